@@ -1,0 +1,237 @@
+"""Seeded synthetic inputs for the verification step.
+
+This module only draws random numbers and lays them out; it holds none of the
+verification arithmetic (no softmax, no acceptance test, no CDF).  Both the
+CUDA path and the CPU oracle are fed from it, in tests and in the benchmark.
+
+Draft tokens are drawn from the draft distribution softmax(draft_logits / T)
+with the Gumbel-max construction (argmax of logits / T plus Gumbel noise),
+which samples that distribution exactly without normalising it.
+
+Logits are returned as float32, or for bf16 workloads as uint16 arrays that
+hold bf16 bit patterns (round-to-nearest-even of the float32 draws).
+
+Workloads (sizes as in the benchmark configurations the project is measured
+on; no public dataset stands behind any of them):
+
+* ``char_level``   B=1 per call, gamma=4, V=256, fp32, T=1; target N(0, 3^2),
+                   draft = 0.8 target + 0.2 fresh N(0, 3^2); ``calls``
+                   independent calls stacked along the batch axis.
+* ``exactness``    B=60000 rows sharing one position, gamma=1, V=4096, fp32;
+                   one fixed target row pair N(0, 3^2) and one fixed draft row
+                   (1-beta) z + beta w, w ~ N(0, 3^2); beta is chosen offline
+                   so that TV(p, q) is the pages' 0.657; fresh tokens and
+                   uniforms per row.
+* ``b8_g3_v32000`` B=8, gamma=3, V=32000, bf16, T=0.7; target N(0, 2.5^2),
+                   draft = 0.9 target + 0.1 N(0, 2.5^2).
+* ``b64_g8_v128256`` B=64, gamma=8, V=128256, bf16, T=1; target N(0, 3^2)
+                   plus +8 on one uniformly chosen token per row; draft =
+                   0.85 target + 0.15 N(0, 3^2).
+* ``multibranch``  32 sequences x 8 branches = 256 rows, gamma=5, V=152064,
+                   bf16, T=1.  Per sequence a branch point bp ~ U{1..gamma}:
+                   target rows, draft rows and draft tokens at positions
+                   j < bp are shared by the sequence's branches; positions
+                   j >= bp are fresh N(0, 3^2) draws per branch.  Draft =
+                   0.8 target + 0.2 N(0, 3^2).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import numpy as np
+
+F32 = "f32"
+BF16 = "bf16"
+
+
+@dataclass
+class Workload:
+    name: str
+    batch: int
+    gamma: int
+    vocab: int
+    dtype: str              # "f32" or "bf16"
+    temperature: float
+    target: np.ndarray      # [B, gamma+1, V] float32 or uint16 (bf16 bits)
+    draft: np.ndarray       # [B, gamma, V]
+    tokens: np.ndarray      # int32 [B, gamma]
+    u_accept: np.ndarray    # float32 [B, gamma]
+    u_resample: np.ndarray  # float32 [B]
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def elem_size(self) -> int:
+        return 4 if self.dtype == F32 else 2
+
+    @property
+    def logit_bytes(self) -> int:
+        """Bytes of logits the step must read at least once."""
+        return self.batch * (2 * self.gamma + 1) * self.vocab * self.elem_size
+
+    def slice(self, lo: int, hi: int) -> "Workload":
+        return Workload(self.name, hi - lo, self.gamma, self.vocab, self.dtype, self.temperature,
+                        self.target[lo:hi], self.draft[lo:hi], self.tokens[lo:hi],
+                        self.u_accept[lo:hi], self.u_resample[lo:hi], dict(self.meta))
+
+
+def bf16_bits(x: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bit patterns, round to nearest even (NaN kept quiet)."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    u = x.view(np.uint32).astype(np.uint64)
+    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    nan = np.isnan(x)
+    out = rounded.astype(np.uint16)
+    if nan.any():
+        out[nan] = ((u[nan] >> 16) | 0x40).astype(np.uint16)
+    return out
+
+
+def bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> the float32 values they denote (exact)."""
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def _normal(rng: np.random.Generator, shape, sigma: float) -> np.ndarray:
+    return rng.standard_normal(shape, dtype=np.float32) * np.float32(sigma)
+
+
+def gumbel_max_tokens(rng: np.random.Generator, logits: np.ndarray, temperature: float,
+                      block_rows: int = 64) -> np.ndarray:
+    """One draw per row from softmax(logits / T) by the Gumbel-max construction.
+
+    ``logits`` is float32 [..., V] (the values the verifier will see).
+    """
+    flat = logits.reshape(-1, logits.shape[-1])
+    out = np.empty(flat.shape[0], np.int32)
+    tiny = np.float32(np.finfo(np.float32).tiny)
+    inv_t = np.float32(1.0 / temperature)
+    for r0 in range(0, flat.shape[0], block_rows):
+        blk = flat[r0:r0 + block_rows]
+        u = rng.random(blk.shape, dtype=np.float32)
+        np.maximum(u, tiny, out=u)
+        g = -np.log(-np.log(u))
+        g += blk * inv_t
+        out[r0:r0 + block_rows] = np.argmax(g, axis=1)
+    return out.reshape(logits.shape[:-1])
+
+
+def _finish(name, dtype, T, target_f32, draft_f32, rng, meta=None, tokens=None) -> Workload:
+    """Round to the storage dtype, draw tokens from the stored draft logits, draw uniforms."""
+    if dtype == BF16:
+        tgt = bf16_bits(target_f32)
+        drf = bf16_bits(draft_f32)
+        drf_seen = bits_to_f32(drf)
+    else:
+        tgt = np.ascontiguousarray(target_f32, dtype=np.float32)
+        drf = np.ascontiguousarray(draft_f32, dtype=np.float32)
+        drf_seen = drf
+    B, G, V = drf.shape
+    if tokens is None:
+        tokens = gumbel_max_tokens(rng, drf_seen, T) if G > 0 else np.zeros((B, 0), np.int32)
+    u_acc = rng.random((B, G), dtype=np.float32)
+    u_res = rng.random(B, dtype=np.float32)
+    return Workload(name, B, G, V, dtype, float(T), tgt, drf, tokens.astype(np.int32),
+                    u_acc, u_res, meta or {})
+
+
+def char_level(calls: int = 1000, seed: int = 0) -> Workload:
+    """B=1 per call, gamma=4, V=256, fp32, T=1; ``calls`` calls stacked on the batch axis."""
+    rng = np.random.default_rng(seed)
+    G, V = 4, 256
+    tgt = _normal(rng, (calls, G + 1, V), 3.0)
+    drf = np.float32(0.8) * tgt[:, :G] + np.float32(0.2) * _normal(rng, (calls, G, V), 3.0)
+    return _finish("char_level_b1_g4_v256_f32", F32, 1.0, tgt, drf, rng, {"calls": calls})
+
+
+def exactness_rows(seed: int = 0, vocab: int = 4096):
+    """The fixed target row pair z (position 0 and the bonus position) and the fixed noise w."""
+    rng = np.random.default_rng(seed)
+    z = _normal(rng, (2, vocab), 3.0)
+    w = _normal(rng, (vocab,), 3.0)
+    return z, w
+
+
+def exactness_draft_row(z: np.ndarray, w: np.ndarray, beta: float) -> np.ndarray:
+    return ((1.0 - beta) * z[0].astype(np.float64) + beta * w.astype(np.float64)).astype(np.float32)
+
+
+def exactness(beta: float, batch: int = 60000, seed: int = 0, vocab: int = 4096) -> Workload:
+    """B rows sharing one position (gamma=1, V=4096, fp32, T=1), fresh tokens/uniforms per row."""
+    z, w = exactness_rows(seed, vocab)
+    d = exactness_draft_row(z, w, beta)
+    rng = np.random.default_rng(seed + 1)
+    tgt = np.broadcast_to(z[None], (batch, 2, vocab))
+    drf = np.broadcast_to(d[None, None], (batch, 1, vocab))
+    tokens = gumbel_max_tokens(rng, np.ascontiguousarray(drf), 1.0, block_rows=2048)
+    return _finish("exactness_b60000_g1_v4096_f32", F32, 1.0, np.ascontiguousarray(tgt),
+                   np.ascontiguousarray(drf), rng, {"beta": beta}, tokens=tokens)
+
+
+def b8_g3_v32000(seed: int = 0) -> Workload:
+    rng = np.random.default_rng(seed)
+    B, G, V = 8, 3, 32000
+    tgt = _normal(rng, (B, G + 1, V), 2.5)
+    drf = np.float32(0.9) * tgt[:, :G] + np.float32(0.1) * _normal(rng, (B, G, V), 2.5)
+    return _finish("b8_g3_v32000_bf16", BF16, 0.7, tgt, drf, rng)
+
+
+def b64_g8_v128256(seed: int = 0, batch: int = 64) -> Workload:
+    rng = np.random.default_rng(seed)
+    B, G, V = batch, 8, 128256
+    tgt = _normal(rng, (B, G + 1, V), 3.0)
+    peak = rng.integers(0, V, size=(B, G + 1))
+    np.add.at(tgt, (np.arange(B)[:, None], np.arange(G + 1)[None, :], peak), np.float32(8.0))
+    drf = np.float32(0.85) * tgt[:, :G] + np.float32(0.15) * _normal(rng, (B, G, V), 3.0)
+    return _finish("b64_g8_v128256_bf16", BF16, 1.0, tgt, drf, rng)
+
+
+def multibranch(seed: int = 0, sequences: int = 32, branches: int = 8, gamma: int = 5,
+                vocab: int = 152064) -> Workload:
+    """sequences x branches rows sharing target/draft rows and tokens before a branch point."""
+    rng = np.random.default_rng(seed)
+    S, K, G, V = sequences, branches, gamma, vocab
+    B = S * K
+    tgt = np.empty((B, G + 1, V), np.float32)
+    drf = np.empty((B, G, V), np.float32)
+    shared = np.zeros((B, G), bool)
+    points = rng.integers(1, G + 1, size=S) if G > 0 else np.zeros(S, np.int64)
+    for s in range(S):
+        bp = int(points[s])
+        base_t = _normal(rng, (bp, V), 3.0)
+        base_d = np.float32(0.8) * base_t + np.float32(0.2) * _normal(rng, (bp, V), 3.0)
+        for k in range(K):
+            b = s * K + k
+            tgt[b, :bp] = base_t
+            drf[b, :bp] = base_d
+            tgt[b, bp:] = _normal(rng, (G + 1 - bp, V), 3.0)
+            if bp < G:
+                drf[b, bp:] = (np.float32(0.8) * tgt[b, bp:G]
+                               + np.float32(0.2) * _normal(rng, (G - bp, V), 3.0))
+            shared[b, :bp] = True
+    # tokens: one draw per (sequence, shared position), one per (row, private position)
+    drf_bits = bf16_bits(drf)
+    seen = bits_to_f32(drf_bits)
+    tokens = np.empty((B, G), np.int32)
+    for s in range(S):
+        bp = int(points[s])
+        rows = slice(s * K, (s + 1) * K)
+        if bp > 0:
+            tokens[rows, :bp] = gumbel_max_tokens(rng, seen[s * K, :bp][None], 1.0)[0][None]
+        if bp < G:
+            tokens[rows, bp:] = gumbel_max_tokens(rng, seen[rows, bp:], 1.0)
+    tgt_bits = bf16_bits(tgt)
+    del tgt
+    u_acc = rng.random((B, G), dtype=np.float32)
+    u_res = rng.random(B, dtype=np.float32)
+    return Workload("multibranch_32x8_g5_v152064_bf16", B, G, V, BF16, 1.0, tgt_bits, drf_bits,
+                    tokens, u_acc, u_res,
+                    {"sequences": S, "branches": K, "branch_points": points.tolist(),
+                     "shared": shared})
+
+
+REGISTRY = {
+    "char_level": char_level,
+    "b8_g3_v32000": b8_g3_v32000,
+    "b64_g8_v128256": b64_g8_v128256,
+    "multibranch": multibranch,
+}
