@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of the batched speculative-sampling verification step.
+
+One step = one verification call over one batch (statistics, acceptance scan,
+residual / bonus draw for every sequence).  Default workload: the multi-branch
+batch, 32 sequences x 8 candidate branches = 256 rows, gamma = 5, V = 152064,
+bf16 logits, T = 1 (the largest of the benchmark configurations with
+V >= 32000; its 856 MB of logits exceed the 126 MB L2, so no flush is needed).
+
+Metric: verified positions per second (B * gamma per step, summed over all
+ranks) and the achieved HBM bandwidth of the fused kernel, algorithmic bytes =
+logits read once = B (2 gamma + 1) V * sizeof(logit).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload multibranch|b64_g8_v128256|b8_g3_v32000|char_level]
+
+N > 1 runs under torch.distributed.run, one rank per GPU: every rank verifies
+its own batch (weak scaling, no data-path collective).  ``--impl reference``
+times the CPU oracle on the host cores on a bounded sample of the workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from speculative_decoding_verification_90_b200 import workloads  # noqa: E402
+
+METRIC = "verified positions/s and achieved HBM GB/s vs B200 peak (spec-verify, 1 GPU)"
+UNIT = "positions/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = [
+    "speculative_decoding_verification_90_b200/csrc/verify_kernel.cuh",
+    "speculative_decoding_verification_90_b200/csrc/specverify.cu",
+]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="multibranch", choices=sorted(workloads.REGISTRY))
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--cluster", type=int, default=0, help="override CTAs per position")
+    ap.add_argument("--threads", type=int, default=0, help="override threads per CTA")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy burst)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def profiled_traffic(workload_name: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches this kernel source."""
+    d = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(d):
+        return None
+    want = kernel_hash()
+    for fn in sorted(os.listdir(d)):
+        if not fn.endswith(".md"):
+            continue
+        text = open(os.path.join(d, fn)).read()
+        w = re.search(r"^workload:\s*(\S+)", text, re.M)
+        hsh = re.search(r"^kernel_source_sha256_16:\s*(\S+)", text, re.M)
+        tr = re.search(r"^dram_bytes_per_launch_full_size:\s*([0-9.eE+]+)", text, re.M)
+        if w and hsh and tr and w.group(1) == workload_name and hsh.group(1) == want:
+            return float(tr.group(1))
+    return None
+
+
+def make_workload(name: str, seed: int):
+    return workloads.REGISTRY[name](seed=seed)
+
+
+def positions_per_step(wl) -> int:
+    return wl.batch * wl.gamma
+
+
+# ----------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return []
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                frac = float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                rows.append({"t": ts + frac, "sm": float(parts[2]), "sm_max": float(parts[3]),
+                             "power": float(parts[4]) if parts[4] not in ("[N/A]", "") else None,
+                             "hw_slowdown": parts[6], "hw_thermal": parts[7],
+                             "sw_thermal": parts[8], "sw_power_cap": parts[9]})
+            except Exception:
+                continue
+        return rows
+
+
+def summarize_clocks(rows, t0, t1):
+    if not rows:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+    inside = [r for r in rows if t0 - 0.06 <= r["t"] <= t1 + 0.06]
+    if not inside:  # timed region shorter than the sampling period: nearest sample
+        inside = [min(rows, key=lambda r: abs(r["t"] - 0.5 * (t0 + t1)))]
+    reasons = set()
+    for r in inside:
+        for key, name in (("hw_slowdown", "hw_slowdown"), ("hw_thermal", "hw_thermal_slowdown"),
+                          ("sw_thermal", "sw_thermal_slowdown"), ("sw_power_cap", "sw_power_cap")):
+            if r[key].lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": float(np.median([r["sm"] for r in inside])),
+            "sm_max_mhz": float(max(r["sm_max"] for r in inside)),
+            "reasons": sorted(reasons), "samples": len(inside)}
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle (reference arm and cpu_baseline)
+# ----------------------------------------------------------------------------
+
+def time_oracle(wl, budget_s: float):
+    """Oracle over the whole batch on all host cores, repeated until `budget_s`
+    of CPU time is reached with at least one pass; bounded to a sample of
+    sequences when one pass would take longer than the budget."""
+    import oracle
+    threads = os.cpu_count() or 1
+    # calibrate on one sequence per thread
+    n_cal = min(wl.batch, threads)
+    t = time.perf_counter()
+    oracle.verify(wl.target[:n_cal], wl.draft[:n_cal], wl.tokens[:n_cal], wl.u_accept[:n_cal],
+                  wl.u_resample[:n_cal], wl.temperature, threads=threads)
+    per_seq_wall = (time.perf_counter() - t) / max(1, math.ceil(n_cal / threads))
+    seqs = wl.batch
+    if per_seq_wall * math.ceil(seqs / threads) > budget_s:
+        seqs = max(threads, int(budget_s / per_seq_wall) * threads)
+        seqs = min(seqs, wl.batch)
+    passes, elapsed = 0, 0.0
+    while passes == 0 or elapsed < budget_s:
+        t = time.perf_counter()
+        oracle.verify(wl.target[:seqs], wl.draft[:seqs], wl.tokens[:seqs], wl.u_accept[:seqs],
+                      wl.u_resample[:seqs], wl.temperature, threads=threads)
+        elapsed += time.perf_counter() - t
+        passes += 1
+    value = passes * seqs * wl.gamma / elapsed
+    sample = (f"{seqs} of {wl.batch} sequences of the workload ({seqs * wl.gamma} positions), "
+              f"{passes} pass(es), {elapsed:.1f} s wall on {threads} threads")
+    return value, threads, sample, elapsed / passes
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    wl = make_workload(args.workload, args.seed)
+    import oracle
+    oracle.build()
+    threads = os.cpu_count() or 1
+    # each step: a bounded sample of the workload's sequences
+    per_step_budget = max(0.5, 120.0 / max(1, args.steps + args.warmup))
+    n_seq = min(wl.batch, threads)
+    t = time.perf_counter()
+    oracle.verify(wl.target[:n_seq], wl.draft[:n_seq], wl.tokens[:n_seq], wl.u_accept[:n_seq],
+                  wl.u_resample[:n_seq], wl.temperature, threads=threads)
+    one = time.perf_counter() - t
+    n_seq = int(min(wl.batch, max(1, per_step_budget / one) * n_seq))
+    for _ in range(args.warmup):
+        oracle.verify(wl.target[:n_seq], wl.draft[:n_seq], wl.tokens[:n_seq],
+                      wl.u_accept[:n_seq], wl.u_resample[:n_seq], wl.temperature, threads=threads)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.verify(wl.target[:n_seq], wl.draft[:n_seq], wl.tokens[:n_seq],
+                      wl.u_accept[:n_seq], wl.u_resample[:n_seq], wl.temperature, threads=threads)
+    el = time.perf_counter() - t
+    value = args.steps * n_seq * wl.gamma / el
+    sample = f"{n_seq} of {wl.batch} sequences per step ({n_seq * wl.gamma} positions)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "batch": wl.batch, "gamma": wl.gamma, "vocab": wl.vocab,
+                   "logits": wl.dtype, "temperature": wl.temperature},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.gpus != world and world > 1:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    from speculative_decoding_verification_90_b200.specverify import SpecVerify
+
+    # every rank verifies its own batch (weak scaling); seeds differ per rank
+    wl = make_workload(args.workload, args.seed + rank)
+    B, G, V = wl.batch, wl.gamma, wl.vocab
+    step_bytes = wl.logit_bytes
+
+    def put(a, logits):
+        if logits and wl.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    # inputs larger than L2 in total: rotate copies when one batch is smaller
+    n_sets = max(1, math.ceil(2 * L2_BYTES / step_bytes)) if step_bytes < 2 * L2_BYTES else 1
+    n_sets = min(n_sets, 256)
+    base = {"target": put(wl.target, True), "draft": put(wl.draft, True),
+            "tokens": put(wl.tokens, False), "u_accept": put(wl.u_accept, False),
+            "u_resample": put(wl.u_resample, False)}
+    sets = [base] + [{k: v.clone() for k, v in base.items()} for _ in range(n_sets - 1)]
+    out_t = torch.empty((B, G + 1), dtype=torch.int32, device=dev)
+    out_n = torch.empty((B,), dtype=torch.int32, device=dev)
+
+    sv = SpecVerify(B, G, V, wl.dtype, local)
+    if args.cluster or args.threads:
+        c0, t0 = sv.launch()
+        sv.set_launch(args.cluster or c0, args.threads or t0)
+    cluster, threads = sv.launch()
+
+    def step(i):
+        s = sets[i % n_sets]
+        sv.run(s["target"], s["draft"], s["tokens"], s["u_accept"], s["u_resample"],
+               wl.temperature, out_t, out_n)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    st, bits = sv.status()
+    if st != 0:
+        raise SystemExit(f"device status {st} (bits {bits}) during warm-up")
+
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local) if rank == 0 else None
+    time.sleep(0.15)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    t_wall1 = time.time()
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    time.sleep(0.12)
+    rows = sampler.stop() if sampler else []
+    ms = ev0.elapsed_time(ev1)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    per_launch_s = ms / 1e3 / args.steps  # this rank's kernel: one launch per step
+
+    # end to end through the host-buffer entry point (pinned host memory)
+    def pinned(a, logits):
+        t = torch.from_numpy(np.ascontiguousarray(a).view(np.int16) if logits and wl.dtype == "bf16"
+                             else np.ascontiguousarray(a))
+        if logits and wl.dtype == "bf16":
+            t = t.view(torch.bfloat16)
+        return t.pin_memory()
+
+    h_in = [pinned(wl.target, True), pinned(wl.draft, True), pinned(wl.tokens, False),
+            pinned(wl.u_accept, False), pinned(wl.u_resample, False)]
+    h_ot = torch.empty((B, G + 1), dtype=torch.int32).pin_memory()
+    h_on = torch.empty((B,), dtype=torch.int32).pin_memory()
+    e2e_steps = max(1, min(args.e2e_steps, args.steps))
+    sv.run_host(*h_in[:5], wl.temperature, h_ot, h_on)  # staging allocation outside the timing
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        sv.run_host(*h_in[:5], wl.temperature, h_ot, h_on)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    h2d = sum(t.numel() * t.element_size() for t in h_in)
+    d2h = h_ot.numel() * 4 + h_on.numel() * 4
+    st, bits = sv.status()
+    sv.close()
+    # tokens settled per step on this rank = accepted + 1 per sequence (last device step)
+    emitted = int((out_n.cpu().numpy().astype(np.int64) + 1).sum())
+
+    line = None
+    if rank == 0:
+        peak, peak_src = measured_peak()
+        achieved = step_bytes / per_launch_s / 1e9
+        traffic = profiled_traffic(wl.name) if args.cluster == 0 and args.threads == 0 else None
+        positions = positions_per_step(wl) * world
+        value = positions * args.steps / (ms_max / 1e3)
+        e2e_value = positions * e2e_steps / (float(e2e_ms.item()) / 1e3)
+        clocks = summarize_clocks(rows, t_wall0, t_wall1)
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            v, cores, sample, _ = time_oracle(wl, budget_s=12.0)
+            cpu = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": B, "gamma": G, "vocab": V,
+                       "logits": wl.dtype, "temperature": wl.temperature,
+                       "parallelism": f"dp{world} (independent batches per GPU)",
+                       "l2": ("inputs larger than L2 (%.0f MB per step, %d rotating set(s))"
+                              % (step_bytes / 1e6, n_sets)),
+                       "launch": {"cluster_ctas": cluster, "threads": threads}},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
+                         "algorithmic_bytes_per_launch": step_bytes,
+                         "kernel": "verify_kernel (fused: stats + accept + scan + draw)"},
+            "hbm_gbs": achieved,
+            "emitted_tokens_per_step": emitted,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "gpu_launches": args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+            "status_after": st,
+        }
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,179 @@
+/*
+ * specverify: batched speculative-sampling verification on NVIDIA B200 (sm_100a).
+ *
+ * The operation (page title and section that define it):
+ *   "Speculative decoding - the small model writes first and the big model
+ *   checks" (blog.mna-game.duckdns.org, deep-learning post 46), section 1:
+ *   accept a draft token t with probability min(1, q(t)/p(t)); on rejection
+ *   draw again from max(0, q - p) / ||max(0, q - p)||_1.
+ *   "Speculative decoding: how to run big models fast" (ai-trend.me), section
+ *   "How it works": judge drafts left to right, stop at the first rejection
+ *   and discard the rest, append one token drawn from q at position gamma+1
+ *   when every draft is accepted, so each call emits 1 .. gamma+1 tokens;
+ *   temperature is handled as sampling from an adjusted distribution.
+ *
+ * For every sequence b of a batch of B:
+ *   q_j = softmax(target_logits[b, j, :] / T),  j = 0 .. gamma
+ *   p_j = softmax(draft_logits[b, j, :] / T),   j = 0 .. gamma-1
+ *   n   = first j with  u_accept[b, j] >= q_j(t_j) / p_j(t_j)  (t_j =
+ *         draft_tokens[b, j]), or gamma if there is none
+ *   if n < gamma: r = max(0, q_n - p_n)   else: r = q_gamma
+ *   s   = smallest i with  sum_{k<=i} r_k  >  u_resample[b] * sum_k r_k
+ *   out_tokens[b, :] = t_0 .. t_{n-1}, s, -1, ..., -1     (gamma+1 entries)
+ *   out_num_accepted[b] = n
+ *
+ * Conventions that the pages leave open:
+ *   - the acceptance comparison is strict (u < ratio); q(t) == 0 gives ratio 0
+ *     and p(t) == 0 < q(t) gives ratio +inf;
+ *   - one uniform per sequence serves both the residual draw and the bonus
+ *     draw, because exactly one of the two happens;
+ *   - if rounding leaves no index with cumulative mass above u * Z, the draw
+ *     returns the last index with r_i > 0; zero-mass tokens are never drawn;
+ *   - if the residual mass is zero at a rejection (reachable only through
+ *     rounding when q and p agree), the draw falls back to q_n and the status
+ *     word records SV_WARN_ZERO_MASS;
+ *   - a sequence with a draft token outside [0, V), or with any logit row
+ *     holding NaN or +inf or no finite entry, emits nothing:
+ *     out_num_accepted[b] = 0 and out_tokens[b, :] = -1, and the status word
+ *     records SV_ERR_TOKEN_RANGE or SV_ERR_NONFINITE.  -inf logits are legal
+ *     (masked vocabulary entries carry zero probability).
+ *
+ * Memory: the caller owns every input and output buffer.  A handle owns a
+ * small device workspace (per-row statistics, per-position decisions, one
+ * ticket per sequence, the status word), allocated by specverify_create and
+ * freed by specverify_destroy.  Device buffers must be device memory of the
+ * handle's device.  A handle may be used by one stream at a time.
+ *
+ * Errors: argument errors are reported before anything is enqueued.  Data
+ * errors found on the device never trap or stall: they set bits of the
+ * handle's status word, read back (and cleared) by specverify_get_status.
+ *
+ * Streams: `stream` is a cudaStream_t passed as void* (NULL is the legacy
+ * default stream).  specverify_run only enqueues work and returns.
+ */
+#ifndef SPECVERIFY_H
+#define SPECVERIFY_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct specverify_ctx *specverify_t;
+
+typedef enum {
+  SV_DTYPE_F32 = 0,  /* IEEE binary32 logits */
+  SV_DTYPE_BF16 = 1  /* bfloat16 logits */
+} sv_dtype;
+
+typedef enum {
+  SV_OK = 0,
+  SV_ERR_INVALID_ARG = 1,  /* bad size, pointer, alignment, temperature or handle */
+  SV_ERR_CUDA = 2,         /* a CUDA runtime call failed; see specverify_last_error() */
+  SV_ERR_OOM = 3,          /* device or host allocation failed */
+  SV_ERR_UNSUPPORTED = 4,  /* the device is not an sm_100 (B200-class) GPU */
+  SV_ERR_TOKEN_RANGE = 16, /* device: some draft token was outside [0, V) */
+  SV_ERR_NONFINITE = 17,   /* device: some logit row held NaN/+inf or only -inf */
+  SV_WARN_ZERO_MASS = 18   /* device: a residual had zero mass; drew from q_n instead */
+} sv_status;
+
+/*
+ * Create a handle for batches of `batch` sequences with `gamma` draft tokens
+ * over a vocabulary of `vocab` entries stored as `dtype`, on CUDA device
+ * `device`.  0 <= batch, 0 <= gamma <= 4096, 1 <= vocab <= 2^30.
+ * Allocates the workspace (about 64 bytes per position plus 16 per sequence)
+ * and chooses a default launch shape.  The caller's current device is left
+ * unchanged.  Returns SV_OK and stores the handle in *out, or an error and
+ * leaves *out NULL.
+ */
+sv_status specverify_create(specverify_t *out, int batch, int gamma, int vocab,
+                            sv_dtype dtype, int device);
+
+/*
+ * Enqueue one verification step on `stream` (device pointers):
+ *   target_logits    [batch, gamma+1, vocab]  dtype, row-major, contiguous
+ *   draft_logits     [batch, gamma,   vocab]  dtype, row-major, contiguous
+ *   draft_tokens     int32 [batch, gamma], expected in [0, vocab)
+ *   u_accept         float [batch, gamma], uniforms in [0, 1)
+ *   u_resample       float [batch],        uniforms in [0, 1)
+ *   temperature      host value, finite and > 0 (divides both logit tensors)
+ *   out_tokens       int32 [batch, gamma+1] (written)
+ *   out_num_accepted int32 [batch]          (written)
+ * Logit pointers must be aligned to their element size; 16-byte aligned
+ * pointers together with vocab * sizeof(dtype) a multiple of 16 take the
+ * vectorised (128-bit load) path, anything else a scalar-load path.
+ * Draft pointers may be NULL when gamma == 0; everything may be NULL when
+ * batch == 0 (nothing is enqueued).  The call is asynchronous.
+ */
+sv_status specverify_run(specverify_t h, const void *target_logits,
+                         const void *draft_logits, const int32_t *draft_tokens,
+                         const float *u_accept, const float *u_resample,
+                         float temperature, int32_t *out_tokens,
+                         int32_t *out_num_accepted, void *stream);
+
+/*
+ * The same step on HOST buffers with the shapes of specverify_run (pinned
+ * host memory gives full copy bandwidth).  Copies the inputs to a device
+ * staging area owned by the handle (allocated on first use, freed by
+ * specverify_destroy), runs the step, copies both outputs back and waits for
+ * `stream`.  Returns after the outputs are in host memory.
+ */
+sv_status specverify_run_host(specverify_t h, const void *target_logits,
+                              const void *draft_logits, const int32_t *draft_tokens,
+                              const float *u_accept, const float *u_resample,
+                              float temperature, int32_t *out_tokens,
+                              int32_t *out_num_accepted, void *stream);
+
+/* Free the handle and everything it owns.  NULL is ignored.  Waits for the
+ * device work of the handle to finish first. */
+void specverify_destroy(specverify_t h);
+
+/*
+ * Wait for `stream`, read and clear the handle's device status word.
+ * Returns the most severe condition seen since the last call:
+ * SV_ERR_TOKEN_RANGE, then SV_ERR_NONFINITE, then SV_WARN_ZERO_MASS, else
+ * SV_OK.  `*bits` (may be NULL) receives the raw bit set (1: token range,
+ * 2: non-finite row, 4: zero residual mass).
+ */
+sv_status specverify_get_status(specverify_t h, void *stream, uint32_t *bits);
+
+/*
+ * Test and debug readback of the last step's intermediate values (waits for
+ * `stream`; host pointers, any may be NULL):
+ *   target_max  float  [batch, gamma+1]  max_i x_i of each target row
+ *   target_sum  double [batch, gamma+1]  sum_i exp((x_i - max) / T)
+ *   draft_max   float  [batch, gamma]
+ *   draft_sum   double [batch, gamma]
+ *   q_tok       double [batch, gamma]    q_j(t_j)
+ *   p_tok       double [batch, gamma]    p_j(t_j)
+ *   ratio       double [batch, gamma]    q_j(t_j) / p_j(t_j) as tested
+ *   resid_mass  double [batch]           mass Z of the distribution drawn from
+ * Positions that the device did not need keep their previous contents.
+ */
+sv_status specverify_debug_readback(specverify_t h, float *target_max, double *target_sum,
+                                   float *draft_max, double *draft_sum, double *q_tok,
+                                   double *p_tok, double *ratio, double *resid_mass,
+                                   void *stream);
+
+/*
+ * Launch shape: `cluster_ctas` thread blocks (1..8, one thread-block cluster)
+ * share each position's vocabulary; `threads` per block is 128, 256 or 512.
+ * specverify_create picks a shape from the problem size and the SM count;
+ * this call overrides it (results do not depend on the shape beyond the
+ * rounding of partial sums).
+ */
+sv_status specverify_set_launch(specverify_t h, int cluster_ctas, int threads);
+sv_status specverify_get_launch(specverify_t h, int *cluster_ctas, int *threads);
+
+/* Static text for a status code. */
+const char *specverify_status_string(sv_status s);
+
+/* Text of the last CUDA runtime error seen by this thread ("" if none). */
+const char *specverify_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPECVERIFY_H */

@@ -1,0 +1,258 @@
+"""Thin Python binding of ``libspecverify.so`` (the C ABI in include/specverify.h).
+
+Argument marshalling only: every step of the verification runs in the CUDA
+library.  The functions keep the C names; ``SpecVerify`` wraps a handle and
+takes torch tensors (device memory and streams come from PyTorch).
+
+Importing this module loads the library and fails loudly if it has not been
+built (``python -m speculative_decoding_verification_90_b200.build``).  There
+is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libspecverify.so")
+
+SV_DTYPE_F32 = 0
+SV_DTYPE_BF16 = 1
+
+SV_OK = 0
+SV_ERR_INVALID_ARG = 1
+SV_ERR_CUDA = 2
+SV_ERR_OOM = 3
+SV_ERR_UNSUPPORTED = 4
+SV_ERR_TOKEN_RANGE = 16
+SV_ERR_NONFINITE = 17
+SV_WARN_ZERO_MASS = 18
+
+# every function declared in include/specverify.h, with its ctypes signature
+_vp, _i, _f, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_uint32)
+SIGNATURES = {
+    "specverify_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
+    "specverify_run": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
+    "specverify_run_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
+    "specverify_destroy": (None, [_vp]),
+    "specverify_get_status": (_i, [_vp, _vp, _u32p]),
+    "specverify_debug_readback": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "specverify_set_launch": (_i, [_vp, _i, _i]),
+    "specverify_get_launch": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "specverify_status_string": (ctypes.c_char_p, [_i]),
+    "specverify_last_error": (ctypes.c_char_p, []),
+}
+
+
+def _load_library():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m speculative_decoding_verification_90_b200.build` (nvcc, sm_100a). "
+            "There is no CPU fallback.")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load_library()
+
+
+class SpecVerifyError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        msg = _lib.specverify_status_string(status).decode()
+        extra = _lib.specverify_last_error().decode()
+        super().__init__(f"{where}: {msg} (status {status})" + (f" [{extra}]" if extra else ""))
+        self.status = status
+
+
+def _check(status: int, where: str) -> int:
+    if status != SV_OK:
+        raise SpecVerifyError(status, where)
+    return status
+
+
+# ---- the C entry points, one Python function each (raw pointers as ints) ----
+
+def specverify_create(batch: int, gamma: int, vocab: int, dtype: int, device: int = 0) -> int:
+    h = ctypes.c_void_p()
+    _check(_lib.specverify_create(ctypes.byref(h), batch, gamma, vocab, dtype, device),
+           "specverify_create")
+    return h.value
+
+
+def specverify_run(h, target, draft, tokens, u_accept, u_resample, temperature, out_tokens,
+                   out_num_accepted, stream=0) -> int:
+    return _check(_lib.specverify_run(h, target, draft, tokens, u_accept, u_resample,
+                                      float(temperature), out_tokens, out_num_accepted, stream),
+                  "specverify_run")
+
+
+def specverify_run_host(h, target, draft, tokens, u_accept, u_resample, temperature, out_tokens,
+                        out_num_accepted, stream=0) -> int:
+    return _check(_lib.specverify_run_host(h, target, draft, tokens, u_accept, u_resample,
+                                           float(temperature), out_tokens, out_num_accepted,
+                                           stream),
+                  "specverify_run_host")
+
+
+def specverify_destroy(h) -> None:
+    _lib.specverify_destroy(h)
+
+
+def specverify_get_status(h, stream=0) -> tuple[int, int]:
+    bits = ctypes.c_uint32()
+    st = _lib.specverify_get_status(h, stream, ctypes.byref(bits))
+    if st in (SV_ERR_INVALID_ARG, SV_ERR_CUDA, SV_ERR_OOM, SV_ERR_UNSUPPORTED):
+        _check(st, "specverify_get_status")
+    return st, bits.value
+
+
+def specverify_debug_readback(h, *ptrs, stream=0) -> int:
+    return _check(_lib.specverify_debug_readback(h, *ptrs, stream), "specverify_debug_readback")
+
+
+def specverify_set_launch(h, cluster_ctas: int, threads: int) -> int:
+    return _check(_lib.specverify_set_launch(h, cluster_ctas, threads), "specverify_set_launch")
+
+
+def specverify_get_launch(h) -> tuple[int, int]:
+    c, t = ctypes.c_int(), ctypes.c_int()
+    _check(_lib.specverify_get_launch(h, ctypes.byref(c), ctypes.byref(t)), "specverify_get_launch")
+    return c.value, t.value
+
+
+def specverify_status_string(status: int) -> str:
+    return _lib.specverify_status_string(status).decode()
+
+
+def specverify_last_error() -> str:
+    return _lib.specverify_last_error().decode()
+
+
+# ---- tensor-level wrapper ----
+
+class SpecVerify:
+    """A handle for fixed (batch, gamma, vocab, dtype) on one CUDA device.
+
+    ``run`` takes torch CUDA tensors and enqueues on the current torch stream
+    (or ``stream``); ``run_host`` takes host numpy arrays or CPU tensors.
+    """
+
+    def __init__(self, batch: int, gamma: int, vocab: int, dtype: str = "bf16", device: int = 0):
+        self.batch, self.gamma, self.vocab, self.dtype = batch, gamma, vocab, dtype
+        self.device = device
+        code = {"f32": SV_DTYPE_F32, "bf16": SV_DTYPE_BF16}[dtype]
+        self.handle = specverify_create(batch, gamma, vocab, code, device)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            specverify_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    # shapes the C ABI expects
+    def _shapes(self):
+        B, G, V = self.batch, self.gamma, self.vocab
+        return {"target": (B, G + 1, V), "draft": (B, G, V), "tokens": (B, G),
+                "u_accept": (B, G), "u_resample": (B,), "out_tokens": (B, G + 1),
+                "out_num_accepted": (B,)}
+
+    def _check_tensor(self, name, t, dtype, cuda):
+        import torch
+        want = self._shapes()[name]
+        if tuple(t.shape) != want:
+            raise ValueError(f"{name}: shape {tuple(t.shape)} != {want}")
+        if t.dtype != dtype:
+            raise ValueError(f"{name}: dtype {t.dtype} != {dtype}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous")
+        if cuda and (t.device.type != "cuda" or t.device.index != self.device):
+            raise ValueError(f"{name}: must live on cuda:{self.device}")
+        if not cuda and t.device.type != "cpu":
+            raise ValueError(f"{name}: must be a host tensor")
+        return t.data_ptr() if t.numel() else 0
+
+    def _logit_dtype(self):
+        import torch
+        return torch.bfloat16 if self.dtype == "bf16" else torch.float32
+
+    def run(self, target, draft, tokens, u_accept, u_resample, temperature, out_tokens,
+            out_num_accepted, stream=None):
+        import torch
+        ld = self._logit_dtype()
+        ptrs = [self._check_tensor("target", target, ld, True),
+                self._check_tensor("draft", draft, ld, True),
+                self._check_tensor("tokens", tokens, torch.int32, True),
+                self._check_tensor("u_accept", u_accept, torch.float32, True),
+                self._check_tensor("u_resample", u_resample, torch.float32, True)]
+        outs = [self._check_tensor("out_tokens", out_tokens, torch.int32, True),
+                self._check_tensor("out_num_accepted", out_num_accepted, torch.int32, True)]
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        specverify_run(self.handle, *ptrs, temperature, *outs, sp)
+
+    def run_host(self, target, draft, tokens, u_accept, u_resample, temperature, out_tokens,
+                 out_num_accepted, stream=None):
+        """Host buffers in and out (torch CPU tensors, ideally pinned); returns when done."""
+        import torch
+        ld = self._logit_dtype()
+        ptrs = [self._check_tensor("target", target, ld, False),
+                self._check_tensor("draft", draft, ld, False),
+                self._check_tensor("tokens", tokens, torch.int32, False),
+                self._check_tensor("u_accept", u_accept, torch.float32, False),
+                self._check_tensor("u_resample", u_resample, torch.float32, False)]
+        outs = [self._check_tensor("out_tokens", out_tokens, torch.int32, False),
+                self._check_tensor("out_num_accepted", out_num_accepted, torch.int32, False)]
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        specverify_run_host(self.handle, *ptrs, temperature, *outs, sp)
+
+    def status(self, stream=None) -> tuple[int, int]:
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        return specverify_get_status(self.handle, sp)
+
+    def set_launch(self, cluster_ctas: int, threads: int):
+        specverify_set_launch(self.handle, cluster_ctas, threads)
+
+    def launch(self) -> tuple[int, int]:
+        return specverify_get_launch(self.handle)
+
+    def readback(self, stream=None) -> dict:
+        """Intermediate values of the last step (see specverify_debug_readback)."""
+        import torch
+        B, G = self.batch, self.gamma
+        out = {"target_max": np.zeros((B, G + 1), np.float32),
+               "target_sum": np.zeros((B, G + 1), np.float64),
+               "draft_max": np.zeros((B, G), np.float32),
+               "draft_sum": np.zeros((B, G), np.float64),
+               "q_tok": np.zeros((B, G), np.float64),
+               "p_tok": np.zeros((B, G), np.float64),
+               "ratio": np.zeros((B, G), np.float64),
+               "resid_mass": np.zeros(B, np.float64)}
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        specverify_debug_readback(self.handle, *[a.ctypes.data for a in out.values()], stream=sp)
+        return out

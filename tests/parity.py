@@ -1,0 +1,132 @@
+"""Shared helpers of the GPU parity tests: run a workload through the C ABI and
+compare it with the CPU oracle decision by decision.
+
+Decision parity (the contract of the tests): for every sequence, the accepted
+count and every emitted token must equal the oracle's, except where the
+oracle's margin at the first differing decision is below ``MARGIN``:
+|u_accept - ratio| for an acceptance test, and for the draw the distance of
+u_resample to the ends of the chosen token's interval of the normalised
+cumulative mass.  Such cases are counted and reported.  Softmax quantities
+must agree within ``PROB_TOL`` absolute (q(t), p(t)) and row sums within
+``SUM_RTOL`` relative.
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+
+MARGIN = 1e-6
+PROB_TOL = 1e-5
+SUM_RTOL = 1e-5
+
+
+def to_device(wl, device=0):
+    import torch
+    dev = torch.device("cuda", device)
+
+    def logits(a):
+        if wl.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    return {
+        "target": logits(wl.target),
+        "draft": logits(wl.draft),
+        "tokens": torch.from_numpy(np.ascontiguousarray(wl.tokens, np.int32)).to(dev),
+        "u_accept": torch.from_numpy(np.ascontiguousarray(wl.u_accept, np.float32)).to(dev),
+        "u_resample": torch.from_numpy(np.ascontiguousarray(wl.u_resample, np.float32)).to(dev),
+    }
+
+
+def gpu_run(wl, cluster=None, threads=None, device=0, inputs=None, sv=None, readback=True):
+    """One verification call of the whole workload; returns numpy outputs."""
+    import torch
+    from speculative_decoding_verification_90_b200.specverify import SpecVerify
+    own = sv is None
+    if own:
+        sv = SpecVerify(wl.batch, wl.gamma, wl.vocab, wl.dtype, device)
+    try:
+        if cluster is not None or threads is not None:
+            c0, t0 = sv.launch()
+            sv.set_launch(cluster or c0, threads or t0)
+        d = inputs if inputs is not None else to_device(wl, device)
+        out_t = torch.full((wl.batch, wl.gamma + 1), -7, dtype=torch.int32, device=f"cuda:{device}")
+        out_n = torch.full((wl.batch,), -7, dtype=torch.int32, device=f"cuda:{device}")
+        sv.run(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
+               wl.temperature, out_t, out_n)
+        torch.cuda.synchronize(device)
+        status, bits = sv.status()
+        res = {"out_tokens": out_t.cpu().numpy(), "out_num_accepted": out_n.cpu().numpy(),
+               "status": status, "bits": bits, "launch": sv.launch()}
+        if readback:
+            res.update(sv.readback())
+        return res
+    finally:
+        if own:
+            sv.close()
+
+
+def oracle_run(wl, b_range=None):
+    import oracle
+    return oracle.verify(wl.target, wl.draft, wl.tokens, wl.u_accept, wl.u_resample,
+                         wl.temperature, threads=os.cpu_count() or 1, b_range=b_range)
+
+
+def compare(wl, gpu, ora, seqs=None, check_probs=True):
+    """Decision parity over the sequences `seqs` (default: all).  Returns a summary dict."""
+    B, G = wl.batch, wl.gamma
+    seqs = np.arange(B) if seqs is None else np.asarray(seqs)
+    hard, margin_cases = [], []
+    for b in seqs:
+        ng, no = int(gpu["out_num_accepted"][b]), int(ora["out_num_accepted"][b])
+        tg, to = gpu["out_tokens"][b], ora["out_tokens"][b]
+        if ora["seq_status"][b] in (16, 17):
+            if ng != 0 or not (tg == -1).all():
+                hard.append((int(b), "error outcome", ng, tg.tolist()))
+            continue
+        if ng != no:
+            j = min(ng, no)
+            m = ora["accept_margin"][b, j]
+            (margin_cases if m < MARGIN else hard).append((int(b), "accept", j, float(m)))
+            continue
+        if not np.array_equal(tg, to):
+            m = ora["cdf_margin_norm"][b]
+            (margin_cases if m < MARGIN else hard).append(
+                (int(b), "draw", int(tg[no]), int(to[no]), float(m)))
+    summary = {"sequences": int(len(seqs)), "hard": hard, "margin_cases": margin_cases}
+    if check_probs and "q_tok" in gpu:
+        ok = ora["seq_status"][seqs] == 0
+        s = seqs[ok]
+        if G > 0 and len(s):
+            tested = ~np.isnan(ora["q_tok"][s])
+            dq = np.abs(gpu["q_tok"][s] - ora["q_tok"][s])[tested]
+            dp = np.abs(gpu["p_tok"][s] - ora["p_tok"][s])[tested]
+            summary["max_dq"] = float(dq.max()) if dq.size else 0.0
+            summary["max_dp"] = float(dp.max()) if dp.size else 0.0
+            rd = np.abs(gpu["draft_sum"][s] / ora["draft_sum"][s] - 1.0)
+            summary["max_draft_sum_rel"] = float(rd.max())
+            summary["draft_max_equal"] = bool(np.array_equal(
+                gpu["draft_max"][s].astype(np.float64), ora["draft_max"][s]))
+        if len(s):
+            rt = np.abs(gpu["target_sum"][s] / ora["target_sum"][s] - 1.0)
+            summary["max_target_sum_rel"] = float(rt.max())
+            summary["target_max_equal"] = bool(np.array_equal(
+                gpu["target_max"][s].astype(np.float64), ora["target_max"][s]))
+            dz = np.abs(gpu["resid_mass"][s] - ora["resid_mass"][s])
+            summary["max_dz"] = float(np.nanmax(dz)) if dz.size else 0.0
+    return summary
+
+
+def assert_parity(summary, max_margin_frac=0.01):
+    assert not summary["hard"], f"decisions differ outside the margin: {summary['hard'][:5]}"
+    assert len(summary["margin_cases"]) <= max(1, max_margin_frac * summary["sequences"]), summary
+    for key in ("max_dq", "max_dp", "max_dz"):
+        if key in summary:
+            assert summary[key] <= PROB_TOL, summary
+    for key in ("max_target_sum_rel", "max_draft_sum_rel"):
+        if key in summary:
+            assert summary[key] <= SUM_RTOL, summary
+    for key in ("target_max_equal", "draft_max_equal"):
+        if key in summary:
+            assert summary[key], summary
