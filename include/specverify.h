@@ -81,9 +81,10 @@ typedef enum {
 /*
  * Create a handle for batches of `batch` sequences with `gamma` draft tokens
  * over a vocabulary of `vocab` entries stored as `dtype`, on CUDA device
- * `device`.  0 <= batch, 0 <= gamma <= 4096, 1 <= vocab <= 2^30.
- * Allocates the workspace (about 64 bytes per position plus 16 per sequence)
- * and chooses a default launch shape.  The caller's current device is left
+ * `device`.  0 <= batch, 0 <= gamma <= 255, 1 <= vocab <= 2^30.
+ * Allocates the workspace (per position: up to 64 partial statistics of
+ * 32 bytes plus about 64 bytes; per sequence 16 bytes per 32 groups of 16
+ * bytes of a row) and chooses a default launch shape.  The caller's current device is left
  * unchanged.  Returns SV_OK and stores the handle in *out, or an error and
  * leaves *out NULL.
  */
@@ -141,30 +142,47 @@ sv_status specverify_get_status(specverify_t h, void *stream, uint32_t *bits);
 /*
  * Test and debug readback of the last step's intermediate values (waits for
  * `stream`; host pointers, any may be NULL):
- *   target_max  float  [batch, gamma+1]  max_i x_i of each target row
- *   target_sum  double [batch, gamma+1]  sum_i exp((x_i - max) / T)
- *   draft_max   float  [batch, gamma]
- *   draft_sum   double [batch, gamma]
+ *   target_lse  double [batch, gamma+1]  log sum_i exp(x_i / T) of each target row
+ *   draft_lse   double [batch, gamma]    the same for each draft row
  *   q_tok       double [batch, gamma]    q_j(t_j)
  *   p_tok       double [batch, gamma]    p_j(t_j)
  *   ratio       double [batch, gamma]    q_j(t_j) / p_j(t_j) as tested
  *   resid_mass  double [batch]           mass Z of the distribution drawn from
  * Positions that the device did not need keep their previous contents.
  */
-sv_status specverify_debug_readback(specverify_t h, float *target_max, double *target_sum,
-                                   float *draft_max, double *draft_sum, double *q_tok,
-                                   double *p_tok, double *ratio, double *resid_mass,
-                                   void *stream);
+sv_status specverify_debug_readback(specverify_t h, double *target_lse, double *draft_lse,
+                                   double *q_tok, double *p_tok, double *ratio,
+                                   double *resid_mass, void *stream);
 
 /*
- * Launch shape: `cluster_ctas` thread blocks (1..8, one thread-block cluster)
- * share each position's vocabulary; `threads` per block is 128, 256 or 512.
- * specverify_create picks a shape from the problem size and the SM count;
- * this call overrides it (results do not depend on the shape beyond the
- * rounding of partial sums).
+ * Launch shape of the statistics kernel (the one that streams every logit):
+ * each position's two rows are split over `slices` thread blocks of
+ * `threads` threads (128, 256 or 512).  1 <= slices
+ * <= min(64, ceil(vocab / group) / 128), group = 8 bf16 or 4 fp32 entries;
+ * larger values return SV_ERR_INVALID_ARG.  specverify_create picks a shape
+ * from the problem size and the SM count; this call overrides it for later
+ * runs (results do not depend on the shape beyond the rounding of partial
+ * sums).  Not stream-ordered: change it only while no run of the handle is
+ * in flight.
  */
-sv_status specverify_set_launch(specverify_t h, int cluster_ctas, int threads);
-sv_status specverify_get_launch(specverify_t h, int *cluster_ctas, int *threads);
+sv_status specverify_set_launch(specverify_t h, int slices, int threads);
+/* Current shape and the largest `slices` this handle accepts (any pointer may be NULL). */
+sv_status specverify_get_launch(specverify_t h, int *slices, int *threads, int *max_slices);
+
+/*
+ * Per-kernel timing of the next `max_runs` runs of the handle: each run then
+ * records CUDA events on its stream around its two kernels (the statistics
+ * kernel, which streams every logit, and the decide-and-draw kernel).  Waits
+ * for the device first; re-arming discards earlier records.
+ */
+sv_status specverify_profile_begin(specverify_t h, int max_runs);
+
+/*
+ * Wait for the last recorded run, store the mean device time per run of each
+ * kernel in milliseconds (any pointer may be NULL) and the number of runs
+ * recorded, and stop recording.
+ */
+sv_status specverify_profile_end(specverify_t h, float *stats_ms, float *draw_ms, int *runs);
 
 /* Static text for a status code. */
 const char *specverify_status_string(sv_status s);

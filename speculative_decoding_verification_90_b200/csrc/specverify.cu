@@ -1,7 +1,7 @@
 // C ABI of the speculative-sampling verification library (see specverify.h).
 //
-// Host side only: argument checks, the workspace, the launch shape, the
-// cluster launch of the fused kernel, host-buffer staging and readbacks.
+// Host side only: argument checks, the workspace, the launch shapes, the
+// three stream-ordered launches of one step, host-buffer staging, readbacks.
 #include "specverify.h"
 
 #include <cuda_runtime.h>
@@ -15,25 +15,36 @@
 
 #include "verify_kernel.cuh"
 
+using specverify::CtaStats;
 using specverify::Params;
 using specverify::PosInfo;
 using specverify::RowStat;
+using specverify::SeqDecision;
 
 struct specverify_ctx {
   int device = 0;
   int batch = 0, gamma = 0, vocab = 0;
   sv_dtype dtype = SV_DTYPE_F32;
-  int cluster = 1, threads = 256;
+  int slices = 1, threads = 128;
+  int max_slices = 1;  // the partial-statistics workspace holds this many per position
+  int draw_slices = 1; // draw blocks per sequence
   int num_sms = 148;
   void* ws = nullptr;  // one device allocation for the whole workspace
+  CtaStats* partial = nullptr;
   RowStat* tstat = nullptr;
   RowStat* dstat = nullptr;
   PosInfo* pos = nullptr;
+  SeqDecision* decision = nullptr;
+  double* draw_mass = nullptr;
+  unsigned* draw_ticket = nullptr;
   double* resid = nullptr;
-  unsigned* ticket = nullptr;
   unsigned* status = nullptr;
   void* stage = nullptr;  // device staging for host-buffer runs
   size_t stage_bytes = 0;
+  // optional per-kernel timing: 3 events per recorded run
+  std::vector<cudaEvent_t> events;
+  int prof_capacity = 0;
+  int prof_runs = 0;
 };
 
 namespace {
@@ -74,57 +85,101 @@ long num_groups(const specverify_ctx* h) {
   return (static_cast<long>(h->vocab) + ve - 1) / ve;
 }
 
-// Default launch shape.  A position's rows are split over `cluster` CTAs;
-// aim for at least eight waves of CTAs over the SMs (so the last partial
-// wave costs little) while keeping every thread at two or more 16-byte
-// groups per row.
+// Default launch shape of the statistics kernel: 128 threads per block, a
+// position's two rows split over `slices` blocks (at most 8) so that the
+// grid holds at least eight waves of blocks where the batch allows (the
+// last, partial wave then costs little), with at least one 16-byte group
+// per thread and row.
 void default_shape(specverify_ctx* h) {
-  const int threads = 256;
+  const int threads = 128;
   const long positions = static_cast<long>(h->batch) * (h->gamma + 1);
-  const long slots = static_cast<long>(h->num_sms) * (2048 / threads);
+  const long slots = static_cast<long>(h->num_sms) * (1024 / threads);
   const long ngroups = num_groups(h);
   int best = 1;
-  for (int c = 1; c <= specverify::kMaxCluster; ++c) {
-    if (ngroups / c < 2L * threads && c > 1) break;
+  // more than 8 slices only lengthens the decision kernel's combine
+  const int cap = h->max_slices < 8 ? h->max_slices : 8;
+  for (int c = 1; c <= cap; ++c) {
+    if (ngroups / c < threads && c > 1) break;
     best = c;
     if (positions * c >= 8 * slots) break;
   }
-  h->cluster = best;
+  h->slices = best;
   h->threads = threads;
 }
 
-template <typename T, int NT, bool A>
-cudaError_t launch_shape(const Params& p, int C, long positions, cudaStream_t s) {
+// Draw blocks per sequence: about 48 KB of the rows drawn from per block,
+// more when the batch is too small to fill the SMs, and at least one
+// 32-group tile per warp.
+int draw_shape(const specverify_ctx* h) {
+  const long bytes = 2L * h->vocab * static_cast<long>(elem_size(h->dtype));
+  long s2 = (bytes + 49151) / 49152;
+  const long slots = static_cast<long>(h->num_sms) * 8;
+  if (h->batch > 0) {
+    const long fill = (slots + h->batch - 1) / h->batch;
+    if (s2 < fill) s2 = fill;
+  }
+  const long ntiles = (num_groups(h) + specverify::kTile - 1) / specverify::kTile;
+  const long by_tiles = ntiles / specverify::kDrawWarps;
+  if (s2 > by_tiles) s2 = by_tiles;
+  if (s2 > 64) s2 = 64;
+  if (s2 < 1) s2 = 1;
+  return static_cast<int>(s2);
+}
+
+template <typename K>
+cudaError_t launch_pdl(K kernel, unsigned blocks, unsigned threads, cudaStream_t s, const Params& p) {
+  // programmatic dependent launch: the kernel may be scheduled before its
+  // predecessor on the stream has finished; it waits in a grid-dependency
+  // barrier before it reads the predecessor's results
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(positions * C), 1, 1);
-  cfg.blockDim = dim3(NT, 1, 1);
+  cfg.gridDim = dim3(blocks, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(C);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, specverify::verify_kernel<T, NT, A>, p);
+  return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
+template <typename T, int NT, bool A>
+cudaError_t launch_stats_nt(const Params& p, long blocks, cudaStream_t s) {
+  specverify::stats_kernel<T, NT, A><<<static_cast<unsigned>(blocks), NT, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// events[0..2] (may be null): before stats, after stats, after draw
 template <typename T, bool A>
-cudaError_t launch_threads(const Params& p, int C, int NT, long positions, cudaStream_t s) {
+cudaError_t launch_step(const Params& p, int NT, cudaStream_t s, cudaEvent_t* ev) {
+  const long positions = static_cast<long>(p.batch) * (p.gamma + 1);
+  const long blocks = positions * p.slices;
+  cudaError_t e = cudaSuccess;
+  if (ev) e = cudaEventRecord(ev[0], s);
+  if (e != cudaSuccess) return e;
   switch (NT) {
-    case 128: return launch_shape<T, 128, A>(p, C, positions, s);
-    case 256: return launch_shape<T, 256, A>(p, C, positions, s);
-    case 512: return launch_shape<T, 512, A>(p, C, positions, s);
+    case 128: e = launch_stats_nt<T, 128, A>(p, blocks, s); break;
+    case 256: e = launch_stats_nt<T, 256, A>(p, blocks, s); break;
+    case 512: e = launch_stats_nt<T, 512, A>(p, blocks, s); break;
     default: return cudaErrorInvalidValue;
   }
+  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
+  if (e != cudaSuccess) return e;
+  const int per = specverify::kDecideThreads / specverify::kWarp;
+  e = launch_pdl(specverify::decide_kernel<T>, static_cast<unsigned>((p.batch + per - 1) / per),
+                 specverify::kDecideThreads, s, p);
+  if (e != cudaSuccess) return e;
+  e = launch_pdl(specverify::draw_kernel<T, A>,
+                 static_cast<unsigned>(static_cast<long>(p.batch) * p.draw_slices),
+                 specverify::kDrawThreads, s, p);
+  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
+  return e;
 }
 
 template <typename T>
-cudaError_t launch_dtype(const Params& p, int C, int NT, bool aligned, long positions,
-                         cudaStream_t s) {
-  return aligned ? launch_threads<T, true>(p, C, NT, positions, s)
-                 : launch_threads<T, false>(p, C, NT, positions, s);
+cudaError_t launch_dtype(const Params& p, int NT, bool aligned, cudaStream_t s, cudaEvent_t* ev) {
+  return aligned ? launch_step<T, true>(p, NT, s, ev) : launch_step<T, false>(p, NT, s, ev);
 }
 
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -159,28 +214,37 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
   p.u_resample = u_resample;
   p.out_tokens = out_tokens;
   p.out_num_accepted = out_num_accepted;
+  p.partial = h->partial;
   p.tstat = h->tstat;
   p.dstat = h->dstat;
   p.pos = h->pos;
+  p.decision = h->decision;
+  p.draw_mass = h->draw_mass;
+  p.draw_ticket = h->draw_ticket;
   p.resid_mass = h->resid;
-  p.ticket = h->ticket;
   p.status = h->status;
   p.batch = h->batch;
   p.gamma = G;
   p.vocab = h->vocab;
   const long ngroups = num_groups(h);
-  p.groups_per_cta = static_cast<int>((ngroups + h->cluster - 1) / h->cluster);
+  p.slices = h->slices;
+  p.groups_per_slice = static_cast<int>((ngroups + h->slices - 1) / h->slices);
+  p.draw_slices = h->draw_slices;
+  {
+    const long ntiles = (ngroups + specverify::kTile - 1) / specverify::kTile;
+    p.groups_per_draw = static_cast<int>((ntiles + h->draw_slices - 1) / h->draw_slices) * specverify::kTile;
+  }
   p.c_hi = c_hi;
   p.c_lo = c_lo;
-  p.c = c;
+  p.c = static_cast<double>(c_hi) + static_cast<double>(c_lo);
 
   const bool aligned = aligned_to(target, 16) && (G == 0 || aligned_to(draft, 16)) &&
                        (static_cast<size_t>(h->vocab) * es) % 16 == 0;
-  const long positions = static_cast<long>(h->batch) * (G + 1);
+  cudaEvent_t* ev = nullptr;
+  if (h->prof_runs < h->prof_capacity) ev = h->events.data() + 3 * (h->prof_runs++);
   cudaError_t e = (h->dtype == SV_DTYPE_BF16)
-                      ? launch_dtype<__nv_bfloat16>(p, h->cluster, h->threads, aligned,
-                                                    positions, stream)
-                      : launch_dtype<float>(p, h->cluster, h->threads, aligned, positions, stream);
+                      ? launch_dtype<__nv_bfloat16>(p, h->threads, aligned, stream, ev)
+                      : launch_dtype<float>(p, h->threads, aligned, stream, ev);
   if (e != cudaSuccess) return cuda_fail(e);
   return SV_OK;
 }
@@ -193,11 +257,11 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
                             int device) {
   if (!out) return SV_ERR_INVALID_ARG;
   *out = nullptr;
-  if (batch < 0 || gamma < 0 || gamma > 4096 || vocab < 1 || vocab > (1 << 30))
+  if (batch < 0 || gamma < 0 || gamma > specverify::kMaxGamma || vocab < 1 || vocab > (1 << 30))
     return SV_ERR_INVALID_ARG;
   if (dtype != SV_DTYPE_F32 && dtype != SV_DTYPE_BF16) return SV_ERR_INVALID_ARG;
   const long positions = static_cast<long>(batch) * (gamma + 1);
-  if (positions * specverify::kMaxCluster > 0x7fffffffL) return SV_ERR_INVALID_ARG;
+  if (positions * specverify::kMaxSlices > 0x7fffffffL) return SV_ERR_INVALID_ARG;
   int ndev = 0;
   cudaError_t e = cudaGetDeviceCount(&ndev);
   if (e != cudaSuccess) return cuda_fail(e);
@@ -222,28 +286,49 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   h->vocab = vocab;
   h->dtype = dtype;
   h->num_sms = prop.multiProcessorCount;
+  {
+    // at most one slice per 128 groups (2 KB of bf16 logits) and 64 in all
+    const long cap = num_groups(h) / 128;
+    h->max_slices = static_cast<int>(cap < 1 ? 1 : (cap > specverify::kMaxSlices ? specverify::kMaxSlices : cap));
+  }
   default_shape(h);
 
   const size_t nT = static_cast<size_t>(batch) * (gamma + 1);
   const size_t nD = static_cast<size_t>(batch) * gamma;
-  const size_t offT = 0;
-  const size_t offD = round_up(offT + nT * sizeof(RowStat), 256);
-  const size_t offP = round_up(offD + nD * sizeof(RowStat), 256);
-  const size_t offR = round_up(offP + nD * sizeof(PosInfo), 256);
-  const size_t offK = round_up(offR + static_cast<size_t>(batch) * sizeof(double), 256);
-  const size_t offS = round_up(offK + static_cast<size_t>(batch) * sizeof(unsigned), 256);
-  const size_t total = offS + 256;
+  const size_t nB = static_cast<size_t>(batch);
+  h->draw_slices = draw_shape(h);
+  const size_t nPart = nT * static_cast<size_t>(h->max_slices);
+  const size_t nDraw = nB * static_cast<size_t>((num_groups(h) + specverify::kTile - 1) / specverify::kTile);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = round_up(off + bytes, 256);
+    return at;
+  };
+  const size_t offA = take(nPart * sizeof(CtaStats));
+  const size_t offT = take(nT * sizeof(RowStat));
+  const size_t offD = take(nD * sizeof(RowStat));
+  const size_t offP = take(nD * sizeof(PosInfo));
+  const size_t offC = take(nB * sizeof(SeqDecision));
+  const size_t offW = take(nDraw * sizeof(double));
+  const size_t offK = take(nB * sizeof(unsigned));
+  const size_t offR = take(nB * sizeof(double));
+  const size_t offS = take(sizeof(unsigned));
+  const size_t total = off;
   e = cudaMalloc(&h->ws, total);
   if (e != cudaSuccess) {
     delete h;
     return cuda_fail(e);
   }
   char* base = static_cast<char*>(h->ws);
+  h->partial = reinterpret_cast<CtaStats*>(base + offA);
   h->tstat = reinterpret_cast<RowStat*>(base + offT);
   h->dstat = reinterpret_cast<RowStat*>(base + offD);
   h->pos = reinterpret_cast<PosInfo*>(base + offP);
+  h->decision = reinterpret_cast<SeqDecision*>(base + offC);
+  h->draw_mass = reinterpret_cast<double*>(base + offW);
+  h->draw_ticket = reinterpret_cast<unsigned*>(base + offK);
   h->resid = reinterpret_cast<double*>(base + offR);
-  h->ticket = reinterpret_cast<unsigned*>(base + offK);
   h->status = reinterpret_cast<unsigned*>(base + offS);
   e = cudaMemset(h->ws, 0, total);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
@@ -331,6 +416,7 @@ void specverify_destroy(specverify_t h) {
     DeviceScope scope(h->device);
     if (scope.ok()) {
       cudaDeviceSynchronize();
+      for (cudaEvent_t ev : h->events) cudaEventDestroy(ev);
       if (h->stage) cudaFree(h->stage);
       if (h->ws) cudaFree(h->ws);
     }
@@ -355,10 +441,9 @@ sv_status specverify_get_status(specverify_t h, void* stream, uint32_t* bits) {
   return SV_OK;
 }
 
-sv_status specverify_debug_readback(specverify_t h, float* target_max, double* target_sum,
-                                   float* draft_max, double* draft_sum, double* q_tok,
-                                   double* p_tok, double* ratio, double* resid_mass,
-                                   void* stream) {
+sv_status specverify_debug_readback(specverify_t h, double* target_lse, double* draft_lse,
+                                   double* q_tok, double* p_tok, double* ratio,
+                                   double* resid_mass, void* stream) {
   if (!h) return SV_ERR_INVALID_ARG;
   DeviceScope scope(h->device);
   if (!scope.ok()) return SV_ERR_CUDA;
@@ -374,13 +459,11 @@ sv_status specverify_debug_readback(specverify_t h, float* target_max, double* t
   if (e == cudaSuccess && nD) e = cudaMemcpy(ps.data(), h->pos, nD * sizeof(PosInfo), cudaMemcpyDeviceToHost);
   if (e == cudaSuccess && h->batch) e = cudaMemcpy(rm.data(), h->resid, h->batch * sizeof(double), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e);
-  for (size_t i = 0; i < nT; ++i) {
-    if (target_max) target_max[i] = ts[i].max;
-    if (target_sum) target_sum[i] = ts[i].sum;
-  }
+  const double ln2 = 0.69314718055994530942;
+  for (size_t i = 0; i < nT; ++i)
+    if (target_lse) target_lse[i] = ts[i].lse2 * ln2;
   for (size_t i = 0; i < nD; ++i) {
-    if (draft_max) draft_max[i] = ds[i].max;
-    if (draft_sum) draft_sum[i] = ds[i].sum;
+    if (draft_lse) draft_lse[i] = ds[i].lse2 * ln2;
     if (q_tok) q_tok[i] = ps[i].q_tok;
     if (p_tok) p_tok[i] = ps[i].p_tok;
     if (ratio) ratio[i] = ps[i].ratio;
@@ -390,19 +473,66 @@ sv_status specverify_debug_readback(specverify_t h, float* target_max, double* t
   return SV_OK;
 }
 
-sv_status specverify_set_launch(specverify_t h, int cluster_ctas, int threads) {
+sv_status specverify_set_launch(specverify_t h, int slices, int threads) {
   if (!h) return SV_ERR_INVALID_ARG;
-  if (cluster_ctas < 1 || cluster_ctas > specverify::kMaxCluster) return SV_ERR_INVALID_ARG;
+  if (slices < 1 || slices > h->max_slices) return SV_ERR_INVALID_ARG;
   if (threads != 128 && threads != 256 && threads != 512) return SV_ERR_INVALID_ARG;
-  h->cluster = cluster_ctas;
+  h->slices = slices;
   h->threads = threads;
   return SV_OK;
 }
 
-sv_status specverify_get_launch(specverify_t h, int* cluster_ctas, int* threads) {
+sv_status specverify_get_launch(specverify_t h, int* slices, int* threads, int* max_slices) {
   if (!h) return SV_ERR_INVALID_ARG;
-  if (cluster_ctas) *cluster_ctas = h->cluster;
+  if (max_slices) *max_slices = h->max_slices;
+  if (slices) *slices = h->slices;
   if (threads) *threads = h->threads;
+  return SV_OK;
+}
+
+sv_status specverify_profile_begin(specverify_t h, int max_runs) {
+  if (!h || max_runs < 0 || max_runs > (1 << 20)) return SV_ERR_INVALID_ARG;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  for (cudaEvent_t ev : h->events) cudaEventDestroy(ev);
+  h->events.clear();
+  h->prof_runs = 0;
+  h->prof_capacity = 0;
+  for (int i = 0; i < 3 * max_runs; ++i) {
+    cudaEvent_t ev;
+    e = cudaEventCreate(&ev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    h->events.push_back(ev);
+  }
+  h->prof_capacity = max_runs;
+  return SV_OK;
+}
+
+sv_status specverify_profile_end(specverify_t h, float* stats_ms, float* draw_ms, int* runs) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  const int n = h->prof_runs;
+  double t[2] = {0.0, 0.0};
+  cudaError_t e = cudaSuccess;
+  if (n > 0) e = cudaEventSynchronize(h->events[3 * (n - 1) + 2]);
+  for (int r = 0; r < n && e == cudaSuccess; ++r) {
+    for (int k = 0; k < 2 && e == cudaSuccess; ++k) {
+      float ms = 0.f;
+      e = cudaEventElapsedTime(&ms, h->events[3 * r + k], h->events[3 * r + k + 1]);
+      t[k] += ms;
+    }
+  }
+  for (cudaEvent_t ev : h->events) cudaEventDestroy(ev);
+  h->events.clear();
+  h->prof_capacity = 0;
+  h->prof_runs = 0;
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (stats_ms) *stats_ms = n ? static_cast<float>(t[0] / n) : 0.f;
+  if (draw_ms) *draw_ms = n ? static_cast<float>(t[1] / n) : 0.f;
+  if (runs) *runs = n;
   return SV_OK;
 }
 

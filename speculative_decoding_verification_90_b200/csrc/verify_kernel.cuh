@@ -1,42 +1,49 @@
-// Fused speculative-sampling verification kernel for sm_100a.
+// Speculative-sampling verification kernels for sm_100a.
 //
-// One thread-block cluster of C CTAs owns one position (b, j), j = 0..gamma,
-// of one sequence: target row (b, j) and, for j < gamma, draft row (b, j).
-// Each CTA owns a contiguous slice of the vocabulary of both rows.
+// One verification step is three stream-ordered kernels (each later one
+// launched early through programmatic dependent launch and waiting for its
+// predecessor with a grid-dependency barrier):
 //
-//   phase 1  single streaming pass over the slice with 128-bit coalesced
-//            loads; online (max, sum of exp) per thread, reduced per CTA and
-//            combined across the cluster through distributed shared memory
-//            ("softmax statistics", step 1 of the round);
-//   phase 2  rank 0 forms q(t), p(t) and the ratio for the position's draft
-//            token and records accept / reject (step 2, min(1, q/p));
-//   phase 3  an atomic ticket per sequence elects the cluster that finishes
-//            last; it scans the gamma decisions with a warp ballot to find
-//            the first rejection n (step 3);
-//   phase 4  that cluster re-reads one row pair (n < gamma: max(0, q_n - p_n))
-//            or one row (n == gamma: q_gamma) - rows that the sequence's other
-//            clusters have just streamed, so they come from L2 - sums the
-//            mass per warp and per CTA, exchanges the CTA sums through
-//            distributed shared memory, and the CTA and warp that hold
-//            u * Z locate the drawn token with a warp prefix scan (step 4).
+//   stats   S blocks per position (b, j), j = 0..gamma, each streaming its
+//           contiguous 1/S of the vocabulary of target row (b, j) and, for
+//           j < gamma, draft row (b, j) with 128-bit coalesced loads; each
+//           thread keeps a running sum of 2^(x c - o) against a lazily raised
+//           offset o; the block writes its (o, sum) partial (step 1 of the
+//           round: softmax statistics).  No atomics, no waits: this is the
+//           kernel that moves all of the logit bytes.
+//   decide  one warp per sequence, one lane per position: the lane combines
+//           the position's partials into log2 sum_i 2^(x_i c), forms q(t),
+//           p(t) and the ratio, and a warp ballot finds the first rejection n
+//           (steps 2 and 3); writes the accepted prefix and what to draw from.
+//   draw    S' blocks per sequence over the rows drawn from (n < gamma:
+//           max(0, q_n - p_n) from target and draft row n; n == gamma: q of
+//           target row gamma); each block publishes the mass of every
+//           32-group tile of its share, and the block that takes the
+//           sequence's ticket last finds, by a block-wide prefix scan over
+//           the tile masses, the tile that holds u * Z and scans it one group
+//           per lane in index order (step 4).
+//
+// No thread ever waits for another block (the only hand-off inside a kernel
+// is an atomic ticket, never a spin).
 //
 // Pages (title, section): "Speculative decoding - the small model writes first
 // and the big model checks", section 1 (rule); "Speculative decoding: how to
 // run big models fast", section "How it works" (steps, bonus token, 1..gamma+1
 // tokens per call, temperature).
 //
-// Numerics: exponentials are base 2 with log2(e)/T split into two floats
-// (c_hi + c_lo, c_lo > 0) so that the argument d * c carries no systematic
-// rounding of the constant; per-thread sums are fp32, everything above a
-// thread (warp, CTA, cluster, ratio, CDF positions) is fp64.  In the residual
-// q - p is formed as p * (2^L - 1) with L = log2(q/p) computed from the logit
-// difference, which keeps it accurate where q and p nearly cancel.
-//
-// No thread ever waits on another cluster: cross-cluster hand-off is a ticket
-// (atomicAdd), never a spin.  Data errors set bits of a status word.
+// Numerics.  c = log2(e)/T is carried as two floats c_hi + c_lo (c_lo > 0).
+// Every exponent argument is x c_hi - o + x c_lo, two FMAs whose only
+// rounding is relative to the (small) result, so no rounding of c or of a
+// large offset ever becomes a systematic factor on the probabilities.  The
+// offset o of a thread is any float near its largest x c seen so far; it is
+// raised only when a group's sum leaves [0, 2^100), so the streaming loop has
+// no max pass.  Per-thread sums are fp32; everything above a thread (warp,
+// block, position, ratio, CDF positions) is fp64.  In the residual q - p is
+// formed as p (2^L - 1) with L = log2(q/p) taken from the logit difference,
+// which keeps it accurate where q and p nearly cancel.  Data errors set bits
+// of a status word; nothing traps.
 #pragma once
 
-#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -45,22 +52,20 @@
 
 namespace specverify {
 
-namespace cg = cooperative_groups;
-
 constexpr int kWarp = 32;
-constexpr int kMaxCluster = 8;
+constexpr int kMaxSlices = 64;
 
 // per-position decision flags
 enum : int { kFlagReject = 0, kFlagAccept = 1, kFlagTokenRange = 2, kFlagNonFinite = 3 };
 // status word bits
 enum : unsigned { kStatTokenRange = 1u, kStatNonFinite = 2u, kStatZeroMass = 4u };
-// what the finishing cluster draws from
+// what the draw kernel draws from
 enum : int { kDrawResidual = 0, kDrawTarget = 1, kDrawNone = 2 };
 
 struct RowStat {
-  double sum;  // sum_i 2^((x_i - max) * c)
-  float max;   // max_i x_i
-  int valid;   // 1 if the row is finite with at least one finite entry
+  double lse2;  // log2 sum_i 2^(x_i c) = log2 sum_i exp(x_i / T) / ln 2
+  int valid;    // 1 if the row is finite with at least one finite entry
+  int pad;
 };
 
 struct PosInfo {
@@ -68,6 +73,23 @@ struct PosInfo {
   double p_tok;
   double ratio;
   int flag;
+  int pad;
+};
+
+// one block's partial statistics of its slice of the position's two rows:
+// sum_i 2^(x_i c - o) against offset o, for the target and the draft row
+struct __align__(16) CtaStats {
+  double sT, sD;
+  float oT, oD;
+  int pad[2];
+};
+
+// per sequence, from the decide kernel to the draw kernel
+struct SeqDecision {
+  double lT, lD;       // log2 sum 2^(x c) of the rows drawn from
+  int n;               // accepted drafts
+  int mode;            // kDraw*
+  unsigned stat_bits;  // data errors found
   int pad;
 };
 
@@ -79,16 +101,22 @@ struct Params {
   const float* u_resample;   // [B]
   int32_t* out_tokens;       // [B, G+1]
   int32_t* out_num_accepted; // [B]
+  CtaStats* partial;         // [B*(G+1)*S] per-block partial statistics
   RowStat* tstat;            // [B*(G+1)]
   RowStat* dstat;            // [B*G]
   PosInfo* pos;              // [B*G]
+  SeqDecision* decision;     // [B]
+  double* draw_mass;         // [B * tiles of a row] mass of each 32-group tile of the draw
+  unsigned* draw_ticket;     // [B], zero between launches
   double* resid_mass;        // [B]
-  unsigned* ticket;          // [B], zero between launches
   unsigned* status;          // [1]
   int batch, gamma, vocab;
-  int groups_per_cta;        // 16-byte groups of the vocabulary per CTA
+  int slices;                // S stats blocks per position
+  int groups_per_slice;      // 16-byte groups of the vocabulary per stats block
+  int draw_slices;           // S2 draw blocks per sequence
+  int groups_per_draw;       // groups per draw block (whole 32-group tiles)
   float c_hi, c_lo;          // log2(e)/T = c_hi + c_lo, c_lo > 0
-  double c;                  // log2(e)/T
+  double c;                  // c_hi + c_lo, exactly
 };
 
 // ---------------------------------------------------------------------------
@@ -175,35 +203,60 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// d * log2(e)/T with the constant carried in two parts; c_lo > 0 keeps
-// d = -inf mapping to -inf (never inf * 0)
-__device__ __forceinline__ float scaled(float d, float c_hi, float c_lo) {
-  return fmaf(d, c_hi, d * c_lo);
+// x c - o with c = c_hi + c_lo: two FMAs; x = -inf gives -inf (c_lo > 0, so
+// never inf * 0), and the rounding is relative to the result only
+__device__ __forceinline__ float arg2(float x, float c_hi, float c_lo, float o) {
+  return fmaf(x, c_lo, fmaf(x, c_hi, -o));
+}
+
+// x c - (l_hi + l_lo), for an offset known to double precision
+__device__ __forceinline__ float arg2l(float x, float c_hi, float c_lo, float l_hi, float l_lo) {
+  return fmaf(x, c_hi, -l_hi) + fmaf(x, c_lo, -l_lo);
 }
 
 // ---------------------------------------------------------------------------
-// phase 1: online softmax statistics
+// phase 1: streaming softmax statistics
 // ---------------------------------------------------------------------------
 
+constexpr float kGroupSumLimit = 1.2676506e30f;  // 2^100
+
+// Adds one group to (o, s): s = sum 2^(x c - o).  The fast path is two FMAs,
+// one ex2 and one add per element; the offset is raised (and the group
+// recomputed) only when the group's sum is not in [0, 2^100): the first
+// group (o = -inf), a much larger logit, +inf or NaN.
 template <typename T>
-__device__ __forceinline__ void accumulate_group(const uint4& v, float& m, float& s, float c_hi,
+__device__ __forceinline__ void accumulate_group(const uint4& v, float& o, float& s, float c_hi,
                                                  float c_lo) {
   constexpr int kVec = Elem<T>::kVec;
   float x[kVec];
   Elem<T>::unpack(v, x);
-  float cm = x[0];
+  float sg = 0.f;
 #pragma unroll
-  for (int k = 1; k < kVec; ++k) cm = fmaxf(cm, x[k]);
-  if (cm > m) {
-    // (m - cm) is -inf while m is -inf: the factor is 0 and s stays 0 (or NaN)
-    s *= ex2(scaled(m - cm, c_hi, c_lo));
-    m = cm;
+  for (int k = 0; k < kVec; ++k) sg += ex2(arg2(x[k], c_hi, c_lo, o));
+  if (!(sg < kGroupSumLimit)) {
+    float gm = -INFINITY;
+    bool nan = false;
+#pragma unroll
+    for (int k = 0; k < kVec; ++k) {
+      gm = fmaxf(gm, x[k]);
+      nan |= (x[k] != x[k]);
+    }
+    if (nan || gm == INFINITY) {
+      sg = NAN;  // the row is invalid; the NaN marks it through every sum
+    } else if (gm == -INFINITY) {
+      sg = 0.f;  // the group has no mass
+    } else {
+      const float on = gm * c_hi;
+      if (on > o) {
+        s *= ex2(o - on);  // o = -inf: s is 0 (or NaN) and stays so
+        o = on;
+      }
+      sg = 0.f;
+#pragma unroll
+      for (int k = 0; k < kVec; ++k) sg += ex2(arg2(x[k], c_hi, c_lo, o));
+    }
   }
-  const float ms = (m == -INFINITY) ? 0.f : m;
-  float acc = 0.f;
-#pragma unroll
-  for (int k = 0; k < kVec; ++k) acc += ex2(scaled(x[k] - ms, c_hi, c_lo));
-  s += acc;
+  s += sg;
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -224,7 +277,7 @@ __device__ __forceinline__ int warp_maxi(int v) {
   return v;
 }
 
-// contiguous group range [lo, hi) of warp `w` inside the CTA range [clo, chi)
+// contiguous group range [lo, hi) of warp `w` inside the range [clo, chi)
 __device__ __forceinline__ void warp_range(long clo, long chi, int w, int nwarps, long& lo,
                                            long& hi) {
   long n = chi - clo;
@@ -235,41 +288,35 @@ __device__ __forceinline__ void warp_range(long clo, long chi, int w, int nwarps
   if (hi > chi) hi = chi;
 }
 
-struct __align__(16) CtaStats {
-  double sT, sD;
-  float mT, mD;
-  int pad[2];
-};
-
-struct __align__(16) Bcast {
-  double sT, sD;       // row sums of the rows drawn from
-  float mT, mD;        // row maxima
-  int last;            // this cluster finishes the sequence
-  int n;               // accepted drafts
-  int mode;            // kDraw*
-  int trow, drow;      // target / draft position of the draw (drow < 0: none)
-  unsigned stat_bits;  // status bits to raise
-  int pad[2];
-};
-
-struct __align__(16) CtaMass {
-  double z;     // residual mass of the CTA slice
-  int last_pos; // last index with r > 0 in the slice, -1 if none
-  int pad;
-};
-
 // ---------------------------------------------------------------------------
 // phase 4 helpers: residual mass of one group
 // ---------------------------------------------------------------------------
 
 struct DrawConsts {
   float c_hi, c_lo;
-  float mT, mD;      // row maxima
-  float invST, invSD;
-  float k_hi, k_lo;  // K = (mT - mD) * c + log2(sT / sD), two-float
+  float lt_hi;   // log2 sum 2^(x c) of the target row, rounded to float ...
+  float ld_hi;   // ... and of the draft row
+  float k_hi, k_lo;  // K = lT - lD, two-float
+  float rD;      // 2^(lt_lo - ld_lo): the draft's share of the two roundings
+  float fT;      // 2^(-lt_lo): applied to every sum of group masses
 };
 
-// r for the VEC elements of one group: residual max(0, q - p) or target q
+// Taylor coefficients of 2^L - 1 = sum_k (ln 2)^k L^k / k!, k = 1..6
+constexpr float kA1 = 0.6931471805599453f;
+constexpr float kA2 = 0.2402265069591007f;
+constexpr float kA3 = 0.055504108664821576f;
+constexpr float kA4 = 0.009618129107628477f;
+constexpr float kA5 = 0.0013333558146428441f;
+constexpr float kA6 = 0.00015403530393381606f;
+
+// r / fT for the VEC elements of one group: residual max(0, q - p) or target
+// q; the caller multiplies sums of r by fT.  Branch-free: L = log2(q/p)
+// comes from the logit difference (exact for bf16 inputs); L <= 0 gives 0,
+// L >= 1/4 gives q - p (q >= 1.19 p, so at most 2.6 bits cancel),
+// 0 < L < 1/4 gives p (2^L - 1) from its Taylor series in L (to L^6,
+// truncation below 6e-9 relative).  The infinite cases need no test: a
+// draft logit of -inf gives L = +inf and r = q - 0; a target logit of -inf
+// gives L = -inf (or NaN) and r = 0.
 template <typename T, int kMode>
 __device__ __forceinline__ void group_mass(const uint4& vt, const uint4& vd, const DrawConsts& k,
                                            float (&r)[Elem<T>::kVec]) {
@@ -278,466 +325,528 @@ __device__ __forceinline__ void group_mass(const uint4& vt, const uint4& vd, con
   Elem<T>::unpack(vt, xt);
   if constexpr (kMode == kDrawTarget) {
 #pragma unroll
-    for (int e = 0; e < kVec; ++e) r[e] = ex2(scaled(xt[e] - k.mT, k.c_hi, k.c_lo)) * k.invST;
+    for (int e = 0; e < kVec; ++e) r[e] = ex2(arg2(xt[e], k.c_hi, k.c_lo, k.lt_hi));
   } else {
     float xd[kVec];
     Elem<T>::unpack(vd, xd);
 #pragma unroll
     for (int e = 0; e < kVec; ++e) {
-      const float q = ex2(scaled(xt[e] - k.mT, k.c_hi, k.c_lo)) * k.invST;
-      const float p = ex2(scaled(xd[e] - k.mD, k.c_hi, k.c_lo)) * k.invSD;
-      float res;
-      if (!(q > 0.f)) {
-        res = 0.f;                     // target gives the token no mass
-      } else if (xd[e] == -INFINITY) {
-        res = q;                       // draft gives it none: all of q is residual
-      } else {
-        // L = log2(q/p) from the logit difference (exact for bf16 inputs)
-        const float dx = xt[e] - xd[e];
-        const float L = fmaf(dx, k.c_hi, -k.k_hi) + fmaf(dx, k.c_lo, -k.k_lo);
-        if (!(L > 0.f)) {
-          res = 0.f;
-        } else if (L >= 1.f) {
-          res = q - p;                 // q >= 2p: no cancellation
-        } else {
-          // 2^L - 1 = e^y - 1, y = L ln 2 in (0, 0.694): Taylor series to y^10
-          const float y = L * 0.69314718055994531f;
-          float t = 2.755731922398589e-7f;           // 1/10!
-          t = fmaf(t, y, 2.755731922398589e-6f);     // 1/9!
-          t = fmaf(t, y, 2.480158730158730e-5f);     // 1/8!
-          t = fmaf(t, y, 1.984126984126984e-4f);     // 1/7!
-          t = fmaf(t, y, 1.388888888888889e-3f);     // 1/6!
-          t = fmaf(t, y, 8.333333333333333e-3f);     // 1/5!
-          t = fmaf(t, y, 4.166666666666667e-2f);     // 1/4!
-          t = fmaf(t, y, 1.666666666666667e-1f);     // 1/3!
-          t = fmaf(t, y, 0.5f);                      // 1/2!
-          t = fmaf(t, y, 1.0f);                      // 1/1!
-          res = p * (t * y);
-        }
-      }
-      r[e] = res;
+      const float q = ex2(arg2(xt[e], k.c_hi, k.c_lo, k.lt_hi));
+      const float p = ex2(arg2(xd[e], k.c_hi, k.c_lo, k.ld_hi)) * k.rD;
+      const float dx = xt[e] - xd[e];
+      const float L = fmaf(dx, k.c_hi, -k.k_hi) + fmaf(dx, k.c_lo, -k.k_lo);
+      float t = kA6;
+      t = fmaf(t, L, kA5);
+      t = fmaf(t, L, kA4);
+      t = fmaf(t, L, kA3);
+      t = fmaf(t, L, kA2);
+      t = fmaf(t, L, kA1);
+      const float small = p * (t * L);
+      const float res = (L >= 0.25f) ? q - p : small;
+      r[e] = (L > 0.f) ? res : 0.f;
     }
   }
 }
 
+__device__ __forceinline__ void split2(double v, float& hi, float& lo) {
+  hi = static_cast<float>(v);
+  lo = static_cast<float>(v - static_cast<double>(hi));
+}
+
 // ---------------------------------------------------------------------------
-// the kernel
+// block-level helpers
 // ---------------------------------------------------------------------------
 
-template <typename T, int NT, bool kAligned>
-__global__ void __launch_bounds__(NT) verify_kernel(const Params P) {
-  constexpr int kVec = Elem<T>::kVec;
+// Streaming statistics of one block's slice of the two rows, reduced to the
+// block (offset = the block's largest thread offset); valid in thread 0.
+template <typename T, int NT, bool kAligned, int kUnroll>
+__device__ __forceinline__ CtaStats slice_stats(const T* rowT, const T* rowD, bool has_draft,
+                                                long glo, long ghi, int V, float c_hi,
+                                                float c_lo) {
   constexpr int kNW = NT / kWarp;
-  constexpr int kUnroll = 4;
-
-  cg::cluster_group cluster = cg::this_cluster();
-  const int C = static_cast<int>(cluster.num_blocks());
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int tid = threadIdx.x;
-  const int lane = tid & (kWarp - 1);
-  const int warp = tid >> 5;
-
-  const int G = P.gamma;
-  const int V = P.vocab;
-  const long position = static_cast<long>(blockIdx.x) / C;  // b * (G+1) + j
-  const int b = static_cast<int>(position / (G + 1));
-  const int j = static_cast<int>(position - static_cast<long>(b) * (G + 1));
-  const bool has_draft = j < G;
-
-  const T* rowT = static_cast<const T*>(P.target) + position * V;
-  const T* rowD = has_draft
-                      ? static_cast<const T*>(P.draft) + (static_cast<long>(b) * G + j) * V
-                      : nullptr;
-
-  const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
-  long clo = static_cast<long>(rank) * P.groups_per_cta;
-  long chi = clo + P.groups_per_cta;
-  if (clo > ngroups) clo = ngroups;
-  if (chi > ngroups) chi = ngroups;
-  long wlo, whi;
-  warp_range(clo, chi, warp, kNW, wlo, whi);
-
-  __shared__ float sm_max[2][kNW];
+  __shared__ float sm_off[2][kNW];
   __shared__ double sm_sum[2][kNW];
-  __shared__ CtaStats part;
-  __shared__ Bcast bc;
-  __shared__ CtaMass mass;
-  __shared__ double sm_wz[kNW];
-  __shared__ int sm_wlast[kNW];
-  __shared__ int sm_owner_warp;
-  __shared__ double sm_target_local;
+  const int tid = threadIdx.x, lane = tid & (kWarp - 1), warp = tid >> 5;
 
-  // ---------------- phase 1: streaming statistics ----------------
-  const float c_hi = P.c_hi, c_lo = P.c_lo;
-  float mT = -INFINITY, sT = 0.f, mD = -INFINITY, sD = 0.f;
-  for (long g0 = wlo + lane; g0 < whi; g0 += static_cast<long>(kWarp) * kUnroll) {
+  float oT = -INFINITY, sT = 0.f, oD = -INFINITY, sD = 0.f;
+  // consecutive threads read consecutive 16-byte groups: each warp-wide load
+  // is 512 contiguous bytes; kUnroll groups per row are in flight per thread
+  for (long g0 = glo + tid; g0 < ghi; g0 += static_cast<long>(NT) * kUnroll) {
     uint4 vt[kUnroll], vd[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const long g = g0 + static_cast<long>(u) * kWarp;
-      if (g < whi) {
+      const long g = g0 + static_cast<long>(u) * NT;
+      if (g < ghi) {
         vt[u] = fetch_group<T, kAligned>(rowT, g, V);
         if (has_draft) vd[u] = fetch_group<T, kAligned>(rowD, g, V);
       }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const long g = g0 + static_cast<long>(u) * kWarp;
-      if (g < whi) {
-        accumulate_group<T>(vt[u], mT, sT, c_hi, c_lo);
-        if (has_draft) accumulate_group<T>(vd[u], mD, sD, c_hi, c_lo);
+      const long g = g0 + static_cast<long>(u) * NT;
+      if (g < ghi) {
+        accumulate_group<T>(vt[u], oT, sT, c_hi, c_lo);
+        if (has_draft) accumulate_group<T>(vd[u], oD, sD, c_hi, c_lo);
       }
     }
   }
-
-  // CTA reduction: max first, then each thread rescales its sum to the CTA max
-  {
-    const float wT = warp_max(mT), wD = warp_max(mD);
-    if (lane == 0) {
-      sm_max[0][warp] = wT;
-      sm_max[1][warp] = wD;
-    }
-    __syncthreads();
-    float McT = sm_max[0][0], McD = sm_max[1][0];
+  // the block's offset is its largest thread offset; each thread rescales
+  const float wT = warp_max(oT), wD = warp_max(oD);
+  if (lane == 0) {
+    sm_off[0][warp] = wT;
+    sm_off[1][warp] = wD;
+  }
+  __syncthreads();
+  float OT = sm_off[0][0], OD = sm_off[1][0];
 #pragma unroll
-    for (int w = 1; w < kNW; ++w) {
-      McT = fmaxf(McT, sm_max[0][w]);
-      McD = fmaxf(McD, sm_max[1][w]);
-    }
-    // s * 2^((m - M) c); a thread with m = -inf holds s = 0 (or NaN, which propagates)
-    const float fT = (mT == -INFINITY) ? 0.f : ex2(scaled(mT - McT, c_hi, c_lo));
-    const float fD = (mD == -INFINITY) ? 0.f : ex2(scaled(mD - McD, c_hi, c_lo));
-    const double zT = warp_sum(static_cast<double>(sT) * static_cast<double>(fT));
-    const double zD = warp_sum(static_cast<double>(sD) * static_cast<double>(fD));
-    if (lane == 0) {
-      sm_sum[0][warp] = zT;
-      sm_sum[1][warp] = zD;
-    }
-    __syncthreads();
-    if (tid == 0) {
-      double a = 0.0, d = 0.0;
-      for (int w = 0; w < kNW; ++w) {
-        a += sm_sum[0][w];
-        d += sm_sum[1][w];
-      }
-      part.sT = a;
-      part.sD = d;
-      part.mT = McT;
-      part.mD = McD;
+  for (int w = 1; w < kNW; ++w) {
+    OT = fmaxf(OT, sm_off[0][w]);
+    OD = fmaxf(OD, sm_off[1][w]);
+  }
+  // a thread with o = -inf holds s = 0 (or NaN, which must propagate)
+  const float fT = (oT == -INFINITY) ? 0.f : ex2(oT - OT);
+  const float fD = (oD == -INFINITY) ? 0.f : ex2(oD - OD);
+  const double zT = warp_sum(static_cast<double>(sT) * static_cast<double>(fT));
+  const double zD = warp_sum(static_cast<double>(sD) * static_cast<double>(fD));
+  if (lane == 0) {
+    sm_sum[0][warp] = zT;
+    sm_sum[1][warp] = zD;
+  }
+  __syncthreads();
+  CtaStats out{0.0, 0.0, OT, OD, {0, 0}};
+  if (tid == 0) {
+    for (int w = 0; w < kNW; ++w) {
+      out.sT += sm_sum[0][w];
+      out.sD += sm_sum[1][w];
     }
   }
-  cluster.sync();  // (1) every CTA's partial statistics are visible
+  return out;
+}
 
-  // ---------------- phases 2-3: rank 0 decides, takes the ticket ----------------
-  if (rank == 0 && warp == 0) {
-    int last = 0;
-    if (lane == 0) {
-      // combine the cluster's partials in rank order (fp64)
-      double ST = 0.0, SD = 0.0;
-      float MT = -INFINITY, MD = -INFINITY;
-      for (int r = 0; r < C; ++r) {
-        const CtaStats* pr = cluster.map_shared_rank(&part, r);
-        MT = fmaxf(MT, pr->mT);
-        MD = fmaxf(MD, pr->mD);
-      }
-      for (int r = 0; r < C; ++r) {
-        const CtaStats* pr = cluster.map_shared_rank(&part, r);
-        const float mt = pr->mT, md = pr->mD;
-        const double st = pr->sT, sd = pr->sD;
-        ST += (mt == -INFINITY) ? st * 0.0 : st * exp2((static_cast<double>(mt) - MT) * P.c);
-        SD += (md == -INFINITY) ? sd * 0.0 : sd * exp2((static_cast<double>(md) - MD) * P.c);
-      }
-      const int validT = (MT != -INFINITY) && isfinite(ST) && ST > 0.0;
-      P.tstat[position] = RowStat{ST, MT, validT};
-      if (has_draft) {
+// (o, s) pairs combined: O = max o, S = sum s 2^(o - O)
+__device__ __forceinline__ void combine_into(float& O, double& S, float o, double s) {
+  if (o == -INFINITY) {
+    S += s * 0.0;  // keeps a NaN partial visible
+    return;
+  }
+  if (o > O) {
+    S = (O == -INFINITY) ? S : S * exp2(static_cast<double>(O) - o);
+    O = o;
+  }
+  S += s * exp2(static_cast<double>(o) - O);
+}
+
+// block-wide scan of one double per thread: inclusive, exclusive, total
+template <int NT>
+__device__ __forceinline__ void block_scan(double v, double& incl, double& excl, double& total) {
+  constexpr int kNW = NT / kWarp;
+  __shared__ double sm_w[kNW];
+  const int tid = threadIdx.x, lane = tid & (kWarp - 1), warp = tid >> 5;
+  double x = v;
+#pragma unroll
+  for (int o = 1; o < kWarp; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  const double prev = __shfl_up_sync(0xffffffffu, x, 1);
+  if (lane == kWarp - 1) sm_w[warp] = x;
+  __syncthreads();
+  double wpre = 0.0;
+  total = 0.0;
+  for (int w = 0; w < kNW; ++w) {
+    if (w < warp) wpre += sm_w[w];
+    total += sm_w[w];
+  }
+  __syncthreads();  // sm_w is reused by the next call
+  incl = wpre + x;
+  excl = (lane == 0) ? wpre : wpre + prev;
+  (void)tid;
+}
+
+// ---------------------------------------------------------------------------
+// kernel 1: streaming statistics
+// ---------------------------------------------------------------------------
+
+template <int NT>
+constexpr int min_blocks() {
+  return 1024 / NT;  // caps registers at 64 per thread
+}
+
+template <typename T, int NT, bool kAligned>
+__global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Params P) {
+  constexpr int kVec = Elem<T>::kVec;
+  const int G = P.gamma, V = P.vocab, S = P.slices;
+  const long unit = blockIdx.x;
+  const long position = unit / S;  // b * (G+1) + j
+  const int slice = static_cast<int>(unit - position * S);
+  const int b = static_cast<int>(position / (G + 1));
+  const int j = static_cast<int>(position - static_cast<long>(b) * (G + 1));
+  const bool has_draft = j < G;
+  const T* rowT = static_cast<const T*>(P.target) + position * V;
+  const T* rowD =
+      has_draft ? static_cast<const T*>(P.draft) + (static_cast<long>(b) * G + j) * V : nullptr;
+  const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
+  long glo = static_cast<long>(slice) * P.groups_per_slice;
+  long ghi = glo + P.groups_per_slice;
+  if (glo > ngroups) glo = ngroups;
+  if (ghi > ngroups) ghi = ngroups;
+  const CtaStats part =
+      slice_stats<T, NT, kAligned, 4>(rowT, rowD, has_draft, glo, ghi, V, P.c_hi, P.c_lo);
+  if (threadIdx.x == 0) P.partial[unit] = part;
+  cudaTriggerProgrammaticLaunchCompletion();
+}
+
+// ---------------------------------------------------------------------------
+// kernel 2: decide (one warp per sequence, one lane per position)
+// ---------------------------------------------------------------------------
+
+constexpr int kDecideThreads = 128;
+constexpr int kMaxGamma = 255;
+
+// (o, s) partials of one row combined in two passes, so that the fp64
+// exponentials of the second pass are independent of one another
+__device__ __forceinline__ double row_lse2(const CtaStats* parts, int S, bool draft, int& valid) {
+  float O = -INFINITY;
+  for (int r = 0; r < S; ++r) O = fmaxf(O, draft ? parts[r].oD : parts[r].oT);
+  double sum = 0.0;
+  for (int r = 0; r < S; ++r) {
+    const float o = draft ? parts[r].oD : parts[r].oT;
+    const double s = draft ? parts[r].sD : parts[r].sT;
+    sum += (o == -INFINITY) ? s * 0.0 : s * exp2(static_cast<double>(o) - O);  // NaN survives
+  }
+  valid = (O != -INFINITY) && isfinite(sum) && sum > 0.0;
+  return static_cast<double>(O) + log2(sum);  // log2 sum_i 2^(x_i c)
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) {
+  // the statistics of the previous kernel must be complete and visible
+  cudaGridDependencySynchronize();
+  const int lane = threadIdx.x & (kWarp - 1);
+  const int b = blockIdx.x * (kDecideThreads / kWarp) + (threadIdx.x >> 5);
+  if (b < P.batch) {  // warp-uniform
+    const int G = P.gamma, V = P.vocab, S = P.slices;
+    const double c = P.c;
+    int n = G;          // first rejection, gamma if none
+    unsigned bits = 0;  // data errors of the sequence
+    double lT_n = 0.0, lD_n = 0.0;
+    for (int base = 0; base <= G; base += kWarp) {
+      const int j = base + lane;
+      int flag = kFlagAccept;
+      bool tok_bad = false, row_bad = false;
+      double lT = 0.0, lD = 0.0;
+      if (j <= G) {
+        const long position = static_cast<long>(b) * (G + 1) + j;
         const long pj = static_cast<long>(b) * G + j;
-        const int validD = (MD != -INFINITY) && isfinite(SD) && SD > 0.0;
-        P.dstat[pj] = RowStat{SD, MD, validD};
-        PosInfo info{0.0, 0.0, 0.0, kFlagReject, 0};
-        const int t = P.tokens[pj];
-        if (t < 0 || t >= V) {
-          info.flag = kFlagTokenRange;
-        } else if (!validT || !validD) {
-          info.flag = kFlagNonFinite;
-        } else {
-          const double xt = static_cast<double>(Elem<T>::load1(rowT, t));
-          const double xd = static_cast<double>(Elem<T>::load1(rowD, t));
-          const double lq = (xt - MT) * P.c - log2(ST);  // log2 q(t)
-          const double lp = (xd - MD) * P.c - log2(SD);  // log2 p(t)
-          info.q_tok = exp2(lq);
-          info.p_tok = exp2(lp);
-          if (!(info.q_tok > 0.0)) info.ratio = 0.0;
-          else if (!(info.p_tok > 0.0)) info.ratio = INFINITY;
-          else info.ratio = exp2(lq - lp);
-          const double u = static_cast<double>(P.u_accept[pj]);
-          info.flag = (u < info.ratio) ? kFlagAccept : kFlagReject;
-        }
-        P.pos[pj] = info;
-      }
-      __threadfence();
-      const unsigned old = atomicAdd(P.ticket + b, 1u);
-      last = (old == static_cast<unsigned>(G)) ? 1 : 0;
-      if (last) __threadfence();
-    }
-    last = __shfl_sync(0xffffffffu, last, 0);
-    Bcast out{};
-    out.last = last;
-    if (last) {
-      // first rejection and any data error, by warp ballot over the flags
-      int n = G;
-      unsigned stat_bits = 0;
-      for (int base = 0; base < G; base += kWarp) {
-        const int jj = base + lane;
-        int f = kFlagAccept;
-        if (jj < G) f = __ldcg(&P.pos[static_cast<long>(b) * G + jj].flag);
-        const unsigned rej = __ballot_sync(0xffffffffu, f == kFlagReject);
-        const unsigned tok = __ballot_sync(0xffffffffu, f == kFlagTokenRange);
-        const unsigned bad = __ballot_sync(0xffffffffu, f == kFlagNonFinite);
-        if (tok) stat_bits |= kStatTokenRange;
-        if (bad) stat_bits |= kStatNonFinite;
-        if (rej && n == G) n = base + __ffs(rej) - 1;
-      }
-      if (lane == 0) {
-        if (!__ldcg(&P.tstat[static_cast<long>(b) * (G + 1) + G].valid)) stat_bits |= kStatNonFinite;
-        out.n = n;
-        out.stat_bits = stat_bits;
-        if (stat_bits) {
-          out.mode = kDrawNone;
-        } else {
-          const long tr = static_cast<long>(b) * (G + 1) + n;
-          out.trow = n;
-          out.mT = __ldcg(&P.tstat[tr].max);
-          out.sT = __ldcg(&P.tstat[tr].sum);
-          if (n < G) {
-            const long dr = static_cast<long>(b) * G + n;
-            out.mode = kDrawResidual;
-            out.drow = n;
-            out.mD = __ldcg(&P.dstat[dr].max);
-            out.sD = __ldcg(&P.dstat[dr].sum);
-          } else {
-            out.mode = kDrawTarget;
-            out.drow = -1;
+        const bool has_draft = j < G;
+        // the acceptance test's inputs first: their loads overlap the combine
+        int t = 0;
+        float u = 0.f, xt = 0.f, xd = 0.f;
+        if (has_draft) {
+          t = P.tokens[pj];
+          u = P.u_accept[pj];
+          tok_bad = (t < 0 || t >= V);
+          if (!tok_bad) {
+            xt = Elem<T>::load1(static_cast<const T*>(P.target) + position * V, t);
+            xd = Elem<T>::load1(static_cast<const T*>(P.draft) + pj * V, t);
           }
         }
-      }
-      // broadcast lane 0's decision to the other lanes
-      out.n = __shfl_sync(0xffffffffu, out.n, 0);
-      out.stat_bits = __shfl_sync(0xffffffffu, out.stat_bits, 0);
-      out.mode = __shfl_sync(0xffffffffu, out.mode, 0);
-      out.trow = __shfl_sync(0xffffffffu, out.trow, 0);
-      out.drow = __shfl_sync(0xffffffffu, out.drow, 0);
-      out.mT = __shfl_sync(0xffffffffu, out.mT, 0);
-      out.mD = __shfl_sync(0xffffffffu, out.mD, 0);
-      out.sT = __shfl_sync(0xffffffffu, out.sT, 0);
-      out.sD = __shfl_sync(0xffffffffu, out.sD, 0);
-    }
-    // push the decision into every CTA of the cluster
-    if (lane < C) *cluster.map_shared_rank(&bc, lane) = out;
-  }
-  cluster.sync();  // (2) the decision is in every CTA's shared memory
-
-  if (!bc.last) return;  // cluster-uniform
-
-  // ---------------- phase 4: the finishing cluster draws the token ----------------
-  const float u_res = P.u_resample[b];
-  int mode = bc.mode;
-  const int n = bc.n;
-  if (mode == kDrawNone) {
-    if (rank == 0 && tid == 0) {
-      int32_t* outt = P.out_tokens + static_cast<long>(b) * (G + 1);
-      for (int k = 0; k <= G; ++k) outt[k] = -1;
-      P.out_num_accepted[b] = 0;
-      P.resid_mass[b] = NAN;
-      atomicOr(P.status, bc.stat_bits);
-      P.ticket[b] = 0u;
-    }
-    return;  // no CTA reads another's shared memory after barrier (2)
-  }
-
-  const T* drawT = static_cast<const T*>(P.target) + (static_cast<long>(b) * (G + 1) + bc.trow) * V;
-  const T* drawD = (bc.drow >= 0)
-                       ? static_cast<const T*>(P.draft) + (static_cast<long>(b) * G + bc.drow) * V
-                       : nullptr;
-  DrawConsts k;
-  k.c_hi = c_hi;
-  k.c_lo = c_lo;
-  k.mT = bc.mT;
-  k.mD = bc.mD;
-  k.invST = static_cast<float>(1.0 / bc.sT);
-  k.invSD = static_cast<float>(1.0 / bc.sD);
-  {
-    const double K = (static_cast<double>(bc.mT) - bc.mD) * P.c + log2(bc.sT / bc.sD);
-    k.k_hi = static_cast<float>(K);
-    k.k_lo = static_cast<float>(K - static_cast<double>(k.k_hi));
-  }
-  unsigned extra_bits = 0;
-  double Z = 0.0, target = 0.0;
-  int owner = -1, last_all = -1;
-  double prefix_owner = 0.0;
-
-  for (int attempt = 0; attempt < 2; ++attempt) {
-    // pass A: mass per warp (contiguous warp ranges) and per CTA
-    double lz = 0.0;
-    int llast = -1;
-    for (long g0 = wlo + lane; g0 < whi; g0 += static_cast<long>(kWarp) * kUnroll) {
-      uint4 vt[kUnroll], vd[kUnroll];
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const long g = g0 + static_cast<long>(u) * kWarp;
-        if (g < whi) {
-          vt[u] = fetch_group<T, kAligned>(drawT, g, V);
-          vd[u] = (mode == kDrawResidual) ? fetch_group<T, kAligned>(drawD, g, V) : vt[u];
+        const CtaStats* parts = P.partial + position * S;
+        int validT = 0, validD = 1;
+        lT = row_lse2(parts, S, false, validT);
+        P.tstat[position] = RowStat{lT, validT, 0};
+        if (has_draft) {
+          lD = row_lse2(parts, S, true, validD);
+          P.dstat[pj] = RowStat{lD, validD, 0};
+        }
+        row_bad = !validT || !validD;
+        if (has_draft) {
+          PosInfo info{0.0, 0.0, 0.0, kFlagReject, 0};
+          if (tok_bad) {
+            info.flag = kFlagTokenRange;
+          } else if (row_bad) {
+            info.flag = kFlagNonFinite;
+          } else {
+            const double lq = static_cast<double>(xt) * c - lT;  // log2 q(t)
+            const double lp = static_cast<double>(xd) * c - lD;  // log2 p(t)
+            info.q_tok = exp2(lq);
+            info.p_tok = exp2(lp);
+            if (!(info.q_tok > 0.0)) info.ratio = 0.0;
+            else if (!(info.p_tok > 0.0)) info.ratio = INFINITY;
+            else info.ratio = exp2(lq - lp);
+            info.flag = (static_cast<double>(u) < info.ratio) ? kFlagAccept : kFlagReject;
+          }
+          P.pos[pj] = info;
+          flag = info.flag;
         }
       }
+      const unsigned rej = __ballot_sync(0xffffffffu, j < G && flag == kFlagReject);
+      if (__ballot_sync(0xffffffffu, tok_bad)) bits |= kStatTokenRange;
+      if (__ballot_sync(0xffffffffu, row_bad)) bits |= kStatNonFinite;
+      // the statistics the draw needs live in lane (n - base) of this chunk
+      const int first = rej ? base + __ffs(rej) - 1 : G;
+      const bool here = (n == G) && (first < G || G < base + kWarp);
+      if (n == G) n = first;
+      const int src = (n - base) & (kWarp - 1);
+      const double lTs = __shfl_sync(0xffffffffu, lT, src);
+      const double lDs = __shfl_sync(0xffffffffu, lD, src);
+      if (here) {
+        lT_n = lTs;
+        lD_n = lDs;
+      }
+    }
+    const long bo = static_cast<long>(b) * (G + 1);
+    if (bits) {
+      for (int q = lane; q <= G; q += kWarp) P.out_tokens[bo + q] = -1;
+      if (lane == 0) {
+        P.out_num_accepted[b] = 0;
+        P.resid_mass[b] = NAN;
+        P.decision[b] = SeqDecision{0.0, 0.0, 0, kDrawNone, bits, 0};
+        atomicOr(P.status, bits);
+      }
+    } else {
+      // accepted prefix and padding; the drawn token at n is the draw kernel's
+      for (int q = lane; q <= G; q += kWarp) {
+        if (q < n) P.out_tokens[bo + q] = P.tokens[static_cast<long>(b) * G + q];
+        else if (q > n) P.out_tokens[bo + q] = -1;
+      }
+      if (lane == 0) {
+        P.out_num_accepted[b] = n;
+        P.decision[b] = SeqDecision{lT_n, lD_n, n, (n < G) ? kDrawResidual : kDrawTarget, 0u, 0};
+      }
+    }
+  }
+  cudaTriggerProgrammaticLaunchCompletion();
+}
+
+// ---------------------------------------------------------------------------
+// kernel 3: draw
+// ---------------------------------------------------------------------------
+
+constexpr int kDrawThreads = 128;
+constexpr int kDrawWarps = kDrawThreads / kWarp;
+constexpr int kTile = 32;  // groups per tile of the draw's mass table
+
+// Mass of each 32-group tile of [tlo, thi) (tiles of the row, warp w takes
+// tiles w, w + 4, ...); lane 0 of the warp stores the tile's mass in `table`.
+template <typename T, bool kAligned>
+__device__ __forceinline__ void tile_masses(int mode, const T* drawT, const T* drawD,
+                                            const DrawConsts& k, long tlo, long thi,
+                                            long ngroups, int V, double* table) {
+  constexpr int kVec = Elem<T>::kVec;
+  constexpr int kUnroll = 4;
+  const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x >> 5;
+  for (long t0 = tlo + warp; t0 < thi; t0 += static_cast<long>(kDrawWarps) * kUnroll) {
+    uint4 vt[kUnroll], vd[kUnroll];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const long g = g0 + static_cast<long>(u) * kWarp;
-        if (g < whi) {
+    for (int u = 0; u < kUnroll; ++u) {
+      const long g = (t0 + static_cast<long>(u) * kDrawWarps) * kTile + lane;
+      if (t0 + u * kDrawWarps < thi && g < ngroups) {
+        vt[u] = fetch_group<T, kAligned>(drawT, g, V);
+        vd[u] = (mode == kDrawResidual) ? fetch_group<T, kAligned>(drawD, g, V) : vt[u];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long tile = t0 + static_cast<long>(u) * kDrawWarps;
+      if (tile < thi) {  // warp-uniform
+        const long g = tile * kTile + lane;
+        float gs = 0.f;
+        if (g < ngroups) {
           float r[kVec];
           if (mode == kDrawResidual) group_mass<T, kDrawResidual>(vt[u], vd[u], k, r);
           else group_mass<T, kDrawTarget>(vt[u], vd[u], k, r);
-          float gs = 0.f;
 #pragma unroll
-          for (int e = 0; e < kVec; ++e) {
-            gs += r[e];
-            if (r[e] > 0.f) llast = static_cast<int>(g * kVec + e);
-          }
-          lz += static_cast<double>(gs);
+          for (int e = 0; e < kVec; ++e) gs += r[e];
+        }
+        const double z = warp_sum(static_cast<double>(gs)) * k.fT;
+        if (lane == 0) table[tile] = z;
+      }
+    }
+  }
+}
+
+// The masses of the 32 groups of `tile`, one per lane of the calling warp:
+// returns the index where the running mass first exceeds tl, else the
+// tile's last index with mass (rounding), else -1 (no mass in the tile).
+template <typename T, bool kAligned>
+__device__ __forceinline__ int scan_tile(int mode, const T* drawT, const T* drawD,
+                                         const DrawConsts& k, long tile, long ngroups, int V,
+                                         double tl_mass) {
+  const double tl = tl_mass / static_cast<double>(k.fT);  // in the units of group_mass
+  constexpr int kVec = Elem<T>::kVec;
+  const int lane = threadIdx.x & (kWarp - 1);
+  const long g = tile * kTile + lane;
+  float r[kVec];
+#pragma unroll
+  for (int e = 0; e < kVec; ++e) r[e] = 0.f;
+  if (g < ngroups) {
+    const uint4 vt = fetch_group<T, kAligned>(drawT, g, V);
+    const uint4 vd = (mode == kDrawResidual) ? fetch_group<T, kAligned>(drawD, g, V) : vt;
+    if (mode == kDrawResidual) group_mass<T, kDrawResidual>(vt, vd, k, r);
+    else group_mass<T, kDrawTarget>(vt, vd, k, r);
+  }
+  float gs = 0.f;
+  int mylast = -1;
+#pragma unroll
+  for (int e = 0; e < kVec; ++e) {
+    gs += r[e];
+    if (r[e] > 0.f) mylast = static_cast<int>(g * kVec + e);
+  }
+  const double ls = static_cast<double>(gs);
+  double incl = ls;
+#pragma unroll
+  for (int o = 1; o < kWarp; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) excl = 0.0;
+  const unsigned hit = __ballot_sync(0xffffffffu, excl <= tl && incl > tl);
+  if (hit) {
+    const int L = __ffs(hit) - 1;
+    int token = -1;
+    if (lane == L) {
+      double acc = excl;
+#pragma unroll
+      for (int e = 0; e < kVec; ++e) {
+        if (r[e] > 0.f) {
+          acc += static_cast<double>(r[e]);
+          if (token < 0 && acc > tl) token = static_cast<int>(g * kVec + e);
         }
       }
+      if (token < 0) token = mylast;  // rounding between the two sums
     }
-    const double wz = warp_sum(lz);
-    const int wl = warp_maxi(llast);
-    if (lane == 0) {
-      sm_wz[warp] = wz;
-      sm_wlast[warp] = wl;
-    }
-    __syncthreads();
-    if (tid == 0) {
-      double z = 0.0;
-      int lp = -1;
-      for (int w = 0; w < kNW; ++w) {
-        z += sm_wz[w];
-        lp = max(lp, sm_wlast[w]);
+    return __shfl_sync(0xffffffffu, token, L);
+  }
+  return warp_maxi(mylast);  // rounding past the tile's end
+}
+
+template <typename T, bool kAligned>
+__global__ void __launch_bounds__(kDrawThreads, 8) draw_kernel(const Params P) {
+  constexpr int kVec = Elem<T>::kVec;
+  const int tid = threadIdx.x;
+  const int G = P.gamma, V = P.vocab, S2 = P.draw_slices;
+  const int b = blockIdx.x / S2;
+  const int s2 = blockIdx.x - b * S2;
+  cudaGridDependencySynchronize();  // the decisions of the previous kernel
+  const SeqDecision d = P.decision[b];
+  if (d.mode == kDrawNone) return;  // the decide kernel wrote the error outcome
+  const int n = d.n;
+  const double lT = d.lT, lD = d.lD;
+  const long bo = static_cast<long>(b) * (G + 1);
+
+  // ---- step 4: residual (n < gamma) or bonus (n == gamma) draw ----
+  int mode = d.mode;
+  const T* drawT = static_cast<const T*>(P.target) + (bo + n) * V;
+  const T* drawD = (mode == kDrawResidual)
+                       ? static_cast<const T*>(P.draft) + (static_cast<long>(b) * G + n) * V
+                       : nullptr;
+  DrawConsts k;
+  k.c_hi = P.c_hi;
+  k.c_lo = P.c_lo;
+  float lt_lo, ld_lo;
+  split2(lT, k.lt_hi, lt_lo);
+  split2(lD, k.ld_hi, ld_lo);
+  split2(lT - lD, k.k_hi, k.k_lo);
+  k.rD = static_cast<float>(exp2(static_cast<double>(lt_lo) - ld_lo));
+  k.fT = static_cast<float>(exp2(-static_cast<double>(lt_lo)));
+
+  const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
+  const long ntiles = (ngroups + kTile - 1) / kTile;
+  const long tiles_per = P.groups_per_draw / kTile;
+  long tlo = static_cast<long>(s2) * tiles_per;
+  long thi = tlo + tiles_per;
+  if (tlo > ntiles) tlo = ntiles;
+  if (thi > ntiles) thi = ntiles;
+  double* table = P.draw_mass + static_cast<long>(b) * ntiles;
+  tile_masses<T, kAligned>(mode, drawT, drawD, k, tlo, thi, ngroups, V, table);
+  __threadfence();  // this block's tiles are published before its ticket
+  __syncthreads();
+  __shared__ int sm_last;
+  if (tid == 0) {
+    const unsigned old = atomicAdd(P.draw_ticket + b, 1u);
+    sm_last = (old == static_cast<unsigned>(S2 - 1));
+    if (sm_last) __threadfence();
+  }
+  __syncthreads();
+  if (!sm_last) return;
+
+  // ---- the block that finishes the sequence locates u * Z ----
+  __shared__ long sm_tile;
+  __shared__ double sm_tl, sm_Z;
+  const long per = (ntiles + kDrawThreads - 1) / kDrawThreads;  // tiles per thread, in order
+  const long a0 = tid * per < ntiles ? tid * per : ntiles;
+  const long a1 = (a0 + per < ntiles) ? a0 + per : ntiles;
+  unsigned extra_bits = 0;
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    double mine = 0.0;
+    for (long t = a0; t < a1; ++t) mine += __ldcg(&table[t]);
+    double incl, excl, tot;
+    block_scan<kDrawThreads>(mine, incl, excl, tot);
+    if (tot > 0.0 || mode != kDrawResidual) {
+      const double target = static_cast<double>(P.u_resample[b]) * tot;
+      if (tid == 0) {
+        sm_Z = tot;
+        sm_tile = -1;
       }
-      mass.z = z;
-      mass.last_pos = lp;
+      __syncthreads();
+      if (excl <= target && incl > target) {
+        // this thread's tiles hold u * Z: walk them in order
+        double acc = excl;
+        for (long t = a0; t < a1; ++t) {
+          const double z = __ldcg(&table[t]);
+          if (z > 0.0 && acc + z > target) {
+            sm_tile = t;
+            sm_tl = target - acc;
+            break;
+          }
+          acc += z;
+        }
+      }
+      // rounding can leave u * Z at or beyond the last tile with mass: use
+      // that tile, with the point at its end
+      const bool has = (a1 > a0) && incl > excl;  // this thread owns mass
+      const unsigned own = __ballot_sync(0xffffffffu, has);
+      __shared__ int sm_lastthread[kDrawWarps];
+      if ((tid & (kWarp - 1)) == 0) sm_lastthread[tid >> 5] = own ? (tid & ~(kWarp - 1)) + 31 - __clz(own) : -1;
+      __syncthreads();
+      if (tid == 0 && sm_tile < 0) {
+        int lt = -1;
+        for (int w = 0; w < kDrawWarps; ++w) lt = max(lt, sm_lastthread[w]);
+        long bt = -1;
+        if (lt >= 0) {
+          const long b0 = static_cast<long>(lt) * per;
+          for (long t = b0; t < b0 + per && t < ntiles; ++t)
+            if (__ldcg(&table[t]) > 0.0) bt = t;
+        }
+        sm_tile = bt;
+        sm_tl = INFINITY;
+      }
+      __syncthreads();
+      break;
     }
-    cluster.sync();  // (3) CTA masses visible
-    // every thread forms the same cluster totals in rank order
-    Z = 0.0;
-    last_all = -1;
-    for (int r = 0; r < C; ++r) {
-      const CtaMass* pr = cluster.map_shared_rank(&mass, r);
-      Z += pr->z;
-      last_all = max(last_all, pr->last_pos);
-    }
-    if (Z > 0.0 || mode != kDrawResidual) break;
-    // zero residual mass (rounding only): draw from q_n instead
+    // zero residual mass (reachable only through rounding): draw from q_n,
+    // this block alone recomputing the row's tiles
     mode = kDrawTarget;
     extra_bits |= kStatZeroMass;
-    cluster.sync();  // (3b) nobody still reads the masses about to be rewritten
-  }
-
-  target = static_cast<double>(u_res) * Z;
-  {
-    double pre = 0.0;
-    for (int r = 0; r < C; ++r) {
-      const CtaMass* pr = cluster.map_shared_rank(&mass, r);
-      if (pr->z > 0.0 && pre + pr->z > target) {
-        owner = r;
-        prefix_owner = pre;
-        break;
-      }
-      pre += pr->z;
-    }
-  }
-
-  if (owner == rank) {
-    if (tid == 0) {
-      const double tl = target - prefix_owner;
-      double pre = 0.0;
-      int ow = -1;
-      for (int w = 0; w < kNW; ++w) {
-        if (sm_wz[w] > 0.0 && pre + sm_wz[w] > tl) {
-          ow = w;
-          break;
-        }
-        pre += sm_wz[w];
-      }
-      sm_owner_warp = ow;
-      sm_target_local = tl - pre;
-    }
+    tile_masses<T, kAligned>(mode, drawT, drawD, k, 0, ntiles, ngroups, V, table);
+    __threadfence();
     __syncthreads();
-    const int ow = sm_owner_warp;
-    if (ow < 0) {
-      if (tid == 0) P.out_tokens[static_cast<long>(b) * (G + 1) + n] = mass.last_pos;
-    } else if (warp == ow) {
-      // pass B: ordered scan of this warp's range
-      const double tw = sm_target_local;
-      double running = 0.0;
-      int token = -1;
-      for (long g0 = wlo; g0 < whi && token < 0; g0 += kWarp) {
-        const long g = g0 + lane;
-        float r[kVec];
-#pragma unroll
-        for (int e = 0; e < kVec; ++e) r[e] = 0.f;
-        if (g < whi) {
-          const uint4 vt = fetch_group<T, kAligned>(drawT, g, V);
-          const uint4 vd = (mode == kDrawResidual) ? fetch_group<T, kAligned>(drawD, g, V) : vt;
-          if (mode == kDrawResidual) group_mass<T, kDrawResidual>(vt, vd, k, r);
-          else group_mass<T, kDrawTarget>(vt, vd, k, r);
-        }
-        float gs = 0.f;
-#pragma unroll
-        for (int e = 0; e < kVec; ++e) gs += r[e];
-        const double ls = static_cast<double>(gs);
-        double incl = ls;
-#pragma unroll
-        for (int o = 1; o < kWarp; o <<= 1) {
-          const double y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const double tot = __shfl_sync(0xffffffffu, incl, kWarp - 1);
-        if (running + tot > tw) {
-          const unsigned hit = __ballot_sync(0xffffffffu, ls > 0.0 && running + incl > tw);
-          const int L = hit ? __ffs(hit) - 1 : kWarp - 1;
-          int found = -1;
-          if (lane == L) {
-            double acc = running + (incl - ls);
-            int lastpos = -1;
-#pragma unroll
-            for (int e = 0; e < kVec; ++e) {
-              if (r[e] > 0.f) {
-                lastpos = static_cast<int>(g * kVec + e);
-                acc += static_cast<double>(r[e]);
-                if (found < 0 && acc > tw) found = lastpos;
-              }
-            }
-            if (found < 0) found = lastpos;  // rounding between the two sums
-          }
-          token = __shfl_sync(0xffffffffu, found, L);
-        }
-        running += tot;
-      }
-      if (token < 0) token = sm_wlast[ow];  // rounding: u * Z beyond this warp's scan
-      if (lane == 0) P.out_tokens[static_cast<long>(b) * (G + 1) + n] = token;
+  }
+
+  // the owning tile: one group per lane, warp 0 scans it in index order
+  if (tid < kWarp) {
+    const long tile = sm_tile;
+    const int token = (tile >= 0) ? scan_tile<T, kAligned>(mode, drawT, drawD, k, tile, ngroups, V, sm_tl)
+                                  : -1;
+    if (tid == 0) {
+      P.out_tokens[bo + n] = token;
+      P.resid_mass[b] = sm_Z;
+      if (extra_bits) atomicOr(P.status, extra_bits);
+      P.draw_ticket[b] = 0u;  // ready for the next launch
     }
   }
-  if (owner < 0 && rank == 0 && tid == 0) {
-    P.out_tokens[static_cast<long>(b) * (G + 1) + n] = last_all;  // rounding: u * Z >= Z
-  }
-  if (rank == 0 && tid == 0) {
-    int32_t* outt = P.out_tokens + static_cast<long>(b) * (G + 1);
-    const int32_t* drafts = P.tokens + static_cast<long>(b) * G;
-    for (int q = 0; q < n; ++q) outt[q] = drafts[q];
-    for (int q = n + 1; q <= G; ++q) outt[q] = -1;
-    P.out_num_accepted[b] = n;
-    P.resid_mass[b] = Z;
-    if (extra_bits) atomicOr(P.status, extra_bits);
-    P.ticket[b] = 0u;  // ready for the next launch
-  }
-  cluster.sync();  // (4) keep shared memory alive until every remote read is done
 }
 
 }  // namespace specverify

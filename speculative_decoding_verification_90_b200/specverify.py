@@ -38,9 +38,11 @@ SIGNATURES = {
     "specverify_run_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
     "specverify_destroy": (None, [_vp]),
     "specverify_get_status": (_i, [_vp, _vp, _u32p]),
-    "specverify_debug_readback": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "specverify_debug_readback": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "specverify_set_launch": (_i, [_vp, _i, _i]),
-    "specverify_get_launch": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "specverify_get_launch": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "specverify_profile_begin": (_i, [_vp, _i]),
+    "specverify_profile_end": (_i, [_vp, ctypes.POINTER(_f), ctypes.POINTER(_f), ctypes.POINTER(_i)]),
     "specverify_status_string": (ctypes.c_char_p, [_i]),
     "specverify_last_error": (ctypes.c_char_p, []),
 }
@@ -117,14 +119,28 @@ def specverify_debug_readback(h, *ptrs, stream=0) -> int:
     return _check(_lib.specverify_debug_readback(h, *ptrs, stream), "specverify_debug_readback")
 
 
-def specverify_set_launch(h, cluster_ctas: int, threads: int) -> int:
-    return _check(_lib.specverify_set_launch(h, cluster_ctas, threads), "specverify_set_launch")
+def specverify_set_launch(h, slices: int, threads: int) -> int:
+    return _check(_lib.specverify_set_launch(h, slices, threads), "specverify_set_launch")
 
 
-def specverify_get_launch(h) -> tuple[int, int]:
-    c, t = ctypes.c_int(), ctypes.c_int()
-    _check(_lib.specverify_get_launch(h, ctypes.byref(c), ctypes.byref(t)), "specverify_get_launch")
-    return c.value, t.value
+def specverify_get_launch(h) -> tuple[int, int, int]:
+    """(slices, threads, max_slices) of the handle."""
+    c, t, m = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(_lib.specverify_get_launch(h, ctypes.byref(c), ctypes.byref(t), ctypes.byref(m)),
+           "specverify_get_launch")
+    return c.value, t.value, m.value
+
+
+def specverify_profile_begin(h, max_runs: int) -> int:
+    return _check(_lib.specverify_profile_begin(h, max_runs), "specverify_profile_begin")
+
+
+def specverify_profile_end(h) -> dict:
+    """Mean device milliseconds per run of each kernel since profile_begin."""
+    a, c, n = ctypes.c_float(), ctypes.c_float(), ctypes.c_int()
+    _check(_lib.specverify_profile_end(h, ctypes.byref(a), ctypes.byref(c), ctypes.byref(n)),
+           "specverify_profile_end")
+    return {"stats_ms": a.value, "draw_ms": c.value, "runs": n.value}
 
 
 def specverify_status_string(status: int) -> str:
@@ -233,20 +249,29 @@ class SpecVerify:
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
         return specverify_get_status(self.handle, sp)
 
-    def set_launch(self, cluster_ctas: int, threads: int):
-        specverify_set_launch(self.handle, cluster_ctas, threads)
+    def set_launch(self, slices: int, threads: int):
+        specverify_set_launch(self.handle, slices, threads)
 
     def launch(self) -> tuple[int, int]:
-        return specverify_get_launch(self.handle)
+        """(slices per position, threads per block)."""
+        return specverify_get_launch(self.handle)[:2]
+
+    def profile_begin(self, max_runs: int):
+        specverify_profile_begin(self.handle, max_runs)
+
+    def profile_end(self) -> dict:
+        return specverify_profile_end(self.handle)
+
+    @property
+    def max_slices(self) -> int:
+        return specverify_get_launch(self.handle)[2]
 
     def readback(self, stream=None) -> dict:
         """Intermediate values of the last step (see specverify_debug_readback)."""
         import torch
         B, G = self.batch, self.gamma
-        out = {"target_max": np.zeros((B, G + 1), np.float32),
-               "target_sum": np.zeros((B, G + 1), np.float64),
-               "draft_max": np.zeros((B, G), np.float32),
-               "draft_sum": np.zeros((B, G), np.float64),
+        out = {"target_lse": np.zeros((B, G + 1), np.float64),
+               "draft_lse": np.zeros((B, G), np.float64),
                "q_tok": np.zeros((B, G), np.float64),
                "p_tok": np.zeros((B, G), np.float64),
                "ratio": np.zeros((B, G), np.float64),

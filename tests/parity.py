@@ -7,8 +7,8 @@ oracle's margin at the first differing decision is below ``MARGIN``:
 |u_accept - ratio| for an acceptance test, and for the draw the distance of
 u_resample to the ends of the chosen token's interval of the normalised
 cumulative mass.  Such cases are counted and reported.  Softmax quantities
-must agree within ``PROB_TOL`` absolute (q(t), p(t)) and row sums within
-``SUM_RTOL`` relative.
+must agree within ``PROB_TOL`` absolute (q(t), p(t), residual mass Z) and the
+log normalisers log sum_i exp(x_i/T) within ``LSE_TOL`` absolute.
 """
 from __future__ import annotations
 
@@ -18,7 +18,7 @@ import numpy as np
 
 MARGIN = 1e-6
 PROB_TOL = 1e-5
-SUM_RTOL = 1e-5
+LSE_TOL = 1e-5   # absolute, i.e. relative on the normaliser
 
 
 def to_device(wl, device=0):
@@ -39,7 +39,7 @@ def to_device(wl, device=0):
     }
 
 
-def gpu_run(wl, cluster=None, threads=None, device=0, inputs=None, sv=None, readback=True):
+def gpu_run(wl, slices=None, threads=None, device=0, inputs=None, sv=None, readback=True):
     """One verification call of the whole workload; returns numpy outputs."""
     import torch
     from speculative_decoding_verification_90_b200.specverify import SpecVerify
@@ -47,9 +47,9 @@ def gpu_run(wl, cluster=None, threads=None, device=0, inputs=None, sv=None, read
     if own:
         sv = SpecVerify(wl.batch, wl.gamma, wl.vocab, wl.dtype, device)
     try:
-        if cluster is not None or threads is not None:
+        if slices is not None or threads is not None:
             c0, t0 = sv.launch()
-            sv.set_launch(cluster or c0, threads or t0)
+            sv.set_launch(min(slices or c0, sv.max_slices), threads or t0)
         d = inputs if inputs is not None else to_device(wl, device)
         out_t = torch.full((wl.batch, wl.gamma + 1), -7, dtype=torch.int32, device=f"cuda:{device}")
         out_n = torch.full((wl.batch,), -7, dtype=torch.int32, device=f"cuda:{device}")
@@ -104,15 +104,12 @@ def compare(wl, gpu, ora, seqs=None, check_probs=True):
             dp = np.abs(gpu["p_tok"][s] - ora["p_tok"][s])[tested]
             summary["max_dq"] = float(dq.max()) if dq.size else 0.0
             summary["max_dp"] = float(dp.max()) if dp.size else 0.0
-            rd = np.abs(gpu["draft_sum"][s] / ora["draft_sum"][s] - 1.0)
-            summary["max_draft_sum_rel"] = float(rd.max())
-            summary["draft_max_equal"] = bool(np.array_equal(
-                gpu["draft_max"][s].astype(np.float64), ora["draft_max"][s]))
+            # log sum_i exp(x_i/T) = max/T + log(sum) in the oracle's terms
+            lse_d = ora["draft_max"][s] / wl.temperature + np.log(ora["draft_sum"][s])
+            summary["max_draft_lse_abs"] = float(np.abs(gpu["draft_lse"][s] - lse_d).max())
         if len(s):
-            rt = np.abs(gpu["target_sum"][s] / ora["target_sum"][s] - 1.0)
-            summary["max_target_sum_rel"] = float(rt.max())
-            summary["target_max_equal"] = bool(np.array_equal(
-                gpu["target_max"][s].astype(np.float64), ora["target_max"][s]))
+            lse_t = ora["target_max"][s] / wl.temperature + np.log(ora["target_sum"][s])
+            summary["max_target_lse_abs"] = float(np.abs(gpu["target_lse"][s] - lse_t).max())
             dz = np.abs(gpu["resid_mass"][s] - ora["resid_mass"][s])
             summary["max_dz"] = float(np.nanmax(dz)) if dz.size else 0.0
     return summary
@@ -124,9 +121,6 @@ def assert_parity(summary, max_margin_frac=0.01):
     for key in ("max_dq", "max_dp", "max_dz"):
         if key in summary:
             assert summary[key] <= PROB_TOL, summary
-    for key in ("max_target_sum_rel", "max_draft_sum_rel"):
+    for key in ("max_target_lse_abs", "max_draft_lse_abs"):
         if key in summary:
-            assert summary[key] <= SUM_RTOL, summary
-    for key in ("target_max_equal", "draft_max_equal"):
-        if key in summary:
-            assert summary[key], summary
+            assert summary[key] <= LSE_TOL, summary
