@@ -35,6 +35,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+from speculative_decoding_verification_90_b200 import dist as svdist  # noqa: E402
 from speculative_decoding_verification_90_b200 import workloads  # noqa: E402
 
 METRIC = "verified positions/s and achieved HBM GB/s vs B200 peak (spec-verify, 1 GPU)"
@@ -201,9 +202,9 @@ def time_oracle(wl, budget_s: float):
 
 
 def run_reference(args):
-    rank = int(os.environ.get("RANK", "0"))
+    rank = svdist.env_rank()[0]
     if rank != 0:
-        return 0
+        return 0  # the CPU reference runs once, on rank 0
     wl = make_workload(args.workload, args.seed)
     import oracle
     oracle.build()
@@ -249,21 +250,18 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, local, world = svdist.env_rank()
     if args.gpus != world and world > 1:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE {world}")
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        svdist.init("nccl", device=dev)
 
     from speculative_decoding_verification_90_b200.specverify import SpecVerify
 
-    # every rank verifies its own batch (weak scaling); seeds differ per rank
-    wl = make_workload(args.workload, args.seed + rank)
+    # every rank verifies its own batch (weak scaling, no data-path collective)
+    wl = make_workload(args.workload, svdist.rank_seed(args.seed, rank))
     B, G, V = wl.batch, wl.gamma, wl.vocab
     step_bytes = wl.logit_bytes
 
@@ -322,10 +320,7 @@ def run_ours(args):
     time.sleep(0.12)
     rows = sampler.stop() if sampler else []
     ms = ev0.elapsed_time(ev1)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = svdist.max_over_ranks(ms, device=dev)  # the job takes as long as its slowest rank
     stats_launch_s = kern["stats_ms"] / 1e3  # the kernel that streams every logit once
 
     # end to end through the host-buffer entry point (pinned host memory)
@@ -351,9 +346,7 @@ def run_ours(args):
         sv.run_host(*h_in[:5], wl.temperature, h_ot, h_on)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_ms, op=dist.ReduceOp.MAX)
+    e2e_ms = svdist.max_over_ranks(e0.elapsed_time(e1), device=dev)
     h2d = sum(t.numel() * t.element_size() for t in h_in)
     d2h = h_ot.numel() * 4 + h_on.numel() * 4
     st, bits = sv.status()
@@ -368,7 +361,7 @@ def run_ours(args):
         traffic = profiled_traffic(wl.name) if args.slices == 0 and args.threads == 0 else None
         positions = positions_per_step(wl) * world
         value = positions * args.steps / (ms_max / 1e3)
-        e2e_value = positions * e2e_steps / (float(e2e_ms.item()) / 1e3)
+        e2e_value = positions * e2e_steps / (e2e_ms / 1e3)
         clocks = summarize_clocks(rows, t_wall0, t_wall1)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
