@@ -184,6 +184,32 @@ sv_status specverify_profile_begin(specverify_t h, int max_runs);
  */
 sv_status specverify_profile_end(specverify_t h, float *stats_ms, float *draw_ms, int *runs);
 
+/*
+ * The verification step without a handle and without allocating: for
+ * callers that cannot call cudaMalloc (code inside a captured graph region
+ * that must not allocate, embedders whose device memory belongs to a pool
+ * they cannot reach from here, serving paths that forbid allocation).  The
+ * pages have no counterpart; this is an interface of this library only.
+ *
+ * Arguments and results are those of specverify_create + specverify_run,
+ * on the CURRENT device (its buffers and `stream` must belong to it), with
+ * the default launch shape.  The workspace is one static device array of
+ * 16 MiB that every GPU loading this library holds until the process exits;
+ * a batch whose workspace does not fit returns SV_ERR_INVALID_ARG with the
+ * needed size in specverify_last_error() and enqueues nothing.  The first
+ * call on a device looks up the array's address (and the SM count); make it
+ * before any stream capture.  The entry point calls no cudaMalloc or
+ * cudaFree.  Every call shares the one array: calls whose work overlaps on
+ * the GPU (other streams, other threads) race and must be serialised by the
+ * caller.  Each call clears what must start at zero.  Data errors show only
+ * in the outputs (num_accepted 0, tokens -1): the status word is not kept.
+ */
+sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_dtype dtype,
+                                 const void *target_logits, const void *draft_logits,
+                                 const int32_t *draft_tokens, const float *u_accept,
+                                 const float *u_resample, float temperature,
+                                 int32_t *out_tokens, int32_t *out_num_accepted, void *stream);
+
 /* Static text for a status code. */
 const char *specverify_status_string(sv_status s);
 

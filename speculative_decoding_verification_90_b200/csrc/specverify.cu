@@ -10,6 +10,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -553,3 +554,138 @@ const char* specverify_status_string(sv_status s) {
 const char* specverify_last_error(void) { return g_last_error; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point
+//
+// For callers that cannot allocate device memory: code running inside a
+// captured CUDA graph region that must not call cudaMalloc, embedders whose
+// device memory is owned by a pool or allocator they cannot reach from this
+// library, and runtimes that forbid allocation on their serving path.  The
+// workspace then lives in one file-scope device array; only its address is
+// looked up, once per device.
+// ---------------------------------------------------------------------------
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t{16} << 20;  // 16 MiB on every device
+constexpr int kNoAllocMaxDevices = 64;
+
+// Device storage of the allocation-free path.  Host code must never pass
+// this name to a kernel: on the host it only stands for the symbol, so its
+// device address is taken with cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+char* g_noalloc_base[kNoAllocMaxDevices] = {};  // device address, per device
+int g_noalloc_sms[kNoAllocMaxDevices] = {};
+
+// First call on the current device: look up the array's device address
+// (with that device current) and the SM count.
+sv_status noalloc_setup(int dev, char** base, int* sms) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (!g_noalloc_base[dev]) {
+    int major = 0, minor = 0, count = 0;
+    cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&count, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (major != 10 || minor != 0) {
+      std::snprintf(g_last_error, sizeof g_last_error,
+                    "device %d is sm_%d%d; this library is built for sm_100a only", dev, major,
+                    minor);
+      return SV_ERR_UNSUPPORTED;
+    }
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e);
+    g_noalloc_sms[dev] = count;
+    g_noalloc_base[dev] = static_cast<char*>(ptr);
+  }
+  *base = g_noalloc_base[dev];
+  *sms = g_noalloc_sms[dev];
+  return SV_OK;
+}
+
+}  // namespace
+
+extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_dtype dtype,
+                                            const void* target_logits, const void* draft_logits,
+                                            const int32_t* draft_tokens, const float* u_accept,
+                                            const float* u_resample, float temperature,
+                                            int32_t* out_tokens, int32_t* out_num_accepted,
+                                            void* stream) {
+  if (batch < 0 || gamma < 0 || gamma > specverify::kMaxGamma || vocab < 1 || vocab > (1 << 30))
+    return SV_ERR_INVALID_ARG;
+  if (dtype != SV_DTYPE_F32 && dtype != SV_DTYPE_BF16) return SV_ERR_INVALID_ARG;
+  if (batch == 0) return SV_OK;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return SV_ERR_UNSUPPORTED;
+  char* base = nullptr;
+  int sms = 0;
+  sv_status st = noalloc_setup(dev, &base, &sms);
+  if (st != SV_OK) return st;
+
+  // the same launch shape and workspace layout a handle would use, carved
+  // out of the static array (a host-side record only: nothing is allocated)
+  specverify_ctx h;
+  h.device = dev;
+  h.batch = batch;
+  h.gamma = gamma;
+  h.vocab = vocab;
+  h.dtype = dtype;
+  h.num_sms = sms;
+  {
+    const long cap = num_groups(&h) / 128;
+    h.max_slices = static_cast<int>(cap < 1 ? 1 : (cap > specverify::kMaxSlices ? specverify::kMaxSlices : cap));
+  }
+  default_shape(&h);
+  h.draw_slices = draw_shape(&h);
+  const size_t nT = static_cast<size_t>(batch) * (gamma + 1);
+  const size_t nD = static_cast<size_t>(batch) * gamma;
+  const size_t nB = static_cast<size_t>(batch);
+  const size_t nDraw =
+      nB * static_cast<size_t>((num_groups(&h) + specverify::kTile - 1) / specverify::kTile);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = round_up(off + bytes, 256);
+    return at;
+  };
+  const size_t offA = take(nT * static_cast<size_t>(h.slices) * sizeof(CtaStats));
+  const size_t offT = take(nT * sizeof(RowStat));
+  const size_t offD = take(nD * sizeof(RowStat));
+  const size_t offP = take(nD * sizeof(PosInfo));
+  const size_t offC = take(nB * sizeof(SeqDecision));
+  const size_t offW = take(nDraw * sizeof(double));
+  const size_t offK = take(nB * sizeof(unsigned));
+  const size_t offR = take(nB * sizeof(double));
+  const size_t offS = take(sizeof(unsigned));
+  if (off > kNoAllocScratchBytes) {
+    std::snprintf(g_last_error, sizeof g_last_error,
+                  "specverify_run_noalloc: this batch needs %zu bytes of scratch; the "
+                  "allocation-free entry point has %zu",
+                  off, kNoAllocScratchBytes);
+    return SV_ERR_INVALID_ARG;
+  }
+  h.partial = reinterpret_cast<CtaStats*>(base + offA);
+  h.tstat = reinterpret_cast<RowStat*>(base + offT);
+  h.dstat = reinterpret_cast<RowStat*>(base + offD);
+  h.pos = reinterpret_cast<PosInfo*>(base + offP);
+  h.decision = reinterpret_cast<SeqDecision*>(base + offC);
+  h.draw_mass = reinterpret_cast<double*>(base + offW);
+  h.draw_ticket = reinterpret_cast<unsigned*>(base + offK);
+  h.resid = reinterpret_cast<double*>(base + offR);
+  h.status = reinterpret_cast<unsigned*>(base + offS);
+
+  // the array keeps the previous call's contents: the draw tickets and the
+  // status word must start at zero
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  e = cudaMemsetAsync(h.draw_ticket, 0, nB * sizeof(unsigned), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h.status, 0, sizeof(unsigned), s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return enqueue(&h, target_logits, draft_logits, draft_tokens, u_accept, u_resample,
+                 temperature, out_tokens, out_num_accepted, s);
+}

@@ -43,6 +43,7 @@ SIGNATURES = {
     "specverify_get_launch": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "specverify_profile_begin": (_i, [_vp, _i]),
     "specverify_profile_end": (_i, [_vp, ctypes.POINTER(_f), ctypes.POINTER(_f), ctypes.POINTER(_i)]),
+    "specverify_run_noalloc": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
     "specverify_status_string": (ctypes.c_char_p, [_i]),
     "specverify_last_error": (ctypes.c_char_p, []),
 }
@@ -141,6 +142,15 @@ def specverify_profile_end(h) -> dict:
     _check(_lib.specverify_profile_end(h, ctypes.byref(a), ctypes.byref(c), ctypes.byref(n)),
            "specverify_profile_end")
     return {"stats_ms": a.value, "draw_ms": c.value, "runs": n.value}
+
+
+def specverify_run_noalloc(batch, gamma, vocab, dtype, target, draft, tokens, u_accept, u_resample,
+                           temperature, out_tokens, out_num_accepted, stream=0) -> int:
+    """The step without a handle; its workspace is a static device array (no allocation)."""
+    return _check(_lib.specverify_run_noalloc(batch, gamma, vocab, dtype, target, draft, tokens,
+                                              u_accept, u_resample, float(temperature), out_tokens,
+                                              out_num_accepted, stream),
+                  "specverify_run_noalloc")
 
 
 def specverify_status_string(status: int) -> str:
