@@ -16,7 +16,7 @@
 
 #include "verify_kernel.cuh"
 
-using specverify::CtaStats;
+using specverify::RowPartial;
 using specverify::Params;
 using specverify::PosInfo;
 using specverify::RowStat;
@@ -31,7 +31,7 @@ struct specverify_ctx {
   int draw_slices = 1; // draw blocks per sequence
   int num_sms = 148;
   void* ws = nullptr;  // one device allocation for the whole workspace
-  CtaStats* partial = nullptr;
+  RowPartial* partial = nullptr;
   RowStat* tstat = nullptr;
   RowStat* dstat = nullptr;
   PosInfo* pos = nullptr;
@@ -86,14 +86,14 @@ long num_groups(const specverify_ctx* h) {
   return (static_cast<long>(h->vocab) + ve - 1) / ve;
 }
 
-// Default launch shape of the statistics kernel: 128 threads per block, a
-// position's two rows split over `slices` blocks (at most 8) so that the
-// grid holds at least eight waves of blocks where the batch allows (the
-// last, partial wave then costs little), with at least one 16-byte group
-// per thread and row.
+// Default launch shape of the statistics kernel: 128 threads per block,
+// every logit row split over `slices` blocks (at most 8) so that the grid
+// holds about four waves of blocks where the batch allows (the last, partial
+// wave then costs little; more, smaller blocks only add per-block overhead),
+// with at least one 16-byte group per thread.
 void default_shape(specverify_ctx* h) {
   const int threads = 128;
-  const long positions = static_cast<long>(h->batch) * (h->gamma + 1);
+  const long rows = static_cast<long>(h->batch) * (2L * h->gamma + 1);
   const long slots = static_cast<long>(h->num_sms) * (1024 / threads);
   const long ngroups = num_groups(h);
   int best = 1;
@@ -102,7 +102,7 @@ void default_shape(specverify_ctx* h) {
   for (int c = 1; c <= cap; ++c) {
     if (ngroups / c < threads && c > 1) break;
     best = c;
-    if (positions * c >= 8 * slots) break;
+    if (rows * c >= 4 * slots) break;
   }
   h->slices = best;
   h->threads = threads;
@@ -154,8 +154,8 @@ cudaError_t launch_stats_nt(const Params& p, long blocks, cudaStream_t s) {
 // events[0..2] (may be null): before stats, after stats, after draw
 template <typename T, bool A>
 cudaError_t launch_step(const Params& p, int NT, cudaStream_t s, cudaEvent_t* ev) {
-  const long positions = static_cast<long>(p.batch) * (p.gamma + 1);
-  const long blocks = positions * p.slices;
+  const long rows = static_cast<long>(p.batch) * (2L * p.gamma + 1);
+  const long blocks = rows * p.slices;
   cudaError_t e = cudaSuccess;
   if (ev) e = cudaEventRecord(ev[0], s);
   if (e != cudaSuccess) return e;
@@ -298,7 +298,7 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   const size_t nD = static_cast<size_t>(batch) * gamma;
   const size_t nB = static_cast<size_t>(batch);
   h->draw_slices = draw_shape(h);
-  const size_t nPart = nT * static_cast<size_t>(h->max_slices);
+  const size_t nPart = (nT + nD) * static_cast<size_t>(h->max_slices);
   const size_t nDraw = nB * static_cast<size_t>((num_groups(h) + specverify::kTile - 1) / specverify::kTile);
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -306,7 +306,7 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
     off = round_up(off + bytes, 256);
     return at;
   };
-  const size_t offA = take(nPart * sizeof(CtaStats));
+  const size_t offA = take(nPart * sizeof(RowPartial));
   const size_t offT = take(nT * sizeof(RowStat));
   const size_t offD = take(nD * sizeof(RowStat));
   const size_t offP = take(nD * sizeof(PosInfo));
@@ -322,7 +322,7 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
     return cuda_fail(e);
   }
   char* base = static_cast<char*>(h->ws);
-  h->partial = reinterpret_cast<CtaStats*>(base + offA);
+  h->partial = reinterpret_cast<RowPartial*>(base + offA);
   h->tstat = reinterpret_cast<RowStat*>(base + offT);
   h->dstat = reinterpret_cast<RowStat*>(base + offD);
   h->pos = reinterpret_cast<PosInfo*>(base + offP);
@@ -654,7 +654,7 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
     off = round_up(off + bytes, 256);
     return at;
   };
-  const size_t offA = take(nT * static_cast<size_t>(h.slices) * sizeof(CtaStats));
+  const size_t offA = take((nT + nD) * static_cast<size_t>(h.slices) * sizeof(RowPartial));
   const size_t offT = take(nT * sizeof(RowStat));
   const size_t offD = take(nD * sizeof(RowStat));
   const size_t offP = take(nD * sizeof(PosInfo));
@@ -670,7 +670,7 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
                   off, kNoAllocScratchBytes);
     return SV_ERR_INVALID_ARG;
   }
-  h.partial = reinterpret_cast<CtaStats*>(base + offA);
+  h.partial = reinterpret_cast<RowPartial*>(base + offA);
   h.tstat = reinterpret_cast<RowStat*>(base + offT);
   h.dstat = reinterpret_cast<RowStat*>(base + offD);
   h.pos = reinterpret_cast<PosInfo*>(base + offP);

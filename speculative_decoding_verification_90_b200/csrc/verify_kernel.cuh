@@ -4,13 +4,13 @@
 // launched early through programmatic dependent launch and waiting for its
 // predecessor with a grid-dependency barrier):
 //
-//   stats   S blocks per position (b, j), j = 0..gamma, each streaming its
-//           contiguous 1/S of the vocabulary of target row (b, j) and, for
-//           j < gamma, draft row (b, j) with 128-bit coalesced loads; each
-//           thread keeps a running sum of 2^(x c - o) against a lazily raised
-//           offset o; the block writes its (o, sum) partial (step 1 of the
-//           round: softmax statistics).  No atomics, no waits: this is the
-//           kernel that moves all of the logit bytes.
+//   stats   S blocks per logit row (every target row, then every draft
+//           row), each streaming its contiguous 1/S of the row with 128-bit
+//           coalesced loads, eight in flight per thread; each thread keeps a
+//           running sum of 2^(x c - o) against a lazily raised offset o; the
+//           block writes its (o, sum) partial (step 1 of the round: softmax
+//           statistics).  No atomics, no waits, the same work in every block:
+//           this is the kernel that moves all of the logit bytes.
 //   decide  one warp per sequence, one lane per position: the lane combines
 //           the position's partials into log2 sum_i 2^(x_i c), forms q(t),
 //           p(t) and the ratio, and a warp ballot finds the first rejection n
@@ -76,12 +76,12 @@ struct PosInfo {
   int pad;
 };
 
-// one block's partial statistics of its slice of the position's two rows:
-// sum_i 2^(x_i c - o) against offset o, for the target and the draft row
-struct __align__(16) CtaStats {
-  double sT, sD;
-  float oT, oD;
-  int pad[2];
+// one block's partial statistics of its slice of one row: sum_i 2^(x_i c - o)
+// against the offset o
+struct __align__(16) RowPartial {
+  double s;
+  float o;
+  int pad;
 };
 
 // per sequence, from the decide kernel to the draw kernel
@@ -101,7 +101,7 @@ struct Params {
   const float* u_resample;   // [B]
   int32_t* out_tokens;       // [B, G+1]
   int32_t* out_num_accepted; // [B]
-  CtaStats* partial;         // [B*(G+1)*S] per-block partial statistics
+  RowPartial* partial;       // [(B*(G+1) + B*G) * S]: target rows, then draft rows
   RowStat* tstat;            // [B*(G+1)]
   RowStat* dstat;            // [B*G]
   PosInfo* pos;              // [B*G]
@@ -357,68 +357,55 @@ __device__ __forceinline__ void split2(double v, float& hi, float& lo) {
 // block-level helpers
 // ---------------------------------------------------------------------------
 
-// Streaming statistics of one block's slice of the two rows, reduced to the
-// block (offset = the block's largest thread offset); valid in thread 0.
+// Streaming statistics of one block's slice [glo, ghi) of one row, reduced to
+// the block (offset = the block's largest thread offset); valid in thread 0.
 template <typename T, int NT, bool kAligned, int kUnroll>
-__device__ __forceinline__ CtaStats slice_stats(const T* rowT, const T* rowD, bool has_draft,
-                                                long glo, long ghi, int V, float c_hi,
-                                                float c_lo) {
+__device__ __forceinline__ RowPartial slice_stats(const T* row, long glo, long ghi, int V,
+                                                  float c_hi, float c_lo) {
   constexpr int kNW = NT / kWarp;
-  __shared__ float sm_off[2][kNW];
-  __shared__ double sm_sum[2][kNW];
+  __shared__ float sm_off[kNW];
+  __shared__ double sm_sum[kNW];
   const int tid = threadIdx.x, lane = tid & (kWarp - 1), warp = tid >> 5;
 
-  float oT = -INFINITY, sT = 0.f, oD = -INFINITY, sD = 0.f;
+  float o = -INFINITY, s = 0.f;
   // consecutive threads read consecutive 16-byte groups: each warp-wide load
-  // is 512 contiguous bytes; kUnroll groups per row are in flight per thread
-  for (long g0 = glo + tid; g0 < ghi; g0 += static_cast<long>(NT) * kUnroll) {
-    uint4 vt[kUnroll], vd[kUnroll];
+  // is 512 contiguous bytes; kUnroll groups are in flight per thread
+  long g0 = glo + tid;
+  for (; g0 + static_cast<long>(NT) * (kUnroll - 1) < ghi; g0 += static_cast<long>(NT) * kUnroll) {
+    uint4 v[kUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const long g = g0 + static_cast<long>(u) * NT;
-      if (g < ghi) {
-        vt[u] = fetch_group<T, kAligned>(rowT, g, V);
-        if (has_draft) vd[u] = fetch_group<T, kAligned>(rowD, g, V);
-      }
-    }
+    for (int u = 0; u < kUnroll; ++u) v[u] = fetch_group<T, kAligned>(row, g0 + static_cast<long>(u) * NT, V);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const long g = g0 + static_cast<long>(u) * NT;
-      if (g < ghi) {
-        accumulate_group<T>(vt[u], oT, sT, c_hi, c_lo);
-        if (has_draft) accumulate_group<T>(vd[u], oD, sD, c_hi, c_lo);
-      }
-    }
+    for (int u = 0; u < kUnroll; ++u) accumulate_group<T>(v[u], o, s, c_hi, c_lo);
   }
+  if (g0 < ghi) {
+    // the last, partial round: all of its loads in flight together
+    uint4 v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long g = g0 + static_cast<long>(u) * NT;
+      if (g < ghi) v[u] = fetch_group<T, kAligned>(row, g, V);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (g0 + static_cast<long>(u) * NT < ghi) accumulate_group<T>(v[u], o, s, c_hi, c_lo);
+  }
+
   // the block's offset is its largest thread offset; each thread rescales
-  const float wT = warp_max(oT), wD = warp_max(oD);
-  if (lane == 0) {
-    sm_off[0][warp] = wT;
-    sm_off[1][warp] = wD;
-  }
+  const float wo = warp_max(o);
+  if (lane == 0) sm_off[warp] = wo;
   __syncthreads();
-  float OT = sm_off[0][0], OD = sm_off[1][0];
+  float O = sm_off[0];
 #pragma unroll
-  for (int w = 1; w < kNW; ++w) {
-    OT = fmaxf(OT, sm_off[0][w]);
-    OD = fmaxf(OD, sm_off[1][w]);
-  }
+  for (int w = 1; w < kNW; ++w) O = fmaxf(O, sm_off[w]);
   // a thread with o = -inf holds s = 0 (or NaN, which must propagate)
-  const float fT = (oT == -INFINITY) ? 0.f : ex2(oT - OT);
-  const float fD = (oD == -INFINITY) ? 0.f : ex2(oD - OD);
-  const double zT = warp_sum(static_cast<double>(sT) * static_cast<double>(fT));
-  const double zD = warp_sum(static_cast<double>(sD) * static_cast<double>(fD));
-  if (lane == 0) {
-    sm_sum[0][warp] = zT;
-    sm_sum[1][warp] = zD;
-  }
+  const float f = (o == -INFINITY) ? 0.f : ex2(o - O);
+  const double z = warp_sum(static_cast<double>(s) * static_cast<double>(f));
+  if (lane == 0) sm_sum[warp] = z;
   __syncthreads();
-  CtaStats out{0.0, 0.0, OT, OD, {0, 0}};
+  RowPartial out{0.0, O, 0};
   if (tid == 0) {
-    for (int w = 0; w < kNW; ++w) {
-      out.sT += sm_sum[0][w];
-      out.sD += sm_sum[1][w];
-    }
+    for (int w = 0; w < kNW; ++w) out.s += sm_sum[w];
   }
   return out;
 }
@@ -476,22 +463,20 @@ template <typename T, int NT, bool kAligned>
 __global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Params P) {
   constexpr int kVec = Elem<T>::kVec;
   const int G = P.gamma, V = P.vocab, S = P.slices;
+  // one unit = one block = one slice of one row; the target tensor's rows
+  // come first, then the draft tensor's, so the grid walks memory in order
   const long unit = blockIdx.x;
-  const long position = unit / S;  // b * (G+1) + j
-  const int slice = static_cast<int>(unit - position * S);
-  const int b = static_cast<int>(position / (G + 1));
-  const int j = static_cast<int>(position - static_cast<long>(b) * (G + 1));
-  const bool has_draft = j < G;
-  const T* rowT = static_cast<const T*>(P.target) + position * V;
-  const T* rowD =
-      has_draft ? static_cast<const T*>(P.draft) + (static_cast<long>(b) * G + j) * V : nullptr;
+  const long r = unit / S;
+  const int slice = static_cast<int>(unit - r * S);
+  const long nT = static_cast<long>(P.batch) * (G + 1);
+  const T* row = (r < nT) ? static_cast<const T*>(P.target) + r * V
+                          : static_cast<const T*>(P.draft) + (r - nT) * V;
   const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
   long glo = static_cast<long>(slice) * P.groups_per_slice;
   long ghi = glo + P.groups_per_slice;
   if (glo > ngroups) glo = ngroups;
   if (ghi > ngroups) ghi = ngroups;
-  const CtaStats part =
-      slice_stats<T, NT, kAligned, 4>(rowT, rowD, has_draft, glo, ghi, V, P.c_hi, P.c_lo);
+  const RowPartial part = slice_stats<T, NT, kAligned, 8>(row, glo, ghi, V, P.c_hi, P.c_lo);
   if (threadIdx.x == 0) P.partial[unit] = part;
   cudaTriggerProgrammaticLaunchCompletion();
 }
@@ -505,13 +490,13 @@ constexpr int kMaxGamma = 255;
 
 // (o, s) partials of one row combined in two passes, so that the fp64
 // exponentials of the second pass are independent of one another
-__device__ __forceinline__ double row_lse2(const CtaStats* parts, int S, bool draft, int& valid) {
+__device__ __forceinline__ double row_lse2(const RowPartial* parts, int S, int& valid) {
   float O = -INFINITY;
-  for (int r = 0; r < S; ++r) O = fmaxf(O, draft ? parts[r].oD : parts[r].oT);
+  for (int r = 0; r < S; ++r) O = fmaxf(O, parts[r].o);
   double sum = 0.0;
   for (int r = 0; r < S; ++r) {
-    const float o = draft ? parts[r].oD : parts[r].oT;
-    const double s = draft ? parts[r].sD : parts[r].sT;
+    const float o = parts[r].o;
+    const double s = parts[r].s;
     sum += (o == -INFINITY) ? s * 0.0 : s * exp2(static_cast<double>(o) - O);  // NaN survives
   }
   valid = (O != -INFINITY) && isfinite(sum) && sum > 0.0;
@@ -551,12 +536,12 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
             xd = Elem<T>::load1(static_cast<const T*>(P.draft) + pj * V, t);
           }
         }
-        const CtaStats* parts = P.partial + position * S;
+        const long nT = static_cast<long>(P.batch) * (G + 1);
         int validT = 0, validD = 1;
-        lT = row_lse2(parts, S, false, validT);
+        lT = row_lse2(P.partial + position * S, S, validT);
         P.tstat[position] = RowStat{lT, validT, 0};
         if (has_draft) {
-          lD = row_lse2(parts, S, true, validD);
+          lD = row_lse2(P.partial + (nT + pj) * S, S, validD);
           P.dstat[pj] = RowStat{lD, validD, 0};
         }
         row_bad = !validT || !validD;
