@@ -58,6 +58,7 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--slices", type=int, default=0, help="override blocks per position")
     ap.add_argument("--threads", type=int, default=0, help="override threads per CTA")
+    ap.add_argument("--draw-slices", type=int, default=0, help="override draw blocks per sequence")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     return ap.parse_args()
@@ -281,10 +282,11 @@ def run_ours(args):
     out_n = torch.empty((B,), dtype=torch.int32, device=dev)
 
     sv = SpecVerify(B, G, V, wl.dtype, local)
-    if args.slices or args.threads:
+    if args.slices or args.threads or args.draw_slices:
         c0, t0 = sv.launch()
-        sv.set_launch(args.slices or c0, args.threads or t0)
+        sv.set_launch(args.slices or c0, args.threads or t0, args.draw_slices)
     slices, threads = sv.launch()
+    sv_draw = sv.draw_slices
 
     def step(i):
         s = sets[i % n_sets]
@@ -358,7 +360,8 @@ def run_ours(args):
     if rank == 0:
         peak, peak_src = measured_peak()
         achieved = step_bytes / stats_launch_s / 1e9
-        traffic = profiled_traffic(wl.name) if args.slices == 0 and args.threads == 0 else None
+        default_shape = not (args.slices or args.threads or args.draw_slices)
+        traffic = profiled_traffic(wl.name) if default_shape else None
         positions = positions_per_step(wl) * world
         value = positions * args.steps / (ms_max / 1e3)
         e2e_value = positions * e2e_steps / (e2e_ms / 1e3)
@@ -376,7 +379,8 @@ def run_ours(args):
                        "parallelism": f"dp{world} (independent batches per GPU)",
                        "l2": ("inputs larger than L2 (%.0f MB per step, %d rotating set(s))"
                               % (step_bytes / 1e6, n_sets)),
-                       "launch": {"blocks_per_position": slices, "threads": threads}},
+                       "launch": {"blocks_per_row": slices, "threads": threads,
+                                  "draw_blocks_per_sequence": sv_draw}},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                          "algorithmic_bytes_per_launch": step_bytes,

@@ -155,19 +155,22 @@ sv_status specverify_debug_readback(specverify_t h, double *target_lse, double *
                                    double *resid_mass, void *stream);
 
 /*
- * Launch shape of the statistics kernel (the one that streams every logit):
- * each position's two rows are split over `slices` thread blocks of
- * `threads` threads (128, 256 or 512).  1 <= slices
- * <= min(64, ceil(vocab / group) / 128), group = 8 bf16 or 4 fp32 entries;
- * larger values return SV_ERR_INVALID_ARG.  specverify_create picks a shape
- * from the problem size and the SM count; this call overrides it for later
- * runs (results do not depend on the shape beyond the rounding of partial
- * sums).  Not stream-ordered: change it only while no run of the handle is
- * in flight.
+ * Launch shape.  The statistics kernel (the one that streams every logit)
+ * splits each logit row over `slices` thread blocks of `threads` threads
+ * (128, 256 or 512); 1 <= slices <= min(64, ceil(vocab / group) / 128),
+ * group = 8 bf16 or 4 fp32 entries.  The draw kernel spreads the rows drawn
+ * from over `draw_slices` blocks per sequence (1..64, at most one per four
+ * 32-group tiles of a row; 0 or less restores the default).  Invalid values
+ * return SV_ERR_INVALID_ARG.  specverify_create picks a shape from the
+ * problem size and the SM count; this call overrides it for later runs
+ * (results do not depend on the shape beyond the rounding of partial sums).
+ * Not stream-ordered: change it only while no run of the handle is in flight.
  */
-sv_status specverify_set_launch(specverify_t h, int slices, int threads);
+sv_status specverify_set_launch(specverify_t h, int slices, int threads, int draw_slices);
+
 /* Current shape and the largest `slices` this handle accepts (any pointer may be NULL). */
-sv_status specverify_get_launch(specverify_t h, int *slices, int *threads, int *max_slices);
+sv_status specverify_get_launch(specverify_t h, int *slices, int *threads, int *max_slices,
+                                int *draw_slices);
 
 /*
  * Per-kernel timing of the next `max_runs` runs of the handle: each run then

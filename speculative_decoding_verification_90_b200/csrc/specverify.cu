@@ -474,20 +474,26 @@ sv_status specverify_debug_readback(specverify_t h, double* target_lse, double* 
   return SV_OK;
 }
 
-sv_status specverify_set_launch(specverify_t h, int slices, int threads) {
+sv_status specverify_set_launch(specverify_t h, int slices, int threads, int draw_slices) {
   if (!h) return SV_ERR_INVALID_ARG;
   if (slices < 1 || slices > h->max_slices) return SV_ERR_INVALID_ARG;
   if (threads != 128 && threads != 256 && threads != 512) return SV_ERR_INVALID_ARG;
+  const long ntiles = (num_groups(h) + specverify::kTile - 1) / specverify::kTile;
+  if (draw_slices > 64 || (draw_slices > 1 && draw_slices > ntiles / specverify::kDrawWarps))
+    return SV_ERR_INVALID_ARG;
   h->slices = slices;
   h->threads = threads;
+  h->draw_slices = (draw_slices >= 1) ? draw_slices : draw_shape(h);
   return SV_OK;
 }
 
-sv_status specverify_get_launch(specverify_t h, int* slices, int* threads, int* max_slices) {
+sv_status specverify_get_launch(specverify_t h, int* slices, int* threads, int* max_slices,
+                                int* draw_slices) {
   if (!h) return SV_ERR_INVALID_ARG;
   if (max_slices) *max_slices = h->max_slices;
   if (slices) *slices = h->slices;
   if (threads) *threads = h->threads;
+  if (draw_slices) *draw_slices = h->draw_slices;
   return SV_OK;
 }
 

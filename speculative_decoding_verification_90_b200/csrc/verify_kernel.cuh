@@ -90,7 +90,8 @@ struct SeqDecision {
   int n;               // accepted drafts
   int mode;            // kDraw*
   unsigned stat_bits;  // data errors found
-  int pad;
+  // the draw's float constants (see DrawConsts), formed once in fp64
+  float lt_hi, k_hi, k_lo, fT;
 };
 
 struct Params {
@@ -294,29 +295,27 @@ __device__ __forceinline__ void warp_range(long clo, long chi, int w, int nwarps
 
 struct DrawConsts {
   float c_hi, c_lo;
-  float lt_hi;   // log2 sum 2^(x c) of the target row, rounded to float ...
-  float ld_hi;   // ... and of the draft row
+  float lt_hi;   // log2 sum 2^(x c) of the target row, rounded to float
   float k_hi, k_lo;  // K = lT - lD, two-float
-  float rD;      // 2^(lt_lo - ld_lo): the draft's share of the two roundings
   float fT;      // 2^(-lt_lo): applied to every sum of group masses
 };
 
-// Taylor coefficients of 2^L - 1 = sum_k (ln 2)^k L^k / k!, k = 1..6
+// Taylor coefficients of 2^L - 1 = sum_k (ln 2)^k L^k / k!, k = 1..5
 constexpr float kA1 = 0.6931471805599453f;
 constexpr float kA2 = 0.2402265069591007f;
 constexpr float kA3 = 0.055504108664821576f;
 constexpr float kA4 = 0.009618129107628477f;
 constexpr float kA5 = 0.0013333558146428441f;
-constexpr float kA6 = 0.00015403530393381606f;
 
 // r / fT for the VEC elements of one group: residual max(0, q - p) or target
-// q; the caller multiplies sums of r by fT.  Branch-free: L = log2(q/p)
-// comes from the logit difference (exact for bf16 inputs); L <= 0 gives 0,
-// L >= 1/4 gives q - p (q >= 1.19 p, so at most 2.6 bits cancel),
-// 0 < L < 1/4 gives p (2^L - 1) from its Taylor series in L (to L^6,
-// truncation below 6e-9 relative).  The infinite cases need no test: a
-// draft logit of -inf gives L = +inf and r = q - 0; a target logit of -inf
-// gives L = -inf (or NaN) and r = 0.
+// q; the caller multiplies sums of r by fT.  L = log2(q/p) comes from the
+// logit difference (exact for bf16 inputs) and p = q 2^-L.  L >= 1/8 gives
+// q - p (q >= 1.09 p: at most 3.6 bits cancel); 0 < L < 1/8 gives
+// p (2^L - 1) from its Taylor series in L (to L^5, truncation below 7e-9
+// relative); L <= 0 gives q - p <= 0, which the final max(., 0) turns into 0.
+// The infinite cases need no test: a draft logit of -inf gives L = +inf,
+// p = 0 and r = q; a target logit of -inf gives q = 0, L = -inf and r = 0
+// (the NaN of 0 * 2^inf is discarded by the selects).
 template <typename T, int kMode>
 __device__ __forceinline__ void group_mass(const uint4& vt, const uint4& vd, const DrawConsts& k,
                                            float (&r)[Elem<T>::kVec]) {
@@ -332,18 +331,17 @@ __device__ __forceinline__ void group_mass(const uint4& vt, const uint4& vd, con
 #pragma unroll
     for (int e = 0; e < kVec; ++e) {
       const float q = ex2(arg2(xt[e], k.c_hi, k.c_lo, k.lt_hi));
-      const float p = ex2(arg2(xd[e], k.c_hi, k.c_lo, k.ld_hi)) * k.rD;
       const float dx = xt[e] - xd[e];
       const float L = fmaf(dx, k.c_hi, -k.k_hi) + fmaf(dx, k.c_lo, -k.k_lo);
-      float t = kA6;
-      t = fmaf(t, L, kA5);
+      const float p = q * ex2(-L);
+      float t = kA5;
       t = fmaf(t, L, kA4);
       t = fmaf(t, L, kA3);
       t = fmaf(t, L, kA2);
       t = fmaf(t, L, kA1);
       const float small = p * (t * L);
-      const float res = (L >= 0.25f) ? q - p : small;
-      r[e] = (L > 0.f) ? res : 0.f;
+      const float res = (L > 0.f && L < 0.125f) ? small : q - p;
+      r[e] = fmaxf(res, 0.f);  // NaN (0 * inf) becomes 0 here
     }
   }
 }
@@ -586,7 +584,7 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
       if (lane == 0) {
         P.out_num_accepted[b] = 0;
         P.resid_mass[b] = NAN;
-        P.decision[b] = SeqDecision{0.0, 0.0, 0, kDrawNone, bits, 0};
+        P.decision[b] = SeqDecision{0.0, 0.0, 0, kDrawNone, bits, 0.f, 0.f, 0.f, 1.f};
         atomicOr(P.status, bits);
       }
     } else {
@@ -597,7 +595,13 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
       }
       if (lane == 0) {
         P.out_num_accepted[b] = n;
-        P.decision[b] = SeqDecision{lT_n, lD_n, n, (n < G) ? kDrawResidual : kDrawTarget, 0u, 0};
+        SeqDecision d{lT_n, lD_n, n, (n < G) ? kDrawResidual : kDrawTarget, 0u,
+                      0.f, 0.f, 0.f, 1.f};
+        float lt_lo;
+        split2(lT_n, d.lt_hi, lt_lo);
+        split2(lT_n - lD_n, d.k_hi, d.k_lo);
+        d.fT = static_cast<float>(exp2(-static_cast<double>(lt_lo)));
+        P.decision[b] = d;
       }
     }
   }
@@ -614,39 +618,54 @@ constexpr int kTile = 32;  // groups per tile of the draw's mass table
 
 // Mass of each 32-group tile of [tlo, thi) (tiles of the row, warp w takes
 // tiles w, w + 4, ...); lane 0 of the warp stores the tile's mass in `table`.
+// Software-pipelined: the next two tiles' loads are in flight while the
+// current two are reduced.
 template <typename T, bool kAligned>
 __device__ __forceinline__ void tile_masses(int mode, const T* drawT, const T* drawD,
                                             const DrawConsts& k, long tlo, long thi,
                                             long ngroups, int V, double* table) {
   constexpr int kVec = Elem<T>::kVec;
-  constexpr int kUnroll = 4;
+  constexpr int kPair = 2;  // tiles per pipeline stage
   const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x >> 5;
-  for (long t0 = tlo + warp; t0 < thi; t0 += static_cast<long>(kDrawWarps) * kUnroll) {
-    uint4 vt[kUnroll], vd[kUnroll];
+  const long first = tlo + warp;
+  if (first >= thi) return;
+  const long count = (thi - first + kDrawWarps - 1) / kDrawWarps;  // this warp's tiles
+  auto load = [&](long kk, uint4 (&vt)[kPair], uint4 (&vd)[kPair]) {
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const long g = (t0 + static_cast<long>(u) * kDrawWarps) * kTile + lane;
-      if (t0 + u * kDrawWarps < thi && g < ngroups) {
+    for (int u = 0; u < kPair; ++u) {
+      const long g = (first + (kk + u) * kDrawWarps) * kTile + lane;
+      if (kk + u < count && g < ngroups) {
         vt[u] = fetch_group<T, kAligned>(drawT, g, V);
         vd[u] = (mode == kDrawResidual) ? fetch_group<T, kAligned>(drawD, g, V) : vt[u];
       }
     }
+  };
+  uint4 ct[kPair], cd[kPair];
+  load(0, ct, cd);
+  for (long kk = 0; kk < count; kk += kPair) {
+    uint4 nt[kPair], nd[kPair];
+    load(kk + kPair, nt, nd);
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const long tile = t0 + static_cast<long>(u) * kDrawWarps;
-      if (tile < thi) {  // warp-uniform
+    for (int u = 0; u < kPair; ++u) {
+      if (kk + u < count) {  // warp-uniform
+        const long tile = first + (kk + u) * kDrawWarps;
         const long g = tile * kTile + lane;
         float gs = 0.f;
         if (g < ngroups) {
           float r[kVec];
-          if (mode == kDrawResidual) group_mass<T, kDrawResidual>(vt[u], vd[u], k, r);
-          else group_mass<T, kDrawTarget>(vt[u], vd[u], k, r);
+          if (mode == kDrawResidual) group_mass<T, kDrawResidual>(ct[u], cd[u], k, r);
+          else group_mass<T, kDrawTarget>(ct[u], cd[u], k, r);
 #pragma unroll
           for (int e = 0; e < kVec; ++e) gs += r[e];
         }
         const double z = warp_sum(static_cast<double>(gs)) * k.fT;
         if (lane == 0) table[tile] = z;
       }
+    }
+#pragma unroll
+    for (int u = 0; u < kPair; ++u) {
+      ct[u] = nt[u];
+      cd[u] = nd[u];
     }
   }
 }
@@ -718,7 +737,6 @@ __global__ void __launch_bounds__(kDrawThreads, 8) draw_kernel(const Params P) {
   const SeqDecision d = P.decision[b];
   if (d.mode == kDrawNone) return;  // the decide kernel wrote the error outcome
   const int n = d.n;
-  const double lT = d.lT, lD = d.lD;
   const long bo = static_cast<long>(b) * (G + 1);
 
   // ---- step 4: residual (n < gamma) or bonus (n == gamma) draw ----
@@ -730,12 +748,10 @@ __global__ void __launch_bounds__(kDrawThreads, 8) draw_kernel(const Params P) {
   DrawConsts k;
   k.c_hi = P.c_hi;
   k.c_lo = P.c_lo;
-  float lt_lo, ld_lo;
-  split2(lT, k.lt_hi, lt_lo);
-  split2(lD, k.ld_hi, ld_lo);
-  split2(lT - lD, k.k_hi, k.k_lo);
-  k.rD = static_cast<float>(exp2(static_cast<double>(lt_lo) - ld_lo));
-  k.fT = static_cast<float>(exp2(-static_cast<double>(lt_lo)));
+  k.lt_hi = d.lt_hi;
+  k.k_hi = d.k_hi;
+  k.k_lo = d.k_lo;
+  k.fT = d.fT;
 
   const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
   const long ntiles = (ngroups + kTile - 1) / kTile;
@@ -760,53 +776,89 @@ __global__ void __launch_bounds__(kDrawThreads, 8) draw_kernel(const Params P) {
   // ---- the block that finishes the sequence locates u * Z ----
   __shared__ long sm_tile;
   __shared__ double sm_tl, sm_Z;
-  const long per = (ntiles + kDrawThreads - 1) / kDrawThreads;  // tiles per thread, in order
-  const long a0 = tid * per < ntiles ? tid * per : ntiles;
-  const long a1 = (a0 + per < ntiles) ? a0 + per : ntiles;
   unsigned extra_bits = 0;
   for (int attempt = 0; attempt < 2; ++attempt) {
-    double mine = 0.0;
-    for (long t = a0; t < a1; ++t) mine += __ldcg(&table[t]);
-    double incl, excl, tot;
-    block_scan<kDrawThreads>(mine, incl, excl, tot);
-    if (tot > 0.0 || mode != kDrawResidual) {
-      const double target = static_cast<double>(P.u_resample[b]) * tot;
-      if (tid == 0) {
-        sm_Z = tot;
-        sm_tile = -1;
-      }
-      __syncthreads();
-      if (excl <= target && incl > target) {
-        // this thread's tiles hold u * Z: walk them in order
-        double acc = excl;
-        for (long t = a0; t < a1; ++t) {
-          const double z = __ldcg(&table[t]);
-          if (z > 0.0 && acc + z > target) {
-            sm_tile = t;
-            sm_tl = target - acc;
-            break;
+    // each thread owns a contiguous run of up to kRun tiles per round, loaded
+    // together (independent loads), summed in index order
+    constexpr int kRun = 8;
+    const long per_round = static_cast<long>(kDrawThreads) * kRun;
+    double base = 0.0;  // mass of the rounds before this one
+    long found_tile = -1;
+    double found_tl = 0.0;
+    bool have_last = false;
+    long last_tile = -1;
+    const double target0 = static_cast<double>(P.u_resample[b]);
+    // pass 1: Z (all rounds)
+    double Z = 0.0;
+    for (long r0 = 0; r0 < ntiles; r0 += per_round) {
+      const long a0 = r0 + static_cast<long>(tid) * kRun;
+      double v[kRun];
+#pragma unroll
+      for (int q = 0; q < kRun; ++q) v[q] = (a0 + q < ntiles) ? __ldcg(&table[a0 + q]) : 0.0;
+      double mine = 0.0;
+#pragma unroll
+      for (int q = 0; q < kRun; ++q) mine += v[q];
+      double incl, excl, tot;
+      block_scan<kDrawThreads>(mine, incl, excl, tot);
+      Z += tot;
+    }
+    if (Z > 0.0 || mode != kDrawResidual) {
+      const double target = target0 * Z;
+      // pass 2: the round, thread and tile holding u * Z
+      for (long r0 = 0; r0 < ntiles; r0 += per_round) {
+        const long a0 = r0 + static_cast<long>(tid) * kRun;
+        double v[kRun];
+#pragma unroll
+        for (int q = 0; q < kRun; ++q) v[q] = (a0 + q < ntiles) ? __ldcg(&table[a0 + q]) : 0.0;
+        double mine = 0.0;
+#pragma unroll
+        for (int q = 0; q < kRun; ++q) mine += v[q];
+        double incl, excl, tot;
+        block_scan<kDrawThreads>(mine, incl, excl, tot);
+        if (base + excl <= target && base + incl > target) {
+          double acc = base + excl;
+#pragma unroll
+          for (int q = 0; q < kRun; ++q) {
+            if (found_tile < 0 && v[q] > 0.0 && acc + v[q] > target) {
+              found_tile = a0 + q;
+              found_tl = target - acc;
+            }
+            acc += v[q];
           }
-          acc += z;
         }
+        // remember the last tile with mass (rounding fallback)
+#pragma unroll
+        for (int q = 0; q < kRun; ++q)
+          if (v[q] > 0.0) {
+            have_last = true;
+            last_tile = a0 + q;
+          }
+        base += tot;
       }
-      // rounding can leave u * Z at or beyond the last tile with mass: use
-      // that tile, with the point at its end
-      const bool has = (a1 > a0) && incl > excl;  // this thread owns mass
-      const unsigned own = __ballot_sync(0xffffffffu, has);
-      __shared__ int sm_lastthread[kDrawWarps];
-      if ((tid & (kWarp - 1)) == 0) sm_lastthread[tid >> 5] = own ? (tid & ~(kWarp - 1)) + 31 - __clz(own) : -1;
+      // publish: the owning tile, else the last tile with mass
+      __shared__ long sm_found, sm_lastt[kDrawThreads / kWarp];
+      if (tid == 0) sm_found = -1;
       __syncthreads();
-      if (tid == 0 && sm_tile < 0) {
-        int lt = -1;
-        for (int w = 0; w < kDrawWarps; ++w) lt = max(lt, sm_lastthread[w]);
-        long bt = -1;
-        if (lt >= 0) {
-          const long b0 = static_cast<long>(lt) * per;
-          for (long t = b0; t < b0 + per && t < ntiles; ++t)
-            if (__ldcg(&table[t]) > 0.0) bt = t;
+      if (found_tile >= 0) {
+        sm_found = found_tile;
+        sm_tl = found_tl;
+      }
+      const long wl = have_last ? last_tile : -1;
+      long m = wl;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if ((tid & (kWarp - 1)) == 0) sm_lastt[tid >> 5] = m;
+      __syncthreads();
+      if (tid == 0) {
+        sm_Z = Z;
+        if (sm_found >= 0) {
+          sm_tile = sm_found;
+        } else {
+          long lt = -1;
+          for (int w = 0; w < kDrawThreads / kWarp; ++w) lt = max(lt, sm_lastt[w]);
+          sm_tile = lt;
+          sm_tl = INFINITY;  // the tile's last index with mass
         }
-        sm_tile = bt;
-        sm_tl = INFINITY;
       }
       __syncthreads();
       break;

@@ -39,8 +39,9 @@ SIGNATURES = {
     "specverify_destroy": (None, [_vp]),
     "specverify_get_status": (_i, [_vp, _vp, _u32p]),
     "specverify_debug_readback": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
-    "specverify_set_launch": (_i, [_vp, _i, _i]),
-    "specverify_get_launch": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "specverify_set_launch": (_i, [_vp, _i, _i, _i]),
+    "specverify_get_launch": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i),
+                                   ctypes.POINTER(_i)]),
     "specverify_profile_begin": (_i, [_vp, _i]),
     "specverify_profile_end": (_i, [_vp, ctypes.POINTER(_f), ctypes.POINTER(_f), ctypes.POINTER(_i)]),
     "specverify_run_noalloc": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
@@ -120,16 +121,17 @@ def specverify_debug_readback(h, *ptrs, stream=0) -> int:
     return _check(_lib.specverify_debug_readback(h, *ptrs, stream), "specverify_debug_readback")
 
 
-def specverify_set_launch(h, slices: int, threads: int) -> int:
-    return _check(_lib.specverify_set_launch(h, slices, threads), "specverify_set_launch")
+def specverify_set_launch(h, slices: int, threads: int, draw_slices: int = 0) -> int:
+    return _check(_lib.specverify_set_launch(h, slices, threads, draw_slices),
+                  "specverify_set_launch")
 
 
-def specverify_get_launch(h) -> tuple[int, int, int]:
-    """(slices, threads, max_slices) of the handle."""
-    c, t, m = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
-    _check(_lib.specverify_get_launch(h, ctypes.byref(c), ctypes.byref(t), ctypes.byref(m)),
-           "specverify_get_launch")
-    return c.value, t.value, m.value
+def specverify_get_launch(h) -> tuple[int, int, int, int]:
+    """(slices, threads, max_slices, draw_slices) of the handle."""
+    c, t, m, k = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(_lib.specverify_get_launch(h, ctypes.byref(c), ctypes.byref(t), ctypes.byref(m),
+                                      ctypes.byref(k)), "specverify_get_launch")
+    return c.value, t.value, m.value, k.value
 
 
 def specverify_profile_begin(h, max_runs: int) -> int:
@@ -259,8 +261,12 @@ class SpecVerify:
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
         return specverify_get_status(self.handle, sp)
 
-    def set_launch(self, slices: int, threads: int):
-        specverify_set_launch(self.handle, slices, threads)
+    def set_launch(self, slices: int, threads: int, draw_slices: int = 0):
+        specverify_set_launch(self.handle, slices, threads, draw_slices)
+
+    @property
+    def draw_slices(self) -> int:
+        return specverify_get_launch(self.handle)[3]
 
     def launch(self) -> tuple[int, int]:
         """(slices per position, threads per block)."""

@@ -85,5 +85,5 @@ def test_null_handle_is_rejected(lib_path):
     lib = S._lib
     assert lib.specverify_run(None, None, None, None, None, None, 1.0, None, None, None) == \
         S.SV_ERR_INVALID_ARG
-    assert lib.specverify_set_launch(None, 1, 256) == S.SV_ERR_INVALID_ARG
+    assert lib.specverify_set_launch(None, 1, 256, 0) == S.SV_ERR_INVALID_ARG
     lib.specverify_destroy(None)

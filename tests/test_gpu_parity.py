@@ -144,6 +144,17 @@ def test_launch_shapes(slices, threads):
     assert_parity(s)
 
 
+@pytest.mark.parametrize("draw_slices", [1, 2, 5, 31])
+def test_draw_shapes(draw_slices):
+    wl = _small(22, 20, 4, 32000, "bf16", T=0.9)
+    from speculative_decoding_verification_90_b200.specverify import SpecVerify
+    with SpecVerify(wl.batch, wl.gamma, wl.vocab, "bf16") as sv:
+        s0, t0 = sv.launch()
+        sv.set_launch(s0, t0, draw_slices)
+        g = gpu_run(wl, sv=sv)
+    assert_parity(compare(wl, g, oracle_run(wl)))
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_misaligned_pointers_take_scalar_path(dtype):
     """Logit tensors offset by one element from a 16-byte boundary."""
@@ -295,9 +306,9 @@ def test_invalid_arguments_rejected_before_launch():
         with pytest.raises(S.SpecVerifyError):
             S.specverify_run(h, x.data_ptr() + 1, x.data_ptr(), i.data_ptr(), x.data_ptr(),
                              x.data_ptr(), 1.0, i.data_ptr(), i.data_ptr(), 0)
-        for c, t in ((0, 256), (9, 256), (2, 100)):
+        for c, t, d in ((0, 256, 0), (9, 256, 0), (2, 100, 0), (1, 128, 65)):
             with pytest.raises(S.SpecVerifyError):
-                S.specverify_set_launch(h, c, t)
+                S.specverify_set_launch(h, c, t, d)
     finally:
         S.specverify_destroy(h)
     for args in ((-1, 2, 100), (4, -1, 100), (4, 2, 0), (4, 256, 100)):
