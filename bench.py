@@ -14,6 +14,10 @@ logits read once = B (2 gamma + 1) V * sizeof(logit).
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload multibranch|b64_g8_v128256|b8_g3_v32000|char_level]
 
+For the multi-branch batch the same positions are also timed through the
+shared-row entry point (each distinct target/draft row once, plus row maps),
+reported under "shared_rows".
+
 N > 1 runs under torch.distributed.run, one rank per GPU: every rank verifies
 its own batch (weak scaling, no data-path collective).  ``--impl reference``
 times the CPU oracle on the host cores on a bounded sample of the workload.
@@ -61,6 +65,8 @@ def parse():
     ap.add_argument("--draw-slices", type=int, default=0, help="override draw blocks per sequence")
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-shared-rows", action="store_true",
+                    help="skip the timing of the shared-row entry point (multibranch)")
     return ap.parse_args()
 
 
@@ -352,6 +358,11 @@ def run_ours(args):
     h2d = sum(t.numel() * t.element_size() for t in h_in)
     d2h = h_ot.numel() * 4 + h_on.numel() * 4
     st, bits = sv.status()
+
+    # the same batch through the shared-row entry point: each distinct row once
+    shared = None
+    if wl.mapped and not args.no_shared_rows:
+        shared = time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local)
     sv.close()
     # tokens settled per step on this rank = accepted + 1 per sequence (last device step)
     emitted = int((out_n.cpu().numpy().astype(np.int64) + 1).sum())
@@ -392,17 +403,70 @@ def run_ours(args):
             "emitted_tokens_per_step": emitted,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-            "gpu_launches": 2 * args.steps,
+            "gpu_launches": 3 * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
             "status_after": st,
         }
+        if shared is not None:
+            sh_bytes = shared["bytes"]
+            sh_ach = sh_bytes / (shared["stats_ms"] / 1e3) / 1e9
+            line["shared_rows"] = {
+                "entry": "specverify_run_mapped", "value": positions * args.steps
+                / (shared["ms_max"] / 1e3), "unit": UNIT,
+                "ms_per_step": shared["ms_max"] / args.steps,
+                "distinct_row_bytes_per_step": sh_bytes,
+                "stats_us": 1e3 * shared["stats_ms"], "decide_and_draw_us": 1e3 * shared["draw_ms"],
+                "stats_hbm_gbs": sh_ach, "stats_frac": sh_ach / peak,
+                "l2": "inputs larger than L2 (%.0f MB per step, %d rotating set(s))"
+                      % (sh_bytes / 1e6, shared["sets"]),
+                "status_after": shared["status"]}
     if world > 1:
         dist.barrier(device_ids=[local])
         dist.destroy_process_group()
     if line is not None:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local):
+    """Time specverify_run_mapped on the workload's distinct rows and row maps."""
+    import torch
+    import torch.distributed as dist
+    m = wl.meta
+    nbytes = wl.unique_logit_bytes
+    n_sets = max(1, math.ceil(2 * L2_BYTES / nbytes)) if nbytes < 2 * L2_BYTES else 1
+    base = {"target_rows": put(m["target_rows"], True), "target_map": put(m["target_map"], False),
+            "draft_rows": put(m["draft_rows"], True), "draft_map": put(m["draft_map"], False),
+            "tokens": put(wl.tokens, False), "u_accept": put(wl.u_accept, False),
+            "u_resample": put(wl.u_resample, False)}
+    sets = [base] + [{k: v.clone() for k, v in base.items()} for _ in range(n_sets - 1)]
+
+    def step(i):
+        d = sets[i % n_sets]
+        sv.run_mapped(d["target_rows"], d["target_map"], d["draft_rows"], d["draft_map"],
+                      d["tokens"], d["u_accept"], d["u_resample"], wl.temperature, out_t, out_n)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sv.profile_begin(args.steps)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for i in range(args.steps):
+        step(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    kern = sv.profile_end()
+    ms_max = svdist.max_over_ranks(ev0.elapsed_time(ev1), device=dev)
+    st, _ = sv.status()
+    del sets, base
+    return {"ms_max": ms_max, "stats_ms": kern["stats_ms"], "draw_ms": kern["draw_ms"],
+            "bytes": nbytes, "sets": n_sets, "status": st}
 
 
 def main():

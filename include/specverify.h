@@ -75,7 +75,8 @@ typedef enum {
   SV_ERR_UNSUPPORTED = 4,  /* the device is not an sm_100 (B200-class) GPU */
   SV_ERR_TOKEN_RANGE = 16, /* device: some draft token was outside [0, V) */
   SV_ERR_NONFINITE = 17,   /* device: some logit row held NaN/+inf or only -inf */
-  SV_WARN_ZERO_MASS = 18   /* device: a residual had zero mass; drew from q_n instead */
+  SV_WARN_ZERO_MASS = 18,  /* device: a residual had zero mass; drew from q_n instead */
+  SV_ERR_ROW_INDEX = 19    /* device: a row map entry was outside the rows given */
 } sv_status;
 
 /*
@@ -126,6 +127,36 @@ sv_status specverify_run_host(specverify_t h, const void *target_logits,
                               float temperature, int32_t *out_tokens,
                               int32_t *out_num_accepted, void *stream);
 
+/*
+ * Multi-branch verification over shared logit rows.  Where many candidate
+ * branches of one sequence share a prefix, their target and draft rows at the
+ * shared positions are the same rows; the SpecFold explainer (blog.ontle.kr,
+ * post 356: the multi-branch paragraph and the implementer's note, where the
+ * shared cache is read through a strided view instead of a per-branch copy)
+ * describes that reuse.  This entry point takes each distinct row once and a
+ * map from every (branch, position) to its row, so the step reads
+ * (n_target_rows + n_draft_rows) rows of V logits instead of B (2 gamma + 1):
+ *   target_rows   [n_target_rows, vocab] dtype, 1 <= n_target_rows <= batch (gamma+1)
+ *   target_map    int32 [batch, gamma+1]: row of target_rows of each position
+ *   draft_rows    [n_draft_rows, vocab]  dtype, 1 <= n_draft_rows <= batch gamma
+ *   draft_map     int32 [batch, gamma]: row of draft_rows of each draft position
+ * and the rest as specverify_run.  Every branch is a sequence b of the batch;
+ * the result equals specverify_run on the rows the maps pick out
+ * (target_logits[b, j] = target_rows[target_map[b, j]], likewise for drafts).
+ * Each distinct row's softmax statistics are computed once and shared by
+ * every position mapped to it.  All pointers are device pointers; the maps
+ * must be 4-byte aligned.  When gamma == 0 the draft arguments are ignored.
+ * A map entry outside [0, n rows) makes that sequence emit nothing (as a
+ * data error does) and records SV_ERR_ROW_INDEX in the status word.
+ */
+sv_status specverify_run_mapped(specverify_t h, const void *target_rows, int n_target_rows,
+                                const int32_t *target_map, const void *draft_rows,
+                                int n_draft_rows, const int32_t *draft_map,
+                                const int32_t *draft_tokens, const float *u_accept,
+                                const float *u_resample, float temperature,
+                                int32_t *out_tokens, int32_t *out_num_accepted,
+                                void *stream);
+
 /* Free the handle and everything it owns.  NULL is ignored.  Waits for the
  * device work of the handle to finish first. */
 void specverify_destroy(specverify_t h);
@@ -133,9 +164,10 @@ void specverify_destroy(specverify_t h);
 /*
  * Wait for `stream`, read and clear the handle's device status word.
  * Returns the most severe condition seen since the last call:
- * SV_ERR_TOKEN_RANGE, then SV_ERR_NONFINITE, then SV_WARN_ZERO_MASS, else
- * SV_OK.  `*bits` (may be NULL) receives the raw bit set (1: token range,
- * 2: non-finite row, 4: zero residual mass).
+ * SV_ERR_ROW_INDEX, then SV_ERR_TOKEN_RANGE, then SV_ERR_NONFINITE, then
+ * SV_WARN_ZERO_MASS, else SV_OK.  `*bits` (may be NULL) receives the raw bit
+ * set (1: token range, 2: non-finite row, 4: zero residual mass, 8: row map
+ * entry out of range).
  */
 sv_status specverify_get_status(specverify_t h, void *stream, uint32_t *bits);
 

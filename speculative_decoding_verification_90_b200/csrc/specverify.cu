@@ -154,7 +154,7 @@ cudaError_t launch_stats_nt(const Params& p, long blocks, cudaStream_t s) {
 // events[0..2] (may be null): before stats, after stats, after draw
 template <typename T, bool A>
 cudaError_t launch_step(const Params& p, int NT, cudaStream_t s, cudaEvent_t* ev) {
-  const long rows = static_cast<long>(p.batch) * (2L * p.gamma + 1);
+  const long rows = p.target_rows + p.draft_rows;
   const long blocks = rows * p.slices;
   cudaError_t e = cudaSuccess;
   if (ev) e = cudaEventRecord(ev[0], s);
@@ -185,13 +185,20 @@ cudaError_t launch_dtype(const Params& p, int NT, bool aligned, cudaStream_t s, 
 
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Row maps null: the logit buffers hold one row per position, [B, G+1, V] and
+// [B, G, V].  Otherwise `target_rows` / `draft_rows` rows that the maps index.
 sv_status enqueue(specverify_t h, const void* target, const void* draft, const int32_t* tokens,
                   const float* u_accept, const float* u_resample, float temperature,
-                  int32_t* out_tokens, int32_t* out_num_accepted, cudaStream_t stream) {
+                  int32_t* out_tokens, int32_t* out_num_accepted, cudaStream_t stream,
+                  const int32_t* target_map = nullptr, const int32_t* draft_map = nullptr,
+                  long target_rows = -1, long draft_rows = -1) {
   const int G = h->gamma;
   const size_t es = elem_size(h->dtype);
   if (!target || !u_resample || !out_tokens || !out_num_accepted) return SV_ERR_INVALID_ARG;
   if (G > 0 && (!draft || !tokens || !u_accept)) return SV_ERR_INVALID_ARG;
+  if (target_rows < 0) target_rows = static_cast<long>(h->batch) * (G + 1);
+  if (draft_rows < 0) draft_rows = static_cast<long>(h->batch) * G;
+  if (!aligned_to(target_map, 4) || !aligned_to(draft_map, 4)) return SV_ERR_INVALID_ARG;
   if (!aligned_to(target, es) || (G > 0 && !aligned_to(draft, es))) return SV_ERR_INVALID_ARG;
   if (!aligned_to(tokens, 4) || !aligned_to(u_accept, 4) || !aligned_to(u_resample, 4) ||
       !aligned_to(out_tokens, 4) || !aligned_to(out_num_accepted, 4))
@@ -210,6 +217,10 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
   Params p;
   p.target = target;
   p.draft = draft;
+  p.target_map = target_map;
+  p.draft_map = draft_map;
+  p.target_rows = target_rows;
+  p.draft_rows = draft_rows;
   p.tokens = tokens;
   p.u_accept = u_accept;
   p.u_resample = u_resample;
@@ -354,6 +365,27 @@ sv_status specverify_run(specverify_t h, const void* target_logits, const void* 
                  temperature, out_tokens, out_num_accepted, static_cast<cudaStream_t>(stream));
 }
 
+sv_status specverify_run_mapped(specverify_t h, const void* target_rows, int n_target_rows,
+                                const int32_t* target_map, const void* draft_rows,
+                                int n_draft_rows, const int32_t* draft_map,
+                                const int32_t* draft_tokens, const float* u_accept,
+                                const float* u_resample, float temperature, int32_t* out_tokens,
+                                int32_t* out_num_accepted, void* stream) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  if (h->batch == 0) return SV_OK;
+  const int G = h->gamma;
+  const long nT = static_cast<long>(h->batch) * (G + 1);
+  const long nD = static_cast<long>(h->batch) * G;
+  if (!target_map || n_target_rows < 1 || n_target_rows > nT) return SV_ERR_INVALID_ARG;
+  if (G > 0 && (!draft_map || n_draft_rows < 1 || n_draft_rows > nD)) return SV_ERR_INVALID_ARG;
+  if (G == 0) n_draft_rows = 0;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  return enqueue(h, target_rows, draft_rows, draft_tokens, u_accept, u_resample, temperature,
+                 out_tokens, out_num_accepted, static_cast<cudaStream_t>(stream), target_map,
+                 G > 0 ? draft_map : nullptr, n_target_rows, n_draft_rows);
+}
+
 sv_status specverify_run_host(specverify_t h, const void* target_logits,
                               const void* draft_logits, const int32_t* draft_tokens,
                               const float* u_accept, const float* u_resample, float temperature,
@@ -436,6 +468,7 @@ sv_status specverify_get_status(specverify_t h, void* stream, uint32_t* bits) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (bits) *bits = v;
+  if (v & specverify::kStatRowIndex) return SV_ERR_ROW_INDEX;
   if (v & specverify::kStatTokenRange) return SV_ERR_TOKEN_RANGE;
   if (v & specverify::kStatNonFinite) return SV_ERR_NONFINITE;
   if (v & specverify::kStatZeroMass) return SV_WARN_ZERO_MASS;
@@ -553,6 +586,7 @@ const char* specverify_status_string(sv_status s) {
     case SV_ERR_TOKEN_RANGE: return "draft token outside [0, vocab)";
     case SV_ERR_NONFINITE: return "logit row with NaN/+inf or no finite entry";
     case SV_WARN_ZERO_MASS: return "zero residual mass; drew from the target distribution";
+    case SV_ERR_ROW_INDEX: return "row map entry outside the logit rows given";
   }
   return "unknown status";
 }

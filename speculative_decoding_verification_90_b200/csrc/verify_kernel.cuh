@@ -58,7 +58,7 @@ constexpr int kMaxSlices = 64;
 // per-position decision flags
 enum : int { kFlagReject = 0, kFlagAccept = 1, kFlagTokenRange = 2, kFlagNonFinite = 3 };
 // status word bits
-enum : unsigned { kStatTokenRange = 1u, kStatNonFinite = 2u, kStatZeroMass = 4u };
+enum : unsigned { kStatTokenRange = 1u, kStatNonFinite = 2u, kStatZeroMass = 4u, kStatRowIndex = 8u };
 // what the draw kernel draws from
 enum : int { kDrawResidual = 0, kDrawTarget = 1, kDrawNone = 2 };
 
@@ -87,6 +87,7 @@ struct __align__(16) RowPartial {
 // per sequence, from the decide kernel to the draw kernel
 struct SeqDecision {
   double lT, lD;       // log2 sum 2^(x c) of the rows drawn from
+  long trow, drow;     // the rows drawn from, as rows of the logit buffers
   int n;               // accepted drafts
   int mode;            // kDraw*
   unsigned stat_bits;  // data errors found
@@ -95,14 +96,17 @@ struct SeqDecision {
 };
 
 struct Params {
-  const void* target;        // [B, G+1, V]
-  const void* draft;         // [B, G, V]
+  const void* target;        // [target_rows, V] logit rows ([B, G+1, V] when unmapped)
+  const void* draft;         // [draft_rows, V] logit rows ([B, G, V] when unmapped)
+  const int32_t* target_map; // [B, G+1] row of `target` of each position, or null (identity)
+  const int32_t* draft_map;  // [B, G] row of `draft` of each draft position, or null
+  long target_rows, draft_rows;
   const int32_t* tokens;     // [B, G]
   const float* u_accept;     // [B, G]
   const float* u_resample;   // [B]
   int32_t* out_tokens;       // [B, G+1]
   int32_t* out_num_accepted; // [B]
-  RowPartial* partial;       // [(B*(G+1) + B*G) * S]: target rows, then draft rows
+  RowPartial* partial;       // [(target_rows + draft_rows) * S]: target rows, then draft rows
   RowStat* tstat;            // [B*(G+1)]
   RowStat* dstat;            // [B*G]
   PosInfo* pos;              // [B*G]
@@ -466,9 +470,10 @@ __global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Param
   const long unit = blockIdx.x;
   const long r = unit / S;
   const int slice = static_cast<int>(unit - r * S);
-  const long nT = static_cast<long>(P.batch) * (G + 1);
+  const long nT = P.target_rows;
   const T* row = (r < nT) ? static_cast<const T*>(P.target) + r * V
                           : static_cast<const T*>(P.draft) + (r - nT) * V;
+  (void)G;
   const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
   long glo = static_cast<long>(slice) * P.groups_per_slice;
   long ghi = glo + P.groups_per_slice;
@@ -513,15 +518,21 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
     int n = G;          // first rejection, gamma if none
     unsigned bits = 0;  // data errors of the sequence
     double lT_n = 0.0, lD_n = 0.0;
+    long tr_n = 0, dr_n = 0;
     for (int base = 0; base <= G; base += kWarp) {
       const int j = base + lane;
       int flag = kFlagAccept;
-      bool tok_bad = false, row_bad = false;
+      bool tok_bad = false, row_bad = false, map_bad = false;
       double lT = 0.0, lD = 0.0;
+      long tr = 0, dr = 0;
       if (j <= G) {
         const long position = static_cast<long>(b) * (G + 1) + j;
         const long pj = static_cast<long>(b) * G + j;
         const bool has_draft = j < G;
+        // rows of the logit buffers that hold this position
+        tr = P.target_map ? static_cast<long>(P.target_map[position]) : position;
+        dr = has_draft ? (P.draft_map ? static_cast<long>(P.draft_map[pj]) : pj) : 0;
+        map_bad = tr < 0 || tr >= P.target_rows || (has_draft && (dr < 0 || dr >= P.draft_rows));
         // the acceptance test's inputs first: their loads overlap the combine
         int t = 0;
         float u = 0.f, xt = 0.f, xd = 0.f;
@@ -529,25 +540,24 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
           t = P.tokens[pj];
           u = P.u_accept[pj];
           tok_bad = (t < 0 || t >= V);
-          if (!tok_bad) {
-            xt = Elem<T>::load1(static_cast<const T*>(P.target) + position * V, t);
-            xd = Elem<T>::load1(static_cast<const T*>(P.draft) + pj * V, t);
+          if (!tok_bad && !map_bad) {
+            xt = Elem<T>::load1(static_cast<const T*>(P.target) + tr * V, t);
+            xd = Elem<T>::load1(static_cast<const T*>(P.draft) + dr * V, t);
           }
         }
-        const long nT = static_cast<long>(P.batch) * (G + 1);
         int validT = 0, validD = 1;
-        lT = row_lse2(P.partial + position * S, S, validT);
-        P.tstat[position] = RowStat{lT, validT, 0};
-        if (has_draft) {
-          lD = row_lse2(P.partial + (nT + pj) * S, S, validD);
-          P.dstat[pj] = RowStat{lD, validD, 0};
+        if (!map_bad) {
+          lT = row_lse2(P.partial + tr * S, S, validT);
+          if (has_draft) lD = row_lse2(P.partial + (P.target_rows + dr) * S, S, validD);
         }
-        row_bad = !validT || !validD;
+        P.tstat[position] = RowStat{lT, validT, 0};
+        if (has_draft) P.dstat[pj] = RowStat{lD, validD, 0};
+        row_bad = !map_bad && (!validT || !validD);
         if (has_draft) {
           PosInfo info{0.0, 0.0, 0.0, kFlagReject, 0};
           if (tok_bad) {
             info.flag = kFlagTokenRange;
-          } else if (row_bad) {
+          } else if (row_bad || map_bad) {
             info.flag = kFlagNonFinite;
           } else {
             const double lq = static_cast<double>(xt) * c - lT;  // log2 q(t)
@@ -566,6 +576,7 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
       const unsigned rej = __ballot_sync(0xffffffffu, j < G && flag == kFlagReject);
       if (__ballot_sync(0xffffffffu, tok_bad)) bits |= kStatTokenRange;
       if (__ballot_sync(0xffffffffu, row_bad)) bits |= kStatNonFinite;
+      if (__ballot_sync(0xffffffffu, map_bad)) bits |= kStatRowIndex;
       // the statistics the draw needs live in lane (n - base) of this chunk
       const int first = rej ? base + __ffs(rej) - 1 : G;
       const bool here = (n == G) && (first < G || G < base + kWarp);
@@ -573,9 +584,13 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
       const int src = (n - base) & (kWarp - 1);
       const double lTs = __shfl_sync(0xffffffffu, lT, src);
       const double lDs = __shfl_sync(0xffffffffu, lD, src);
+      const long trs = __shfl_sync(0xffffffffu, tr, src);
+      const long drs = __shfl_sync(0xffffffffu, dr, src);
       if (here) {
         lT_n = lTs;
         lD_n = lDs;
+        tr_n = trs;
+        dr_n = drs;
       }
     }
     const long bo = static_cast<long>(b) * (G + 1);
@@ -584,7 +599,7 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
       if (lane == 0) {
         P.out_num_accepted[b] = 0;
         P.resid_mass[b] = NAN;
-        P.decision[b] = SeqDecision{0.0, 0.0, 0, kDrawNone, bits, 0.f, 0.f, 0.f, 1.f};
+        P.decision[b] = SeqDecision{0.0, 0.0, 0, 0, 0, kDrawNone, bits, 0.f, 0.f, 0.f, 1.f};
         atomicOr(P.status, bits);
       }
     } else {
@@ -595,7 +610,7 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
       }
       if (lane == 0) {
         P.out_num_accepted[b] = n;
-        SeqDecision d{lT_n, lD_n, n, (n < G) ? kDrawResidual : kDrawTarget, 0u,
+        SeqDecision d{lT_n, lD_n, tr_n, dr_n, n, (n < G) ? kDrawResidual : kDrawTarget, 0u,
                       0.f, 0.f, 0.f, 1.f};
         float lt_lo;
         split2(lT_n, d.lt_hi, lt_lo);
@@ -741,10 +756,8 @@ __global__ void __launch_bounds__(kDrawThreads, 8) draw_kernel(const Params P) {
 
   // ---- step 4: residual (n < gamma) or bonus (n == gamma) draw ----
   int mode = d.mode;
-  const T* drawT = static_cast<const T*>(P.target) + (bo + n) * V;
-  const T* drawD = (mode == kDrawResidual)
-                       ? static_cast<const T*>(P.draft) + (static_cast<long>(b) * G + n) * V
-                       : nullptr;
+  const T* drawT = static_cast<const T*>(P.target) + d.trow * V;
+  const T* drawD = (mode == kDrawResidual) ? static_cast<const T*>(P.draft) + d.drow * V : nullptr;
   DrawConsts k;
   k.c_hi = P.c_hi;
   k.c_lo = P.c_lo;

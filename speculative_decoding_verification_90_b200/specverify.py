@@ -29,6 +29,7 @@ SV_ERR_UNSUPPORTED = 4
 SV_ERR_TOKEN_RANGE = 16
 SV_ERR_NONFINITE = 17
 SV_WARN_ZERO_MASS = 18
+SV_ERR_ROW_INDEX = 19
 
 # every function declared in include/specverify.h, with its ctypes signature
 _vp, _i, _f, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_uint32)
@@ -36,6 +37,8 @@ SIGNATURES = {
     "specverify_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
     "specverify_run": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
     "specverify_run_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
+    "specverify_run_mapped": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _vp,
+                                   _vp]),
     "specverify_destroy": (None, [_vp]),
     "specverify_get_status": (_i, [_vp, _vp, _u32p]),
     "specverify_debug_readback": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -103,6 +106,16 @@ def specverify_run_host(h, target, draft, tokens, u_accept, u_resample, temperat
                                            float(temperature), out_tokens, out_num_accepted,
                                            stream),
                   "specverify_run_host")
+
+
+def specverify_run_mapped(h, target_rows, n_target_rows, target_map, draft_rows, n_draft_rows,
+                          draft_map, tokens, u_accept, u_resample, temperature, out_tokens,
+                          out_num_accepted, stream=0) -> int:
+    return _check(_lib.specverify_run_mapped(h, target_rows, n_target_rows, target_map, draft_rows,
+                                             n_draft_rows, draft_map, tokens, u_accept, u_resample,
+                                             float(temperature), out_tokens, out_num_accepted,
+                                             stream),
+                  "specverify_run_mapped")
 
 
 def specverify_destroy(h) -> None:
@@ -236,6 +249,45 @@ class SpecVerify:
             stream = torch.cuda.current_stream(self.device)
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
         specverify_run(self.handle, *ptrs, temperature, *outs, sp)
+
+    def run_mapped(self, target_rows, target_map, draft_rows, draft_map, tokens, u_accept,
+                   u_resample, temperature, out_tokens, out_num_accepted, stream=None):
+        """Shared-row step: ``target_rows[target_map[b, j]]`` is position (b, j)'s target row."""
+        import torch
+        B, G, V = self.batch, self.gamma, self.vocab
+        ld = self._logit_dtype()
+
+        def rows(name, t, cap):
+            if t.dim() != 2 or t.shape[1] != V or not 1 <= t.shape[0] <= cap:
+                raise ValueError(f"{name}: shape {tuple(t.shape)} is not [1..{cap}, {V}]")
+            if t.dtype != ld or not t.is_contiguous() or t.device.type != "cuda" \
+                    or t.device.index != self.device:
+                raise ValueError(f"{name}: must be a contiguous {ld} tensor on cuda:{self.device}")
+            return t.data_ptr(), t.shape[0]
+
+        def index(name, t, shape):
+            if tuple(t.shape) != shape or t.dtype != torch.int32 or not t.is_contiguous() \
+                    or t.device.type != "cuda" or t.device.index != self.device:
+                raise ValueError(f"{name}: must be a contiguous int32 {shape} tensor on "
+                                 f"cuda:{self.device}")
+            return t.data_ptr() if t.numel() else 0
+
+        tp, nt = rows("target_rows", target_rows, B * (G + 1))
+        tm = index("target_map", target_map, (B, G + 1))
+        if G > 0:
+            dp, nd = rows("draft_rows", draft_rows, B * G)
+            dm = index("draft_map", draft_map, (B, G))
+        else:
+            dp, nd, dm = 0, 0, 0
+        ptrs = [self._check_tensor("tokens", tokens, torch.int32, True),
+                self._check_tensor("u_accept", u_accept, torch.float32, True),
+                self._check_tensor("u_resample", u_resample, torch.float32, True)]
+        outs = [self._check_tensor("out_tokens", out_tokens, torch.int32, True),
+                self._check_tensor("out_num_accepted", out_num_accepted, torch.int32, True)]
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        specverify_run_mapped(self.handle, tp, nt, tm, dp, nd, dm, *ptrs, temperature, *outs, sp)
 
     def run_host(self, target, draft, tokens, u_accept, u_resample, temperature, out_tokens,
                  out_num_accepted, stream=None):

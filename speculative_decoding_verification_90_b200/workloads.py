@@ -32,7 +32,8 @@ on; no public dataset stands behind any of them):
                    target rows, draft rows and draft tokens at positions
                    j < bp are shared by the sequence's branches; positions
                    j >= bp are fresh N(0, 3^2) draws per branch.  Draft =
-                   0.8 target + 0.2 N(0, 3^2).
+                   0.8 target + 0.2 N(0, 3^2).  Also given as distinct rows
+                   plus row maps, for the shared-row entry point.
 """
 from __future__ import annotations
 
@@ -42,6 +43,7 @@ import numpy as np
 
 F32 = "f32"
 BF16 = "bf16"
+MAPPED_KEYS = ("target_rows", "target_map", "draft_rows", "draft_map")
 
 
 @dataclass
@@ -69,9 +71,25 @@ class Workload:
         return self.batch * (2 * self.gamma + 1) * self.vocab * self.elem_size
 
     def slice(self, lo: int, hi: int) -> "Workload":
+        # the distinct-row tables index the whole batch: a slice keeps only the
+        # per-position arrays
+        meta = {k: v for k, v in self.meta.items() if k not in MAPPED_KEYS}
         return Workload(self.name, hi - lo, self.gamma, self.vocab, self.dtype, self.temperature,
                         self.target[lo:hi], self.draft[lo:hi], self.tokens[lo:hi],
-                        self.u_accept[lo:hi], self.u_resample[lo:hi], dict(self.meta))
+                        self.u_accept[lo:hi], self.u_resample[lo:hi], meta)
+
+    @property
+    def mapped(self) -> bool:
+        """True if ``meta`` holds distinct rows and row maps (shared-row layout)."""
+        return all(k in self.meta for k in MAPPED_KEYS)
+
+    @property
+    def unique_logit_bytes(self) -> int:
+        """Bytes of the distinct logit rows (the shared-row step reads each once)."""
+        if not self.mapped:
+            return self.logit_bytes
+        rows = self.meta["target_rows"].shape[0] + self.meta["draft_rows"].shape[0]
+        return rows * self.vocab * self.elem_size
 
 
 def bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -187,46 +205,105 @@ def b64_g8_v128256(seed: int = 0, batch: int = 64) -> Workload:
 
 def multibranch(seed: int = 0, sequences: int = 32, branches: int = 8, gamma: int = 5,
                 vocab: int = 152064) -> Workload:
-    """sequences x branches rows sharing target/draft rows and tokens before a branch point."""
+    """sequences x branches rows sharing target/draft rows and tokens before a branch point.
+
+    Besides the per-position arrays, ``meta`` holds each distinct row once:
+    ``target_rows`` / ``draft_rows`` (bf16 bits) and ``target_map`` [B, G+1] /
+    ``draft_map`` [B, G] (int32), with ``target[b, j] == target_rows[target_map[b, j]]``.
+    """
     rng = np.random.default_rng(seed)
     S, K, G, V = sequences, branches, gamma, vocab
     B = S * K
-    tgt = np.empty((B, G + 1, V), np.float32)
-    drf = np.empty((B, G, V), np.float32)
-    shared = np.zeros((B, G), bool)
     points = rng.integers(1, G + 1, size=S) if G > 0 else np.zeros(S, np.int64)
+    t_parts, d_parts = [], []
+    t_map = np.empty((B, G + 1), np.int32)
+    d_map = np.empty((B, G), np.int32)
+    shared = np.zeros((B, G), bool)
+    nt = nd = 0
     for s in range(S):
         bp = int(points[s])
         base_t = _normal(rng, (bp, V), 3.0)
         base_d = np.float32(0.8) * base_t + np.float32(0.2) * _normal(rng, (bp, V), 3.0)
+        t_parts.append(base_t)
+        d_parts.append(base_d)
+        t0, d0 = nt, nd
+        nt += bp
+        nd += bp
         for k in range(K):
             b = s * K + k
-            tgt[b, :bp] = base_t
-            drf[b, :bp] = base_d
-            tgt[b, bp:] = _normal(rng, (G + 1 - bp, V), 3.0)
+            t_map[b, :bp] = t0 + np.arange(bp)
+            d_map[b, :bp] = d0 + np.arange(bp)
+            own_t = _normal(rng, (G + 1 - bp, V), 3.0)
+            t_parts.append(own_t)
+            t_map[b, bp:] = nt + np.arange(G + 1 - bp)
+            nt += G + 1 - bp
             if bp < G:
-                drf[b, bp:] = (np.float32(0.8) * tgt[b, bp:G]
+                d_parts.append(np.float32(0.8) * own_t[:G - bp]
                                + np.float32(0.2) * _normal(rng, (G - bp, V), 3.0))
+                d_map[b, bp:] = nd + np.arange(G - bp)
+                nd += G - bp
             shared[b, :bp] = True
+    t_rows = bf16_bits(np.concatenate(t_parts))
+    del t_parts
+    d_rows = bf16_bits(np.concatenate(d_parts)) if d_parts else np.zeros((0, V), np.uint16)
+    del d_parts
     # tokens: one draw per (sequence, shared position), one per (row, private position)
-    drf_bits = bf16_bits(drf)
-    seen = bits_to_f32(drf_bits)
+    seen = bits_to_f32(d_rows)
     tokens = np.empty((B, G), np.int32)
     for s in range(S):
         bp = int(points[s])
         rows = slice(s * K, (s + 1) * K)
         if bp > 0:
-            tokens[rows, :bp] = gumbel_max_tokens(rng, seen[s * K, :bp][None], 1.0)[0][None]
+            tokens[rows, :bp] = gumbel_max_tokens(rng, seen[d_map[s * K, :bp]][None], 1.0)[0][None]
         if bp < G:
-            tokens[rows, bp:] = gumbel_max_tokens(rng, seen[rows, bp:], 1.0)
-    tgt_bits = bf16_bits(tgt)
-    del tgt
+            tokens[rows, bp:] = gumbel_max_tokens(rng, seen[d_map[rows, bp:]], 1.0)
+    del seen
     u_acc = rng.random((B, G), dtype=np.float32)
     u_res = rng.random(B, dtype=np.float32)
-    return Workload("multibranch_32x8_g5_v152064_bf16", B, G, V, BF16, 1.0, tgt_bits, drf_bits,
-                    tokens, u_acc, u_res,
+    return Workload("multibranch_32x8_g5_v152064_bf16", B, G, V, BF16, 1.0, t_rows[t_map],
+                    d_rows[d_map], tokens, u_acc, u_res,
                     {"sequences": S, "branches": K, "branch_points": points.tolist(),
-                     "shared": shared})
+                     "shared": shared, "target_rows": t_rows, "target_map": t_map,
+                     "draft_rows": d_rows, "draft_map": d_map})
+
+
+def random_maps(seed: int = 0, batch: int = 24, gamma: int = 4, vocab: int = 5000,
+                target_rows: int = 40, draft_rows: int = 30, dtype: str = F32,
+                temperature: float = 1.0) -> Workload:
+    """Distinct rows with arbitrary many-to-one row maps (positions of different
+    sequences, and a target and a bonus position, may share a row).
+
+    Target rows N(0, 3^2); each draft row is 0.8 x a random target row + 0.2
+    N(0, 3^2).  Maps are uniform over the rows, then the first rows are pinned
+    so that every row is used at least once.  Tokens are drawn from the
+    materialised draft rows.
+    """
+    rng = np.random.default_rng(seed)
+    B, G, V = batch, gamma, vocab
+    if not 1 <= target_rows <= B * (G + 1) or (G > 0 and not 1 <= draft_rows <= B * G):
+        raise ValueError("row counts must be within [1, positions]")
+    t_f = _normal(rng, (target_rows, V), 3.0)
+    d_rows_n = draft_rows if G > 0 else 0
+    src = rng.integers(0, target_rows, size=d_rows_n)
+    d_f = np.float32(0.8) * t_f[src] + np.float32(0.2) * _normal(rng, (d_rows_n, V), 3.0)
+    t_map = rng.integers(0, target_rows, size=(B, G + 1)).astype(np.int32)
+    t_map.reshape(-1)[rng.permutation(B * (G + 1))[:target_rows]] = np.arange(target_rows)
+    d_map = rng.integers(0, max(d_rows_n, 1), size=(B, G)).astype(np.int32)
+    if G > 0:
+        d_map.reshape(-1)[rng.permutation(B * G)[:d_rows_n]] = np.arange(d_rows_n)
+    if dtype == BF16:
+        t_st, d_st = bf16_bits(t_f), bf16_bits(d_f)
+        d_seen = bits_to_f32(d_st)
+    else:
+        t_st, d_st, d_seen = t_f, d_f, d_f
+    tokens = (gumbel_max_tokens(rng, d_seen[d_map], temperature) if G > 0
+              else np.zeros((B, 0), np.int32))
+    u_acc = rng.random((B, G), dtype=np.float32)
+    u_res = rng.random(B, dtype=np.float32)
+    return Workload(f"random_maps_b{B}_g{G}_v{V}_{dtype}", B, G, V, dtype, float(temperature),
+                    t_st[t_map], d_st[d_map], tokens.astype(np.int32), u_acc, u_res,
+                    {"target_rows": t_st, "target_map": t_map, "draft_rows": d_st,
+                     "draft_map": d_map})
 
 
 REGISTRY = {

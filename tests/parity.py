@@ -30,7 +30,14 @@ def to_device(wl, device=0):
             return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
         return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
 
-    return {
+    out = {}
+    if getattr(wl, "mapped", False):
+        m = wl.meta
+        out = {"target_rows": logits(m["target_rows"]),
+               "target_map": torch.from_numpy(np.ascontiguousarray(m["target_map"], np.int32)).to(dev),
+               "draft_rows": logits(m["draft_rows"]),
+               "draft_map": torch.from_numpy(np.ascontiguousarray(m["draft_map"], np.int32)).to(dev)}
+    return out | {
         "target": logits(wl.target),
         "draft": logits(wl.draft),
         "tokens": torch.from_numpy(np.ascontiguousarray(wl.tokens, np.int32)).to(dev),
@@ -39,8 +46,12 @@ def to_device(wl, device=0):
     }
 
 
-def gpu_run(wl, slices=None, threads=None, device=0, inputs=None, sv=None, readback=True):
-    """One verification call of the whole workload; returns numpy outputs."""
+def gpu_run(wl, slices=None, threads=None, device=0, inputs=None, sv=None, readback=True,
+            mapped=False):
+    """One verification call of the whole workload; returns numpy outputs.
+
+    ``mapped``: call the shared-row entry point on the workload's distinct rows
+    and row maps instead of the per-position arrays."""
     import torch
     from speculative_decoding_verification_90_b200.specverify import SpecVerify
     own = sv is None
@@ -53,8 +64,13 @@ def gpu_run(wl, slices=None, threads=None, device=0, inputs=None, sv=None, readb
         d = inputs if inputs is not None else to_device(wl, device)
         out_t = torch.full((wl.batch, wl.gamma + 1), -7, dtype=torch.int32, device=f"cuda:{device}")
         out_n = torch.full((wl.batch,), -7, dtype=torch.int32, device=f"cuda:{device}")
-        sv.run(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
-               wl.temperature, out_t, out_n)
+        if mapped:
+            sv.run_mapped(d["target_rows"], d["target_map"], d["draft_rows"], d["draft_map"],
+                          d["tokens"], d["u_accept"], d["u_resample"], wl.temperature, out_t,
+                          out_n)
+        else:
+            sv.run(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
+                   wl.temperature, out_t, out_n)
         torch.cuda.synchronize(device)
         status, bits = sv.status()
         res = {"out_tokens": out_t.cpu().numpy(), "out_num_accepted": out_n.cpu().numpy(),
