@@ -23,6 +23,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
+_SRCS = [_SRC, os.path.join(_HERE, "gate.c")]
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 DTYPE_F32 = 0
@@ -35,10 +36,12 @@ WARN_ZERO_MASS = 18
 
 
 def build(force: bool = False) -> str:
-    """Compile ``oracle.c`` into ``liboracle.so`` (plain gcc, IEEE semantics)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    """Compile ``oracle.c`` and ``gate.c`` into ``liboracle.so`` (plain gcc, IEEE semantics)."""
+    stale = not os.path.exists(_LIB) or any(
+        os.path.getmtime(_LIB) < os.path.getmtime(src) for src in _SRCS)
+    if force or stale:
         cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-Wall", "-Wextra",
-               "-o", _LIB, _SRC, "-lm"]
+               "-o", _LIB, *_SRCS, "-lm"]
         subprocess.run(cmd, check=True)
     return _LIB
 
@@ -69,6 +72,29 @@ class _Result(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in _RESULT_FIELDS]
 
 
+class _GateProblem(ctypes.Structure):
+    _fields_ = [
+        ("branches", ctypes.c_int),
+        ("positions", ctypes.c_int),
+        ("dim", ctypes.c_int),
+        ("dtype", ctypes.c_int),
+        ("hidden", ctypes.c_void_p),
+        ("parent", ctypes.c_void_p),
+        ("tau", ctypes.c_double),
+    ]
+
+
+_GATE_FIELDS = ["rel_diff", "margin", "recompute", "provenance", "source", "packed", "n_packed",
+                "parent_used"]
+
+
+class _GateResult(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in _GATE_FIELDS]
+
+
+GATE_OK = 0
+GATE_ERR_PARENT = 20
+
 _lib = None
 _lib_lock = threading.Lock()
 
@@ -85,6 +111,8 @@ def _load():
                                                ctypes.c_int, ctypes.c_double, ctypes.c_void_p,
                                                ctypes.c_void_p, ctypes.c_void_p]
             lib.oracle_softmax_row.restype = ctypes.c_int
+            lib.oracle_gate.argtypes = [ctypes.POINTER(_GateProblem), ctypes.POINTER(_GateResult)]
+            lib.oracle_gate.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -177,4 +205,40 @@ def verify(target: np.ndarray, draft: np.ndarray, tokens: np.ndarray, u_accept: 
     if any(e < 0 for e in errs):
         raise MemoryError("oracle could not allocate its row buffers")
     out["errors"] = int(sum(errs))
+    return out
+
+
+def gate(hidden: np.ndarray, parent: np.ndarray, tau: float) -> dict:
+    """The multi-branch fold gate (``gate.c``) on hidden states [branches, positions, dim]
+    (float32, or uint16 bf16 bits) with one parent index per branch (-1: none).
+
+    Returns numpy arrays ``rel_diff``, ``margin`` (float64 [branches, positions]),
+    ``recompute``, ``provenance``, ``source`` (int32 [branches, positions]),
+    ``packed`` (int32 [n_packed]), ``parent_used`` (int32 [branches]) and
+    ``status`` (GATE_OK or GATE_ERR_PARENT).
+    """
+    hidden = np.ascontiguousarray(hidden)
+    parent = np.ascontiguousarray(parent, dtype=np.int32)
+    nb, npos, dim = hidden.shape
+    if parent.shape != (nb,):
+        raise ValueError("parent must hold one entry per branch")
+    out = {
+        "rel_diff": np.empty((nb, npos), np.float64),
+        "margin": np.empty((nb, npos), np.float64),
+        "recompute": np.empty((nb, npos), np.int32),
+        "provenance": np.empty((nb, npos), np.int32),
+        "source": np.empty((nb, npos), np.int32),
+        "packed": np.empty(max(1, nb * npos), np.int32),
+        "n_packed": np.zeros(1, np.int32),
+        "parent_used": np.empty(max(1, nb), np.int32),
+    }
+    prob = _GateProblem(nb, npos, dim, _dtype_code(hidden), _ptr(hidden), _ptr(parent), float(tau))
+    res = _GateResult(*[_ptr(out[name]) for name in _GATE_FIELDS])
+    st = _load().oracle_gate(ctypes.byref(prob), ctypes.byref(res))
+    if st < 0:
+        raise MemoryError("oracle could not allocate its buffers")
+    n = int(out.pop("n_packed")[0])
+    out["packed"] = out["packed"][:n]
+    out["parent_used"] = out["parent_used"][:nb]
+    out["status"] = st
     return out

@@ -34,6 +34,10 @@ on; no public dataset stands behind any of them):
                    j >= bp are fresh N(0, 3^2) draws per branch.  Draft =
                    0.8 target + 0.2 N(0, 3^2).  Also given as distinct rows
                    plus row maps, for the shared-row entry point.
+* ``gate_tree``    fold-gate inputs: 128 sequences x 8 candidate branches, one
+                   block of 32 positions, hidden size 4096, bf16; a random
+                   tree per sequence and a perturbation that peaks at each
+                   child's newly revealed position (see the function).
 """
 from __future__ import annotations
 
@@ -304,6 +308,80 @@ def random_maps(seed: int = 0, batch: int = 24, gamma: int = 4, vocab: int = 500
                     t_st[t_map], d_st[d_map], tokens.astype(np.int32), u_acc, u_res,
                     {"target_rows": t_st, "target_map": t_map, "draft_rows": d_st,
                      "draft_map": d_map})
+
+
+@dataclass
+class GateWorkload:
+    """Hidden states of candidate branches at one layer input, and their tree."""
+    name: str
+    branches: int
+    positions: int
+    dim: int
+    dtype: str              # "f32" or "bf16"
+    tau: float
+    hidden: np.ndarray      # [branches, positions, dim] float32 or uint16 (bf16 bits)
+    parent: np.ndarray      # int32 [branches], -1 for a branch without a parent
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def elem_size(self) -> int:
+        return 4 if self.dtype == F32 else 2
+
+    @property
+    def rows(self) -> int:
+        return self.branches * self.positions
+
+    def rows_read(self) -> int:
+        """Rows the gate must read at least once: every row of a branch that has a
+        parent (as the child) or that is some branch's parent."""
+        nb = self.branches
+        p = self.parent
+        has_parent = (p >= 0) & (p < nb)
+        is_parent = np.zeros(nb, bool)
+        is_parent[p[has_parent]] = True
+        return int((has_parent | is_parent).sum()) * self.positions
+
+
+def gate_tree(seed: int = 0, sequences: int = 128, branches: int = 8, positions: int = 32,
+              dim: int = 4096, dtype: str = BF16, tau: float = 0.05, amplitude: float = 0.5,
+              width: float = 2.0, floor: float = 0.01) -> GateWorkload:
+    """Per sequence a tree of ``branches`` candidates over one block of ``positions``.
+
+    Branch 0 of a sequence has no parent and holds N(0, 1) hidden states; branch
+    k >= 1 takes a parent uniformly among branches 0..k-1 of its sequence and a
+    revealed position r ~ U{0..positions-1}, and its hidden state at position j
+    is the parent's plus N(0, 1) noise scaled by
+    amplitude * exp(-|j - r| / width) + floor, so the difference is largest at
+    the newly revealed position and ripples out to its neighbours.  States are
+    stored in ``dtype`` (bf16: round to nearest even); a child is built from its
+    parent's stored values.
+    """
+    rng = np.random.default_rng(seed)
+    nb = sequences * branches
+    parent = np.empty(nb, np.int32)
+    revealed = np.full(nb, -1, np.int64)
+    store = bf16_bits if dtype == BF16 else (lambda a: np.ascontiguousarray(a, np.float32))
+    seen = bits_to_f32 if dtype == BF16 else (lambda a: a)
+    hidden = np.empty((nb, positions, dim), np.uint16 if dtype == BF16 else np.float32)
+    j = np.arange(positions, dtype=np.float32)[:, None]
+    for s in range(sequences):
+        b0 = s * branches
+        parent[b0] = -1
+        hidden[b0] = store(rng.standard_normal((positions, dim), dtype=np.float32))
+        for k in range(1, branches):
+            c = b0 + k
+            p = b0 + int(rng.integers(0, k))
+            r = int(rng.integers(0, positions))
+            parent[c] = p
+            revealed[c] = r
+            scale = (np.float32(amplitude) * np.exp(-np.abs(j - np.float32(r)) / np.float32(width))
+                     + np.float32(floor)).astype(np.float32)
+            noise = rng.standard_normal((positions, dim), dtype=np.float32)
+            hidden[c] = store(seen(hidden[p]) + scale * noise)
+    name = f"gate_{sequences}x{branches}_p{positions}_d{dim}_{dtype}"
+    return GateWorkload(name, nb, positions, dim, dtype, float(tau), hidden, parent,
+                        {"sequences": sequences, "branches_per_sequence": branches,
+                         "revealed": revealed})
 
 
 REGISTRY = {
