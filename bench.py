@@ -16,7 +16,10 @@ logits read once = B (2 gamma + 1) V * sizeof(logit).
 
 For the multi-branch batch the same positions are also timed through the
 shared-row entry point (each distinct target/draft row once, plus row maps),
-reported under "shared_rows".
+reported under "shared_rows".  The fold gate (relative hidden-state difference
+per branch and position, provenance, packing of the rows to recompute) is
+timed on 128 sequences x 8 branches x 32 positions x 4096 bf16 hidden states,
+reported under "specfold_gate".
 
 N > 1 runs under torch.distributed.run, one rank per GPU: every rank verifies
 its own batch (weak scaling, no data-path collective).  ``--impl reference``
@@ -67,6 +70,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-shared-rows", action="store_true",
                     help="skip the timing of the shared-row entry point (multibranch)")
+    ap.add_argument("--no-gate", action="store_true",
+                    help="skip the timing of the fold gate (128 x 8 branches, 32 x 4096 bf16)")
     return ap.parse_args()
 
 
@@ -364,6 +369,7 @@ def run_ours(args):
     if wl.mapped and not args.no_shared_rows:
         shared = time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local)
     sv.close()
+    gate = None if args.no_gate else time_gate(args, dev, world, local)
     # tokens settled per step on this rank = accepted + 1 per sequence (last device step)
     emitted = int((out_n.cpu().numpy().astype(np.int64) + 1).sum())
 
@@ -408,6 +414,8 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "status_after": st,
         }
+        if gate is not None:
+            line["specfold_gate"] = gate_summary(gate, peak)
         if shared is not None:
             sh_bytes = shared["bytes"]
             sh_ach = sh_bytes / (shared["stats_ms"] / 1e3) / 1e9
@@ -467,6 +475,74 @@ def time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local):
     del sets, base
     return {"ms_max": ms_max, "stats_ms": kern["stats_ms"], "draw_ms": kern["draw_ms"],
             "bytes": nbytes, "sets": n_sets, "status": st}
+
+
+def time_gate(args, dev, world, local):
+    """Time the fold gate on its benchmark tree (every rank its own copy)."""
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_verification_90_b200.specverify import FoldGate
+    w = workloads.gate_tree(seed=svdist.rank_seed(args.seed, svdist.env_rank()[0]))
+    H = torch.from_numpy(w.hidden.view(np.int16)).view(torch.bfloat16).to(dev)
+    par = torch.from_numpy(w.parent).to(dev)
+    rows = w.rows
+    packed = torch.empty(rows, dtype=torch.int32, device=dev)
+    n = torch.empty(1, dtype=torch.int32, device=dev)
+    rel = torch.empty((w.branches, w.positions), dtype=torch.float32, device=dev)
+    prov = torch.empty((w.branches, w.positions), dtype=torch.int32, device=dev)
+    src = torch.empty((w.branches, w.positions), dtype=torch.int32, device=dev)
+    ph = torch.empty((rows, w.dim), dtype=torch.bfloat16, device=dev)
+    gate = FoldGate(w.branches, w.positions, w.dim, w.dtype, local)
+
+    def step():
+        gate.run(H, par, w.tau, packed, n, rel_diff=rel, provenance=prov, source=src,
+                 packed_hidden=ph)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(10, min(args.steps, 200))
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gate.profile_begin(steps)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    kern = gate.profile_end()
+    ms_max = svdist.max_over_ranks(ev0.elapsed_time(ev1), device=dev)
+    st, _ = gate.status()
+    gate.close()
+    k = int(n.item())
+    return {"workload": w.name, "steps": steps, "ms_max": ms_max, "rows_ms": kern["rows_ms"],
+            "pack_ms": kern["pack_ms"], "rows": rows, "packed": k,
+            "read_bytes": w.rows_read() * w.dim * w.elem_size,
+            "packed_bytes": k * w.dim * w.elem_size, "hidden_bytes": w.hidden.nbytes,
+            "status": st, "world": world}
+
+
+def gate_summary(g, peak):
+    rows_gbs = g["read_bytes"] / (g["rows_ms"] / 1e3) / 1e9
+    # the packing kernel writes the packed batch (its algorithmic bytes); it
+    # re-reads those rows, which is not counted
+    pack_gbs = g["packed_bytes"] / (g["pack_ms"] / 1e3) / 1e9 if g["pack_ms"] > 0 else None
+    ms = g["ms_max"] / g["steps"]
+    return {
+        "workload": g["workload"], "entry": "specfold_gate_run",
+        "rows_per_s": g["rows"] * g["world"] / (ms / 1e3), "ms_per_pass": ms,
+        "rows": g["rows"], "packed_rows": g["packed"],
+        "difference_kernel": {"us": 1e3 * g["rows_ms"], "algorithmic_bytes": g["read_bytes"],
+                              "achieved_gbs": rows_gbs, "peak_gbs": peak,
+                              "frac": rows_gbs / peak},
+        "pack_kernel": {"us": 1e3 * g["pack_ms"], "algorithmic_bytes": g["packed_bytes"],
+                        "achieved_gbs": pack_gbs},
+        "l2": "inputs larger than L2 (%.0f MB of hidden states per pass)" % (g["hidden_bytes"] / 1e6),
+        "status_after": g["status"],
+    }
 
 
 def main():

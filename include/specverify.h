@@ -76,7 +76,8 @@ typedef enum {
   SV_ERR_TOKEN_RANGE = 16, /* device: some draft token was outside [0, V) */
   SV_ERR_NONFINITE = 17,   /* device: some logit row held NaN/+inf or only -inf */
   SV_WARN_ZERO_MASS = 18,  /* device: a residual had zero mass; drew from q_n instead */
-  SV_ERR_ROW_INDEX = 19    /* device: a row map entry was outside the rows given */
+  SV_ERR_ROW_INDEX = 19,   /* device: a row map entry was outside the rows given */
+  SV_ERR_PARENT = 20       /* device (fold gate): a parent entry out of range, a self link or a cycle */
 } sv_status;
 
 /*

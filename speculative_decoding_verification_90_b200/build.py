@@ -35,8 +35,9 @@ def sources() -> list[str]:
 
 
 def deps() -> list[str]:
-    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [
-        os.path.join(INCLUDE, "specverify.h"), __file__]
+    return (sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh")))
+            + sorted(glob.glob(os.path.join(CSRC, "*.h")))
+            + sorted(glob.glob(os.path.join(INCLUDE, "*.h"))) + [__file__])
 
 
 def up_to_date() -> bool:

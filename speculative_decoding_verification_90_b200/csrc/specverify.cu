@@ -14,6 +14,7 @@
 #include <new>
 #include <vector>
 
+#include "host_common.h"
 #include "verify_kernel.cuh"
 
 using specverify::RowPartial;
@@ -48,7 +49,7 @@ struct specverify_ctx {
   int prof_runs = 0;
 };
 
-namespace {
+namespace svhost {
 
 thread_local char g_last_error[256] = "";
 
@@ -58,28 +59,17 @@ sv_status cuda_fail(cudaError_t e) {
   return (e == cudaErrorMemoryAllocation) ? SV_ERR_OOM : SV_ERR_CUDA;
 }
 
-// makes the handle's device current for the scope, restores the caller's
-class DeviceScope {
- public:
-  explicit DeviceScope(int dev) {
-    ok_ = cudaGetDevice(&prev_) == cudaSuccess;
-    if (ok_ && prev_ != dev) ok_ = cudaSetDevice(dev) == cudaSuccess;
-    switched_ = ok_ && prev_ != dev;
-  }
-  ~DeviceScope() {
-    if (switched_) cudaSetDevice(prev_);
-  }
-  bool ok() const { return ok_; }
+}  // namespace svhost
 
- private:
-  int prev_ = 0;
-  bool ok_ = false;
-  bool switched_ = false;
-};
+namespace {
+
+using svhost::cuda_fail;
+using svhost::DeviceScope;
+using svhost::g_last_error;
+using svhost::round_up;
 
 size_t elem_size(sv_dtype d) { return d == SV_DTYPE_BF16 ? 2 : 4; }
 int group_elems(sv_dtype d) { return d == SV_DTYPE_BF16 ? 8 : 4; }
-size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 long num_groups(const specverify_ctx* h) {
   const int ve = group_elems(h->dtype);
@@ -587,6 +577,7 @@ const char* specverify_status_string(sv_status s) {
     case SV_ERR_NONFINITE: return "logit row with NaN/+inf or no finite entry";
     case SV_WARN_ZERO_MASS: return "zero residual mass; drew from the target distribution";
     case SV_ERR_ROW_INDEX: return "row map entry outside the logit rows given";
+    case SV_ERR_PARENT: return "parent index out of range, self link or cycle";
   }
   return "unknown status";
 }

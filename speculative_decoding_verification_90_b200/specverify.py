@@ -30,8 +30,9 @@ SV_ERR_TOKEN_RANGE = 16
 SV_ERR_NONFINITE = 17
 SV_WARN_ZERO_MASS = 18
 SV_ERR_ROW_INDEX = 19
+SV_ERR_PARENT = 20
 
-# every function declared in include/specverify.h, with its ctypes signature
+# every function declared in include/*.h, with its ctypes signature
 _vp, _i, _f, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_uint32)
 SIGNATURES = {
     "specverify_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
@@ -48,6 +49,13 @@ SIGNATURES = {
     "specverify_profile_begin": (_i, [_vp, _i]),
     "specverify_profile_end": (_i, [_vp, ctypes.POINTER(_f), ctypes.POINTER(_f), ctypes.POINTER(_i)]),
     "specverify_run_noalloc": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
+    "specfold_gate_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
+    "specfold_gate_run": (_i, [_vp, _vp, _vp, _f, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "specfold_gate_get_status": (_i, [_vp, _vp, _u32p]),
+    "specfold_gate_profile_begin": (_i, [_vp, _i]),
+    "specfold_gate_profile_end": (_i, [_vp, ctypes.POINTER(_f), ctypes.POINTER(_f),
+                                       ctypes.POINTER(_i)]),
+    "specfold_gate_destroy": (None, [_vp]),
     "specverify_status_string": (ctypes.c_char_p, [_i]),
     "specverify_last_error": (ctypes.c_char_p, []),
 }
@@ -166,6 +174,45 @@ def specverify_run_noalloc(batch, gamma, vocab, dtype, target, draft, tokens, u_
                                               u_accept, u_resample, float(temperature), out_tokens,
                                               out_num_accepted, stream),
                   "specverify_run_noalloc")
+
+
+def specfold_gate_create(branches: int, positions: int, dim: int, dtype: int,
+                         device: int = 0) -> int:
+    h = ctypes.c_void_p()
+    _check(_lib.specfold_gate_create(ctypes.byref(h), branches, positions, dim, dtype, device),
+           "specfold_gate_create")
+    return h.value
+
+
+def specfold_gate_run(h, hidden, parent, tau, rel_diff, provenance, source, packed_rows,
+                      n_packed, packed_hidden, stream=0) -> int:
+    return _check(_lib.specfold_gate_run(h, hidden, parent, float(tau), rel_diff, provenance,
+                                         source, packed_rows, n_packed, packed_hidden, stream),
+                  "specfold_gate_run")
+
+
+def specfold_gate_get_status(h, stream=0) -> tuple[int, int]:
+    bits = ctypes.c_uint32()
+    st = _lib.specfold_gate_get_status(h, stream, ctypes.byref(bits))
+    if st in (SV_ERR_INVALID_ARG, SV_ERR_CUDA, SV_ERR_OOM, SV_ERR_UNSUPPORTED):
+        _check(st, "specfold_gate_get_status")
+    return st, bits.value
+
+
+def specfold_gate_profile_begin(h, max_runs: int) -> int:
+    return _check(_lib.specfold_gate_profile_begin(h, max_runs), "specfold_gate_profile_begin")
+
+
+def specfold_gate_profile_end(h) -> dict:
+    """Mean device milliseconds per run of the difference and packing kernels."""
+    a, c, n = ctypes.c_float(), ctypes.c_float(), ctypes.c_int()
+    _check(_lib.specfold_gate_profile_end(h, ctypes.byref(a), ctypes.byref(c), ctypes.byref(n)),
+           "specfold_gate_profile_end")
+    return {"rows_ms": a.value, "pack_ms": c.value, "runs": n.value}
+
+
+def specfold_gate_destroy(h) -> None:
+    _lib.specfold_gate_destroy(h)
 
 
 def specverify_status_string(status: int) -> str:
@@ -349,3 +396,78 @@ class SpecVerify:
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
         specverify_debug_readback(self.handle, *[a.ctypes.data for a in out.values()], stream=sp)
         return out
+
+
+class FoldGate:
+    """A fold-gate handle for fixed (branches, positions, dim, dtype) on one CUDA device.
+
+    ``run`` takes torch CUDA tensors and enqueues on the current torch stream
+    (or ``stream``).
+    """
+
+    def __init__(self, branches: int, positions: int, dim: int, dtype: str = "bf16",
+                 device: int = 0):
+        self.branches, self.positions, self.dim, self.dtype = branches, positions, dim, dtype
+        self.device = device
+        code = {"f32": SV_DTYPE_F32, "bf16": SV_DTYPE_BF16}[dtype]
+        self.handle = specfold_gate_create(branches, positions, dim, code, device)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            specfold_gate_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def _ptr(self, name, t, shape, dtype, optional=False):
+        if t is None:
+            if optional:
+                return 0
+            raise ValueError(f"{name} is required")
+        if tuple(t.shape) != shape or t.dtype != dtype or not t.is_contiguous() \
+                or t.device.type != "cuda" or t.device.index != self.device:
+            raise ValueError(f"{name}: must be a contiguous {dtype} {shape} tensor on "
+                             f"cuda:{self.device}")
+        return t.data_ptr()
+
+    def run(self, hidden, parent, tau, packed_rows, n_packed, rel_diff=None, provenance=None,
+            source=None, packed_hidden=None, stream=None):
+        import torch
+        nb, npos, dim = self.branches, self.positions, self.dim
+        hd = torch.bfloat16 if self.dtype == "bf16" else torch.float32
+        rows = nb * npos
+        args = [self._ptr("hidden", hidden, (nb, npos, dim), hd),
+                self._ptr("parent", parent, (nb,), torch.int32), float(tau),
+                self._ptr("rel_diff", rel_diff, (nb, npos), torch.float32, True),
+                self._ptr("provenance", provenance, (nb, npos), torch.int32, True),
+                self._ptr("source", source, (nb, npos), torch.int32, True),
+                self._ptr("packed_rows", packed_rows, (rows,), torch.int32),
+                self._ptr("n_packed", n_packed, (1,), torch.int32),
+                self._ptr("packed_hidden", packed_hidden, (rows, dim), hd, True)]
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        specfold_gate_run(self.handle, *args, sp)
+
+    def status(self, stream=None) -> tuple[int, int]:
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        return specfold_gate_get_status(self.handle, sp)
+
+    def profile_begin(self, max_runs: int):
+        specfold_gate_profile_begin(self.handle, max_runs)
+
+    def profile_end(self) -> dict:
+        return specfold_gate_profile_end(self.handle)

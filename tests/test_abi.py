@@ -2,6 +2,7 @@
 function that include/specverify.h declares, and the binding covers them all.
 No compute call is made here."""
 import ctypes
+import glob
 import os
 import re
 import subprocess
@@ -9,13 +10,17 @@ import subprocess
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "specverify.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
+PREFIX = r"(?:specverify|specfold_gate)_\w+"
 
 
 def _declared():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(specverify_\w+)\s*\(", text)))
+    names = set()
+    for header in HEADERS:
+        text = open(header).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names |= set(re.findall(rf"\b({PREFIX})\s*\(", text))
+    return sorted(names)
 
 
 @pytest.fixture(scope="module")
@@ -37,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib_path):
         assert hasattr(lib, name), name
     out = subprocess.run(["nm", "-D", "--defined-only", lib_path], capture_output=True,
                          text=True, check=True).stdout
-    exported = set(re.findall(r"\bT (specverify_\w+)", out))
+    exported = set(re.findall(rf"\bT ({PREFIX})", out))
     assert set(_declared()) == exported
 
 
