@@ -23,7 +23,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "oracle.c")
-_SRCS = [_SRC, os.path.join(_HERE, "gate.c")]
+_SRCS = [_SRC, os.path.join(_HERE, "gate.c"), os.path.join(_HERE, "sampling.c")]
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 DTYPE_F32 = 0
@@ -36,7 +36,7 @@ WARN_ZERO_MASS = 18
 
 
 def build(force: bool = False) -> str:
-    """Compile ``oracle.c`` and ``gate.c`` into ``liboracle.so`` (plain gcc, IEEE semantics)."""
+    """Compile the oracle's C files into ``liboracle.so`` (plain gcc, IEEE semantics)."""
     stale = not os.path.exists(_LIB) or any(
         os.path.getmtime(_LIB) < os.path.getmtime(src) for src in _SRCS)
     if force or stale:
@@ -92,6 +92,34 @@ class _GateResult(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in _GATE_FIELDS]
 
 
+class _SampProblem(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int),
+        ("gamma", ctypes.c_int),
+        ("vocab", ctypes.c_int),
+        ("dtype", ctypes.c_int),
+        ("target_logits", ctypes.c_void_p),
+        ("draft_logits", ctypes.c_void_p),
+        ("draft_tokens", ctypes.c_void_p),
+        ("u_accept", ctypes.c_void_p),
+        ("u_resample", ctypes.c_void_p),
+        ("temperature", ctypes.c_void_p),
+        ("top_k", ctypes.c_int),
+        ("top_p", ctypes.c_double),
+    ]
+
+
+_SAMP_FIELDS = ["out_tokens", "out_num_accepted", "seq_status", "q_tok", "p_tok",
+                "accept_margin", "resid_mass", "cdf_margin_norm", "kept_target", "kept_draft",
+                "filter_margin"]
+
+
+class _SampResult(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in _SAMP_FIELDS]
+
+
+ERR_TEMPERATURE = 21
+
 GATE_OK = 0
 GATE_ERR_PARENT = 20
 
@@ -113,6 +141,10 @@ def _load():
             lib.oracle_softmax_row.restype = ctypes.c_int
             lib.oracle_gate.argtypes = [ctypes.POINTER(_GateProblem), ctypes.POINTER(_GateResult)]
             lib.oracle_gate.restype = ctypes.c_int
+            lib.oracle_verify_sampling.argtypes = [ctypes.POINTER(_SampProblem),
+                                                   ctypes.POINTER(_SampResult),
+                                                   ctypes.c_int, ctypes.c_int]
+            lib.oracle_verify_sampling.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -241,4 +273,53 @@ def gate(hidden: np.ndarray, parent: np.ndarray, tau: float) -> dict:
     out["packed"] = out["packed"][:n]
     out["parent_used"] = out["parent_used"][:nb]
     out["status"] = st
+    return out
+
+
+def verify_sampling(target: np.ndarray, draft: np.ndarray, tokens: np.ndarray,
+                    u_accept: np.ndarray, u_resample: np.ndarray, temperature,
+                    top_k: int = 0, top_p: float = 1.0, threads: int = 1,
+                    b_range: tuple[int, int] | None = None) -> dict:
+    """The verification step on adjusted distributions (``sampling.c``): a
+    temperature per sequence (0: greedy), top-k (0: off) and top-p (1: off)
+    applied to every target and draft row.  Shapes as in ``verify``;
+    ``temperature`` is a scalar or float32 [B]."""
+    target = np.ascontiguousarray(target)
+    draft = np.ascontiguousarray(draft)
+    tokens = np.ascontiguousarray(tokens, dtype=np.int32)
+    u_accept = np.ascontiguousarray(u_accept, dtype=np.float32)
+    u_resample = np.ascontiguousarray(u_resample, dtype=np.float32)
+    B, Gp1, V = target.shape
+    G = Gp1 - 1
+    temps = np.ascontiguousarray(np.broadcast_to(np.asarray(temperature, np.float32), (B,)))
+    if draft.shape != (B, G, V) or draft.dtype != target.dtype:
+        raise ValueError("draft logits must be [B, gamma, V] with the target's dtype")
+    lo, hi = (0, B) if b_range is None else b_range
+    out = {
+        "out_tokens": np.full((B, G + 1), -1, np.int32),
+        "out_num_accepted": np.zeros(B, np.int32),
+        "seq_status": np.zeros(B, np.int32),
+        "q_tok": np.full((B, G), np.nan),
+        "p_tok": np.full((B, G), np.nan),
+        "accept_margin": np.full((B, G), np.nan),
+        "resid_mass": np.full(B, np.nan),
+        "cdf_margin_norm": np.full(B, np.nan),
+        "kept_target": np.zeros((B, G + 1), np.int32),
+        "kept_draft": np.zeros((B, G), np.int32),
+        "filter_margin": np.full(B, np.inf),
+    }
+    prob = _SampProblem(B, G, V, _dtype_code(target), _ptr(target), _ptr(draft), _ptr(tokens),
+                        _ptr(u_accept), _ptr(u_resample), _ptr(temps), int(top_k), float(top_p))
+    res = _SampResult(*[_ptr(out[name]) for name in _SAMP_FIELDS])
+    lib = _load()
+    threads = max(1, min(int(threads), hi - lo)) if hi > lo else 1
+    bounds = np.linspace(lo, hi, threads + 1).astype(int)
+    with ThreadPoolExecutor(threads) as ex:
+        errs = list(ex.map(
+            lambda k: lib.oracle_verify_sampling(ctypes.byref(prob), ctypes.byref(res),
+                                                 int(bounds[k]), int(bounds[k + 1])),
+            range(threads)))
+    if any(e < 0 for e in errs):
+        raise MemoryError("oracle could not allocate its row buffers")
+    out["errors"] = int(sum(errs))
     return out

@@ -85,8 +85,10 @@ def gpu_run(wl, slices=None, threads=None, device=0, inputs=None, sv=None, readb
 
 def oracle_run(wl, b_range=None):
     import oracle
+    # the C ABI takes the temperature as a float: the oracle gets the same value
     return oracle.verify(wl.target, wl.draft, wl.tokens, wl.u_accept, wl.u_resample,
-                         wl.temperature, threads=os.cpu_count() or 1, b_range=b_range)
+                         float(np.float32(wl.temperature)), threads=os.cpu_count() or 1,
+                         b_range=b_range)
 
 
 def compare(wl, gpu, ora, seqs=None, check_probs=True):
