@@ -77,7 +77,8 @@ typedef enum {
   SV_ERR_NONFINITE = 17,   /* device: some logit row held NaN/+inf or only -inf */
   SV_WARN_ZERO_MASS = 18,  /* device: a residual had zero mass; drew from q_n instead */
   SV_ERR_ROW_INDEX = 19,   /* device: a row map entry was outside the rows given */
-  SV_ERR_PARENT = 20       /* device (fold gate): a parent entry out of range, a self link or a cycle */
+  SV_ERR_PARENT = 20,      /* device (fold gate): a parent entry out of range, a self link or a cycle */
+  SV_ERR_TEMPERATURE = 21  /* device (sampling variants): a temperature < 0, NaN or infinite */
 } sv_status;
 
 /*
@@ -127,6 +128,45 @@ sv_status specverify_run_host(specverify_t h, const void *target_logits,
                               const float *u_accept, const float *u_resample,
                               float temperature, int32_t *out_tokens,
                               int32_t *out_num_accepted, void *stream);
+
+/*
+ * The step under sampling variants.  Argmax, top-k, nucleus and temperature
+ * sampling are standard sampling from an adjusted distribution, so the same
+ * rule verifies them ("Speculative decoding: how to run big models fast",
+ * section "How it works", guarantee paragraph).  Every target row q_j and draft
+ * row p_j of sequence b is replaced by its adjusted distribution:
+ *   temperatures[b] == 0: the point mass on the first index of the row's
+ *     largest logit (greedy; top_k and top_p do not change it);
+ *   temperatures[b] > 0: softmax(x / T) restricted to the entries with
+ *     x >= the k-th largest logit (top_k in [1, vocab); entries tied with it
+ *     are kept), then, within those, to the entries >= the largest logit value
+ *     v whose cumulative mass (all kept entries >= v) reaches top_p of the
+ *     kept mass (top_p in (0, 1); ties at v are kept), and renormalised.
+ * top_k == 0 or >= vocab and top_p >= 1 switch the filters off.  Then the
+ * rule of specverify_run: accept while u_accept < q(t)/p(t) (q(t) == 0 gives
+ * 0, p(t) == 0 < q(t) gives +inf), draw from max(0, q_n - p_n) at the first
+ * rejection or from q_gamma, by the inverse CDF with u_resample.
+ * Arguments as specverify_run, plus
+ *   temperatures  float [batch] device array, one per sequence
+ *   top_k         host value >= 0
+ *   top_p         host value in (0, inf); values >= 1 switch it off
+ * A sequence with a temperature < 0, NaN or infinite emits nothing and sets
+ * status bit 16 (SV_ERR_TEMPERATURE).  Each row is read several times (the
+ * threshold search); the kernels are separate from the plain step's.
+ */
+sv_status specverify_run_sampling(specverify_t h, const void *target_logits,
+                                  const void *draft_logits, const int32_t *draft_tokens,
+                                  const float *u_accept, const float *u_resample,
+                                  const float *temperatures, int top_k, float top_p,
+                                  int32_t *out_tokens, int32_t *out_num_accepted, void *stream);
+
+/*
+ * After specverify_run_sampling: wait for `stream` and copy the number of
+ * entries each row's adjusted distribution keeps ([batch, gamma+1] and
+ * [batch, gamma] int32 host arrays; either may be NULL).  Diagnostic.
+ */
+sv_status specverify_debug_kept(specverify_t h, int32_t *kept_target, int32_t *kept_draft,
+                                void *stream);
 
 /*
  * Multi-branch verification over shared logit rows.  Where many candidate

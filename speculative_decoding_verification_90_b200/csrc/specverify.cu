@@ -15,6 +15,7 @@
 #include <vector>
 
 #include "host_common.h"
+#include "sampling_kernel.cuh"
 #include "verify_kernel.cuh"
 
 using specverify::RowPartial;
@@ -41,6 +42,8 @@ struct specverify_ctx {
   unsigned* draw_ticket = nullptr;
   double* resid = nullptr;
   unsigned* status = nullptr;
+  specsamp::SampRow* samp_rows = nullptr;          // sampling variants: per-row filter
+  specsamp::SampDecision* samp_decision = nullptr; // sampling variants: per sequence
   void* stage = nullptr;  // device staging for host-buffer runs
   size_t stage_bytes = 0;
   // optional per-kernel timing: 3 events per recorded run
@@ -117,8 +120,8 @@ int draw_shape(const specverify_ctx* h) {
   return static_cast<int>(s2);
 }
 
-template <typename K>
-cudaError_t launch_pdl(K kernel, unsigned blocks, unsigned threads, cudaStream_t s, const Params& p) {
+template <typename K, typename PP>
+cudaError_t launch_pdl(K kernel, unsigned blocks, unsigned threads, cudaStream_t s, const PP& p) {
   // programmatic dependent launch: the kernel may be scheduled before its
   // predecessor on the stream has finished; it waits in a grid-dependency
   // barrier before it reads the predecessor's results
@@ -316,6 +319,8 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   const size_t offK = take(nB * sizeof(unsigned));
   const size_t offR = take(nB * sizeof(double));
   const size_t offS = take(sizeof(unsigned));
+  const size_t offSR = take((nT + nD) * sizeof(specsamp::SampRow));
+  const size_t offSD = take(nB * sizeof(specsamp::SampDecision));
   const size_t total = off;
   e = cudaMalloc(&h->ws, total);
   if (e != cudaSuccess) {
@@ -332,6 +337,8 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   h->draw_ticket = reinterpret_cast<unsigned*>(base + offK);
   h->resid = reinterpret_cast<double*>(base + offR);
   h->status = reinterpret_cast<unsigned*>(base + offS);
+  h->samp_rows = reinterpret_cast<specsamp::SampRow*>(base + offSR);
+  h->samp_decision = reinterpret_cast<specsamp::SampDecision*>(base + offSD);
   e = cudaMemset(h->ws, 0, total);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
@@ -353,6 +360,102 @@ sv_status specverify_run(specverify_t h, const void* target_logits, const void* 
   if (!scope.ok()) return SV_ERR_CUDA;
   return enqueue(h, target_logits, draft_logits, draft_tokens, u_accept, u_resample,
                  temperature, out_tokens, out_num_accepted, static_cast<cudaStream_t>(stream));
+}
+
+sv_status specverify_run_sampling(specverify_t h, const void* target_logits,
+                                  const void* draft_logits, const int32_t* draft_tokens,
+                                  const float* u_accept, const float* u_resample,
+                                  const float* temperatures, int top_k, float top_p,
+                                  int32_t* out_tokens, int32_t* out_num_accepted, void* stream) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  if (h->batch == 0) return SV_OK;
+  const int G = h->gamma;
+  const size_t es = elem_size(h->dtype);
+  if (!target_logits || !u_resample || !temperatures || !out_tokens || !out_num_accepted)
+    return SV_ERR_INVALID_ARG;
+  if (G > 0 && (!draft_logits || !draft_tokens || !u_accept)) return SV_ERR_INVALID_ARG;
+  if (!aligned_to(target_logits, es) || (G > 0 && !aligned_to(draft_logits, es)))
+    return SV_ERR_INVALID_ARG;
+  if (!aligned_to(draft_tokens, 4) || !aligned_to(u_accept, 4) || !aligned_to(u_resample, 4) ||
+      !aligned_to(temperatures, 4) || !aligned_to(out_tokens, 4) ||
+      !aligned_to(out_num_accepted, 4))
+    return SV_ERR_INVALID_ARG;
+  if (top_k < 0 || std::isnan(top_p) || !(top_p > 0.f)) return SV_ERR_INVALID_ARG;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  specsamp::SampParams p;
+  p.target = target_logits;
+  p.draft = draft_logits;
+  p.tokens = draft_tokens;
+  p.u_accept = u_accept;
+  p.u_resample = u_resample;
+  p.temperature = temperatures;
+  p.out_tokens = out_tokens;
+  p.out_num_accepted = out_num_accepted;
+  p.rows = h->samp_rows;
+  p.decision = h->samp_decision;
+  p.tstat = h->tstat;
+  p.dstat = h->dstat;
+  p.pos = h->pos;
+  p.resid_mass = h->resid;
+  p.status = h->status;
+  p.batch = h->batch;
+  p.gamma = G;
+  p.vocab = h->vocab;
+  p.top_k = (top_k >= h->vocab) ? 0 : top_k;
+  p.top_p = (top_p >= 1.f) ? 1.0 : static_cast<double>(top_p);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long rows = static_cast<long>(h->batch) * (2L * G + 1);
+  const int per = specsamp::kDecideThreads / specsamp::kWarp;
+  cudaError_t e;
+  if (h->dtype == SV_DTYPE_BF16) {
+    e = cudaFuncSetAttribute(specsamp::select_kernel<__nv_bfloat16>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, specsamp::kCandSmem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    specsamp::select_kernel<__nv_bfloat16>
+        <<<static_cast<unsigned>(rows), specsamp::kSelThreads, specsamp::kCandSmem, s>>>(p);
+    e = cudaGetLastError();
+    if (e == cudaSuccess)
+      e = launch_pdl(specsamp::decide_kernel<__nv_bfloat16>,
+                     static_cast<unsigned>((h->batch + per - 1) / per), specsamp::kDecideThreads, s, p);
+    if (e == cudaSuccess)
+      e = launch_pdl(specsamp::draw_kernel<__nv_bfloat16>, static_cast<unsigned>(h->batch),
+                     specsamp::kDrawThreads, s, p);
+  } else {
+    e = cudaFuncSetAttribute(specsamp::select_kernel<float>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, specsamp::kCandSmem);
+    if (e != cudaSuccess) return cuda_fail(e);
+    specsamp::select_kernel<float>
+        <<<static_cast<unsigned>(rows), specsamp::kSelThreads, specsamp::kCandSmem, s>>>(p);
+    e = cudaGetLastError();
+    if (e == cudaSuccess)
+      e = launch_pdl(specsamp::decide_kernel<float>,
+                     static_cast<unsigned>((h->batch + per - 1) / per), specsamp::kDecideThreads, s, p);
+    if (e == cudaSuccess)
+      e = launch_pdl(specsamp::draw_kernel<float>, static_cast<unsigned>(h->batch),
+                     specsamp::kDrawThreads, s, p);
+  }
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SV_OK;
+}
+
+sv_status specverify_debug_kept(specverify_t h, int32_t* kept_target, int32_t* kept_draft,
+                                void* stream) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  const size_t nT = static_cast<size_t>(h->batch) * (h->gamma + 1);
+  const size_t nD = static_cast<size_t>(h->batch) * h->gamma;
+  std::vector<RowStat> ts(nT), ds(nD);
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess && nT) e = cudaMemcpy(ts.data(), h->tstat, nT * sizeof(RowStat), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && nD) e = cudaMemcpy(ds.data(), h->dstat, nD * sizeof(RowStat), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  for (size_t i = 0; i < nT; ++i)
+    if (kept_target) kept_target[i] = ts[i].pad;
+  for (size_t i = 0; i < nD; ++i)
+    if (kept_draft) kept_draft[i] = ds[i].pad;
+  return SV_OK;
 }
 
 sv_status specverify_run_mapped(specverify_t h, const void* target_rows, int n_target_rows,
@@ -459,6 +562,7 @@ sv_status specverify_get_status(specverify_t h, void* stream, uint32_t* bits) {
   if (e != cudaSuccess) return cuda_fail(e);
   if (bits) *bits = v;
   if (v & specverify::kStatRowIndex) return SV_ERR_ROW_INDEX;
+  if (v & specsamp::kStatTemperature) return SV_ERR_TEMPERATURE;
   if (v & specverify::kStatTokenRange) return SV_ERR_TOKEN_RANGE;
   if (v & specverify::kStatNonFinite) return SV_ERR_NONFINITE;
   if (v & specverify::kStatZeroMass) return SV_WARN_ZERO_MASS;
@@ -578,6 +682,7 @@ const char* specverify_status_string(sv_status s) {
     case SV_WARN_ZERO_MASS: return "zero residual mass; drew from the target distribution";
     case SV_ERR_ROW_INDEX: return "row map entry outside the logit rows given";
     case SV_ERR_PARENT: return "parent index out of range, self link or cycle";
+    case SV_ERR_TEMPERATURE: return "temperature negative, NaN or infinite";
   }
   return "unknown status";
 }

@@ -31,6 +31,7 @@ SV_ERR_NONFINITE = 17
 SV_WARN_ZERO_MASS = 18
 SV_ERR_ROW_INDEX = 19
 SV_ERR_PARENT = 20
+SV_ERR_TEMPERATURE = 21
 
 # every function declared in include/*.h, with its ctypes signature
 _vp, _i, _f, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_uint32)
@@ -38,6 +39,8 @@ SIGNATURES = {
     "specverify_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
     "specverify_run": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
     "specverify_run_host": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
+    "specverify_run_sampling": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _f, _vp, _vp, _vp]),
+    "specverify_debug_kept": (_i, [_vp, _vp, _vp, _vp]),
     "specverify_run_mapped": (_i, [_vp, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp, _vp, _f, _vp, _vp,
                                    _vp]),
     "specverify_destroy": (None, [_vp]),
@@ -124,6 +127,19 @@ def specverify_run_mapped(h, target_rows, n_target_rows, target_map, draft_rows,
                                              float(temperature), out_tokens, out_num_accepted,
                                              stream),
                   "specverify_run_mapped")
+
+
+def specverify_run_sampling(h, target, draft, tokens, u_accept, u_resample, temperatures, top_k,
+                            top_p, out_tokens, out_num_accepted, stream=0) -> int:
+    return _check(_lib.specverify_run_sampling(h, target, draft, tokens, u_accept, u_resample,
+                                               temperatures, int(top_k), float(top_p), out_tokens,
+                                               out_num_accepted, stream),
+                  "specverify_run_sampling")
+
+
+def specverify_debug_kept(h, kept_target, kept_draft, stream=0) -> int:
+    return _check(_lib.specverify_debug_kept(h, kept_target, kept_draft, stream),
+                  "specverify_debug_kept")
 
 
 def specverify_destroy(h) -> None:
@@ -259,7 +275,8 @@ class SpecVerify:
     def _shapes(self):
         B, G, V = self.batch, self.gamma, self.vocab
         return {"target": (B, G + 1, V), "draft": (B, G, V), "tokens": (B, G),
-                "u_accept": (B, G), "u_resample": (B,), "out_tokens": (B, G + 1),
+                "u_accept": (B, G), "u_resample": (B,), "temperatures": (B,),
+                "out_tokens": (B, G + 1),
                 "out_num_accepted": (B,)}
 
     def _check_tensor(self, name, t, dtype, cuda):
@@ -335,6 +352,36 @@ class SpecVerify:
             stream = torch.cuda.current_stream(self.device)
         sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
         specverify_run_mapped(self.handle, tp, nt, tm, dp, nd, dm, *ptrs, temperature, *outs, sp)
+
+    def run_sampling(self, target, draft, tokens, u_accept, u_resample, temperatures, out_tokens,
+                     out_num_accepted, top_k=0, top_p=1.0, stream=None):
+        """Sampling variants: ``temperatures`` float32 [B] on the device (0: greedy)."""
+        import torch
+        ld = self._logit_dtype()
+        ptrs = [self._check_tensor("target", target, ld, True),
+                self._check_tensor("draft", draft, ld, True),
+                self._check_tensor("tokens", tokens, torch.int32, True),
+                self._check_tensor("u_accept", u_accept, torch.float32, True),
+                self._check_tensor("u_resample", u_resample, torch.float32, True),
+                self._check_tensor("temperatures", temperatures, torch.float32, True)]
+        outs = [self._check_tensor("out_tokens", out_tokens, torch.int32, True),
+                self._check_tensor("out_num_accepted", out_num_accepted, torch.int32, True)]
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        specverify_run_sampling(self.handle, *ptrs, top_k, top_p, *outs, sp)
+
+    def kept(self, stream=None):
+        """Entries kept by each row's adjusted distribution after run_sampling."""
+        import torch
+        B, G = self.batch, self.gamma
+        kt = np.zeros((B, G + 1), np.int32)
+        kd = np.zeros((B, G), np.int32)
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        sp = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+        specverify_debug_kept(self.handle, kt.ctypes.data, kd.ctypes.data if kd.size else None, sp)
+        return kt, kd
 
     def run_host(self, target, draft, tokens, u_accept, u_resample, temperature, out_tokens,
                  out_num_accepted, stream=None):

@@ -142,3 +142,87 @@ def assert_parity(summary, max_margin_frac=0.01):
     for key in ("max_target_lse_abs", "max_draft_lse_abs"):
         if key in summary:
             assert summary[key] <= LSE_TOL, summary
+
+
+FILTER_MARGIN = 1e-6   # top-p boundary: |cumulative mass - top_p| below this is a margin case
+
+
+def gpu_run_sampling(wl, temperatures, top_k=0, top_p=1.0, device=0, inputs=None, sv=None):
+    """One call of the sampling-variant entry point; numpy outputs plus readbacks."""
+    import torch
+    from speculative_decoding_verification_90_b200.specverify import SpecVerify
+    own = sv is None
+    if own:
+        sv = SpecVerify(wl.batch, wl.gamma, wl.vocab, wl.dtype, device)
+    try:
+        d = inputs if inputs is not None else to_device(wl, device)
+        temps = torch.from_numpy(np.ascontiguousarray(
+            np.broadcast_to(np.asarray(temperatures, np.float32), (wl.batch,)))).to(f"cuda:{device}")
+        out_t = torch.full((wl.batch, wl.gamma + 1), -7, dtype=torch.int32, device=f"cuda:{device}")
+        out_n = torch.full((wl.batch,), -7, dtype=torch.int32, device=f"cuda:{device}")
+        sv.run_sampling(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
+                        temps, out_t, out_n, top_k=top_k, top_p=top_p)
+        torch.cuda.synchronize(device)
+        status, bits = sv.status()
+        res = {"out_tokens": out_t.cpu().numpy(), "out_num_accepted": out_n.cpu().numpy(),
+               "status": status, "bits": bits}
+        res.update(sv.readback())
+        res["kept_target"], res["kept_draft"] = sv.kept()
+        return res
+    finally:
+        if own:
+            sv.close()
+
+
+def oracle_run_sampling(wl, temperatures, top_k=0, top_p=1.0):
+    import oracle
+    return oracle.verify_sampling(wl.target, wl.draft, wl.tokens, wl.u_accept, wl.u_resample,
+                                  np.asarray(temperatures, np.float32), top_k=top_k,
+                                  top_p=float(np.float32(top_p)), threads=os.cpu_count() or 1)
+
+
+def compare_sampling(wl, gpu, ora):
+    """Decision parity of the sampling variants.  A sequence with a row whose
+    top-p boundary margin (|cumulative mass - top_p| at the chosen cut, relative
+    to the kept mass) is below FILTER_MARGIN may cut one group differently: its
+    kept counts and probabilities are not compared, and a differing decision
+    counts as a margin case.  Everything else must agree as in the plain step."""
+    B, G = wl.batch, wl.gamma
+    hard, margin_cases = [], []
+    ok = []
+    for b in range(B):
+        ng, no = int(gpu["out_num_accepted"][b]), int(ora["out_num_accepted"][b])
+        tg, to = gpu["out_tokens"][b], ora["out_tokens"][b]
+        if ora["seq_status"][b] in (16, 17, 21):
+            if ng != 0 or not (tg == -1).all():
+                hard.append((b, "error outcome", ng, tg.tolist()))
+            continue
+        near_cut = ora["filter_margin"][b] < FILTER_MARGIN
+        if not near_cut:
+            if ora["seq_status"][b] == 0:
+                ok.append(b)   # a zero-mass fallback's residual mass is rounding
+            if not (np.array_equal(gpu["kept_target"][b], ora["kept_target"][b])
+                    and np.array_equal(gpu["kept_draft"][b], ora["kept_draft"][b])):
+                hard.append((b, "kept", gpu["kept_target"][b].tolist(),
+                             ora["kept_target"][b].tolist()))
+                continue
+        if ng != no:
+            j = min(ng, no)
+            m = ora["accept_margin"][b, j]
+            (margin_cases if (m < MARGIN or near_cut) else hard).append((b, "accept", j, float(m)))
+            continue
+        if not np.array_equal(tg, to):
+            m = ora["cdf_margin_norm"][b]
+            (margin_cases if (m < MARGIN or near_cut) else hard).append(
+                (b, "draw", int(tg[no]), int(to[no]), float(m)))
+    summary = {"sequences": B, "hard": hard, "margin_cases": margin_cases,
+               "near_cut": int((ora["filter_margin"] < FILTER_MARGIN).sum())}
+    s = np.asarray(ok, dtype=np.int64)
+    if G > 0 and len(s):
+        tested = ~np.isnan(ora["q_tok"][s])
+        summary["max_dq"] = float(np.abs(gpu["q_tok"][s] - ora["q_tok"][s])[tested].max(initial=0.0))
+        summary["max_dp"] = float(np.abs(gpu["p_tok"][s] - ora["p_tok"][s])[tested].max(initial=0.0))
+    if len(s):
+        dz = np.abs(gpu["resid_mass"][s] - ora["resid_mass"][s])
+        summary["max_dz"] = float(np.nanmax(dz)) if dz.size else 0.0
+    return summary
