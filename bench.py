@@ -19,7 +19,8 @@ shared-row entry point (each distinct target/draft row once, plus row maps),
 reported under "shared_rows".  The fold gate (relative hidden-state difference
 per branch and position, provenance, packing of the rows to recompute) is
 timed on 128 sequences x 8 branches x 32 positions x 4096 bf16 hidden states,
-reported under "specfold_gate".
+reported under "specfold_gate".  The sampling-variant entry point (greedy;
+top-k 50 with top-p 0.9) is timed on the same batch under "sampling_variants".
 
 N > 1 runs under torch.distributed.run, one rank per GPU: every rank verifies
 its own batch (weak scaling, no data-path collective).  ``--impl reference``
@@ -49,9 +50,9 @@ METRIC = "verified positions/s and achieved HBM GB/s vs B200 peak (spec-verify, 
 UNIT = "positions/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_HBM_GBS = 6650.0
+# the source of the kernel whose DRAM traffic the committed ncu summary records
 KERNEL_SOURCES = [
     "speculative_decoding_verification_90_b200/csrc/verify_kernel.cuh",
-    "speculative_decoding_verification_90_b200/csrc/specverify.cu",
 ]
 
 
@@ -70,6 +71,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-shared-rows", action="store_true",
                     help="skip the timing of the shared-row entry point (multibranch)")
+    ap.add_argument("--no-sampling", action="store_true",
+                    help="skip the timing of the sampling variants (greedy, top-k + top-p)")
     ap.add_argument("--no-gate", action="store_true",
                     help="skip the timing of the fold gate (128 x 8 branches, 32 x 4096 bf16)")
     return ap.parse_args()
@@ -364,6 +367,11 @@ def run_ours(args):
     d2h = h_ot.numel() * 4 + h_on.numel() * 4
     st, bits = sv.status()
 
+    # the same batch under sampling variants (separate kernels)
+    sampling = None
+    if not args.no_sampling:
+        sampling = time_sampling(args, wl, sv, sets, n_sets, out_t, out_n, dev, world, local)
+
     # the same batch through the shared-row entry point: each distinct row once
     shared = None
     if wl.mapped and not args.no_shared_rows:
@@ -416,6 +424,16 @@ def run_ours(args):
         }
         if gate is not None:
             line["specfold_gate"] = gate_summary(gate, peak)
+        if sampling is not None:
+            line["sampling_variants"] = {
+                name: {"entry": "specverify_run_sampling", "settings": v["settings"],
+                       "value": positions * args.steps / (v["ms_max"] / 1e3), "unit": UNIT,
+                       "ms_per_step": v["ms_max"] / args.steps,
+                       "logit_gbs": step_bytes / (v["ms_max"] / 1e3 / args.steps) / 1e9,
+                       "select_us": v["select_us"],
+                       "decide_and_draw_us": v["decide_and_draw_us"],
+                       "status_after": v["status"]}
+                for name, v in sampling.items()}
         if shared is not None:
             sh_bytes = shared["bytes"]
             sh_ach = sh_bytes / (shared["stats_ms"] / 1e3) / 1e9
@@ -475,6 +493,44 @@ def time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local):
     del sets, base
     return {"ms_max": ms_max, "stats_ms": kern["stats_ms"], "draw_ms": kern["draw_ms"],
             "bytes": nbytes, "sets": n_sets, "status": st}
+
+
+def time_sampling(args, wl, sv, sets, n_sets, out_t, out_n, dev, world, local):
+    """Time the sampling-variant entry point on the bench batch: greedy, and
+    top-k 50 with top-p 0.9 at the workload's temperature."""
+    import torch
+    import torch.distributed as dist
+    res = {}
+    configs = {"greedy": (0.0, 0, 1.0), "top_k50_top_p0.9": (wl.temperature, 50, 0.9)}
+    for name, (T, k, p) in configs.items():
+        temps = torch.full((wl.batch,), T, dtype=torch.float32, device=dev)
+
+        def step(i):
+            d = sets[i % n_sets]
+            sv.run_sampling(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
+                            temps, out_t, out_n, top_k=k, top_p=p)
+
+        for i in range(max(3, args.warmup)):
+            step(i)
+        torch.cuda.synchronize()
+        stream = torch.cuda.current_stream()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize()
+        sv.profile_begin(args.steps)
+        ev0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        kern = sv.profile_end()
+        ms_max = svdist.max_over_ranks(ev0.elapsed_time(ev1), device=dev)
+        st, _ = sv.status()
+        res[name] = {"settings": {"temperature": T, "top_k": k, "top_p": p}, "ms_max": ms_max,
+                     "select_us": 1e3 * kern["stats_ms"], "decide_and_draw_us": 1e3 * kern["draw_ms"],
+                     "status": st}
+    return res
 
 
 def time_gate(args, dev, world, local):

@@ -9,11 +9,12 @@
 // Three stream-ordered kernels per pass:
 //   tree_kernel  one block: validates every branch's parent chain by pointer
 //                jumping in shared memory;
-//   rows_kernel  one warp per row (c, j): streams H[c, j] and H[parent, j]
-//                with 128-bit loads, sum of squares in fp32 per lane, fp64
-//                across the warp; decides recompute = !(d <= tau); ranks the
-//                recomputed rows of the block; the block that takes the last
-//                ticket turns the per-block counts into offsets;
+//   rows_kernel  persistent blocks over contiguous row ranges; each warp
+//                streams its rows' H[c, j] and H[parent, j] through a ring of
+//                cp.async stages, sums squares in fp32 per lane and fp64
+//                across the warp, and decides recompute = !(d <= tau); the
+//                block ranks its recomputed rows, and the block that takes
+//                the last ticket turns the per-block counts into offsets;
 //   pack_kernel  one warp per row: writes the packed row index, follows the
 //                fold chain to the source row, copies recomputed rows into the
 //                packed batch.
@@ -42,7 +43,8 @@ struct GateParams {
   double tau;
   int branches, positions, dim;
   long rows;
-  int blocks;               // rows_kernel / pack_kernel grid
+  int blocks;               // rows_kernel grid (persistent; each block a contiguous row range)
+  int pack_blocks;          // pack_kernel grid (8 rows per block)
   // outputs (rel_diff, provenance, source, packed_hidden may be null)
   float* rel_diff;
   int32_t* provenance;
@@ -53,7 +55,7 @@ struct GateParams {
   // workspace
   int32_t* eff_parent;      // [branches] parent after validation, -1 if none
   uint8_t* flag;            // [rows] 1: recompute
-  uint8_t* rank;            // [rows] rank among the recomputed rows of its block
+  int32_t* rank;            // [rows] rank among the recomputed rows of its block
   int32_t* prov;            // [rows] provenance (always kept for the chain walk)
   int32_t* block_count;     // [blocks]
   int32_t* block_offset;    // [blocks]
@@ -160,86 +162,181 @@ __global__ void __launch_bounds__(kTreeThreads) tree_kernel(const GateParams P) 
 // kernel 2: difference test
 // ---------------------------------------------------------------------------
 
-template <typename T, bool kAligned>
-__device__ __forceinline__ void row_sums(const T* hc, const T* hp, int dim, double& num,
-                                         double& den) {
-  const int lane = threadIdx.x & (kWarp - 1);
-  float d0 = 0.f, d1 = 0.f, n0 = 0.f, n1 = 0.f;
-  if constexpr (kAligned) {
-    constexpr int kU = 4;
-    const int groups = dim / HElem<T>::kPerVec;
-    const uint4* gc = reinterpret_cast<const uint4*>(hc);
-    const uint4* gp = reinterpret_cast<const uint4*>(hp);
-    int g = lane;
-    for (; g + (kU - 1) * kWarp < groups; g += kU * kWarp) {
-      uint4 c[kU], p[kU];
-#pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        c[u] = ld_v4(gc + g + u * kWarp);
-        p[u] = ld_v4(gp + g + u * kWarp);
-      }
-#pragma unroll
-      for (int u = 0; u < kU; ++u) HElem<T>::accumulate(c[u], p[u], d0, d1, n0, n1);
-    }
-    for (; g < groups; g += kWarp) HElem<T>::accumulate(ld_v4(gc + g), ld_v4(gp + g), d0, d1, n0, n1);
-  } else {
-    for (int k = lane; k < dim; k += kWarp) {
-      const float c = HElem<T>::scalar(hc, k), p = HElem<T>::scalar(hp, k);
-      const float e = c - p;
-      d0 = fmaf(e, e, d0);
-      n0 = fmaf(p, p, n0);
-    }
-  }
-  num = static_cast<double>(d0) + static_cast<double>(d1);
-  den = static_cast<double>(n0) + static_cast<double>(n1);
-#pragma unroll
-  for (int o = kWarp / 2; o > 0; o >>= 1) {
-    num += __shfl_xor_sync(0xffffffffu, num, o);
-    den += __shfl_xor_sync(0xffffffffu, den, o);
-  }
+constexpr int kStages = 8;  // cp.async stages in flight per warp
+constexpr int kStageBytes = kWarp * 32;  // one 16-byte group of child and parent per lane
+constexpr int kRowsSmem = kStages * kStageBytes * (kThreads / kWarp);
+
+// rows of block b: [row_start(b), row_start(b + 1))
+__device__ __forceinline__ long row_start(long b, long rows, int nblk) { return b * rows / nblk; }
+
+__device__ __forceinline__ int block_of(long row, long rows, int nblk) {
+  long b = row * nblk / rows;
+  while (b + 1 < nblk && row_start(b + 1, rows, nblk) <= row) ++b;
+  while (b > 0 && row_start(b, rows, nblk) > row) --b;
+  return static_cast<int>(b);
 }
 
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  const int n = valid ? 16 : 0;  // 0: fill with zeros, read nothing
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(gmem), "r"(n));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 1));
+}
+
+// lane 0's per-row epilogue: the decision and its records
+__device__ __forceinline__ bool finish_row(const GateParams& P, long row, int par, int j,
+                                           double num, double den) {
+  double d = INFINITY;
+  if (par >= 0) d = (den == 0.0) ? ((num == 0.0) ? 0.0 : INFINITY) : sqrt(num / den);
+  const bool rec = par < 0 || !(d <= P.tau);
+  const int32_t prov = rec ? -1 : static_cast<int32_t>(static_cast<long>(par) * P.positions + j);
+  P.prov[row] = prov;
+  P.flag[row] = rec ? 1 : 0;
+  if (P.provenance) P.provenance[row] = prov;
+  if (P.rel_diff) P.rel_diff[row] = static_cast<float>(d);
+  return rec;
+}
+
+// One persistent block per slot: block b owns the contiguous rows
+// [row_start(b), row_start(b + 1)); warp w takes every 8th of them.  With
+// 128-bit rows a warp streams its rows' (child, parent) groups through a ring
+// of kStages cp.async stages in shared memory, so loads stay in flight across
+// row boundaries without holding registers.
 template <typename T, bool kAligned>
 __global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
-  __shared__ unsigned s_flags;
+  extern __shared__ uint4 ring[];  // [warps][kStages][2][kWarp]
   __shared__ bool s_last;
+  __shared__ int s_count;
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x & (kWarp - 1);
-  const long row = static_cast<long>(blockIdx.x) * kRowsPerBlock + warp;
-  if (threadIdx.x == 0) s_flags = 0u;
+  const long r0 = row_start(blockIdx.x, P.rows, P.blocks);
+  const long r1 = row_start(blockIdx.x + 1, P.rows, P.blocks);
+  const T* base = static_cast<const T*>(P.hidden);
+  cudaGridDependencySynchronize();  // validated parents
 
-  // the validated parents come from the tree kernel
-  cudaGridDependencySynchronize();
-  __syncthreads();
-  bool rec = false;
-  if (row < P.rows) {
-    const int c = static_cast<int>(row / P.positions);
-    const int j = static_cast<int>(row - static_cast<long>(c) * P.positions);
-    const int par = P.eff_parent[c];
-    double d = INFINITY;
-    if (par >= 0) {
-      const T* base = static_cast<const T*>(P.hidden);
+  // rows of this warp: r0 + warp, r0 + warp + 8, ...; those without a parent
+  // are decided without reading anything
+  auto parent_of = [&](long row) -> int { return P.eff_parent[row / P.positions]; };
+  if (lane == 0)
+    for (long row = r0 + warp; row < r1; row += kRowsPerBlock)
+      if (parent_of(row) < 0) finish_row(P, row, -1, 0, 0.0, 0.0);
+  // next row at or after `row` (in this warp's sequence) that has a parent
+  auto next_row = [&](long row) -> long {
+    while (row < r1 && parent_of(row) < 0) row += kRowsPerBlock;
+    return row;
+  };
+
+  if constexpr (kAligned) {
+    constexpr int kVec = HElem<T>::kPerVec;
+    const int groups = P.dim / kVec;
+    const int chunks = (groups + kWarp - 1) / kWarp;  // units per row
+    uint4* my = ring + static_cast<long>(warp) * kStages * 2 * kWarp;
+    // issue pointer: the row being fetched, its two group pointers (this
+    // lane's group of chunk 0) and the chunk; all set once per row
+    long irow = next_row(r0 + warp);
+    int ichunk = 0;
+    const uint4* igc = nullptr;  // this lane's next group of the child row
+    const uint4* igp = nullptr;  // and of the parent row
+    const uint4* rc = nullptr;   // first group of each row: the (unread) source
+    const uint4* rp = nullptr;   // address of a zero-filling copy
+    auto set_issue_row = [&]() {
+      if (irow < r1) {
+        const int par = parent_of(irow);
+        const long j = irow - (irow / P.positions) * P.positions;
+        rc = reinterpret_cast<const uint4*>(base + irow * P.dim);
+        rp = reinterpret_cast<const uint4*>(base + (static_cast<long>(par) * P.positions + j) * P.dim);
+        igc = rc + lane;
+        igp = rp + lane;
+      }
+    };
+    set_issue_row();
+    int g_left = groups - lane;  // groups of the row at or after this lane's
+    auto issue = [&](int slot) {
+      if (irow < r1) {
+        const bool ok = g_left > 0;
+        cp_async16(my + (slot * 2 + 0) * kWarp + lane, ok ? igc : rc, ok);
+        cp_async16(my + (slot * 2 + 1) * kWarp + lane, ok ? igp : rp, ok);
+        igc += kWarp;
+        igp += kWarp;
+        g_left -= kWarp;
+        if (++ichunk == chunks) {
+          ichunk = 0;
+          g_left = groups - lane;
+          irow = next_row(irow + kRowsPerBlock);
+          set_issue_row();
+        }
+      }
+      cp_async_commit();  // an empty group keeps the wait count uniform
+    };
+#pragma unroll 1
+    for (int st = 0; st < kStages - 1; ++st) issue(st);
+    long crow = next_row(r0 + warp);
+    int cchunk = 0, slot = 0;
+    float d0 = 0.f, d1 = 0.f, n0 = 0.f, n1 = 0.f;
+    while (crow < r1) {
+      issue(slot == 0 ? kStages - 1 : slot - 1);
+      cp_async_wait();
+      const uint4 c = my[(slot * 2 + 0) * kWarp + lane];
+      const uint4 p = my[(slot * 2 + 1) * kWarp + lane];
+      HElem<T>::accumulate(c, p, d0, d1, n0, n1);
+      slot = (slot == kStages - 1) ? 0 : slot + 1;
+      if (++cchunk == chunks) {
+        double num = static_cast<double>(d0) + static_cast<double>(d1);
+        double den = static_cast<double>(n0) + static_cast<double>(n1);
+#pragma unroll
+        for (int o = kWarp / 2; o > 0; o >>= 1) {
+          num += __shfl_xor_sync(0xffffffffu, num, o);
+          den += __shfl_xor_sync(0xffffffffu, den, o);
+        }
+        if (lane == 0)
+          finish_row(P, crow, parent_of(crow), static_cast<int>(crow % P.positions), num, den);
+        d0 = d1 = n0 = n1 = 0.f;
+        cchunk = 0;
+        crow = next_row(crow + kRowsPerBlock);
+      }
+    }
+    asm volatile("cp.async.wait_all;");
+  } else {
+    for (long row = next_row(r0 + warp); row < r1; row = next_row(row + kRowsPerBlock)) {
+      const int par = parent_of(row);
+      const int j = static_cast<int>(row % P.positions);
       const T* hc = base + row * P.dim;
       const T* hp = base + (static_cast<long>(par) * P.positions + j) * P.dim;
-      double num, den;
-      row_sums<T, kAligned>(hc, hp, P.dim, num, den);
-      d = (den == 0.0) ? ((num == 0.0) ? 0.0 : INFINITY) : sqrt(num / den);
-    }
-    rec = par < 0 || !(d <= P.tau);
-    if (lane == 0) {
-      const int32_t prov = rec ? -1 : static_cast<int32_t>(static_cast<long>(par) * P.positions + j);
-      P.prov[row] = prov;
-      P.flag[row] = rec ? 1 : 0;
-      if (P.provenance) P.provenance[row] = prov;
-      if (P.rel_diff) P.rel_diff[row] = static_cast<float>(d);
-      if (rec) atomicOr(&s_flags, 1u << warp);
+      float dd = 0.f, nn = 0.f;
+      for (int k = lane; k < P.dim; k += kWarp) {
+        const float c = HElem<T>::scalar(hc, k), p = HElem<T>::scalar(hp, k);
+        const float e = c - p;
+        dd = fmaf(e, e, dd);
+        nn = fmaf(p, p, nn);
+      }
+      double num = dd, den = nn;
+#pragma unroll
+      for (int o = kWarp / 2; o > 0; o >>= 1) {
+        num += __shfl_xor_sync(0xffffffffu, num, o);
+        den += __shfl_xor_sync(0xffffffffu, den, o);
+      }
+      if (lane == 0) finish_row(P, row, par, j, num, den);
     }
   }
+
+  // ranks of the recomputed rows inside the block, in row order
   __syncthreads();
-  const unsigned flags = s_flags;
-  if (row < P.rows && lane == 0)
-    P.rank[row] = static_cast<uint8_t>(__popc(flags & ((1u << warp) - 1u)));
+  if (warp == 0) {
+    int running = 0;
+    for (long base_row = r0; base_row < r1; base_row += kWarp) {
+      const long row = base_row + lane;
+      const bool f = row < r1 && P.flag[row] != 0;
+      const unsigned m = __ballot_sync(0xffffffffu, f);
+      if (row < r1) P.rank[row] = running + __popc(m & ((1u << lane) - 1u));
+      running += __popc(m);
+    }
+    if (lane == 0) s_count = running;
+  }
+  __syncthreads();
   if (threadIdx.x == 0) {
-    P.block_count[blockIdx.x] = __popc(flags);
+    P.block_count[blockIdx.x] = s_count;
     __threadfence();
     // atomicInc wraps to 0 at the last block, so the ticket resets itself
     s_last = atomicInc(P.ticket, static_cast<unsigned>(P.blocks - 1)) ==
@@ -254,8 +351,8 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
   __shared__ int32_t s_carry;
   if (threadIdx.x == 0) s_carry = 0;
   __syncthreads();
-  for (int base = 0; base < P.blocks; base += kScanThreads) {
-    const int i = base + threadIdx.x;
+  for (int b0 = 0; b0 < P.blocks; b0 += kScanThreads) {
+    const int i = b0 + threadIdx.x;
     const int v = (i < P.blocks) ? __ldcg(P.block_count + i) : 0;
     int x = v;
 #pragma unroll
@@ -288,6 +385,7 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
 // kernel 3: packing and fold-chain resolution
 // ---------------------------------------------------------------------------
 
+// one warp per row; the row's slot is its block's offset plus its rank
 template <typename T, bool kAligned>
 __global__ void __launch_bounds__(kThreads) pack_kernel(const GateParams P) {
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x & (kWarp - 1);
@@ -296,7 +394,9 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const GateParams P) {
   if (row >= P.rows) return;
   const bool rec = __ldcg(P.flag + row) != 0;
   long slot = 0;
-  if (rec) slot = static_cast<long>(__ldcg(P.block_offset + blockIdx.x)) + __ldcg(P.rank + row);
+  if (rec)
+    slot = static_cast<long>(__ldcg(P.block_offset + block_of(row, P.rows, P.blocks))) +
+           __ldcg(P.rank + row);
   if (lane == 0) {
     if (rec) P.packed[slot] = static_cast<int32_t>(row);
     if (P.source) {

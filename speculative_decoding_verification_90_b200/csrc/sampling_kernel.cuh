@@ -153,6 +153,20 @@ __device__ __forceinline__ unsigned block_max_u(unsigned v, unsigned* sm) {
 }
 
 template <int NT>
+__device__ __forceinline__ unsigned block_min_u(unsigned v, unsigned* sm) {
+  const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();
+  if (lane == 0) sm[warp] = v;
+  __syncthreads();
+  unsigned t = 0xffffffffu;
+#pragma unroll
+  for (int w = 0; w < NT / kWarp; ++w) t = min(t, sm[w]);
+  return t;
+}
+
+template <int NT>
 __device__ __forceinline__ int block_min_i(int v, int* sm) {
   const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x >> 5;
 #pragma unroll
@@ -180,15 +194,63 @@ __device__ __forceinline__ int block_max_i(int v, int* sm) {
   return t;
 }
 
+// Row scans.  With 16-byte aligned rows a thread reads one 16-byte group per
+// step (consecutive threads, consecutive groups); otherwise one element.
+// `f(x, i)` sees every element once.  The loop count is the same for all
+// threads of the block, so `f` may use warp collectives when `kUniform`.
+template <typename T, bool kAligned, bool kUniform, typename F>
+__device__ __forceinline__ void scan_row(const T* row, int V, F&& f) {
+  if constexpr (kAligned) {
+    // four groups per thread in flight per round
+    constexpr int kVec = Elem<T>::kVec;
+    constexpr int kU = 4;
+    const long groups = V / kVec;
+    const uint4* g4 = reinterpret_cast<const uint4*>(row);
+    const long stride = static_cast<long>(blockDim.x) * kU;
+    const long end = kUniform ? ((groups + stride - 1) / stride) * stride : groups;
+    for (long g0 = threadIdx.x; g0 < end; g0 += stride) {
+      uint4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const long g = g0 + static_cast<long>(u) * blockDim.x;
+        if (g < groups) v[u] = __ldg(g4 + g);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const long g = g0 + static_cast<long>(u) * blockDim.x;
+        const bool in = g < groups;
+        if (!kUniform && !in) break;
+        float x[kVec];
+        if (in) {
+          Elem<T>::unpack(v[u], x);
+        } else {
+#pragma unroll
+          for (int e = 0; e < kVec; ++e) x[e] = NAN;
+        }
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) f(x[e], in ? g * kVec + e : -1L);
+      }
+    }
+  } else {
+    const long end = kUniform ? ((static_cast<long>(V) + blockDim.x - 1) / blockDim.x) * blockDim.x : V;
+    for (long i = threadIdx.x; i < end; i += blockDim.x) {
+      const bool in = i < V;
+      f(in ? elem<T>(row, i) : NAN, in ? i : -1L);
+    }
+  }
+}
+
 // The count-based radix select: the `rank`-th largest key (1-based) among the
 // row's entries with key >= `floor_key`, for keys whose low `low_bits` bits are
 // zero (bf16 values widened to float).  Histograms of 256 bins per 8-bit digit
 // in shared memory; each warp adds a bin's lanes once (match_any).  Returns the
 // key, and in *count_eq the number of entries equal to it.
-template <typename T>
+template <typename T, bool kAligned>
 __device__ unsigned radix_select(const T* row, int V, unsigned floor_key, long rank, int low_bits,
                                  int* hist, int* count_eq) {
-  const int lane = threadIdx.x & (kWarp - 1);
+  // hist: kSelWarps private histograms of 256 bins (plain shared atomics; a
+  // warp's lanes that share a bin are serialised by the hardware)
+  const int warp = threadIdx.x >> 5;
   __shared__ unsigned s_prefix, s_mask;
   __shared__ long s_rank;
   __shared__ int s_eq;
@@ -199,41 +261,55 @@ __device__ unsigned radix_select(const T* row, int V, unsigned floor_key, long r
     s_eq = 0;
   }
   __syncthreads();
+  int* mine = hist + warp * 256;
   for (int shift = 24; shift >= low_bits; shift -= 8) {
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < 256 * kSelWarps; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     const unsigned prefix = s_prefix, mask = s_mask;
-    const long nV = V;
-    for (long base = 0; base < nV; base += blockDim.x) {
-      const long i = base + threadIdx.x;
-      bool in = false;
-      unsigned bin = 0;
-      if (i < nV) {
-        const unsigned k = fkey(elem<T>(row, i));
-        in = k >= floor_key && (k & mask) == prefix;
-        bin = (k >> shift) & 255u;
-      }
-      const unsigned act = __ballot_sync(0xffffffffu, in);
-      if (in) {
-        const unsigned grp = __match_any_sync(act, bin);
-        if (lane == __ffs(grp) - 1) atomicAdd(&hist[bin], __popc(grp));
-      }
+    scan_row<T, kAligned, false>(row, V, [&](float x, long) {
+      const unsigned k = fkey(x);
+      if (k >= floor_key && (k & mask) == prefix) atomicAdd(&mine[(k >> shift) & 255u], 1);
+    });
+    __syncthreads();
+    // totals into the first histogram
+    for (int bin = threadIdx.x; bin < 256; bin += blockDim.x) {
+      int t = 0;
+      for (int w = 0; w < kSelWarps; ++w) t += hist[w * 256 + bin];
+      hist[bin] = t;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      long need = s_rank, cum = 0;
-      int sel = 0;
-      for (int b = 255; b >= 0; --b) {
-        if (cum + hist[b] >= need) {
-          sel = b;
-          break;
+    if (threadIdx.x < kWarp) {
+      // the bin holding the rank-th largest: warp scan from the top bin down
+      const int lane = threadIdx.x;
+      long need = s_rank;
+      long cum = 0;
+      int sel = -1;
+      for (int base = 255; base >= 0 && sel < 0; base -= kWarp) {
+        const int bin = base - lane;
+        long c = hist[bin];
+        long incl = c;
+#pragma unroll
+        for (int o = 1; o < kWarp; o <<= 1) {
+          const long y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
         }
-        cum += hist[b];
+        const unsigned hit = __ballot_sync(0xffffffffu, cum + incl >= need);
+        if (hit) {
+          const int l = __ffs(hit) - 1;
+          const long before = __shfl_sync(0xffffffffu, incl - c, l);
+          sel = base - l;
+          cum += before;
+        } else {
+          cum += __shfl_sync(0xffffffffu, incl, kWarp - 1);
+        }
       }
-      s_rank = need - cum;
-      s_prefix = prefix | (static_cast<unsigned>(sel) << shift);
-      s_mask = mask | (255u << shift);
-      s_eq = hist[sel];
+      if (lane == 0) {
+        if (sel < 0) sel = 0;
+        s_rank = need - cum;
+        s_prefix = prefix | (static_cast<unsigned>(sel) << shift);
+        s_mask = mask | (255u << shift);
+        s_eq = hist[sel];
+      }
     }
     __syncthreads();
   }
@@ -241,17 +317,15 @@ __device__ unsigned radix_select(const T* row, int V, unsigned floor_key, long r
   return s_prefix;
 }
 
-// sum over the row of 2^(x c - o) for entries with key >= lo (and key < hi
-// when hi != 0), per thread in fp32, over the block in fp64
-template <typename T>
-__device__ double masked_mass(const T* row, int V, unsigned lo, unsigned hi, float c_hi,
-                              float c_lo, float o, double* sm) {
+// sum over the row of 2^(x c - o) for entries with key >= lo, per thread in
+// fp32, over the block in fp64
+template <typename T, bool kAligned>
+__device__ double masked_mass(const T* row, int V, unsigned lo, float c_hi, float c_lo, float o,
+                              double* sm) {
   float s = 0.f;
-  for (long i = threadIdx.x; i < V; i += blockDim.x) {
-    const float x = elem<T>(row, i);
-    const unsigned k = fkey(x);
-    if (k >= lo && (hi == 0u || k < hi)) s += ex2(specverify::arg2(x, c_hi, c_lo, o));
-  }
+  scan_row<T, kAligned, false>(row, V, [&](float x, long) {
+    if (fkey(x) >= lo) s += ex2(specverify::arg2(x, c_hi, c_lo, o));
+  });
   return block_sum<kSelThreads>(static_cast<double>(s), sm);
 }
 
@@ -266,15 +340,260 @@ __device__ __forceinline__ void put_row(const SampParams& P, long r, long nT, co
   else P.dstat[r - nT] = st;
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const SampParams P) {
-  __shared__ int hist[256];
+// Candidates: entries gathered into shared memory (key, weight in double
+// precision rounded to float) when their key is above `above` and at least
+// `floor_key`; the count may exceed kCand (then only the first kCand are kept
+// and the caller falls back).  Entries equal to `above` are counted in *n_eq.
+template <typename T, bool kAligned, bool kTail>
+__device__ int gather(const T* row, int V, unsigned above, unsigned floor_key, double c, double od,
+                      unsigned* cand_key, float* cand_w, int* cand_n, float c_hi, float c_lo,
+                      float o, double* sm, double* n_eq_out, double* tail_out) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  if (threadIdx.x == 0) *cand_n = 0;
+  __syncthreads();
+  int n_eq = 0;
+  float tail = 0.f;  // entries floor_key <= key < above
+  scan_row<T, kAligned, true>(row, V, [&](float x, long i) {
+    const unsigned k = fkey(x);
+    const bool valid = i >= 0;
+    const bool take = valid && k > above && k >= floor_key;
+    n_eq += (valid && k == above && k >= floor_key);
+    if (kTail && valid && k < above && k >= floor_key) tail += ex2(specverify::arg2(x, c_hi, c_lo, o));
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (m) {
+      int at = 0;
+      if (lane == __ffs(m) - 1) at = atomicAdd(cand_n, __popc(m));
+      at = __shfl_sync(0xffffffffu, at, __ffs(m) - 1);
+      if (take) {
+        const int slot = at + __popc(m & ((1u << lane) - 1u));
+        if (slot < kCand) cand_key[slot] = k;
+      }
+    }
+  });
+  __syncthreads();
+  const int n = *cand_n;
+  // the candidates' weights in double precision (rounded to float), after the
+  // scan so that no lane waits on another's exp2
+  for (int i = threadIdx.x; i < min(n, kCand); i += blockDim.x)
+    cand_w[i] = static_cast<float>(exp2(static_cast<double>(key_value(cand_key[i])) * c - od));
+  *n_eq_out = block_sum<kSelThreads>(static_cast<double>(n_eq), sm);
+  *tail_out = block_sum<kSelThreads>(static_cast<double>(tail), sm) * exp2(static_cast<double>(o) - od);
+  return n;
+}
+
+// A reduction over either warp 0 alone (kW) or the whole block.
+template <bool kW>
+struct Red {
+  double* sm;
+  __device__ __forceinline__ double sum(double v) const {
+    if constexpr (kW) return specverify::warp_sum(v);
+    else return block_sum<kSelThreads>(v, sm);
+  }
+  __device__ __forceinline__ int first() const { return kW ? (threadIdx.x & (kWarp - 1)) : threadIdx.x; }
+  __device__ __forceinline__ int stride() const { return kW ? kWarp : static_cast<int>(blockDim.x); }
+};
+
+constexpr int kWarpCands = 2048;  // candidate sets up to this size: warp 0 alone
+
+struct CandSet {
+  const unsigned* key;
+  const float* w;   // weights 2^(x c - od), double-precision exp2 rounded to float
+  int n;
+  unsigned above;   // every entry with key > above is a candidate
+  double n_eq;      // entries equal to `above` (not stored; one weight)
+  double w_above;
+  double tail;      // mass of the entries theta <= key < above
+  unsigned kmax, step;
+};
+
+struct StageOut {
+  unsigned theta;
+  float margin;
+  double Z, kept;   // mass (when z_valid) and count (when kept_valid) of the kept set
+  double Zk, goal;  // for the whole-row fallback, when below
+  int z_valid, kept_valid, below;
+};
+
+// The top-k cut (when `do_k`: the k-th largest candidate key, searched from
+// `theta` = a lower bound) and the nucleus cut (when `do_p`) over the
+// candidates; run by warp 0 alone or by the whole block.  Thread 0 writes *out.
+template <bool kW>
+__device__ void cand_stage(const Red<kW>& R, const CandSet& cs, bool do_k, int top_k, bool do_p,
+                           double top_p, unsigned theta, StageOut* out) {
+  const int f = R.first(), st = R.stride();
+  const unsigned step = cs.step;
+  if (do_k) {
+    unsigned lo = theta, hi = cs.kmax;
+    while (lo < hi) {
+      const unsigned mid = lo + (((hi - lo) / step + 1) / 2) * step;
+      double cnt = 0.0;
+      for (int i = f; i < cs.n; i += st) cnt += cs.key[i] >= mid ? 1.0 : 0.0;
+      if (R.sum(cnt) >= top_k) lo = mid;
+      else hi = mid - step;
+    }
+    theta = lo;
+  }
+  // M(>= v): candidates >= max(v, theta), plus the group at `above`
+  auto mass_ge = [&](unsigned v) -> double {
+    double sv = 0.0;
+    for (int i = f; i < cs.n; i += st)
+      if (cs.key[i] >= v && cs.key[i] >= theta) sv += static_cast<double>(cs.w[i]);
+    double t = R.sum(sv);
+    if (v <= cs.above && cs.above >= theta) t += cs.n_eq * cs.w_above;
+    return t;
+  };
+  StageOut o{theta, INFINITY, 0.0, 0.0, 0.0, 0.0, 0, 0, 0};
+  if (do_p) {
+    const unsigned v0 = max(theta, cs.above);
+    const double m0 = mass_ge(v0);
+    const double Zk = cs.tail + m0;  // mass of the entries >= theta
+    const double goal = top_p * Zk;
+    o.Zk = Zk;
+    o.goal = goal;
+    if (m0 >= goal) {
+      unsigned lo = v0, hi = cs.kmax;
+      while (lo < hi) {
+        const unsigned mid = lo + (((hi - lo) / step + 1) / 2) * step;
+        if (mass_ge(mid) >= goal) lo = mid;
+        else hi = mid - step;
+      }
+      const double m_ge = mass_ge(lo);
+      const double m_gt = (lo >= cs.kmax) ? 0.0 : mass_ge(lo + step);
+      o.margin = static_cast<float>(fmin(top_p - m_gt / Zk, m_ge / Zk - top_p));
+      o.theta = max(theta, lo);
+    } else {
+      o.below = 1;
+    }
+  }
+  // the kept set's mass and size, when every kept entry is a candidate
+  if (!o.below && o.theta > cs.above) {
+    double sv = 0.0, cnt = 0.0;
+    for (int i = f; i < cs.n; i += st)
+      if (cs.key[i] >= o.theta && key_value(cs.key[i]) != -INFINITY) {
+        sv += static_cast<double>(cs.w[i]);
+        cnt += 1.0;
+      }
+    o.Z = R.sum(sv);
+    o.kept = R.sum(cnt);
+    o.z_valid = 1;
+    o.kept_valid = 1;
+  } else if (!o.below && do_p) {
+    o.Z = mass_ge(o.theta);  // includes the group at `above`; the count comes from a pass
+    o.z_valid = 1;
+  }
+  if (threadIdx.x == 0) *out = o;
+}
+
+struct PassA {
+  float mx;     // largest value of the thread's entries
+  long am;      // its first index
+  bool bad;     // a NaN or +inf entry
+  float t[4];   // the thread's four largest values, descending (-inf: empty)
+  float o, s;   // with kSum: s = sum 2^(x c - o) over the thread's entries
+  int ninf;     // with kSum: entries equal to -inf
+};
+
+// One scan of the row: each thread's maximum, first argmax and invalid
+// entries; with kTrack also its four largest values, inserted only when a
+// 16-byte group's maximum beats the fourth (rare after the first groups).
+template <typename T, bool kAligned, bool kTrack, bool kSum>
+__device__ __forceinline__ PassA pass_a(const T* row, int V, float c_hi, float c_lo) {
+  PassA a{-INFINITY, 0x7fffffff, false, {-INFINITY, -INFINITY, -INFINITY, -INFINITY},
+          -INFINITY, 0.f, 0};
+  auto insert = [&](float x) {
+    if (x > a.t[3]) {  // old values on the right
+      a.t[3] = fmaxf(a.t[3], fminf(a.t[2], x));
+      a.t[2] = fmaxf(a.t[2], fminf(a.t[1], x));
+      a.t[1] = fmaxf(a.t[1], fminf(a.t[0], x));
+      a.t[0] = fmaxf(a.t[0], x);
+    }
+  };
+  if constexpr (kAligned) {
+    constexpr int kVec = Elem<T>::kVec;
+    constexpr int kU = 4;
+    const long groups = V / kVec;
+    const uint4* g4 = reinterpret_cast<const uint4*>(row);
+    const long stride = static_cast<long>(blockDim.x) * kU;
+    for (long g0 = threadIdx.x; g0 < groups; g0 += stride) {
+      uint4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const long g = g0 + static_cast<long>(u) * blockDim.x;
+        if (g < groups) v[u] = __ldg(g4 + g);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const long g = g0 + static_cast<long>(u) * blockDim.x;
+        if (g >= groups) break;
+        float x[kVec];
+        Elem<T>::unpack(v[u], x);
+        float gm = x[0];
+        bool gb = (x[0] != x[0]) || x[0] == INFINITY;
+#pragma unroll
+        for (int e = 1; e < kVec; ++e) {
+          gm = fmaxf(gm, x[e]);
+          gb |= (x[e] != x[e]) || x[e] == INFINITY;
+        }
+        a.bad |= gb;
+        if (gm > a.mx) {  // the first index of the group's maximum
+          a.mx = gm;
+#pragma unroll
+          for (int e = kVec - 1; e >= 0; --e)
+            if (x[e] == gm) a.am = g * kVec + e;
+        }
+        if (kTrack && gm > a.t[3]) {
+#pragma unroll
+          for (int e = 0; e < kVec; ++e) insert(x[e]);
+        }
+        if constexpr (kSum) {
+          const float on = gm * c_hi;
+          if (on > a.o) {  // raise the offset (a.o = -inf: a.s is 0 and stays so)
+            a.s *= ex2(a.o - on);
+            a.o = on;
+          }
+#pragma unroll
+          for (int e = 0; e < kVec; ++e) {
+            a.s += ex2(specverify::arg2(x[e], c_hi, c_lo, a.o));
+            a.ninf += x[e] == -INFINITY;
+          }
+        }
+      }
+    }
+  } else {
+    for (long i = threadIdx.x; i < V; i += blockDim.x) {
+      const float x = elem<T>(row, i);
+      a.bad |= (x != x) || x == INFINITY;
+      if (x > a.mx) {
+        a.mx = x;
+        a.am = i;
+      }
+      if (kTrack) insert(x);
+      if constexpr (kSum) {
+        const float on = x * c_hi;
+        if (on > a.o) {
+          a.s *= ex2(a.o - on);
+          a.o = on;
+        }
+        a.s += ex2(specverify::arg2(x, c_hi, c_lo, a.o));
+        a.ninf += x == -INFINITY;
+      }
+    }
+  }
+  return a;
+}
+
+template <typename T, bool kAligned>
+__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SampParams P) {
   __shared__ double smd[kSelWarps];
   __shared__ unsigned smu[kSelWarps];
   __shared__ int smi[kSelWarps];
+  __shared__ unsigned s_tmax[kSelThreads];
   extern __shared__ unsigned cand_smem[];  // kCand keys, then kCand weights
   unsigned* cand_key = cand_smem;
   float* cand_w = reinterpret_cast<float*>(cand_smem + kCand);
+  // the radix select's per-warp histograms reuse the candidate area: every
+  // radix select runs before the candidates it serves are gathered
+  int* hist = reinterpret_cast<int*>(cand_smem);
   __shared__ int cand_n;
 
   const int G = P.gamma, V = P.vocab;
@@ -286,23 +605,30 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SampParams P)
                       : static_cast<const T*>(P.draft) + (r - nT) * V;
   const float temp = P.temperature[b];
   const int low_bits = sizeof(T) == 2 ? 16 : 0;
+  const unsigned step = 1u << low_bits;
 
-  // pass A: maximum, first argmax, invalid entries
-  float mx = -INFINITY;
-  int am = 0x7fffffff;
-  bool bad = false;
-  for (long i = threadIdx.x; i < V; i += blockDim.x) {
-    const float x = elem<T>(row, i);
-    bad |= (x != x) || x == INFINITY;
-    if (x > mx) {
-      mx = x;
-      am = static_cast<int>(i);
-    }
-  }
+  // pass A: maximum, first argmax, invalid entries, and (for a top-k cut)
+  // each thread's four largest values
+  PassA a;
+  float c_hi = 0.f, c_lo = 0.f;
+  double c = 0.0;
+  if (temp_ok(temp) && temp > 0.f) temp_consts(temp, c_hi, c_lo, c);
+  const bool any_filter = (P.top_k > 0 && P.top_k < V) || P.top_p < 1.0;
+  if (P.top_k > 0 && P.top_k <= kSelThreads && P.top_k < V && temp > 0.f)
+    a = pass_a<T, kAligned, true, false>(row, V, c_hi, c_lo);
+  else if (!any_filter && temp > 0.f && temp_ok(temp))
+    a = pass_a<T, kAligned, false, true>(row, V, c_hi, c_lo);  // the normaliser in the same scan
+  else
+    a = pass_a<T, kAligned, false, false>(row, V, c_hi, c_lo);
+  const float mx = a.mx;
+  const long am = a.am;
+  const bool bad = a.bad;
+  const unsigned t0 = fkey(a.t[0]), t1 = fkey(a.t[1]), t2 = fkey(a.t[2]), t3 = fkey(a.t[3]);
+  s_tmax[threadIdx.x] = fkey(mx);
   const unsigned kmax = block_max_u<kSelThreads>(bad ? 0u : fkey(mx), smu);
   const bool any_bad = __syncthreads_or(bad);
   const float gmx = key_value(kmax);
-  const int arg = block_min_i<kSelThreads>(mx == gmx ? am : 0x7fffffff, smi);
+  const int arg = block_min_i<kSelThreads>(mx == gmx ? static_cast<int>(am) : 0x7fffffff, smi);
   SampRow out{0.0, 0u, arg, 1, V, INFINITY, 0};
   if (!temp_ok(temp)) {
     out.valid = 0;
@@ -325,131 +651,186 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SampParams P)
     if (threadIdx.x == 0) put_row(P, r, nT, out);
     return;
   }
-  float c_hi, c_lo;
-  double c;
-  temp_consts(temp, c_hi, c_lo, c);
-  const float o = gmx * c_hi;  // weights 2^(x c - o) are at most about 1
+  if (!any_filter) {
+    // no filter: the normaliser of the whole row from pass A
+    const float O = key_value(block_max_u<kSelThreads>(a.o == -INFINITY ? 0u : fkey(a.o), smu));
+    const double S = block_sum<kSelThreads>(
+        a.o == -INFINITY ? 0.0 : static_cast<double>(a.s) * exp2(static_cast<double>(a.o) - O), smd);
+    const double ninf = block_sum<kSelThreads>(static_cast<double>(a.ninf), smd);
+    if (threadIdx.x == 0) {
+      out.l2 = static_cast<double>(O) + log2(S);
+      out.theta = 0u;
+      out.kept = V - static_cast<int>(ninf);
+      put_row(P, r, nT, out);
+    }
+    return;
+  }
+  const float o = gmx * c_hi;                       // fp32 weights 2^(x c - o)
+  const double od = static_cast<double>(gmx) * c;   // fp64 weights 2^(x c - od)
+  const bool use_k = P.top_k > 0 && P.top_k < V;
+  const bool use_p = P.top_p < 1.0;
 
-  // top-k threshold
+  // The candidate set in shared memory: every entry with key > `above` (and
+  // >= theta), plus the group of entries equal to `above`, all of one weight.
+  __shared__ StageOut s_st;
   unsigned theta = 0u;
+  unsigned above = 0u;
+  int nc = -1;  // candidates gathered (-1: none)
+  double n_eq = 0.0, tail = 0.0;
   int eq = 0;
-  if (P.top_k > 0 && P.top_k < V) theta = radix_select<T>(row, V, 0u, P.top_k, low_bits, hist, &eq);
+  if (use_k && P.top_k <= kSelThreads) {
+    // The threads' four largest keys hold every entry >= their k-th largest
+    // value theta4 when no thread's fourth key reaches theta4 (a thread with
+    // more entries >= theta4 would have its fourth key >= theta4).  Then
+    // theta4 is the row's k-th largest key and the lists are the candidates.
+    cand_key[4 * threadIdx.x + 0] = t0;
+    cand_key[4 * threadIdx.x + 1] = t1;
+    cand_key[4 * threadIdx.x + 2] = t2;
+    cand_key[4 * threadIdx.x + 3] = t3;
+    __syncthreads();
+    __shared__ unsigned s_t4;
+    __shared__ int s_t4_ok;
+    if (threadIdx.x < kWarp) {
+      unsigned lo = 0u, hi = kmax, m3 = 0u;
+      while (lo < hi) {
+        const unsigned mid = lo + (((hi - lo) / step + 1) / 2) * step;
+        int cnt = 0;
+        for (int i = threadIdx.x; i < 4 * kSelThreads; i += kWarp) cnt += cand_key[i] >= mid;
+        if (__reduce_add_sync(0xffffffffu, cnt) >= P.top_k) lo = mid;
+        else hi = mid - step;
+      }
+      for (int i = threadIdx.x; i < kSelThreads; i += kWarp) m3 = max(m3, cand_key[4 * i + 3]);
+      m3 = __reduce_max_sync(0xffffffffu, m3);
+      if (threadIdx.x == 0) {
+        s_t4 = lo;
+        s_t4_ok = (m3 < lo) && lo > fkey(-INFINITY);  // empty places are -inf
+      }
+    }
+    __syncthreads();
+    if (s_t4_ok) {
+      const unsigned t4 = s_t4;
+      for (int i = threadIdx.x; i < 4 * kSelThreads; i += blockDim.x) {
+        const unsigned k = cand_key[i];
+        cand_w[i] = (k >= t4) ? static_cast<float>(exp2(static_cast<double>(key_value(k)) * c - od)) : 0.f;
+      }
+      __syncthreads();
+      nc = 4 * kSelThreads;
+      above = t4 - 1u;  // every entry >= t4 is in the lists
+      theta = t4;
+      n_eq = 0.0;
+      tail = 0.0;
+    }
+  }
+  if (use_k && P.top_k <= kSelThreads && nc < 0) {
+    // a lower bound on the k-th largest: the k-th largest of the threads'
+    // maxima (k distinct entries are at or above it); a short row is
+    // gathered whole.  Warp 0 searches the kSelThreads maxima.
+    __shared__ unsigned s_lb;
+    if (threadIdx.x < kWarp) {
+      unsigned lo = 0u, hi = (V > kCand) ? kmax : 0u;
+      while (lo < hi) {
+        const unsigned mid = lo + (((hi - lo) / step + 1) / 2) * step;
+        int cnt = 0;
+        for (int i = threadIdx.x; i < kSelThreads; i += kWarp) cnt += s_tmax[i] >= mid;
+        if (__reduce_add_sync(0xffffffffu, cnt) >= P.top_k) lo = mid;
+        else hi = mid - step;
+      }
+      if (threadIdx.x == 0) s_lb = lo;
+    }
+    __syncthreads();
+    const unsigned lb = s_lb;
+    const unsigned lb_floor = lb > 0u ? lb - 1u : 0u;  // gather keys >= lb
+    const int n = gather<T, kAligned, false>(row, V, lb_floor, 0u, c, od, cand_key, cand_w, &cand_n,
+                                             c_hi, c_lo, o, smd, &n_eq, &tail);
+    if (n <= kCand) {
+      nc = n;
+      above = lb_floor;
+      theta = lb;    // raised to the k-th largest candidate below
+      n_eq = 0.0;    // the candidates hold every entry >= lb
+      tail = 0.0;
+    }
+  }
+  if (use_k && nc < 0) theta = radix_select<T, kAligned>(row, V, 0u, P.top_k, low_bits, hist, &eq);
+  const bool k_in_cands = use_k && nc >= 0;
 
-  // nucleus threshold
-  float margin = INFINITY;
-  bool z_known = false;
-  double Z_kept = 0.0;
-  if (P.top_p < 1.0) {
-    // candidate key vc: the kCand-th largest key >= theta (theta itself when
-    // fewer entries are kept).  The entries strictly above vc (fewer than
-    // kCand) go to shared memory with weights from the double-precision exp2;
-    // the entries equal to vc form one group of equal weight.
+  if (use_p && nc < 0) {
+    // candidate key: the kCand-th largest key >= theta (theta itself when
+    // fewer entries are kept)
     unsigned vc = theta;
-    {
+    double nd = V;  // without a top-k cut every entry is >= theta = 0
+    if (theta > 0u) {
       int n_ge = 0;
-      for (long i = threadIdx.x; i < V; i += blockDim.x) n_ge += fkey(elem<T>(row, i)) >= theta;
-      const double nd = block_sum<kSelThreads>(static_cast<double>(n_ge), smd);
-      int eq_c = 0;
-      if (nd > kCand) vc = radix_select<T>(row, V, theta, kCand, low_bits, hist, &eq_c);
+      scan_row<T, kAligned, false>(row, V, [&](float x, long) { n_ge += fkey(x) >= theta; });
+      nd = block_sum<kSelThreads>(static_cast<double>(n_ge), smd);
     }
-    if (threadIdx.x == 0) cand_n = 0;
-    __syncthreads();
-    const int lane = threadIdx.x & (kWarp - 1);
-    const double od = static_cast<double>(gmx) * c;
-    int n_eq = 0;
-    float tail = 0.f;  // entries theta <= key < vc (all lighter than every candidate)
-    for (long base = 0; base < V; base += blockDim.x) {
-      const long i = base + threadIdx.x;
-      float x = -INFINITY;
-      unsigned k = 0u;
-      if (i < V) {
-        x = elem<T>(row, i);
-        k = fkey(x);
-      }
-      const bool take = i < V && k > vc && k >= theta;
-      n_eq += (i < V && k == vc && k >= theta);
-      if (i < V && k < vc && k >= theta) tail += ex2(specverify::arg2(x, c_hi, c_lo, o));
-      const unsigned m = __ballot_sync(0xffffffffu, take);
-      int at = 0;
-      if (lane == 0 && m) at = atomicAdd(&cand_n, __popc(m));
-      at = __shfl_sync(0xffffffffu, at, 0);
-      if (take) {
-        const int slot = at + __popc(m & ((1u << lane) - 1u));
-        if (slot < kCand) {
-          cand_key[slot] = k;
-          cand_w[slot] = static_cast<float>(exp2(static_cast<double>(x) * c - od));
-        }
-      }
-    }
-    __syncthreads();
-    const int nc = min(cand_n, kCand);
-    const double n_vc = block_sum<kSelThreads>(static_cast<double>(n_eq), smd);
-    const double z_tail = block_sum<kSelThreads>(static_cast<double>(tail), smd) *
-                          exp2(static_cast<double>(o) - od);
-    // (no entry equals vc when every entry is a candidate: vc may then be a key
-    // that decodes to no finite value)
-    const float xv = key_value(vc);
-    const double w_vc = (n_vc > 0.0 && xv != -INFINITY) ? exp2(static_cast<double>(xv) * c - od) : 0.0;
-    // M(>= v) for v >= vc: the candidates at or above v, plus the vc group
-    auto mass_ge = [&](unsigned v) -> double {
-      double sv = 0.0;
-      for (int i = threadIdx.x; i < nc; i += blockDim.x)
-        if (cand_key[i] >= v) sv += static_cast<double>(cand_w[i]);
-      double t = block_sum<kSelThreads>(sv, smd);
-      if (v <= vc) t += n_vc * w_vc;
-      return t;
-    };
-    const double m_vc = mass_ge(vc);
-    const double Zk = z_tail + m_vc;   // mass of the entries >= theta
-    const double goal = P.top_p * Zk;
-    const unsigned step = 1u << low_bits;
-    unsigned lo, hi;  // the largest v in [lo, hi] with M(>= v) >= goal
-    double m_ge, m_gt;
-    if (m_vc >= goal) {
-      lo = vc;
-      hi = kmax;
-      while (lo < hi) {
-        const unsigned mid = lo + (((hi - lo) / step + 1) / 2) * step;
-        if (mass_ge(mid) >= goal) lo = mid;
-        else hi = mid - step;
-      }
-      m_ge = mass_ge(lo);
-      m_gt = (lo >= kmax) ? 0.0 : mass_ge(lo + step);
-      Z_kept = m_ge;
-      z_known = true;
-    } else {
-      // the boundary lies below the candidates: whole-row passes (fp32 weights)
-      const double sc = exp2(static_cast<double>(o) - od);
-      lo = theta;
-      hi = vc;
-      while (lo < hi) {
-        const unsigned mid = lo + (((hi - lo) / step + 1) / 2) * step;
-        if (masked_mass<T>(row, V, mid, 0u, c_hi, c_lo, o, smd) * sc >= goal) lo = mid;
-        else hi = mid - step;
-      }
-      m_ge = masked_mass<T>(row, V, lo, 0u, c_hi, c_lo, o, smd) * sc;
-      m_gt = masked_mass<T>(row, V, lo + step, 0u, c_hi, c_lo, o, smd) * sc;
-    }
-    margin = static_cast<float>(fmin(P.top_p - m_gt / Zk, m_ge / Zk - P.top_p));
-    theta = max(theta, lo);
+    int eq_c = 0;
+    if (nd > kCand) vc = radix_select<T, kAligned>(row, V, theta, kCand, low_bits, hist, &eq_c);
+    nc = min(gather<T, kAligned, true>(row, V, vc, theta, c, od, cand_key, cand_w, &cand_n, c_hi,
+                                       c_lo, o, smd, &n_eq, &tail),
+             kCand);
+    above = vc;
   }
 
-  // log-normaliser and size of the kept set
-  float s = 0.f;
-  int kept = 0;
-  for (long i = threadIdx.x; i < V; i += blockDim.x) {
-    const float x = elem<T>(row, i);
-    if (fkey(x) >= theta && x != -INFINITY) {
-      s += ex2(specverify::arg2(x, c_hi, c_lo, o));
-      ++kept;
+  float margin = INFINITY;
+  double Z_kept = -1.0;  // from the candidates when they hold the kept set
+  double nk = -1.0;
+  if (nc >= 0 && (k_in_cands || use_p)) {
+    // (no entry equals `above` when every entry is a candidate: it may then
+    // be a key that decodes to no finite value)
+    const float xv = key_value(above);
+    const double w_above = (n_eq > 0.0 && xv != -INFINITY) ? exp2(static_cast<double>(xv) * c - od) : 0.0;
+    CandSet cs{cand_key, cand_w, nc, above, n_eq, w_above, tail, kmax, step};
+    if (nc <= kWarpCands) {
+      if (threadIdx.x < kWarp)
+        cand_stage(Red<true>{smd}, cs, k_in_cands, P.top_k, use_p, P.top_p, theta, &s_st);
+    } else {
+      cand_stage(Red<false>{smd}, cs, k_in_cands, P.top_k, use_p, P.top_p, theta, &s_st);
+    }
+    __syncthreads();
+    const StageOut st = s_st;
+    theta = st.theta;
+    if (st.below) {
+      // the nucleus boundary lies below the candidates: whole-row passes
+      // over [theta, boundary of the candidates) with fp32 weights
+      const double sc = exp2(static_cast<double>(o) - od);
+      const double goal = st.goal, Zk = st.Zk;
+      unsigned lo = theta, hi = max(theta, above);
+      while (lo < hi) {
+        const unsigned mid = lo + (((hi - lo) / step + 1) / 2) * step;
+        if (masked_mass<T, kAligned>(row, V, mid, c_hi, c_lo, o, smd) * sc >= goal) lo = mid;
+        else hi = mid - step;
+      }
+      const double m_ge = masked_mass<T, kAligned>(row, V, lo, c_hi, c_lo, o, smd) * sc;
+      const double m_gt = masked_mass<T, kAligned>(row, V, lo + step, c_hi, c_lo, o, smd) * sc;
+      margin = static_cast<float>(fmin(P.top_p - m_gt / Zk, m_ge / Zk - P.top_p));
+      theta = lo;
+      Z_kept = m_ge;
+    } else {
+      margin = st.margin;
+      if (st.z_valid) Z_kept = st.Z;
+      if (st.kept_valid) nk = st.kept;
     }
   }
-  const double Zs = block_sum<kSelThreads>(static_cast<double>(s), smd);
-  const double nk = block_sum<kSelThreads>(static_cast<double>(kept), smd);
+
+  // log-normaliser and size of the kept set, when the candidates do not hold it
+  double Z = Z_kept;
+  if (nk < 0.0) {
+    float sf = 0.f;
+    int kept = 0;
+    scan_row<T, kAligned, false>(row, V, [&](float x, long) {
+      if (fkey(x) >= theta && x != -INFINITY) {
+        sf += ex2(specverify::arg2(x, c_hi, c_lo, o));
+        ++kept;
+      }
+    });
+    const double zs = block_sum<kSelThreads>(static_cast<double>(sf), smd) * exp2(static_cast<double>(o) - od);
+    nk = block_sum<kSelThreads>(static_cast<double>(kept), smd);
+    if (Z < 0.0) Z = zs;
+  }
   if (threadIdx.x == 0) {
-    // log2 sum 2^(x c): from the double-precision candidate masses when the
-    // nucleus ends among them, else from this pass
-    out.l2 = z_known ? static_cast<double>(gmx) * c + log2(Z_kept) : static_cast<double>(o) + log2(Zs);
+    // log2 sum 2^(x c): the double-precision candidate masses where they hold
+    // the kept set, else the streaming pass
+    out.l2 = od + log2(Z);
     out.theta = theta;
     out.kept = static_cast<int>(nk);
     out.margin = margin;

@@ -24,12 +24,13 @@ struct specfold_gate_ctx {
   int device = 0;
   int branches = 0, positions = 0, dim = 0;
   long rows = 0;
-  int blocks = 0;
+  int blocks = 0;       // difference kernel (persistent)
+  int pack_blocks = 0;  // packing kernel
   sv_dtype dtype = SV_DTYPE_F32;
   void* ws = nullptr;
   int32_t* eff_parent = nullptr;
   uint8_t* flag = nullptr;
-  uint8_t* rank = nullptr;
+  int32_t* rank = nullptr;
   int32_t* prov = nullptr;
   int32_t* block_count = nullptr;
   int32_t* block_offset = nullptr;
@@ -47,12 +48,12 @@ size_t gate_elem_size(sv_dtype d) { return d == SV_DTYPE_BF16 ? 2 : 4; }
 bool gate_aligned(const void* p, size_t a) { return reinterpret_cast<uintptr_t>(p) % a == 0; }
 
 template <typename K>
-cudaError_t launch_pdl(K kernel, unsigned grid, unsigned block, cudaStream_t s,
+cudaError_t launch_pdl(K kernel, unsigned grid, unsigned block, size_t smem, cudaStream_t s,
                        const GateParams& p) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(block);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -71,11 +72,11 @@ cudaError_t launch_pass(const GateParams& p, cudaStream_t s, cudaEvent_t* ev) {
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[0], s);
   if (e == cudaSuccess)
     e = launch_pdl(specfold::rows_kernel<T, A>, static_cast<unsigned>(p.blocks),
-                   specfold::kThreads, s, p);
+                   specfold::kThreads, A ? specfold::kRowsSmem : 0, s, p);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
   if (e == cudaSuccess)
-    e = launch_pdl(specfold::pack_kernel<T, A>, static_cast<unsigned>(p.blocks),
-                   specfold::kThreads, s, p);
+    e = launch_pdl(specfold::pack_kernel<T, A>, static_cast<unsigned>(p.pack_blocks),
+                   specfold::kThreads, 0, s, p);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
   return e;
 }
@@ -118,8 +119,28 @@ sv_status specfold_gate_create(specfold_gate_t* out, int branches, int positions
   h->positions = positions;
   h->dim = dim;
   h->rows = rows;
-  h->blocks = static_cast<int>((rows + specfold::kRowsPerBlock - 1) / specfold::kRowsPerBlock);
+  h->pack_blocks = static_cast<int>((rows + specfold::kRowsPerBlock - 1) / specfold::kRowsPerBlock);
   h->dtype = dtype;
+  // the difference kernel is persistent: as many blocks as fit on the GPU at
+  // once (its cp.async ring sets the limit), never more than there are rows
+  {
+    int sms = 0, occ = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+    const void* k = (dtype == SV_DTYPE_BF16)
+                        ? reinterpret_cast<const void*>(specfold::rows_kernel<__nv_bfloat16, true>)
+                        : reinterpret_cast<const void*>(specfold::rows_kernel<float, true>);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, specfold::kRowsSmem);
+    if (e == cudaSuccess)
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, specfold::kThreads,
+                                                        specfold::kRowsSmem);
+    if (e != cudaSuccess) {
+      delete h;
+      return cuda_fail(e);
+    }
+    const long want = static_cast<long>(sms) * (occ > 0 ? occ : 1);
+    h->blocks = static_cast<int>(want < rows ? want : rows);
+  }
 
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -129,7 +150,7 @@ sv_status specfold_gate_create(specfold_gate_t* out, int branches, int positions
   };
   const size_t oE = take(sizeof(int32_t) * branches);
   const size_t oF = take(static_cast<size_t>(rows));
-  const size_t oR = take(static_cast<size_t>(rows));
+  const size_t oR = take(sizeof(int32_t) * rows);
   const size_t oP = take(sizeof(int32_t) * rows);
   const size_t oC = take(sizeof(int32_t) * h->blocks);
   const size_t oO = take(sizeof(int32_t) * h->blocks);
@@ -143,7 +164,7 @@ sv_status specfold_gate_create(specfold_gate_t* out, int branches, int positions
   char* b = static_cast<char*>(h->ws);
   h->eff_parent = reinterpret_cast<int32_t*>(b + oE);
   h->flag = reinterpret_cast<uint8_t*>(b + oF);
-  h->rank = reinterpret_cast<uint8_t*>(b + oR);
+  h->rank = reinterpret_cast<int32_t*>(b + oR);
   h->prov = reinterpret_cast<int32_t*>(b + oP);
   h->block_count = reinterpret_cast<int32_t*>(b + oC);
   h->block_offset = reinterpret_cast<int32_t*>(b + oO);
@@ -188,6 +209,7 @@ sv_status specfold_gate_run(specfold_gate_t h, const void* hidden, const int32_t
   p.dim = h->dim;
   p.rows = h->rows;
   p.blocks = h->blocks;
+  p.pack_blocks = h->pack_blocks;
   p.rel_diff = rel_diff;
   p.provenance = provenance;
   p.source = source;

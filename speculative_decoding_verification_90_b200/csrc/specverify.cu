@@ -178,6 +178,30 @@ cudaError_t launch_dtype(const Params& p, int NT, bool aligned, cudaStream_t s, 
 
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// the sampling-variant step: select (one block per row), decide, draw
+// events (may be null): before select, after select, after draw
+template <typename T, bool A>
+cudaError_t launch_sampling(const specsamp::SampParams& p, long rows, int per, cudaStream_t s,
+                            cudaEvent_t* ev) {
+  cudaError_t e = cudaFuncSetAttribute(specsamp::select_kernel<T, A>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       specsamp::kCandSmem);
+  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[0], s);
+  if (e != cudaSuccess) return e;
+  specsamp::select_kernel<T, A>
+      <<<static_cast<unsigned>(rows), specsamp::kSelThreads, specsamp::kCandSmem, s>>>(p);
+  e = cudaGetLastError();
+  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
+  if (e == cudaSuccess)
+    e = launch_pdl(specsamp::decide_kernel<T>, static_cast<unsigned>((p.batch + per - 1) / per),
+                   specsamp::kDecideThreads, s, p);
+  if (e == cudaSuccess)
+    e = launch_pdl(specsamp::draw_kernel<T>, static_cast<unsigned>(p.batch),
+                   specsamp::kDrawThreads, s, p);
+  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
+  return e;
+}
+
 // Row maps null: the logit buffers hold one row per position, [B, G+1, V] and
 // [B, G, V].  Otherwise `target_rows` / `draft_rows` rows that the maps index.
 sv_status enqueue(specverify_t h, const void* target, const void* draft, const int32_t* tokens,
@@ -408,33 +432,16 @@ sv_status specverify_run_sampling(specverify_t h, const void* target_logits,
   const long rows = static_cast<long>(h->batch) * (2L * G + 1);
   const int per = specsamp::kDecideThreads / specsamp::kWarp;
   cudaError_t e;
-  if (h->dtype == SV_DTYPE_BF16) {
-    e = cudaFuncSetAttribute(specsamp::select_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, specsamp::kCandSmem);
-    if (e != cudaSuccess) return cuda_fail(e);
-    specsamp::select_kernel<__nv_bfloat16>
-        <<<static_cast<unsigned>(rows), specsamp::kSelThreads, specsamp::kCandSmem, s>>>(p);
-    e = cudaGetLastError();
-    if (e == cudaSuccess)
-      e = launch_pdl(specsamp::decide_kernel<__nv_bfloat16>,
-                     static_cast<unsigned>((h->batch + per - 1) / per), specsamp::kDecideThreads, s, p);
-    if (e == cudaSuccess)
-      e = launch_pdl(specsamp::draw_kernel<__nv_bfloat16>, static_cast<unsigned>(h->batch),
-                     specsamp::kDrawThreads, s, p);
-  } else {
-    e = cudaFuncSetAttribute(specsamp::select_kernel<float>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, specsamp::kCandSmem);
-    if (e != cudaSuccess) return cuda_fail(e);
-    specsamp::select_kernel<float>
-        <<<static_cast<unsigned>(rows), specsamp::kSelThreads, specsamp::kCandSmem, s>>>(p);
-    e = cudaGetLastError();
-    if (e == cudaSuccess)
-      e = launch_pdl(specsamp::decide_kernel<float>,
-                     static_cast<unsigned>((h->batch + per - 1) / per), specsamp::kDecideThreads, s, p);
-    if (e == cudaSuccess)
-      e = launch_pdl(specsamp::draw_kernel<float>, static_cast<unsigned>(h->batch),
-                     specsamp::kDrawThreads, s, p);
-  }
+  const bool aligned = aligned_to(target_logits, 16) && (G == 0 || aligned_to(draft_logits, 16)) &&
+                       (static_cast<size_t>(h->vocab) * es) % 16 == 0;
+  cudaEvent_t* ev = nullptr;
+  if (h->prof_runs < h->prof_capacity) ev = h->events.data() + 3 * (h->prof_runs++);
+  if (h->dtype == SV_DTYPE_BF16)
+    e = aligned ? launch_sampling<__nv_bfloat16, true>(p, rows, per, s, ev)
+                : launch_sampling<__nv_bfloat16, false>(p, rows, per, s, ev);
+  else
+    e = aligned ? launch_sampling<float, true>(p, rows, per, s, ev)
+                : launch_sampling<float, false>(p, rows, per, s, ev);
   if (e != cudaSuccess) return cuda_fail(e);
   return SV_OK;
 }
