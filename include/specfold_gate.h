@@ -34,7 +34,7 @@
  *
  * Memory: the caller owns every input and output.  A handle owns a small
  * device workspace (per-branch validated parents, per-row flags, provenance
- * and ranks, per-block counts, a ticket, a status word).  Errors: argument
+ * and packed slots, a status word).  Errors: argument
  * errors return before anything is enqueued; a bad parent array never traps:
  * it sets status bit 1, read (and cleared) by specfold_gate_get_status.
  */
@@ -91,7 +91,8 @@ sv_status specfold_gate_get_status(specfold_gate_t h, void *stream, uint32_t *bi
 sv_status specfold_gate_profile_begin(specfold_gate_t h, int max_runs);
 
 /* Wait for the recorded runs and return the mean device milliseconds per run
- * of the difference kernel (`rows_ms`) and of the packing kernel (`pack_ms`),
+ * of the difference kernel (`rows_ms`) and of the slot scan plus the packing
+ * kernel (`pack_ms`),
  * and the number of runs averaged. */
 sv_status specfold_gate_profile_end(specfold_gate_t h, float *rows_ms, float *pack_ms, int *runs);
 

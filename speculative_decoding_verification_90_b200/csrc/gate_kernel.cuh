@@ -6,20 +6,19 @@
 // above tau from all branches are packed into one batch), the implementer's
 // note (the gate records provenance; a resolution step follows fold chains).
 //
-// Three stream-ordered kernels per pass:
+// Four stream-ordered kernels per pass:
 //   tree_kernel  one block: validates every branch's parent chain by pointer
 //                jumping in shared memory;
-//   rows_kernel  persistent blocks over contiguous row ranges; each warp
-//                streams its rows' H[c, j] and H[parent, j] through a ring of
-//                cp.async stages, sums squares in fp32 per lane and fp64
-//                across the warp, and decides recompute = !(d <= tau); the
-//                block ranks its recomputed rows, and the block that takes
-//                the last ticket turns the per-block counts into offsets;
+//   rows_kernel  persistent warps, global warp w taking rows w, w + W, ...;
+//                each warp streams its rows' H[c, j] and H[parent, j] through
+//                a ring of cp.async stages, sums squares in fp32 per lane and
+//                fp64 across the warp, and decides recompute = !(d <= tau);
+//   scan_kernel  one block: the packed slot of every recomputed row (an
+//                exclusive prefix sum of the flags) and their count;
 //   pack_kernel  one warp per row: writes the packed row index, follows the
 //                fold chain to the source row, copies recomputed rows into the
 //                packed batch.
-// The only hand-off inside a kernel is the ticket (the last arriver proceeds);
-// nothing waits on another block.
+// Nothing waits on another block inside a kernel.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -33,7 +32,6 @@ constexpr int kRowsPerBlock = 8;  // one warp per row
 constexpr int kThreads = kRowsPerBlock * kWarp;
 constexpr int kTreeThreads = 1024;
 constexpr int kMaxBranches = 16384;
-constexpr int kScanThreads = kThreads;
 
 enum : unsigned { kStatParent = 1u };
 
@@ -43,7 +41,7 @@ struct GateParams {
   double tau;
   int branches, positions, dim;
   long rows;
-  int blocks;               // rows_kernel grid (persistent; each block a contiguous row range)
+  int blocks;               // rows_kernel grid (persistent warps)
   int pack_blocks;          // pack_kernel grid (8 rows per block)
   // outputs (rel_diff, provenance, source, packed_hidden may be null)
   float* rel_diff;
@@ -55,11 +53,8 @@ struct GateParams {
   // workspace
   int32_t* eff_parent;      // [branches] parent after validation, -1 if none
   uint8_t* flag;            // [rows] 1: recompute
-  int32_t* rank;            // [rows] rank among the recomputed rows of its block
+  int32_t* rank;            // [rows] packed slot of each recomputed row
   int32_t* prov;            // [rows] provenance (always kept for the chain walk)
-  int32_t* block_count;     // [blocks]
-  int32_t* block_offset;    // [blocks]
-  unsigned* ticket;
   unsigned* status;
 };
 
@@ -166,16 +161,6 @@ constexpr int kStages = 8;  // cp.async stages in flight per warp
 constexpr int kStageBytes = kWarp * 32;  // one 16-byte group of child and parent per lane
 constexpr int kRowsSmem = kStages * kStageBytes * (kThreads / kWarp);
 
-// rows of block b: [row_start(b), row_start(b + 1))
-__device__ __forceinline__ long row_start(long b, long rows, int nblk) { return b * rows / nblk; }
-
-__device__ __forceinline__ int block_of(long row, long rows, int nblk) {
-  long b = row * nblk / rows;
-  while (b + 1 < nblk && row_start(b + 1, rows, nblk) <= row) ++b;
-  while (b > 0 && row_start(b, rows, nblk) > row) --b;
-  return static_cast<int>(b);
-}
-
 __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
   const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem));
   const int n = valid ? 16 : 0;  // 0: fill with zeros, read nothing
@@ -200,31 +185,30 @@ __device__ __forceinline__ bool finish_row(const GateParams& P, long row, int pa
   return rec;
 }
 
-// One persistent block per slot: block b owns the contiguous rows
-// [row_start(b), row_start(b + 1)); warp w takes every 8th of them.  With
-// 128-bit rows a warp streams its rows' (child, parent) groups through a ring
-// of kStages cp.async stages in shared memory, so loads stay in flight across
-// row boundaries without holding registers.
+// Persistent warps: global warp w takes rows w, w + W, w + 2W, ... (W warps
+// in the grid), so all warps move through the tensor together and a parent
+// row, a few hundred rows before its children, is still in L2 when they read
+// it.  With 128-bit rows a warp streams its rows' (child, parent) groups
+// through a ring of kStages cp.async stages in shared memory, so loads stay in
+// flight across row boundaries without holding registers.
 template <typename T, bool kAligned>
 __global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
   extern __shared__ uint4 ring[];  // [warps][kStages][2][kWarp]
-  __shared__ bool s_last;
-  __shared__ int s_count;
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x & (kWarp - 1);
-  const long r0 = row_start(blockIdx.x, P.rows, P.blocks);
-  const long r1 = row_start(blockIdx.x + 1, P.rows, P.blocks);
+  const long W = static_cast<long>(gridDim.x) * (kThreads / kWarp);
+  const long r0 = static_cast<long>(blockIdx.x) * (kThreads / kWarp) + warp;
+  const long r1 = P.rows;
   const T* base = static_cast<const T*>(P.hidden);
   cudaGridDependencySynchronize();  // validated parents
 
-  // rows of this warp: r0 + warp, r0 + warp + 8, ...; those without a parent
-  // are decided without reading anything
+  // rows without a parent are decided without reading anything
   auto parent_of = [&](long row) -> int { return P.eff_parent[row / P.positions]; };
   if (lane == 0)
-    for (long row = r0 + warp; row < r1; row += kRowsPerBlock)
+    for (long row = r0; row < r1; row += W)
       if (parent_of(row) < 0) finish_row(P, row, -1, 0, 0.0, 0.0);
   // next row at or after `row` (in this warp's sequence) that has a parent
   auto next_row = [&](long row) -> long {
-    while (row < r1 && parent_of(row) < 0) row += kRowsPerBlock;
+    while (row < r1 && parent_of(row) < 0) row += W;
     return row;
   };
 
@@ -235,7 +219,7 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
     uint4* my = ring + static_cast<long>(warp) * kStages * 2 * kWarp;
     // issue pointer: the row being fetched, its two group pointers (this
     // lane's group of chunk 0) and the chunk; all set once per row
-    long irow = next_row(r0 + warp);
+    long irow = next_row(r0);
     int ichunk = 0;
     const uint4* igc = nullptr;  // this lane's next group of the child row
     const uint4* igp = nullptr;  // and of the parent row
@@ -264,7 +248,7 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
         if (++ichunk == chunks) {
           ichunk = 0;
           g_left = groups - lane;
-          irow = next_row(irow + kRowsPerBlock);
+          irow = next_row(irow + W);
           set_issue_row();
         }
       }
@@ -272,7 +256,7 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
     };
 #pragma unroll 1
     for (int st = 0; st < kStages - 1; ++st) issue(st);
-    long crow = next_row(r0 + warp);
+    long crow = next_row(r0);
     int cchunk = 0, slot = 0;
     float d0 = 0.f, d1 = 0.f, n0 = 0.f, n1 = 0.f;
     while (crow < r1) {
@@ -294,12 +278,12 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
           finish_row(P, crow, parent_of(crow), static_cast<int>(crow % P.positions), num, den);
         d0 = d1 = n0 = n1 = 0.f;
         cchunk = 0;
-        crow = next_row(crow + kRowsPerBlock);
+        crow = next_row(crow + W);
       }
     }
     asm volatile("cp.async.wait_all;");
   } else {
-    for (long row = next_row(r0 + warp); row < r1; row = next_row(row + kRowsPerBlock)) {
+    for (long row = next_row(r0); row < r1; row = next_row(row + W)) {
       const int par = parent_of(row);
       const int j = static_cast<int>(row % P.positions);
       const T* hc = base + row * P.dim;
@@ -321,71 +305,53 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
     }
   }
 
-  // ranks of the recomputed rows inside the block, in row order
-  __syncthreads();
-  if (warp == 0) {
-    int running = 0;
-    for (long base_row = r0; base_row < r1; base_row += kWarp) {
-      const long row = base_row + lane;
-      const bool f = row < r1 && P.flag[row] != 0;
-      const unsigned m = __ballot_sync(0xffffffffu, f);
-      if (row < r1) P.rank[row] = running + __popc(m & ((1u << lane) - 1u));
-      running += __popc(m);
-    }
-    if (lane == 0) s_count = running;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    P.block_count[blockIdx.x] = s_count;
-    __threadfence();
-    // atomicInc wraps to 0 at the last block, so the ticket resets itself
-    s_last = atomicInc(P.ticket, static_cast<unsigned>(P.blocks - 1)) ==
-             static_cast<unsigned>(P.blocks - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-
-  // last block: exclusive prefix sum of the per-block counts
-  __threadfence();
-  __shared__ int32_t s_warp[kScanThreads / kWarp];
-  __shared__ int32_t s_carry;
-  if (threadIdx.x == 0) s_carry = 0;
-  __syncthreads();
-  for (int b0 = 0; b0 < P.blocks; b0 += kScanThreads) {
-    const int i = b0 + threadIdx.x;
-    const int v = (i < P.blocks) ? __ldcg(P.block_count + i) : 0;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < kWarp; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, o);
-      if (lane >= o) x += y;
-    }
-    if (lane == kWarp - 1) s_warp[warp] = x;
-    __syncthreads();
-    if (warp == 0) {
-      int w = (lane < kScanThreads / kWarp) ? s_warp[lane] : 0;
-#pragma unroll
-      for (int o = 1; o < kWarp; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, w, o);
-        if (lane >= o) w += y;
-      }
-      if (lane < kScanThreads / kWarp) s_warp[lane] = w;  // inclusive over warps
-    }
-    __syncthreads();
-    const int before = s_carry + (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
-    if (i < P.blocks) P.block_offset[i] = before;
-    __syncthreads();
-    if (threadIdx.x == 0) s_carry += s_warp[kScanThreads / kWarp - 1];
-    __syncthreads();
-  }
-  if (threadIdx.x == 0) *P.n_packed = s_carry;
 }
 
 // ---------------------------------------------------------------------------
-// kernel 3: packing and fold-chain resolution
+// kernel 3: the packed slots (one block): exclusive prefix sum of the flags
 // ---------------------------------------------------------------------------
 
-// one warp per row; the row's slot is its block's offset plus its rank
+// each thread owns a contiguous chunk of rows: its count, one block-wide
+// exclusive scan of the counts, then its slots in row order
+constexpr int kSlotThreads = 1024;
+
+__global__ void __launch_bounds__(kSlotThreads) scan_kernel(const GateParams P) {
+  __shared__ int32_t s_warp[kSlotThreads / kWarp];
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x & (kWarp - 1);
+  cudaGridDependencySynchronize();
+  const long chunk = (P.rows + kSlotThreads - 1) / kSlotThreads;
+  const long lo = min(P.rows, chunk * threadIdx.x), hi = min(P.rows, lo + chunk);
+  int v = 0;
+  for (long i = lo; i < hi; ++i) v += __ldcg(P.flag + i) != 0;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < kWarp; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == kWarp - 1) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = s_warp[lane];  // kSlotThreads / kWarp == kWarp warps
+#pragma unroll
+    for (int o = 1; o < kWarp; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    s_warp[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  int slot = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
+  for (long i = lo; i < hi; ++i)
+    if (__ldcg(P.flag + i) != 0) P.rank[i] = slot++;
+  if (threadIdx.x == kSlotThreads - 1) *P.n_packed = s_warp[kWarp - 1];
+}
+
+// ---------------------------------------------------------------------------
+// kernel 4: packing and fold-chain resolution
+// ---------------------------------------------------------------------------
+
+// one warp per row; the row's slot comes from the scan
 template <typename T, bool kAligned>
 __global__ void __launch_bounds__(kThreads) pack_kernel(const GateParams P) {
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x & (kWarp - 1);
@@ -394,9 +360,7 @@ __global__ void __launch_bounds__(kThreads) pack_kernel(const GateParams P) {
   if (row >= P.rows) return;
   const bool rec = __ldcg(P.flag + row) != 0;
   long slot = 0;
-  if (rec)
-    slot = static_cast<long>(__ldcg(P.block_offset + block_of(row, P.rows, P.blocks))) +
-           __ldcg(P.rank + row);
+  if (rec) slot = __ldcg(P.rank + row);
   if (lane == 0) {
     if (rec) P.packed[slot] = static_cast<int32_t>(row);
     if (P.source) {

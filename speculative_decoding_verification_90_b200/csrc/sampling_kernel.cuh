@@ -36,10 +36,11 @@ using specverify::Elem;
 using specverify::ex2;
 using specverify::kWarp;
 
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / kWarp;
-constexpr int kCand = 12288;         // top-p candidates kept in shared memory
+constexpr int kCand = 12288;         // most candidates kept in shared memory
 constexpr int kCandSmem = kCand * 8; // their keys and weights (dynamic shared memory)
+constexpr int kCandSmall = 2048;     // the candidate room of a call whose cuts need no more
 constexpr int kDrawThreads = 512;
 constexpr int kDecideThreads = 128;
 
@@ -88,6 +89,7 @@ struct SampParams {
   int batch, gamma, vocab;
   int top_k;                 // 0: off
   double top_p;              // >= 1: off
+  int cand_cap;              // candidates that fit in the launch's dynamic shared memory
 };
 
 // ---------------------------------------------------------------------------
@@ -317,6 +319,81 @@ __device__ unsigned radix_select(const T* row, int V, unsigned floor_key, long r
   return s_prefix;
 }
 
+// The nucleus cut below the candidates: the largest key v in [lo, hi) with
+// above + M(lo <= key, v <= key < hi) >= goal, where M sums the fp32 weights
+// 2^(x c - o).  An 8-bit digit descent over the key with per-warp mass
+// histograms in shared memory (one pass per digit).  Returns v, and the masses
+// at or above v and strictly above v (both including `above`).
+template <typename T, bool kAligned>
+__device__ unsigned mass_descent(const T* row, int V, unsigned lo, unsigned hi, double above,
+                                 double goal, int low_bits, float c_hi, float c_lo, float o,
+                                 float* histw, double* m_ge, double* m_gt) {
+  const int warp = threadIdx.x >> 5;
+  __shared__ unsigned d_prefix, d_mask;
+  __shared__ double d_above, d_bin;
+  if (threadIdx.x == 0) {
+    d_prefix = 0u;
+    d_mask = 0u;
+    d_above = above;
+    d_bin = 0.0;
+  }
+  __syncthreads();
+  float* mine = histw + warp * 256;
+  for (int shift = 24; shift >= low_bits; shift -= 8) {
+    for (int i = threadIdx.x; i < 256 * kSelWarps; i += blockDim.x) histw[i] = 0.f;
+    __syncthreads();
+    const unsigned prefix = d_prefix, mask = d_mask;
+    scan_row<T, kAligned, false>(row, V, [&](float x, long) {
+      const unsigned k = fkey(x);
+      if (k >= lo && k < hi && (k & mask) == prefix)
+        atomicAdd(&mine[(k >> shift) & 255u], ex2(specverify::arg2(x, c_hi, c_lo, o)));
+    });
+    __syncthreads();
+    if (threadIdx.x < kWarp) {
+      // bins from the top down, 32 at a time: the first whose cumulative mass
+      // (after everything above it) reaches the goal
+      const int lane = threadIdx.x;
+      double cum = d_above;
+      int sel = -1;
+      double sel_mass = 0.0;
+      for (int base = 255; base >= 0 && sel < 0; base -= kWarp) {
+        const int bin = base - lane;
+        double m = 0.0;
+        for (int w = 0; w < kSelWarps; ++w) m += static_cast<double>(histw[w * 256 + bin]);
+        double incl = m;
+#pragma unroll
+        for (int off = 1; off < kWarp; off <<= 1) {
+          const double y = __shfl_up_sync(0xffffffffu, incl, off);
+          if (lane >= off) incl += y;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, cum + incl >= goal);
+        if (hit) {
+          const int l = __ffs(hit) - 1;
+          sel = base - l;
+          sel_mass = __shfl_sync(0xffffffffu, m, l);
+          cum += __shfl_sync(0xffffffffu, incl - m, l);
+        } else {
+          cum += __shfl_sync(0xffffffffu, incl, kWarp - 1);
+        }
+      }
+      if (lane == 0) {
+        if (sel < 0) {  // rounding: the goal is not reached; take the lowest bin
+          sel = 0;
+          sel_mass = 0.0;
+        }
+        d_above = cum;
+        d_bin = sel_mass;
+        d_prefix = prefix | (static_cast<unsigned>(sel) << shift);
+        d_mask = mask | (255u << shift);
+      }
+    }
+    __syncthreads();
+  }
+  *m_gt = d_above;
+  *m_ge = d_above + d_bin;
+  return d_prefix;
+}
+
 // sum over the row of 2^(x c - o) for entries with key >= lo, per thread in
 // fp32, over the block in fp64
 template <typename T, bool kAligned>
@@ -347,7 +424,7 @@ __device__ __forceinline__ void put_row(const SampParams& P, long r, long nT, co
 template <typename T, bool kAligned, bool kTail>
 __device__ int gather(const T* row, int V, unsigned above, unsigned floor_key, double c, double od,
                       unsigned* cand_key, float* cand_w, int* cand_n, float c_hi, float c_lo,
-                      float o, double* sm, double* n_eq_out, double* tail_out) {
+                      float o, double* sm, double* n_eq_out, double* tail_out, int cap) {
   const int lane = threadIdx.x & (kWarp - 1);
   if (threadIdx.x == 0) *cand_n = 0;
   __syncthreads();
@@ -366,7 +443,7 @@ __device__ int gather(const T* row, int V, unsigned above, unsigned floor_key, d
       at = __shfl_sync(0xffffffffu, at, __ffs(m) - 1);
       if (take) {
         const int slot = at + __popc(m & ((1u << lane) - 1u));
-        if (slot < kCand) cand_key[slot] = k;
+        if (slot < cap) cand_key[slot] = k;
       }
     }
   });
@@ -374,7 +451,7 @@ __device__ int gather(const T* row, int V, unsigned above, unsigned floor_key, d
   const int n = *cand_n;
   // the candidates' weights in double precision (rounded to float), after the
   // scan so that no lane waits on another's exp2
-  for (int i = threadIdx.x; i < min(n, kCand); i += blockDim.x)
+  for (int i = threadIdx.x; i < min(n, cap); i += blockDim.x)
     cand_w[i] = static_cast<float>(exp2(static_cast<double>(key_value(cand_key[i])) * c - od));
   *n_eq_out = block_sum<kSelThreads>(static_cast<double>(n_eq), sm);
   *tail_out = block_sum<kSelThreads>(static_cast<double>(tail), sm) * exp2(static_cast<double>(o) - od);
@@ -410,7 +487,7 @@ struct StageOut {
   unsigned theta;
   float margin;
   double Z, kept;   // mass (when z_valid) and count (when kept_valid) of the kept set
-  double Zk, goal;  // for the whole-row fallback, when below
+  double Zk, goal, m0;  // for the whole-row fallback, when below
   int z_valid, kept_valid, below;
 };
 
@@ -442,7 +519,7 @@ __device__ void cand_stage(const Red<kW>& R, const CandSet& cs, bool do_k, int t
     if (v <= cs.above && cs.above >= theta) t += cs.n_eq * cs.w_above;
     return t;
   };
-  StageOut o{theta, INFINITY, 0.0, 0.0, 0.0, 0.0, 0, 0, 0};
+  StageOut o{theta, INFINITY, 0.0, 0.0, 0.0, 0.0, 0.0, 0, 0, 0};
   if (do_p) {
     const unsigned v0 = max(theta, cs.above);
     const double m0 = mass_ge(v0);
@@ -450,6 +527,7 @@ __device__ void cand_stage(const Red<kW>& R, const CandSet& cs, bool do_k, int t
     const double goal = top_p * Zk;
     o.Zk = Zk;
     o.goal = goal;
+    o.m0 = m0;
     if (m0 >= goal) {
       unsigned lo = v0, hi = cs.kmax;
       while (lo < hi) {
@@ -583,14 +661,15 @@ __device__ __forceinline__ PassA pass_a(const T* row, int V, float c_hi, float c
 }
 
 template <typename T, bool kAligned>
-__global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SampParams P) {
+__global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams P) {
   __shared__ double smd[kSelWarps];
   __shared__ unsigned smu[kSelWarps];
   __shared__ int smi[kSelWarps];
   __shared__ unsigned s_tmax[kSelThreads];
-  extern __shared__ unsigned cand_smem[];  // kCand keys, then kCand weights
+  extern __shared__ unsigned cand_smem[];  // cap keys, then cap weights
+  const int kCap = P.cand_cap;
   unsigned* cand_key = cand_smem;
-  float* cand_w = reinterpret_cast<float*>(cand_smem + kCand);
+  float* cand_w = reinterpret_cast<float*>(cand_smem + kCap);
   // the radix select's per-warp histograms reuse the candidate area: every
   // radix select runs before the candidates it serves are gathered
   int* hist = reinterpret_cast<int*>(cand_smem);
@@ -727,7 +806,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SampParams
     // gathered whole.  Warp 0 searches the kSelThreads maxima.
     __shared__ unsigned s_lb;
     if (threadIdx.x < kWarp) {
-      unsigned lo = 0u, hi = (V > kCand) ? kmax : 0u;
+      unsigned lo = 0u, hi = (V > kCap) ? kmax : 0u;
       while (lo < hi) {
         const unsigned mid = lo + (((hi - lo) / step + 1) / 2) * step;
         int cnt = 0;
@@ -741,8 +820,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SampParams
     const unsigned lb = s_lb;
     const unsigned lb_floor = lb > 0u ? lb - 1u : 0u;  // gather keys >= lb
     const int n = gather<T, kAligned, false>(row, V, lb_floor, 0u, c, od, cand_key, cand_w, &cand_n,
-                                             c_hi, c_lo, o, smd, &n_eq, &tail);
-    if (n <= kCand) {
+                                             c_hi, c_lo, o, smd, &n_eq, &tail, kCap);
+    if (n <= kCap) {
       nc = n;
       above = lb_floor;
       theta = lb;    // raised to the k-th largest candidate below
@@ -754,7 +833,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SampParams
   const bool k_in_cands = use_k && nc >= 0;
 
   if (use_p && nc < 0) {
-    // candidate key: the kCand-th largest key >= theta (theta itself when
+    // candidate key: the kCap-th largest key >= theta (theta itself when
     // fewer entries are kept)
     unsigned vc = theta;
     double nd = V;  // without a top-k cut every entry is >= theta = 0
@@ -764,10 +843,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SampParams
       nd = block_sum<kSelThreads>(static_cast<double>(n_ge), smd);
     }
     int eq_c = 0;
-    if (nd > kCand) vc = radix_select<T, kAligned>(row, V, theta, kCand, low_bits, hist, &eq_c);
+    if (nd > kCap) vc = radix_select<T, kAligned>(row, V, theta, kCap, low_bits, hist, &eq_c);
     nc = min(gather<T, kAligned, true>(row, V, vc, theta, c, od, cand_key, cand_w, &cand_n, c_hi,
-                                       c_lo, o, smd, &n_eq, &tail),
-             kCand);
+                                       c_lo, o, smd, &n_eq, &tail, kCap),
+             kCap);
     above = vc;
   }
 
@@ -790,18 +869,18 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_kernel(const SampParams
     const StageOut st = s_st;
     theta = st.theta;
     if (st.below) {
-      // the nucleus boundary lies below the candidates: whole-row passes
-      // over [theta, boundary of the candidates) with fp32 weights
+      // the nucleus boundary lies below the candidates: a mass descent over
+      // the keys in [theta, v0), everything at or above v0 (mass m0) counted
+      // (fp32 weights relative to o; the candidates' room holds the histograms)
       const double sc = exp2(static_cast<double>(o) - od);
-      const double goal = st.goal, Zk = st.Zk;
-      unsigned lo = theta, hi = max(theta, above);
-      while (lo < hi) {
-        const unsigned mid = lo + (((hi - lo) / step + 1) / 2) * step;
-        if (masked_mass<T, kAligned>(row, V, mid, c_hi, c_lo, o, smd) * sc >= goal) lo = mid;
-        else hi = mid - step;
-      }
-      const double m_ge = masked_mass<T, kAligned>(row, V, lo, c_hi, c_lo, o, smd) * sc;
-      const double m_gt = masked_mass<T, kAligned>(row, V, lo + step, c_hi, c_lo, o, smd) * sc;
+      const double Zk = st.Zk;
+      const unsigned v0 = max(theta, above);
+      double m_ge, m_gt;
+      const unsigned lo = mass_descent<T, kAligned>(
+          row, V, theta, v0, st.m0 / sc, st.goal / sc, low_bits, c_hi, c_lo, o,
+          reinterpret_cast<float*>(cand_smem), &m_ge, &m_gt);
+      m_ge *= sc;
+      m_gt *= sc;
       margin = static_cast<float>(fmin(P.top_p - m_gt / Zk, m_ge / Zk - P.top_p));
       theta = lo;
       Z_kept = m_ge;

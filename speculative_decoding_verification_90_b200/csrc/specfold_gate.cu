@@ -32,9 +32,6 @@ struct specfold_gate_ctx {
   uint8_t* flag = nullptr;
   int32_t* rank = nullptr;
   int32_t* prov = nullptr;
-  int32_t* block_count = nullptr;
-  int32_t* block_offset = nullptr;
-  unsigned* ticket = nullptr;
   unsigned* status = nullptr;
   // optional timing: 3 events per recorded run (before rows, after rows, after pack)
   std::vector<cudaEvent_t> events;
@@ -74,6 +71,8 @@ cudaError_t launch_pass(const GateParams& p, cudaStream_t s, cudaEvent_t* ev) {
     e = launch_pdl(specfold::rows_kernel<T, A>, static_cast<unsigned>(p.blocks),
                    specfold::kThreads, A ? specfold::kRowsSmem : 0, s, p);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
+  if (e == cudaSuccess)
+    e = launch_pdl(specfold::scan_kernel, 1u, specfold::kSlotThreads, 0, s, p);
   if (e == cudaSuccess)
     e = launch_pdl(specfold::pack_kernel<T, A>, static_cast<unsigned>(p.pack_blocks),
                    specfold::kThreads, 0, s, p);
@@ -152,9 +151,6 @@ sv_status specfold_gate_create(specfold_gate_t* out, int branches, int positions
   const size_t oF = take(static_cast<size_t>(rows));
   const size_t oR = take(sizeof(int32_t) * rows);
   const size_t oP = take(sizeof(int32_t) * rows);
-  const size_t oC = take(sizeof(int32_t) * h->blocks);
-  const size_t oO = take(sizeof(int32_t) * h->blocks);
-  const size_t oT = take(sizeof(unsigned));
   const size_t oS = take(sizeof(unsigned));
   e = cudaMalloc(&h->ws, off);
   if (e != cudaSuccess) {
@@ -166,9 +162,6 @@ sv_status specfold_gate_create(specfold_gate_t* out, int branches, int positions
   h->flag = reinterpret_cast<uint8_t*>(b + oF);
   h->rank = reinterpret_cast<int32_t*>(b + oR);
   h->prov = reinterpret_cast<int32_t*>(b + oP);
-  h->block_count = reinterpret_cast<int32_t*>(b + oC);
-  h->block_offset = reinterpret_cast<int32_t*>(b + oO);
-  h->ticket = reinterpret_cast<unsigned*>(b + oT);
   h->status = reinterpret_cast<unsigned*>(b + oS);
   // the attribute is per function, shared by all handles: allow the largest tree
   e = cudaFuncSetAttribute(specfold::tree_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -220,9 +213,6 @@ sv_status specfold_gate_run(specfold_gate_t h, const void* hidden, const int32_t
   p.flag = h->flag;
   p.rank = h->rank;
   p.prov = h->prov;
-  p.block_count = h->block_count;
-  p.block_offset = h->block_offset;
-  p.ticket = h->ticket;
   p.status = h->status;
 
   const bool aligned = gate_aligned(hidden, 16) && (!packed_hidden || gate_aligned(packed_hidden, 16)) &&

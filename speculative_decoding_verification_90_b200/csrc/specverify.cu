@@ -188,8 +188,8 @@ cudaError_t launch_sampling(const specsamp::SampParams& p, long rows, int per, c
                                        specsamp::kCandSmem);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[0], s);
   if (e != cudaSuccess) return e;
-  specsamp::select_kernel<T, A>
-      <<<static_cast<unsigned>(rows), specsamp::kSelThreads, specsamp::kCandSmem, s>>>(p);
+  specsamp::select_kernel<T, A><<<static_cast<unsigned>(rows), specsamp::kSelThreads,
+                                  static_cast<size_t>(p.cand_cap) * 8, s>>>(p);
   e = cudaGetLastError();
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
   if (e == cudaSuccess)
@@ -428,6 +428,10 @@ sv_status specverify_run_sampling(specverify_t h, const void* target_logits,
   p.vocab = h->vocab;
   p.top_k = (top_k >= h->vocab) ? 0 : top_k;
   p.top_p = (top_p >= 1.f) ? 1.0 : static_cast<double>(top_p);
+  // a nucleus cut outside a small top-k set needs the large candidate room
+  // (fewer blocks per SM); every other setting fits in the small one
+  const bool small_k = p.top_k > 0 && p.top_k <= specsamp::kSelThreads;
+  p.cand_cap = (p.top_p < 1.0 && !small_k) ? specsamp::kCand : specsamp::kCandSmall;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long rows = static_cast<long>(h->batch) * (2L * G + 1);
   const int per = specsamp::kDecideThreads / specsamp::kWarp;
