@@ -319,10 +319,19 @@ __global__ void __launch_bounds__(kSlotThreads) scan_kernel(const GateParams P) 
   __shared__ int32_t s_warp[kSlotThreads / kWarp];
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x & (kWarp - 1);
   cudaGridDependencySynchronize();
-  const long chunk = (P.rows + kSlotThreads - 1) / kSlotThreads;
+  // chunks of a multiple of 4 rows: the flags are read four per 32-bit load
+  // (the flag array is 256-byte aligned and padded to a multiple of 4)
+  const long chunk = ((P.rows + kSlotThreads - 1) / kSlotThreads + 3) & ~3L;
   const long lo = min(P.rows, chunk * threadIdx.x), hi = min(P.rows, lo + chunk);
   int v = 0;
-  for (long i = lo; i < hi; ++i) v += __ldcg(P.flag + i) != 0;
+  for (long i = lo; i < hi; i += 4) {
+    const unsigned w = __ldcg(reinterpret_cast<const unsigned*>(P.flag + i));
+    // bytes past `hi` (the next chunk's rows, or padding past the last row)
+    // are masked off
+    const long left = hi - i;
+    const unsigned keep = left >= 4 ? 0xffffffffu : ((1u << (8 * left)) - 1u);
+    v += __popc(w & keep & 0x01010101u);
+  }
   int x = v;
 #pragma unroll
   for (int o = 1; o < kWarp; o <<= 1) {

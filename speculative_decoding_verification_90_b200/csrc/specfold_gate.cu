@@ -148,7 +148,7 @@ sv_status specfold_gate_create(specfold_gate_t* out, int branches, int positions
     return at;
   };
   const size_t oE = take(sizeof(int32_t) * branches);
-  const size_t oF = take(static_cast<size_t>(rows));
+  const size_t oF = take(static_cast<size_t>(rows) + 4);  // + padding for 4-byte reads
   const size_t oR = take(sizeof(int32_t) * rows);
   const size_t oP = take(sizeof(int32_t) * rows);
   const size_t oS = take(sizeof(unsigned));
