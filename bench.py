@@ -79,10 +79,15 @@ def parse():
 
 
 def kernel_hash() -> str:
+    """Hash of the statistics kernel's code: its part of the source, from the
+    streaming-statistics helpers through the kernel itself."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel)) as f:
+            text = f.read()
+        a = text.find("// phase 1: streaming softmax statistics")
+        b = text.find("// kernel 2:")
+        h.update(text[a:b].encode() if 0 <= a < b else text.encode())
     return h.hexdigest()[:16]
 
 

@@ -78,7 +78,8 @@ typedef enum {
   SV_WARN_ZERO_MASS = 18,  /* device: a residual had zero mass; drew from q_n instead */
   SV_ERR_ROW_INDEX = 19,   /* device: a row map entry was outside the rows given */
   SV_ERR_PARENT = 20,      /* device (fold gate): a parent entry out of range, a self link or a cycle */
-  SV_ERR_TEMPERATURE = 21  /* device (sampling variants): a temperature < 0, NaN or infinite */
+  SV_ERR_TEMPERATURE = 21, /* device (sampling variants): a temperature < 0, NaN or infinite */
+  SV_ERR_PIPELINE = 22     /* device (fused LM head): a tensor-core pipeline wait gave up */
 } sv_status;
 
 /*

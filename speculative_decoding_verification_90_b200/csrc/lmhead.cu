@@ -1,0 +1,531 @@
+// C ABI of the verification step fused with the LM head (see specverify_lmhead.h).
+//
+// Host side only: argument checks, the workspace, the TMA tensor maps, and the
+// stream-ordered launches of one step:
+//   1. statistics GEMMs (target rows, then draft rows): per-(row, vocabulary
+//      tile) softmax partials and the logits at the draft tokens;
+//   2. the decide kernel of the plain step on those partials;
+//   3. a gather of the two hidden rows each sequence draws from;
+//   4. logit GEMMs for those rows (fp32, [batch, vocab] each);
+//   5. the draw kernel of the plain step on them.
+#include "specverify_lmhead.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <new>
+#include <vector>
+
+#include "host_common.h"
+#include "lmhead_kernel.cuh"
+#include "verify_kernel.cuh"
+
+using specverify::Params;
+using specverify::PosInfo;
+using specverify::RowPartial;
+using specverify::RowStat;
+using specverify::SeqDecision;
+using svhost::cuda_fail;
+using svhost::DeviceScope;
+using svhost::g_last_error;
+using svhost::round_up;
+
+struct specverify_lmhead_ctx {
+  int device = 0;
+  int batch = 0, gamma = 0, vocab = 0, hidden = 0;
+  int ntiles = 0;
+  int num_sms = 148;
+  int draw_slices = 1;
+  void* ws = nullptr;
+  RowPartial* partial = nullptr;
+  float* gathered = nullptr;   // [nT + nD]
+  RowStat* tstat = nullptr;
+  RowStat* dstat = nullptr;
+  PosInfo* pos = nullptr;
+  SeqDecision* decision = nullptr;
+  double* draw_mass = nullptr;
+  unsigned* draw_ticket = nullptr;
+  double* resid = nullptr;
+  unsigned* status = nullptr;
+  unsigned* gemm_error = nullptr;
+  __nv_bfloat16* xt = nullptr;  // [B, hidden] the rows drawn from
+  __nv_bfloat16* xd = nullptr;
+  float* lt = nullptr;          // [B, vocab] their logits
+  float* ld = nullptr;
+  std::vector<cudaEvent_t> events;  // 3 per recorded run
+  int prof_capacity = 0;
+  int prof_runs = 0;
+};
+
+namespace {
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encode_fn() {
+  static EncodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(p);
+  });
+  return fn;
+}
+
+// a row-major [rows, cols] bf16 matrix, loaded in boxes of box_rows x 64
+// (128-byte rows, 128-byte swizzle); rows past the end read as zeros
+bool make_map(CUtensorMap* map, const void* base, long rows, int cols, int box_rows) {
+  EncodeTiled fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(lmhead::kBK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
+
+template <int kMode>
+cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const lmhead::LmParams& p,
+                        cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(lmhead::gemm_kernel<kMode>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       lmhead::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(static_cast<unsigned>(p.ntiles),
+                  static_cast<unsigned>((p.rows + lmhead::kBM - 1) / lmhead::kBM));
+  lmhead::gemm_kernel<kMode><<<grid, lmhead::kThreads, lmhead::kSmemBytes, s>>>(ma, mb, p);
+  return cudaGetLastError();
+}
+
+// the rows each sequence draws from: target row n and draft row n
+__global__ void gather_rows_kernel(const __nv_bfloat16* ht, const __nv_bfloat16* hd,
+                                   const SeqDecision* decision, int gamma, int hidden,
+                                   __nv_bfloat16* xt, __nv_bfloat16* xd) {
+  const int b = blockIdx.x;
+  const SeqDecision d = decision[b];
+  const int n = (d.mode == specverify::kDrawNone) ? 0 : d.n;
+  const uint4* st = reinterpret_cast<const uint4*>(ht + (static_cast<long>(b) * (gamma + 1) + n) * hidden);
+  uint4* dt = reinterpret_cast<uint4*>(xt + static_cast<long>(b) * hidden);
+  const int groups = hidden / 8;
+  for (int g = threadIdx.x; g < groups; g += blockDim.x) dt[g] = st[g];
+  if (gamma > 0) {
+    const int nd = n < gamma ? n : gamma - 1;
+    const uint4* sd = reinterpret_cast<const uint4*>(hd + (static_cast<long>(b) * gamma + nd) * hidden);
+    uint4* dd = reinterpret_cast<uint4*>(xd + static_cast<long>(b) * hidden);
+    for (int g = threadIdx.x; g < groups; g += blockDim.x) dd[g] = sd[g];
+  }
+}
+
+template <typename K>
+cudaError_t launch_plain(K kernel, unsigned grid, unsigned block, cudaStream_t s, const Params& p) {
+  kernel<<<grid, block, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+void split_c(float temperature, float& c_hi, float& c_lo, double& c) {
+  const double cd = 1.4426950408889634074 / static_cast<double>(temperature);
+  c_hi = static_cast<float>(cd);
+  if (static_cast<double>(c_hi) > cd) c_hi = std::nextafter(c_hi, 0.f);
+  c_lo = static_cast<float>(cd - static_cast<double>(c_hi));
+  if (!(c_lo >= 1e-30f)) c_lo = 1e-30f;
+  c = static_cast<double>(c_hi) + static_cast<double>(c_lo);
+}
+
+}  // namespace
+
+extern "C" {
+
+sv_status specverify_lmhead_create(specverify_lmhead_t* out, int batch, int gamma, int vocab,
+                                   int hidden, int device) {
+  if (!out) return SV_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (batch < 1 || gamma < 0 || gamma > specverify::kMaxGamma || vocab < 1 ||
+      vocab > (1 << 24) || hidden < lmhead::kBK || hidden % lmhead::kBK != 0 || hidden > (1 << 16))
+    return SV_ERR_INVALID_ARG;
+  const long nT = static_cast<long>(batch) * (gamma + 1), nD = static_cast<long>(batch) * gamma;
+  if (nT + nD > (1L << 30)) return SV_ERR_INVALID_ARG;
+  int ndev = 0;
+  cudaError_t e = cudaGetDeviceCount(&ndev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (device < 0 || device >= ndev) return SV_ERR_INVALID_ARG;
+  int major = 0, minor = 0, sms = 0;
+  e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
+  if (e != cudaSuccess) return cuda_fail(e);
+  if (major != 10 || minor != 0) {
+    std::snprintf(g_last_error, sizeof g_last_error,
+                  "device %d is sm_%d%d; this library is built for sm_100a only", device, major,
+                  minor);
+    return SV_ERR_UNSUPPORTED;
+  }
+  if (!encode_fn()) {
+    std::snprintf(g_last_error, sizeof g_last_error, "cuTensorMapEncodeTiled is not available");
+    return SV_ERR_UNSUPPORTED;
+  }
+  DeviceScope scope(device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  specverify_lmhead_ctx* h = new (std::nothrow) specverify_lmhead_ctx;
+  if (!h) return SV_ERR_OOM;
+  h->device = device;
+  h->batch = batch;
+  h->gamma = gamma;
+  h->vocab = vocab;
+  h->hidden = hidden;
+  h->num_sms = sms;
+  h->ntiles = (vocab + lmhead::kBN - 1) / lmhead::kBN;
+  // draw blocks per sequence for fp32 rows (the plain step's rule: about 48 KB
+  // of a row per block, at most one block per 4 tiles of 32 groups, at most 64)
+  {
+    const long groups = (vocab + 3) / 4;
+    const long tiles = (groups + specverify::kTile - 1) / specverify::kTile;
+    long ds = (2L * vocab * 4 + 48 * 1024 - 1) / (48 * 1024);
+    if (ds > tiles / 4) ds = tiles / 4;
+    if (ds > 64) ds = 64;
+    h->draw_slices = static_cast<int>(ds < 1 ? 1 : ds);
+  }
+  const size_t nB = static_cast<size_t>(batch);
+  const size_t tiles32 = static_cast<size_t>(((vocab + 3) / 4 + specverify::kTile - 1) / specverify::kTile);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = round_up(off + bytes, 256);
+    return at;
+  };
+  const size_t oP = take(static_cast<size_t>(nT + nD) * h->ntiles * sizeof(RowPartial));
+  const size_t oG = take(static_cast<size_t>(nT + nD) * sizeof(float));
+  const size_t oT = take(static_cast<size_t>(nT) * sizeof(RowStat));
+  const size_t oD = take(static_cast<size_t>(nD > 0 ? nD : 1) * sizeof(RowStat));
+  const size_t oQ = take(static_cast<size_t>(nD > 0 ? nD : 1) * sizeof(PosInfo));
+  const size_t oC = take(nB * sizeof(SeqDecision));
+  const size_t oW = take(nB * tiles32 * sizeof(double));
+  const size_t oK = take(nB * sizeof(unsigned));
+  const size_t oR = take(nB * sizeof(double));
+  const size_t oS = take(sizeof(unsigned));
+  const size_t oE = take(sizeof(unsigned));
+  const size_t oXT = take(nB * hidden * 2);
+  const size_t oXD = take(nB * hidden * 2);
+  const size_t oLT = take(nB * static_cast<size_t>(vocab) * 4);
+  const size_t oLD = take(nB * static_cast<size_t>(vocab) * 4);
+  e = cudaMalloc(&h->ws, off);
+  if (e != cudaSuccess) {
+    delete h;
+    return cuda_fail(e);
+  }
+  char* b = static_cast<char*>(h->ws);
+  h->partial = reinterpret_cast<RowPartial*>(b + oP);
+  h->gathered = reinterpret_cast<float*>(b + oG);
+  h->tstat = reinterpret_cast<RowStat*>(b + oT);
+  h->dstat = reinterpret_cast<RowStat*>(b + oD);
+  h->pos = reinterpret_cast<PosInfo*>(b + oQ);
+  h->decision = reinterpret_cast<SeqDecision*>(b + oC);
+  h->draw_mass = reinterpret_cast<double*>(b + oW);
+  h->draw_ticket = reinterpret_cast<unsigned*>(b + oK);
+  h->resid = reinterpret_cast<double*>(b + oR);
+  h->status = reinterpret_cast<unsigned*>(b + oS);
+  h->gemm_error = reinterpret_cast<unsigned*>(b + oE);
+  h->xt = reinterpret_cast<__nv_bfloat16*>(b + oXT);
+  h->xd = reinterpret_cast<__nv_bfloat16*>(b + oXD);
+  h->lt = reinterpret_cast<float*>(b + oLT);
+  h->ld = reinterpret_cast<float*>(b + oLD);
+  e = cudaMemset(h->ws, 0, off);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    cudaFree(h->ws);
+    delete h;
+    return cuda_fail(e);
+  }
+  *out = h;
+  return SV_OK;
+}
+
+sv_status specverify_lmhead_logits(specverify_lmhead_t h, const void* hidden_rows, int rows,
+                                   const void* weight, float* out_logits, void* stream) {
+  if (!h || !hidden_rows || !weight || !out_logits || rows < 1) return SV_ERR_INVALID_ARG;
+  if (!aligned16(hidden_rows) || !aligned16(weight) || !aligned16(out_logits))
+    return SV_ERR_INVALID_ARG;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  CUtensorMap ma, mb;
+  if (!make_map(&ma, hidden_rows, rows, h->hidden, lmhead::kBM) ||
+      !make_map(&mb, weight, h->vocab, h->hidden, lmhead::kBN))
+    return SV_ERR_INVALID_ARG;
+  lmhead::LmParams p{};
+  p.rows = rows;
+  p.vocab = h->vocab;
+  p.hidden = h->hidden;
+  p.ntiles = h->ntiles;
+  p.logits = out_logits;
+  p.error = h->gemm_error;
+  cudaError_t e = launch_gemm<lmhead::kModeLogits>(ma, mb, p, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SV_OK;
+}
+
+sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden,
+                                const void* target_weight, const void* draft_hidden,
+                                const void* draft_weight, const int32_t* draft_tokens,
+                                const float* u_accept, const float* u_resample, float temperature,
+                                int32_t* out_tokens, int32_t* out_num_accepted, void* stream) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  const int B = h->batch, G = h->gamma, V = h->vocab, D = h->hidden;
+  if (!target_hidden || !target_weight || !u_resample || !out_tokens || !out_num_accepted)
+    return SV_ERR_INVALID_ARG;
+  if (G > 0 && (!draft_hidden || !draft_weight || !draft_tokens || !u_accept))
+    return SV_ERR_INVALID_ARG;
+  if (!aligned16(target_hidden) || !aligned16(target_weight) ||
+      (G > 0 && (!aligned16(draft_hidden) || !aligned16(draft_weight))))
+    return SV_ERR_INVALID_ARG;
+  if (!std::isfinite(temperature) || !(temperature > 0.f)) return SV_ERR_INVALID_ARG;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const long nT = static_cast<long>(B) * (G + 1), nD = static_cast<long>(B) * G;
+
+  float c_hi, c_lo;
+  double c;
+  split_c(temperature, c_hi, c_lo, c);
+  if (!(c < 1e30)) return SV_ERR_INVALID_ARG;
+
+  CUtensorMap mht, mwt, mhd, mwd, mxt, mxd;
+  if (!make_map(&mht, target_hidden, nT, D, lmhead::kBM) ||
+      !make_map(&mwt, target_weight, V, D, lmhead::kBN) ||
+      !make_map(&mxt, h->xt, B, D, lmhead::kBM))
+    return SV_ERR_INVALID_ARG;
+  if (G > 0 && (!make_map(&mhd, draft_hidden, nD, D, lmhead::kBM) ||
+                !make_map(&mwd, draft_weight, V, D, lmhead::kBN) ||
+                !make_map(&mxd, h->xd, B, D, lmhead::kBM)))
+    return SV_ERR_INVALID_ARG;
+
+  cudaEvent_t* ev = nullptr;
+  if (h->prof_runs < h->prof_capacity) ev = h->events.data() + 3 * (h->prof_runs++);
+  cudaError_t e = ev ? cudaEventRecord(ev[0], s) : cudaSuccess;
+
+  // 1. statistics GEMMs
+  lmhead::LmParams g{};
+  g.vocab = V;
+  g.hidden = D;
+  g.ntiles = h->ntiles;
+  g.partial = h->partial;
+  g.tokens = draft_tokens;
+  g.token_stride = G;
+  g.gathered = h->gathered;
+  g.c_hi = c_hi;
+  g.c_lo = c_lo;
+  g.error = h->gemm_error;
+  g.rows = static_cast<int>(nT);
+  g.row_offset = 0;
+  g.positions = G + 1;
+  if (e == cudaSuccess) e = launch_gemm<lmhead::kModeStats>(mht, mwt, g, s);
+  if (G > 0) {
+    g.rows = static_cast<int>(nD);
+    g.row_offset = nT;
+    g.positions = G;
+    if (e == cudaSuccess) e = launch_gemm<lmhead::kModeStats>(mhd, mwd, g, s);
+  }
+  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
+
+  // 2. the decision, on the partials (one per 256-column tile of each row)
+  Params p{};
+  p.target = h->lt;  // the compact rows drawn from (written in step 4)
+  p.draft = h->ld;
+  p.target_map = nullptr;
+  p.draft_map = nullptr;
+  p.target_rows = nT;
+  p.draft_rows = nD;
+  p.tokens = draft_tokens;
+  p.u_accept = u_accept;
+  p.u_resample = u_resample;
+  p.out_tokens = out_tokens;
+  p.out_num_accepted = out_num_accepted;
+  p.partial = h->partial;
+  p.tstat = h->tstat;
+  p.dstat = h->dstat;
+  p.pos = h->pos;
+  p.decision = h->decision;
+  p.draw_mass = h->draw_mass;
+  p.draw_ticket = h->draw_ticket;
+  p.resid_mass = h->resid;
+  p.status = h->status;
+  p.batch = B;
+  p.gamma = G;
+  p.vocab = V;
+  p.slices = h->ntiles;
+  p.groups_per_slice = 0;
+  p.draw_slices = h->draw_slices;
+  {
+    const long groups = (V + 3) / 4;
+    const long ntiles32 = (groups + specverify::kTile - 1) / specverify::kTile;
+    p.groups_per_draw = static_cast<int>((ntiles32 + h->draw_slices - 1) / h->draw_slices) * specverify::kTile;
+  }
+  p.c_hi = c_hi;
+  p.c_lo = c_lo;
+  p.c = c;
+  p.gathered_target = h->gathered;
+  p.gathered_draft = h->gathered + nT;
+  p.draw_compact = 1;
+  const int per = specverify::kDecideThreads / specverify::kWarp;
+  if (e == cudaSuccess)
+    e = launch_plain(specverify::decide_kernel<float>, static_cast<unsigned>((B + per - 1) / per),
+                     specverify::kDecideThreads, s, p);
+
+  // 3-4. the two rows each sequence draws from, and their logits
+  if (e == cudaSuccess) {
+    gather_rows_kernel<<<B, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(target_hidden),
+                                         static_cast<const __nv_bfloat16*>(draft_hidden),
+                                         h->decision, G, D, h->xt, h->xd);
+    e = cudaGetLastError();
+  }
+  lmhead::LmParams l{};
+  l.rows = B;
+  l.vocab = V;
+  l.hidden = D;
+  l.ntiles = h->ntiles;
+  l.error = h->gemm_error;
+  l.logits = h->lt;
+  if (e == cudaSuccess) e = launch_gemm<lmhead::kModeLogits>(mxt, mwt, l, s);
+  if (G > 0) {
+    l.logits = h->ld;
+    if (e == cudaSuccess) e = launch_gemm<lmhead::kModeLogits>(mxd, mwd, l, s);
+  }
+
+  // 5. the draw on fp32 rows
+  const bool aligned = (static_cast<size_t>(V) * 4) % 16 == 0;
+  if (e == cudaSuccess)
+    e = aligned ? launch_plain(specverify::draw_kernel<float, true>,
+                               static_cast<unsigned>(static_cast<long>(B) * h->draw_slices),
+                               specverify::kDrawThreads, s, p)
+                : launch_plain(specverify::draw_kernel<float, false>,
+                               static_cast<unsigned>(static_cast<long>(B) * h->draw_slices),
+                               specverify::kDrawThreads, s, p);
+  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  return SV_OK;
+}
+
+sv_status specverify_lmhead_get_status(specverify_lmhead_t h, void* stream, uint32_t* bits) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned v[2] = {0, 0};
+  cudaError_t e = cudaMemcpyAsync(&v[0], h->status, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(&v[1], h->gemm_error, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->status, 0, sizeof(unsigned), s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->gemm_error, 0, sizeof(unsigned), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const unsigned all = v[0] | (v[1] ? 32u : 0u);
+  if (bits) *bits = all;
+  if (v[1]) return SV_ERR_PIPELINE;
+  if (v[0] & specverify::kStatTokenRange) return SV_ERR_TOKEN_RANGE;
+  if (v[0] & specverify::kStatNonFinite) return SV_ERR_NONFINITE;
+  if (v[0] & specverify::kStatZeroMass) return SV_WARN_ZERO_MASS;
+  return SV_OK;
+}
+
+sv_status specverify_lmhead_readback(specverify_lmhead_t h, double* target_lse,
+                                     double* draft_lse, double* q_tok, double* p_tok,
+                                     double* resid_mass, void* stream) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  const size_t nT = static_cast<size_t>(h->batch) * (h->gamma + 1);
+  const size_t nD = static_cast<size_t>(h->batch) * h->gamma;
+  std::vector<RowStat> ts(nT), ds(nD);
+  std::vector<PosInfo> ps(nD);
+  std::vector<double> rm(h->batch);
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess) e = cudaMemcpy(ts.data(), h->tstat, nT * sizeof(RowStat), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && nD) e = cudaMemcpy(ds.data(), h->dstat, nD * sizeof(RowStat), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess && nD) e = cudaMemcpy(ps.data(), h->pos, nD * sizeof(PosInfo), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(rm.data(), h->resid, h->batch * sizeof(double), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const double ln2 = 0.69314718055994530942;
+  for (size_t i = 0; i < nT; ++i)
+    if (target_lse) target_lse[i] = ts[i].lse2 * ln2;
+  for (size_t i = 0; i < nD; ++i) {
+    if (draft_lse) draft_lse[i] = ds[i].lse2 * ln2;
+    if (q_tok) q_tok[i] = ps[i].q_tok;
+    if (p_tok) p_tok[i] = ps[i].p_tok;
+  }
+  if (resid_mass)
+    for (int b = 0; b < h->batch; ++b) resid_mass[b] = rm[b];
+  return SV_OK;
+}
+
+sv_status specverify_lmhead_profile_begin(specverify_lmhead_t h, int max_runs) {
+  if (!h || max_runs < 0 || max_runs > (1 << 20)) return SV_ERR_INVALID_ARG;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e);
+  for (cudaEvent_t ev : h->events) cudaEventDestroy(ev);
+  h->events.clear();
+  h->prof_capacity = 0;
+  h->prof_runs = 0;
+  for (int i = 0; i < 3 * max_runs; ++i) {
+    cudaEvent_t ev;
+    e = cudaEventCreate(&ev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    h->events.push_back(ev);
+  }
+  h->prof_capacity = max_runs;
+  return SV_OK;
+}
+
+sv_status specverify_lmhead_profile_end(specverify_lmhead_t h, float* stats_ms, float* rest_ms,
+                                        int* runs) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  DeviceScope scope(h->device);
+  if (!scope.ok()) return SV_ERR_CUDA;
+  double a = 0.0, c = 0.0;
+  for (int r = 0; r < h->prof_runs; ++r) {
+    cudaEvent_t* ev = h->events.data() + 3 * r;
+    float t1 = 0.f, t2 = 0.f;
+    cudaError_t e = cudaEventSynchronize(ev[2]);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t1, ev[0], ev[1]);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t2, ev[1], ev[2]);
+    if (e != cudaSuccess) return cuda_fail(e);
+    a += t1;
+    c += t2;
+  }
+  const int n = h->prof_runs;
+  if (stats_ms) *stats_ms = n ? static_cast<float>(a / n) : 0.f;
+  if (rest_ms) *rest_ms = n ? static_cast<float>(c / n) : 0.f;
+  if (runs) *runs = n;
+  for (cudaEvent_t ev : h->events) cudaEventDestroy(ev);
+  h->events.clear();
+  h->prof_capacity = 0;
+  h->prof_runs = 0;
+  return SV_OK;
+}
+
+void specverify_lmhead_destroy(specverify_lmhead_t h) {
+  if (!h) return;
+  {
+    DeviceScope scope(h->device);
+    if (scope.ok()) {
+      cudaDeviceSynchronize();
+      for (cudaEvent_t ev : h->events) cudaEventDestroy(ev);
+      if (h->ws) cudaFree(h->ws);
+    }
+  }
+  delete h;
+}
+
+}  // extern "C"

@@ -1,0 +1,306 @@
+// The LM-head GEMM of the fused verification step, on the 5th-generation
+// tensor cores (tcgen05) of sm_100a.
+//
+// logits[r, v] = sum_k hidden[r, k] * weight[v, k]   (bf16 inputs, fp32 accumulation)
+//
+// One CTA computes a 128 x 256 tile of logits (rows x vocabulary): TMA loads
+// 128 x 64 and 256 x 64 bf16 tiles (128-byte swizzle) into a 4-stage ring of
+// shared memory; one thread issues tcgen05.mma (M = 128, N = 256, K = 16) with
+// the accumulator in tensor memory (256 columns); the four warps then read the
+// accumulator back with tcgen05.ld, 32 columns at a time, each warp its 32
+// rows (TMEM lanes).  The epilogue either
+//   - folds the tile into per-row softmax statistics (s = sum 2^(x c - o) with
+//     a running offset o, as the streaming statistics kernel does), and picks
+//     out the logit at the row's draft token when the token falls in the tile
+//     (the logits never reach global memory), or
+//   - writes the fp32 logits (the rows the draw needs).
+//
+// Every wait on an mbarrier is bounded: after kSpinLimit tries the thread sets
+// the error flag and leaves the loop, the kernel skips its remaining work, and
+// warp 0 still frees the tensor memory.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "verify_kernel.cuh"
+
+namespace lmhead {
+
+constexpr int kBM = 128;     // rows per tile (UMMA M)
+constexpr int kBN = 256;     // vocabulary columns per tile (UMMA N)
+constexpr int kBK = 64;      // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int kUK = 16;      // K per tcgen05.mma (bf16)
+constexpr int kStages = 4;
+constexpr int kThreads = 128;
+constexpr int kABytes = kBM * kBK * 2;   // 16 KB
+constexpr int kBBytes = kBN * kBK * 2;   // 32 KB
+constexpr int kStageBytes = kABytes + kBBytes;
+constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + room to align to 1024
+constexpr int kTmemCols = 256;
+constexpr unsigned kSpinLimit = 1u << 20;  // tries per wait (well under a second)
+
+enum : int { kModeStats = 0, kModeLogits = 1 };
+
+struct LmParams {
+  int rows;                 // M: rows of hidden
+  int vocab;                // N: rows of weight
+  int hidden;               // K (a multiple of 64)
+  int ntiles;               // vocabulary tiles = ceil(vocab / 256)
+  // statistics mode
+  specverify::RowPartial* partial;  // [(row_offset + rows) * ntiles]
+  long row_offset;
+  const int32_t* tokens;    // token whose logit is picked out for row r, or null
+  int token_stride;         // row r -> tokens[(r / (G+1)) * G + r % (G+1)] via the two fields
+  int positions;            // G + 1 for target rows (the last position has no token), G for draft
+  float* gathered;          // [row_offset + rows] logit at the row's token
+  float c_hi, c_lo;
+  // logits mode
+  float* logits;            // [rows, vocab] fp32
+  unsigned* error;          // set when a wait gives up
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// wait for the phase with the given parity to complete; false after the limit
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+  const uint32_t a = smem_u32(bar);
+  for (unsigned i = 0; i < kSpinLimit; ++i) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// K-major operand tile with 128-byte swizzle: rows of 128 bytes, 8-row groups
+// 1024 bytes apart (stride byte offset), descriptor version 1, swizzle mode 2
+__device__ __forceinline__ uint64_t umma_desc(uint32_t saddr) {
+  return (static_cast<uint64_t>((saddr >> 4) & 0x3FFFu)) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+// kind::f16 instruction descriptor: fp32 accumulator, bf16 A and B, both
+// K-major, M = 128, N = 256
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                            (static_cast<uint32_t>(kBN >> 3) << 17) |
+                            (static_cast<uint32_t>(kBM >> 4) << 24);
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t da, uint64_t db, bool accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(da), "l"(db), "r"(kIdesc), "r"(accum ? 1u : 0u));
+}
+
+// arrive on `bar` once every tcgen05.mma issued so far by this thread is done
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---------------------------------------------------------------------------
+// the kernel
+// ---------------------------------------------------------------------------
+
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_hidden,
+                const __grid_constant__ CUtensorMap tm_weight, const LmParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];
+  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int s_failed;
+
+  const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kBN;   // vocabulary tile
+  const int m0 = blockIdx.y * kBM;   // row tile
+  const int nk = P.hidden / kBK;
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&accum_bar, 1);
+    s_failed = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&tmem_base_s)),
+                 "r"(kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+
+  if (warp == 0 && lane == 0) {
+    // producer: TMA loads into the ring
+    for (int kt = 0; kt < nk; ++kt) {
+      const int s = kt % kStages;
+      if (kt >= kStages && !mbar_wait(&empty_bar[s], ((kt / kStages) - 1) & 1)) {
+        s_failed = 1;
+        break;
+      }
+      uint8_t* a = smem + s * kStageBytes;
+      uint8_t* b = a + kABytes;
+      mbar_expect_tx(&full_bar[s], kStageBytes);
+      tma_load_2d(a, &tm_hidden, &full_bar[s], kt * kBK, m0);
+      tma_load_2d(b, &tm_weight, &full_bar[s], kt * kBK, n0);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // MMA issuer
+    for (int kt = 0; kt < nk; ++kt) {
+      const int s = kt % kStages;
+      if (!mbar_wait(&full_bar[s], (kt / kStages) & 1)) {
+        s_failed = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t a = smem_u32(smem + s * kStageBytes);
+      const uint32_t b = a + kABytes;
+#pragma unroll
+      for (int k = 0; k < kBK / kUK; ++k)
+        umma_f16(tmem, umma_desc(a + k * kUK * 2), umma_desc(b + k * kUK * 2), kt > 0 || k > 0);
+      umma_commit(&empty_bar[s]);  // the stage is free once these MMAs are done
+    }
+    umma_commit(&accum_bar);  // the accumulator is complete
+  }
+
+  // epilogue: all four warps, each its 32 TMEM lanes (rows); the decision to
+  // read the accumulator is block-uniform (the loads are warp-collective)
+  const bool ok = mbar_wait(&accum_bar, 0);
+  const bool good = __syncthreads_and(ok) && !*static_cast<volatile int*>(&s_failed);
+  tc_fence_after();
+  const int r = m0 + warp * 32 + lane;
+  if (good) {
+    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    if constexpr (kMode == kModeStats) {
+      int t = -1;
+      if (r < P.rows && P.tokens) {
+        const int pos = r % P.positions, seq = r / P.positions;
+        if (pos < P.token_stride) t = P.tokens[static_cast<long>(seq) * P.token_stride + pos];
+      }
+      float o = -INFINITY, sum = 0.f, xt = 0.f;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBN; c0 += 32) {
+        float v[32];
+        tmem_ld32(lane_addr + c0, v);
+        float cm = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int col = n0 + c0 + i;
+          if (col >= P.vocab) v[i] = -INFINITY;
+          if (col == t) xt = v[i];
+          cm = fmaxf(cm, v[i]);
+        }
+        const float on = cm * P.c_hi;
+        if (cm != -INFINITY && on > o) {
+          sum *= specverify::ex2(o - on);
+          o = on;
+        }
+        if (o != -INFINITY) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) sum += specverify::ex2(specverify::arg2(v[i], P.c_hi, P.c_lo, o));
+        }
+      }
+      if (r < P.rows) {
+        P.partial[(P.row_offset + r) * P.ntiles + blockIdx.x] =
+            specverify::RowPartial{static_cast<double>(sum), o, 0};
+        if (t >= n0 && t < n0 + kBN) P.gathered[P.row_offset + r] = xt;
+      }
+    } else {
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBN; c0 += 32) {
+        float v[32];
+        tmem_ld32(lane_addr + c0, v);
+        if (r < P.rows) {
+          float* out = P.logits + static_cast<long>(r) * P.vocab + n0 + c0;
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (n0 + c0 + i < P.vocab) out[i] = v[i];
+        }
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    atomicOr(P.error, 1u);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols));
+  }
+}
+
+}  // namespace lmhead

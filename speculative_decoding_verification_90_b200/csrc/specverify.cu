@@ -266,6 +266,9 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
   p.c_hi = c_hi;
   p.c_lo = c_lo;
   p.c = static_cast<double>(c_hi) + static_cast<double>(c_lo);
+  p.gathered_target = nullptr;
+  p.gathered_draft = nullptr;
+  p.draw_compact = 0;
 
   const bool aligned = aligned_to(target, 16) && (G == 0 || aligned_to(draft, 16)) &&
                        (static_cast<size_t>(h->vocab) * es) % 16 == 0;
@@ -694,6 +697,7 @@ const char* specverify_status_string(sv_status s) {
     case SV_ERR_ROW_INDEX: return "row map entry outside the logit rows given";
     case SV_ERR_PARENT: return "parent index out of range, self link or cycle";
     case SV_ERR_TEMPERATURE: return "temperature negative, NaN or infinite";
+    case SV_ERR_PIPELINE: return "a tensor-core pipeline wait gave up";
   }
   return "unknown status";
 }

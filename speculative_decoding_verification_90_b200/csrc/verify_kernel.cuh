@@ -122,6 +122,12 @@ struct Params {
   int groups_per_draw;       // groups per draw block (whole 32-group tiles)
   float c_hi, c_lo;          // log2(e)/T = c_hi + c_lo, c_lo > 0
   double c;                  // c_hi + c_lo, exactly
+  // fused LM-head form: the logits at the draft tokens were picked out by the
+  // GEMM ([target_rows] and [draft_rows] floats; null: read the logit rows),
+  // and the draw reads row b of compact [B, V] logit buffers
+  const float* gathered_target;
+  const float* gathered_draft;
+  int draw_compact;
 };
 
 // ---------------------------------------------------------------------------
@@ -541,8 +547,10 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
           u = P.u_accept[pj];
           tok_bad = (t < 0 || t >= V);
           if (!tok_bad && !map_bad) {
-            xt = Elem<T>::load1(static_cast<const T*>(P.target) + tr * V, t);
-            xd = Elem<T>::load1(static_cast<const T*>(P.draft) + dr * V, t);
+            xt = P.gathered_target ? P.gathered_target[tr]
+                                   : Elem<T>::load1(static_cast<const T*>(P.target) + tr * V, t);
+            xd = P.gathered_draft ? P.gathered_draft[dr]
+                                  : Elem<T>::load1(static_cast<const T*>(P.draft) + dr * V, t);
           }
         }
         int validT = 0, validD = 1;
@@ -610,8 +618,8 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
       }
       if (lane == 0) {
         P.out_num_accepted[b] = n;
-        SeqDecision d{lT_n, lD_n, tr_n, dr_n, n, (n < G) ? kDrawResidual : kDrawTarget, 0u,
-                      0.f, 0.f, 0.f, 1.f};
+        SeqDecision d{lT_n, lD_n, P.draw_compact ? b : tr_n, P.draw_compact ? b : dr_n, n,
+                      (n < G) ? kDrawResidual : kDrawTarget, 0u, 0.f, 0.f, 0.f, 1.f};
         float lt_lo;
         split2(lT_n, d.lt_hi, lt_lo);
         split2(lT_n - lD_n, d.k_hi, d.k_lo);

@@ -32,6 +32,7 @@ SV_WARN_ZERO_MASS = 18
 SV_ERR_ROW_INDEX = 19
 SV_ERR_PARENT = 20
 SV_ERR_TEMPERATURE = 21
+SV_ERR_PIPELINE = 22
 
 # every function declared in include/*.h, with its ctypes signature
 _vp, _i, _f, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_uint32)
@@ -59,6 +60,15 @@ SIGNATURES = {
     "specfold_gate_profile_end": (_i, [_vp, ctypes.POINTER(_f), ctypes.POINTER(_f),
                                        ctypes.POINTER(_i)]),
     "specfold_gate_destroy": (None, [_vp]),
+    "specverify_lmhead_create": (_i, [ctypes.POINTER(_vp), _i, _i, _i, _i, _i]),
+    "specverify_lmhead_run": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
+    "specverify_lmhead_logits": (_i, [_vp, _vp, _i, _vp, _vp, _vp]),
+    "specverify_lmhead_get_status": (_i, [_vp, _vp, _u32p]),
+    "specverify_lmhead_readback": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "specverify_lmhead_profile_begin": (_i, [_vp, _i]),
+    "specverify_lmhead_profile_end": (_i, [_vp, ctypes.POINTER(_f), ctypes.POINTER(_f),
+                                           ctypes.POINTER(_i)]),
+    "specverify_lmhead_destroy": (None, [_vp]),
     "specverify_status_string": (ctypes.c_char_p, [_i]),
     "specverify_last_error": (ctypes.c_char_p, []),
 }
@@ -229,6 +239,56 @@ def specfold_gate_profile_end(h) -> dict:
 
 def specfold_gate_destroy(h) -> None:
     _lib.specfold_gate_destroy(h)
+
+
+def specverify_lmhead_create(batch, gamma, vocab, hidden, device=0) -> int:
+    h = ctypes.c_void_p()
+    _check(_lib.specverify_lmhead_create(ctypes.byref(h), batch, gamma, vocab, hidden, device),
+           "specverify_lmhead_create")
+    return h.value
+
+
+def specverify_lmhead_run(h, target_hidden, target_weight, draft_hidden, draft_weight, tokens,
+                          u_accept, u_resample, temperature, out_tokens, out_num_accepted,
+                          stream=0) -> int:
+    return _check(_lib.specverify_lmhead_run(h, target_hidden, target_weight, draft_hidden,
+                                             draft_weight, tokens, u_accept, u_resample,
+                                             float(temperature), out_tokens, out_num_accepted,
+                                             stream),
+                  "specverify_lmhead_run")
+
+
+def specverify_lmhead_logits(h, hidden_rows, rows, weight, out_logits, stream=0) -> int:
+    return _check(_lib.specverify_lmhead_logits(h, hidden_rows, rows, weight, out_logits, stream),
+                  "specverify_lmhead_logits")
+
+
+def specverify_lmhead_get_status(h, stream=0) -> tuple[int, int]:
+    bits = ctypes.c_uint32()
+    st = _lib.specverify_lmhead_get_status(h, stream, ctypes.byref(bits))
+    if st in (SV_ERR_INVALID_ARG, SV_ERR_CUDA, SV_ERR_OOM, SV_ERR_UNSUPPORTED):
+        _check(st, "specverify_lmhead_get_status")
+    return st, bits.value
+
+
+def specverify_lmhead_readback(h, *ptrs, stream=0) -> int:
+    return _check(_lib.specverify_lmhead_readback(h, *ptrs, stream), "specverify_lmhead_readback")
+
+
+def specverify_lmhead_profile_begin(h, max_runs: int) -> int:
+    return _check(_lib.specverify_lmhead_profile_begin(h, max_runs),
+                  "specverify_lmhead_profile_begin")
+
+
+def specverify_lmhead_profile_end(h) -> dict:
+    a, c, n = ctypes.c_float(), ctypes.c_float(), ctypes.c_int()
+    _check(_lib.specverify_lmhead_profile_end(h, ctypes.byref(a), ctypes.byref(c),
+                                              ctypes.byref(n)), "specverify_lmhead_profile_end")
+    return {"stats_ms": a.value, "rest_ms": c.value, "runs": n.value}
+
+
+def specverify_lmhead_destroy(h) -> None:
+    _lib.specverify_lmhead_destroy(h)
 
 
 def specverify_status_string(status: int) -> str:
@@ -518,3 +578,87 @@ class FoldGate:
 
     def profile_end(self) -> dict:
         return specfold_gate_profile_end(self.handle)
+
+
+class LmHeadVerify:
+    """The verification step fused with the LM head, for fixed (batch, gamma,
+    vocab, hidden) on one CUDA device; bf16 hidden states and weights."""
+
+    def __init__(self, batch: int, gamma: int, vocab: int, hidden: int, device: int = 0):
+        self.batch, self.gamma, self.vocab, self.hidden = batch, gamma, vocab, hidden
+        self.device = device
+        self.handle = specverify_lmhead_create(batch, gamma, vocab, hidden, device)
+
+    def close(self):
+        if getattr(self, "handle", None):
+            specverify_lmhead_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def _t(self, name, t, shape, dtype):
+        if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous() \
+                or t.device.type != "cuda" or t.device.index != self.device:
+            raise ValueError(f"{name}: must be a contiguous {dtype} {tuple(shape)} tensor on "
+                             f"cuda:{self.device}")
+        return t.data_ptr() if t.numel() else 0
+
+    def _stream(self, stream):
+        import torch
+        if stream is None:
+            stream = torch.cuda.current_stream(self.device)
+        return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+    def run(self, target_hidden, target_weight, draft_hidden, draft_weight, tokens, u_accept,
+            u_resample, temperature, out_tokens, out_num_accepted, stream=None):
+        import torch
+        B, G, V, D = self.batch, self.gamma, self.vocab, self.hidden
+        bf = torch.bfloat16
+        args = [self._t("target_hidden", target_hidden, (B, G + 1, D), bf),
+                self._t("target_weight", target_weight, (V, D), bf),
+                self._t("draft_hidden", draft_hidden, (B, G, D), bf),
+                self._t("draft_weight", draft_weight, (V, D), bf),
+                self._t("tokens", tokens, (B, G), torch.int32),
+                self._t("u_accept", u_accept, (B, G), torch.float32),
+                self._t("u_resample", u_resample, (B,), torch.float32)]
+        outs = [self._t("out_tokens", out_tokens, (B, G + 1), torch.int32),
+                self._t("out_num_accepted", out_num_accepted, (B,), torch.int32)]
+        specverify_lmhead_run(self.handle, *args, temperature, *outs, self._stream(stream))
+
+    def logits(self, hidden_rows, weight, out, stream=None):
+        import torch
+        rows = hidden_rows.shape[0]
+        specverify_lmhead_logits(
+            self.handle, self._t("hidden_rows", hidden_rows, (rows, self.hidden), torch.bfloat16),
+            rows, self._t("weight", weight, (self.vocab, self.hidden), torch.bfloat16),
+            self._t("out", out, (rows, self.vocab), torch.float32), self._stream(stream))
+
+    def status(self, stream=None) -> tuple[int, int]:
+        return specverify_lmhead_get_status(self.handle, self._stream(stream))
+
+    def readback(self, stream=None) -> dict:
+        B, G = self.batch, self.gamma
+        out = {"target_lse": np.zeros((B, G + 1)), "draft_lse": np.zeros((B, G)),
+               "q_tok": np.zeros((B, G)), "p_tok": np.zeros((B, G)),
+               "resid_mass": np.zeros(B)}
+        specverify_lmhead_readback(self.handle, *[out[k].ctypes.data if out[k].size else None
+                                                  for k in ("target_lse", "draft_lse", "q_tok",
+                                                            "p_tok", "resid_mass")],
+                                   stream=self._stream(stream))
+        return out
+
+    def profile_begin(self, max_runs: int):
+        specverify_lmhead_profile_begin(self.handle, max_runs)
+
+    def profile_end(self) -> dict:
+        return specverify_lmhead_profile_end(self.handle)

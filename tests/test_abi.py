@@ -11,7 +11,7 @@ import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
-PREFIX = r"(?:specverify|specfold_gate)_\w+"
+PREFIX = r"(?:specverify|specfold_gate|specverify_lmhead)_\w+"
 
 
 def _declared():
