@@ -28,6 +28,7 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 DTYPE_F32 = 0
 DTYPE_BF16 = 1
+DTYPE_F64 = 2
 
 OK = 0
 ERR_TOKEN_RANGE = 16
@@ -158,7 +159,20 @@ def _dtype_code(arr: np.ndarray) -> int:
         return DTYPE_F32
     if arr.dtype == np.uint16:
         return DTYPE_BF16
-    raise TypeError(f"logits must be float32 or uint16 (bf16 bits), got {arr.dtype}")
+    if arr.dtype == np.float64:
+        return DTYPE_F64
+    raise TypeError(f"logits must be float32, float64 or uint16 (bf16 bits), got {arr.dtype}")
+
+
+def lm_logits(hidden: np.ndarray, weight: np.ndarray) -> np.ndarray:
+    """Logits of an output layer, exactly as the plain definition states them:
+    hidden [..., d] . weight [V, d]^T in float64 (hidden and weight given as
+    float32 values, e.g. the values of bf16 inputs).  A library matmul is the
+    one step; the product of two bf16 values is exact in float64 and the sum
+    of d of them is rounded at most d times at double precision."""
+    h = np.asarray(hidden, np.float64)
+    w = np.asarray(weight, np.float64)
+    return np.ascontiguousarray(h @ w.T)
 
 
 def softmax(row: np.ndarray, temperature: float = 1.0):

@@ -55,6 +55,7 @@
 
 #define ORACLE_DTYPE_F32 0
 #define ORACLE_DTYPE_BF16 1
+#define ORACLE_DTYPE_F64 2 /* logits computed exactly from an output layer */
 
 #define ORACLE_OK 0
 #define ORACLE_ERR_TOKEN_RANGE 16
@@ -105,6 +106,7 @@ static double oracle_bf16_to_double(uint16_t bits) {
 static double oracle_load(const void *base, int dtype, size_t index) {
   if (dtype == ORACLE_DTYPE_BF16)
     return oracle_bf16_to_double(((const uint16_t *)base)[index]);
+  if (dtype == ORACLE_DTYPE_F64) return ((const double *)base)[index];
   return (double)((const float *)base)[index];
 }
 

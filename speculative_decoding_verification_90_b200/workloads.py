@@ -34,6 +34,9 @@ on; no public dataset stands behind any of them):
                    j >= bp are fresh N(0, 3^2) draws per branch.  Draft =
                    0.8 target + 0.2 N(0, 3^2).  Also given as distinct rows
                    plus row maps, for the shared-row entry point.
+* ``lmhead``       fused-step inputs: 64 sequences, gamma=8, V=128256,
+                   hidden 4096, bf16 hidden states and output layer whose
+                   logits are N(0, 3^2) (see the function).
 * ``gate_tree``    fold-gate inputs: 128 sequences x 8 candidate branches, one
                    block of 32 positions, hidden size 4096, bf16; a random
                    tree per sequence and a perturbation that peaks at each
@@ -382,6 +385,80 @@ def gate_tree(seed: int = 0, sequences: int = 128, branches: int = 8, positions:
     return GateWorkload(name, nb, positions, dim, dtype, float(tau), hidden, parent,
                         {"sequences": sequences, "branches_per_sequence": branches,
                          "revealed": revealed})
+
+
+@dataclass
+class LmWorkload:
+    """Hidden states and output-layer weights (bf16 bits) for the fused step."""
+    name: str
+    batch: int
+    gamma: int
+    vocab: int
+    hidden: int
+    temperature: float
+    target_hidden: np.ndarray   # uint16 [B, gamma+1, hidden]
+    target_weight: np.ndarray   # uint16 [vocab, hidden]
+    draft_hidden: np.ndarray    # uint16 [B, gamma, hidden]
+    draft_weight: np.ndarray    # uint16 [vocab, hidden] (the target's when shared)
+    tokens: np.ndarray          # int32 [B, gamma]
+    u_accept: np.ndarray        # float32 [B, gamma]
+    u_resample: np.ndarray      # float32 [B]
+    meta: dict = field(default_factory=dict)
+
+
+def lmhead(seed: int = 0, batch: int = 64, gamma: int = 8, vocab: int = 128256,
+           hidden: int = 4096, shared_weight: bool = True, temperature: float = 1.0) -> LmWorkload:
+    """Output-layer inputs with logits distributed like the b64_g8_v128256 batch.
+
+    Target hidden states N(0, 1); weights N(0, (3/sqrt(hidden))^2), so a logit
+    is N(0, 3^2); draft hidden states 0.9 x the target's at the same position +
+    0.1 x N(0, 1); the draft uses the target's output layer (shared) or
+    0.85 x it + 0.15 x fresh noise.  All stored as bf16.  Draft tokens are drawn
+    from softmax(draft logits / T) by Gumbel-max on float32 logits of the stored
+    values (computed here in row blocks).
+    """
+    rng = np.random.default_rng(seed)
+    B, G, V, D = batch, gamma, vocab, hidden
+    ht = bf16_bits(rng.standard_normal((B, G + 1, D), dtype=np.float32))
+    w = np.empty((V, D), np.uint16)
+    sigma = np.float32(3.0 / np.sqrt(D))
+    for v0 in range(0, V, 8192):
+        w[v0:v0 + 8192] = bf16_bits(rng.standard_normal((min(8192, V - v0), D), dtype=np.float32)
+                                    * sigma)
+    hd = bf16_bits(np.float32(0.9) * bits_to_f32(ht[:, :G])
+                   + np.float32(0.1) * rng.standard_normal((B, G, D), dtype=np.float32))
+    if shared_weight:
+        wd = w
+    else:
+        wd = np.empty_like(w)
+        for v0 in range(0, V, 8192):
+            n = min(8192, V - v0)
+            wd[v0:v0 + n] = bf16_bits(np.float32(0.85) * bits_to_f32(w[v0:v0 + n])
+                                      + np.float32(0.15) * sigma
+                                      * rng.standard_normal((n, D), dtype=np.float32))
+    tokens = np.zeros((B, G), np.int32)
+    if G > 0:
+        hdf = bits_to_f32(hd).reshape(B * G, D)
+        best = np.full(B * G, -np.inf, np.float32)
+        arg = np.zeros(B * G, np.int64)
+        tiny = np.float32(np.finfo(np.float32).tiny)
+        for v0 in range(0, V, 8192):
+            n = min(8192, V - v0)
+            logits = hdf @ bits_to_f32(wd[v0:v0 + n]).T
+            u = rng.random(logits.shape, dtype=np.float32)
+            np.maximum(u, tiny, out=u)
+            g = logits / np.float32(temperature) - np.log(-np.log(u))
+            j = np.argmax(g, axis=1)
+            val = g[np.arange(g.shape[0]), j]
+            better = val > best
+            best[better] = val[better]
+            arg[better] = v0 + j[better]
+        tokens = arg.astype(np.int32).reshape(B, G)
+    u_acc = rng.random((B, G), dtype=np.float32)
+    u_res = rng.random(B, dtype=np.float32)
+    name = f"lmhead_b{B}_g{G}_v{V}_d{D}_bf16" + ("" if shared_weight else "_two_heads")
+    return LmWorkload(name, B, G, V, D, float(temperature), ht, w, hd, wd, tokens, u_acc, u_res,
+                      {"shared_weight": shared_weight})
 
 
 REGISTRY = {
