@@ -1,0 +1,177 @@
+"""GPU parity of the verification step fused with the LM head
+(specverify_lmhead_run) against the CPU oracle run on float64 logits
+x = h . W^T computed from the same bf16 hidden states and weights.
+
+The GPU forms the logits with fp32 accumulation on tensor cores.  The bound
+used here: |x_gpu - x| <= 4e-6 * sum_k |h_k w_k| per logit (the largest
+ratio measured on B200 is 6.4e-7; at hidden 4096 with logits N(0, 3^2) the
+scale sum |h w| is about 120, so logits differ by up to about 5e-4 and
+probabilities by a relative 7e-4).  Decisions must therefore agree outside a
+margin of FUSED_MARGIN, probabilities within FUSED_PROB_TOL absolute and log
+normalisers within FUSED_LSE_TOL.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+
+from speculative_decoding_verification_90_b200 import workloads
+
+from parity import assert_parity, compare
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover - collected on CPU hosts
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+GEMM_REL = 4e-6
+FUSED_MARGIN = 2e-3
+FUSED_PROB_TOL = 1e-3
+FUSED_LSE_TOL = 1e-3
+
+
+def _bf(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def _f(a, dtype=np.float32):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype)).cuda()
+
+
+def run_fused(w, lm=None):
+    from speculative_decoding_verification_90_b200.specverify import LmHeadVerify
+    own = lm is None
+    if own:
+        lm = LmHeadVerify(w.batch, w.gamma, w.vocab, w.hidden)
+    try:
+        B, G = w.batch, w.gamma
+        ht, wt = _bf(w.target_hidden), _bf(w.target_weight)
+        hd = _bf(w.draft_hidden)
+        wd = wt if w.draft_weight is w.target_weight else _bf(w.draft_weight)
+        ot = torch.full((B, G + 1), -7, dtype=torch.int32, device="cuda")
+        on = torch.full((B,), -7, dtype=torch.int32, device="cuda")
+        lm.run(ht, wt, hd, wd, _f(w.tokens, np.int32), _f(w.u_accept), _f(w.u_resample),
+               w.temperature, ot, on)
+        torch.cuda.synchronize()
+        st, bits = lm.status()
+        res = {"out_tokens": ot.cpu().numpy(), "out_num_accepted": on.cpu().numpy(),
+               "status": st, "bits": bits}
+        res.update(lm.readback())
+        return res
+    finally:
+        if own:
+            lm.close()
+
+
+def oracle_fused(w):
+    import os
+    import oracle
+    t = oracle.lm_logits(workloads.bits_to_f32(w.target_hidden), workloads.bits_to_f32(w.target_weight))
+    d = oracle.lm_logits(workloads.bits_to_f32(w.draft_hidden), workloads.bits_to_f32(w.draft_weight))
+    return oracle.verify(t, d, w.tokens, w.u_accept, w.u_resample,
+                         float(np.float32(w.temperature)), threads=os.cpu_count() or 1)
+
+
+def _parity(w, name):
+    import parity
+    g = run_fused(w)
+    o = oracle_fused(w)
+    old = parity.MARGIN
+    parity.MARGIN = FUSED_MARGIN
+    try:
+        wl = workloads.Workload(w.name, w.batch, w.gamma, w.vocab, "f32", w.temperature,
+                                np.zeros((w.batch, w.gamma + 1, 1), np.float32),
+                                np.zeros((w.batch, w.gamma, 1), np.float32), w.tokens,
+                                w.u_accept, w.u_resample)
+        s = compare(wl, g, o)
+    finally:
+        parity.MARGIN = old
+    print(f"\n[{name}] seqs={s['sequences']} hard={len(s['hard'])} margin={len(s['margin_cases'])} "
+          f"dq={s.get('max_dq')} dp={s.get('max_dp')} lseT={s.get('max_target_lse_abs')} "
+          f"lseD={s.get('max_draft_lse_abs')} dz={s.get('max_dz')}")
+    assert not s["hard"], s["hard"][:5]
+    assert len(s["margin_cases"]) <= max(1, 0.05 * s["sequences"]), s
+    for k in ("max_dq", "max_dp", "max_dz"):
+        if k in s:
+            assert s[k] <= FUSED_PROB_TOL, s
+    for k in ("max_target_lse_abs", "max_draft_lse_abs"):
+        if k in s:
+            assert s[k] <= FUSED_LSE_TOL, s
+    return g, o, s
+
+
+@pytest.mark.parametrize("rows,hidden,vocab", [(200, 64, 1000), (300, 1024, 5003), (130, 4096, 32000)])
+def test_gemm_against_float64_logits(rows, hidden, vocab):
+    from speculative_decoding_verification_90_b200.specverify import LmHeadVerify
+    import oracle
+    rng = np.random.default_rng(rows + hidden)
+    h = workloads.bf16_bits(rng.standard_normal((rows, hidden)).astype(np.float32))
+    wt = workloads.bf16_bits((rng.standard_normal((vocab, hidden)) * 3 / np.sqrt(hidden)).astype(np.float32))
+    out = torch.full((rows, vocab), float("nan"), device="cuda")
+    with LmHeadVerify(1, 1, vocab, hidden) as lm:
+        lm.logits(_bf(h), _bf(wt), out)
+        torch.cuda.synchronize()
+        assert lm.status()[0] == 0
+    hf, wf = workloads.bits_to_f32(h), workloads.bits_to_f32(wt)
+    ref = oracle.lm_logits(hf, wf)
+    scale = np.abs(hf).astype(np.float64) @ np.abs(wf).astype(np.float64).T
+    err = np.abs(out.cpu().numpy().astype(np.float64) - ref) / scale
+    assert not np.isnan(err).any()
+    print(f"\n[gemm {rows}x{hidden}x{vocab}] max error / scale = {err.max():.3e}")
+    assert err.max() <= GEMM_REL
+
+
+@pytest.mark.parametrize("B,G,V,D,shared", [
+    (8, 4, 32000, 1024, True),
+    (5, 3, 5003, 256, False),     # ragged vocabulary, two output layers
+    (3, 0, 2000, 128, True),      # bonus draw only
+    (6, 9, 1000, 64, True),       # the smallest hidden size
+])
+def test_fused_parity(B, G, V, D, shared):
+    w = workloads.lmhead(seed=B + G + V, batch=B, gamma=G, vocab=V, hidden=D, shared_weight=shared)
+    g, o, s = _parity(w, f"fused B={B} G={G} V={V} D={D} shared={shared}")
+    assert g["status"] == 0
+
+
+def test_fused_parity_full_size():
+    """64 sequences, gamma 8, V = 128256, hidden 4096 (the benchmark case)."""
+    w = workloads.lmhead()
+    g, o, s = _parity(w, "fused full size")
+    assert g["status"] == 0
+
+
+def test_fused_token_range_and_repeat():
+    from speculative_decoding_verification_90_b200.specverify import LmHeadVerify
+    w = workloads.lmhead(seed=5, batch=6, gamma=3, vocab=3000, hidden=128)
+    w.tokens[2, 1] = 3000
+    with LmHeadVerify(w.batch, w.gamma, w.vocab, w.hidden) as lm:
+        a = run_fused(w, lm)
+        b = run_fused(w, lm)
+    assert a["status"] == 16 and a["bits"] & 1
+    assert a["out_num_accepted"][2] == 0 and (a["out_tokens"][2] == -1).all()
+    np.testing.assert_array_equal(a["out_tokens"], b["out_tokens"])
+
+
+def test_fused_invalid_arguments():
+    from speculative_decoding_verification_90_b200 import specverify as m
+    for args in ((2, 2, 1000, 100), (2, 2, 1000, 0), (0, 2, 1000, 64), (2, 2, 0, 64)):
+        with pytest.raises(m.SpecVerifyError):
+            m.specverify_lmhead_create(*args, 0)
+    with m.LmHeadVerify(2, 1, 500, 64) as lm:
+        ht = torch.zeros((2, 2, 64), dtype=torch.bfloat16, device="cuda")
+        wt = torch.zeros((500 * 64 + 8,), dtype=torch.bfloat16, device="cuda")
+        tok = torch.zeros((2, 1), dtype=torch.int32, device="cuda")
+        ua = torch.zeros((2, 1), device="cuda")
+        ur = torch.zeros((2,), device="cuda")
+        ot = torch.zeros((2, 2), dtype=torch.int32, device="cuda")
+        on = torch.zeros((2,), dtype=torch.int32, device="cuda")
+        # a weight pointer that is not 16-byte aligned
+        assert m._lib.specverify_lmhead_run(lm.handle, ht.data_ptr(), wt.data_ptr() + 2,
+                                            ht.data_ptr(), wt.data_ptr(), tok.data_ptr(),
+                                            ua.data_ptr(), ur.data_ptr(), ctypes.c_float(1.0),
+                                            ot.data_ptr(), on.data_ptr(), None) == m.SV_ERR_INVALID_ARG
+        assert m._lib.specverify_lmhead_run(lm.handle, ht.data_ptr(), wt.data_ptr(),
+                                            ht.data_ptr(), wt.data_ptr(), tok.data_ptr(),
+                                            ua.data_ptr(), ur.data_ptr(), ctypes.c_float(0.0),
+                                            ot.data_ptr(), on.data_ptr(), None) == m.SV_ERR_INVALID_ARG
