@@ -20,7 +20,9 @@ reported under "shared_rows".  The fold gate (relative hidden-state difference
 per branch and position, provenance, packing of the rows to recompute) is
 timed on 128 sequences x 8 branches x 32 positions x 4096 bf16 hidden states,
 reported under "specfold_gate".  The sampling-variant entry point (greedy;
-top-k 50 with top-p 0.9) is timed on the same batch under "sampling_variants".
+top-k 50 with top-p 0.9) is timed on the same batch under "sampling_variants",
+and the step fused with a 128256 x 4096 LM head on tensor cores (64
+sequences, gamma 8) under "lmhead_fused".
 
 N > 1 runs under torch.distributed.run, one rank per GPU: every rank verifies
 its own batch (weak scaling, no data-path collective).  ``--impl reference``
@@ -73,6 +75,8 @@ def parse():
                     help="skip the timing of the shared-row entry point (multibranch)")
     ap.add_argument("--no-sampling", action="store_true",
                     help="skip the timing of the sampling variants (greedy, top-k + top-p)")
+    ap.add_argument("--no-lmhead", action="store_true",
+                    help="skip the timing of the LM-head-fused step (64 x 8, V 128256, d 4096)")
     ap.add_argument("--no-gate", action="store_true",
                     help="skip the timing of the fold gate (128 x 8 branches, 32 x 4096 bf16)")
     return ap.parse_args()
@@ -383,6 +387,7 @@ def run_ours(args):
         shared = time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local)
     sv.close()
     gate = None if args.no_gate else time_gate(args, dev, world, local)
+    lmh = None if args.no_lmhead else time_lmhead(args, dev, world, local)
     # tokens settled per step on this rank = accepted + 1 per sequence (last device step)
     emitted = int((out_n.cpu().numpy().astype(np.int64) + 1).sum())
 
@@ -429,6 +434,8 @@ def run_ours(args):
         }
         if gate is not None:
             line["specfold_gate"] = gate_summary(gate, peak)
+        if lmh is not None:
+            line["lmhead_fused"] = lmhead_summary(lmh)
         if sampling is not None:
             line["sampling_variants"] = {
                 name: {"entry": "specverify_run_sampling", "settings": v["settings"],
@@ -536,6 +543,86 @@ def time_sampling(args, wl, sv, sets, n_sets, out_t, out_n, dev, world, local):
                      "select_us": 1e3 * kern["stats_ms"], "decide_and_draw_us": 1e3 * kern["draw_ms"],
                      "status": st}
     return res
+
+
+def bf16_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d["bf16_tflops_sustained"]), "measured"
+    except Exception:
+        return 1590.0, 1400.0, "fallback (1.59 PFLOP/s burst, 1.4 sustained)"
+
+
+def time_lmhead(args, dev, world, local):
+    """Time the verification step fused with the LM head (every rank its own copy)."""
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_verification_90_b200.specverify import LmHeadVerify
+    w = workloads.lmhead(seed=svdist.rank_seed(args.seed, svdist.env_rank()[0]))
+
+    def bf(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+
+    ht, wt, hd = bf(w.target_hidden), bf(w.target_weight), bf(w.draft_hidden)
+    wd = wt if w.draft_weight is w.target_weight else bf(w.draft_weight)
+    tok = torch.from_numpy(w.tokens).to(dev)
+    ua = torch.from_numpy(w.u_accept).to(dev)
+    ur = torch.from_numpy(w.u_resample).to(dev)
+    B, G = w.batch, w.gamma
+    ot = torch.empty((B, G + 1), dtype=torch.int32, device=dev)
+    on = torch.empty((B,), dtype=torch.int32, device=dev)
+    lm = LmHeadVerify(B, G, w.vocab, w.hidden, local)
+
+    def step():
+        lm.run(ht, wt, hd, wd, tok, ua, ur, w.temperature, ot, on)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(5, min(args.steps, 50))
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lm.profile_begin(steps)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    kern = lm.profile_end()
+    ms_max = svdist.max_over_ranks(ev0.elapsed_time(ev1), device=dev)
+    st, _ = lm.status()
+    lm.close()
+    rows = B * (2 * G + 1)
+    return {"workload": w.name, "steps": steps, "ms_max": ms_max, "stats_ms": kern["stats_ms"],
+            "rest_ms": kern["rest_ms"], "positions": B * G * world,
+            "stats_flops": 2.0 * rows * w.vocab * w.hidden,
+            "draw_flops": 2.0 * 2 * B * w.vocab * w.hidden,
+            "weight_bytes": w.vocab * w.hidden * 2 * (1 if w.draft_weight is w.target_weight else 2),
+            "status": st}
+
+
+def lmhead_summary(g):
+    peak, peak_sus, src = bf16_peak()
+    ms = g["ms_max"] / g["steps"]
+    stats_tf = g["stats_flops"] / (g["stats_ms"] / 1e3) / 1e12
+    step_tf = (g["stats_flops"] + g["draw_flops"]) / (ms / 1e3) / 1e12
+    return {
+        "workload": g["workload"], "entry": "specverify_lmhead_run",
+        "value": g["positions"] / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+        "roofline": {"bound": "tensor", "kernel": "LM-head statistics GEMMs (tcgen05)",
+                     "achieved": stats_tf, "peak": peak, "unit": "TFLOP/s",
+                     "frac": stats_tf / peak, "peak_source": f"{src} bf16 (burst)",
+                     "algorithmic_flops_per_step": g["stats_flops"]},
+        "step_tflops": step_tf,
+        "stats_gemm_us": 1e3 * g["stats_ms"], "rest_us": 1e3 * g["rest_ms"],
+        "logits_written_per_step": "only the 2 drawn rows per sequence (fp32)",
+        "status_after": g["status"],
+    }
 
 
 def time_gate(args, dev, world, local):

@@ -17,7 +17,7 @@
  * target and draft rows at the first rejection, or the bonus row) are
  * recomputed as fp32 logits for the draw.
  *
- * Shapes: hidden is a multiple of 64 (<= 65536); vocab <= 2^24.  Layouts
+ * Shapes: hidden is a multiple of 64 (<= 65536); vocab <= 65535 x 256.  Layouts
  * (device pointers, 16-byte aligned, row-major, contiguous):
  *   target_hidden [batch, gamma+1, hidden] bf16;  target_weight [vocab, hidden] bf16
  *   draft_hidden  [batch, gamma, hidden]   bf16;  draft_weight  [vocab, hidden] bf16

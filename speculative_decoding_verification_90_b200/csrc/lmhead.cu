@@ -4,7 +4,8 @@
 // stream-ordered launches of one step:
 //   1. statistics GEMMs (target rows, then draft rows): per-(row, vocabulary
 //      tile) softmax partials and the logits at the draft tokens;
-//   2. the decide kernel of the plain step on those partials;
+//   2. the per-tile partials folded to one per row, and the decide kernel of
+//      the plain step on them;
 //   3. a gather of the two hidden rows each sequence draws from;
 //   4. logit GEMMs for those rows (fp32, [batch, vocab] each);
 //   5. the draw kernel of the plain step on them.
@@ -41,7 +42,8 @@ struct specverify_lmhead_ctx {
   int num_sms = 148;
   int draw_slices = 1;
   void* ws = nullptr;
-  RowPartial* partial = nullptr;
+  RowPartial* partial = nullptr;   // [(nT + nD) * ntiles] one per row and 256-column tile
+  RowPartial* combined = nullptr;  // [nT + nD] one per row
   float* gathered = nullptr;   // [nT + nD]
   RowStat* tstat = nullptr;
   RowStat* dstat = nullptr;
@@ -98,16 +100,19 @@ bool make_map(CUtensorMap* map, const void* base, long rows, int cols, int box_r
 
 bool aligned16(const void* p) { return reinterpret_cast<uintptr_t>(p) % 16 == 0; }
 
+// ma: the first hidden tensor (p.rows rows); ma2: the second (p.rows2 rows,
+// statistics mode only; pass ma again when there is none); mb: the weight
 template <int kMode>
-cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb, const lmhead::LmParams& p,
-                        cudaStream_t s) {
+cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& ma2, const CUtensorMap& mb,
+                        const lmhead::LmParams& p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(lmhead::gemm_kernel<kMode>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        lmhead::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>(p.ntiles),
-                  static_cast<unsigned>((p.rows + lmhead::kBM - 1) / lmhead::kBM));
-  lmhead::gemm_kernel<kMode><<<grid, lmhead::kThreads, lmhead::kSmemBytes, s>>>(ma, mb, p);
+  const int tiles = (p.rows + lmhead::kBM - 1) / lmhead::kBM +
+                    (p.rows2 + lmhead::kBM - 1) / lmhead::kBM;
+  const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(p.ntiles));
+  lmhead::gemm_kernel<kMode><<<grid, lmhead::kThreads, lmhead::kSmemBytes, s>>>(ma, ma2, mb, p);
   return cudaGetLastError();
 }
 
@@ -128,6 +133,28 @@ __global__ void gather_rows_kernel(const __nv_bfloat16* ht, const __nv_bfloat16*
     uint4* dd = reinterpret_cast<uint4*>(xd + static_cast<long>(b) * hidden);
     for (int g = threadIdx.x; g < groups; g += blockDim.x) dd[g] = sd[g];
   }
+}
+
+// one warp per row: the row's per-tile partials (o_t, s_t) folded into one,
+// O = max o_t, S = sum s_t 2^(o_t - O) in fp64 (a NaN partial stays visible)
+__global__ void __launch_bounds__(256) combine_rows_kernel(const RowPartial* in, int ntiles,
+                                                           long rows, RowPartial* out) {
+  const int lane = threadIdx.x & 31;
+  const long r = static_cast<long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  if (r >= rows) return;
+  const RowPartial* p = in + r * ntiles;
+  float O = -INFINITY;
+  for (int t = lane; t < ntiles; t += 32) O = fmaxf(O, p[t].o);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) O = fmaxf(O, __shfl_xor_sync(0xffffffffu, O, o));
+  double S = 0.0;
+  for (int t = lane; t < ntiles; t += 32) {
+    const RowPartial q = p[t];
+    S += (q.o == -INFINITY) ? q.s * 0.0 : q.s * exp2(static_cast<double>(q.o) - O);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) S += __shfl_xor_sync(0xffffffffu, S, o);
+  if (lane == 0) out[r] = RowPartial{S, O, 0};
 }
 
 template <typename K>
@@ -154,7 +181,7 @@ sv_status specverify_lmhead_create(specverify_lmhead_t* out, int batch, int gamm
   if (!out) return SV_ERR_INVALID_ARG;
   *out = nullptr;
   if (batch < 1 || gamma < 0 || gamma > specverify::kMaxGamma || vocab < 1 ||
-      vocab > (1 << 24) || hidden < lmhead::kBK || hidden % lmhead::kBK != 0 || hidden > (1 << 16))
+      vocab > 65535 * lmhead::kBN || hidden < lmhead::kBK || hidden % lmhead::kBK != 0 || hidden > (1 << 16))
     return SV_ERR_INVALID_ARG;
   const long nT = static_cast<long>(batch) * (gamma + 1), nD = static_cast<long>(batch) * gamma;
   if (nT + nD > (1L << 30)) return SV_ERR_INVALID_ARG;
@@ -207,6 +234,7 @@ sv_status specverify_lmhead_create(specverify_lmhead_t* out, int batch, int gamm
     return at;
   };
   const size_t oP = take(static_cast<size_t>(nT + nD) * h->ntiles * sizeof(RowPartial));
+  const size_t oM = take(static_cast<size_t>(nT + nD) * sizeof(RowPartial));
   const size_t oG = take(static_cast<size_t>(nT + nD) * sizeof(float));
   const size_t oT = take(static_cast<size_t>(nT) * sizeof(RowStat));
   const size_t oD = take(static_cast<size_t>(nD > 0 ? nD : 1) * sizeof(RowStat));
@@ -228,6 +256,7 @@ sv_status specverify_lmhead_create(specverify_lmhead_t* out, int batch, int gamm
   }
   char* b = static_cast<char*>(h->ws);
   h->partial = reinterpret_cast<RowPartial*>(b + oP);
+  h->combined = reinterpret_cast<RowPartial*>(b + oM);
   h->gathered = reinterpret_cast<float*>(b + oG);
   h->tstat = reinterpret_cast<RowStat*>(b + oT);
   h->dstat = reinterpret_cast<RowStat*>(b + oD);
@@ -271,7 +300,7 @@ sv_status specverify_lmhead_logits(specverify_lmhead_t h, const void* hidden_row
   p.ntiles = h->ntiles;
   p.logits = out_logits;
   p.error = h->gemm_error;
-  cudaError_t e = launch_gemm<lmhead::kModeLogits>(ma, mb, p, static_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_gemm<lmhead::kModeLogits>(ma, ma, mb, p, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e);
   return SV_OK;
 }
@@ -330,12 +359,21 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   g.rows = static_cast<int>(nT);
   g.row_offset = 0;
   g.positions = G + 1;
-  if (e == cudaSuccess) e = launch_gemm<lmhead::kModeStats>(mht, mwt, g, s);
-  if (G > 0) {
-    g.rows = static_cast<int>(nD);
-    g.row_offset = nT;
-    g.positions = G;
-    if (e == cudaSuccess) e = launch_gemm<lmhead::kModeStats>(mhd, mwd, g, s);
+  g.rows2 = 0;
+  if (G > 0 && draft_weight == target_weight) {
+    // one output layer: target and draft rows in one launch, the weight read once
+    g.rows2 = static_cast<int>(nD);
+    g.row_offset2 = nT;
+    g.positions2 = G;
+    if (e == cudaSuccess) e = launch_gemm<lmhead::kModeStats>(mht, mhd, mwt, g, s);
+  } else {
+    if (e == cudaSuccess) e = launch_gemm<lmhead::kModeStats>(mht, mht, mwt, g, s);
+    if (G > 0) {
+      g.rows = static_cast<int>(nD);
+      g.row_offset = nT;
+      g.positions = G;
+      if (e == cudaSuccess) e = launch_gemm<lmhead::kModeStats>(mhd, mhd, mwd, g, s);
+    }
   }
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
 
@@ -352,7 +390,7 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   p.u_resample = u_resample;
   p.out_tokens = out_tokens;
   p.out_num_accepted = out_num_accepted;
-  p.partial = h->partial;
+  p.partial = h->combined;
   p.tstat = h->tstat;
   p.dstat = h->dstat;
   p.pos = h->pos;
@@ -364,7 +402,7 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   p.batch = B;
   p.gamma = G;
   p.vocab = V;
-  p.slices = h->ntiles;
+  p.slices = 1;  // the per-tile partials are folded first
   p.groups_per_slice = 0;
   p.draw_slices = h->draw_slices;
   {
@@ -378,6 +416,11 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   p.gathered_target = h->gathered;
   p.gathered_draft = h->gathered + nT;
   p.draw_compact = 1;
+  if (e == cudaSuccess) {
+    combine_rows_kernel<<<static_cast<unsigned>((nT + nD + 7) / 8), 256, 0, s>>>(
+        h->partial, h->ntiles, nT + nD, h->combined);
+    e = cudaGetLastError();
+  }
   const int per = specverify::kDecideThreads / specverify::kWarp;
   if (e == cudaSuccess)
     e = launch_plain(specverify::decide_kernel<float>, static_cast<unsigned>((B + per - 1) / per),
@@ -397,10 +440,17 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   l.ntiles = h->ntiles;
   l.error = h->gemm_error;
   l.logits = h->lt;
-  if (e == cudaSuccess) e = launch_gemm<lmhead::kModeLogits>(mxt, mwt, l, s);
-  if (G > 0) {
-    l.logits = h->ld;
-    if (e == cudaSuccess) e = launch_gemm<lmhead::kModeLogits>(mxd, mwd, l, s);
+  if (G > 0 && draft_weight == target_weight) {
+    // one output layer: both drawn rows of every sequence in one launch
+    l.rows2 = B;
+    l.logits2 = h->ld;
+    if (e == cudaSuccess) e = launch_gemm<lmhead::kModeLogits>(mxt, mxd, mwt, l, s);
+  } else {
+    if (e == cudaSuccess) e = launch_gemm<lmhead::kModeLogits>(mxt, mxt, mwt, l, s);
+    if (G > 0) {
+      l.logits = h->ld;
+      if (e == cudaSuccess) e = launch_gemm<lmhead::kModeLogits>(mxd, mxd, mwd, l, s);
+    }
   }
 
   // 5. the draw on fp32 rows

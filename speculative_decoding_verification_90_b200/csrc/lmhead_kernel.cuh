@@ -45,7 +45,10 @@ constexpr unsigned kSpinLimit = 1u << 20;  // tries per wait (well under a secon
 enum : int { kModeStats = 0, kModeLogits = 1 };
 
 struct LmParams {
-  int rows;                 // M: rows of hidden
+  int rows;                 // M: rows of hidden (the first segment)
+  int rows2;                // rows of the second hidden tensor (statistics mode; 0: none)
+  long row_offset2;         // its first row in the partial / gathered arrays
+  int positions2;           // its positions per sequence (rows of one sequence)
   int vocab;                // N: rows of weight
   int hidden;               // K (a multiple of 64)
   int ntiles;               // vocabulary tiles = ceil(vocab / 256)
@@ -59,6 +62,7 @@ struct LmParams {
   float c_hi, c_lo;
   // logits mode
   float* logits;            // [rows, vocab] fp32
+  float* logits2;           // [rows2, vocab] fp32: the second hidden tensor's
   unsigned* error;          // set when a wait gives up
 };
 
@@ -165,10 +169,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 // the kernel
 // ---------------------------------------------------------------------------
 
+// Grid: x = row tiles of the first hidden tensor, then of the second (which
+// shares the weight), y = vocabulary tiles.  The row tiles of one vocabulary
+// tile run next to each other, so the weight tile comes from HBM once and from
+// L2 for the other rows.
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_hidden,
-                const __grid_constant__ CUtensorMap tm_weight, const LmParams P) {
+                const __grid_constant__ CUtensorMap tm_hidden2,
+                const __grid_constant__ CUtensorMap tm_weight, const LmParams P0) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
@@ -177,8 +186,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   __shared__ int s_failed;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kBN;   // vocabulary tile
-  const int m0 = blockIdx.y * kBM;   // row tile
+  const int tiles1 = (P0.rows + kBM - 1) / kBM;
+  const bool second = static_cast<int>(blockIdx.x) >= tiles1;
+  LmParams P = P0;
+  if (second) {  // the second hidden tensor: its own rows, offset, positions, output
+    P.rows = P0.rows2;
+    P.row_offset = P0.row_offset2;
+    P.positions = P0.positions2;
+    P.logits = P0.logits2;
+  }
+  const CUtensorMap* tm_a = second ? &tm_hidden2 : &tm_hidden;
+  const int vt = blockIdx.y;                                     // vocabulary tile
+  const int n0 = vt * kBN;
+  const int m0 = (second ? static_cast<int>(blockIdx.x) - tiles1 : static_cast<int>(blockIdx.x)) * kBM;
   const int nk = P.hidden / kBK;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -214,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* a = smem + s * kStageBytes;
       uint8_t* b = a + kABytes;
       mbar_expect_tx(&full_bar[s], kStageBytes);
-      tma_load_2d(a, &tm_hidden, &full_bar[s], kt * kBK, m0);
+      tma_load_2d(a, tm_a, &full_bar[s], kt * kBK, m0);
       tma_load_2d(b, &tm_weight, &full_bar[s], kt * kBK, n0);
     }
   } else if (warp == 1 && lane == 0) {
@@ -235,6 +255,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     umma_commit(&accum_bar);  // the accumulator is complete
   }
+  // the other lanes of the producer and MMA warps wait here, not spinning on
+  // the accumulator barrier next to their lane 0 (a diverged warp would
+  // interleave the two paths and slow the pipeline loop)
+  __syncwarp();
 
   // epilogue: all four warps, each its 32 TMEM lanes (rows); the decision to
   // read the accumulator is block-uniform (the loads are warp-collective)
@@ -274,7 +298,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (r < P.rows) {
-        P.partial[(P.row_offset + r) * P.ntiles + blockIdx.x] =
+        P.partial[(P.row_offset + r) * P.ntiles + vt] =
             specverify::RowPartial{static_cast<double>(sum), o, 0};
         if (t >= n0 && t < n0 + kBN) P.gathered[P.row_offset + r] = xt;
       }
