@@ -109,10 +109,12 @@ cudaError_t launch_gemm(const CUtensorMap& ma, const CUtensorMap& ma2, const CUt
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        lmhead::kSmemBytes);
   if (e != cudaSuccess) return e;
-  const int tiles = (p.rows + lmhead::kBM - 1) / lmhead::kBM +
-                    (p.rows2 + lmhead::kBM - 1) / lmhead::kBM;
-  const dim3 grid(static_cast<unsigned>(tiles), static_cast<unsigned>(p.ntiles));
-  lmhead::gemm_kernel<kMode><<<grid, lmhead::kThreads, lmhead::kSmemBytes, s>>>(ma, ma2, mb, p);
+  const long tiles = static_cast<long>((p.rows + lmhead::kBM - 1) / lmhead::kBM +
+                                       (p.rows2 + lmhead::kBM - 1) / lmhead::kBM) *
+                     p.ntiles;
+  const long grid = tiles < p.num_sms ? tiles : p.num_sms;  // persistent: one CTA per SM
+  lmhead::gemm_kernel<kMode><<<static_cast<unsigned>(grid), lmhead::kPThreads,
+                               lmhead::kSmemBytes, s>>>(ma, ma2, mb, p);
   return cudaGetLastError();
 }
 
@@ -298,6 +300,7 @@ sv_status specverify_lmhead_logits(specverify_lmhead_t h, const void* hidden_row
   p.vocab = h->vocab;
   p.hidden = h->hidden;
   p.ntiles = h->ntiles;
+  p.num_sms = h->num_sms;
   p.logits = out_logits;
   p.error = h->gemm_error;
   cudaError_t e = launch_gemm<lmhead::kModeLogits>(ma, ma, mb, p, static_cast<cudaStream_t>(stream));
@@ -349,6 +352,7 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   g.vocab = V;
   g.hidden = D;
   g.ntiles = h->ntiles;
+  g.num_sms = h->num_sms;
   g.partial = h->partial;
   g.tokens = draft_tokens;
   g.token_stride = G;
@@ -438,6 +442,7 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   l.vocab = V;
   l.hidden = D;
   l.ntiles = h->ntiles;
+  l.num_sms = h->num_sms;
   l.error = h->gemm_error;
   l.logits = h->lt;
   if (G > 0 && draft_weight == target_weight) {

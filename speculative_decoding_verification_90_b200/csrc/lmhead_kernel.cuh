@@ -3,12 +3,13 @@
 //
 // logits[r, v] = sum_k hidden[r, k] * weight[v, k]   (bf16 inputs, fp32 accumulation)
 //
-// One CTA computes a 128 x 256 tile of logits (rows x vocabulary): TMA loads
-// 128 x 64 and 256 x 64 bf16 tiles (128-byte swizzle) into a 4-stage ring of
-// shared memory; one thread issues tcgen05.mma (M = 128, N = 256, K = 16) with
-// the accumulator in tensor memory (256 columns); the four warps then read the
-// accumulator back with tcgen05.ld, 32 columns at a time, each warp its 32
-// rows (TMEM lanes).  The epilogue either
+// Persistent CTAs (one per SM) walk 128 x 256 tiles of logits (rows x
+// vocabulary): TMA loads 128 x 64 and 256 x 64 bf16 tiles (128-byte swizzle)
+// into a 4-stage ring of shared memory; one thread issues tcgen05.mma (M = 128,
+// N = 256, K = 16) into one of two 256-column accumulators in tensor memory;
+// four epilogue warps read the other accumulator back with tcgen05.ld, 32
+// columns at a time, each warp its 32 rows (TMEM lanes), while the next
+// tile's MMAs run.  The epilogue either
 //   - folds the tile into per-row softmax statistics (s = sum 2^(x c - o) with
 //     a running offset o, as the streaming statistics kernel does), and picks
 //     out the logit at the row's draft token when the token falls in the tile
@@ -17,7 +18,7 @@
 //
 // Every wait on an mbarrier is bounded: after kSpinLimit tries the thread sets
 // the error flag and leaves the loop, the kernel skips its remaining work, and
-// warp 0 still frees the tensor memory.
+// warp 1 still frees the tensor memory.
 #pragma once
 
 #include <cuda.h>
@@ -34,12 +35,10 @@ constexpr int kBN = 256;     // vocabulary columns per tile (UMMA N)
 constexpr int kBK = 64;      // K per stage: 64 bf16 = one 128-byte swizzle row
 constexpr int kUK = 16;      // K per tcgen05.mma (bf16)
 constexpr int kStages = 4;
-constexpr int kThreads = 128;
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB
 constexpr int kBBytes = kBN * kBK * 2;   // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + room to align to 1024
-constexpr int kTmemCols = 256;
 constexpr unsigned kSpinLimit = 1u << 20;  // tries per wait (well under a second)
 
 enum : int { kModeStats = 0, kModeLogits = 1 };
@@ -52,6 +51,7 @@ struct LmParams {
   int vocab;                // N: rows of weight
   int hidden;               // K (a multiple of 64)
   int ntiles;               // vocabulary tiles = ceil(vocab / 256)
+  int num_sms;              // persistent grid size
   // statistics mode
   specverify::RowPartial* partial;  // [(row_offset + rows) * ntiles]
   long row_offset;
@@ -165,41 +165,104 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // ---------------------------------------------------------------------------
-// the kernel
+// the epilogue of one tile (one warp: its 32 TMEM lanes = rows q*32 .. q*32+31)
 // ---------------------------------------------------------------------------
 
-// Grid: x = row tiles of the first hidden tensor, then of the second (which
-// shares the weight), y = vocabulary tiles.  The row tiles of one vocabulary
-// tile run next to each other, so the weight tile comes from HBM once and from
-// L2 for the other rows.
 template <int kMode>
-__global__ void __launch_bounds__(kThreads, 1)
+__device__ __forceinline__ void epilogue_tile(const LmParams& P, uint32_t acc_addr, int m0, int n0,
+                                              int vt, int q, int lane) {
+  const int r = m0 + q * 32 + lane;
+  const uint32_t lane_addr = acc_addr + (static_cast<uint32_t>(q * 32) << 16);
+  if constexpr (kMode == kModeStats) {
+    int t = -1;
+    if (r < P.rows && P.tokens) {
+      const int pos = r % P.positions, seq = r / P.positions;
+      if (pos < P.token_stride) t = P.tokens[static_cast<long>(seq) * P.token_stride + pos];
+    }
+    float o = -INFINITY, sum = 0.f, xt = 0.f;
+#pragma unroll 1
+    for (int c0 = 0; c0 < kBN; c0 += 32) {
+      float v[32];
+      tmem_ld32(lane_addr + c0, v);
+      float cm = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int col = n0 + c0 + i;
+        if (col >= P.vocab) v[i] = -INFINITY;
+        if (col == t) xt = v[i];
+        cm = fmaxf(cm, v[i]);
+      }
+      const float on = cm * P.c_hi;
+      if (cm != -INFINITY && on > o) {
+        sum *= specverify::ex2(o - on);
+        o = on;
+      }
+      if (o != -INFINITY) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sum += specverify::ex2(specverify::arg2(v[i], P.c_hi, P.c_lo, o));
+      }
+    }
+    if (r < P.rows) {
+      P.partial[(P.row_offset + r) * P.ntiles + vt] =
+          specverify::RowPartial{static_cast<double>(sum), o, 0};
+      if (t >= n0 && t < n0 + kBN) P.gathered[P.row_offset + r] = xt;
+    }
+  } else {
+#pragma unroll 1
+    for (int c0 = 0; c0 < kBN; c0 += 32) {
+      float v[32];
+      tmem_ld32(lane_addr + c0, v);
+      if (r < P.rows) {
+        float* out = P.logits + static_cast<long>(r) * P.vocab + n0 + c0;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (n0 + c0 + i < P.vocab) out[i] = v[i];
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the kernel: persistent, one CTA per SM, tiles in the order (vocabulary tile,
+// row tile) with row tiles fastest, so that concurrently running CTAs share a
+// weight tile through L2
+// ---------------------------------------------------------------------------
+//
+// warp 0 lane 0: TMA producer over a 4-stage ring, continuous across tiles
+// warp 1: allocates 512 TMEM columns (two 256-column accumulators); lane 0
+//         issues the MMAs of tile i into accumulator i % 2 once the epilogue of
+//         tile i - 2 has released it
+// warps 2-5: the epilogue; warp w reads TMEM lanes 32 (w % 4) .. + 31, so the
+//         four cover the 128 rows, while the MMAs of the next tile run
+
+constexpr int kPThreads = 192;
+constexpr int kAccCols = 2 * kBN;
+
+template <int kMode>
+__global__ void __launch_bounds__(kPThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_hidden,
                 const __grid_constant__ CUtensorMap tm_hidden2,
                 const __grid_constant__ CUtensorMap tm_weight, const LmParams P0) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
-  __shared__ __align__(8) uint64_t accum_bar;
+  __shared__ __align__(8) uint64_t tfull_bar[2];
+  __shared__ __align__(8) uint64_t tempty_bar[2];
   __shared__ uint32_t tmem_base_s;
   __shared__ int s_failed;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int tiles1 = (P0.rows + kBM - 1) / kBM;
-  const bool second = static_cast<int>(blockIdx.x) >= tiles1;
-  LmParams P = P0;
-  if (second) {  // the second hidden tensor: its own rows, offset, positions, output
-    P.rows = P0.rows2;
-    P.row_offset = P0.row_offset2;
-    P.positions = P0.positions2;
-    P.logits = P0.logits2;
-  }
-  const CUtensorMap* tm_a = second ? &tm_hidden2 : &tm_hidden;
-  const int vt = blockIdx.y;                                     // vocabulary tile
-  const int n0 = vt * kBN;
-  const int m0 = (second ? static_cast<int>(blockIdx.x) - tiles1 : static_cast<int>(blockIdx.x)) * kBM;
-  const int nk = P.hidden / kBK;
+  const int tiles2 = (P0.rows2 + kBM - 1) / kBM;
+  const int n_rt = tiles1 + tiles2;
+  const long n_tiles = static_cast<long>(n_rt) * P0.ntiles;
+  const int nk = P0.hidden / kBK;
+  volatile int* failed = &s_failed;
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
@@ -208,14 +271,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    mbar_init(&accum_bar, 1);
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull_bar[a], 1);
+      mbar_init(&tempty_bar[a], 4);  // one arrival per epilogue warp
+    }
     s_failed = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 0) {
+  if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                      smem_u32(&tmem_base_s)),
-                 "r"(kTmemCols));
+                 "r"(kAccCols));
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
   }
   tc_fence_before();
@@ -223,107 +289,94 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
 
-  if (warp == 0 && lane == 0) {
-    // producer: TMA loads into the ring
-    for (int kt = 0; kt < nk; ++kt) {
-      const int s = kt % kStages;
-      if (kt >= kStages && !mbar_wait(&empty_bar[s], ((kt / kStages) - 1) & 1)) {
-        s_failed = 1;
-        break;
+  if (warp == 0) {
+    if (lane == 0) {
+      long it = 0;
+      for (long t = blockIdx.x; t < n_tiles && !*failed; t += gridDim.x) {
+        const int rt = static_cast<int>(t % n_rt), vt = static_cast<int>(t / n_rt);
+        const bool second = rt >= tiles1;
+        const CUtensorMap* tm_a = second ? &tm_hidden2 : &tm_hidden;
+        const int m0 = (second ? rt - tiles1 : rt) * kBM, n0 = vt * kBN;
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          const int s = static_cast<int>(it % kStages);
+          if (it >= kStages && !mbar_wait(&empty_bar[s], static_cast<unsigned>((it / kStages) - 1) & 1)) {
+            *failed = 1;
+            break;
+          }
+          uint8_t* a = smem + s * kStageBytes;
+          mbar_expect_tx(&full_bar[s], kStageBytes);
+          tma_load_2d(a, tm_a, &full_bar[s], kt * kBK, m0);
+          tma_load_2d(a + kABytes, &tm_weight, &full_bar[s], kt * kBK, n0);
+        }
       }
-      uint8_t* a = smem + s * kStageBytes;
-      uint8_t* b = a + kABytes;
-      mbar_expect_tx(&full_bar[s], kStageBytes);
-      tma_load_2d(a, tm_a, &full_bar[s], kt * kBK, m0);
-      tma_load_2d(b, &tm_weight, &full_bar[s], kt * kBK, n0);
     }
-  } else if (warp == 1 && lane == 0) {
-    // MMA issuer
-    for (int kt = 0; kt < nk; ++kt) {
-      const int s = kt % kStages;
-      if (!mbar_wait(&full_bar[s], (kt / kStages) & 1)) {
-        s_failed = 1;
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      long it = 0;
+      long i = 0;  // this CTA's tile count
+      for (long t = blockIdx.x; t < n_tiles && !*failed; t += gridDim.x, ++i) {
+        const int acc = static_cast<int>(i & 1);
+        if (i >= 2 && !mbar_wait(&tempty_bar[acc], static_cast<unsigned>((i / 2) - 1) & 1)) {
+          *failed = 1;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + static_cast<uint32_t>(acc * kBN);
+        for (int kt = 0; kt < nk; ++kt, ++it) {
+          const int s = static_cast<int>(it % kStages);
+          if (!mbar_wait(&full_bar[s], static_cast<unsigned>(it / kStages) & 1)) {
+            *failed = 1;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + s * kStageBytes);
+          const uint32_t b = a + kABytes;
+#pragma unroll
+          for (int k = 0; k < kBK / kUK; ++k)
+            umma_f16(d, umma_desc(a + k * kUK * 2), umma_desc(b + k * kUK * 2), kt > 0 || k > 0);
+          umma_commit(&empty_bar[s]);  // the stage is free once these MMAs are done
+        }
+        umma_commit(&tfull_bar[acc]);  // accumulator `acc` holds tile t
+      }
+    }
+    __syncwarp();
+  } else {
+    const int q = warp % 4;  // TMEM lane quarter of this warp
+    long i = 0;
+    for (long t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+      const int acc = static_cast<int>(i & 1);
+      bool ok = mbar_wait(&tfull_bar[acc], static_cast<unsigned>(i / 2) & 1);
+      ok = __all_sync(0xffffffffu, ok) && !*failed;
+      if (!ok) {
+        if (lane == 0) *failed = 1;
         break;
       }
       tc_fence_after();
-      const uint32_t a = smem_u32(smem + s * kStageBytes);
-      const uint32_t b = a + kABytes;
-#pragma unroll
-      for (int k = 0; k < kBK / kUK; ++k)
-        umma_f16(tmem, umma_desc(a + k * kUK * 2), umma_desc(b + k * kUK * 2), kt > 0 || k > 0);
-      umma_commit(&empty_bar[s]);  // the stage is free once these MMAs are done
+      const int rt = static_cast<int>(t % n_rt), vt = static_cast<int>(t / n_rt);
+      const bool second = rt >= tiles1;
+      LmParams P = P0;
+      if (second) {
+        P.rows = P0.rows2;
+        P.row_offset = P0.row_offset2;
+        P.positions = P0.positions2;
+        P.logits = P0.logits2;
+      }
+      epilogue_tile<kMode>(P, tmem + static_cast<uint32_t>(acc * kBN),
+                           (second ? rt - tiles1 : rt) * kBM, vt * kBN, vt, q, lane);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty_bar[acc]);
     }
-    umma_commit(&accum_bar);  // the accumulator is complete
   }
-  // the other lanes of the producer and MMA warps wait here, not spinning on
-  // the accumulator barrier next to their lane 0 (a diverged warp would
-  // interleave the two paths and slow the pipeline loop)
-  __syncwarp();
 
-  // epilogue: all four warps, each its 32 TMEM lanes (rows); the decision to
-  // read the accumulator is block-uniform (the loads are warp-collective)
-  const bool ok = mbar_wait(&accum_bar, 0);
-  const bool good = __syncthreads_and(ok) && !*static_cast<volatile int*>(&s_failed);
-  tc_fence_after();
-  const int r = m0 + warp * 32 + lane;
-  if (good) {
-    const uint32_t lane_addr = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-    if constexpr (kMode == kModeStats) {
-      int t = -1;
-      if (r < P.rows && P.tokens) {
-        const int pos = r % P.positions, seq = r / P.positions;
-        if (pos < P.token_stride) t = P.tokens[static_cast<long>(seq) * P.token_stride + pos];
-      }
-      float o = -INFINITY, sum = 0.f, xt = 0.f;
-#pragma unroll 1
-      for (int c0 = 0; c0 < kBN; c0 += 32) {
-        float v[32];
-        tmem_ld32(lane_addr + c0, v);
-        float cm = -INFINITY;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const int col = n0 + c0 + i;
-          if (col >= P.vocab) v[i] = -INFINITY;
-          if (col == t) xt = v[i];
-          cm = fmaxf(cm, v[i]);
-        }
-        const float on = cm * P.c_hi;
-        if (cm != -INFINITY && on > o) {
-          sum *= specverify::ex2(o - on);
-          o = on;
-        }
-        if (o != -INFINITY) {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sum += specverify::ex2(specverify::arg2(v[i], P.c_hi, P.c_lo, o));
-        }
-      }
-      if (r < P.rows) {
-        P.partial[(P.row_offset + r) * P.ntiles + vt] =
-            specverify::RowPartial{static_cast<double>(sum), o, 0};
-        if (t >= n0 && t < n0 + kBN) P.gathered[P.row_offset + r] = xt;
-      }
-    } else {
-#pragma unroll 1
-      for (int c0 = 0; c0 < kBN; c0 += 32) {
-        float v[32];
-        tmem_ld32(lane_addr + c0, v);
-        if (r < P.rows) {
-          float* out = P.logits + static_cast<long>(r) * P.vocab + n0 + c0;
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (n0 + c0 + i < P.vocab) out[i] = v[i];
-        }
-      }
-    }
-  } else if (threadIdx.x == 0) {
-    atomicOr(P.error, 1u);
-  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (threadIdx.x == 0 && *failed) atomicOr(P0.error, 1u);
+  if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"(kTmemCols));
+                 "r"(kAccCols));
   }
 }
 
