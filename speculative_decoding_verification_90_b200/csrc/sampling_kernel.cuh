@@ -15,12 +15,15 @@
 // the first index of the largest logit.
 //
 // Three stream-ordered kernels:
-//   select_kernel  one block per row: maximum and first argmax; count-based
-//                  radix select of the top-k threshold; for top-p, the entries
-//                  above a count-selected candidate key gathered into shared
-//                  memory and a binary search over keys on their fp64 masses
-//                  (whole-row passes when the boundary lies below the
-//                  candidates); the log-normaliser of the kept entries.
+//   select_kernel  one block per row: one scan for the maximum, the first
+//                  argmax and (top-k <= 256) each thread's four largest values,
+//                  which hold the top-k set whenever no thread's fourth value
+//                  reaches the cut (else a candidate gather or a radix select
+//                  with per-warp histograms); for top-p, candidates with
+//                  double-precision weights in shared memory and a binary
+//                  search over keys on their masses (a mass-histogram digit
+//                  descent when the cut lies below the candidates); the
+//                  log-normaliser of the kept entries.
 //   decide_kernel  one warp per sequence, one lane per position: adjusted
 //                  q(t), p(t), the acceptance test and the first rejection by
 //                  ballot; greedy sequences emit the argmax here.
@@ -151,20 +154,6 @@ __device__ __forceinline__ unsigned block_max_u(unsigned v, unsigned* sm) {
   unsigned t = 0;
 #pragma unroll
   for (int w = 0; w < NT / kWarp; ++w) t = max(t, sm[w]);
-  return t;
-}
-
-template <int NT>
-__device__ __forceinline__ unsigned block_min_u(unsigned v, unsigned* sm) {
-  const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
-  __syncthreads();
-  if (lane == 0) sm[warp] = v;
-  __syncthreads();
-  unsigned t = 0xffffffffu;
-#pragma unroll
-  for (int w = 0; w < NT / kWarp; ++w) t = min(t, sm[w]);
   return t;
 }
 
@@ -392,18 +381,6 @@ __device__ unsigned mass_descent(const T* row, int V, unsigned lo, unsigned hi, 
   *m_gt = d_above;
   *m_ge = d_above + d_bin;
   return d_prefix;
-}
-
-// sum over the row of 2^(x c - o) for entries with key >= lo, per thread in
-// fp32, over the block in fp64
-template <typename T, bool kAligned>
-__device__ double masked_mass(const T* row, int V, unsigned lo, float c_hi, float c_lo, float o,
-                              double* sm) {
-  float s = 0.f;
-  scan_row<T, kAligned, false>(row, V, [&](float x, long) {
-    if (fkey(x) >= lo) s += ex2(specverify::arg2(x, c_hi, c_lo, o));
-  });
-  return block_sum<kSelThreads>(static_cast<double>(s), sm);
 }
 
 // ---------------------------------------------------------------------------
