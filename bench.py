@@ -25,7 +25,9 @@ and the step fused with a 128256 x 4096 LM head on tensor cores (64
 sequences, gamma 8) under "lmhead_fused".
 
 N > 1 runs under torch.distributed.run, one rank per GPU: every rank verifies
-its own batch (weak scaling, no data-path collective).  ``--impl reference``
+its own batch (weak scaling, no data-path collective); the extra measurements
+(shared rows, sampling variants, fold gate, LM-head-fused step) run at N = 1
+only.  ``--impl reference``
 times the CPU oracle on the host cores on a bounded sample of the workload.
 """
 from __future__ import annotations
@@ -376,18 +378,21 @@ def run_ours(args):
     d2h = h_ot.numel() * 4 + h_on.numel() * 4
     st, bits = sv.status()
 
+    # the extra measurements run at one GPU only: a scaling run times the
+    # headline step (each rank would otherwise build every extra workload)
+    extras = world == 1
     # the same batch under sampling variants (separate kernels)
     sampling = None
-    if not args.no_sampling:
+    if extras and not args.no_sampling:
         sampling = time_sampling(args, wl, sv, sets, n_sets, out_t, out_n, dev, world, local)
 
     # the same batch through the shared-row entry point: each distinct row once
     shared = None
-    if wl.mapped and not args.no_shared_rows:
+    if extras and wl.mapped and not args.no_shared_rows:
         shared = time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local)
     sv.close()
-    gate = None if args.no_gate else time_gate(args, dev, world, local)
-    lmh = None if args.no_lmhead else time_lmhead(args, dev, world, local)
+    gate = None if (args.no_gate or not extras) else time_gate(args, dev, world, local)
+    lmh = None if (args.no_lmhead or not extras) else time_lmhead(args, dev, world, local)
     # tokens settled per step on this rank = accepted + 1 per sequence (last device step)
     emitted = int((out_n.cpu().numpy().astype(np.int64) + 1).sum())
 
