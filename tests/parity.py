@@ -19,6 +19,31 @@ import numpy as np
 MARGIN = 1e-6
 PROB_TOL = 1e-5
 LSE_TOL = 1e-5   # absolute, i.e. relative on the normaliser
+# A residual draw is determined at the kernels' precision only when the
+# residual mass Z is well above the rounding of q - p: the fp32 normalisers
+# agree with the oracle's to about 1e-7, so below Z = 1e-6 the residual's
+# relative error passes 10% (the oracle's own Z there is often fp64 rounding,
+# e.g. 1e-80 when q and p are nearly the same point mass).  Such draws are
+# checked for validity only and reported as "unresolved".
+RESID_RESOLVE = 1e-6
+
+
+def _unresolved(ora, b, no, G):
+    return no < G and float(ora["resid_mass"][b]) < RESID_RESOLVE
+
+
+def _valid_draw(tg, no, V, logit_row=None, top_k=0):
+    """The emitted token lies in [0, V), everything after it is -1 and (given the
+    target row) its logit is finite and not below the k-th largest."""
+    tok = int(tg[no])
+    if not (0 <= tok < V) or not (np.asarray(tg[no + 1:]) == -1).all():
+        return False
+    if logit_row is None:
+        return True
+    x = np.asarray(logit_row, np.float32)
+    if not np.isfinite(x[tok]):
+        return False
+    return not (0 < top_k < V) or x[tok] >= np.partition(x, V - top_k)[V - top_k]
 
 
 def to_device(wl, device=0):
@@ -95,7 +120,7 @@ def compare(wl, gpu, ora, seqs=None, check_probs=True):
     """Decision parity over the sequences `seqs` (default: all).  Returns a summary dict."""
     B, G = wl.batch, wl.gamma
     seqs = np.arange(B) if seqs is None else np.asarray(seqs)
-    hard, margin_cases = [], []
+    hard, margin_cases, unresolved = [], [], []
     for b in seqs:
         ng, no = int(gpu["out_num_accepted"][b]), int(ora["out_num_accepted"][b])
         tg, to = gpu["out_tokens"][b], ora["out_tokens"][b]
@@ -109,10 +134,16 @@ def compare(wl, gpu, ora, seqs=None, check_probs=True):
             (margin_cases if m < MARGIN else hard).append((int(b), "accept", j, float(m)))
             continue
         if not np.array_equal(tg, to):
+            if _unresolved(ora, b, no, G):
+                ok_draw = np.array_equal(tg[:no], to[:no]) and _valid_draw(tg, no, wl.vocab)
+                (unresolved if ok_draw else hard).append(
+                    (int(b), "unresolved draw", int(tg[no]), int(to[no]), float(ora["resid_mass"][b])))
+                continue
             m = ora["cdf_margin_norm"][b]
             (margin_cases if m < MARGIN else hard).append(
                 (int(b), "draw", int(tg[no]), int(to[no]), float(m)))
-    summary = {"sequences": int(len(seqs)), "hard": hard, "margin_cases": margin_cases}
+    summary = {"sequences": int(len(seqs)), "hard": hard, "margin_cases": margin_cases,
+               "unresolved": unresolved}
     if check_probs and "q_tok" in gpu:
         ok = ora["seq_status"][seqs] == 0
         s = seqs[ok]
@@ -181,14 +212,20 @@ def oracle_run_sampling(wl, temperatures, top_k=0, top_p=1.0):
                                   top_p=float(np.float32(top_p)), threads=os.cpu_count() or 1)
 
 
-def compare_sampling(wl, gpu, ora):
+def _target_row(wl, b, n):
+    from speculative_decoding_verification_90_b200 import workloads
+    row = wl.target[b, n]
+    return workloads.bits_to_f32(row) if wl.dtype == "bf16" else row
+
+
+def compare_sampling(wl, gpu, ora, top_k=0):
     """Decision parity of the sampling variants.  A sequence with a row whose
     top-p boundary margin (|cumulative mass - top_p| at the chosen cut, relative
     to the kept mass) is below FILTER_MARGIN may cut one group differently: its
     kept counts and probabilities are not compared, and a differing decision
     counts as a margin case.  Everything else must agree as in the plain step."""
     B, G = wl.batch, wl.gamma
-    hard, margin_cases = [], []
+    hard, margin_cases, unresolved = [], [], []
     ok = []
     for b in range(B):
         ng, no = int(gpu["out_num_accepted"][b]), int(ora["out_num_accepted"][b])
@@ -212,10 +249,17 @@ def compare_sampling(wl, gpu, ora):
             (margin_cases if (m < MARGIN or near_cut) else hard).append((b, "accept", j, float(m)))
             continue
         if not np.array_equal(tg, to):
+            if _unresolved(ora, b, no, G):
+                row = _target_row(wl, b, no)
+                ok_draw = np.array_equal(tg[:no], to[:no]) and _valid_draw(tg, no, wl.vocab, row, top_k)
+                (unresolved if ok_draw else hard).append(
+                    (b, "unresolved draw", int(tg[no]), int(to[no]), float(ora["resid_mass"][b])))
+                continue
             m = ora["cdf_margin_norm"][b]
             (margin_cases if (m < MARGIN or near_cut) else hard).append(
                 (b, "draw", int(tg[no]), int(to[no]), float(m)))
     summary = {"sequences": B, "hard": hard, "margin_cases": margin_cases,
+               "unresolved": unresolved,
                "near_cut": int((ora["filter_margin"] < FILTER_MARGIN).sum())}
     s = np.asarray(ok, dtype=np.int64)
     if G > 0 and len(s):
