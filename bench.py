@@ -20,9 +20,9 @@ reported under "shared_rows".  The fold gate (relative hidden-state difference
 per branch and position, provenance, packing of the rows to recompute) is
 timed on 128 sequences x 8 branches x 32 positions x 4096 bf16 hidden states,
 reported under "specfold_gate".  The sampling-variant entry point (greedy;
-top-k 50 with top-p 0.9) is timed on the same batch under "sampling_variants",
-and the step fused with a 128256 x 4096 LM head on tensor cores (64
-sequences, gamma 8) under "lmhead_fused".
+top-k 50 with top-p 0.9; top-p 0.9 alone; top-k 2000 alone) is timed on the
+same batch under "sampling_variants", and the step fused with a 128256 x 4096
+LM head on tensor cores (64 sequences, gamma 8) under "lmhead_fused".
 
 N > 1 runs under torch.distributed.run, one rank per GPU: every rank verifies
 its own batch (weak scaling, no data-path collective); the extra measurements
@@ -77,6 +77,9 @@ def parse():
                     help="skip the timing of the shared-row entry point (multibranch)")
     ap.add_argument("--no-sampling", action="store_true",
                     help="skip the timing of the sampling variants (greedy, top-k + top-p)")
+    ap.add_argument("--sampling", default=None,
+                    help="comma-separated sampling settings to time (greedy, top_k50_top_p0.9, "
+                         "top_p0.9, top_k2000; default: all)")
     ap.add_argument("--no-lmhead", action="store_true",
                     help="skip the timing of the LM-head-fused step (64 x 8, V 128256, d 4096)")
     ap.add_argument("--no-gate", action="store_true",
@@ -513,12 +516,16 @@ def time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local):
 
 
 def time_sampling(args, wl, sv, sets, n_sets, out_t, out_n, dev, world, local):
-    """Time the sampling-variant entry point on the bench batch: greedy, and
-    top-k 50 with top-p 0.9 at the workload's temperature."""
+    """Time the sampling-variant entry point on the bench batch: greedy; top-k
+    50 with top-p 0.9; top-p 0.9 alone; top-k 2000 alone (the last three at the
+    workload's temperature)."""
     import torch
     import torch.distributed as dist
     res = {}
-    configs = {"greedy": (0.0, 0, 1.0), "top_k50_top_p0.9": (wl.temperature, 50, 0.9)}
+    configs = {"greedy": (0.0, 0, 1.0), "top_k50_top_p0.9": (wl.temperature, 50, 0.9),
+               "top_p0.9": (wl.temperature, 0, 0.9), "top_k2000": (wl.temperature, 2000, 1.0)}
+    if args.sampling:
+        configs = {name: configs[name] for name in args.sampling.split(",")}
     for name, (T, k, p) in configs.items():
         temps = torch.full((wl.batch,), T, dtype=torch.float32, device=dev)
 

@@ -18,12 +18,15 @@
 //   select_kernel  one block per row: one scan for the maximum, the first
 //                  argmax and (top-k <= 256) each thread's four largest values,
 //                  which hold the top-k set whenever no thread's fourth value
-//                  reaches the cut (else a candidate gather or a radix select
-//                  with per-warp histograms); for top-p, candidates with
-//                  double-precision weights in shared memory and a binary
-//                  search over keys on their masses (a mass-histogram digit
-//                  descent when the cut lies below the candidates); the
-//                  log-normaliser of the kept entries.
+//                  reaches the cut.  Otherwise a band histogram: one scan
+//                  counts (top-k) or weighs (top-p alone) the entries in bands
+//                  of their distance below the maximum, and a second gathers
+//                  the bands that hold the cut as candidates.  The cuts
+//                  themselves are binary searches over keys on the candidates'
+//                  counts and double-precision masses.  A count radix select
+//                  and a mass-histogram digit descent remain as fallbacks
+//                  (candidates that do not fit; a cut outside them).  Last,
+//                  the log-normaliser of the kept entries.
 //   decide_kernel  one warp per sequence, one lane per position: adjusted
 //                  q(t), p(t), the acceptance test and the first rejection by
 //                  ballot; greedy sequences emit the argmax here.
@@ -41,7 +44,7 @@ using specverify::kWarp;
 
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / kWarp;
-constexpr int kCand = 12288;         // most candidates kept in shared memory
+constexpr int kCand = 12288;         // most candidates kept in shared memory (large top-k sets)
 constexpr int kCandSmem = kCand * 8; // their keys and weights (dynamic shared memory)
 constexpr int kCandSmall = 2048;     // the candidate room of a call whose cuts need no more
 constexpr int kDrawThreads = 512;
@@ -383,6 +386,268 @@ __device__ unsigned mass_descent(const T* row, int V, unsigned lo, unsigned hi, 
   return d_prefix;
 }
 
+// Bands of an entry's distance below the row maximum gmx: j = the nearest
+// integer to min(max((gmx - x) s, 0), kBands - 1), with (gmx - x) s formed as
+// one fused multiply-add and the rounding done by adding 2^23.  Every step is
+// monotone, so j never increases with x and a run of bands is a run of keys;
+// -inf lands in the last band.  s = kBandsPerUnit for counts (bands of 1/32
+// logit) and kBandsPerUnit log2(e)/T for masses (1/32 of a factor 2 in weight).
+constexpr int kBands = 4 * kSelThreads;  // 1024
+constexpr float kBandsPerUnit = 32.f;
+constexpr int kBandCap = kBands * kSelWarps / 2;  // candidate room whose area holds the histograms
+constexpr double kBandSlack = 4e-6;      // relative room around the nucleus goal
+
+__device__ __forceinline__ int band_of(float x, float s, float gs) {
+  const float d = fminf(fmaxf(fmaf(-x, s, gs), 0.f), static_cast<float>(kBands - 1));
+  return __float_as_int(d + 8388608.f) - 0x4b000000;
+}
+
+// Row scan by groups: `f(x, n, i0)` sees the n (0 past the end) elements
+// i0 .. i0 + n - 1 in x[0 .. n); the loop count is the same for every thread
+// of the block, so `f` may use warp collectives.
+template <typename T, bool kAligned>
+struct Groups {
+  static constexpr int kN = kAligned ? Elem<T>::kVec : 1;
+};
+
+template <typename T, bool kAligned, typename F>
+__device__ __forceinline__ void scan_groups(const T* row, int V, F&& f) {
+  constexpr int kN = Groups<T, kAligned>::kN;
+  if constexpr (kAligned) {
+    constexpr int kU = 4;
+    const long groups = V / kN;
+    const uint4* g4 = reinterpret_cast<const uint4*>(row);
+    const long stride = static_cast<long>(blockDim.x) * kU;
+    const long end = ((groups + stride - 1) / stride) * stride;
+    for (long g0 = threadIdx.x; g0 < end; g0 += stride) {
+      uint4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const long g = g0 + static_cast<long>(u) * blockDim.x;
+        if (g < groups) v[u] = __ldg(g4 + g);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const long g = g0 + static_cast<long>(u) * blockDim.x;
+        float x[kN];
+        int n = 0;
+        if (g < groups) {
+          Elem<T>::unpack(v[u], x);
+          n = kN;
+        } else {
+#pragma unroll
+          for (int e = 0; e < kN; ++e) x[e] = 0.f;
+        }
+        f(x, n, g * kN);
+      }
+    }
+  } else {
+    const long end = ((static_cast<long>(V) + blockDim.x - 1) / blockDim.x) * blockDim.x;
+    for (long i = threadIdx.x; i < end; i += blockDim.x) {
+      const int n = i < V ? 1 : 0;
+      float x[1] = {n ? elem<T>(row, i) : 0.f};
+      f(x, n, i);
+    }
+  }
+}
+
+struct BandCut {
+  int lo, hi;         // the bands holding the cut (lo = -1: none found)
+  double end;         // running total (count or mass) through band hi
+  double head, tail;  // mass: of the bands before lo, and after hi
+};
+
+// One scan: per-warp histograms over bands of the entry count (kMass false)
+// or of the fp32 weight 2^(x c - o) (kMass true), in `smem` (kSelWarps x
+// kBands words); then warp 0 walks the bands from the largest values down,
+// each lane over kBands / 32 consecutive bands, and takes the first band where
+// the running total reaches the goal: `goal` entries (count), or `goal` times
+// the row's mass (mass).  With kMass the range spans the bands holding the
+// goal -/+ kBandSlack of the mass (the cut itself is settled later on
+// double-precision candidate weights), and the masses before and after it
+// come from the same histogram.
+template <typename T, bool kAligned, bool kMass>
+__device__ BandCut band_cut(const T* row, int V, float s, float gs, float c_hi, float c_lo,
+                            float o, double goal, unsigned* smem) {
+  float* hw = reinterpret_cast<float*>(smem);
+  int* hc = reinterpret_cast<int*>(smem);
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < kBands * kSelWarps; i += blockDim.x) smem[i] = 0u;
+  __syncthreads();
+  float* hwm = hw + warp * kBands;
+  int* hcm = hc + warp * kBands;
+  // the last band (everything far below the maximum; most of the row at a
+  // low temperature) is summed in registers, not by atomics on one word
+  float last_w = 0.f;
+  int last_c = 0;
+  scan_row<T, kAligned, false>(row, V, [&](float x, long) {
+    const int j = band_of(x, s, gs);
+    if constexpr (kMass) {
+      const float w = ex2(specverify::arg2(x, c_hi, c_lo, o));
+      if (j == kBands - 1) last_w += w;
+      else atomicAdd(hwm + j, w);
+    } else {
+      if (j == kBands - 1) ++last_c;
+      else atomicAdd(hcm + j, 1);
+    }
+  });
+  if constexpr (kMass) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) last_w += __shfl_xor_sync(0xffffffffu, last_w, off);
+    if ((threadIdx.x & (kWarp - 1)) == 0) atomicAdd(hwm + kBands - 1, last_w);
+  } else {
+    last_c = __reduce_add_sync(0xffffffffu, last_c);
+    if ((threadIdx.x & (kWarp - 1)) == 0) atomicAdd(hcm + kBands - 1, last_c);
+  }
+  __syncthreads();
+  // totals over the warps (fp64) into the first kBands doubles of `smem`
+  constexpr int kPerT = kBands / kSelThreads;
+  const int b0 = kPerT * threadIdx.x;
+  double a[kPerT];
+#pragma unroll
+  for (int e = 0; e < kPerT; ++e) {
+    a[e] = 0.0;
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w)
+      a[e] += kMass ? static_cast<double>(hw[w * kBands + b0 + e])
+                    : static_cast<double>(hc[w * kBands + b0 + e]);
+  }
+  __syncthreads();
+  double* tot = reinterpret_cast<double*>(smem);
+#pragma unroll
+  for (int e = 0; e < kPerT; ++e) tot[b0 + e] = a[e];
+  __syncthreads();
+  __shared__ BandCut s_bc;
+  if (threadIdx.x < kWarp) {
+    constexpr int kPer = kBands / kWarp;
+    const int lane = threadIdx.x;
+    const double* mine = tot + lane * kPer;
+    double sl = 0.0;
+#pragma unroll 8
+    for (int i = 0; i < kPer; ++i) sl += mine[i];
+    double incl = sl;
+#pragma unroll
+    for (int off = 1; off < kWarp; off <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    // each lane's bands run from the previous lane's end to its own, so the
+    // lanes' intervals chain and cover (0, total]
+    double start = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) start = 0.0;
+    const double total = __shfl_sync(0xffffffffu, incl, kWarp - 1);
+    const double g = kMass ? goal * total : goal;
+    const double slack = kMass ? kBandSlack * total : 0.0;
+    // first band j with end(j - 1) < h <= end(j); its start and end
+    auto find = [&](double h, double* s_out, double* e_out) -> int {
+      int found = -1;
+      double fs = 0.0, fe = 0.0, cum = start;
+      for (int i = 0; i < kPer; ++i) {
+        const double nxt = (i == kPer - 1) ? incl : cum + mine[i];
+        if (found < 0 && cum < h && h <= nxt) {
+          found = lane * kPer + i;
+          fs = cum;
+          fe = nxt;
+        }
+        cum = nxt;
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, found >= 0);
+      if (!m) return -1;
+      const int l = __ffs(m) - 1;
+      *s_out = __shfl_sync(0xffffffffu, fs, l);
+      *e_out = __shfl_sync(0xffffffffu, fe, l);
+      return __shfl_sync(0xffffffffu, found, l);
+    };
+    double s_lo = 0.0, e_lo = 0.0, s_hi = 0.0, e_hi = 0.0;
+    const double h_lo = g - slack;
+    int lo = h_lo <= 0.0 ? 0 : find(h_lo, &s_lo, &e_lo);
+    const int hi = find(fmin(g + slack, total), &s_hi, &e_hi);
+    if (hi < 0 || lo > hi) lo = -1;
+    if (lane == 0) s_bc = BandCut{lo, hi, e_hi, s_lo, fmax(total - e_hi, 0.0)};
+  }
+  __syncthreads();
+  return s_bc;
+}
+
+struct BandGather {
+  int n;                   // entries in the bands (may exceed the room)
+  unsigned kmin, kmax;     // their smallest and largest keys
+  unsigned hkmin;          // smallest key of the entries in earlier bands
+  double head, nhead;      // mass (fp64 weights 2^(x c - od)) and count of those entries
+};
+
+// Candidates: the entries in bands [j_lo, j_hi], keys into shared memory and
+// then their weights in double precision (rounded to float).  With kHead also
+// the count and smallest key of the entries in earlier bands (larger values).
+// One vote per group of elements: most groups hold no candidate.
+template <typename T, bool kAligned, bool kHead>
+__device__ BandGather gather_bands(const T* row, int V, float s, float gs, int j_lo, int j_hi,
+                                   double c, double od, unsigned* cand_key, float* cand_w,
+                                   int* cand_n, double* smd, unsigned* smu, int cap) {
+  constexpr int kN = Groups<T, kAligned>::kN;
+  const int lane = threadIdx.x & (kWarp - 1);
+  if (threadIdx.x == 0) *cand_n = 0;
+  __syncthreads();
+  int nh = 0;
+  unsigned kmx = 0u, nkmn = 0u, nhk = 0u;  // maxima of k, ~k, ~k
+  scan_groups<T, kAligned>(row, V, [&](const float* x, int n, long) {
+    unsigned tmask = 0u;
+    unsigned key[kN];
+#pragma unroll
+    for (int e = 0; e < kN; ++e) {
+      key[e] = fkey(x[e]);
+      if (e < n) {
+        const int j = band_of(x[e], s, gs);
+        if (j >= j_lo && j <= j_hi) {
+          tmask |= 1u << e;
+          kmx = max(kmx, key[e]);
+          nkmn = max(nkmn, ~key[e]);
+        }
+        if (kHead && j < j_lo) {
+          ++nh;
+          nhk = max(nhk, ~key[e]);
+        }
+      }
+    }
+    if (__any_sync(0xffffffffu, tmask != 0u)) {
+      // the lanes' takes in lane order: a warp scan of their counts, one
+      // shared atomic for the warp's run of slots
+      const int cnt = __popc(tmask);
+      int incl = cnt;
+#pragma unroll
+      for (int off = 1; off < kWarp; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      int base = 0;
+      if (lane == kWarp - 1) base = atomicAdd(cand_n, incl);
+      int slot = __shfl_sync(0xffffffffu, base, kWarp - 1) + incl - cnt;
+#pragma unroll
+      for (int e = 0; e < kN; ++e) {
+        if ((tmask >> e) & 1u) {
+          if (slot < cap) cand_key[slot] = key[e];
+          ++slot;
+        }
+      }
+    }
+  });
+  __syncthreads();
+  BandGather out;
+  out.n = *cand_n;
+  for (int i = threadIdx.x; i < min(out.n, cap); i += blockDim.x)
+    cand_w[i] = static_cast<float>(exp2(static_cast<double>(key_value(cand_key[i])) * c - od));
+  out.kmax = block_max_u<kSelThreads>(kmx, smu);
+  out.kmin = ~block_max_u<kSelThreads>(nkmn, smu);
+  out.head = 0.0;
+  out.nhead = 0.0;
+  out.hkmin = 0u;
+  if constexpr (kHead) {
+    out.nhead = block_sum<kSelThreads>(static_cast<double>(nh), smd);
+    out.hkmin = ~block_max_u<kSelThreads>(nhk, smu);
+  }
+  return out;
+}
+
 // ---------------------------------------------------------------------------
 // kernel 1: per-row adjusted distribution
 // ---------------------------------------------------------------------------
@@ -457,7 +722,8 @@ struct CandSet {
   double n_eq;      // entries equal to `above` (not stored; one weight)
   double w_above;
   double tail;      // mass of the entries theta <= key < above
-  unsigned kmax, step;
+  unsigned kmax, step;  // largest candidate key; spacing of keys
+  double head, nhead;   // mass and count of entries above every candidate (not stored)
 };
 
 struct StageOut {
@@ -465,7 +731,8 @@ struct StageOut {
   float margin;
   double Z, kept;   // mass (when z_valid) and count (when kept_valid) of the kept set
   double Zk, goal, m0;  // for the whole-row fallback, when below
-  int z_valid, kept_valid, below;
+  int z_valid, kept_valid;
+  int below;        // 1: the nucleus cut lies below the candidates; 2: above them
 };
 
 // The top-k cut (when `do_k`: the k-th largest candidate key, searched from
@@ -487,12 +754,13 @@ __device__ void cand_stage(const Red<kW>& R, const CandSet& cs, bool do_k, int t
     }
     theta = lo;
   }
-  // M(>= v): candidates >= max(v, theta), plus the group at `above`
+  // M(>= v) for v up to the largest candidate: candidates >= max(v, theta),
+  // the group at `above`, and the entries above every candidate
   auto mass_ge = [&](unsigned v) -> double {
     double sv = 0.0;
     for (int i = f; i < cs.n; i += st)
       if (cs.key[i] >= v && cs.key[i] >= theta) sv += static_cast<double>(cs.w[i]);
-    double t = R.sum(sv);
+    double t = R.sum(sv) + cs.head;
     if (v <= cs.above && cs.above >= theta) t += cs.n_eq * cs.w_above;
     return t;
   };
@@ -505,7 +773,9 @@ __device__ void cand_stage(const Red<kW>& R, const CandSet& cs, bool do_k, int t
     o.Zk = Zk;
     o.goal = goal;
     o.m0 = m0;
-    if (m0 >= goal) {
+    if (cs.head > 0.0 && cs.head >= goal) {
+      o.below = 2;
+    } else if (m0 >= goal) {
       unsigned lo = v0, hi = cs.kmax;
       while (lo < hi) {
         const unsigned mid = lo + (((hi - lo) / step + 1) / 2) * step;
@@ -513,23 +783,24 @@ __device__ void cand_stage(const Red<kW>& R, const CandSet& cs, bool do_k, int t
         else hi = mid - step;
       }
       const double m_ge = mass_ge(lo);
-      const double m_gt = (lo >= cs.kmax) ? 0.0 : mass_ge(lo + step);
+      const double m_gt = (lo >= cs.kmax) ? cs.head : mass_ge(lo + step);
       o.margin = static_cast<float>(fmin(top_p - m_gt / Zk, m_ge / Zk - top_p));
       o.theta = max(theta, lo);
     } else {
       o.below = 1;
     }
   }
-  // the kept set's mass and size, when every kept entry is a candidate
-  if (!o.below && o.theta > cs.above) {
+  // the kept set's mass and size, when every kept entry is a candidate or
+  // above them
+  if (!o.below && (o.theta > cs.above || (o.theta == cs.above && cs.n_eq == 0.0))) {
     double sv = 0.0, cnt = 0.0;
     for (int i = f; i < cs.n; i += st)
       if (cs.key[i] >= o.theta && key_value(cs.key[i]) != -INFINITY) {
         sv += static_cast<double>(cs.w[i]);
         cnt += 1.0;
       }
-    o.Z = R.sum(sv);
-    o.kept = R.sum(cnt);
+    o.Z = R.sum(sv) + cs.head;
+    o.kept = R.sum(cnt) + cs.nhead;
     o.z_valid = 1;
     o.kept_valid = 1;
   } else if (!o.below && do_p) {
@@ -806,6 +1077,54 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams
       tail = 0.0;
     }
   }
+  // Band histograms (when the candidate room holds them).  A top-k cut the
+  // lists did not settle: every entry down to the band holding the k-th
+  // largest is a candidate.  A nucleus cut alone: the candidates are the
+  // bands around the cut, the masses above and below them from the histogram.
+  // (kept in shared memory: read only after the scans)
+  __shared__ BandGather s_bg;
+  if (threadIdx.x == 0) s_bg = BandGather{0, 0u, kmax, 0u, 0.0, 0.0};
+  if (use_k && nc < 0 && P.top_k <= kCap && kCap >= kBandCap) {
+    const float sb = kBandsPerUnit;
+    const float gs = gmx * sb;
+    const BandCut bc = band_cut<T, kAligned, false>(row, V, sb, gs, c_hi, c_lo, o,
+                                                   static_cast<double>(P.top_k), cand_smem);
+    if (bc.lo >= 0 && bc.end <= kCap) {
+      const BandGather g = gather_bands<T, kAligned, false>(row, V, sb, gs, 0, bc.hi, c, od,
+                                                            cand_key, cand_w, &cand_n, smd, smu,
+                                                            kCap);
+      if (g.n > 0 && g.n <= kCap) {
+        nc = g.n;
+        above = g.kmin;  // the candidates hold every entry >= kmin, at least k of them
+        theta = g.kmin;
+        n_eq = 0.0;
+        tail = 0.0;
+        if (threadIdx.x == 0) s_bg.kmax = g.kmax;
+      }
+    }
+  }
+  if (use_p && !use_k && nc < 0 && kCap >= kBandCap) {
+    const float sb = fminf(kBandsPerUnit * c_hi, 1e30f);
+    const float gs = gmx * sb;
+    const BandCut bc = band_cut<T, kAligned, true>(row, V, sb, gs, c_hi, c_lo, o, P.top_p, cand_smem);
+    if (bc.lo >= 0) {
+      const BandGather g = gather_bands<T, kAligned, true>(row, V, sb, gs, bc.lo, bc.hi, c, od,
+                                                           cand_key, cand_w, &cand_n, smd, smu,
+                                                           kCap);
+      if (g.n > 0 && g.n <= kCap) {
+        // histogram masses are relative to o; the candidates' to od
+        const double sc = exp2(static_cast<double>(o) - od);
+        nc = g.n;
+        above = g.kmin;      // entries below kmin: the later bands (mass `tail`);
+        n_eq = 0.0;          // entries above kmax: the earlier bands (head)
+        tail = bc.tail * sc;
+        if (threadIdx.x == 0) {
+          s_bg = g;
+          s_bg.head = bc.head * sc;
+        }
+      }
+    }
+  }
   if (use_k && nc < 0) theta = radix_select<T, kAligned>(row, V, 0u, P.top_k, low_bits, hist, &eq);
   const bool k_in_cands = use_k && nc >= 0;
 
@@ -835,7 +1154,8 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams
     // be a key that decodes to no finite value)
     const float xv = key_value(above);
     const double w_above = (n_eq > 0.0 && xv != -INFINITY) ? exp2(static_cast<double>(xv) * c - od) : 0.0;
-    CandSet cs{cand_key, cand_w, nc, above, n_eq, w_above, tail, kmax, step};
+    __syncthreads();
+    CandSet cs{cand_key, cand_w, nc, above, n_eq, w_above, tail, s_bg.kmax, step, s_bg.head, s_bg.nhead};
     if (nc <= kWarpCands) {
       if (threadIdx.x < kWarp)
         cand_stage(Red<true>{smd}, cs, k_in_cands, P.top_k, use_p, P.top_p, theta, &s_st);
@@ -846,20 +1166,23 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams
     const StageOut st = s_st;
     theta = st.theta;
     if (st.below) {
-      // the nucleus boundary lies below the candidates: a mass descent over
+      // the nucleus boundary lies outside the candidates: a mass descent over
       // the keys in [theta, v0), everything at or above v0 (mass m0) counted
-      // (fp32 weights relative to o; the candidates' room holds the histograms)
+      // (below), or over the keys above every candidate (above); fp32 weights
+      // relative to o, the candidates' room holds the histograms
       const double sc = exp2(static_cast<double>(o) - od);
       const double Zk = st.Zk;
-      const unsigned v0 = max(theta, above);
+      const bool up = st.below == 2;
+      const unsigned lo_key = up ? s_bg.hkmin : theta;
+      const unsigned hi_key = up ? 0xffffffffu : max(theta, above);
       double m_ge, m_gt;
       const unsigned lo = mass_descent<T, kAligned>(
-          row, V, theta, v0, st.m0 / sc, st.goal / sc, low_bits, c_hi, c_lo, o,
+          row, V, lo_key, hi_key, up ? 0.0 : st.m0 / sc, st.goal / sc, low_bits, c_hi, c_lo, o,
           reinterpret_cast<float*>(cand_smem), &m_ge, &m_gt);
       m_ge *= sc;
       m_gt *= sc;
       margin = static_cast<float>(fmin(P.top_p - m_gt / Zk, m_ge / Zk - P.top_p));
-      theta = lo;
+      theta = max(lo, lo_key);  // (a goal missed by rounding keeps the whole range)
       Z_kept = m_ge;
     } else {
       margin = st.margin;

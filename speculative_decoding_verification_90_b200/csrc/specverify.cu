@@ -6,6 +6,7 @@
 
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdio>
 #include <cstdlib>
@@ -431,10 +432,17 @@ sv_status specverify_run_sampling(specverify_t h, const void* target_logits,
   p.vocab = h->vocab;
   p.top_k = (top_k >= h->vocab) ? 0 : top_k;
   p.top_p = (top_p >= 1.f) ? 1.0 : static_cast<double>(top_p);
-  // a nucleus cut outside a small top-k set needs the large candidate room
-  // (fewer blocks per SM); every other setting fits in the small one
+  // Candidate room (dynamic shared memory, so blocks per SM): a small top-k
+  // set or no filter fits in the small one; a nucleus cut alone takes the
+  // room of the band histograms; a larger top-k set, room for its k entries
+  // and a band or so beyond them.
   const bool small_k = p.top_k > 0 && p.top_k <= specsamp::kSelThreads;
-  p.cand_cap = (p.top_p < 1.0 && !small_k) ? specsamp::kCand : specsamp::kCandSmall;
+  if (small_k || (p.top_k == 0 && p.top_p >= 1.0)) {
+    p.cand_cap = specsamp::kCandSmall;
+  } else {
+    const int want = p.top_k > 0 ? static_cast<int>(svhost::round_up(static_cast<size_t>(p.top_k) + p.top_k / 4 + 256, 1024)) : 0;
+    p.cand_cap = std::min(specsamp::kCand, std::max(specsamp::kBandCap, want));
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const long rows = static_cast<long>(h->batch) * (2L * G + 1);
   const int per = specsamp::kDecideThreads / specsamp::kWarp;

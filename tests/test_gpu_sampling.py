@@ -21,8 +21,9 @@ if not torch.cuda.is_available():  # pragma: no cover - collected on CPU hosts
 def _check(wl, temps, name, top_k=0, top_p=1.0, max_margin_frac=0.02):
     g = gpu_run_sampling(wl, temps, top_k, top_p)
     o = oracle_run_sampling(wl, temps, top_k, top_p)
-    s = compare_sampling(wl, g, o)
+    s = compare_sampling(wl, g, o, top_k)
     print(f"\n[{name}] seqs={s['sequences']} hard={len(s['hard'])} margin={len(s['margin_cases'])} "
+          f"unresolved={len(s['unresolved'])} "
           f"dq={s.get('max_dq')} dp={s.get('max_dp')} dz={s.get('max_dz')} "
           f"kept_t(mean)={float(np.mean(o['kept_target'])):.1f}")
     assert_parity(s, max_margin_frac=max_margin_frac)
@@ -50,6 +51,35 @@ def test_b64_greedy_full_size():
 def test_b64_filters_full_size(top_k, top_p):
     wl = workloads.b64_g8_v128256(seed=2)
     _check(wl, wl.temperature, f"b64 k={top_k} p={top_p}", top_k, top_p)
+
+
+@pytest.mark.parametrize("T,top_k,top_p", [(1.0, 2000, 1.0), (0.7, 2000, 0.9), (1.3, 5000, 0.95),
+                                           (0.05, 0, 0.9), (2.5, 0, 0.5), (1.0, 0, 0.9999),
+                                           (1.0, 0, 0.02), (0.05, 3000, 1.0)])
+def test_b64_band_cuts_full_size(T, top_k, top_p):
+    """Large top-k sets (count bands) and nucleus cuts alone (mass bands) over
+    temperatures that move the cut from the top band to the far tail."""
+    wl = workloads.b64_g8_v128256(seed=5)
+    _check(wl, T, f"b64 T={T} k={top_k} p={top_p}", top_k, top_p)
+
+
+def test_flat_and_neg_inf_rows():
+    """Rows of one repeated value (every entry in one band: more candidates than
+    fit) and rows mostly -inf (the last band), with large top-k and nucleus cuts."""
+    rng = np.random.default_rng(31)
+    B, G, V = 6, 3, 40000
+    tgt = (rng.standard_normal((B, G + 1, V)) * 2.0).astype(np.float32)
+    drf = (0.8 * tgt[:, :G] + 0.2 * rng.standard_normal((B, G, V)) * 2.0).astype(np.float32)
+    tgt[0] = 1.5
+    drf[0] = 1.5
+    tgt[1, :, 100:] = -np.inf
+    drf[1, :, 200:] = -np.inf
+    tgt[2, 1, :] = np.where(np.arange(V) % 3 == 0, 0.25, -np.inf)
+    tok = workloads.gumbel_max_tokens(rng, drf, 1.0)
+    wl = workloads.Workload("flat_inf", B, G, V, "f32", 1.0, tgt, drf, tok,
+                            rng.random((B, G), dtype=np.float32), rng.random(B, dtype=np.float32))
+    for k, p in ((0, 0.5), (0, 0.97), (3000, 1.0), (20000, 0.9), (300, 0.8)):
+        _check(wl, 1.0, f"flat/-inf k={k} p={p}", k, p)
 
 
 def test_multibranch_filters_full_size():
