@@ -105,7 +105,8 @@ struct SampParams {
 // order-preserving unsigned key of a float (NaN excluded by the callers)
 __device__ __forceinline__ unsigned fkey(float x) {
   const unsigned u = __float_as_uint(x);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  // negative: all bits flipped; otherwise the sign bit set
+  return u ^ (static_cast<unsigned>(static_cast<int>(u) >> 31) | 0x80000000u);
 }
 
 __device__ __forceinline__ float key_value(unsigned k) {
@@ -455,7 +456,32 @@ struct BandCut {
   int lo, hi;         // the bands holding the cut (lo = -1: none found)
   double end;         // running total (count or mass) through band hi
   double head, tail;  // mass: of the bands before lo, and after hi
+  unsigned k_lo;      // smallest key in a band <= hi
+  unsigned k_head;    // mass: smallest key in a band < lo (kmax + step when lo = 0);
+                      // count: kmax + step (every band down to hi is wanted)
 };
+
+// Smallest key K in [key(-inf), kmax] with band_of(K) <= j, by warp 0 (every
+// lane calls it): each round probes 32 evenly spaced keys of the remaining
+// range, whose predicate runs false ... true since the band never increases
+// with the key, and band(kmax) = 0.  Rounded up to a multiple of `step`,
+// which selects the same entries when every key is such a multiple.
+__device__ __forceinline__ unsigned band_floor_key(int j, float s, float gs, unsigned kmax,
+                                                   unsigned step) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  unsigned lo = 0x007fffffu, hi = kmax;  // key(-inf) .. key(max): no NaN in between
+  while (lo < hi) {
+    const unsigned w = (hi - lo) / kWarp + 1u;
+    const unsigned p = min(hi, lo + (static_cast<unsigned>(lane) + 1u) * w - 1u);
+    const unsigned ok = __ballot_sync(0xffffffffu, band_of(key_value(p), s, gs) <= j);
+    const int l = __ffs(ok) - 1;  // lane 31 probes hi, whose band is <= j
+    const unsigned p_hit = __shfl_sync(0xffffffffu, p, l);
+    const unsigned p_before = __shfl_sync(0xffffffffu, p, max(l - 1, 0));
+    lo = (l == 0) ? lo : p_before + 1u;
+    hi = p_hit;
+  }
+  return ((lo + step - 1u) / step) * step;
+}
 
 // One scan: per-warp histograms over bands of the entry count (kMass false)
 // or of the fp32 weight 2^(x c - o) (kMass true), in `smem` (kSelWarps x
@@ -468,7 +494,7 @@ struct BandCut {
 // come from the same histogram.
 template <typename T, bool kAligned, bool kMass>
 __device__ BandCut band_cut(const T* row, int V, float s, float gs, float c_hi, float c_lo,
-                            float o, double goal, unsigned* smem) {
+                            float o, double goal, unsigned kmax, unsigned step, unsigned* smem) {
   float* hw = reinterpret_cast<float*>(smem);
   int* hc = reinterpret_cast<int*>(smem);
   const int warp = threadIdx.x >> 5;
@@ -563,55 +589,46 @@ __device__ BandCut band_cut(const T* row, int V, float s, float gs, float c_hi, 
     int lo = h_lo <= 0.0 ? 0 : find(h_lo, &s_lo, &e_lo);
     const int hi = find(fmin(g + slack, total), &s_hi, &e_hi);
     if (hi < 0 || lo > hi) lo = -1;
-    if (lane == 0) s_bc = BandCut{lo, hi, e_hi, s_lo, fmax(total - e_hi, 0.0)};
+    unsigned k_lo = 0u, k_head = 0u;
+    if (lo >= 0) {
+      k_lo = band_floor_key(hi, s, gs, kmax, step);
+      k_head = (kMass && lo > 0) ? band_floor_key(lo - 1, s, gs, kmax, step) : kmax + step;
+    }
+    if (lane == 0) s_bc = BandCut{lo, hi, e_hi, s_lo, fmax(total - e_hi, 0.0), k_lo, k_head};
   }
   __syncthreads();
   return s_bc;
 }
 
-struct BandGather {
-  int n;                   // entries in the bands (may exceed the room)
-  unsigned kmin, kmax;     // their smallest and largest keys
-  unsigned hkmin;          // smallest key of the entries in earlier bands
-  double head, nhead;      // mass (fp64 weights 2^(x c - od)) and count of those entries
-};
-
-// Candidates: the entries in bands [j_lo, j_hi], keys into shared memory and
-// then their weights in double precision (rounded to float).  With kHead also
-// the count and smallest key of the entries in earlier bands (larger values).
-// One vote per group of elements: most groups hold no candidate.
+// Candidates: the entries with k_lo <= key < k_head (exactly the entries of
+// the bands holding the cut), keys into shared memory and then their weights
+// in double precision (rounded to float); the count in the return value (may
+// exceed the room).  With kHead also the number of entries with key >= k_head
+// (the earlier bands) in *nhead.  One vote per group of elements: where a lane
+// holds candidates, one warp scan of the lanes' counts and one shared atomic
+// per warp place them.
 template <typename T, bool kAligned, bool kHead>
-__device__ BandGather gather_bands(const T* row, int V, float s, float gs, int j_lo, int j_hi,
-                                   double c, double od, unsigned* cand_key, float* cand_w,
-                                   int* cand_n, double* smd, unsigned* smu, int cap) {
+__device__ int gather_range(const T* row, int V, unsigned k_lo, unsigned k_head, double c,
+                            double od, unsigned* cand_key, float* cand_w, int* cand_n, double* smd,
+                            double* nhead, int cap) {
   constexpr int kN = Groups<T, kAligned>::kN;
   const int lane = threadIdx.x & (kWarp - 1);
   if (threadIdx.x == 0) *cand_n = 0;
   __syncthreads();
   int nh = 0;
-  unsigned kmx = 0u, nkmn = 0u, nhk = 0u;  // maxima of k, ~k, ~k
   scan_groups<T, kAligned>(row, V, [&](const float* x, int n, long) {
     unsigned tmask = 0u;
-    unsigned key[kN];
+    if (n == kN) {
 #pragma unroll
-    for (int e = 0; e < kN; ++e) {
-      key[e] = fkey(x[e]);
-      if (e < n) {
-        const int j = band_of(x[e], s, gs);
-        if (j >= j_lo && j <= j_hi) {
-          tmask |= 1u << e;
-          kmx = max(kmx, key[e]);
-          nkmn = max(nkmn, ~key[e]);
-        }
-        if (kHead && j < j_lo) {
-          ++nh;
-          nhk = max(nhk, ~key[e]);
-        }
+      for (int e = 0; e < kN; ++e) {
+        const unsigned key = fkey(x[e]);
+        const bool above_lo = key >= k_lo;
+        const bool in_head = key >= k_head;
+        tmask |= static_cast<unsigned>(above_lo && !in_head) << e;
+        if constexpr (kHead) nh += in_head;
       }
     }
     if (__any_sync(0xffffffffu, tmask != 0u)) {
-      // the lanes' takes in lane order: a warp scan of their counts, one
-      // shared atomic for the warp's run of slots
       const int cnt = __popc(tmask);
       int incl = cnt;
 #pragma unroll
@@ -625,28 +642,27 @@ __device__ BandGather gather_bands(const T* row, int V, float s, float gs, int j
 #pragma unroll
       for (int e = 0; e < kN; ++e) {
         if ((tmask >> e) & 1u) {
-          if (slot < cap) cand_key[slot] = key[e];
+          if (slot < cap) cand_key[slot] = fkey(x[e]);
           ++slot;
         }
       }
     }
   });
   __syncthreads();
-  BandGather out;
-  out.n = *cand_n;
-  for (int i = threadIdx.x; i < min(out.n, cap); i += blockDim.x)
+  const int nc = *cand_n;
+  for (int i = threadIdx.x; i < min(nc, cap); i += blockDim.x)
     cand_w[i] = static_cast<float>(exp2(static_cast<double>(key_value(cand_key[i])) * c - od));
-  out.kmax = block_max_u<kSelThreads>(kmx, smu);
-  out.kmin = ~block_max_u<kSelThreads>(nkmn, smu);
-  out.head = 0.0;
-  out.nhead = 0.0;
-  out.hkmin = 0u;
-  if constexpr (kHead) {
-    out.nhead = block_sum<kSelThreads>(static_cast<double>(nh), smd);
-    out.hkmin = ~block_max_u<kSelThreads>(nhk, smu);
-  }
-  return out;
+  *nhead = kHead ? block_sum<kSelThreads>(static_cast<double>(nh), smd) : 0.0;
+  return nc;
 }
+
+// What the candidate stage needs besides the candidates of a band cut
+// (kept in shared memory: read only after the scans).
+struct BandSide {
+  unsigned kmax;     // a key at or above every candidate
+  unsigned hkmin;    // smallest key above the candidates' bands
+  double head, nhead;  // mass (fp64 weights 2^(x c - od)) and count of those entries
+};
 
 // ---------------------------------------------------------------------------
 // kernel 1: per-row adjusted distribution
@@ -1081,47 +1097,45 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams
   // lists did not settle: every entry down to the band holding the k-th
   // largest is a candidate.  A nucleus cut alone: the candidates are the
   // bands around the cut, the masses above and below them from the histogram.
-  // (kept in shared memory: read only after the scans)
-  __shared__ BandGather s_bg;
-  if (threadIdx.x == 0) s_bg = BandGather{0, 0u, kmax, 0u, 0.0, 0.0};
+  __shared__ BandSide s_bs;
+  if (threadIdx.x == 0) s_bs = BandSide{kmax, 0u, 0.0, 0.0};
   if (use_k && nc < 0 && P.top_k <= kCap && kCap >= kBandCap) {
     const float sb = kBandsPerUnit;
     const float gs = gmx * sb;
     const BandCut bc = band_cut<T, kAligned, false>(row, V, sb, gs, c_hi, c_lo, o,
-                                                   static_cast<double>(P.top_k), cand_smem);
+                                                   static_cast<double>(P.top_k), kmax, step,
+                                                   cand_smem);
     if (bc.lo >= 0 && bc.end <= kCap) {
-      const BandGather g = gather_bands<T, kAligned, false>(row, V, sb, gs, 0, bc.hi, c, od,
-                                                            cand_key, cand_w, &cand_n, smd, smu,
-                                                            kCap);
-      if (g.n > 0 && g.n <= kCap) {
-        nc = g.n;
-        above = g.kmin;  // the candidates hold every entry >= kmin, at least k of them
-        theta = g.kmin;
+      double unused;
+      const int n = gather_range<T, kAligned, false>(row, V, bc.k_lo, kmax + step, c, od,
+                                                     cand_key, cand_w, &cand_n, smd, &unused, kCap);
+      if (n > 0 && n <= kCap) {
+        nc = n;
+        above = bc.k_lo;  // the candidates hold every entry >= k_lo, at least k of them
+        theta = bc.k_lo;
         n_eq = 0.0;
         tail = 0.0;
-        if (threadIdx.x == 0) s_bg.kmax = g.kmax;
       }
     }
   }
   if (use_p && !use_k && nc < 0 && kCap >= kBandCap) {
     const float sb = fminf(kBandsPerUnit * c_hi, 1e30f);
     const float gs = gmx * sb;
-    const BandCut bc = band_cut<T, kAligned, true>(row, V, sb, gs, c_hi, c_lo, o, P.top_p, cand_smem);
+    const BandCut bc = band_cut<T, kAligned, true>(row, V, sb, gs, c_hi, c_lo, o, P.top_p, kmax,
+                                                  step, cand_smem);
     if (bc.lo >= 0) {
-      const BandGather g = gather_bands<T, kAligned, true>(row, V, sb, gs, bc.lo, bc.hi, c, od,
-                                                           cand_key, cand_w, &cand_n, smd, smu,
-                                                           kCap);
-      if (g.n > 0 && g.n <= kCap) {
+      double nh = 0.0;
+      const int n = gather_range<T, kAligned, true>(row, V, bc.k_lo, bc.k_head, c, od, cand_key,
+                                                    cand_w, &cand_n, smd, &nh, kCap);
+      if (n > 0 && n <= kCap) {
         // histogram masses are relative to o; the candidates' to od
         const double sc = exp2(static_cast<double>(o) - od);
-        nc = g.n;
-        above = g.kmin;      // entries below kmin: the later bands (mass `tail`);
-        n_eq = 0.0;          // entries above kmax: the earlier bands (head)
+        nc = n;
+        above = bc.k_lo;   // entries below k_lo: the later bands (mass `tail`);
+        n_eq = 0.0;        // entries from k_head on: the earlier bands (head)
         tail = bc.tail * sc;
-        if (threadIdx.x == 0) {
-          s_bg = g;
-          s_bg.head = bc.head * sc;
-        }
+        if (threadIdx.x == 0)
+          s_bs = BandSide{bc.lo > 0 ? bc.k_head - step : kmax, bc.k_head, bc.head * sc, nh};
       }
     }
   }
@@ -1155,7 +1169,7 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams
     const float xv = key_value(above);
     const double w_above = (n_eq > 0.0 && xv != -INFINITY) ? exp2(static_cast<double>(xv) * c - od) : 0.0;
     __syncthreads();
-    CandSet cs{cand_key, cand_w, nc, above, n_eq, w_above, tail, s_bg.kmax, step, s_bg.head, s_bg.nhead};
+    CandSet cs{cand_key, cand_w, nc, above, n_eq, w_above, tail, s_bs.kmax, step, s_bs.head, s_bs.nhead};
     if (nc <= kWarpCands) {
       if (threadIdx.x < kWarp)
         cand_stage(Red<true>{smd}, cs, k_in_cands, P.top_k, use_p, P.top_p, theta, &s_st);
@@ -1173,7 +1187,7 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams
       const double sc = exp2(static_cast<double>(o) - od);
       const double Zk = st.Zk;
       const bool up = st.below == 2;
-      const unsigned lo_key = up ? s_bg.hkmin : theta;
+      const unsigned lo_key = up ? s_bs.hkmin : theta;
       const unsigned hi_key = up ? 0xffffffffu : max(theta, above);
       double m_ge, m_gt;
       const unsigned lo = mass_descent<T, kAligned>(
