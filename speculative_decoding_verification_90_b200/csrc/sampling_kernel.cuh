@@ -677,8 +677,9 @@ __device__ __forceinline__ void put_row(const SampParams& P, long r, long nT, co
 
 // Candidates: entries gathered into shared memory (key, weight in double
 // precision rounded to float) when their key is above `above` and at least
-// `floor_key`; the count may exceed kCand (then only the first kCand are kept
-// and the caller falls back).  Entries equal to `above` are counted in *n_eq.
+// `floor_key`; the count may exceed the room `cap` (then only the first `cap`
+// are kept and the caller falls back).  Entries equal to `above` are counted
+// in *n_eq.
 template <typename T, bool kAligned, bool kTail>
 __device__ int gather(const T* row, int V, unsigned above, unsigned floor_key, double c, double od,
                       unsigned* cand_key, float* cand_w, int* cand_n, float c_hi, float c_lo,
@@ -1099,7 +1100,9 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams
   // bands around the cut, the masses above and below them from the histogram.
   __shared__ BandSide s_bs;
   if (threadIdx.x == 0) s_bs = BandSide{kmax, 0u, 0.0, 0.0};
-  if (use_k && nc < 0 && P.top_k <= kCap && kCap >= kBandCap) {
+  // (gs must be finite for the bands to follow the keys: an overflow there
+  // means logits beyond 1e37, left to the fallbacks)
+  if (use_k && nc < 0 && P.top_k <= kCap && kCap >= kBandCap && isfinite(gmx * kBandsPerUnit)) {
     const float sb = kBandsPerUnit;
     const float gs = gmx * sb;
     const BandCut bc = band_cut<T, kAligned, false>(row, V, sb, gs, c_hi, c_lo, o,
@@ -1118,8 +1121,9 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams
       }
     }
   }
-  if (use_p && !use_k && nc < 0 && kCap >= kBandCap) {
-    const float sb = fminf(kBandsPerUnit * c_hi, 1e30f);
+  const float sb_p = fminf(kBandsPerUnit * c_hi, 1e30f);
+  if (use_p && !use_k && nc < 0 && kCap >= kBandCap && isfinite(gmx * sb_p)) {
+    const float sb = sb_p;
     const float gs = gmx * sb;
     const BandCut bc = band_cut<T, kAligned, true>(row, V, sb, gs, c_hi, c_lo, o, P.top_p, kmax,
                                                   step, cand_smem);
