@@ -60,6 +60,12 @@ KERNEL_SOURCES = [
 ]
 
 
+# sampling-variant settings timed by the bench: name -> (temperature, top_k, top_p);
+# None = the workload's temperature
+SAMPLING_SETTINGS = {"greedy": (0.0, 0, 1.0), "top_k50_top_p0.9": (None, 50, 0.9),
+                     "top_p0.9": (None, 0, 0.9), "top_k2000": (None, 2000, 1.0)}
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -76,15 +82,20 @@ def parse():
     ap.add_argument("--no-shared-rows", action="store_true",
                     help="skip the timing of the shared-row entry point (multibranch)")
     ap.add_argument("--no-sampling", action="store_true",
-                    help="skip the timing of the sampling variants (greedy, top-k + top-p)")
+                    help="skip the timing of the sampling variants")
     ap.add_argument("--sampling", default=None,
-                    help="comma-separated sampling settings to time (greedy, top_k50_top_p0.9, "
-                         "top_p0.9, top_k2000; default: all)")
+                    help="comma-separated sampling settings to time (" + ", ".join(SAMPLING_SETTINGS)
+                         + "; default: all)")
     ap.add_argument("--no-lmhead", action="store_true",
                     help="skip the timing of the LM-head-fused step (64 x 8, V 128256, d 4096)")
     ap.add_argument("--no-gate", action="store_true",
                     help="skip the timing of the fold gate (128 x 8 branches, 32 x 4096 bf16)")
-    return ap.parse_args()
+    args = ap.parse_args()
+    if args.sampling:
+        unknown = [n for n in args.sampling.split(",") if n not in SAMPLING_SETTINGS]
+        if unknown:
+            ap.error(f"--sampling: unknown setting(s) {unknown}; known: {list(SAMPLING_SETTINGS)}")
+    return args
 
 
 def kernel_hash() -> str:
@@ -522,8 +533,8 @@ def time_sampling(args, wl, sv, sets, n_sets, out_t, out_n, dev, world, local):
     import torch
     import torch.distributed as dist
     res = {}
-    configs = {"greedy": (0.0, 0, 1.0), "top_k50_top_p0.9": (wl.temperature, 50, 0.9),
-               "top_p0.9": (wl.temperature, 0, 0.9), "top_k2000": (wl.temperature, 2000, 1.0)}
+    configs = {name: (wl.temperature if T is None else T, k, p)
+               for name, (T, k, p) in SAMPLING_SETTINGS.items()}
     if args.sampling:
         configs = {name: configs[name] for name in args.sampling.split(",")}
     for name, (T, k, p) in configs.items():
