@@ -237,6 +237,43 @@ def test_disjoint_supports_reject_first_and_draw_from_target(oracle_mod):
     assert np.allclose(out["resid_mass"], 1.0, atol=1e-12)
 
 
+def test_zero_residual_mass_falls_back_to_target(oracle_mod):
+    """A rejection whose residual max(0, q - p) has no mass in double precision:
+    target and draft rows equal except at the drafted token t, where q(t)
+    underflows to 0 (logit -1000) and p(t) is about 1e-301 (logit -690).  The
+    ratio is 0, so t is rejected; every other q(i) equals p(i) bit for bit
+    (the tiny p(t) does not move the draft's normaliser), so Z = 0.  The draw
+    then comes from q at that position (inverse CDF with the same uniform,
+    checked against a library softmax) and the ZERO_MASS warning is set."""
+    rng = np.random.default_rng(12)
+    B, G, V, T = 24, 2, 64, 1.0
+    tgt = (rng.standard_normal((B, G + 1, V)) * 2).astype(np.float32)
+    drf = tgt[:, :G].copy()
+    n = rng.integers(0, G, size=B)          # the position that rejects
+    tok = np.zeros((B, G), np.int32)
+    for b in range(B):
+        for j in range(G):
+            tok[b, j] = int(np.argmax(tgt[b, j]))  # accepted (ratio 1) before n
+        t = int(rng.integers(0, V))
+        tok[b, n[b]] = t
+        tgt[b, n[b], t] = -1000.0
+        drf[b, n[b], t] = -690.0
+    u_acc = np.full((B, G), 0.5, np.float32)
+    u_res = rng.random(B, dtype=np.float32)
+    out = oracle_mod.verify(tgt, drf, tok, u_acc, u_res, T)
+    np.testing.assert_array_equal(out["out_num_accepted"], n)
+    assert (out["seq_status"] == 18).all()
+    for b in range(B):
+        q = torch.softmax(torch.from_numpy(tgt[b, n[b]].astype(np.float64)) / T, 0).numpy()
+        c = np.cumsum(q)
+        expect = int(np.searchsorted(c, float(u_res[b]) * c[-1], side="right"))
+        assert abs(float(u_res[b]) * c[-1] - c[min(expect, V - 1)]) > 1e-9   # away from an edge
+        assert out["out_tokens"][b, n[b]] == expect
+        np.testing.assert_array_equal(out["out_tokens"][b, :n[b]], tok[b, :n[b]])
+        assert (out["out_tokens"][b, n[b] + 1:] == -1).all()
+        assert out["q_tok"][b, n[b]] == 0.0 and out["p_tok"][b, n[b]] > 0.0
+
+
 def test_data_errors(oracle_mod):
     rng = np.random.default_rng(6)
     tgt, drf, tok, ua, ur = _random_problem(rng, 4, 3, 16, "f32", 0.5)
