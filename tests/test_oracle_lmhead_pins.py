@@ -48,3 +48,34 @@ def test_lmhead_workload_layout():
     assert ((w.tokens >= 0) & (w.tokens < 500)).all()
     w2 = workloads.lmhead(seed=1, batch=3, gamma=2, vocab=500, hidden=128, shared_weight=False)
     assert w2.draft_weight is not w2.target_weight
+
+
+def test_integer_valued_inputs_give_exact_dot_products():
+    """Small integers are exact in bf16 and every partial sum below 2^53 is exact
+    in float64: the logits equal Python integer arithmetic (brute force)."""
+    rng = np.random.default_rng(7)
+    D, V, R = 96, 33, 5
+    h = rng.integers(-8, 9, size=(R, D))
+    w = rng.integers(-8, 9, size=(V, D))
+    hb = workloads.bits_to_f32(workloads.bf16_bits(h.astype(np.float32)))
+    wb = workloads.bits_to_f32(workloads.bf16_bits(w.astype(np.float32)))
+    assert (hb == h).all() and (wb == w).all()
+    x = oracle.lm_logits(hb, wb)
+    for r in range(R):
+        for v in range(V):
+            assert x[r, v] == sum(int(h[r, k]) * int(w[v, k]) for k in range(D))
+
+
+def test_scaling_a_hidden_row_scales_its_logits():
+    """h -> 2h doubles every logit exactly (a power of two is exact in both
+    bf16 and float64); the other rows are untouched."""
+    rng = np.random.default_rng(8)
+    D, V = 64, 50
+    h = workloads.bits_to_f32(workloads.bf16_bits(rng.standard_normal((2, D)).astype(np.float32)))
+    w = workloads.bits_to_f32(workloads.bf16_bits(rng.standard_normal((V, D)).astype(np.float32)))
+    x = oracle.lm_logits(h, w)
+    h2 = h.copy()
+    h2[1] *= 2.0
+    x2 = oracle.lm_logits(h2, w)
+    np.testing.assert_array_equal(x2[0], x[0])
+    np.testing.assert_array_equal(x2[1], 2.0 * x[1])
