@@ -216,3 +216,23 @@ def test_bruteforce_law_equals_adjusted_target(top_k, top_p):
                 res = np.zeros(V)
             law += p[t] * (acc * np.eye(V)[t] + (1.0 - acc) * res)
         assert np.max(np.abs(law - q)) < 3.0 * V / n, (trial, law, q)
+
+
+def test_top_p_keeps_tied_values_together():
+    """Probabilities (0.4, 0.2, 0.2, 0.2): top_p 0.4 stops at the first value
+    (mass 0.4 reaches it) and keeps one entry; top_p 0.5 must take the next
+    value, which three entries share, so all four are kept (q(t) = 0.2)."""
+    probs = np.array([0.4, 0.2, 0.2, 0.2])
+    x = np.log(probs).astype(np.float32)
+    tgt = np.stack([x, x])[None]
+    drf = tgt[:, :1].copy()
+    tok = np.array([[2]], np.int32)
+    ua = np.array([[0.0]], np.float32)
+    ur = np.array([0.3], np.float32)
+    seen = np.exp(x.astype(np.float64))
+    seen /= seen.sum()
+    for top_p, keep in ((0.39, 1), (0.5, 4), (0.9, 4)):
+        r = oracle.verify_sampling(tgt, drf, tok, ua, ur, 1.0, top_p=top_p)
+        assert r["kept_target"][0].tolist() == [keep, keep]
+        expect = seen[2] / seen[:keep].sum() if keep > 2 else 0.0
+        assert r["q_tok"][0, 0] == pytest.approx(expect, rel=1e-12, abs=1e-300)
