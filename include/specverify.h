@@ -7,7 +7,7 @@
  *   accept a draft token t with probability min(1, q(t)/p(t)); on rejection
  *   draw again from max(0, q - p) / ||max(0, q - p)||_1.
  *   "Speculative decoding: how to run big models fast" (ai-trend.me), section
- *   "How it works": judge drafts left to right, stop at the first rejection
+ *   "How it works": check the drafts left to right, stop at the first rejection
  *   and discard the rest, append one token drawn from q at position gamma+1
  *   when every draft is accepted, so each call emits 1 .. gamma+1 tokens;
  *   temperature is handled as sampling from an adjusted distribution.
