@@ -464,7 +464,9 @@ struct BandCut {
 // Smallest key K in [key(-inf), kmax] with band_of(K) <= j, by warp 0 (every
 // lane calls it): each round probes 32 evenly spaced keys of the remaining
 // range, whose predicate runs false ... true since the band never increases
-// with the key, and band(kmax) = 0.  Rounded up to a multiple of `step`,
+// with the key, and band(kmax) = 0.  (Should the rounding of gs put the
+// maximum in a later band, no lane votes, lo only grows and the loop still
+// ends, past kmax: no key qualifies.)  Rounded up to a multiple of `step`,
 // which selects the same entries when every key is such a multiple.
 __device__ __forceinline__ unsigned band_floor_key(int j, float s, float gs, unsigned kmax,
                                                    unsigned step) {
