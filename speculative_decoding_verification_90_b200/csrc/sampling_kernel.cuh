@@ -465,8 +465,8 @@ struct BandCut {
 // lane calls it): each round probes 32 evenly spaced keys of the remaining
 // range, whose predicate runs false ... true since the band never increases
 // with the key, and band(kmax) = 0.  (Should the rounding of gs put the
-// maximum in a later band, no lane votes, lo only grows and the loop still
-// ends, past kmax: no key qualifies.)  Rounded up to a multiple of `step`,
+// maximum in a later band, no lane votes and lo only grows, so the loop still
+// ends, at kmax.)  Rounded up to a multiple of `step`,
 // which selects the same entries when every key is such a multiple.
 __device__ __forceinline__ unsigned band_floor_key(int j, float s, float gs, unsigned kmax,
                                                    unsigned step) {
