@@ -89,3 +89,91 @@ def test_shard_covers_the_batch_once():
             assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
     with pytest.raises(ValueError):
         svdist.shard(10, 2, 2)
+
+
+# ---------------------------------------------------------------------------
+# the sampling variants and the fold gate shard the same way: whole sequences
+# per rank, no data-path collective; gathered results equal one whole run
+# ---------------------------------------------------------------------------
+
+_GATE = dict(seed=2, sequences=4, branches=8, positions=4, dim=64, dtype="f32", tau=0.2)
+
+
+def _variants_worker(rank, world, port, result_q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    try:
+        import oracle
+        from speculative_decoding_verification_90_b200 import workloads
+        svdist.init("gloo", timeout_s=60)
+        # sampling variants: per-sequence temperatures travel with the shard
+        wl = workloads.b8_g3_v32000(seed=21)
+        temps = np.array([0.7, 0.0, 1.3, 0.9, 0.0, 2.0, 0.5, 1.0], np.float32)
+        lo, hi = svdist.shard(wl.batch, world, rank)
+        part = oracle.verify_sampling(wl.target[lo:hi], wl.draft[lo:hi], wl.tokens[lo:hi],
+                                      wl.u_accept[lo:hi], wl.u_resample[lo:hi], temps[lo:hi],
+                                      top_k=20, top_p=0.9)
+        # fold gate: whole sequences (blocks of branches) per rank, parents rebased
+        g = workloads.gate_tree(**_GATE)
+        per = _GATE["branches"]
+        s_lo, s_hi = svdist.shard(_GATE["sequences"], world, rank)
+        b_lo, b_hi = s_lo * per, s_hi * per
+        par = g.parent[b_lo:b_hi].copy()
+        par[par >= 0] -= b_lo
+        gate = oracle.gate(g.hidden[b_lo:b_hi], par, g.tau)
+        mine = {"lo": lo, "tokens": part["out_tokens"], "n": part["out_num_accepted"],
+                "b_lo": b_lo, "gate": gate}
+        everyone = [None] * world
+        dist.all_gather_object(everyone, mine)
+        dist.barrier()
+        result_q.put((rank, everyone))
+        dist.destroy_process_group()
+    except Exception as e:  # report, never hang the parent
+        result_q.put((rank, "error: " + repr(e)))
+
+
+def test_two_rank_gloo_variants_and_gate():
+    import oracle
+    from speculative_decoding_verification_90_b200 import workloads
+    oracle.build()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_variants_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=240) for _ in range(2))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank in (0, 1):
+        assert not isinstance(results[rank], str), results[rank]
+    shards = sorted(results[0], key=lambda m: m["lo"])
+
+    wl = workloads.b8_g3_v32000(seed=21)
+    temps = np.array([0.7, 0.0, 1.3, 0.9, 0.0, 2.0, 0.5, 1.0], np.float32)
+    ref = oracle.verify_sampling(wl.target, wl.draft, wl.tokens, wl.u_accept, wl.u_resample,
+                                 temps, top_k=20, top_p=0.9)
+    np.testing.assert_array_equal(np.concatenate([m["tokens"] for m in shards]), ref["out_tokens"])
+    np.testing.assert_array_equal(np.concatenate([m["n"] for m in shards]), ref["out_num_accepted"])
+
+    g = workloads.gate_tree(**_GATE)
+    per = _GATE["branches"]
+    assert all(p < 0 or p // per == b // per for b, p in enumerate(g.parent))  # within a sequence
+    whole = oracle.gate(g.hidden, g.parent, g.tau)
+    npos = _GATE["positions"]
+
+    def rebase(a, off):
+        a = a.copy()
+        a[a >= 0] += off
+        return a
+
+    for key in ("rel_diff", "recompute"):
+        np.testing.assert_array_equal(np.concatenate([m["gate"][key] for m in shards]), whole[key])
+    for key in ("provenance", "source"):
+        np.testing.assert_array_equal(
+            np.concatenate([rebase(m["gate"][key], m["b_lo"] * npos) for m in shards]), whole[key])
+    np.testing.assert_array_equal(
+        np.concatenate([m["gate"]["packed"] + m["b_lo"] * npos for m in shards]), whole["packed"])
+    assert whole["packed"].size > 0 and whole["recompute"].sum() < whole["recompute"].size
