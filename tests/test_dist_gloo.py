@@ -97,6 +97,17 @@ def test_shard_covers_the_batch_once():
 # ---------------------------------------------------------------------------
 
 _GATE = dict(seed=2, sequences=4, branches=8, positions=4, dim=64, dtype="f32", tau=0.2)
+_LM = dict(seed=5, batch=6, gamma=3, vocab=700, hidden=128)
+
+
+def _lm_verify(oracle, workloads, lm, lo, hi):
+    """Sequences [lo, hi) of the LM-head workload: float64 logits of the
+    output layer, then the verification on them."""
+    f = workloads.bits_to_f32
+    t = oracle.lm_logits(f(lm.target_hidden[lo:hi]), f(lm.target_weight))
+    d = oracle.lm_logits(f(lm.draft_hidden[lo:hi]), f(lm.draft_weight))
+    return oracle.verify(t, d, lm.tokens[lo:hi], lm.u_accept[lo:hi], lm.u_resample[lo:hi],
+                         lm.temperature)
 
 
 def _variants_worker(rank, world, port, result_q):
@@ -122,8 +133,13 @@ def _variants_worker(rank, world, port, result_q):
         par = g.parent[b_lo:b_hi].copy()
         par[par >= 0] -= b_lo
         gate = oracle.gate(g.hidden[b_lo:b_hi], par, g.tau)
+        # the step fused with the output layer: the batch split, the layer replicated
+        lm = workloads.lmhead(**_LM)
+        m_lo, m_hi = svdist.shard(lm.batch, world, rank)
+        lm_part = _lm_verify(oracle, workloads, lm, m_lo, m_hi)
         mine = {"lo": lo, "tokens": part["out_tokens"], "n": part["out_num_accepted"],
-                "b_lo": b_lo, "gate": gate}
+                "b_lo": b_lo, "gate": gate, "lm_lo": m_lo, "lm_tokens": lm_part["out_tokens"],
+                "lm_n": lm_part["out_num_accepted"]}
         everyone = [None] * world
         dist.all_gather_object(everyone, mine)
         dist.barrier()
@@ -177,3 +193,11 @@ def test_two_rank_gloo_variants_and_gate():
     np.testing.assert_array_equal(
         np.concatenate([m["gate"]["packed"] + m["b_lo"] * npos for m in shards]), whole["packed"])
     assert whole["packed"].size > 0 and whole["recompute"].sum() < whole["recompute"].size
+
+    lm = workloads.lmhead(**_LM)
+    lm_ref = _lm_verify(oracle, workloads, lm, 0, lm.batch)
+    lm_shards = sorted(results[0], key=lambda m: m["lm_lo"])
+    np.testing.assert_array_equal(np.concatenate([m["lm_tokens"] for m in lm_shards]),
+                                  lm_ref["out_tokens"])
+    np.testing.assert_array_equal(np.concatenate([m["lm_n"] for m in lm_shards]),
+                                  lm_ref["out_num_accepted"])
