@@ -539,9 +539,16 @@ def time_sampling(args, wl, sv, sets, n_sets, out_t, out_n, dev, world, local):
         configs = {name: configs[name] for name in args.sampling.split(",")}
     for name, (T, k, p) in configs.items():
         temps = torch.full((wl.batch,), T, dtype=torch.float32, device=dev)
+        # greedy: the draft "samples" its argmax, which is the method's
+        # precondition (t drawn from the adjusted p); tokens drawn at T = 1
+        # would hand the rule tokens that p gives no mass
+        use = sets
+        if T == 0.0:
+            use = [dict(d, tokens=d["draft"].argmax(dim=-1).to(torch.int32).contiguous())
+                   for d in sets]
 
-        def step(i):
-            d = sets[i % n_sets]
+        def step(i, use=use):
+            d = use[i % n_sets]
             sv.run_sampling(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
                             temps, out_t, out_n, top_k=k, top_p=p)
 

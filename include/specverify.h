@@ -29,9 +29,12 @@
  *     draw, because exactly one of the two happens;
  *   - if rounding leaves no index with cumulative mass above u * Z, the draw
  *     returns the last index with r_i > 0; zero-mass tokens are never drawn;
- *   - if the residual mass is zero at a rejection (reachable only through
- *     rounding when q and p agree), the draw falls back to q_n and the status
- *     word records SV_WARN_ZERO_MASS;
+ *   - if the residual mass is zero at a rejection, the draw falls back to q_n
+ *     and the status word records SV_WARN_ZERO_MASS.  With draft tokens drawn
+ *     from p, as the method requires, this is reachable only through rounding
+ *     when q and p agree; a token that p gives no mass can also reach it (for
+ *     instance under greedy sampling, a token that is not the draft's argmax
+ *     while the two argmaxes agree);
  *   - a sequence with a draft token outside [0, V), or with any logit row
  *     holding NaN or +inf or no finite entry, emits nothing:
  *     out_num_accepted[b] = 0 and out_tokens[b, :] = -1, and the status word

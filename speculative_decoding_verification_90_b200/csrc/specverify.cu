@@ -205,28 +205,44 @@ cudaError_t launch_sampling(const specsamp::SampParams& p, long rows, int per, c
 
 // Row maps null: the logit buffers hold one row per position, [B, G+1, V] and
 // [B, G, V].  Otherwise `target_rows` / `draft_rows` rows that the maps index.
-sv_status enqueue(specverify_t h, const void* target, const void* draft, const int32_t* tokens,
-                  const float* u_accept, const float* u_resample, float temperature,
-                  int32_t* out_tokens, int32_t* out_num_accepted, cudaStream_t stream,
-                  const int32_t* target_map = nullptr, const int32_t* draft_map = nullptr,
-                  long target_rows = -1, long draft_rows = -1) {
+// Every argument check of a verification call: null and alignment tests,
+// the temperature and log2(e)/T range.  Runs before anything is enqueued.
+sv_status check_args(const specverify_ctx* h, const void* target, const void* draft,
+                     const int32_t* tokens, const float* u_accept, const float* u_resample,
+                     float temperature, const int32_t* out_tokens,
+                     const int32_t* out_num_accepted, const int32_t* target_map,
+                     const int32_t* draft_map) {
   const int G = h->gamma;
   const size_t es = elem_size(h->dtype);
   if (!target || !u_resample || !out_tokens || !out_num_accepted) return SV_ERR_INVALID_ARG;
   if (G > 0 && (!draft || !tokens || !u_accept)) return SV_ERR_INVALID_ARG;
-  if (target_rows < 0) target_rows = static_cast<long>(h->batch) * (G + 1);
-  if (draft_rows < 0) draft_rows = static_cast<long>(h->batch) * G;
   if (!aligned_to(target_map, 4) || !aligned_to(draft_map, 4)) return SV_ERR_INVALID_ARG;
   if (!aligned_to(target, es) || (G > 0 && !aligned_to(draft, es))) return SV_ERR_INVALID_ARG;
   if (!aligned_to(tokens, 4) || !aligned_to(u_accept, 4) || !aligned_to(u_resample, 4) ||
       !aligned_to(out_tokens, 4) || !aligned_to(out_num_accepted, 4))
     return SV_ERR_INVALID_ARG;
   if (!std::isfinite(temperature) || !(temperature > 0.f)) return SV_ERR_INVALID_ARG;
+  const double c = 1.4426950408889634074 / static_cast<double>(temperature);
+  if (!(c < 1e30)) return SV_ERR_INVALID_ARG;
+  return SV_OK;
+}
+
+sv_status enqueue(specverify_t h, const void* target, const void* draft, const int32_t* tokens,
+                  const float* u_accept, const float* u_resample, float temperature,
+                  int32_t* out_tokens, int32_t* out_num_accepted, cudaStream_t stream,
+                  const int32_t* target_map = nullptr, const int32_t* draft_map = nullptr,
+                  long target_rows = -1, long draft_rows = -1) {
+  const int G = h->gamma;
+  const sv_status chk = check_args(h, target, draft, tokens, u_accept, u_resample, temperature,
+                                   out_tokens, out_num_accepted, target_map, draft_map);
+  if (chk != SV_OK) return chk;
+  const size_t es = elem_size(h->dtype);
+  if (target_rows < 0) target_rows = static_cast<long>(h->batch) * (G + 1);
+  if (draft_rows < 0) draft_rows = static_cast<long>(h->batch) * G;
 
   // log2(e)/T = c_hi + c_lo with c_hi rounded toward zero, so c_lo >= 0;
   // c_lo is kept a normal positive float so that -inf * c_lo stays -inf
   const double c = 1.4426950408889634074 / static_cast<double>(temperature);
-  if (!(c < 1e30)) return SV_ERR_INVALID_ARG;
   float c_hi = static_cast<float>(c);
   if (static_cast<double>(c_hi) > c) c_hi = std::nextafter(c_hi, 0.f);
   float c_lo = static_cast<float>(c - static_cast<double>(c_hi));
@@ -838,6 +854,13 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
   h.draw_ticket = reinterpret_cast<unsigned*>(base + offK);
   h.resid = reinterpret_cast<double*>(base + offR);
   h.status = reinterpret_cast<unsigned*>(base + offS);
+
+  // a rejected call enqueues nothing: every argument check runs before the
+  // array is touched
+  const sv_status chk = check_args(&h, target_logits, draft_logits, draft_tokens, u_accept,
+                                   u_resample, temperature, out_tokens, out_num_accepted,
+                                   nullptr, nullptr);
+  if (chk != SV_OK) return chk;
 
   // the array keeps the previous call's contents: the draw tickets and the
   // status word must start at zero

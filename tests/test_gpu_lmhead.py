@@ -64,11 +64,17 @@ def run_fused(w, lm=None):
             lm.close()
 
 
-def oracle_fused(w):
-    import os
+def oracle_logits(w):
     import oracle
     t = oracle.lm_logits(workloads.bits_to_f32(w.target_hidden), workloads.bits_to_f32(w.target_weight))
     d = oracle.lm_logits(workloads.bits_to_f32(w.draft_hidden), workloads.bits_to_f32(w.draft_weight))
+    return t, d
+
+
+def oracle_fused(w, logits=None):
+    import os
+    import oracle
+    t, d = logits if logits is not None else oracle_logits(w)
     return oracle.verify(t, d, w.tokens, w.u_accept, w.u_resample,
                          float(np.float32(w.temperature)), threads=os.cpu_count() or 1)
 
@@ -76,7 +82,8 @@ def oracle_fused(w):
 def _parity(w, name):
     import parity
     g = run_fused(w)
-    o = oracle_fused(w)
+    logits = oracle_logits(w)
+    o = oracle_fused(w, logits)
     old = parity.MARGIN
     parity.MARGIN = FUSED_MARGIN
     try:
@@ -84,14 +91,16 @@ def _parity(w, name):
                                 np.zeros((w.batch, w.gamma + 1, 1), np.float32),
                                 np.zeros((w.batch, w.gamma, 1), np.float32), w.tokens,
                                 w.u_accept, w.u_resample)
-        s = compare(wl, g, o)
+        s = compare(wl, g, o, logits=logits)
     finally:
         parity.MARGIN = old
+    parity.record(s, name)
     print(f"\n[{name}] seqs={s['sequences']} hard={len(s['hard'])} margin={len(s['margin_cases'])} "
           f"dq={s.get('max_dq')} dp={s.get('max_dp')} lseT={s.get('max_target_lse_abs')} "
           f"lseD={s.get('max_draft_lse_abs')} dz={s.get('max_dz')}")
     assert not s["hard"], s["hard"][:5]
     assert len(s["margin_cases"]) <= max(1, 0.05 * s["sequences"]), s
+    assert len(s["unresolved"]) <= max(1, 0.01 * s["sequences"]), s
     for k in ("max_dq", "max_dp", "max_dz"):
         if k in s:
             assert s[k] <= FUSED_PROB_TOL, s

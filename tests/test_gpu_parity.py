@@ -224,6 +224,43 @@ def test_masked_vocab_entries_and_temperatures():
         _check(wl, f"masked T={T}")
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("V", [64, 4099, 152064])
+def test_zero_residual_mass_falls_back_to_target(dtype, V):
+    """Rows equal except at the drafted token t of the rejecting position, where
+    the target logit is -1000 (q(t) underflows to 0) and the draft's -690
+    (-688 in bf16; p(t) about 1e-300): t is rejected with ratio 0, every other
+    q(i) equals p(i), so the residual max(0, q - p) has no mass.  The draw then
+    comes from q at that position with the same uniform, and the ZERO_MASS
+    warning is raised.  At V = 152064 the draw's recomputation of q's tile
+    masses covers the whole row in one place (the rows the other draw warps
+    had covered)."""
+    rng = np.random.default_rng(V)
+    B, G = 24, 2
+    tgt = (rng.standard_normal((B, G + 1, V)) * 2).astype(np.float32)
+    drf = tgt[:, :G].copy()
+    n = rng.integers(0, G, size=B)
+    tok = np.zeros((B, G), np.int32)
+    for b in range(B):
+        for j in range(G):
+            tok[b, j] = int(np.argmax(tgt[b, j]))
+        t = int(rng.integers(0, V))
+        tok[b, n[b]] = t
+        tgt[b, n[b], t] = -1000.0
+        drf[b, n[b], t] = -690.0
+    wl = workloads._finish(f"zero_mass_{V}_{dtype}", dtype, 1.0, tgt, drf, rng, tokens=tok)
+    wl.u_accept[:] = 0.5
+    g = gpu_run(wl)
+    o = oracle_run(wl)
+    assert (o["seq_status"] == 18).all()
+    assert g["bits"] == 4 and g["status"] == 18
+    np.testing.assert_array_equal(g["out_num_accepted"], n)
+    s = compare(wl, g, o, check_probs=False)
+    _report(f"zero mass V={V} {dtype}", s)
+    assert not s["unresolved"]
+    assert_parity(s)
+
+
 def test_tokens_at_vocab_edges():
     wl = _small(17, 30, 3, 777, "f32", mix=0.6)
     wl.tokens[:, 0] = 0

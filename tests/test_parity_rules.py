@@ -7,7 +7,7 @@ import pytest
 
 from speculative_decoding_verification_90_b200 import workloads
 
-from parity import RESID_RESOLVE, compare, compare_sampling, oracle_run_sampling
+from parity import RESID_RESOLVE, compare, compare_sampling, oracle_run, oracle_run_sampling
 
 oracle = pytest.importorskip("oracle")
 
@@ -69,3 +69,45 @@ def test_unresolved_draw_checks_validity():
     g["out_tokens"][b, n] = wl.vocab        # out of range
     s = compare(wl, g, o, check_probs=False)
     assert [h[0] for h in s["hard"]] == [b]
+
+
+def test_unresolved_plain_draw_needs_residual_support():
+    """Plain step: an unresolved residual draw passes only with a token of the
+    residual's support (q_n > p_n at fp32 precision); a token the draft
+    favours, or one outside [0, V), is a hard difference; the count of
+    unresolved draws is capped."""
+    from parity import assert_parity
+    wl = _small()
+    o = oracle_run(wl)
+    b = _rejected(o, wl.gamma)[0]
+    n = int(o["out_num_accepted"][b])
+    o["resid_mass"][b] = 1e-12
+    T = float(np.float32(wl.temperature))
+    q = oracle.softmax(wl.target[b, n], T)[0]
+    p = oracle.softmax(wl.draft[b, n], T)[0]
+    d = q - p
+    d[int(o["out_tokens"][b, n])] = 0.0
+    favoured_by_q, favoured_by_p = int(np.argmax(d)), int(np.argmin(d))
+    assert d[favoured_by_q] > 0 > d[favoured_by_p]
+    g = _copy(o)
+    g["out_tokens"][b, n] = favoured_by_q
+    s = compare(wl, g, o, check_probs=False)
+    assert not s["hard"] and [u[0] for u in s["unresolved"]] == [b]
+    assert_parity(s, max_unresolved_frac=0.0, report=False)   # one unresolved draw is allowed
+    g["out_tokens"][b, n] = favoured_by_p
+    s = compare(wl, g, o, check_probs=False)
+    assert [h[0] for h in s["hard"]] == [b]
+    # a second unresolved sequence exceeds the cap of max(1, 1% of 8)
+    b2 = [c for c in _rejected(o, wl.gamma) if c != b][0]
+    n2 = int(o["out_num_accepted"][b2])
+    o["resid_mass"][b2] = 1e-12
+    q2 = oracle.softmax(wl.target[b2, n2], T)[0]
+    p2 = oracle.softmax(wl.draft[b2, n2], T)[0]
+    d2 = q2 - p2
+    d2[int(o["out_tokens"][b2, n2])] = 0.0
+    g["out_tokens"][b, n] = favoured_by_q
+    g["out_tokens"][b2, n2] = int(np.argmax(d2))
+    s = compare(wl, g, o, check_probs=False)
+    assert not s["hard"] and len(s["unresolved"]) == 2
+    with pytest.raises(AssertionError):
+        assert_parity(s, report=False)
