@@ -60,6 +60,10 @@ KERNEL_SOURCES = [
 ]
 
 
+# kernels of one plain step: statistics (which also takes each sequence's
+# decision) and draw
+LAUNCHES_PER_STEP = 2
+
 # sampling-variant settings timed by the bench: name -> (temperature, top_k, top_p);
 # None = the workload's temperature
 SAMPLING_SETTINGS = {"greedy": (0.0, 0, 1.0), "top_k50_top_p0.9": (None, 50, 0.9),
@@ -434,19 +438,20 @@ def run_ours(args):
                        "l2": ("inputs larger than L2 (%.0f MB per step, %d rotating set(s))"
                               % (step_bytes / 1e6, n_sets)),
                        "launch": {"blocks_per_row": slices, "threads": threads,
-                                  "draw_blocks_per_sequence": sv_draw}},
+                                  "draw_blocks_per_sequence_max": sv_draw}},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                          "algorithmic_bytes_per_launch": step_bytes,
                          "kernel": "stats_kernel (streams every logit once)"},
-            "kernels_us_per_step": {"stats": 1e3 * kern["stats_ms"],
-                                    "decide_and_draw": 1e3 * kern["draw_ms"],
+            "kernels_us_per_step": {"stats_and_decide": 1e3 * kern["stats_ms"],
+                                    "draw": 1e3 * kern["draw_ms"],
                                     "runs": kern["runs"]},
             "step_hbm_gbs": step_bytes / (ms / 1e3 / args.steps) / 1e9,
+            "step_frac": step_bytes / (ms / 1e3 / args.steps) / 1e9 / peak,
             "emitted_tokens_per_step": emitted,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
             "status_after": st,

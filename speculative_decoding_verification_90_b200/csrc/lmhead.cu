@@ -40,7 +40,8 @@ struct specverify_lmhead_ctx {
   int batch = 0, gamma = 0, vocab = 0, hidden = 0;
   int ntiles = 0;
   int num_sms = 148;
-  int draw_slices = 1;
+  int draw_slices = 1;  // the draw kernel's grid (blocks)
+  long draw_tiles = 1;  // tiles per fp32 row drawn from
   void* ws = nullptr;
   RowPartial* partial = nullptr;   // [(nT + nD) * ntiles] one per row and 256-column tile
   RowPartial* combined = nullptr;  // [nT + nD] one per row
@@ -217,18 +218,12 @@ sv_status specverify_lmhead_create(specverify_lmhead_t* out, int batch, int gamm
   h->hidden = hidden;
   h->num_sms = sms;
   h->ntiles = (vocab + lmhead::kBN - 1) / lmhead::kBN;
-  // draw blocks per sequence for fp32 rows (the plain step's rule: about 48 KB
-  // of a row per block, at most one block per 4 tiles of 32 groups, at most 64)
-  {
-    const long groups = (vocab + 3) / 4;
-    const long tiles = (groups + specverify::kTile - 1) / specverify::kTile;
-    long ds = (2L * vocab * 4 + 48 * 1024 - 1) / (48 * 1024);
-    if (ds > tiles / 4) ds = tiles / 4;
-    if (ds > 64) ds = 64;
-    h->draw_slices = static_cast<int>(ds < 1 ? 1 : ds);
-  }
+  // the draw on fp32 rows: the plain step's grid rule (one resident wave at
+  // most, one warp per tile at least)
+  h->draw_tiles = specverify::draw_tiles_per_row(vocab, 4);
+  h->draw_slices = static_cast<int>(specverify::draw_grid(batch, h->draw_tiles, 64, sms));
   const size_t nB = static_cast<size_t>(batch);
-  const size_t tiles32 = static_cast<size_t>(((vocab + 3) / 4 + specverify::kTile - 1) / specverify::kTile);
+  const size_t tiles32 = static_cast<size_t>(h->draw_tiles);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -401,6 +396,7 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   p.decision = h->decision;
   p.draw_mass = h->draw_mass;
   p.draw_ticket = h->draw_ticket;
+  p.seq_ticket = nullptr;
   p.resid_mass = h->resid;
   p.status = h->status;
   p.batch = B;
@@ -408,12 +404,7 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   p.vocab = V;
   p.slices = 1;  // the per-tile partials are folded first
   p.groups_per_slice = 0;
-  p.draw_slices = h->draw_slices;
-  {
-    const long groups = (V + 3) / 4;
-    const long ntiles32 = (groups + specverify::kTile - 1) / specverify::kTile;
-    p.groups_per_draw = static_cast<int>((ntiles32 + h->draw_slices - 1) / h->draw_slices) * specverify::kTile;
-  }
+  p.draw_tiles = h->draw_tiles;
   p.c_hi = c_hi;
   p.c_lo = c_lo;
   p.c = c;
@@ -462,11 +453,9 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   const bool aligned = (static_cast<size_t>(V) * 4) % 16 == 0;
   if (e == cudaSuccess)
     e = aligned ? launch_plain(specverify::draw_kernel<float, true>,
-                               static_cast<unsigned>(static_cast<long>(B) * h->draw_slices),
-                               specverify::kDrawThreads, s, p)
+                               static_cast<unsigned>(h->draw_slices), specverify::kDrawThreads, s, p)
                 : launch_plain(specverify::draw_kernel<float, false>,
-                               static_cast<unsigned>(static_cast<long>(B) * h->draw_slices),
-                               specverify::kDrawThreads, s, p);
+                               static_cast<unsigned>(h->draw_slices), specverify::kDrawThreads, s, p);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
   if (e != cudaSuccess) return cuda_fail(e);
   return SV_OK;

@@ -31,7 +31,7 @@ struct specverify_ctx {
   sv_dtype dtype = SV_DTYPE_F32;
   int slices = 1, threads = 128;
   int max_slices = 1;  // the partial-statistics workspace holds this many per position
-  int draw_slices = 1; // draw blocks per sequence
+  int draw_slices = 64; // at most this many draw blocks per sequence
   int num_sms = 148;
   void* ws = nullptr;  // one device allocation for the whole workspace
   RowPartial* partial = nullptr;
@@ -41,6 +41,7 @@ struct specverify_ctx {
   SeqDecision* decision = nullptr;
   double* draw_mass = nullptr;
   unsigned* draw_ticket = nullptr;
+  unsigned* seq_ticket = nullptr;
   double* resid = nullptr;
   unsigned* status = nullptr;
   specsamp::SampRow* samp_rows = nullptr;          // sampling variants: per-row filter
@@ -102,23 +103,16 @@ void default_shape(specverify_ctx* h) {
   h->threads = threads;
 }
 
-// Draw blocks per sequence: about 48 KB of the rows drawn from per block,
-// more when the batch is too small to fill the SMs, and at least one
-// 32-group tile per warp.
-int draw_shape(const specverify_ctx* h) {
-  const long bytes = 2L * h->vocab * static_cast<long>(elem_size(h->dtype));
-  long s2 = (bytes + 49151) / 49152;
-  const long slots = static_cast<long>(h->num_sms) * 8;
-  if (h->batch > 0) {
-    const long fill = (slots + h->batch - 1) / h->batch;
-    if (s2 < fill) s2 = fill;
-  }
-  const long ntiles = (num_groups(h) + specverify::kTile - 1) / specverify::kTile;
-  const long by_tiles = ntiles / specverify::kDrawWarps;
-  if (s2 > by_tiles) s2 = by_tiles;
-  if (s2 > 64) s2 = 64;
-  if (s2 < 1) s2 = 1;
-  return static_cast<int>(s2);
+// Draw blocks per sequence, at most: the draw kernel's grid is also capped at
+// one resident wave and at one warp per tile, so the default only bounds it.
+int draw_shape(const specverify_ctx*) { return 64; }
+
+long draw_tiles(const specverify_ctx* h) {
+  return specverify::draw_tiles_per_row(h->vocab, group_elems(h->dtype));
+}
+
+unsigned draw_blocks(const specverify_ctx* h) {
+  return specverify::draw_grid(h->batch, draw_tiles(h), h->draw_slices, h->num_sms);
 }
 
 template <typename K, typename PP>
@@ -139,42 +133,50 @@ cudaError_t launch_pdl(K kernel, unsigned blocks, unsigned threads, cudaStream_t
   return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
-template <typename T, int NT, bool A>
+template <typename T, int NT, bool A, bool D>
 cudaError_t launch_stats_nt(const Params& p, long blocks, cudaStream_t s) {
-  specverify::stats_kernel<T, NT, A><<<static_cast<unsigned>(blocks), NT, 0, s>>>(p);
+  specverify::stats_kernel<T, NT, A, D><<<static_cast<unsigned>(blocks), NT, 0, s>>>(p);
   return cudaGetLastError();
 }
 
-// events[0..2] (may be null): before stats, after stats, after draw
+// One step.  Unmapped rows: the statistics kernel also takes each sequence's
+// decision; with row maps a decide kernel runs after it.  events[0..2] (may
+// be null): before stats, after stats (and decide), after draw.
 template <typename T, bool A>
-cudaError_t launch_step(const Params& p, int NT, cudaStream_t s, cudaEvent_t* ev) {
+cudaError_t launch_step(const Params& p, int NT, unsigned draw_blocks, cudaStream_t s,
+                        cudaEvent_t* ev) {
   const long rows = p.target_rows + p.draft_rows;
   const long blocks = rows * p.slices;
+  const bool fused = p.target_map == nullptr && p.draft_map == nullptr;
   cudaError_t e = cudaSuccess;
   if (ev) e = cudaEventRecord(ev[0], s);
   if (e != cudaSuccess) return e;
-  switch (NT) {
-    case 128: e = launch_stats_nt<T, 128, A>(p, blocks, s); break;
-    case 256: e = launch_stats_nt<T, 256, A>(p, blocks, s); break;
-    case 512: e = launch_stats_nt<T, 512, A>(p, blocks, s); break;
+  switch (NT * 2 + (fused ? 1 : 0)) {
+    case 256: e = launch_stats_nt<T, 128, A, false>(p, blocks, s); break;
+    case 257: e = launch_stats_nt<T, 128, A, true>(p, blocks, s); break;
+    case 512: e = launch_stats_nt<T, 256, A, false>(p, blocks, s); break;
+    case 513: e = launch_stats_nt<T, 256, A, true>(p, blocks, s); break;
+    case 1024: e = launch_stats_nt<T, 512, A, false>(p, blocks, s); break;
+    case 1025: e = launch_stats_nt<T, 512, A, true>(p, blocks, s); break;
     default: return cudaErrorInvalidValue;
+  }
+  if (e == cudaSuccess && !fused) {
+    const int per = specverify::kDecideThreads / specverify::kWarp;
+    e = launch_pdl(specverify::decide_kernel<T>, static_cast<unsigned>((p.batch + per - 1) / per),
+                   specverify::kDecideThreads, s, p);
   }
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
   if (e != cudaSuccess) return e;
-  const int per = specverify::kDecideThreads / specverify::kWarp;
-  e = launch_pdl(specverify::decide_kernel<T>, static_cast<unsigned>((p.batch + per - 1) / per),
-                 specverify::kDecideThreads, s, p);
-  if (e != cudaSuccess) return e;
-  e = launch_pdl(specverify::draw_kernel<T, A>,
-                 static_cast<unsigned>(static_cast<long>(p.batch) * p.draw_slices),
-                 specverify::kDrawThreads, s, p);
+  e = launch_pdl(specverify::draw_kernel<T, A>, draw_blocks, specverify::kDrawThreads, s, p);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
   return e;
 }
 
 template <typename T>
-cudaError_t launch_dtype(const Params& p, int NT, bool aligned, cudaStream_t s, cudaEvent_t* ev) {
-  return aligned ? launch_step<T, true>(p, NT, s, ev) : launch_step<T, false>(p, NT, s, ev);
+cudaError_t launch_dtype(const Params& p, int NT, unsigned draw_blocks, bool aligned,
+                         cudaStream_t s, cudaEvent_t* ev) {
+  return aligned ? launch_step<T, true>(p, NT, draw_blocks, s, ev)
+                 : launch_step<T, false>(p, NT, draw_blocks, s, ev);
 }
 
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -267,6 +269,7 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
   p.decision = h->decision;
   p.draw_mass = h->draw_mass;
   p.draw_ticket = h->draw_ticket;
+  p.seq_ticket = h->seq_ticket;
   p.resid_mass = h->resid;
   p.status = h->status;
   p.batch = h->batch;
@@ -275,11 +278,7 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
   const long ngroups = num_groups(h);
   p.slices = h->slices;
   p.groups_per_slice = static_cast<int>((ngroups + h->slices - 1) / h->slices);
-  p.draw_slices = h->draw_slices;
-  {
-    const long ntiles = (ngroups + specverify::kTile - 1) / specverify::kTile;
-    p.groups_per_draw = static_cast<int>((ntiles + h->draw_slices - 1) / h->draw_slices) * specverify::kTile;
-  }
+  p.draw_tiles = draw_tiles(h);
   p.c_hi = c_hi;
   p.c_lo = c_lo;
   p.c = static_cast<double>(c_hi) + static_cast<double>(c_lo);
@@ -291,9 +290,10 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
                        (static_cast<size_t>(h->vocab) * es) % 16 == 0;
   cudaEvent_t* ev = nullptr;
   if (h->prof_runs < h->prof_capacity) ev = h->events.data() + 3 * (h->prof_runs++);
+  const unsigned nd = draw_blocks(h);
   cudaError_t e = (h->dtype == SV_DTYPE_BF16)
-                      ? launch_dtype<__nv_bfloat16>(p, h->threads, aligned, stream, ev)
-                      : launch_dtype<float>(p, h->threads, aligned, stream, ev);
+                      ? launch_dtype<__nv_bfloat16>(p, h->threads, nd, aligned, stream, ev)
+                      : launch_dtype<float>(p, h->threads, nd, aligned, stream, ev);
   if (e != cudaSuccess) return cuda_fail(e);
   return SV_OK;
 }
@@ -347,7 +347,7 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   const size_t nB = static_cast<size_t>(batch);
   h->draw_slices = draw_shape(h);
   const size_t nPart = (nT + nD) * static_cast<size_t>(h->max_slices);
-  const size_t nDraw = nB * static_cast<size_t>((num_groups(h) + specverify::kTile - 1) / specverify::kTile);
+  const size_t nDraw = nB * static_cast<size_t>(draw_tiles(h));
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -360,7 +360,7 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   const size_t offP = take(nD * sizeof(PosInfo));
   const size_t offC = take(nB * sizeof(SeqDecision));
   const size_t offW = take(nDraw * sizeof(double));
-  const size_t offK = take(nB * sizeof(unsigned));
+  const size_t offK = take(2 * nB * sizeof(unsigned));  // draw tickets, then sequence tickets
   const size_t offR = take(nB * sizeof(double));
   const size_t offS = take(sizeof(unsigned));
   const size_t offSR = take((nT + nD) * sizeof(specsamp::SampRow));
@@ -379,6 +379,7 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   h->decision = reinterpret_cast<SeqDecision*>(base + offC);
   h->draw_mass = reinterpret_cast<double*>(base + offW);
   h->draw_ticket = reinterpret_cast<unsigned*>(base + offK);
+  h->seq_ticket = h->draw_ticket + nB;
   h->resid = reinterpret_cast<double*>(base + offR);
   h->status = reinterpret_cast<unsigned*>(base + offS);
   h->samp_rows = reinterpret_cast<specsamp::SampRow*>(base + offSR);
@@ -643,9 +644,7 @@ sv_status specverify_set_launch(specverify_t h, int slices, int threads, int dra
   if (!h) return SV_ERR_INVALID_ARG;
   if (slices < 1 || slices > h->max_slices) return SV_ERR_INVALID_ARG;
   if (threads != 128 && threads != 256 && threads != 512) return SV_ERR_INVALID_ARG;
-  const long ntiles = (num_groups(h) + specverify::kTile - 1) / specverify::kTile;
-  if (draw_slices > 64 || (draw_slices > 1 && draw_slices > ntiles / specverify::kDrawWarps))
-    return SV_ERR_INVALID_ARG;
+  if (draw_slices > 64) return SV_ERR_INVALID_ARG;
   h->slices = slices;
   h->threads = threads;
   h->draw_slices = (draw_slices >= 1) ? draw_slices : draw_shape(h);
@@ -821,8 +820,7 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
   const size_t nT = static_cast<size_t>(batch) * (gamma + 1);
   const size_t nD = static_cast<size_t>(batch) * gamma;
   const size_t nB = static_cast<size_t>(batch);
-  const size_t nDraw =
-      nB * static_cast<size_t>((num_groups(&h) + specverify::kTile - 1) / specverify::kTile);
+  const size_t nDraw = nB * static_cast<size_t>(draw_tiles(&h));
   size_t off = 0;
   auto take = [&](size_t bytes) {
     const size_t at = off;
@@ -835,7 +833,7 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
   const size_t offP = take(nD * sizeof(PosInfo));
   const size_t offC = take(nB * sizeof(SeqDecision));
   const size_t offW = take(nDraw * sizeof(double));
-  const size_t offK = take(nB * sizeof(unsigned));
+  const size_t offK = take(2 * nB * sizeof(unsigned));  // draw tickets, then sequence tickets
   const size_t offR = take(nB * sizeof(double));
   const size_t offS = take(sizeof(unsigned));
   if (off > kNoAllocScratchBytes) {
@@ -852,6 +850,7 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
   h.decision = reinterpret_cast<SeqDecision*>(base + offC);
   h.draw_mass = reinterpret_cast<double*>(base + offW);
   h.draw_ticket = reinterpret_cast<unsigned*>(base + offK);
+  h.seq_ticket = h.draw_ticket + nB;
   h.resid = reinterpret_cast<double*>(base + offR);
   h.status = reinterpret_cast<unsigned*>(base + offS);
 
@@ -862,10 +861,10 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
                                    nullptr, nullptr);
   if (chk != SV_OK) return chk;
 
-  // the array keeps the previous call's contents: the draw tickets and the
+  // the array keeps the previous call's contents: the tickets and the
   // status word must start at zero
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  e = cudaMemsetAsync(h.draw_ticket, 0, nB * sizeof(unsigned), s);
+  e = cudaMemsetAsync(h.draw_ticket, 0, 2 * nB * sizeof(unsigned), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h.status, 0, sizeof(unsigned), s);
   if (e != cudaSuccess) return cuda_fail(e);
   return enqueue(&h, target_logits, draft_logits, draft_tokens, u_accept, u_resample,

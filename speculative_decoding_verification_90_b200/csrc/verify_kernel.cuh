@@ -1,27 +1,30 @@
 // Speculative-sampling verification kernels for sm_100a.
 //
-// One verification step is three stream-ordered kernels (each later one
-// launched early through programmatic dependent launch and waiting for its
-// predecessor with a grid-dependency barrier):
+// One verification step of unmapped rows is two stream-ordered kernels (the
+// second launched early through programmatic dependent launch and waiting for
+// the first with a grid-dependency barrier):
 //
 //   stats   S blocks per logit row (every target row, then every draft
 //           row), each streaming its contiguous 1/S of the row with 128-bit
 //           coalesced loads, eight in flight per thread; each thread keeps a
 //           running sum of 2^(x c - o) against a lazily raised offset o; the
 //           block writes its (o, sum) partial (step 1 of the round: softmax
-//           statistics).  No atomics, no waits, the same work in every block:
-//           this is the kernel that moves all of the logit bytes.
-//   decide  one warp per sequence, one lane per position: the lane combines
-//           the position's partials into log2 sum_i 2^(x_i c), forms q(t),
-//           p(t) and the ratio, and a warp ballot finds the first rejection n
-//           (steps 2 and 3); writes the accepted prefix and what to draw from.
-//   draw    S' blocks per sequence over the rows drawn from (n < gamma:
-//           max(0, q_n - p_n) from target and draft row n; n == gamma: q of
-//           target row gamma); each block publishes the mass of every
-//           32-group tile of its share, and the block that takes the
-//           sequence's ticket last finds, by a block-wide prefix scan over
-//           the tile masses, the tile that holds u * Z and scans it one group
-//           per lane in index order (step 4).
+//           statistics).  This is the kernel that moves all of the logit
+//           bytes.  The block that finishes a sequence's last slice (an
+//           atomic ticket per sequence) then takes its decision with one
+//           warp, one lane per position: the lane combines the position's
+//           partials into log2 sum_i 2^(x_i c), forms q(t), p(t) and the
+//           ratio, and a warp ballot finds the first rejection n (steps 2
+//           and 3); it writes the accepted prefix and what to draw from.
+//   draw    the grid's warps split every tile of every sequence's rows drawn
+//           from (n < gamma: max(0, q_n - p_n) from target and draft row n;
+//           n == gamma: q of target row gamma) into even contiguous runs,
+//           write each tile's mass, and the warp that completes a sequence's
+//           tiles (an atomic ticket) locates u * Z by a warp scan over the
+//           tile masses and one re-read tile (step 4).
+//
+// With row maps (rows shared between positions) or the LM-head-fused step, a
+// separate decide kernel (one warp per sequence) runs between the two.
 //
 // No thread ever waits for another block (the only hand-off inside a kernel
 // is an atomic ticket, never a spin).
@@ -113,13 +116,13 @@ struct Params {
   SeqDecision* decision;     // [B]
   double* draw_mass;         // [B * tiles of a row] mass of each 32-group tile of the draw
   unsigned* draw_ticket;     // [B], zero between launches
+  unsigned* seq_ticket;      // [B], zero between launches (statistics slices done)
   double* resid_mass;        // [B]
   unsigned* status;          // [1]
   int batch, gamma, vocab;
   int slices;                // S stats blocks per position
   int groups_per_slice;      // 16-byte groups of the vocabulary per stats block
-  int draw_slices;           // S2 draw blocks per sequence
-  int groups_per_draw;       // groups per draw block (whole 32-group tiles)
+  long draw_tiles;           // tiles of kTile groups per row drawn from
   float c_hi, c_lo;          // log2(e)/T = c_hi + c_lo, c_lo > 0
   double c;                  // c_hi + c_lo, exactly
   // fused LM-head form: the logits at the draft tokens were picked out by the
@@ -317,45 +320,6 @@ constexpr float kA3 = 0.055504108664821576f;
 constexpr float kA4 = 0.009618129107628477f;
 constexpr float kA5 = 0.0013333558146428441f;
 
-// r / fT for the VEC elements of one group: residual max(0, q - p) or target
-// q; the caller multiplies sums of r by fT.  L = log2(q/p) comes from the
-// logit difference (exact for bf16 inputs) and p = q 2^-L.  L >= 1/8 gives
-// q - p (q >= 1.09 p: at most 3.6 bits cancel); 0 < L < 1/8 gives
-// p (2^L - 1) from its Taylor series in L (to L^5, truncation below 7e-9
-// relative); L <= 0 gives q - p <= 0, which the final max(., 0) turns into 0.
-// The infinite cases need no test: a draft logit of -inf gives L = +inf,
-// p = 0 and r = q; a target logit of -inf gives q = 0, L = -inf and r = 0
-// (the NaN of 0 * 2^inf is discarded by the selects).
-template <typename T, int kMode>
-__device__ __forceinline__ void group_mass(const uint4& vt, const uint4& vd, const DrawConsts& k,
-                                           float (&r)[Elem<T>::kVec]) {
-  constexpr int kVec = Elem<T>::kVec;
-  float xt[kVec];
-  Elem<T>::unpack(vt, xt);
-  if constexpr (kMode == kDrawTarget) {
-#pragma unroll
-    for (int e = 0; e < kVec; ++e) r[e] = ex2(arg2(xt[e], k.c_hi, k.c_lo, k.lt_hi));
-  } else {
-    float xd[kVec];
-    Elem<T>::unpack(vd, xd);
-#pragma unroll
-    for (int e = 0; e < kVec; ++e) {
-      const float q = ex2(arg2(xt[e], k.c_hi, k.c_lo, k.lt_hi));
-      const float dx = xt[e] - xd[e];
-      const float L = fmaf(dx, k.c_hi, -k.k_hi) + fmaf(dx, k.c_lo, -k.k_lo);
-      const float p = q * ex2(-L);
-      float t = kA5;
-      t = fmaf(t, L, kA4);
-      t = fmaf(t, L, kA3);
-      t = fmaf(t, L, kA2);
-      t = fmaf(t, L, kA1);
-      const float small = p * (t * L);
-      const float res = (L > 0.f && L < 0.125f) ? small : q - p;
-      r[e] = fmaxf(res, 0.f);  // NaN (0 * inf) becomes 0 here
-    }
-  }
-}
-
 __device__ __forceinline__ void split2(double v, float& hi, float& lo) {
   hi = static_cast<float>(v);
   lo = static_cast<float>(v - static_cast<double>(hi));
@@ -459,7 +423,176 @@ __device__ __forceinline__ void block_scan(double v, double& incl, double& excl,
 }
 
 // ---------------------------------------------------------------------------
-// kernel 1: streaming statistics
+// steps 2 and 3: the decision of one sequence (one warp, one lane per position)
+// ---------------------------------------------------------------------------
+
+constexpr int kDecideThreads = 128;
+constexpr int kMaxGamma = 255;
+
+// One row's partial.  kL2: read through L2 only, for partials that other
+// blocks of the running kernel wrote (L1 is not coherent with their stores).
+template <bool kL2>
+__device__ __forceinline__ void load_partial(const RowPartial* p, float& o, double& s) {
+  if constexpr (kL2) {
+    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p));
+    s = __hiloint2double(static_cast<int>(v.y), static_cast<int>(v.x));
+    o = __uint_as_float(v.z);
+  } else {
+    s = p->s;
+    o = p->o;
+  }
+}
+
+// (o, s) partials of one row combined in two passes, so that the fp64
+// exponentials of the second pass are independent of one another
+template <bool kL2>
+__device__ __forceinline__ double row_lse2(const RowPartial* parts, int S, int& valid) {
+  float O = -INFINITY;
+  for (int r = 0; r < S; ++r) {
+    float o;
+    double s;
+    load_partial<kL2>(parts + r, o, s);
+    O = fmaxf(O, o);
+  }
+  double sum = 0.0;
+  for (int r = 0; r < S; ++r) {
+    float o;
+    double s;
+    load_partial<kL2>(parts + r, o, s);
+    sum += (o == -INFINITY) ? s * 0.0 : s * exp2(static_cast<double>(o) - O);  // NaN survives
+  }
+  valid = (O != -INFINITY) && isfinite(sum) && sum > 0.0;
+  return static_cast<double>(O) + log2(sum);  // log2 sum_i 2^(x_i c)
+}
+
+// The decision of sequence b by the calling warp (all 32 lanes): lane j
+// combines the partials of position j's rows, forms q(t), p(t) and the ratio
+// in fp64 and tests u < ratio (step 2); a warp ballot finds the first
+// rejection n (step 3).  Writes the accepted prefix, the padding, the count,
+// the per-position readback records and what the draw kernel draws from.
+template <typename T, bool kL2>
+__device__ __forceinline__ void decide_sequence(const Params& P, int b) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  const int G = P.gamma, V = P.vocab, S = P.slices;
+  const double c = P.c;
+  int n = G;          // first rejection, gamma if none
+  unsigned bits = 0;  // data errors of the sequence
+  double lT_n = 0.0, lD_n = 0.0;
+  long tr_n = 0, dr_n = 0;
+  for (int base = 0; base <= G; base += kWarp) {
+    const int j = base + lane;
+    int flag = kFlagAccept;
+    bool tok_bad = false, row_bad = false, map_bad = false;
+    double lT = 0.0, lD = 0.0;
+    long tr = 0, dr = 0;
+    if (j <= G) {
+      const long position = static_cast<long>(b) * (G + 1) + j;
+      const long pj = static_cast<long>(b) * G + j;
+      const bool has_draft = j < G;
+      // rows of the logit buffers that hold this position
+      tr = P.target_map ? static_cast<long>(P.target_map[position]) : position;
+      dr = has_draft ? (P.draft_map ? static_cast<long>(P.draft_map[pj]) : pj) : 0;
+      map_bad = tr < 0 || tr >= P.target_rows || (has_draft && (dr < 0 || dr >= P.draft_rows));
+      // the acceptance test's inputs first: their loads overlap the combine
+      int t = 0;
+      float u = 0.f, xt = 0.f, xd = 0.f;
+      if (has_draft) {
+        t = P.tokens[pj];
+        u = P.u_accept[pj];
+        tok_bad = (t < 0 || t >= V);
+        if (!tok_bad && !map_bad) {
+          xt = P.gathered_target ? P.gathered_target[tr]
+                                 : Elem<T>::load1(static_cast<const T*>(P.target) + tr * V, t);
+          xd = P.gathered_draft ? P.gathered_draft[dr]
+                                : Elem<T>::load1(static_cast<const T*>(P.draft) + dr * V, t);
+        }
+      }
+      int validT = 0, validD = 1;
+      if (!map_bad) {
+        lT = row_lse2<kL2>(P.partial + tr * S, S, validT);
+        if (has_draft) lD = row_lse2<kL2>(P.partial + (P.target_rows + dr) * S, S, validD);
+      }
+      P.tstat[position] = RowStat{lT, validT, 0};
+      if (has_draft) P.dstat[pj] = RowStat{lD, validD, 0};
+      row_bad = !map_bad && (!validT || !validD);
+      if (has_draft) {
+        PosInfo info{0.0, 0.0, 0.0, kFlagReject, 0};
+        if (tok_bad) {
+          info.flag = kFlagTokenRange;
+        } else if (row_bad || map_bad) {
+          info.flag = kFlagNonFinite;
+        } else {
+          const double lq = static_cast<double>(xt) * c - lT;  // log2 q(t)
+          const double lp = static_cast<double>(xd) * c - lD;  // log2 p(t)
+          info.q_tok = exp2(lq);
+          info.p_tok = exp2(lp);
+          if (!(info.q_tok > 0.0)) info.ratio = 0.0;
+          else if (!(info.p_tok > 0.0)) info.ratio = INFINITY;
+          else info.ratio = exp2(lq - lp);
+          info.flag = (static_cast<double>(u) < info.ratio) ? kFlagAccept : kFlagReject;
+        }
+        P.pos[pj] = info;
+        flag = info.flag;
+      }
+    }
+    const unsigned rej = __ballot_sync(0xffffffffu, j < G && flag == kFlagReject);
+    if (__ballot_sync(0xffffffffu, tok_bad)) bits |= kStatTokenRange;
+    if (__ballot_sync(0xffffffffu, row_bad)) bits |= kStatNonFinite;
+    if (__ballot_sync(0xffffffffu, map_bad)) bits |= kStatRowIndex;
+    // the statistics the draw needs live in lane (n - base) of this chunk
+    const int first = rej ? base + __ffs(rej) - 1 : G;
+    const bool here = (n == G) && (first < G || G < base + kWarp);
+    if (n == G) n = first;
+    const int src = (n - base) & (kWarp - 1);
+    const double lTs = __shfl_sync(0xffffffffu, lT, src);
+    const double lDs = __shfl_sync(0xffffffffu, lD, src);
+    const long trs = __shfl_sync(0xffffffffu, tr, src);
+    const long drs = __shfl_sync(0xffffffffu, dr, src);
+    if (here) {
+      lT_n = lTs;
+      lD_n = lDs;
+      tr_n = trs;
+      dr_n = drs;
+    }
+  }
+  const long bo = static_cast<long>(b) * (G + 1);
+  if (bits) {
+    for (int q = lane; q <= G; q += kWarp) P.out_tokens[bo + q] = -1;
+    if (lane == 0) {
+      P.out_num_accepted[b] = 0;
+      P.resid_mass[b] = NAN;
+      P.decision[b] = SeqDecision{0.0, 0.0, 0, 0, 0, kDrawNone, bits, 0.f, 0.f, 0.f, 1.f};
+      atomicOr(P.status, bits);
+    }
+  } else {
+    // accepted prefix and padding; the drawn token at n is the draw kernel's
+    for (int q = lane; q <= G; q += kWarp) {
+      if (q < n) P.out_tokens[bo + q] = P.tokens[static_cast<long>(b) * G + q];
+      else if (q > n) P.out_tokens[bo + q] = -1;
+    }
+    if (lane == 0) {
+      P.out_num_accepted[b] = n;
+      SeqDecision d{lT_n, lD_n, P.draw_compact ? b : tr_n, P.draw_compact ? b : dr_n, n,
+                    (n < G) ? kDrawResidual : kDrawTarget, 0u, 0.f, 0.f, 0.f, 1.f};
+      float lt_lo;
+      split2(lT_n, d.lt_hi, lt_lo);
+      split2(lT_n - lD_n, d.k_hi, d.k_lo);
+      d.fT = static_cast<float>(exp2(-static_cast<double>(lt_lo)));
+      P.decision[b] = d;
+    }
+  }
+}
+
+// Called from the statistics kernel: kept out of line so that the streaming
+// loop's register allocation does not carry the decision's.
+template <typename T>
+__device__ __noinline__ void decide_sequence_l2(const Params* P, int b) {
+  __threadfence();  // every lane reads the other blocks' partials after the ticket
+  decide_sequence<T, true>(*P, b);
+}
+
+// ---------------------------------------------------------------------------
+// kernel 1: streaming statistics (and, unmapped, each sequence's decision)
 // ---------------------------------------------------------------------------
 
 template <int NT>
@@ -467,10 +600,14 @@ constexpr int min_blocks() {
   return 1024 / NT;  // caps registers at 64 per thread
 }
 
-template <typename T, int NT, bool kAligned>
-__global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Params P) {
+// kDecide (unmapped rows only): the block that completes the last slice of a
+// sequence's 2 gamma + 1 rows takes that sequence's decision with its first
+// warp, so the decisions are made while the other rows still stream and no
+// separate decide launch sits between the statistics and the draw.
+template <typename T, int NT, bool kAligned, bool kDecide>
+__global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const __grid_constant__ Params P) {
   constexpr int kVec = Elem<T>::kVec;
-  const int G = P.gamma, V = P.vocab, S = P.slices;
+  const int V = P.vocab, S = P.slices;
   // one unit = one block = one slice of one row; the target tensor's rows
   // come first, then the draft tensor's, so the grid walks memory in order
   const long unit = blockIdx.x;
@@ -479,7 +616,6 @@ __global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Param
   const long nT = P.target_rows;
   const T* row = (r < nT) ? static_cast<const T*>(P.target) + r * V
                           : static_cast<const T*>(P.draft) + (r - nT) * V;
-  (void)G;
   const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
   long glo = static_cast<long>(slice) * P.groups_per_slice;
   long ghi = glo + P.groups_per_slice;
@@ -487,423 +623,394 @@ __global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Param
   if (ghi > ngroups) ghi = ngroups;
   const RowPartial part = slice_stats<T, NT, kAligned, 8>(row, glo, ghi, V, P.c_hi, P.c_lo);
   if (threadIdx.x == 0) P.partial[unit] = part;
+  if constexpr (kDecide) {
+    __shared__ int sm_b;
+    if (threadIdx.x == 0) {
+      const int G = P.gamma;
+      const int b = (r < nT || G == 0) ? static_cast<int>(r / (G + 1))
+                                       : static_cast<int>((r - nT) / G);
+      __threadfence();  // this block's partial is visible before its ticket
+      const unsigned need = static_cast<unsigned>((2 * G + 1) * S);
+      const unsigned old = atomicAdd(P.seq_ticket + b, 1u);
+      sm_b = (old == need - 1) ? b : -1;
+      if (sm_b >= 0) {
+        __threadfence();        // every partial of the sequence is visible
+        P.seq_ticket[b] = 0u;   // ready for the next launch
+      }
+    }
+    __syncthreads();
+    if (sm_b >= 0 && threadIdx.x < kWarp) decide_sequence_l2<T>(&P, sm_b);
+  }
   cudaTriggerProgrammaticLaunchCompletion();
 }
 
 // ---------------------------------------------------------------------------
-// kernel 2: decide (one warp per sequence, one lane per position)
+// kernel 2: decide (mapped rows, the LM-head-fused step): one warp per sequence
 // ---------------------------------------------------------------------------
-
-constexpr int kDecideThreads = 128;
-constexpr int kMaxGamma = 255;
-
-// (o, s) partials of one row combined in two passes, so that the fp64
-// exponentials of the second pass are independent of one another
-__device__ __forceinline__ double row_lse2(const RowPartial* parts, int S, int& valid) {
-  float O = -INFINITY;
-  for (int r = 0; r < S; ++r) O = fmaxf(O, parts[r].o);
-  double sum = 0.0;
-  for (int r = 0; r < S; ++r) {
-    const float o = parts[r].o;
-    const double s = parts[r].s;
-    sum += (o == -INFINITY) ? s * 0.0 : s * exp2(static_cast<double>(o) - O);  // NaN survives
-  }
-  valid = (O != -INFINITY) && isfinite(sum) && sum > 0.0;
-  return static_cast<double>(O) + log2(sum);  // log2 sum_i 2^(x_i c)
-}
 
 template <typename T>
 __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) {
   // the statistics of the previous kernel must be complete and visible
   cudaGridDependencySynchronize();
-  const int lane = threadIdx.x & (kWarp - 1);
   const int b = blockIdx.x * (kDecideThreads / kWarp) + (threadIdx.x >> 5);
-  if (b < P.batch) {  // warp-uniform
-    const int G = P.gamma, V = P.vocab, S = P.slices;
-    const double c = P.c;
-    int n = G;          // first rejection, gamma if none
-    unsigned bits = 0;  // data errors of the sequence
-    double lT_n = 0.0, lD_n = 0.0;
-    long tr_n = 0, dr_n = 0;
-    for (int base = 0; base <= G; base += kWarp) {
-      const int j = base + lane;
-      int flag = kFlagAccept;
-      bool tok_bad = false, row_bad = false, map_bad = false;
-      double lT = 0.0, lD = 0.0;
-      long tr = 0, dr = 0;
-      if (j <= G) {
-        const long position = static_cast<long>(b) * (G + 1) + j;
-        const long pj = static_cast<long>(b) * G + j;
-        const bool has_draft = j < G;
-        // rows of the logit buffers that hold this position
-        tr = P.target_map ? static_cast<long>(P.target_map[position]) : position;
-        dr = has_draft ? (P.draft_map ? static_cast<long>(P.draft_map[pj]) : pj) : 0;
-        map_bad = tr < 0 || tr >= P.target_rows || (has_draft && (dr < 0 || dr >= P.draft_rows));
-        // the acceptance test's inputs first: their loads overlap the combine
-        int t = 0;
-        float u = 0.f, xt = 0.f, xd = 0.f;
-        if (has_draft) {
-          t = P.tokens[pj];
-          u = P.u_accept[pj];
-          tok_bad = (t < 0 || t >= V);
-          if (!tok_bad && !map_bad) {
-            xt = P.gathered_target ? P.gathered_target[tr]
-                                   : Elem<T>::load1(static_cast<const T*>(P.target) + tr * V, t);
-            xd = P.gathered_draft ? P.gathered_draft[dr]
-                                  : Elem<T>::load1(static_cast<const T*>(P.draft) + dr * V, t);
-          }
-        }
-        int validT = 0, validD = 1;
-        if (!map_bad) {
-          lT = row_lse2(P.partial + tr * S, S, validT);
-          if (has_draft) lD = row_lse2(P.partial + (P.target_rows + dr) * S, S, validD);
-        }
-        P.tstat[position] = RowStat{lT, validT, 0};
-        if (has_draft) P.dstat[pj] = RowStat{lD, validD, 0};
-        row_bad = !map_bad && (!validT || !validD);
-        if (has_draft) {
-          PosInfo info{0.0, 0.0, 0.0, kFlagReject, 0};
-          if (tok_bad) {
-            info.flag = kFlagTokenRange;
-          } else if (row_bad || map_bad) {
-            info.flag = kFlagNonFinite;
-          } else {
-            const double lq = static_cast<double>(xt) * c - lT;  // log2 q(t)
-            const double lp = static_cast<double>(xd) * c - lD;  // log2 p(t)
-            info.q_tok = exp2(lq);
-            info.p_tok = exp2(lp);
-            if (!(info.q_tok > 0.0)) info.ratio = 0.0;
-            else if (!(info.p_tok > 0.0)) info.ratio = INFINITY;
-            else info.ratio = exp2(lq - lp);
-            info.flag = (static_cast<double>(u) < info.ratio) ? kFlagAccept : kFlagReject;
-          }
-          P.pos[pj] = info;
-          flag = info.flag;
-        }
-      }
-      const unsigned rej = __ballot_sync(0xffffffffu, j < G && flag == kFlagReject);
-      if (__ballot_sync(0xffffffffu, tok_bad)) bits |= kStatTokenRange;
-      if (__ballot_sync(0xffffffffu, row_bad)) bits |= kStatNonFinite;
-      if (__ballot_sync(0xffffffffu, map_bad)) bits |= kStatRowIndex;
-      // the statistics the draw needs live in lane (n - base) of this chunk
-      const int first = rej ? base + __ffs(rej) - 1 : G;
-      const bool here = (n == G) && (first < G || G < base + kWarp);
-      if (n == G) n = first;
-      const int src = (n - base) & (kWarp - 1);
-      const double lTs = __shfl_sync(0xffffffffu, lT, src);
-      const double lDs = __shfl_sync(0xffffffffu, lD, src);
-      const long trs = __shfl_sync(0xffffffffu, tr, src);
-      const long drs = __shfl_sync(0xffffffffu, dr, src);
-      if (here) {
-        lT_n = lTs;
-        lD_n = lDs;
-        tr_n = trs;
-        dr_n = drs;
-      }
-    }
-    const long bo = static_cast<long>(b) * (G + 1);
-    if (bits) {
-      for (int q = lane; q <= G; q += kWarp) P.out_tokens[bo + q] = -1;
-      if (lane == 0) {
-        P.out_num_accepted[b] = 0;
-        P.resid_mass[b] = NAN;
-        P.decision[b] = SeqDecision{0.0, 0.0, 0, 0, 0, kDrawNone, bits, 0.f, 0.f, 0.f, 1.f};
-        atomicOr(P.status, bits);
-      }
-    } else {
-      // accepted prefix and padding; the drawn token at n is the draw kernel's
-      for (int q = lane; q <= G; q += kWarp) {
-        if (q < n) P.out_tokens[bo + q] = P.tokens[static_cast<long>(b) * G + q];
-        else if (q > n) P.out_tokens[bo + q] = -1;
-      }
-      if (lane == 0) {
-        P.out_num_accepted[b] = n;
-        SeqDecision d{lT_n, lD_n, P.draw_compact ? b : tr_n, P.draw_compact ? b : dr_n, n,
-                      (n < G) ? kDrawResidual : kDrawTarget, 0u, 0.f, 0.f, 0.f, 1.f};
-        float lt_lo;
-        split2(lT_n, d.lt_hi, lt_lo);
-        split2(lT_n - lD_n, d.k_hi, d.k_lo);
-        d.fT = static_cast<float>(exp2(-static_cast<double>(lt_lo)));
-        P.decision[b] = d;
-      }
-    }
-  }
+  if (b < P.batch) decide_sequence<T, false>(P, b);  // warp-uniform
   cudaTriggerProgrammaticLaunchCompletion();
 }
 
 // ---------------------------------------------------------------------------
-// kernel 3: draw
+// kernel 3: draw (step 4)
 // ---------------------------------------------------------------------------
+//
+// The rows drawn from are cut into tiles of kTile 16-byte groups: lane l of a
+// warp takes groups k * 32 + l of the tile, k = 0 .. kDrawK - 1 (every load
+// instruction of the warp reads 512 contiguous bytes).  All tiles of the
+// batch, sequence by sequence, form one index range that the grid's warps
+// split into contiguous runs, so the work is even whatever mix of residual
+// draws (two rows), bonus draws (one row) and error outcomes (none) the batch
+// holds.  A warp writes the fp64 mass of each tile of its run to the
+// sequence's table, then adds the number of tiles it finished to the
+// sequence's ticket; the warp that completes the count locates u * Z: a warp
+// scan over the table finds the tile, and a re-read of that one tile finds
+// the index.
 
-constexpr int kDrawThreads = 128;
+constexpr int kDrawThreads = 256;
 constexpr int kDrawWarps = kDrawThreads / kWarp;
-constexpr int kTile = 32;  // groups per tile of the draw's mass table
+constexpr int kDrawK = 2;                 // groups per lane per tile
+constexpr int kTile = kWarp * kDrawK;     // groups per tile of the mass table
+constexpr int kDrawBlocksPerSM = 2;
 
-// Mass of each 32-group tile of [tlo, thi) (tiles of the row, warp w takes
-// tiles w, w + 4, ...); lane 0 of the warp stores the tile's mass in `table`.
-// Software-pipelined: the next two tiles' loads are in flight while the
-// current two are reduced.
-template <typename T, bool kAligned>
-__device__ __forceinline__ void tile_masses(int mode, const T* drawT, const T* drawD,
-                                            const DrawConsts& k, long tlo, long thi,
-                                            long ngroups, int V, double* table) {
+// tiles of one row of V entries stored `vec` to a 16-byte group
+inline long draw_tiles_per_row(long V, int vec) {
+  const long groups = (V + vec - 1) / vec;
+  return (groups + kTile - 1) / kTile;
+}
+
+// Grid of the draw kernel: at most `draw_blocks` blocks per sequence, at most
+// one resident wave, and at least one tile per warp.
+inline unsigned draw_grid(long batch, long tiles_per_row, int draw_blocks, int num_sms) {
+  long g = batch * static_cast<long>(draw_blocks);
+  const long wave = static_cast<long>(num_sms) * kDrawBlocksPerSM;
+  const long by_tiles = (batch * tiles_per_row + kDrawWarps - 1) / kDrawWarps;
+  if (g > wave) g = wave;
+  if (g > by_tiles) g = by_tiles;
+  if (g < 1) g = 1;
+  return static_cast<unsigned>(g);
+}
+
+// r (in units of 1/fT) for the kVec elements of one group: residual
+// max(0, q - p) or target q.  Pairs of elements go through the packed fp32
+// instructions (two lanes of arithmetic per instruction); the exponentials
+// are one MUFU ex2 each.  L = log2(q/p) comes from the logit difference
+// (exact for bf16 inputs) and p = q 2^-L.  L < 1/8 takes p (2^L - 1) from its
+// Taylor series in L to L^5 (truncation below 7e-9 relative on (0, 1/8); for
+// L <= 0 the series factor stays above 0.31, so the product is <= 0 and the
+// final max(., 0) makes it 0); L >= 1/8 takes q - p (q >= 1.09 p: at most 3.6
+// bits cancel).  Infinite logits need no test: a draft logit of -inf gives
+// L = +inf, p = 0 and r = q; a target logit of -inf gives q = 0 and r = 0
+// (the NaN of 0 * 2^inf is discarded by the final max).
+template <typename T, int kMode>
+__device__ __forceinline__ void group_r(const uint4& vt, const uint4& vd, const DrawConsts& k,
+                                        float (&r)[Elem<T>::kVec]) {
   constexpr int kVec = Elem<T>::kVec;
-  constexpr int kPair = 2;  // tiles per pipeline stage
-  const int lane = threadIdx.x & (kWarp - 1), warp = threadIdx.x >> 5;
-  const long first = tlo + warp;
-  if (first >= thi) return;
-  const long count = (thi - first + kDrawWarps - 1) / kDrawWarps;  // this warp's tiles
-  auto load = [&](long kk, uint4 (&vt)[kPair], uint4 (&vd)[kPair]) {
+  float xt[kVec];
+  Elem<T>::unpack(vt, xt);
+  const float2 chi = make_float2(k.c_hi, k.c_hi), clo = make_float2(k.c_lo, k.c_lo);
+  const float2 mlt = make_float2(-k.lt_hi, -k.lt_hi);
+  if constexpr (kMode == kDrawTarget) {
 #pragma unroll
-    for (int u = 0; u < kPair; ++u) {
-      const long g = (first + (kk + u) * kDrawWarps) * kTile + lane;
-      if (kk + u < count && g < ngroups) {
-        vt[u] = fetch_group<T, kAligned>(drawT, g, V);
-        vd[u] = (mode == kDrawResidual) ? fetch_group<T, kAligned>(drawD, g, V) : vt[u];
-      }
+    for (int e = 0; e < kVec; e += 2) {
+      const float2 x = make_float2(xt[e], xt[e + 1]);
+      const float2 y = __ffma2_rn(x, clo, __ffma2_rn(x, chi, mlt));
+      r[e] = ex2(y.x);
+      r[e + 1] = ex2(y.y);
     }
-  };
-  uint4 ct[kPair], cd[kPair];
-  load(0, ct, cd);
-  for (long kk = 0; kk < count; kk += kPair) {
-    uint4 nt[kPair], nd[kPair];
-    load(kk + kPair, nt, nd);
+  } else {
+    float xd[kVec];
+    Elem<T>::unpack(vd, xd);
+    const float2 mkhi = make_float2(-k.k_hi, -k.k_hi), mklo = make_float2(-k.k_lo, -k.k_lo);
+    const float2 one_neg = make_float2(-1.f, -1.f);
+    const float2 a1 = make_float2(kA1, kA1), a2 = make_float2(kA2, kA2);
+    const float2 a3 = make_float2(kA3, kA3), a4 = make_float2(kA4, kA4);
+    const float2 a5 = make_float2(kA5, kA5);
 #pragma unroll
-    for (int u = 0; u < kPair; ++u) {
-      if (kk + u < count) {  // warp-uniform
-        const long tile = first + (kk + u) * kDrawWarps;
-        const long g = tile * kTile + lane;
-        float gs = 0.f;
-        if (g < ngroups) {
-          float r[kVec];
-          if (mode == kDrawResidual) group_mass<T, kDrawResidual>(ct[u], cd[u], k, r);
-          else group_mass<T, kDrawTarget>(ct[u], cd[u], k, r);
-#pragma unroll
-          for (int e = 0; e < kVec; ++e) gs += r[e];
-        }
-        const double z = warp_sum(static_cast<double>(gs)) * k.fT;
-        if (lane == 0) table[tile] = z;
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kPair; ++u) {
-      ct[u] = nt[u];
-      cd[u] = nd[u];
+    for (int e = 0; e < kVec; e += 2) {
+      const float2 x = make_float2(xt[e], xt[e + 1]);
+      const float2 xdp = make_float2(xd[e], xd[e + 1]);
+      const float2 y = __ffma2_rn(x, clo, __ffma2_rn(x, chi, mlt));
+      float2 q;
+      q.x = ex2(y.x);
+      q.y = ex2(y.y);
+      const float2 dx = __ffma2_rn(xdp, one_neg, x);  // xt - xd, exact for bf16
+      const float2 L = __fadd2_rn(__ffma2_rn(dx, chi, mkhi), __ffma2_rn(dx, clo, mklo));
+      float2 w;
+      w.x = ex2(-L.x);
+      w.y = ex2(-L.y);
+      const float2 p = __fmul2_rn(q, w);
+      float2 t = __ffma2_rn(a5, L, a4);
+      t = __ffma2_rn(t, L, a3);
+      t = __ffma2_rn(t, L, a2);
+      t = __ffma2_rn(t, L, a1);
+      const float2 small = __fmul2_rn(p, __fmul2_rn(t, L));
+      const float2 big = __ffma2_rn(p, one_neg, q);  // q - p
+      r[e] = fmaxf((L.x < 0.125f) ? small.x : big.x, 0.f);
+      r[e + 1] = fmaxf((L.y < 0.125f) ? small.y : big.y, 0.f);
     }
   }
 }
 
-// The masses of the 32 groups of `tile`, one per lane of the calling warp:
-// returns the index where the running mass first exceeds tl, else the
-// tile's last index with mass (rounding), else -1 (no mass in the tile).
-template <typename T, bool kAligned>
-__device__ __forceinline__ int scan_tile(int mode, const T* drawT, const T* drawD,
-                                         const DrawConsts& k, long tile, long ngroups, int V,
-                                         double tl_mass) {
-  const double tl = tl_mass / static_cast<double>(k.fT);  // in the units of group_mass
+// fp32 sum of a group's r, pairwise
+template <int kVec>
+__device__ __forceinline__ float group_sum(const float (&r)[kVec]) {
+  float2 acc = make_float2(r[0], r[1]);
+#pragma unroll
+  for (int e = 2; e < kVec; e += 2) acc = __fadd2_rn(acc, make_float2(r[e], r[e + 1]));
+  return acc.x + acc.y;
+}
+
+// One tile's loads for the calling lane: its kDrawK groups of the target row
+// (and of the draft row for a residual draw); groups past the row end are
+// not read.
+template <typename T, bool kAligned, int kMode>
+__device__ __forceinline__ void load_tile(const T* rowT, const T* rowD, long tile, long ngroups,
+                                          int V, uint4 (&vt)[kDrawK], uint4 (&vd)[kDrawK]) {
+  const int lane = threadIdx.x & (kWarp - 1);
+#pragma unroll
+  for (int kk = 0; kk < kDrawK; ++kk) {
+    const long g = tile * kTile + kk * kWarp + lane;
+    if (g < ngroups) {
+      vt[kk] = fetch_group<T, kAligned>(rowT, g, V);
+      if constexpr (kMode == kDrawResidual) vd[kk] = fetch_group<T, kAligned>(rowD, g, V);
+    }
+  }
+}
+
+// fp64 mass (times fT) of one tile whose loads are in vt / vd, valid in every lane
+template <typename T, int kMode>
+__device__ __forceinline__ double tile_mass_of(const uint4 (&vt)[kDrawK], const uint4 (&vd)[kDrawK],
+                                               const DrawConsts& k, long tile, long ngroups) {
   constexpr int kVec = Elem<T>::kVec;
   const int lane = threadIdx.x & (kWarp - 1);
-  const long g = tile * kTile + lane;
-  float r[kVec];
+  double m = 0.0;
 #pragma unroll
-  for (int e = 0; e < kVec; ++e) r[e] = 0.f;
-  if (g < ngroups) {
-    const uint4 vt = fetch_group<T, kAligned>(drawT, g, V);
-    const uint4 vd = (mode == kDrawResidual) ? fetch_group<T, kAligned>(drawD, g, V) : vt;
-    if (mode == kDrawResidual) group_mass<T, kDrawResidual>(vt, vd, k, r);
-    else group_mass<T, kDrawTarget>(vt, vd, k, r);
+  for (int kk = 0; kk < kDrawK; ++kk) {
+    const long g = tile * kTile + kk * kWarp + lane;
+    if (g < ngroups) {
+      float r[kVec];
+      group_r<T, kMode>(vt[kk], vd[kk], k, r);
+      m += static_cast<double>(group_sum<kVec>(r));
+    }
   }
-  float gs = 0.f;
+  return warp_sum(m) * static_cast<double>(k.fT);
+}
+
+// Masses of tiles [t0, t1) of one row into table[t0 .. t1) (lane 0 stores),
+// software-pipelined: the next tile's loads are in flight while the current
+// tile is reduced (two register buffers, alternated).
+template <typename T, bool kAligned, int kMode>
+__device__ __forceinline__ void tile_masses_mode(const T* rowT, const T* rowD, const DrawConsts& k,
+                                                 long t0, long t1, long ngroups, int V,
+                                                 double* table) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  uint4 at[kDrawK], ad[kDrawK], bt[kDrawK], bd[kDrawK];
+  long t = t0;
+  if (t < t1) load_tile<T, kAligned, kMode>(rowT, rowD, t, ngroups, V, at, ad);
+  while (t < t1) {
+    if (t + 1 < t1) load_tile<T, kAligned, kMode>(rowT, rowD, t + 1, ngroups, V, bt, bd);
+    const double za = tile_mass_of<T, kMode>(at, ad, k, t, ngroups);
+    if (lane == 0) table[t] = za;
+    if (++t >= t1) break;
+    if (t + 1 < t1) load_tile<T, kAligned, kMode>(rowT, rowD, t + 1, ngroups, V, at, ad);
+    const double zb = tile_mass_of<T, kMode>(bt, bd, k, t, ngroups);
+    if (lane == 0) table[t] = zb;
+    ++t;
+  }
+}
+
+template <typename T, bool kAligned>
+__device__ __forceinline__ void tile_masses(int mode, const T* rowT, const T* rowD,
+                                            const DrawConsts& k, long t0, long t1, long ngroups,
+                                            int V, double* table) {
+  if (mode == kDrawResidual)
+    tile_masses_mode<T, kAligned, kDrawResidual>(rowT, rowD, k, t0, t1, ngroups, V, table);
+  else
+    tile_masses_mode<T, kAligned, kDrawTarget>(rowT, rowD, k, t0, t1, ngroups, V, table);
+}
+
+// The index inside `tile` where the running mass first exceeds tl_mass (in
+// table units); else the tile's last index with mass (rounding between the
+// table's sum and this scan's); else -1.  The calling warp re-reads the
+// tile: lane l's groups k * 32 + l, scanned in index order (k, then lane,
+// then element).
+template <typename T, bool kAligned, int kMode>
+__device__ __forceinline__ int scan_tile(const T* rowT, const T* rowD, const DrawConsts& k,
+                                         long tile, long ngroups, int V, double tl_mass) {
+  constexpr int kVec = Elem<T>::kVec;
+  const int lane = threadIdx.x & (kWarp - 1);
+  const double tl = tl_mass / static_cast<double>(k.fT);  // in the units of group_r
+  uint4 vt[kDrawK], vd[kDrawK];
+  load_tile<T, kAligned, kMode>(rowT, rowD, tile, ngroups, V, vt, vd);
+  double base = 0.0;
   int mylast = -1;
 #pragma unroll
-  for (int e = 0; e < kVec; ++e) {
-    gs += r[e];
-    if (r[e] > 0.f) mylast = static_cast<int>(g * kVec + e);
-  }
-  const double ls = static_cast<double>(gs);
-  double incl = ls;
+  for (int kk = 0; kk < kDrawK; ++kk) {
+    const long g = tile * kTile + kk * kWarp + lane;
+    float r[kVec];
 #pragma unroll
-  for (int o = 1; o < kWarp; o <<= 1) {
-    const double y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
-  if (lane == 0) excl = 0.0;
-  const unsigned hit = __ballot_sync(0xffffffffu, excl <= tl && incl > tl);
-  if (hit) {
-    const int L = __ffs(hit) - 1;
-    int token = -1;
-    if (lane == L) {
-      double acc = excl;
+    for (int e = 0; e < kVec; ++e) r[e] = 0.f;
+    if (g < ngroups) group_r<T, kMode>(vt[kk], vd[kk], k, r);
+    const double v = static_cast<double>(group_sum<kVec>(r));
 #pragma unroll
-      for (int e = 0; e < kVec; ++e) {
-        if (r[e] > 0.f) {
-          acc += static_cast<double>(r[e]);
-          if (token < 0 && acc > tl) token = static_cast<int>(g * kVec + e);
-        }
-      }
-      if (token < 0) token = mylast;  // rounding between the two sums
+    for (int e = 0; e < kVec; ++e)
+      if (r[e] > 0.f) mylast = static_cast<int>(g * kVec + e);
+    double incl = v;
+#pragma unroll
+    for (int o = 1; o < kWarp; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
-    return __shfl_sync(0xffffffffu, token, L);
+    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.0;
+    const unsigned hit =
+        __ballot_sync(0xffffffffu, v > 0.0 && base + excl <= tl && base + incl > tl);
+    if (hit) {
+      const int Ln = __ffs(hit) - 1;
+      int token = -1;
+      if (lane == Ln) {
+        double acc = base + excl;
+        int last = -1;
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) {
+          if (r[e] > 0.f) {
+            acc += static_cast<double>(r[e]);
+            last = static_cast<int>(g * kVec + e);
+            if (token < 0 && acc > tl) token = last;
+          }
+        }
+        if (token < 0) token = last;  // rounding between the two sums
+      }
+      return __shfl_sync(0xffffffffu, token, Ln);
+    }
+    base += __shfl_sync(0xffffffffu, incl, kWarp - 1);
   }
   return warp_maxi(mylast);  // rounding past the tile's end
 }
 
+// Step 4's last part for sequence b, by the warp that finished its table:
+// Z = sum of the tile masses; the tile holding u * Z (a warp scan over the
+// table in index order); the index inside it.  Z = 0 at a rejection: the
+// warp recomputes the table for q_n and draws from it (ZERO_MASS warning).
 template <typename T, bool kAligned>
-__global__ void __launch_bounds__(kDrawThreads, 8) draw_kernel(const Params P) {
-  constexpr int kVec = Elem<T>::kVec;
-  const int tid = threadIdx.x;
-  const int G = P.gamma, V = P.vocab, S2 = P.draw_slices;
-  const int b = blockIdx.x / S2;
-  const int s2 = blockIdx.x - b * S2;
-  cudaGridDependencySynchronize();  // the decisions of the previous kernel
-  const SeqDecision d = P.decision[b];
-  if (d.mode == kDrawNone) return;  // the decide kernel wrote the error outcome
-  const int n = d.n;
-  const long bo = static_cast<long>(b) * (G + 1);
-
-  // ---- step 4: residual (n < gamma) or bonus (n == gamma) draw ----
-  int mode = d.mode;
-  const T* drawT = static_cast<const T*>(P.target) + d.trow * V;
-  const T* drawD = (mode == kDrawResidual) ? static_cast<const T*>(P.draft) + d.drow * V : nullptr;
-  DrawConsts k;
-  k.c_hi = P.c_hi;
-  k.c_lo = P.c_lo;
-  k.lt_hi = d.lt_hi;
-  k.k_hi = d.k_hi;
-  k.k_lo = d.k_lo;
-  k.fT = d.fT;
-
-  const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
-  const long ntiles = (ngroups + kTile - 1) / kTile;
-  const long tiles_per = P.groups_per_draw / kTile;
-  long tlo = static_cast<long>(s2) * tiles_per;
-  long thi = tlo + tiles_per;
-  if (tlo > ntiles) tlo = ntiles;
-  if (thi > ntiles) thi = ntiles;
+__device__ __noinline__ void locate(const Params* Pp, int b, int mode, const T* rowT,
+                                    const T* rowD, const DrawConsts k, long ntiles,
+                                    long ngroups) {
+  const Params& P = *Pp;
+  const int lane = threadIdx.x & (kWarp - 1);
+  const int V = P.vocab, G = P.gamma;
   double* table = P.draw_mass + static_cast<long>(b) * ntiles;
-  tile_masses<T, kAligned>(mode, drawT, drawD, k, tlo, thi, ngroups, V, table);
-  __threadfence();  // this block's tiles are published before its ticket
-  __syncthreads();
-  __shared__ int sm_last;
-  if (tid == 0) {
-    const unsigned old = atomicAdd(P.draw_ticket + b, 1u);
-    sm_last = (old == static_cast<unsigned>(S2 - 1));
-    if (sm_last) __threadfence();
-  }
-  __syncthreads();
-  if (!sm_last) return;
-
-  // ---- the block that finishes the sequence locates u * Z ----
-  __shared__ long sm_tile;
-  __shared__ double sm_tl, sm_Z;
   unsigned extra_bits = 0;
-  for (int attempt = 0; attempt < 2; ++attempt) {
-    // each thread owns a contiguous run of up to kRun tiles per round, loaded
-    // together (independent loads), summed in index order
-    constexpr int kRun = 8;
-    const long per_round = static_cast<long>(kDrawThreads) * kRun;
-    double base = 0.0;  // mass of the rounds before this one
-    long found_tile = -1;
-    double found_tl = 0.0;
-    bool have_last = false;
-    long last_tile = -1;
-    const double target0 = static_cast<double>(P.u_resample[b]);
-    // pass 1: Z (all rounds)
-    double Z = 0.0;
-    for (long r0 = 0; r0 < ntiles; r0 += per_round) {
-      const long a0 = r0 + static_cast<long>(tid) * kRun;
-      double v[kRun];
-#pragma unroll
-      for (int q = 0; q < kRun; ++q) v[q] = (a0 + q < ntiles) ? __ldcg(&table[a0 + q]) : 0.0;
-      double mine = 0.0;
-#pragma unroll
-      for (int q = 0; q < kRun; ++q) mine += v[q];
-      double incl, excl, tot;
-      block_scan<kDrawThreads>(mine, incl, excl, tot);
-      Z += tot;
-    }
-    if (Z > 0.0 || mode != kDrawResidual) {
-      const double target = target0 * Z;
-      // pass 2: the round, thread and tile holding u * Z
-      for (long r0 = 0; r0 < ntiles; r0 += per_round) {
-        const long a0 = r0 + static_cast<long>(tid) * kRun;
-        double v[kRun];
-#pragma unroll
-        for (int q = 0; q < kRun; ++q) v[q] = (a0 + q < ntiles) ? __ldcg(&table[a0 + q]) : 0.0;
-        double mine = 0.0;
-#pragma unroll
-        for (int q = 0; q < kRun; ++q) mine += v[q];
-        double incl, excl, tot;
-        block_scan<kDrawThreads>(mine, incl, excl, tot);
-        if (base + excl <= target && base + incl > target) {
-          double acc = base + excl;
-#pragma unroll
-          for (int q = 0; q < kRun; ++q) {
-            if (found_tile < 0 && v[q] > 0.0 && acc + v[q] > target) {
-              found_tile = a0 + q;
-              found_tl = target - acc;
-            }
-            acc += v[q];
-          }
-        }
-        // remember the last tile with mass (rounding fallback)
-#pragma unroll
-        for (int q = 0; q < kRun; ++q)
-          if (v[q] > 0.0) {
-            have_last = true;
-            last_tile = a0 + q;
-          }
-        base += tot;
-      }
-      // publish: the owning tile, else the last tile with mass
-      __shared__ long sm_found, sm_lastt[kDrawThreads / kWarp];
-      if (tid == 0) sm_found = -1;
-      __syncthreads();
-      if (found_tile >= 0) {
-        sm_found = found_tile;
-        sm_tl = found_tl;
-      }
-      const long wl = have_last ? last_tile : -1;
-      long m = wl;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if ((tid & (kWarp - 1)) == 0) sm_lastt[tid >> 5] = m;
-      __syncthreads();
-      if (tid == 0) {
-        sm_Z = Z;
-        if (sm_found >= 0) {
-          sm_tile = sm_found;
-        } else {
-          long lt = -1;
-          for (int w = 0; w < kDrawThreads / kWarp; ++w) lt = max(lt, sm_lastt[w]);
-          sm_tile = lt;
-          sm_tl = INFINITY;  // the tile's last index with mass
-        }
-      }
-      __syncthreads();
-      break;
-    }
-    // zero residual mass (reachable only through rounding): draw from q_n,
-    // this block alone recomputing the row's tiles
+  double Z = 0.0;
+  for (long i = lane; i < ntiles; i += kWarp) Z += __ldcg(table + i);
+  Z = warp_sum(Z);
+  if (!(Z > 0.0) && mode == kDrawResidual) {
     mode = kDrawTarget;
     extra_bits |= kStatZeroMass;
-    tile_masses<T, kAligned>(mode, drawT, drawD, k, 0, ntiles, ngroups, V, table);
-    __threadfence();
-    __syncthreads();
+    tile_masses<T, kAligned>(mode, rowT, rowD, k, 0, ntiles, ngroups, V, table);
+    __syncwarp();
+    Z = 0.0;
+    for (long i = lane; i < ntiles; i += kWarp) Z += __ldcg(table + i);
+    Z = warp_sum(Z);
   }
-
-  // the owning tile: one group per lane, warp 0 scans it in index order
-  if (tid < kWarp) {
-    const long tile = sm_tile;
-    const int token = (tile >= 0) ? scan_tile<T, kAligned>(mode, drawT, drawD, k, tile, ngroups, V, sm_tl)
-                                  : -1;
-    if (tid == 0) {
-      P.out_tokens[bo + n] = token;
-      P.resid_mass[b] = sm_Z;
-      if (extra_bits) atomicOr(P.status, extra_bits);
-      P.draw_ticket[b] = 0u;  // ready for the next launch
+  const double target = static_cast<double>(P.u_resample[b]) * Z;
+  long found = -1, last_mass = -1;
+  double tl = 0.0, base = 0.0;
+  for (long c0 = 0; c0 < ntiles; c0 += kWarp) {
+    const long i = c0 + lane;
+    const double v = (i < ntiles) ? __ldcg(table + i) : 0.0;
+    double incl = v;
+#pragma unroll
+    for (int o = 1; o < kWarp; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
+    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.0;
+    const unsigned hit =
+        __ballot_sync(0xffffffffu, v > 0.0 && base + excl <= target && base + incl > target);
+    const unsigned has = __ballot_sync(0xffffffffu, v > 0.0);
+    if (has) last_mass = c0 + (31 - __clz(has));
+    if (hit) {
+      const int Ln = __ffs(hit) - 1;
+      found = c0 + Ln;
+      tl = __shfl_sync(0xffffffffu, target - (base + excl), Ln);
+      break;
+    }
+    base += __shfl_sync(0xffffffffu, incl, kWarp - 1);
+  }
+  if (found < 0) {  // rounding: the tile's last index with mass
+    found = last_mass;
+    tl = INFINITY;
+  }
+  int token = -1;
+  if (found >= 0) {
+    token = (mode == kDrawResidual)
+                ? scan_tile<T, kAligned, kDrawResidual>(rowT, rowD, k, found, ngroups, V, tl)
+                : scan_tile<T, kAligned, kDrawTarget>(rowT, rowD, k, found, ngroups, V, tl);
+  }
+  if (lane == 0) {
+    const SeqDecision& d = P.decision[b];
+    P.out_tokens[static_cast<long>(b) * (G + 1) + d.n] = token;
+    P.resid_mass[b] = Z;
+    if (extra_bits) atomicOr(P.status, extra_bits);
+    P.draw_ticket[b] = 0u;  // ready for the next launch
+  }
+}
+
+template <typename T, bool kAligned>
+__global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(const __grid_constant__ Params P) {
+  constexpr int kVec = Elem<T>::kVec;
+  const int lane = threadIdx.x & (kWarp - 1);
+  const int V = P.vocab;
+  const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
+  const long ntiles = P.draw_tiles;
+  const long total = static_cast<long>(P.batch) * ntiles;
+  const long W = static_cast<long>(gridDim.x) * kDrawWarps;
+  const long w = static_cast<long>(blockIdx.x) * kDrawWarps + (threadIdx.x >> 5);
+  const long lo = total * w / W, hi = total * (w + 1) / W;
+  cudaGridDependencySynchronize();  // the decisions of the previous kernel
+  for (long t = lo; t < hi;) {
+    const int b = static_cast<int>(t / ntiles);
+    const long row0 = static_cast<long>(b) * ntiles;
+    const long end = (hi < row0 + ntiles) ? hi : row0 + ntiles;
+    const SeqDecision d = P.decision[b];
+    if (d.mode != kDrawNone) {
+      const T* rowT = static_cast<const T*>(P.target) + d.trow * V;
+      const T* rowD = (d.mode == kDrawResidual) ? static_cast<const T*>(P.draft) + d.drow * V
+                                                : nullptr;
+      DrawConsts k;
+      k.c_hi = P.c_hi;
+      k.c_lo = P.c_lo;
+      k.lt_hi = d.lt_hi;
+      k.k_hi = d.k_hi;
+      k.k_lo = d.k_lo;
+      k.fT = d.fT;
+      double* table = P.draw_mass + row0;
+      tile_masses<T, kAligned>(d.mode, rowT, rowD, k, t - row0, end - row0, ngroups, V, table);
+      // publish this run's tiles; the warp that completes the row locates
+      unsigned last = 0;
+      if (lane == 0) {
+        __threadfence();
+        const unsigned cnt = static_cast<unsigned>(end - t);
+        const unsigned old = atomicAdd(P.draw_ticket + b, cnt);
+        last = (old + cnt == static_cast<unsigned>(ntiles));
+        if (last) __threadfence();
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (last) {
+        __threadfence();  // every lane reads the other warps' tiles after the ticket
+        locate<T, kAligned>(&P, b, d.mode, rowT, rowD, k, ntiles, ngroups);
+      }
+    }
+    t = end;
   }
 }
 
