@@ -60,9 +60,8 @@ KERNEL_SOURCES = [
 ]
 
 
-# kernels of one plain step: statistics (which also takes each sequence's
-# decision) and draw
-LAUNCHES_PER_STEP = 2
+# kernels of one plain step: statistics, decide, draw
+LAUNCHES_PER_STEP = 3
 
 # sampling-variant settings timed by the bench: name -> (temperature, top_k, top_p);
 # None = the workload's temperature
@@ -94,6 +93,9 @@ def parse():
                     help="skip the timing of the LM-head-fused step (64 x 8, V 128256, d 4096)")
     ap.add_argument("--no-gate", action="store_true",
                     help="skip the timing of the fold gate (128 x 8 branches, 32 x 4096 bf16)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other benchmark configurations (64 x 8 at V 128256, 8 x 3 at "
+                         "V 32000, the char-level calls, the 60000-row exactness batch)")
     args = ap.parse_args()
     if args.sampling:
         unknown = [n for n in args.sampling.split(",") if n not in SAMPLING_SETTINGS]
@@ -409,6 +411,7 @@ def run_ours(args):
     if extras and wl.mapped and not args.no_shared_rows:
         shared = time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local)
     sv.close()
+    others = None if (args.no_configs or not extras) else time_other_configs(args, dev)
     gate = None if (args.no_gate or not extras) else time_gate(args, dev, world, local)
     lmh = None if (args.no_lmhead or not extras) else time_lmhead(args, dev, world, local)
     # tokens settled per step on this rank = accepted + 1 per sequence (last device step)
@@ -443,8 +446,8 @@ def run_ours(args):
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                          "algorithmic_bytes_per_launch": step_bytes,
                          "kernel": "stats_kernel (streams every logit once)"},
-            "kernels_us_per_step": {"stats_and_decide": 1e3 * kern["stats_ms"],
-                                    "draw": 1e3 * kern["draw_ms"],
+            "kernels_us_per_step": {"stats": 1e3 * kern["stats_ms"],
+                                    "decide_and_draw": 1e3 * kern["draw_ms"],
                                     "runs": kern["runs"]},
             "step_hbm_gbs": step_bytes / (ms / 1e3 / args.steps) / 1e9,
             "step_frac": step_bytes / (ms / 1e3 / args.steps) / 1e9 / peak,
@@ -456,6 +459,8 @@ def run_ours(args):
             "cpu_baseline": cpu,
             "status_after": st,
         }
+        if others is not None:
+            line["other_configs"] = others_summary(others, peak)
         if gate is not None:
             line["specfold_gate"] = gate_summary(gate, peak)
         if lmh is not None:
@@ -489,6 +494,162 @@ def run_ours(args):
     if line is not None:
         print(json.dumps(line), flush=True)
     return 0
+
+
+def _device_inputs(wl, dev):
+    import torch
+
+    def put(a, logits):
+        if logits and wl.dtype == "bf16":
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    return {"target": put(wl.target, True), "draft": put(wl.draft, True),
+            "tokens": put(wl.tokens, False), "u_accept": put(wl.u_accept, False),
+            "u_resample": put(wl.u_resample, False)}
+
+
+def _time_calls(sv, sets, wl, calls, warmup, out_t, out_n, slices=None):
+    """Device time of `calls` verification calls (CUDA events on the launch
+    stream), cycling through the input sets; returns (ms, per-kernel means)."""
+    import torch
+    n = len(sets)
+
+    def call(i):
+        d = sets[i % n]
+        if slices is None:
+            sv.run(d["target"], d["draft"], d["tokens"], d["u_accept"], d["u_resample"],
+                   wl.temperature, out_t, out_n)
+        else:
+            b0, b1 = slices[i % len(slices)]
+            sv.run(d["target"][b0:b1], d["draft"][b0:b1], d["tokens"][b0:b1],
+                   d["u_accept"][b0:b1], d["u_resample"][b0:b1], wl.temperature, out_t, out_n)
+
+    for i in range(max(3, warmup)):
+        call(i)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sv.profile_begin(calls)
+    ev0.record(stream)
+    for i in range(calls):
+        call(i)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    kern = sv.profile_end()
+    return ev0.elapsed_time(ev1), kern
+
+
+def time_other_configs(args, dev):
+    """The other benchmark configurations, one GPU: the 64-sequence gamma-8
+    batch at V = 128256 (a plain step like the headline's); the 8-sequence
+    batch at V = 32000 and the char-level calls (B = 1, V = 256), both
+    launch-bound, as calls per second over rotating input copies larger than
+    L2 in total; the 60000-row exactness batch (one call) with the total
+    variation distance of its emitted tokens to q."""
+    import torch
+    from speculative_decoding_verification_90_b200.specverify import SpecVerify
+    res = {}
+    steps = max(1, args.steps)
+    # configuration 4: a bandwidth-bound step (279 MB of logits > 2 x L2)
+    wl = workloads.b64_g8_v128256(seed=args.seed)
+    d = _device_inputs(wl, dev)
+    n_sets = max(1, math.ceil(2 * L2_BYTES / wl.logit_bytes)) if wl.logit_bytes < 2 * L2_BYTES else 1
+    sets = [d] + [{k: v.clone() for k, v in d.items()} for _ in range(n_sets - 1)]
+    out_t = torch.empty((wl.batch, wl.gamma + 1), dtype=torch.int32, device=dev)
+    out_n = torch.empty((wl.batch,), dtype=torch.int32, device=dev)
+    with SpecVerify(wl.batch, wl.gamma, wl.vocab, wl.dtype, dev.index) as sv:
+        ms, kern = _time_calls(sv, sets, wl, steps, args.warmup, out_t, out_n)
+        st, _ = sv.status()
+    res["b64_g8_v128256"] = {"wl": wl, "ms": ms, "calls": steps, "kern": kern, "sets": n_sets,
+                             "status": st}
+    del sets, d
+    # configuration 3: 3.6 MB per call, launch-bound; copies rotate past L2
+    wl = workloads.b8_g3_v32000(seed=args.seed)
+    d = _device_inputs(wl, dev)
+    n_sets = min(256, max(1, math.ceil(2 * L2_BYTES / wl.logit_bytes)))
+    sets = [d] + [{k: v.clone() for k, v in d.items()} for _ in range(n_sets - 1)]
+    out_t = torch.empty((wl.batch, wl.gamma + 1), dtype=torch.int32, device=dev)
+    out_n = torch.empty((wl.batch,), dtype=torch.int32, device=dev)
+    calls = max(200, 4 * steps)
+    with SpecVerify(wl.batch, wl.gamma, wl.vocab, wl.dtype, dev.index) as sv:
+        ms, kern = _time_calls(sv, sets, wl, calls, args.warmup, out_t, out_n)
+        st, _ = sv.status()
+    res["b8_g3_v32000"] = {"wl": wl, "ms": ms, "calls": calls, "kern": kern, "sets": n_sets,
+                           "status": st}
+    del sets, d
+    # configuration 1: 1000 independent calls of one sequence each
+    wl = workloads.char_level(calls=1000, seed=args.seed)
+    d = _device_inputs(wl, dev)
+    out_t = torch.empty((1, wl.gamma + 1), dtype=torch.int32, device=dev)
+    out_n = torch.empty((1,), dtype=torch.int32, device=dev)
+    with SpecVerify(1, wl.gamma, wl.vocab, wl.dtype, dev.index) as sv:
+        ms, kern = _time_calls(sv, [d], wl, wl.batch, args.warmup, out_t, out_n,
+                               slices=[(b, b + 1) for b in range(wl.batch)])
+        st, _ = sv.status()
+    res["char_level"] = {"wl": wl, "ms": ms, "calls": wl.batch, "kern": kern, "sets": 1,
+                         "status": st}
+    del d
+    # configuration 2: the exactness batch, one call; the law of its outputs
+    with open(os.path.join(ROOT, "tests", "golden", "exactness_beta.json")) as f:
+        beta = json.load(f)["beta"]
+    wl = workloads.exactness(beta, seed=args.seed)
+    d = _device_inputs(wl, dev)
+    out_t = torch.empty((wl.batch, wl.gamma + 1), dtype=torch.int32, device=dev)
+    out_n = torch.empty((wl.batch,), dtype=torch.int32, device=dev)
+    with SpecVerify(wl.batch, wl.gamma, wl.vocab, wl.dtype, dev.index) as sv:
+        ms, kern = _time_calls(sv, [d], wl, max(3, steps // 10), args.warmup, out_t, out_n)
+        st, _ = sv.status()
+    sv_out = out_t[:, 0].cpu().numpy()
+    x = wl.target[0, 0].astype(np.float64) / wl.temperature
+    q = np.exp(x - x.max())
+    q /= q.sum()
+    N, V = wl.batch, wl.vocab
+    tv = 0.5 * float(np.abs(np.bincount(sv_out, minlength=V)[:V] / N - q).sum())
+    rng = np.random.default_rng(1234)
+    direct = [0.5 * float(np.abs(np.bincount(rng.choice(V, N, p=q), minlength=V) / N - q).sum())
+              for _ in range(20)]
+    res["exactness"] = {"wl": wl, "ms": ms, "calls": max(3, steps // 10), "kern": kern, "sets": 1,
+                        "status": st, "tv": tv, "tv_direct_mean": float(np.mean(direct)),
+                        "tv_direct_sd": float(np.std(direct))}
+    del d
+    return res
+
+
+def others_summary(res, peak):
+    out = {}
+    for name, r in res.items():
+        wl = r["wl"]
+        per_call_s = r["ms"] / 1e3 / r["calls"]
+        positions = wl.batch * wl.gamma
+        e = {"workload": wl.name, "batch": wl.batch, "gamma": wl.gamma, "vocab": wl.vocab,
+             "logits": wl.dtype, "temperature": wl.temperature,
+             "calls": r["calls"], "us_per_call": per_call_s * 1e6,
+             "kernels_us_per_call": {"stats": 1e3 * r["kern"]["stats_ms"],
+                                     "decide_and_draw": 1e3 * r["kern"]["draw_ms"]},
+             "status_after": r["status"]}
+        if name == "char_level":
+            # one sequence per call
+            e["calls_per_s"] = 1.0 / per_call_s
+            e["value"] = wl.gamma / per_call_s
+            e["unit"] = "positions/s"
+            e["l2"] = "one sequence per call (9 KB); launch-bound"
+        else:
+            step_bytes = wl.logit_bytes
+            e["value"] = positions / per_call_s
+            e["unit"] = "positions/s"
+            e["calls_per_s"] = 1.0 / per_call_s
+            e["step_hbm_gbs"] = step_bytes / per_call_s / 1e9
+            e["step_frac"] = e["step_hbm_gbs"] / peak
+            e["stats_hbm_gbs"] = step_bytes / (r["kern"]["stats_ms"] / 1e3) / 1e9
+            e["l2"] = ("inputs larger than L2 (%.1f MB per call, %d rotating set(s))"
+                       % (step_bytes / 1e6, r["sets"]))
+        if name == "exactness":
+            e["tv_emitted_vs_q"] = r["tv"]
+            e["tv_direct_sampling"] = {"mean": r["tv_direct_mean"], "sd": r["tv_direct_sd"],
+                                       "reps": 20}
+        out[name] = e
+    return out
 
 
 def time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local):

@@ -10,9 +10,10 @@
 //   tree_kernel  one block: validates every branch's parent chain by pointer
 //                jumping in shared memory;
 //   rows_kernel  persistent warps, global warp w taking rows w, w + W, ...;
-//                each warp streams its rows' H[c, j] and H[parent, j] through
-//                a ring of cp.async stages, sums squares in fp32 per lane and
-//                fp64 across the warp, and decides recompute = !(d <= tau);
+//                each warp streams its rows' H[c, j] and H[parent, j] with
+//                128-bit loads, eight in flight per lane, sums squares with
+//                packed fp32 pairs per lane and in fp64 across the warp, and
+//                decides recompute = !(d <= tau);
 //   scan_kernel  one block: the packed slot of every recomputed row (an
 //                exclusive prefix sum of the flags) and their count;
 //   pack_kernel  one warp per row: writes the packed row index, follows the
@@ -78,6 +79,20 @@ struct HElem<float> {
   static constexpr int kPerVec = 4;
   __device__ static float scalar(const float* p, long i) { return __ldg(p + i); }
   // d += (c - p)^2, n += p^2 over one 16-byte group of each row
+  // d += (c - p)^2, n += p^2 on pairs of entries (packed fp32 instructions)
+  __device__ static void accumulate2(uint4 c, uint4 p, float2& d, float2& n) {
+    const float2 m1 = make_float2(-1.f, -1.f);
+    float2 cc = make_float2(__uint_as_float(c.x), __uint_as_float(c.y));
+    float2 pp = make_float2(__uint_as_float(p.x), __uint_as_float(p.y));
+    float2 e = __ffma2_rn(pp, m1, cc);
+    d = __ffma2_rn(e, e, d);
+    n = __ffma2_rn(pp, pp, n);
+    cc = make_float2(__uint_as_float(c.z), __uint_as_float(c.w));
+    pp = make_float2(__uint_as_float(p.z), __uint_as_float(p.w));
+    e = __ffma2_rn(pp, m1, cc);
+    d = __ffma2_rn(e, e, d);
+    n = __ffma2_rn(pp, pp, n);
+  }
   __device__ static void accumulate(uint4 c, uint4 p, float& d0, float& d1, float& n0, float& n1) {
     const float c0 = __uint_as_float(c.x), c1 = __uint_as_float(c.y);
     const float c2 = __uint_as_float(c.z), c3 = __uint_as_float(c.w);
@@ -104,6 +119,20 @@ struct HElem<__nv_bfloat16> {
     float e;
     e = cl - pl; d0 = fmaf(e, e, d0); n0 = fmaf(pl, pl, n0);
     e = ch - ph; d1 = fmaf(e, e, d1); n1 = fmaf(ph, ph, n1);
+  }
+  __device__ static void pair2(unsigned c, unsigned p, float2& d, float2& n) {
+    const float2 cc = make_float2(__uint_as_float(c << 16), __uint_as_float(c & 0xffff0000u));
+    const float2 pp = make_float2(__uint_as_float(p << 16), __uint_as_float(p & 0xffff0000u));
+    const float2 e = __ffma2_rn(pp, make_float2(-1.f, -1.f), cc);  // exact: bf16 differences
+    d = __ffma2_rn(e, e, d);
+    n = __ffma2_rn(pp, pp, n);
+  }
+  // d += (c - p)^2, n += p^2 on pairs of entries (packed fp32 instructions)
+  __device__ static void accumulate2(uint4 c, uint4 p, float2& d, float2& n) {
+    pair2(c.x, p.x, d, n);
+    pair2(c.y, p.y, d, n);
+    pair2(c.z, p.z, d, n);
+    pair2(c.w, p.w, d, n);
   }
   __device__ static void accumulate(uint4 c, uint4 p, float& d0, float& d1, float& n0, float& n1) {
     pair(c.x, p.x, d0, d1, n0, n1);
@@ -157,19 +186,8 @@ __global__ void __launch_bounds__(kTreeThreads) tree_kernel(const GateParams P) 
 // kernel 2: difference test
 // ---------------------------------------------------------------------------
 
-constexpr int kStages = 8;  // cp.async stages in flight per warp
-constexpr int kStageBytes = kWarp * 32;  // one 16-byte group of child and parent per lane
-constexpr int kRowsSmem = kStages * kStageBytes * (kThreads / kWarp);
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
-  const unsigned dst = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-  const int n = valid ? 16 : 0;  // 0: fill with zeros, read nothing
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(gmem), "r"(n));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(kStages - 1));
-}
+constexpr int kRowUnroll = 4;  // 16-byte groups of each row in flight per lane
+constexpr int kRowsBlocksPerSM = 4;
 
 // lane 0's per-row epilogue: the decision and its records
 __device__ __forceinline__ bool finish_row(const GateParams& P, long row, int par, int j,
@@ -188,12 +206,11 @@ __device__ __forceinline__ bool finish_row(const GateParams& P, long row, int pa
 // Persistent warps: global warp w takes rows w, w + W, w + 2W, ... (W warps
 // in the grid), so all warps move through the tensor together and a parent
 // row, a few hundred rows before its children, is still in L2 when they read
-// it.  With 128-bit rows a warp streams its rows' (child, parent) groups
-// through a ring of kStages cp.async stages in shared memory, so loads stay in
-// flight across row boundaries without holding registers.
+// it.  With 128-bit rows each lane keeps kRowUnroll groups of the child row
+// and kRowUnroll of the parent row in flight (the statistics kernel's load
+// scheme: independent non-coherent 16-byte loads, coalesced across the warp).
 template <typename T, bool kAligned>
-__global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
-  extern __shared__ uint4 ring[];  // [warps][kStages][2][kWarp]
+__global__ void __launch_bounds__(kThreads, kRowsBlocksPerSM) rows_kernel(const GateParams P) {
   const int warp = threadIdx.x / kWarp, lane = threadIdx.x & (kWarp - 1);
   const long W = static_cast<long>(gridDim.x) * (kThreads / kWarp);
   const long r0 = static_cast<long>(blockIdx.x) * (kThreads / kWarp) + warp;
@@ -215,73 +232,37 @@ __global__ void __launch_bounds__(kThreads) rows_kernel(const GateParams P) {
   if constexpr (kAligned) {
     constexpr int kVec = HElem<T>::kPerVec;
     const int groups = P.dim / kVec;
-    const int chunks = (groups + kWarp - 1) / kWarp;  // units per row
-    uint4* my = ring + static_cast<long>(warp) * kStages * 2 * kWarp;
-    // issue pointer: the row being fetched, its two group pointers (this
-    // lane's group of chunk 0) and the chunk; all set once per row
-    long irow = next_row(r0);
-    int ichunk = 0;
-    const uint4* igc = nullptr;  // this lane's next group of the child row
-    const uint4* igp = nullptr;  // and of the parent row
-    const uint4* rc = nullptr;   // first group of each row: the (unread) source
-    const uint4* rp = nullptr;   // address of a zero-filling copy
-    auto set_issue_row = [&]() {
-      if (irow < r1) {
-        const int par = parent_of(irow);
-        const long j = irow - (irow / P.positions) * P.positions;
-        rc = reinterpret_cast<const uint4*>(base + irow * P.dim);
-        rp = reinterpret_cast<const uint4*>(base + (static_cast<long>(par) * P.positions + j) * P.dim);
-        igc = rc + lane;
-        igp = rp + lane;
-      }
-    };
-    set_issue_row();
-    int g_left = groups - lane;  // groups of the row at or after this lane's
-    auto issue = [&](int slot) {
-      if (irow < r1) {
-        const bool ok = g_left > 0;
-        cp_async16(my + (slot * 2 + 0) * kWarp + lane, ok ? igc : rc, ok);
-        cp_async16(my + (slot * 2 + 1) * kWarp + lane, ok ? igp : rp, ok);
-        igc += kWarp;
-        igp += kWarp;
-        g_left -= kWarp;
-        if (++ichunk == chunks) {
-          ichunk = 0;
-          g_left = groups - lane;
-          irow = next_row(irow + W);
-          set_issue_row();
-        }
-      }
-      cp_async_commit();  // an empty group keeps the wait count uniform
-    };
-#pragma unroll 1
-    for (int st = 0; st < kStages - 1; ++st) issue(st);
-    long crow = next_row(r0);
-    int cchunk = 0, slot = 0;
-    float d0 = 0.f, d1 = 0.f, n0 = 0.f, n1 = 0.f;
-    while (crow < r1) {
-      issue(slot == 0 ? kStages - 1 : slot - 1);
-      cp_async_wait();
-      const uint4 c = my[(slot * 2 + 0) * kWarp + lane];
-      const uint4 p = my[(slot * 2 + 1) * kWarp + lane];
-      HElem<T>::accumulate(c, p, d0, d1, n0, n1);
-      slot = (slot == kStages - 1) ? 0 : slot + 1;
-      if (++cchunk == chunks) {
-        double num = static_cast<double>(d0) + static_cast<double>(d1);
-        double den = static_cast<double>(n0) + static_cast<double>(n1);
+    for (long row = next_row(r0); row < r1; row = next_row(row + W)) {
+      const int par = parent_of(row);
+      const int j = static_cast<int>(row % P.positions);
+      const uint4* hc = reinterpret_cast<const uint4*>(base + row * P.dim);
+      const uint4* hp = reinterpret_cast<const uint4*>(base + (static_cast<long>(par) * P.positions + j) * P.dim);
+      float2 d = make_float2(0.f, 0.f), n = make_float2(0.f, 0.f);
+      for (int g0 = lane; g0 < groups; g0 += kWarp * kRowUnroll) {
+        uint4 c[kRowUnroll], q[kRowUnroll];
 #pragma unroll
-        for (int o = kWarp / 2; o > 0; o >>= 1) {
-          num += __shfl_xor_sync(0xffffffffu, num, o);
-          den += __shfl_xor_sync(0xffffffffu, den, o);
+        for (int u = 0; u < kRowUnroll; ++u) {
+          const int g = g0 + u * kWarp;
+          if (g < groups) {
+            c[u] = ld_v4(hc + g);
+            q[u] = ld_v4(hp + g);
+          } else {
+            c[u] = make_uint4(0u, 0u, 0u, 0u);
+            q[u] = c[u];
+          }
         }
-        if (lane == 0)
-          finish_row(P, crow, parent_of(crow), static_cast<int>(crow % P.positions), num, den);
-        d0 = d1 = n0 = n1 = 0.f;
-        cchunk = 0;
-        crow = next_row(crow + W);
+#pragma unroll
+        for (int u = 0; u < kRowUnroll; ++u) HElem<T>::accumulate2(c[u], q[u], d, n);
       }
+      double num = static_cast<double>(d.x) + static_cast<double>(d.y);
+      double den = static_cast<double>(n.x) + static_cast<double>(n.y);
+#pragma unroll
+      for (int o = kWarp / 2; o > 0; o >>= 1) {
+        num += __shfl_xor_sync(0xffffffffu, num, o);
+        den += __shfl_xor_sync(0xffffffffu, den, o);
+      }
+      if (lane == 0) finish_row(P, row, par, j, num, den);
     }
-    asm volatile("cp.async.wait_all;");
   } else {
     for (long row = next_row(r0); row < r1; row = next_row(row + W)) {
       const int par = parent_of(row);

@@ -396,7 +396,6 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   p.decision = h->decision;
   p.draw_mass = h->draw_mass;
   p.draw_ticket = h->draw_ticket;
-  p.seq_ticket = nullptr;
   p.resid_mass = h->resid;
   p.status = h->status;
   p.batch = B;
@@ -452,10 +451,8 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   // 5. the draw on fp32 rows
   const bool aligned = (static_cast<size_t>(V) * 4) % 16 == 0;
   if (e == cudaSuccess)
-    e = aligned ? launch_plain(specverify::draw_kernel<float, true>,
-                               static_cast<unsigned>(h->draw_slices), specverify::kDrawThreads, s, p)
-                : launch_plain(specverify::draw_kernel<float, false>,
-                               static_cast<unsigned>(h->draw_slices), specverify::kDrawThreads, s, p);
+    e = aligned ? specverify::launch_draw<float, true>(p, static_cast<unsigned>(h->draw_slices), s, false)
+                : specverify::launch_draw<float, false>(p, static_cast<unsigned>(h->draw_slices), s, false);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
   if (e != cudaSuccess) return cuda_fail(e);
   return SV_OK;

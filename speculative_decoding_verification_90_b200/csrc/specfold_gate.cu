@@ -69,7 +69,7 @@ cudaError_t launch_pass(const GateParams& p, cudaStream_t s, cudaEvent_t* ev) {
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[0], s);
   if (e == cudaSuccess)
     e = launch_pdl(specfold::rows_kernel<T, A>, static_cast<unsigned>(p.blocks),
-                   specfold::kThreads, A ? specfold::kRowsSmem : 0, s, p);
+                   specfold::kThreads, 0, s, p);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
   if (e == cudaSuccess)
     e = launch_pdl(specfold::scan_kernel, 1u, specfold::kSlotThreads, 0, s, p);
@@ -121,7 +121,7 @@ sv_status specfold_gate_create(specfold_gate_t* out, int branches, int positions
   h->pack_blocks = static_cast<int>((rows + specfold::kRowsPerBlock - 1) / specfold::kRowsPerBlock);
   h->dtype = dtype;
   // the difference kernel is persistent: as many blocks as fit on the GPU at
-  // once (its cp.async ring sets the limit), never more than there are rows
+  // once (its registers set the limit), never more than there are rows
   {
     int sms = 0, occ = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device);
@@ -129,10 +129,7 @@ sv_status specfold_gate_create(specfold_gate_t* out, int branches, int positions
                         ? reinterpret_cast<const void*>(specfold::rows_kernel<__nv_bfloat16, true>)
                         : reinterpret_cast<const void*>(specfold::rows_kernel<float, true>);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, specfold::kRowsSmem);
-    if (e == cudaSuccess)
-      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, specfold::kThreads,
-                                                        specfold::kRowsSmem);
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, specfold::kThreads, 0);
     if (e != cudaSuccess) {
       delete h;
       return cuda_fail(e);

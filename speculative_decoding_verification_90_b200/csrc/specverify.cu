@@ -41,7 +41,6 @@ struct specverify_ctx {
   SeqDecision* decision = nullptr;
   double* draw_mass = nullptr;
   unsigned* draw_ticket = nullptr;
-  unsigned* seq_ticket = nullptr;
   double* resid = nullptr;
   unsigned* status = nullptr;
   specsamp::SampRow* samp_rows = nullptr;          // sampling variants: per-row filter
@@ -133,41 +132,37 @@ cudaError_t launch_pdl(K kernel, unsigned blocks, unsigned threads, cudaStream_t
   return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
-template <typename T, int NT, bool A, bool D>
+template <typename T, int NT, bool A>
 cudaError_t launch_stats_nt(const Params& p, long blocks, cudaStream_t s) {
-  specverify::stats_kernel<T, NT, A, D><<<static_cast<unsigned>(blocks), NT, 0, s>>>(p);
+  specverify::stats_kernel<T, NT, A><<<static_cast<unsigned>(blocks), NT, 0, s>>>(p);
   return cudaGetLastError();
 }
 
-// One step.  Unmapped rows: the statistics kernel also takes each sequence's
-// decision; with row maps a decide kernel runs after it.  events[0..2] (may
-// be null): before stats, after stats (and decide), after draw.
+// One step: statistics, decide, draw.  events[0..2] (may be null): before
+// stats, after stats, after draw.
 template <typename T, bool A>
 cudaError_t launch_step(const Params& p, int NT, unsigned draw_blocks, cudaStream_t s,
                         cudaEvent_t* ev) {
   const long rows = p.target_rows + p.draft_rows;
   const long blocks = rows * p.slices;
-  const bool fused = p.target_map == nullptr && p.draft_map == nullptr;
   cudaError_t e = cudaSuccess;
   if (ev) e = cudaEventRecord(ev[0], s);
   if (e != cudaSuccess) return e;
-  switch (NT * 2 + (fused ? 1 : 0)) {
-    case 256: e = launch_stats_nt<T, 128, A, false>(p, blocks, s); break;
-    case 257: e = launch_stats_nt<T, 128, A, true>(p, blocks, s); break;
-    case 512: e = launch_stats_nt<T, 256, A, false>(p, blocks, s); break;
-    case 513: e = launch_stats_nt<T, 256, A, true>(p, blocks, s); break;
-    case 1024: e = launch_stats_nt<T, 512, A, false>(p, blocks, s); break;
-    case 1025: e = launch_stats_nt<T, 512, A, true>(p, blocks, s); break;
+  switch (NT) {
+    case 128: e = launch_stats_nt<T, 128, A>(p, blocks, s); break;
+    case 256: e = launch_stats_nt<T, 256, A>(p, blocks, s); break;
+    case 512: e = launch_stats_nt<T, 512, A>(p, blocks, s); break;
     default: return cudaErrorInvalidValue;
   }
-  if (e == cudaSuccess && !fused) {
+  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
+  if (e != cudaSuccess) return e;
+  {
     const int per = specverify::kDecideThreads / specverify::kWarp;
     e = launch_pdl(specverify::decide_kernel<T>, static_cast<unsigned>((p.batch + per - 1) / per),
                    specverify::kDecideThreads, s, p);
   }
-  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
   if (e != cudaSuccess) return e;
-  e = launch_pdl(specverify::draw_kernel<T, A>, draw_blocks, specverify::kDrawThreads, s, p);
+  e = specverify::launch_draw<T, A>(p, draw_blocks, s, true);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
   return e;
 }
@@ -269,7 +264,6 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
   p.decision = h->decision;
   p.draw_mass = h->draw_mass;
   p.draw_ticket = h->draw_ticket;
-  p.seq_ticket = h->seq_ticket;
   p.resid_mass = h->resid;
   p.status = h->status;
   p.batch = h->batch;
@@ -360,7 +354,7 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   const size_t offP = take(nD * sizeof(PosInfo));
   const size_t offC = take(nB * sizeof(SeqDecision));
   const size_t offW = take(nDraw * sizeof(double));
-  const size_t offK = take(2 * nB * sizeof(unsigned));  // draw tickets, then sequence tickets
+  const size_t offK = take(nB * sizeof(unsigned));
   const size_t offR = take(nB * sizeof(double));
   const size_t offS = take(sizeof(unsigned));
   const size_t offSR = take((nT + nD) * sizeof(specsamp::SampRow));
@@ -379,7 +373,6 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   h->decision = reinterpret_cast<SeqDecision*>(base + offC);
   h->draw_mass = reinterpret_cast<double*>(base + offW);
   h->draw_ticket = reinterpret_cast<unsigned*>(base + offK);
-  h->seq_ticket = h->draw_ticket + nB;
   h->resid = reinterpret_cast<double*>(base + offR);
   h->status = reinterpret_cast<unsigned*>(base + offS);
   h->samp_rows = reinterpret_cast<specsamp::SampRow*>(base + offSR);
@@ -833,7 +826,7 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
   const size_t offP = take(nD * sizeof(PosInfo));
   const size_t offC = take(nB * sizeof(SeqDecision));
   const size_t offW = take(nDraw * sizeof(double));
-  const size_t offK = take(2 * nB * sizeof(unsigned));  // draw tickets, then sequence tickets
+  const size_t offK = take(nB * sizeof(unsigned));
   const size_t offR = take(nB * sizeof(double));
   const size_t offS = take(sizeof(unsigned));
   if (off > kNoAllocScratchBytes) {
@@ -850,7 +843,6 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
   h.decision = reinterpret_cast<SeqDecision*>(base + offC);
   h.draw_mass = reinterpret_cast<double*>(base + offW);
   h.draw_ticket = reinterpret_cast<unsigned*>(base + offK);
-  h.seq_ticket = h.draw_ticket + nB;
   h.resid = reinterpret_cast<double*>(base + offR);
   h.status = reinterpret_cast<unsigned*>(base + offS);
 
@@ -861,10 +853,10 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
                                    nullptr, nullptr);
   if (chk != SV_OK) return chk;
 
-  // the array keeps the previous call's contents: the tickets and the
+  // the array keeps the previous call's contents: the draw tickets and the
   // status word must start at zero
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  e = cudaMemsetAsync(h.draw_ticket, 0, 2 * nB * sizeof(unsigned), s);
+  e = cudaMemsetAsync(h.draw_ticket, 0, nB * sizeof(unsigned), s);
   if (e == cudaSuccess) e = cudaMemsetAsync(h.status, 0, sizeof(unsigned), s);
   if (e != cudaSuccess) return cuda_fail(e);
   return enqueue(&h, target_logits, draft_logits, draft_tokens, u_accept, u_resample,

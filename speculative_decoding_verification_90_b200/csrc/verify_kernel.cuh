@@ -1,30 +1,26 @@
 // Speculative-sampling verification kernels for sm_100a.
 //
-// One verification step of unmapped rows is two stream-ordered kernels (the
-// second launched early through programmatic dependent launch and waiting for
-// the first with a grid-dependency barrier):
+// One verification step is three stream-ordered kernels (each later one
+// launched early through programmatic dependent launch and waiting for its
+// predecessor with a grid-dependency barrier):
 //
 //   stats   S blocks per logit row (every target row, then every draft
 //           row), each streaming its contiguous 1/S of the row with 128-bit
 //           coalesced loads, eight in flight per thread; each thread keeps a
 //           running sum of 2^(x c - o) against a lazily raised offset o; the
 //           block writes its (o, sum) partial (step 1 of the round: softmax
-//           statistics).  This is the kernel that moves all of the logit
-//           bytes.  The block that finishes a sequence's last slice (an
-//           atomic ticket per sequence) then takes its decision with one
-//           warp, one lane per position: the lane combines the position's
-//           partials into log2 sum_i 2^(x_i c), forms q(t), p(t) and the
-//           ratio, and a warp ballot finds the first rejection n (steps 2
-//           and 3); it writes the accepted prefix and what to draw from.
+//           statistics).  No atomics, no waits, the same work in every block:
+//           this is the kernel that moves all of the logit bytes.
+//   decide  one warp per sequence, one lane per position: the lane combines
+//           the position's partials into log2 sum_i 2^(x_i c), forms q(t),
+//           p(t) and the ratio, and a warp ballot finds the first rejection n
+//           (steps 2 and 3); writes the accepted prefix and what to draw from.
 //   draw    the grid's warps split every tile of every sequence's rows drawn
 //           from (n < gamma: max(0, q_n - p_n) from target and draft row n;
 //           n == gamma: q of target row gamma) into even contiguous runs,
 //           write each tile's mass, and the warp that completes a sequence's
 //           tiles (an atomic ticket) locates u * Z by a warp scan over the
 //           tile masses and one re-read tile (step 4).
-//
-// With row maps (rows shared between positions) or the LM-head-fused step, a
-// separate decide kernel (one warp per sequence) runs between the two.
 //
 // No thread ever waits for another block (the only hand-off inside a kernel
 // is an atomic ticket, never a spin).
@@ -116,7 +112,6 @@ struct Params {
   SeqDecision* decision;     // [B]
   double* draw_mass;         // [B * tiles of a row] mass of each 32-group tile of the draw
   unsigned* draw_ticket;     // [B], zero between launches
-  unsigned* seq_ticket;      // [B], zero between launches (statistics slices done)
   double* resid_mass;        // [B]
   unsigned* status;          // [1]
   int batch, gamma, vocab;
@@ -429,36 +424,15 @@ __device__ __forceinline__ void block_scan(double v, double& incl, double& excl,
 constexpr int kDecideThreads = 128;
 constexpr int kMaxGamma = 255;
 
-// One row's partial.  kL2: read through L2 only, for partials that other
-// blocks of the running kernel wrote (L1 is not coherent with their stores).
-template <bool kL2>
-__device__ __forceinline__ void load_partial(const RowPartial* p, float& o, double& s) {
-  if constexpr (kL2) {
-    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(p));
-    s = __hiloint2double(static_cast<int>(v.y), static_cast<int>(v.x));
-    o = __uint_as_float(v.z);
-  } else {
-    s = p->s;
-    o = p->o;
-  }
-}
-
 // (o, s) partials of one row combined in two passes, so that the fp64
 // exponentials of the second pass are independent of one another
-template <bool kL2>
 __device__ __forceinline__ double row_lse2(const RowPartial* parts, int S, int& valid) {
   float O = -INFINITY;
-  for (int r = 0; r < S; ++r) {
-    float o;
-    double s;
-    load_partial<kL2>(parts + r, o, s);
-    O = fmaxf(O, o);
-  }
+  for (int r = 0; r < S; ++r) O = fmaxf(O, parts[r].o);
   double sum = 0.0;
   for (int r = 0; r < S; ++r) {
-    float o;
-    double s;
-    load_partial<kL2>(parts + r, o, s);
+    const float o = parts[r].o;
+    const double s = parts[r].s;
     sum += (o == -INFINITY) ? s * 0.0 : s * exp2(static_cast<double>(o) - O);  // NaN survives
   }
   valid = (O != -INFINITY) && isfinite(sum) && sum > 0.0;
@@ -470,7 +444,7 @@ __device__ __forceinline__ double row_lse2(const RowPartial* parts, int S, int& 
 // in fp64 and tests u < ratio (step 2); a warp ballot finds the first
 // rejection n (step 3).  Writes the accepted prefix, the padding, the count,
 // the per-position readback records and what the draw kernel draws from.
-template <typename T, bool kL2>
+template <typename T>
 __device__ __forceinline__ void decide_sequence(const Params& P, int b) {
   const int lane = threadIdx.x & (kWarp - 1);
   const int G = P.gamma, V = P.vocab, S = P.slices;
@@ -509,8 +483,8 @@ __device__ __forceinline__ void decide_sequence(const Params& P, int b) {
       }
       int validT = 0, validD = 1;
       if (!map_bad) {
-        lT = row_lse2<kL2>(P.partial + tr * S, S, validT);
-        if (has_draft) lD = row_lse2<kL2>(P.partial + (P.target_rows + dr) * S, S, validD);
+        lT = row_lse2(P.partial + tr * S, S, validT);
+        if (has_draft) lD = row_lse2(P.partial + (P.target_rows + dr) * S, S, validD);
       }
       P.tstat[position] = RowStat{lT, validT, 0};
       if (has_draft) P.dstat[pj] = RowStat{lD, validD, 0};
@@ -583,16 +557,8 @@ __device__ __forceinline__ void decide_sequence(const Params& P, int b) {
   }
 }
 
-// Called from the statistics kernel: kept out of line so that the streaming
-// loop's register allocation does not carry the decision's.
-template <typename T>
-__device__ __noinline__ void decide_sequence_l2(const Params* P, int b) {
-  __threadfence();  // every lane reads the other blocks' partials after the ticket
-  decide_sequence<T, true>(*P, b);
-}
-
 // ---------------------------------------------------------------------------
-// kernel 1: streaming statistics (and, unmapped, each sequence's decision)
+// kernel 1: streaming statistics
 // ---------------------------------------------------------------------------
 
 template <int NT>
@@ -600,12 +566,8 @@ constexpr int min_blocks() {
   return 1024 / NT;  // caps registers at 64 per thread
 }
 
-// kDecide (unmapped rows only): the block that completes the last slice of a
-// sequence's 2 gamma + 1 rows takes that sequence's decision with its first
-// warp, so the decisions are made while the other rows still stream and no
-// separate decide launch sits between the statistics and the draw.
-template <typename T, int NT, bool kAligned, bool kDecide>
-__global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const __grid_constant__ Params P) {
+template <typename T, int NT, bool kAligned>
+__global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Params P) {
   constexpr int kVec = Elem<T>::kVec;
   const int V = P.vocab, S = P.slices;
   // one unit = one block = one slice of one row; the target tensor's rows
@@ -623,29 +585,11 @@ __global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const __gri
   if (ghi > ngroups) ghi = ngroups;
   const RowPartial part = slice_stats<T, NT, kAligned, 8>(row, glo, ghi, V, P.c_hi, P.c_lo);
   if (threadIdx.x == 0) P.partial[unit] = part;
-  if constexpr (kDecide) {
-    __shared__ int sm_b;
-    if (threadIdx.x == 0) {
-      const int G = P.gamma;
-      const int b = (r < nT || G == 0) ? static_cast<int>(r / (G + 1))
-                                       : static_cast<int>((r - nT) / G);
-      __threadfence();  // this block's partial is visible before its ticket
-      const unsigned need = static_cast<unsigned>((2 * G + 1) * S);
-      const unsigned old = atomicAdd(P.seq_ticket + b, 1u);
-      sm_b = (old == need - 1) ? b : -1;
-      if (sm_b >= 0) {
-        __threadfence();        // every partial of the sequence is visible
-        P.seq_ticket[b] = 0u;   // ready for the next launch
-      }
-    }
-    __syncthreads();
-    if (sm_b >= 0 && threadIdx.x < kWarp) decide_sequence_l2<T>(&P, sm_b);
-  }
   cudaTriggerProgrammaticLaunchCompletion();
 }
 
 // ---------------------------------------------------------------------------
-// kernel 2: decide (mapped rows, the LM-head-fused step): one warp per sequence
+// kernel 2: decide (one warp per sequence)
 // ---------------------------------------------------------------------------
 
 template <typename T>
@@ -653,7 +597,7 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
   // the statistics of the previous kernel must be complete and visible
   cudaGridDependencySynchronize();
   const int b = blockIdx.x * (kDecideThreads / kWarp) + (threadIdx.x >> 5);
-  if (b < P.batch) decide_sequence<T, false>(P, b);  // warp-uniform
+  if (b < P.batch) decide_sequence<T>(P, b);  // warp-uniform
   cudaTriggerProgrammaticLaunchCompletion();
 }
 
@@ -667,17 +611,23 @@ __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) 
 // batch, sequence by sequence, form one index range that the grid's warps
 // split into contiguous runs, so the work is even whatever mix of residual
 // draws (two rows), bonus draws (one row) and error outcomes (none) the batch
-// holds.  A warp writes the fp64 mass of each tile of its run to the
-// sequence's table, then adds the number of tiles it finished to the
-// sequence's ticket; the warp that completes the count locates u * Z: a warp
-// scan over the table finds the tile, and a re-read of that one tile finds
-// the index.
+// holds.  A warp streams its run through a private ring of kStages tiles in
+// shared memory filled by asynchronous 16-byte copies (cp.async; each lane
+// copies and later reads only its own slots), so about three tiles per warp
+// are in flight while one is reduced, without holding them in registers.  It
+// writes the fp64 mass of each tile of its run to the sequence's table, then
+// adds the number of tiles it finished to the sequence's ticket; the warp
+// that completes the count locates u * Z: a warp scan over the table finds
+// the tile, and a re-read of that one tile finds the index.
 
 constexpr int kDrawThreads = 256;
 constexpr int kDrawWarps = kDrawThreads / kWarp;
 constexpr int kDrawK = 2;                 // groups per lane per tile
 constexpr int kTile = kWarp * kDrawK;     // groups per tile of the mass table
 constexpr int kDrawBlocksPerSM = 2;
+constexpr int kStages = 4;                          // ring depth per warp
+constexpr int kStageU4 = 2 * kDrawK * kWarp;        // 16-byte slots per warp per stage
+constexpr size_t kDrawSmem = sizeof(uint4) * kStageU4 * kStages * kDrawWarps;
 
 // tiles of one row of V entries stored `vec` to a 16-byte group
 inline long draw_tiles_per_row(long V, int vec) {
@@ -826,6 +776,71 @@ __device__ __forceinline__ void tile_masses_mode(const T* rowT, const T* rowD, c
   }
 }
 
+__device__ __forceinline__ void cp_async16(uint4* smem, const uint4* gmem) {
+  const unsigned sa = static_cast<unsigned>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// One tile's copies into a ring slot: target groups at [kk * 32 + lane],
+// draft groups at [(kDrawK + kk) * 32 + lane]; groups past the row end are
+// not copied (and not read).
+template <int kMode>
+__device__ __forceinline__ void issue_tile(uint4* slot, const uint4* rowT, const uint4* rowD,
+                                           long tile, long ngroups) {
+  const int lane = threadIdx.x & (kWarp - 1);
+#pragma unroll
+  for (int kk = 0; kk < kDrawK; ++kk) {
+    const long g = tile * kTile + kk * kWarp + lane;
+    if (g < ngroups) {
+      cp_async16(slot + kk * kWarp + lane, rowT + g);
+      if constexpr (kMode == kDrawResidual) cp_async16(slot + (kDrawK + kk) * kWarp + lane, rowD + g);
+    }
+  }
+}
+
+// Masses of tiles [t0, t1) of one row (16-byte aligned rows) into table,
+// through the calling warp's ring: kStages - 1 tiles are in flight while one
+// is reduced.  Every iteration commits one copy group (possibly empty), so
+// waiting until at most kStages - 1 groups are pending means the oldest
+// tile has landed.  Returns with no copy in flight.
+template <typename T, int kMode>
+__device__ __forceinline__ void tile_masses_ring(const T* rowT, const T* rowD, const DrawConsts& k,
+                                                 long t0, long t1, long ngroups, double* table,
+                                                 uint4* ring) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  const uint4* gT = reinterpret_cast<const uint4*>(rowT);
+  const uint4* gD = reinterpret_cast<const uint4*>(rowD);
+  const long n = t1 - t0;
+#pragma unroll
+  for (int i = 0; i < kStages - 1; ++i) {
+    if (i < n) issue_tile<kMode>(ring + i * kStageU4, gT, gD, t0 + i, ngroups);
+    cp_async_commit();
+  }
+  for (long i = 0; i < n; ++i) {
+    const long nx = i + kStages - 1;
+    if (nx < n) issue_tile<kMode>(ring + (nx % kStages) * kStageU4, gT, gD, t0 + nx, ngroups);
+    cp_async_commit();
+    cp_async_wait<kStages - 1>();
+    const uint4* slot = ring + (i % kStages) * kStageU4;
+    uint4 vt[kDrawK], vd[kDrawK];
+#pragma unroll
+    for (int kk = 0; kk < kDrawK; ++kk) {
+      vt[kk] = slot[kk * kWarp + lane];
+      if constexpr (kMode == kDrawResidual) vd[kk] = slot[(kDrawK + kk) * kWarp + lane];
+    }
+    const double z = tile_mass_of<T, kMode>(vt, vd, k, t0 + i, ngroups);
+    if (lane == 0) table[t0 + i] = z;
+  }
+  cp_async_wait<0>();
+}
+
 template <typename T, bool kAligned>
 __device__ __forceinline__ void tile_masses(int mode, const T* rowT, const T* rowD,
                                             const DrawConsts& k, long t0, long t1, long ngroups,
@@ -895,6 +910,148 @@ __device__ __forceinline__ int scan_tile(const T* rowT, const T* rowD, const Dra
   return warp_maxi(mylast);  // rounding past the tile's end
 }
 
+constexpr int kLocRun = 10;  // table entries per lane per round of the scans below
+
+// Sum of table[0 .. ntiles) by the calling warp: each lane loads a contiguous
+// run of kLocRun entries per round (all loads of a round in flight together)
+// and adds it in index order; lane sums are combined across the warp.
+__device__ __forceinline__ double table_total(const double* table, long ntiles) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  double tot = 0.0;
+  for (long r0 = 0; r0 < ntiles; r0 += static_cast<long>(kWarp) * kLocRun) {
+    const long a = r0 + static_cast<long>(lane) * kLocRun;
+    double v[kLocRun];
+#pragma unroll
+    for (int q = 0; q < kLocRun; ++q) v[q] = (a + q < ntiles) ? __ldcg(table + a + q) : 0.0;
+    double sm = 0.0;
+#pragma unroll
+    for (int q = 0; q < kLocRun; ++q) sm += v[q];
+    tot += warp_sum(sm);
+  }
+  return tot;
+}
+
+// The first entry i of table[0 .. ntiles) with positive mass whose running
+// sum in index order passes `target` (found = i, tl = target minus the mass
+// before i), by the calling warp: per round, lane runs as in table_total, a
+// warp scan of the lane sums picks the lane and that lane walks its run.  If
+// rounding leaves no such entry, the last entry with mass and tl = +inf.
+__device__ __forceinline__ void find_in_table(const double* table, long ntiles, double target,
+                                              long& found, double& tl) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  double base = 0.0;
+  long last_mass = -1;
+  found = -1;
+  tl = INFINITY;
+  for (long r0 = 0; r0 < ntiles; r0 += static_cast<long>(kWarp) * kLocRun) {
+    const long a = r0 + static_cast<long>(lane) * kLocRun;
+    double v[kLocRun];
+#pragma unroll
+    for (int q = 0; q < kLocRun; ++q) v[q] = (a + q < ntiles) ? __ldcg(table + a + q) : 0.0;
+    double sm = 0.0;
+    long mylast = -1;
+#pragma unroll
+    for (int q = 0; q < kLocRun; ++q) {
+      sm += v[q];
+      if (v[q] > 0.0) mylast = a + q;
+    }
+    double incl = sm;
+#pragma unroll
+    for (int o = 1; o < kWarp; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.0;
+    long lm = mylast;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lm = max(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+    if (lm >= 0) last_mass = lm;
+    const unsigned hit =
+        __ballot_sync(0xffffffffu, sm > 0.0 && base + excl <= target && base + incl > target);
+    if (hit) {
+      const int Ln = __ffs(hit) - 1;
+      long f = -1;
+      double t = INFINITY;
+      if (lane == Ln) {
+        double acc = base + excl;
+#pragma unroll
+        for (int q = 0; q < kLocRun; ++q) {
+          if (f < 0 && v[q] > 0.0 && acc + v[q] > target) {
+            f = a + q;
+            t = target - acc;
+          }
+          acc += v[q];
+        }
+        if (f < 0) f = mylast;  // rounding between the lane sum and this walk
+      }
+      found = __shfl_sync(0xffffffffu, f, Ln);
+      tl = __shfl_sync(0xffffffffu, t, Ln);
+      return;
+    }
+    base += __shfl_sync(0xffffffffu, incl, kWarp - 1);
+  }
+  found = last_mass;  // rounding past the table's end
+  tl = INFINITY;
+}
+
+// find_in_table for a table of at most kWarp * kLocRun entries, with the
+// total computed from the same loads; returns Z (found = -1 if Z is 0).
+__device__ __forceinline__ double locate_one_round(const double* table, long ntiles, double u,
+                                                   long& found, double& tl) {
+  const int lane = threadIdx.x & (kWarp - 1);
+  const long a = static_cast<long>(lane) * kLocRun;
+  double v[kLocRun];
+#pragma unroll
+  for (int q = 0; q < kLocRun; ++q) v[q] = (a + q < ntiles) ? __ldcg(table + a + q) : 0.0;
+  double sm = 0.0;
+  long mylast = -1;
+#pragma unroll
+  for (int q = 0; q < kLocRun; ++q) {
+    sm += v[q];
+    if (v[q] > 0.0) mylast = a + q;
+  }
+  double incl = sm;
+#pragma unroll
+  for (int o = 1; o < kWarp; o <<= 1) {
+    const double y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  double excl = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) excl = 0.0;
+  const double Z = __shfl_sync(0xffffffffu, incl, kWarp - 1);
+  found = -1;
+  tl = INFINITY;
+  if (!(Z > 0.0)) return Z;
+  const double target = u * Z;
+  const unsigned hit = __ballot_sync(0xffffffffu, sm > 0.0 && excl <= target && incl > target);
+  if (hit) {
+    const int Ln = __ffs(hit) - 1;
+    long f = -1;
+    double t = INFINITY;
+    if (lane == Ln) {
+      double acc = excl;
+#pragma unroll
+      for (int q = 0; q < kLocRun; ++q) {
+        if (f < 0 && v[q] > 0.0 && acc + v[q] > target) {
+          f = a + q;
+          t = target - acc;
+        }
+        acc += v[q];
+      }
+      if (f < 0) f = mylast;  // rounding between the lane sum and this walk
+    }
+    found = __shfl_sync(0xffffffffu, f, Ln);
+    tl = __shfl_sync(0xffffffffu, t, Ln);
+  } else {
+    long lm = mylast;  // rounding past the table's end: the last entry with mass
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lm = max(lm, __shfl_xor_sync(0xffffffffu, lm, o));
+    found = lm;
+  }
+  return Z;
+}
+
 // Step 4's last part for sequence b, by the warp that finished its table:
 // Z = sum of the tile masses; the tile holding u * Z (a warp scan over the
 // table in index order); the index inside it.  Z = 0 at a rejection: the
@@ -908,48 +1065,23 @@ __device__ __noinline__ void locate(const Params* Pp, int b, int mode, const T* 
   const int V = P.vocab, G = P.gamma;
   double* table = P.draw_mass + static_cast<long>(b) * ntiles;
   unsigned extra_bits = 0;
-  double Z = 0.0;
-  for (long i = lane; i < ntiles; i += kWarp) Z += __ldcg(table + i);
-  Z = warp_sum(Z);
+  const double u = static_cast<double>(P.u_resample[b]);
+  long found = -1;
+  double tl = INFINITY, Z = 0.0;
+  // a table of at most one round of lane runs is read once: Z and the place
+  // of u * Z come from the same loads
+  const bool one_round = ntiles <= static_cast<long>(kWarp) * kLocRun;
+  if (one_round) Z = locate_one_round(table, ntiles, u, found, tl);
+  else Z = table_total(table, ntiles);
   if (!(Z > 0.0) && mode == kDrawResidual) {
     mode = kDrawTarget;
     extra_bits |= kStatZeroMass;
     tile_masses<T, kAligned>(mode, rowT, rowD, k, 0, ntiles, ngroups, V, table);
     __syncwarp();
-    Z = 0.0;
-    for (long i = lane; i < ntiles; i += kWarp) Z += __ldcg(table + i);
-    Z = warp_sum(Z);
+    if (one_round) Z = locate_one_round(table, ntiles, u, found, tl);
+    else Z = table_total(table, ntiles);
   }
-  const double target = static_cast<double>(P.u_resample[b]) * Z;
-  long found = -1, last_mass = -1;
-  double tl = 0.0, base = 0.0;
-  for (long c0 = 0; c0 < ntiles; c0 += kWarp) {
-    const long i = c0 + lane;
-    const double v = (i < ntiles) ? __ldcg(table + i) : 0.0;
-    double incl = v;
-#pragma unroll
-    for (int o = 1; o < kWarp; o <<= 1) {
-      const double y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    double excl = __shfl_up_sync(0xffffffffu, incl, 1);
-    if (lane == 0) excl = 0.0;
-    const unsigned hit =
-        __ballot_sync(0xffffffffu, v > 0.0 && base + excl <= target && base + incl > target);
-    const unsigned has = __ballot_sync(0xffffffffu, v > 0.0);
-    if (has) last_mass = c0 + (31 - __clz(has));
-    if (hit) {
-      const int Ln = __ffs(hit) - 1;
-      found = c0 + Ln;
-      tl = __shfl_sync(0xffffffffu, target - (base + excl), Ln);
-      break;
-    }
-    base += __shfl_sync(0xffffffffu, incl, kWarp - 1);
-  }
-  if (found < 0) {  // rounding: the tile's last index with mass
-    found = last_mass;
-    tl = INFINITY;
-  }
+  if (!one_round) find_in_table(table, ntiles, u * Z, found, tl);
   int token = -1;
   if (found >= 0) {
     token = (mode == kDrawResidual)
@@ -968,6 +1100,8 @@ __device__ __noinline__ void locate(const Params* Pp, int b, int mode, const T* 
 template <typename T, bool kAligned>
 __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(const __grid_constant__ Params P) {
   constexpr int kVec = Elem<T>::kVec;
+  extern __shared__ uint4 draw_smem[];
+  uint4* ring = draw_smem + (threadIdx.x >> 5) * (kStageU4 * kStages);  // this warp's ring
   const int lane = threadIdx.x & (kWarp - 1);
   const int V = P.vocab;
   const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
@@ -994,7 +1128,14 @@ __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(co
       k.k_lo = d.k_lo;
       k.fT = d.fT;
       double* table = P.draw_mass + row0;
-      tile_masses<T, kAligned>(d.mode, rowT, rowD, k, t - row0, end - row0, ngroups, V, table);
+      if constexpr (kAligned) {
+        if (d.mode == kDrawResidual)
+          tile_masses_ring<T, kDrawResidual>(rowT, rowD, k, t - row0, end - row0, ngroups, table, ring);
+        else
+          tile_masses_ring<T, kDrawTarget>(rowT, rowD, k, t - row0, end - row0, ngroups, table, ring);
+      } else {
+        tile_masses<T, kAligned>(d.mode, rowT, rowD, k, t - row0, end - row0, ngroups, V, table);
+      }
       // publish this run's tiles; the warp that completes the row locates
       unsigned last = 0;
       if (lane == 0) {
@@ -1012,6 +1153,30 @@ __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(co
     }
     t = end;
   }
+}
+
+// Host: launch the draw kernel (its ring needs more than the default 48 KB of
+// dynamic shared memory per block), optionally as a programmatic dependent
+// launch of the previous kernel on the stream.
+template <typename T, bool kAligned>
+inline cudaError_t launch_draw(const Params& p, unsigned grid, cudaStream_t s, bool pdl) {
+  const size_t smem = kAligned ? kDrawSmem : 0;
+  cudaError_t e = cudaSuccess;
+  if (kAligned)
+    e = cudaFuncSetAttribute(draw_kernel<T, kAligned>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kDrawThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, draw_kernel<T, kAligned>, p);
 }
 
 }  // namespace specverify
