@@ -60,9 +60,6 @@ KERNEL_SOURCES = [
 ]
 
 
-# kernels of one plain step: statistics, decide, draw
-LAUNCHES_PER_STEP = 3
-
 # sampling-variant settings timed by the bench: name -> (temperature, top_k, top_p);
 # None = the workload's temperature
 SAMPLING_SETTINGS = {"greedy": (0.0, 0, 1.0), "top_k50_top_p0.9": (None, 50, 0.9),
@@ -93,6 +90,9 @@ def parse():
                     help="skip the timing of the LM-head-fused step (64 x 8, V 128256, d 4096)")
     ap.add_argument("--no-gate", action="store_true",
                     help="skip the timing of the fold gate (128 x 8 branches, 32 x 4096 bf16)")
+    ap.add_argument("--oracle-table", action="store_true",
+                    help="with --impl reference: time the CPU oracle on every benchmark "
+                         "configuration at one thread and at all host threads (bounded samples)")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other benchmark configurations (64 x 8 at V 128256, 8 x 3 at "
                          "V 32000, the char-level calls, the 60000-row exactness batch)")
@@ -104,16 +104,24 @@ def parse():
     return args
 
 
+# the parts of the kernel source that make up the statistics kernel
+STATS_SOURCE_RANGES = [
+    ("// phase 1: streaming softmax statistics", "// phase 4 helpers"),
+    ("// block-level helpers", "// block-wide scan of one double"),
+    ("// kernel 1: streaming statistics", "// kernel 2:"),
+]
+
+
 def kernel_hash() -> str:
-    """Hash of the statistics kernel's code: its part of the source, from the
-    streaming-statistics helpers through the kernel itself."""
+    """Hash of the statistics kernel's code: the streaming-statistics helpers,
+    the block reduction and the kernel itself."""
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
         with open(os.path.join(ROOT, rel)) as f:
             text = f.read()
-        a = text.find("// phase 1: streaming softmax statistics")
-        b = text.find("// kernel 2:")
-        h.update(text[a:b].encode() if 0 <= a < b else text.encode())
+        for start, end in STATS_SOURCE_RANGES:
+            a, b = text.find(start), text.find(end)
+            h.update(text[a:b].encode() if 0 <= a < b else text.encode())
     return h.hexdigest()[:16]
 
 
@@ -247,10 +255,46 @@ def time_oracle(wl, budget_s: float):
     return value, threads, sample, elapsed / passes
 
 
+def oracle_table(args):
+    """Oracle positions/s on every configuration, one thread and all host
+    threads, each a bounded sample (about 2 s of wall time per entry)."""
+    import oracle
+    oracle.build()
+    threads = os.cpu_count() or 1
+    with open(os.path.join(ROOT, "tests", "golden", "exactness_beta.json")) as f:
+        beta = json.load(f)["beta"]
+    wls = {"char_level": workloads.char_level(seed=args.seed),
+           "exactness": workloads.exactness(beta, seed=args.seed, batch=4096),
+           "b8_g3_v32000": workloads.b8_g3_v32000(seed=args.seed),
+           "b64_g8_v128256": workloads.b64_g8_v128256(seed=args.seed),
+           "multibranch": workloads.multibranch(seed=args.seed)}
+    out = {}
+    for name, wl in wls.items():
+        row = {"workload": wl.name}
+        for th in (1, threads):
+            n = min(wl.batch, th)
+            t = time.perf_counter()
+            oracle.verify(wl.target[:n], wl.draft[:n], wl.tokens[:n], wl.u_accept[:n],
+                          wl.u_resample[:n], wl.temperature, threads=th)
+            one = max(1e-6, time.perf_counter() - t)
+            n = int(min(wl.batch, max(1, 2.0 / one) * n))
+            t = time.perf_counter()
+            oracle.verify(wl.target[:n], wl.draft[:n], wl.tokens[:n], wl.u_accept[:n],
+                          wl.u_resample[:n], wl.temperature, threads=th)
+            el = time.perf_counter() - t
+            row[f"threads_{th}"] = {"positions_per_s": n * wl.gamma / el, "sequences": n,
+                                    "seconds": el}
+        out[name] = row
+    print(json.dumps({"impl": "reference", "oracle_table": out, "cores": threads}), flush=True)
+    return 0
+
+
 def run_reference(args):
     rank = svdist.env_rank()[0]
     if rank != 0:
         return 0  # the CPU reference runs once, on rank 0
+    if args.oracle_table:
+        return oracle_table(args)
     wl = make_workload(args.workload, args.seed)
     import oracle
     oracle.build()
@@ -332,6 +376,7 @@ def run_ours(args):
         sv.set_launch(args.slices or c0, args.threads or t0, args.draw_slices)
     slices, threads = sv.launch()
     sv_draw = sv.draw_slices
+    kernels_per_step = sv.kernels_per_run()
 
     def step(i):
         s = sets[i % n_sets]
@@ -454,7 +499,7 @@ def run_ours(args):
             "emitted_tokens_per_step": emitted,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": kernels_per_step * args.steps,
             "clocks": clocks,
             "cpu_baseline": cpu,
             "status_after": st,
@@ -540,6 +585,46 @@ def _time_calls(sv, sets, wl, calls, warmup, out_t, out_n, slices=None):
     return ev0.elapsed_time(ev1), kern
 
 
+def _time_graph(sv, sets, wl, calls, out_t, out_n, slices=None):
+    """Device time of `calls` calls captured once in a CUDA graph and replayed
+    (launch-bound configurations: the host's per-call overhead is left out).
+    Returns milliseconds per replay of all calls, or None if capture fails."""
+    import torch
+    n = len(sets)
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    try:
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for i in range(calls):
+                    d = sets[i % n]
+                    if slices is None:
+                        sv.run(d["target"], d["draft"], d["tokens"], d["u_accept"],
+                               d["u_resample"], wl.temperature, out_t, out_n)
+                    else:
+                        b0, b1 = slices[i % len(slices)]
+                        sv.run(d["target"][b0:b1], d["draft"][b0:b1], d["tokens"][b0:b1],
+                               d["u_accept"][b0:b1], d["u_resample"][b0:b1], wl.temperature,
+                               out_t, out_n)
+    except Exception as exc:  # capture not possible here: report eager timing only
+        torch.cuda.synchronize()
+        return None, f"{type(exc).__name__}: {exc}"[:200]
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    reps = 5
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for _ in range(reps):
+        g.replay()
+    ev1.record()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1) / reps
+    del g
+    return ms, None
+
+
 def time_other_configs(args, dev):
     """The other benchmark configurations, one GPU: the 64-sequence gamma-8
     batch at V = 128256 (a plain step like the headline's); the 8-sequence
@@ -574,21 +659,24 @@ def time_other_configs(args, dev):
     calls = max(200, 4 * steps)
     with SpecVerify(wl.batch, wl.gamma, wl.vocab, wl.dtype, dev.index) as sv:
         ms, kern = _time_calls(sv, sets, wl, calls, args.warmup, out_t, out_n)
+        gms, gerr = _time_graph(sv, sets, wl, calls, out_t, out_n)
         st, _ = sv.status()
     res["b8_g3_v32000"] = {"wl": wl, "ms": ms, "calls": calls, "kern": kern, "sets": n_sets,
-                           "status": st}
+                           "status": st, "graph_ms": gms, "graph_err": gerr}
     del sets, d
     # configuration 1: 1000 independent calls of one sequence each
     wl = workloads.char_level(calls=1000, seed=args.seed)
     d = _device_inputs(wl, dev)
     out_t = torch.empty((1, wl.gamma + 1), dtype=torch.int32, device=dev)
     out_n = torch.empty((1,), dtype=torch.int32, device=dev)
+    one_by_one = [(b, b + 1) for b in range(wl.batch)]
     with SpecVerify(1, wl.gamma, wl.vocab, wl.dtype, dev.index) as sv:
         ms, kern = _time_calls(sv, [d], wl, wl.batch, args.warmup, out_t, out_n,
-                               slices=[(b, b + 1) for b in range(wl.batch)])
+                               slices=one_by_one)
+        gms, gerr = _time_graph(sv, [d], wl, wl.batch, out_t, out_n, slices=one_by_one)
         st, _ = sv.status()
     res["char_level"] = {"wl": wl, "ms": ms, "calls": wl.batch, "kern": kern, "sets": 1,
-                         "status": st}
+                         "status": st, "graph_ms": gms, "graph_err": gerr}
     del d
     # configuration 2: the exactness batch, one call; the law of its outputs
     with open(os.path.join(ROOT, "tests", "golden", "exactness_beta.json")) as f:
@@ -628,6 +716,16 @@ def others_summary(res, peak):
              "kernels_us_per_call": {"stats": 1e3 * r["kern"]["stats_ms"],
                                      "decide_and_draw": 1e3 * r["kern"]["draw_ms"]},
              "status_after": r["status"]}
+        if r.get("graph_ms") is not None or r.get("graph_err"):
+            # launch-bound: the same calls captured once in a CUDA graph and
+            # replayed, so the host's per-call overhead is left out
+            if r.get("graph_ms") is not None:
+                gcall = r["graph_ms"] / 1e3 / r["calls"]
+                e["graph"] = {"us_per_call": gcall * 1e6, "calls_per_s": 1.0 / gcall,
+                              "value": (wl.gamma if name == "char_level" else positions) / gcall,
+                              "unit": "positions/s"}
+            else:
+                e["graph"] = {"unavailable": r["graph_err"]}
         if name == "char_level":
             # one sequence per call
             e["calls_per_s"] = 1.0 / per_call_s

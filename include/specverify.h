@@ -250,6 +250,13 @@ sv_status specverify_get_launch(specverify_t h, int *slices, int *threads, int *
                                 int *draw_slices);
 
 /*
+ * Number of kernels one run of the handle enqueues (`mapped` nonzero: a run
+ * of specverify_run_mapped): statistics, decide and draw; none for an empty
+ * batch.
+ */
+sv_status specverify_kernels_per_run(specverify_t h, int mapped, int *kernels);
+
+/*
  * Per-kernel timing of the next `max_runs` runs of the handle: each run then
  * records CUDA events on its stream around its two kernels (the statistics
  * kernel, which streams every logit, and the decide-and-draw kernel).  Waits

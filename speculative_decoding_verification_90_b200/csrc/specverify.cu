@@ -273,6 +273,7 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
   p.slices = h->slices;
   p.groups_per_slice = static_cast<int>((ngroups + h->slices - 1) / h->slices);
   p.draw_tiles = draw_tiles(h);
+  const unsigned nd = draw_blocks(h);
   p.c_hi = c_hi;
   p.c_lo = c_lo;
   p.c = static_cast<double>(c_hi) + static_cast<double>(c_lo);
@@ -284,7 +285,6 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
                        (static_cast<size_t>(h->vocab) * es) % 16 == 0;
   cudaEvent_t* ev = nullptr;
   if (h->prof_runs < h->prof_capacity) ev = h->events.data() + 3 * (h->prof_runs++);
-  const unsigned nd = draw_blocks(h);
   cudaError_t e = (h->dtype == SV_DTYPE_BF16)
                       ? launch_dtype<__nv_bfloat16>(p, h->threads, nd, aligned, stream, ev)
                       : launch_dtype<float>(p, h->threads, nd, aligned, stream, ev);
@@ -651,6 +651,13 @@ sv_status specverify_get_launch(specverify_t h, int* slices, int* threads, int* 
   if (slices) *slices = h->slices;
   if (threads) *threads = h->threads;
   if (draw_slices) *draw_slices = h->draw_slices;
+  return SV_OK;
+}
+
+sv_status specverify_kernels_per_run(specverify_t h, int mapped, int* kernels) {
+  if (!h || !kernels) return SV_ERR_INVALID_ARG;
+  (void)mapped;  // the mapped form launches the same kernels
+  *kernels = h->batch == 0 ? 0 : 3;  // statistics, decide, draw
   return SV_OK;
 }
 

@@ -50,6 +50,7 @@ SIGNATURES = {
     "specverify_set_launch": (_i, [_vp, _i, _i, _i]),
     "specverify_get_launch": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i),
                                    ctypes.POINTER(_i)]),
+    "specverify_kernels_per_run": (_i, [_vp, _i, ctypes.POINTER(_i)]),
     "specverify_profile_begin": (_i, [_vp, _i]),
     "specverify_profile_end": (_i, [_vp, ctypes.POINTER(_f), ctypes.POINTER(_f), ctypes.POINTER(_i)]),
     "specverify_run_noalloc": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
@@ -179,6 +180,14 @@ def specverify_get_launch(h) -> tuple[int, int, int, int]:
     _check(_lib.specverify_get_launch(h, ctypes.byref(c), ctypes.byref(t), ctypes.byref(m),
                                       ctypes.byref(k)), "specverify_get_launch")
     return c.value, t.value, m.value, k.value
+
+
+def specverify_kernels_per_run(h, mapped: bool = False) -> int:
+    """Kernels one run of the handle enqueues."""
+    k = ctypes.c_int()
+    _check(_lib.specverify_kernels_per_run(h, 1 if mapped else 0, ctypes.byref(k)),
+           "specverify_kernels_per_run")
+    return k.value
 
 
 def specverify_profile_begin(h, max_runs: int) -> int:
@@ -477,6 +486,9 @@ class SpecVerify:
     def launch(self) -> tuple[int, int]:
         """(slices per position, threads per block)."""
         return specverify_get_launch(self.handle)[:2]
+
+    def kernels_per_run(self, mapped: bool = False) -> int:
+        return specverify_kernels_per_run(self.handle, mapped)
 
     def profile_begin(self, max_runs: int):
         specverify_profile_begin(self.handle, max_runs)
