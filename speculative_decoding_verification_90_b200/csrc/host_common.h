@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <cstddef>
 
@@ -37,5 +38,16 @@ class DeviceScope {
 };
 
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// An NVTX range around the host side of one entry point (the enqueue, not the
+// kernels' device time): named ranges in a profiler's timeline.  NVTX v3 is
+// header-only; without a profiler attached each push / pop is a no-op call.
+class NvtxRange {
+ public:
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 }  // namespace svhost

@@ -308,6 +308,7 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
                                 const void* draft_weight, const int32_t* draft_tokens,
                                 const float* u_accept, const float* u_resample, float temperature,
                                 int32_t* out_tokens, int32_t* out_num_accepted, void* stream) {
+  svhost::NvtxRange nvtx_range("specverify_lmhead_run");
   if (!h) return SV_ERR_INVALID_ARG;
   const int B = h->batch, G = h->gamma, V = h->vocab, D = h->hidden;
   if (!target_hidden || !target_weight || !u_resample || !out_tokens || !out_num_accepted)

@@ -16,9 +16,14 @@
 //     (the logits never reach global memory), or
 //   - writes the fp32 logits (the rows the draw needs).
 //
-// Every wait on an mbarrier is bounded: after kSpinLimit tries the thread sets
-// the error flag and leaves the loop, the kernel skips its remaining work, and
-// warp 1 still frees the tensor memory.
+// Every wait on an mbarrier is bounded in time (kWaitLimitNs of the global
+// nanosecond timer): a wait that runs out sets the CTA's failure flag and its
+// thread leaves its loop; the other roles see the flag and stop too.  Before
+// the tensor memory is freed, a failed CTA drains what it still has in
+// flight: the producer waits (bounded again) for every TMA load it issued
+// that the MMA thread had not consumed, and the MMA thread commits its last
+// MMAs to a drain barrier and waits for it (bounded).  Then warp 1 frees the
+// tensor memory and the error flag reaches the host.
 #pragma once
 
 #include <cuda.h>
@@ -39,7 +44,7 @@ constexpr int kABytes = kBM * kBK * 2;   // 16 KB
 constexpr int kBBytes = kBN * kBK * 2;   // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + room to align to 1024
-constexpr unsigned kSpinLimit = 1u << 20;  // tries per wait (well under a second)
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 enum : int { kModeStats = 0, kModeLogits = 1 };
 
@@ -84,10 +89,18 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, unsigned bytes) {
                : "memory");
 }
 
-// wait for the phase with the given parity to complete; false after the limit
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// wait for the phase with the given parity to complete; false once the wait
+// has lasted kWaitLimitNs (the timer is read every 256 tries)
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
   const uint32_t a = smem_u32(bar);
-  for (unsigned i = 0; i < kSpinLimit; ++i) {
+  unsigned long long t0 = 0;
+  for (unsigned i = 0;; ++i) {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -97,8 +110,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
         : "r"(a), "r"(parity)
         : "memory");
     if (done) return true;
+    if ((i & 255u) == 0u) {
+      const unsigned long long now = global_ns();
+      if (i == 0u) t0 = now;
+      else if (now - t0 > kWaitLimitNs) return false;
+    }
   }
-  return false;
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
@@ -253,8 +270,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
   __shared__ __align__(8) uint64_t empty_bar[kStages];
   __shared__ __align__(8) uint64_t tfull_bar[2];
   __shared__ __align__(8) uint64_t tempty_bar[2];
+  __shared__ __align__(8) uint64_t drain_bar;
   __shared__ uint32_t tmem_base_s;
   __shared__ int s_failed;
+  __shared__ long s_issued, s_consumed;  // TMA stage loads issued / waited for by the MMA thread
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x & 31;
   const int tiles1 = (P0.rows + kBM - 1) / kBM;
@@ -275,7 +294,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
       mbar_init(&tfull_bar[a], 1);
       mbar_init(&tempty_bar[a], 4);  // one arrival per epilogue warp
     }
+    mbar_init(&drain_bar, 1);
     s_failed = 0;
+    s_issued = 0;
+    s_consumed = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 1) {
@@ -307,6 +329,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
           mbar_expect_tx(&full_bar[s], kStageBytes);
           tma_load_2d(a, tm_a, &full_bar[s], kt * kBK, m0);
           tma_load_2d(a + kABytes, &tm_weight, &full_bar[s], kt * kBK, n0);
+          s_issued = it + 1;
         }
       }
     }
@@ -329,6 +352,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
             *failed = 1;
             break;
           }
+          s_consumed = it + 1;
           tc_fence_after();
           const uint32_t a = smem_u32(smem + s * kStageBytes);
           const uint32_t b = a + kABytes;
@@ -372,7 +396,21 @@ __global__ void __launch_bounds__(kPThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 0 && *failed) atomicOr(P0.error, 1u);
+  if (*failed) {  // uniform: the flag is read after the barrier
+    // drain before the shared memory and the tensor memory are given back:
+    // the TMA loads the MMA thread never waited for, then the MMAs issued
+    if (threadIdx.x == 0) {
+      for (long j = s_consumed; j < s_issued; ++j)
+        if (!mbar_wait(&full_bar[j % kStages], static_cast<unsigned>(j / kStages) & 1)) break;
+    }
+    if (warp == 1 && lane == 0) {
+      umma_commit(&drain_bar);
+      mbar_wait(&drain_bar, 0);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) atomicOr(P0.error, 1u);
+  }
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),

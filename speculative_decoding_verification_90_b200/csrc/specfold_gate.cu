@@ -178,6 +178,7 @@ sv_status specfold_gate_run(specfold_gate_t h, const void* hidden, const int32_t
                             float tau, float* rel_diff, int32_t* provenance, int32_t* source,
                             int32_t* packed_rows, int32_t* n_packed, void* packed_hidden,
                             void* stream) {
+  svhost::NvtxRange nvtx_range("specfold_gate_run");
   if (!h) return SV_ERR_INVALID_ARG;
   if (!hidden || !parent || !packed_rows || !n_packed) return SV_ERR_INVALID_ARG;
   if (std::isnan(tau) || !(tau >= 0.f)) return SV_ERR_INVALID_ARG;

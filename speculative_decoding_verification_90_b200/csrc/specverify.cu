@@ -392,6 +392,7 @@ sv_status specverify_run(specverify_t h, const void* target_logits, const void* 
                          const int32_t* draft_tokens, const float* u_accept,
                          const float* u_resample, float temperature, int32_t* out_tokens,
                          int32_t* out_num_accepted, void* stream) {
+  svhost::NvtxRange nvtx_range("specverify_run");
   if (!h) return SV_ERR_INVALID_ARG;
   if (h->batch == 0) return SV_OK;
   DeviceScope scope(h->device);
@@ -405,6 +406,7 @@ sv_status specverify_run_sampling(specverify_t h, const void* target_logits,
                                   const float* u_accept, const float* u_resample,
                                   const float* temperatures, int top_k, float top_p,
                                   int32_t* out_tokens, int32_t* out_num_accepted, void* stream) {
+  svhost::NvtxRange nvtx_range("specverify_run_sampling");
   if (!h) return SV_ERR_INVALID_ARG;
   if (h->batch == 0) return SV_OK;
   const int G = h->gamma;
@@ -496,6 +498,7 @@ sv_status specverify_run_mapped(specverify_t h, const void* target_rows, int n_t
                                 const int32_t* draft_tokens, const float* u_accept,
                                 const float* u_resample, float temperature, int32_t* out_tokens,
                                 int32_t* out_num_accepted, void* stream) {
+  svhost::NvtxRange nvtx_range("specverify_run_mapped");
   if (!h) return SV_ERR_INVALID_ARG;
   if (h->batch == 0) return SV_OK;
   const int G = h->gamma;
@@ -515,6 +518,7 @@ sv_status specverify_run_host(specverify_t h, const void* target_logits,
                               const void* draft_logits, const int32_t* draft_tokens,
                               const float* u_accept, const float* u_resample, float temperature,
                               int32_t* out_tokens, int32_t* out_num_accepted, void* stream) {
+  svhost::NvtxRange nvtx_range("specverify_run_host");
   if (!h) return SV_ERR_INVALID_ARG;
   if (h->batch == 0) return SV_OK;
   const int G = h->gamma;
@@ -789,6 +793,7 @@ extern "C" sv_status specverify_run_noalloc(int batch, int gamma, int vocab, sv_
                                             const float* u_resample, float temperature,
                                             int32_t* out_tokens, int32_t* out_num_accepted,
                                             void* stream) {
+  svhost::NvtxRange nvtx_range("specverify_run_noalloc");
   if (batch < 0 || gamma < 0 || gamma > specverify::kMaxGamma || vocab < 1 || vocab > (1 << 30))
     return SV_ERR_INVALID_ARG;
   if (dtype != SV_DTYPE_F32 && dtype != SV_DTYPE_BF16) return SV_ERR_INVALID_ARG;
