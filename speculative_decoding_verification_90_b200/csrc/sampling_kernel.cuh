@@ -927,6 +927,246 @@ __device__ __forceinline__ PassA pass_a(const T* row, int V, float c_hi, float c
   return a;
 }
 
+// ---------------------------------------------------------------------------
+// bf16 rows: the cuts in one scan, over exact values
+// ---------------------------------------------------------------------------
+//
+// A bf16 logit takes one of at most 65536 values, and the entries near the
+// row maximum hold the mass that top-k and top-p cut.  One scan counts, per
+// value, the entries of every value in a window of kXBins consecutive bf16
+// values (counts in shared memory), placed from a sample of the row: kXAbove
+// values above the sample's maximum, the rest below it.  Entries below the
+// window only add to a per-thread fp32 mass (a nucleus cut alone needs the
+// row's total); an entry above it means the sample missed the maximum by
+// more than the window allows, and the row takes the general path.  After
+// the scan every value of the window has an exact count, so its mass
+// count * 2^(x c - od) is exact in fp64, and the cuts are walks over the
+// window from the largest value down: the k-th largest value (cumulative
+// counts), then the first value whose cumulative mass reaches top_p of the
+// kept set's mass (or the row's): the walk over distinct values, ties
+// included, that defines the cut.  A cut that would fall below the window
+// takes the general path too, and so does a row holding NaN or +inf (an
+// entry above the window) or no entry in the window (the general path also
+// reports the invalid rows).  The row maximum is the largest value with a
+// count; the first argmax is not needed (only greedy rows use it, and they do
+// not come here).
+
+constexpr int kXBins = 4096;                   // values in the window (16 KB of counts)
+constexpr int kXAbove = 1024;                  // of which above the sample's maximum
+constexpr int kXPer = kXBins / kSelThreads;    // window values per thread in the walks
+constexpr unsigned kKeyNegInf = 0x007fu;       // 16-bit key of -inf
+constexpr unsigned kKeyPosInf = 0xff80u;       // 16-bit key of +inf (NaN keys lie outside both)
+
+// order-preserving 16-bit key of a bf16 value (its bits in the low half of h):
+// the top half of fkey of the value widened to float
+__device__ __forceinline__ unsigned bf16_key(unsigned h) {
+  return (h & 0x8000u) ? (~h & 0xffffu) : (h | 0x8000u);
+}
+__device__ __forceinline__ float key16_value(unsigned k) {
+  const unsigned h = (k & 0x8000u) ? (k & 0x7fffu) : (~k & 0xffffu);
+  return __uint_as_float(h << 16);
+}
+
+struct XState {
+  bool off = false;  // an entry above the window, NaN or +inf: the general path takes the row
+  float tail = 0.f;  // kTail: sum 2^(x c - o) below the window
+};
+
+// One 32-bit word of two bf16 entries, branch-free: both keys in one register
+// (each half h -> h ^ 0x8000 for a positive value, ~h for a negative one);
+// a key in the window [klo, klo + span] adds 1 to its count (a predicated
+// shared atomic at index key - klo); one unsigned compare flags a key above
+// the window, +inf or NaN of either sign; the mass below the window is an ex2
+// of -inf where it does not apply.
+template <bool kTail>
+__device__ __forceinline__ void x_word(unsigned w, unsigned klo, unsigned span, unsigned top,
+                                       unsigned* hist, float c_hi, float c_lo, float o,
+                                       XState& st) {
+  const unsigned neg = (w >> 15) & 0x00010001u;              // sign of each half
+  const unsigned k2 = w ^ (0x80008000u | (neg * 0x7fffu));   // both keys
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const unsigned k = half ? (k2 >> 16) : (k2 & 0xffffu);
+    const unsigned i = k - klo;
+    const bool in = i <= span;
+    if (in) atomicAdd(hist + i, 1u);
+    st.off |= (k - kKeyNegInf) > top;  // top = window top - key(-inf)
+    if constexpr (kTail) {
+      const float x = __uint_as_float(half ? (w & 0xffff0000u) : (w << 16));
+      st.tail += ex2(in ? -INFINITY : specverify::arg2(x, c_hi, c_lo, o));
+    }
+  }
+}
+
+// Returns true when the row's adjusted distribution is settled (and written),
+// false when the general path must take the row.  Every thread of the block
+// calls it and gets the same answer.
+template <bool kTail>
+__device__ bool exact_select(const SampParams& P, long r, long nT, const __nv_bfloat16* row, int V,
+                             float c_hi, float c_lo, double c, bool use_k, bool use_p,
+                             unsigned* hist) {
+  __shared__ double smd[kSelWarps];
+  __shared__ unsigned smu[kSelWarps];
+  __shared__ int s_cut;        // window value of the cut (-1: the general path)
+  __shared__ double s_zcut;    // mass through it
+  __shared__ double s_ncut;    // entries through it
+  __shared__ float s_margin;
+  const int tid = threadIdx.x;
+  const long groups = V / 8;
+  const uint4* g4 = reinterpret_cast<const uint4*>(row);
+
+  // the window: from the largest finite key among the row's first kSelThreads groups
+  unsigned ks = 0u;
+  if (tid < groups) {
+    const uint4 v = __ldg(g4 + tid);
+    const unsigned w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const unsigned k0 = bf16_key(w[q] & 0xffffu), k1 = bf16_key(w[q] >> 16);
+      if (k0 < kKeyPosInf) ks = max(ks, k0);
+      if (k1 < kKeyPosInf) ks = max(ks, k1);
+    }
+  }
+  for (int i = tid; i < kXBins; i += kSelThreads) hist[i] = 0u;
+  ks = block_max_u<kSelThreads>(ks, smu);  // (barriers inside: hist is clear after it)
+  if (ks <= kKeyNegInf) ks = 0x8000u;      // no finite entry sampled: centre on 0
+  const int khi = min(static_cast<int>(ks) + kXAbove, static_cast<int>(kKeyPosInf) - 1);
+  // the window: keys klo .. khi (never the key of -inf); count index = key - klo
+  const int klo = max(khi - kXBins + 1, static_cast<int>(kKeyNegInf) + 1);
+  const unsigned span = static_cast<unsigned>(khi - klo);
+  const unsigned top = static_cast<unsigned>(khi) - kKeyNegInf;
+  const float o = key16_value(ks) * c_hi;  // weights of the entries below the window
+
+  XState st;
+  {
+    constexpr int kU = 4;
+    const long stride = static_cast<long>(kSelThreads) * kU;
+    for (long g0 = tid; g0 < groups; g0 += stride) {
+      uint4 v[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const long g = g0 + static_cast<long>(u) * kSelThreads;
+        if (g < groups) v[u] = __ldg(g4 + g);
+      }
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const long g = g0 + static_cast<long>(u) * kSelThreads;
+        if (g >= groups) break;
+        x_word<kTail>(v[u].x, static_cast<unsigned>(klo), span, top, hist, c_hi, c_lo, o, st);
+        x_word<kTail>(v[u].y, static_cast<unsigned>(klo), span, top, hist, c_hi, c_lo, o, st);
+        x_word<kTail>(v[u].z, static_cast<unsigned>(klo), span, top, hist, c_hi, c_lo, o, st);
+        x_word<kTail>(v[u].w, static_cast<unsigned>(klo), span, top, hist, c_hi, c_lo, o, st);
+      }
+    }
+  }
+  // rows with an entry above the window, NaN or +inf go to the general path
+  // (which also reports the invalid ones)
+  if (__syncthreads_or(st.off)) return false;
+  const double tail_o = kTail ? block_sum<kSelThreads>(static_cast<double>(st.tail), smd) : 0.0;
+  // the window in descending order: rank q = khi - key, count hist[span - q]
+  // (ranks past span lie below the window: no count); the row maximum is the
+  // first rank with a count (none: every entry is below the window or -inf,
+  // and the general path takes the row)
+  const int b0 = tid * kXPer;
+  auto count_at = [&](int q) -> unsigned {
+    return q <= static_cast<int>(span) ? hist[static_cast<int>(span) - q] : 0u;
+  };
+  unsigned first = 0xffffffffu;
+  for (int i = kXPer - 1; i >= 0; --i)
+    if (count_at(b0 + i)) first = static_cast<unsigned>(b0 + i);
+  first = 0xffffffffu - block_max_u<kSelThreads>(0xffffffffu - first, smu);
+  if (first == 0xffffffffu) return false;
+  const unsigned kmax = static_cast<unsigned>(khi) - first;
+  SampRow out{0.0, 0u, -1, 1, V, INFINITY, 0};
+
+  // exact masses of the window's values, relative to the maximum
+  const double od = static_cast<double>(key16_value(kmax)) * c;
+  double cnt_t = 0.0, mass_t = 0.0;
+#pragma unroll 4
+  for (int i = 0; i < kXPer; ++i) {
+    const unsigned n = count_at(b0 + i);
+    if (n) {
+      const double x = key16_value(static_cast<unsigned>(khi - (b0 + i)));
+      cnt_t += n;
+      mass_t += n * exp2(x * c - od);
+    }
+  }
+  double c_in, c_ex, c_tot, m_in, m_ex, m_tot;
+  specverify::block_scan<kSelThreads>(cnt_t, c_in, c_ex, c_tot);
+  specverify::block_scan<kSelThreads>(mass_t, m_in, m_ex, m_tot);
+  if (tid == 0) {
+    s_cut = -1;
+    s_margin = INFINITY;
+  }
+  __syncthreads();
+  // top-k: the window value where the cumulative count reaches k
+  int kcut = kXBins - 1;
+  double zk = m_tot;
+  if (use_k) {
+    const double k = static_cast<double>(P.top_k);
+    if (c_ex < k && k <= c_in) {
+      double cc = c_ex, mm = m_ex;
+      for (int i = 0; i < kXPer; ++i) {
+        const unsigned n = count_at(b0 + i);
+        if (!n) continue;
+        cc += n;
+        mm += n * exp2(static_cast<double>(key16_value(static_cast<unsigned>(khi - (b0 + i)))) * c - od);
+        if (cc >= k) {
+          s_cut = b0 + i;
+          s_zcut = mm;
+          s_ncut = cc;
+          break;
+        }
+      }
+    }
+    __syncthreads();
+    if (s_cut < 0) return false;  // the k-th largest lies below the window
+    kcut = s_cut;
+    zk = s_zcut;
+  }
+  if (use_p) {
+    // the row's mass (nucleus alone, with the entries below the window) or
+    // the top-k set's; the first window value whose cumulative mass, divided
+    // by it, reaches top_p, and never past the top-k cut
+    const double Z = use_k ? zk : m_tot + tail_o * exp2(static_cast<double>(o) - od);
+    const double tp = P.top_p;
+    __syncthreads();
+    if (tid == 0) s_cut = -1;
+    __syncthreads();
+    const bool mine = b0 <= kcut && (m_ex / Z < tp || b0 == 0) &&
+                      (m_in / Z >= tp || (b0 <= kcut && kcut < b0 + kXPer));
+    if (mine) {
+      double cc = c_ex, mm = m_ex;
+      for (int i = 0; i < kXPer && b0 + i <= kcut; ++i) {
+        const unsigned n = count_at(b0 + i);
+        if (!n) continue;
+        const double before = mm;
+        cc += n;
+        mm += n * exp2(static_cast<double>(key16_value(static_cast<unsigned>(khi - (b0 + i)))) * c - od);
+        if (mm / Z >= tp || b0 + i == kcut) {
+          if (atomicCAS(&s_cut, -1, b0 + i) == -1) {
+            s_zcut = mm;
+            s_ncut = cc;
+            s_margin = static_cast<float>(fmin(tp - before / Z, mm / Z - tp));
+          }
+          break;
+        }
+      }
+    }
+    __syncthreads();
+    if (s_cut < 0) return false;  // the nucleus reaches below the window
+  }
+  if (tid == 0) {
+    const int cut = s_cut;
+    out.theta = fkey(key16_value(static_cast<unsigned>(khi - cut)));
+    out.l2 = od + log2(s_zcut);
+    out.kept = static_cast<int>(s_ncut);
+    out.margin = s_margin;
+    put_row(P, r, nT, out);
+  }
+  return true;
+}
+
 template <typename T, bool kAligned>
 __global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams P) {
   __shared__ double smd[kSelWarps];
@@ -952,6 +1192,25 @@ __global__ void __launch_bounds__(kSelThreads, 4) select_kernel(const SampParams
   const float temp = P.temperature[b];
   const int low_bits = sizeof(T) == 2 ? 16 : 0;
   const unsigned step = 1u << low_bits;
+
+  // bf16 rows with a filter: the one-scan cut over exact values first
+  if constexpr (sizeof(T) == 2 && kAligned) {
+    const bool filter = (P.top_k > 0 && P.top_k < V) || P.top_p < 1.0;
+    // (a top-k cut of at most kSelThreads keeps the per-thread lists below:
+    // one lighter scan settles it)
+    const bool lists = P.top_k > 0 && P.top_k <= kSelThreads && P.top_k < V;
+    if (filter && !lists && temp > 0.f && temp_ok(temp)) {
+      float xc_hi, xc_lo;
+      double xc;
+      temp_consts(temp, xc_hi, xc_lo, xc);
+      const bool uk = P.top_k > 0 && P.top_k < V, up = P.top_p < 1.0;
+      const bool done =
+          (up && !uk) ? exact_select<true>(P, r, nT, row, V, xc_hi, xc_lo, xc, uk, up, cand_smem)
+                      : exact_select<false>(P, r, nT, row, V, xc_hi, xc_lo, xc, uk, up, cand_smem);
+      if (done) return;
+      __syncthreads();  // the general path reuses the candidate area
+    }
+  }
 
   // pass A: maximum, first argmax, invalid entries, and (for a top-k cut)
   // each thread's four largest values
