@@ -242,10 +242,11 @@ sv_status specverify_lmhead_create(specverify_lmhead_t* out, int batch, int gamm
   const size_t oR = take(nB * sizeof(double));
   const size_t oS = take(sizeof(unsigned));
   const size_t oE = take(sizeof(unsigned));
-  const size_t oXT = take(nB * hidden * 2);
-  const size_t oXD = take(nB * hidden * 2);
-  const size_t oLT = take(nB * static_cast<size_t>(vocab) * 4);
-  const size_t oLD = take(nB * static_cast<size_t>(vocab) * 4);
+  // the drawn rows: the B target rows then the B draft rows, contiguous, so
+  // that with one output layer a single GEMM tile holds both rows of a
+  // sequence pair (hidden states bf16, logits fp32)
+  const size_t oXT = take(2 * nB * hidden * 2);
+  const size_t oLT = take(2 * nB * static_cast<size_t>(vocab) * 4);
   e = cudaMalloc(&h->ws, off);
   if (e != cudaSuccess) {
     delete h;
@@ -265,9 +266,9 @@ sv_status specverify_lmhead_create(specverify_lmhead_t* out, int batch, int gamm
   h->status = reinterpret_cast<unsigned*>(b + oS);
   h->gemm_error = reinterpret_cast<unsigned*>(b + oE);
   h->xt = reinterpret_cast<__nv_bfloat16*>(b + oXT);
-  h->xd = reinterpret_cast<__nv_bfloat16*>(b + oXD);
+  h->xd = h->xt + nB * hidden;
   h->lt = reinterpret_cast<float*>(b + oLT);
-  h->ld = reinterpret_cast<float*>(b + oLD);
+  h->ld = h->lt + nB * static_cast<size_t>(vocab);
   e = cudaMemset(h->ws, 0, off);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
@@ -329,10 +330,11 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   split_c(temperature, c_hi, c_lo, c);
   if (!(c < 1e30)) return SV_ERR_INVALID_ARG;
 
-  CUtensorMap mht, mwt, mhd, mwd, mxt, mxd;
+  CUtensorMap mht, mwt, mhd, mwd, mxt, mxd, mx2;
   if (!make_map(&mht, target_hidden, nT, D, lmhead::kBM) ||
       !make_map(&mwt, target_weight, V, D, lmhead::kBN) ||
-      !make_map(&mxt, h->xt, B, D, lmhead::kBM))
+      !make_map(&mxt, h->xt, B, D, lmhead::kBM) ||
+      !make_map(&mx2, h->xt, 2L * B, D, lmhead::kBM))
     return SV_ERR_INVALID_ARG;
   if (G > 0 && (!make_map(&mhd, draft_hidden, nD, D, lmhead::kBM) ||
                 !make_map(&mwd, draft_weight, V, D, lmhead::kBN) ||
@@ -437,10 +439,11 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   l.error = h->gemm_error;
   l.logits = h->lt;
   if (G > 0 && draft_weight == target_weight) {
-    // one output layer: both drawn rows of every sequence in one launch
-    l.rows2 = B;
-    l.logits2 = h->ld;
-    if (e == cudaSuccess) e = launch_gemm<lmhead::kModeLogits>(mxt, mxd, mwt, l, s);
+    // one output layer: the 2B drawn rows (target rows, then draft rows, one
+    // tensor) as one GEMM, so each weight tile is read once for both
+    l.rows = 2 * B;
+    l.rows2 = 0;
+    if (e == cudaSuccess) e = launch_gemm<lmhead::kModeLogits>(mx2, mx2, mwt, l, s);
   } else {
     if (e == cudaSuccess) e = launch_gemm<lmhead::kModeLogits>(mxt, mxt, mwt, l, s);
     if (G > 0) {

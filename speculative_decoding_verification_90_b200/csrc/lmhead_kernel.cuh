@@ -230,15 +230,24 @@ __device__ __forceinline__ void epilogue_tile(const LmParams& P, uint32_t acc_ad
       if (t >= n0 && t < n0 + kBN) P.gathered[P.row_offset + r] = xt;
     }
   } else {
+    // 16-byte stores when the row's 32 columns are 16-byte aligned and inside
+    // the vocabulary (every full tile of a vocabulary that is a multiple of 4)
+    const bool vec = (P.vocab % 4) == 0;
 #pragma unroll 1
     for (int c0 = 0; c0 < kBN; c0 += 32) {
       float v[32];
       tmem_ld32(lane_addr + c0, v);
       if (r < P.rows) {
         float* out = P.logits + static_cast<long>(r) * P.vocab + n0 + c0;
+        if (vec && n0 + c0 + 32 <= P.vocab) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-          if (n0 + c0 + i < P.vocab) out[i] = v[i];
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(out + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (n0 + c0 + i < P.vocab) out[i] = v[i];
+        }
       }
     }
   }
