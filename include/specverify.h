@@ -82,7 +82,7 @@ typedef enum {
   SV_ERR_ROW_INDEX = 19,   /* device: a row map entry was outside the rows given */
   SV_ERR_PARENT = 20,      /* device (fold gate): a parent entry out of range, a self link or a cycle */
   SV_ERR_TEMPERATURE = 21, /* device (sampling variants): a temperature < 0, NaN or infinite */
-  SV_ERR_PIPELINE = 22     /* device (fused LM head): a tensor-core pipeline wait gave up */
+  SV_ERR_PIPELINE = 22     /* device: a bounded wait gave up (LM-head pipeline, single-launch step) */
 } sv_status;
 
 /*
@@ -251,16 +251,46 @@ sv_status specverify_get_launch(specverify_t h, int *slices, int *threads, int *
 
 /*
  * Number of kernels one run of the handle enqueues (`mapped` nonzero: a run
- * of specverify_run_mapped): statistics, decide and draw; none for an empty
- * batch.
+ * of specverify_run_mapped): statistics, decide and draw; one for an aligned
+ * unmapped run in the single-launch form (specverify_set_fused); none for an
+ * empty batch.
  */
 sv_status specverify_kernels_per_run(specverify_t h, int mapped, int *kernels);
 
 /*
+ * Single-launch form of the step (default off).  With `enable` nonzero, a run
+ * of specverify_run (or specverify_run_host) whose logit pointers are 16-byte
+ * aligned with vocab * sizeof(dtype) a multiple of 16 is one persistent
+ * kernel: its warps take statistics units (runs of `unit_groups` 16-byte
+ * groups of one row, 128 .. 2^20, with at most `max_slices` units per row;
+ * 0 picks 1024) and draw chunks (`chunk_tiles` tiles of 64 groups of the
+ * rows drawn from; 0 picks 8) from one ordered list, sequence by sequence,
+ * the draw chunks of a sequence `lag` sequences after its statistics (-1
+ * derives it from the grid).  The warp that finishes a sequence's statistics
+ * decides it; the rows drawn from are then re-read from L2 while later
+ * sequences stream.  Results equal the three-kernel form's up to the rounding
+ * of partial sums.  Waits between warps are bounded; one that runs out (it
+ * never should) makes specverify_get_status return SV_ERR_PIPELINE and reset
+ * the form's control words.  `enable` zero: three kernels (statistics,
+ * decide, draw) as for unaligned or mapped runs.  Invalid values return
+ * SV_ERR_INVALID_ARG.  Not stream-ordered: change it only while no run of
+ * the handle is in flight.
+ */
+sv_status specverify_set_fused(specverify_t h, int enable, int unit_groups, int chunk_tiles,
+                               int lag);
+
+/* Whether an aligned unmapped run takes the single launch, and its shape
+ * (the lag as derived); any pointer may be NULL. */
+sv_status specverify_get_fused(specverify_t h, int *enabled, int *unit_groups, int *chunk_tiles,
+                               int *lag);
+
+/*
  * Per-kernel timing of the next `max_runs` runs of the handle: each run then
  * records CUDA events on its stream around its two kernels (the statistics
- * kernel, which streams every logit, and the decide-and-draw kernel).  Waits
- * for the device first; re-arming discards earlier records.
+ * kernel, which streams every logit, and the decide-and-draw kernel; a
+ * single-launch run records its one kernel as the statistics time and zero
+ * for the other).  Waits for the device first; re-arming discards earlier
+ * records.
  */
 sv_status specverify_profile_begin(specverify_t h, int max_runs);
 

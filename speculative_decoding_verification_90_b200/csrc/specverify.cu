@@ -15,6 +15,7 @@
 #include <new>
 #include <vector>
 
+#include "fused_kernel.cuh"
 #include "host_common.h"
 #include "sampling_kernel.cuh"
 #include "verify_kernel.cuh"
@@ -44,6 +45,14 @@ struct specverify_ctx {
   double* resid = nullptr;
   unsigned* status = nullptr;
   specsamp::SampRow* samp_rows = nullptr;          // sampling variants: per-row filter
+  // single-launch step (fused_kernel): used for 16-byte aligned, unmapped
+  // runs when `fused` is set; its own partial table and control words
+  int fused = 0;  // off by default (specverify_set_fused)
+  int fused_unit_groups = 1024;  // 16-byte groups per statistics unit
+  int fused_chunk_tiles = 8;     // mass-table tiles per draw chunk
+  int fused_lag = -1;            // sequences between statistics and draw (-1: derived)
+  int fused_blocks_per_sm = 0;   // resident blocks of fused_kernel per SM
+  unsigned* fctl = nullptr;      // task counter, exit count, then 3 words per sequence
   specsamp::SampDecision* samp_decision = nullptr; // sampling variants: per sequence
   void* stage = nullptr;  // device staging for host-buffer runs
   size_t stage_bytes = 0;
@@ -200,6 +209,56 @@ cudaError_t launch_sampling(const specsamp::SampParams& p, long rows, int per, c
   return e;
 }
 
+// The single-launch step's task layout for this handle's batch.
+specverify::FusedShape fused_shape_of(const specverify_ctx* h) {
+  const long warps = static_cast<long>(h->num_sms) * h->fused_blocks_per_sm * specverify::kFusedWarps;
+  return specverify::fused_shape(h->batch, h->gamma, num_groups(h), draw_tiles(h),
+                                 h->fused_unit_groups, h->fused_chunk_tiles, h->fused_lag, warps);
+}
+
+// Whether an (aligned) run of the handle takes the single launch: the fused
+// mode is on, the rows are not mapped, and the task list fits its counters.
+bool use_fused(const specverify_ctx* h, const int32_t* target_map) {
+  if (!h->fused || target_map || !h->fctl || h->fused_blocks_per_sm < 1) return false;
+  const specverify::FusedShape fs = fused_shape_of(h);
+  return fs.units_per_row <= h->max_slices && fs.total_tasks < (1L << 31);
+}
+
+// The single-launch step.  events (may be null): [0] before, [1] and [2]
+// after the kernel (the whole step is reported as the statistics time).
+template <typename T>
+cudaError_t launch_fused(const specverify_ctx* h, Params p, cudaStream_t s, cudaEvent_t* ev) {
+  const specverify::FusedShape fs = fused_shape_of(h);
+  p.slices = fs.units_per_row;  // the partial table holds max_slices >= this per row
+  specverify::FusedParams f;
+  f.task_next = h->fctl;
+  f.exit_count = h->fctl + 1;
+  f.stats_done = h->fctl + 2;
+  f.ready = h->fctl + 2 + h->batch;
+  f.draw_done = h->fctl + 2 + 2L * h->batch;
+  f.total_tasks = static_cast<unsigned>(fs.total_tasks);
+  f.units_per_row = fs.units_per_row;
+  f.groups_per_unit = fs.groups_per_unit;
+  f.units_per_seq = fs.units_per_seq;
+  f.chunk_tiles = fs.chunk_tiles;
+  f.chunks_per_seq = fs.chunks_per_seq;
+  f.lag = fs.lag;
+  long blocks = static_cast<long>(h->num_sms) * h->fused_blocks_per_sm;
+  const long need = (fs.total_tasks + specverify::kFusedWarps - 1) / specverify::kFusedWarps;
+  if (blocks > need) blocks = need;
+  if (blocks < 1) blocks = 1;
+  f.total_warps = static_cast<unsigned>(blocks * specverify::kFusedWarps);
+  cudaError_t e = cudaSuccess;
+  if (ev) e = cudaEventRecord(ev[0], s);
+  if (e != cudaSuccess) return e;
+  specverify::fused_kernel<T><<<static_cast<unsigned>(blocks), specverify::kFusedThreads,
+                                specverify::kFusedSmem, s>>>(p, f);
+  e = cudaGetLastError();
+  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
+  if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
+  return e;
+}
+
 // Row maps null: the logit buffers hold one row per position, [B, G+1, V] and
 // [B, G, V].  Otherwise `target_rows` / `draft_rows` rows that the maps index.
 // Every argument check of a verification call: null and alignment tests,
@@ -285,6 +344,13 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
                        (static_cast<size_t>(h->vocab) * es) % 16 == 0;
   cudaEvent_t* ev = nullptr;
   if (h->prof_runs < h->prof_capacity) ev = h->events.data() + 3 * (h->prof_runs++);
+  if (aligned && use_fused(h, target_map)) {
+    const cudaError_t fe = (h->dtype == SV_DTYPE_BF16)
+                               ? launch_fused<__nv_bfloat16>(h, p, stream, ev)
+                               : launch_fused<float>(h, p, stream, ev);
+    if (fe != cudaSuccess) return cuda_fail(fe);
+    return SV_OK;
+  }
   cudaError_t e = (h->dtype == SV_DTYPE_BF16)
                       ? launch_dtype<__nv_bfloat16>(p, h->threads, nd, aligned, stream, ev)
                       : launch_dtype<float>(p, h->threads, nd, aligned, stream, ev);
@@ -359,6 +425,7 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   const size_t offS = take(sizeof(unsigned));
   const size_t offSR = take((nT + nD) * sizeof(specsamp::SampRow));
   const size_t offSD = take(nB * sizeof(specsamp::SampDecision));
+  const size_t offF = take((2 + 3 * nB) * sizeof(unsigned));
   const size_t total = off;
   e = cudaMalloc(&h->ws, total);
   if (e != cudaSuccess) {
@@ -377,6 +444,28 @@ sv_status specverify_create(specverify_t* out, int batch, int gamma, int vocab, 
   h->status = reinterpret_cast<unsigned*>(base + offS);
   h->samp_rows = reinterpret_cast<specsamp::SampRow*>(base + offSR);
   h->samp_decision = reinterpret_cast<specsamp::SampDecision*>(base + offSD);
+  h->fctl = reinterpret_cast<unsigned*>(base + offF);
+  {
+    // resident blocks of the single-launch kernel (its grid is one wave)
+    int nb = 0;
+    e = (dtype == SV_DTYPE_BF16)
+            ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                  &nb, specverify::fused_kernel<__nv_bfloat16>, specverify::kFusedThreads,
+                  specverify::kFusedSmem)
+            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                  &nb, specverify::fused_kernel<float>, specverify::kFusedThreads,
+                  specverify::kFusedSmem);
+    if (e != cudaSuccess) {
+      cudaFree(h->ws);
+      delete h;
+      return cuda_fail(e);
+    }
+    h->fused_blocks_per_sm = nb;
+    h->fused = 0;  // opt-in: the three kernels are faster on every measured batch
+    long ug = 1024;
+    while ((num_groups(h) + ug - 1) / ug > h->max_slices) ug *= 2;
+    h->fused_unit_groups = static_cast<int>(ug);
+  }
   e = cudaMemset(h->ws, 0, total);
   if (e == cudaSuccess) e = cudaDeviceSynchronize();
   if (e != cudaSuccess) {
@@ -597,6 +686,14 @@ sv_status specverify_get_status(specverify_t h, void* stream, uint32_t* bits) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (bits) *bits = v;
+  if (v & specverify::kStatWait) {
+    // a wait of the single launch ran out: its control words may be left
+    // nonzero; clear them so that the next run starts clean
+    e = cudaMemsetAsync(h->fctl, 0, (2 + 3 * static_cast<size_t>(h->batch)) * sizeof(unsigned), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return SV_ERR_PIPELINE;
+  }
   if (v & specverify::kStatRowIndex) return SV_ERR_ROW_INDEX;
   if (v & specsamp::kStatTemperature) return SV_ERR_TEMPERATURE;
   if (v & specverify::kStatTokenRange) return SV_ERR_TOKEN_RANGE;
@@ -660,8 +757,46 @@ sv_status specverify_get_launch(specverify_t h, int* slices, int* threads, int* 
 
 sv_status specverify_kernels_per_run(specverify_t h, int mapped, int* kernels) {
   if (!h || !kernels) return SV_ERR_INVALID_ARG;
-  (void)mapped;  // the mapped form launches the same kernels
-  *kernels = h->batch == 0 ? 0 : 3;  // statistics, decide, draw
+  // statistics, decide, draw; one launch for an unmapped run in fused mode
+  // (the count for 16-byte aligned logits with vocab * sizeof(dtype) a
+  // multiple of 16)
+  if (h->batch == 0) *kernels = 0;
+  else *kernels = (!mapped && use_fused(h, nullptr)) ? 1 : 3;
+  return SV_OK;
+}
+
+sv_status specverify_set_fused(specverify_t h, int enable, int unit_groups, int chunk_tiles,
+                               int lag) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  if (unit_groups != 0) {
+    if (unit_groups < 128 || unit_groups > (1 << 20)) return SV_ERR_INVALID_ARG;
+    const long nu = (num_groups(h) + unit_groups - 1) / unit_groups;
+    if (nu > h->max_slices) return SV_ERR_INVALID_ARG;
+  }
+  if (chunk_tiles < 0 || chunk_tiles > 4096) return SV_ERR_INVALID_ARG;
+  if (lag < -1) return SV_ERR_INVALID_ARG;
+  if (enable && h->fused_blocks_per_sm < 1) return SV_ERR_UNSUPPORTED;
+  h->fused = enable ? 1 : 0;
+  if (unit_groups != 0) h->fused_unit_groups = unit_groups;
+  else {
+    // default: 1024 groups (16 KB), fewer units if the table has no room
+    long ug = 1024;
+    while ((num_groups(h) + ug - 1) / ug > h->max_slices) ug *= 2;
+    h->fused_unit_groups = static_cast<int>(ug);
+  }
+  h->fused_chunk_tiles = chunk_tiles ? chunk_tiles : 8;
+  h->fused_lag = lag;
+  return SV_OK;
+}
+
+sv_status specverify_get_fused(specverify_t h, int* enabled, int* unit_groups, int* chunk_tiles,
+                               int* lag) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  const specverify::FusedShape fs = fused_shape_of(h);
+  if (enabled) *enabled = use_fused(h, nullptr) ? 1 : 0;
+  if (unit_groups) *unit_groups = h->fused_unit_groups;
+  if (chunk_tiles) *chunk_tiles = h->fused_chunk_tiles;
+  if (lag) *lag = fs.lag;
   return SV_OK;
 }
 
@@ -724,7 +859,7 @@ const char* specverify_status_string(sv_status s) {
     case SV_ERR_ROW_INDEX: return "row map entry outside the logit rows given";
     case SV_ERR_PARENT: return "parent index out of range, self link or cycle";
     case SV_ERR_TEMPERATURE: return "temperature negative, NaN or infinite";
-    case SV_ERR_PIPELINE: return "a tensor-core pipeline wait gave up";
+    case SV_ERR_PIPELINE: return "a bounded device wait gave up (tensor-core pipeline or single-launch step)";
   }
   return "unknown status";
 }

@@ -57,7 +57,15 @@ constexpr int kMaxSlices = 64;
 // per-position decision flags
 enum : int { kFlagReject = 0, kFlagAccept = 1, kFlagTokenRange = 2, kFlagNonFinite = 3 };
 // status word bits
-enum : unsigned { kStatTokenRange = 1u, kStatNonFinite = 2u, kStatZeroMass = 4u, kStatRowIndex = 8u };
+// (16 is the sampling variants' temperature bit; 32: a bounded wait of the
+// single-launch step gave up)
+enum : unsigned {
+  kStatTokenRange = 1u,
+  kStatNonFinite = 2u,
+  kStatZeroMass = 4u,
+  kStatRowIndex = 8u,
+  kStatWait = 32u
+};
 // what the draw kernel draws from
 enum : int { kDrawResidual = 0, kDrawTarget = 1, kDrawNone = 2 };
 
@@ -425,14 +433,17 @@ constexpr int kDecideThreads = 128;
 constexpr int kMaxGamma = 255;
 
 // (o, s) partials of one row combined in two passes, so that the fp64
-// exponentials of the second pass are independent of one another
+// exponentials of the second pass are independent of one another.  kCg: the
+// partials were written by other warps of the same launch, so they are read
+// through L2 (ld.global.cg), never from a possibly stale L1 line.
+template <bool kCg>
 __device__ __forceinline__ double row_lse2(const RowPartial* parts, int S, int& valid) {
   float O = -INFINITY;
-  for (int r = 0; r < S; ++r) O = fmaxf(O, parts[r].o);
+  for (int r = 0; r < S; ++r) O = fmaxf(O, kCg ? __ldcg(&parts[r].o) : parts[r].o);
   double sum = 0.0;
   for (int r = 0; r < S; ++r) {
-    const float o = parts[r].o;
-    const double s = parts[r].s;
+    const float o = kCg ? __ldcg(&parts[r].o) : parts[r].o;
+    const double s = kCg ? __ldcg(&parts[r].s) : parts[r].s;
     sum += (o == -INFINITY) ? s * 0.0 : s * exp2(static_cast<double>(o) - O);  // NaN survives
   }
   valid = (O != -INFINITY) && isfinite(sum) && sum > 0.0;
@@ -444,8 +455,12 @@ __device__ __forceinline__ double row_lse2(const RowPartial* parts, int S, int& 
 // in fp64 and tests u < ratio (step 2); a warp ballot finds the first
 // rejection n (step 3).  Writes the accepted prefix, the padding, the count,
 // the per-position readback records and what the draw kernel draws from.
-template <typename T>
-__device__ __forceinline__ void decide_sequence(const Params& P, int b) {
+// kCg: the partials come from other warps of the same launch (see row_lse2).
+// staged (unmapped rows only): the sequence's partials were copied to shared
+// memory, its gamma+1 target rows then its gamma draft rows, S per row.
+template <typename T, bool kCg = false>
+__device__ __forceinline__ void decide_sequence(const Params& P, int b,
+                                                const RowPartial* staged = nullptr) {
   const int lane = threadIdx.x & (kWarp - 1);
   const int G = P.gamma, V = P.vocab, S = P.slices;
   const double c = P.c;
@@ -483,8 +498,13 @@ __device__ __forceinline__ void decide_sequence(const Params& P, int b) {
       }
       int validT = 0, validD = 1;
       if (!map_bad) {
-        lT = row_lse2(P.partial + tr * S, S, validT);
-        if (has_draft) lD = row_lse2(P.partial + (P.target_rows + dr) * S, S, validD);
+        if (staged) {
+          lT = row_lse2<false>(staged + static_cast<long>(j) * S, S, validT);
+          if (has_draft) lD = row_lse2<false>(staged + static_cast<long>(G + 1 + j) * S, S, validD);
+        } else {
+          lT = row_lse2<kCg>(P.partial + tr * S, S, validT);
+          if (has_draft) lD = row_lse2<kCg>(P.partial + (P.target_rows + dr) * S, S, validD);
+        }
       }
       P.tstat[position] = RowStat{lT, validT, 0};
       if (has_draft) P.dstat[pj] = RowStat{lD, validD, 0};
@@ -806,11 +826,11 @@ __device__ __forceinline__ void issue_tile(uint4* slot, const uint4* rowT, const
 }
 
 // Masses of tiles [t0, t1) of one row (16-byte aligned rows) into table,
-// through the calling warp's ring: kStages - 1 tiles are in flight while one
-// is reduced.  Every iteration commits one copy group (possibly empty), so
-// waiting until at most kStages - 1 groups are pending means the oldest
-// tile has landed.  Returns with no copy in flight.
-template <typename T, int kMode>
+// through the calling warp's ring of NS stages: NS - 1 tiles are in flight
+// while one is reduced.  Every iteration commits one copy group (possibly
+// empty), so waiting until at most NS - 1 groups are pending means the
+// oldest tile has landed.  Returns with no copy in flight.
+template <typename T, int kMode, int NS = kStages>
 __device__ __forceinline__ void tile_masses_ring(const T* rowT, const T* rowD, const DrawConsts& k,
                                                  long t0, long t1, long ngroups, double* table,
                                                  uint4* ring) {
@@ -819,16 +839,16 @@ __device__ __forceinline__ void tile_masses_ring(const T* rowT, const T* rowD, c
   const uint4* gD = reinterpret_cast<const uint4*>(rowD);
   const long n = t1 - t0;
 #pragma unroll
-  for (int i = 0; i < kStages - 1; ++i) {
+  for (int i = 0; i < NS - 1; ++i) {
     if (i < n) issue_tile<kMode>(ring + i * kStageU4, gT, gD, t0 + i, ngroups);
     cp_async_commit();
   }
   for (long i = 0; i < n; ++i) {
-    const long nx = i + kStages - 1;
-    if (nx < n) issue_tile<kMode>(ring + (nx % kStages) * kStageU4, gT, gD, t0 + nx, ngroups);
+    const long nx = i + NS - 1;
+    if (nx < n) issue_tile<kMode>(ring + (nx % NS) * kStageU4, gT, gD, t0 + nx, ngroups);
     cp_async_commit();
-    cp_async_wait<kStages - 1>();
-    const uint4* slot = ring + (i % kStages) * kStageU4;
+    cp_async_wait<NS - 1>();
+    const uint4* slot = ring + (i % NS) * kStageU4;
     uint4 vt[kDrawK], vd[kDrawK];
 #pragma unroll
     for (int kk = 0; kk < kDrawK; ++kk) {
@@ -1057,7 +1077,7 @@ __device__ __forceinline__ double locate_one_round(const double* table, long nti
 // table in index order); the index inside it.  Z = 0 at a rejection: the
 // warp recomputes the table for q_n and draws from it (ZERO_MASS warning).
 template <typename T, bool kAligned>
-__device__ __noinline__ void locate(const Params* Pp, int b, int mode, const T* rowT,
+__device__ __noinline__ void locate(const Params* Pp, int b, int n, int mode, const T* rowT,
                                     const T* rowD, const DrawConsts k, long ntiles,
                                     long ngroups) {
   const Params& P = *Pp;
@@ -1089,8 +1109,7 @@ __device__ __noinline__ void locate(const Params* Pp, int b, int mode, const T* 
                 : scan_tile<T, kAligned, kDrawTarget>(rowT, rowD, k, found, ngroups, V, tl);
   }
   if (lane == 0) {
-    const SeqDecision& d = P.decision[b];
-    P.out_tokens[static_cast<long>(b) * (G + 1) + d.n] = token;
+    P.out_tokens[static_cast<long>(b) * (G + 1) + n] = token;
     P.resid_mass[b] = Z;
     if (extra_bits) atomicOr(P.status, extra_bits);
     P.draw_ticket[b] = 0u;  // ready for the next launch
@@ -1148,7 +1167,7 @@ __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(co
       last = __shfl_sync(0xffffffffu, last, 0);
       if (last) {
         __threadfence();  // every lane reads the other warps' tiles after the ticket
-        locate<T, kAligned>(&P, b, d.mode, rowT, rowD, k, ntiles, ngroups);
+        locate<T, kAligned>(&P, b, d.n, d.mode, rowT, rowD, k, ntiles, ngroups);
       }
     }
     t = end;

@@ -51,6 +51,9 @@ SIGNATURES = {
     "specverify_get_launch": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i),
                                    ctypes.POINTER(_i)]),
     "specverify_kernels_per_run": (_i, [_vp, _i, ctypes.POINTER(_i)]),
+    "specverify_set_fused": (_i, [_vp, _i, _i, _i, _i]),
+    "specverify_get_fused": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i),
+                                  ctypes.POINTER(_i)]),
     "specverify_profile_begin": (_i, [_vp, _i]),
     "specverify_profile_end": (_i, [_vp, ctypes.POINTER(_f), ctypes.POINTER(_f), ctypes.POINTER(_i)]),
     "specverify_run_noalloc": (_i, [_i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _f, _vp, _vp, _vp]),
@@ -188,6 +191,20 @@ def specverify_kernels_per_run(h, mapped: bool = False) -> int:
     _check(_lib.specverify_kernels_per_run(h, 1 if mapped else 0, ctypes.byref(k)),
            "specverify_kernels_per_run")
     return k.value
+
+
+def specverify_set_fused(h, enable: bool, unit_groups: int = 0, chunk_tiles: int = 0,
+                         lag: int = -1) -> int:
+    return _check(_lib.specverify_set_fused(h, 1 if enable else 0, unit_groups, chunk_tiles, lag),
+                  "specverify_set_fused")
+
+
+def specverify_get_fused(h) -> tuple[int, int, int, int]:
+    """(enabled for an aligned unmapped run, unit_groups, chunk_tiles, lag) of the handle."""
+    e, u, c, g = ctypes.c_int(), ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    _check(_lib.specverify_get_fused(h, ctypes.byref(e), ctypes.byref(u), ctypes.byref(c),
+                                     ctypes.byref(g)), "specverify_get_fused")
+    return e.value, u.value, c.value, g.value
 
 
 def specverify_profile_begin(h, max_runs: int) -> int:
@@ -489,6 +506,13 @@ class SpecVerify:
 
     def kernels_per_run(self, mapped: bool = False) -> int:
         return specverify_kernels_per_run(self.handle, mapped)
+
+    def set_fused(self, enable: bool, unit_groups: int = 0, chunk_tiles: int = 0, lag: int = -1):
+        """Single launch (True) or three kernels (False) for aligned unmapped runs."""
+        specverify_set_fused(self.handle, enable, unit_groups, chunk_tiles, lag)
+
+    def fused(self) -> tuple[int, int, int, int]:
+        return specverify_get_fused(self.handle)
 
     def profile_begin(self, max_runs: int):
         specverify_profile_begin(self.handle, max_runs)

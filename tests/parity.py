@@ -106,11 +106,13 @@ def to_device(wl, device=0):
 
 
 def gpu_run(wl, slices=None, threads=None, device=0, inputs=None, sv=None, readback=True,
-            mapped=False):
+            mapped=False, fused=None):
     """One verification call of the whole workload; returns numpy outputs.
 
     ``mapped``: call the shared-row entry point on the workload's distinct rows
-    and row maps instead of the per-position arrays."""
+    and row maps instead of the per-position arrays.  ``fused``: True or a
+    (unit_groups, chunk_tiles, lag) tuple selects the single-launch form,
+    False the three kernels; None keeps the handle's setting."""
     import torch
     from speculative_decoding_verification_90_b200.specverify import SpecVerify
     own = sv is None
@@ -120,6 +122,11 @@ def gpu_run(wl, slices=None, threads=None, device=0, inputs=None, sv=None, readb
         if slices is not None or threads is not None:
             c0, t0 = sv.launch()
             sv.set_launch(min(slices or c0, sv.max_slices), threads or t0)
+        if fused is not None:
+            if isinstance(fused, tuple):
+                sv.set_fused(True, *fused)
+            else:
+                sv.set_fused(bool(fused))
         d = inputs if inputs is not None else to_device(wl, device)
         out_t = torch.full((wl.batch, wl.gamma + 1), -7, dtype=torch.int32, device=f"cuda:{device}")
         out_n = torch.full((wl.batch,), -7, dtype=torch.int32, device=f"cuda:{device}")
