@@ -12,10 +12,14 @@
  * bandwidth argument for verification (one read of the parameters scores many
  * positions) is what the fusion exploits: the softmax statistics and the
  * draft tokens' logits are taken from each 128 x 256 accumulator tile in
- * tensor memory, so the logits of the B (2 gamma + 1) positions are never
- * written to global memory.  Only the two rows each sequence draws from (its
- * target and draft rows at the first rejection, or the bonus row) are
- * recomputed as fp32 logits for the draw.
+ * tensor memory.  The draw needs the fp32 logits of two rows per sequence
+ * (its target and draft rows at the first rejection, or the bonus row), known
+ * only after the decision.  Two forms (specverify_lmhead_set_keep_logits):
+ * kept logits (the default when the buffer takes at most 16 GB): the
+ * statistics GEMMs also store every row's fp32 logits, which the GEMM's
+ * tensor-bound time leaves the memory bandwidth to write, and the draw reads
+ * its rows there; recomputed: nothing but the statistics leaves tensor
+ * memory, and a second GEMM over the output layer recomputes the drawn rows.
  *
  * Shapes: hidden is a multiple of 64 (<= 65536); vocab <= 65535 x 256.  Layouts
  * (device pointers, 16-byte aligned, row-major, contiguous):
@@ -27,7 +31,8 @@
  *
  * Memory: the handle owns a workspace of per-(row, 256-column tile) partial
  * statistics (16 B each), the picked-out logits, the plain step's decision
- * records, and 2 x batch x (hidden x 2 + vocab x 4) bytes for the drawn rows.
+ * records, 2 x batch x (hidden x 2 + vocab x 4) bytes for the drawn rows, and
+ * with kept logits batch x (2 gamma + 1) x vocab x 4 bytes.
  * Errors: argument errors return before anything is enqueued; data errors set
  * the status word as in specverify.h; a tensor-core pipeline wait that gives
  * up (it never should) sets SV_ERR_PIPELINE instead of hanging.
@@ -48,6 +53,14 @@ typedef struct specverify_lmhead_ctx *specverify_lmhead_t;
 /* Create a handle for (batch, gamma, vocab, hidden) on `device`. */
 sv_status specverify_lmhead_create(specverify_lmhead_t *out, int batch, int gamma, int vocab,
                                    int hidden, int device);
+
+/* Kept logits (nonzero, allocating their buffer if the handle has none;
+ * SV_ERR_OOM if that fails) or the recomputing form (zero).  Results are the
+ * same: the drawn rows' logits come from the same tensor-core arithmetic.
+ * Not stream-ordered: change it only while no run of the handle is in
+ * flight. */
+sv_status specverify_lmhead_set_keep_logits(specverify_lmhead_t h, int keep);
+sv_status specverify_lmhead_get_keep_logits(specverify_lmhead_t h, int *keep);
 
 /* Enqueue one fused step on `stream` (asynchronous). */
 sv_status specverify_lmhead_run(specverify_lmhead_t h, const void *target_hidden,
@@ -75,7 +88,8 @@ sv_status specverify_lmhead_readback(specverify_lmhead_t h, double *target_lse,
                                      double *resid_mass, void *stream);
 
 /* CUDA-event timing of the next `max_runs` runs: the statistics GEMMs, and
- * the rest (decision, row gather, logit GEMMs, draw), mean ms per run. */
+ * the rest (decision, and the draw; without kept logits also the row gather
+ * and the logit GEMMs), mean ms per run. */
 sv_status specverify_lmhead_profile_begin(specverify_lmhead_t h, int max_runs);
 sv_status specverify_lmhead_profile_end(specverify_lmhead_t h, float *stats_ms, float *rest_ms,
                                         int *runs);

@@ -3,12 +3,13 @@
 // Host side only: argument checks, the workspace, the TMA tensor maps, and the
 // stream-ordered launches of one step:
 //   1. statistics GEMMs (target rows, then draft rows): per-(row, vocabulary
-//      tile) softmax partials and the logits at the draft tokens;
+//      tile) softmax partials and the logits at the draft tokens; with kept
+//      logits (the default) every row's fp32 logits are stored as well;
 //   2. the per-tile partials folded to one per row, and the decide kernel of
 //      the plain step on them;
-//   3. a gather of the two hidden rows each sequence draws from;
-//   4. logit GEMMs for those rows (fp32, [batch, vocab] each);
-//   5. the draw kernel of the plain step on them.
+//   3. without kept logits: a gather of the two hidden rows each sequence
+//      draws from, and logit GEMMs for those rows (fp32, [batch, vocab] each);
+//   4. the draw kernel of the plain step on the rows drawn from.
 #include "specverify_lmhead.h"
 
 #include <cuda.h>
@@ -59,6 +60,11 @@ struct specverify_lmhead_ctx {
   __nv_bfloat16* xd = nullptr;
   float* lt = nullptr;          // [B, vocab] their logits
   float* ld = nullptr;
+  // kept logits: every row's fp32 logits [nT + nD, vocab] (target rows, then
+  // draft rows), written by the statistics GEMMs; the draw reads its rows
+  // there instead of recomputing them
+  int keep_logits = 0;
+  float* all_logits = nullptr;
   std::vector<cudaEvent_t> events;  // 3 per recorded run
   int prof_capacity = 0;
   int prof_runs = 0;
@@ -165,6 +171,9 @@ cudaError_t launch_plain(K kernel, unsigned grid, unsigned block, cudaStream_t s
   kernel<<<grid, block, 0, s>>>(p);
   return cudaGetLastError();
 }
+
+// the kept-logits buffer is allocated by default up to this size
+constexpr size_t kKeepDefaultBytes = size_t{16} << 30;
 
 void split_c(float temperature, float& c_hi, float& c_lo, double& c) {
   const double cd = 1.4426950408889634074 / static_cast<double>(temperature);
@@ -276,7 +285,41 @@ sv_status specverify_lmhead_create(specverify_lmhead_t* out, int batch, int gamm
     delete h;
     return cuda_fail(e);
   }
+  // kept logits by default when they take at most kKeepDefaultBytes; an
+  // allocation that fails leaves the recomputing form (no error)
+  const size_t keep_bytes = static_cast<size_t>(nT + nD) * static_cast<size_t>(vocab) * 4;
+  if (keep_bytes <= kKeepDefaultBytes) {
+    void* kl = nullptr;
+    if (cudaMalloc(&kl, keep_bytes) == cudaSuccess) {
+      h->all_logits = static_cast<float*>(kl);
+      h->keep_logits = 1;
+    } else {
+      (void)cudaGetLastError();
+    }
+  }
   *out = h;
+  return SV_OK;
+}
+
+sv_status specverify_lmhead_set_keep_logits(specverify_lmhead_t h, int keep) {
+  if (!h) return SV_ERR_INVALID_ARG;
+  if (keep && !h->all_logits) {
+    DeviceScope scope(h->device);
+    if (!scope.ok()) return SV_ERR_CUDA;
+    const size_t bytes = static_cast<size_t>(h->batch) * (2L * h->gamma + 1) *
+                         static_cast<size_t>(h->vocab) * 4;
+    void* kl = nullptr;
+    const cudaError_t e = cudaMalloc(&kl, bytes);
+    if (e != cudaSuccess) return cuda_fail(e);
+    h->all_logits = static_cast<float*>(kl);
+  }
+  h->keep_logits = keep ? 1 : 0;
+  return SV_OK;
+}
+
+sv_status specverify_lmhead_get_keep_logits(specverify_lmhead_t h, int* keep) {
+  if (!h || !keep) return SV_ERR_INVALID_ARG;
+  *keep = h->keep_logits;
   return SV_OK;
 }
 
@@ -362,6 +405,9 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   g.row_offset = 0;
   g.positions = G + 1;
   g.rows2 = 0;
+  const bool keep = h->keep_logits && h->all_logits;
+  g.logits = keep ? h->all_logits : nullptr;  // every row's logits, indexed by row_offset + r
+  g.logits2 = g.logits;
   if (G > 0 && draft_weight == target_weight) {
     // one output layer: target and draft rows in one launch, the weight read once
     g.rows2 = static_cast<int>(nD);
@@ -381,8 +427,10 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
 
   // 2. the decision, on the partials (one per 256-column tile of each row)
   Params p{};
-  p.target = h->lt;  // the compact rows drawn from (written in step 4)
-  p.draft = h->ld;
+  // the rows drawn from: with kept logits, rows of the [nT + nD, vocab]
+  // buffer (unmapped layout); else the compact rows written in step 3
+  p.target = keep ? h->all_logits : h->lt;
+  p.draft = keep ? h->all_logits + nT * static_cast<long>(V) : h->ld;
   p.target_map = nullptr;
   p.draft_map = nullptr;
   p.target_rows = nT;
@@ -412,7 +460,7 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   p.c = c;
   p.gathered_target = h->gathered;
   p.gathered_draft = h->gathered + nT;
-  p.draw_compact = 1;
+  p.draw_compact = keep ? 0 : 1;
   if (e == cudaSuccess) {
     combine_rows_kernel<<<static_cast<unsigned>((nT + nD + 7) / 8), 256, 0, s>>>(
         h->partial, h->ntiles, nT + nD, h->combined);
@@ -423,8 +471,8 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
     e = launch_plain(specverify::decide_kernel<float>, static_cast<unsigned>((B + per - 1) / per),
                      specverify::kDecideThreads, s, p);
 
-  // 3-4. the two rows each sequence draws from, and their logits
-  if (e == cudaSuccess) {
+  // 3. without kept logits: the two rows each sequence draws from, and their logits
+  if (e == cudaSuccess && !keep) {
     gather_rows_kernel<<<B, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(target_hidden),
                                          static_cast<const __nv_bfloat16*>(draft_hidden),
                                          h->decision, G, D, h->xt, h->xd);
@@ -438,7 +486,9 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   l.num_sms = h->num_sms;
   l.error = h->gemm_error;
   l.logits = h->lt;
-  if (G > 0 && draft_weight == target_weight) {
+  if (keep) {
+    // the rows drawn from are in the kept logits
+  } else if (G > 0 && draft_weight == target_weight) {
     // one output layer: the 2B drawn rows (target rows, then draft rows, one
     // tensor) as one GEMM, so each weight tile is read once for both
     l.rows = 2 * B;
@@ -452,7 +502,7 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
     }
   }
 
-  // 5. the draw on fp32 rows
+  // 4. the draw on fp32 rows
   const bool aligned = (static_cast<size_t>(V) * 4) % 16 == 0;
   if (e == cudaSuccess)
     e = aligned ? specverify::launch_draw<float, true>(p, static_cast<unsigned>(h->draw_slices), s, false)
@@ -568,6 +618,7 @@ void specverify_lmhead_destroy(specverify_lmhead_t h) {
       cudaDeviceSynchronize();
       for (cudaEvent_t ev : h->events) cudaEventDestroy(ev);
       if (h->ws) cudaFree(h->ws);
+      if (h->all_logits) cudaFree(h->all_logits);
     }
   }
   delete h;

@@ -65,7 +65,8 @@ struct LmParams {
   int positions;            // G + 1 for target rows (the last position has no token), G for draft
   float* gathered;          // [row_offset + rows] logit at the row's token
   float c_hi, c_lo;
-  // logits mode
+  // logits mode; statistics mode: null, or [row_offset + rows, vocab] fp32
+  // where the tile's logits are stored as well
   float* logits;            // [rows, vocab] fp32
   float* logits2;           // [rows2, vocab] fp32: the second hidden tensor's
   unsigned* error;          // set when a wait gives up
@@ -190,6 +191,25 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 // the epilogue of one tile (one warp: its 32 TMEM lanes = rows q*32 .. q*32+31)
 // ---------------------------------------------------------------------------
 
+// columns c .. c+31 of one fp32 logit row: 16-byte stores when they are
+// 16-byte aligned and inside the vocabulary (every full tile of a vocabulary
+// that is a multiple of 4), else one store per column inside it.  Streaming
+// stores (evict-first in L2): the logits are read back at most once, later,
+// and must not push the operand tiles that concurrent CTAs share out of L2.
+__device__ __forceinline__ void store_logits32(float* row, int c, int vocab, bool vec,
+                                               const float (&v)[32]) {
+  float* out = row + c;
+  if (vec && c + 32 <= vocab) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 4)
+      __stcs(reinterpret_cast<float4*>(out + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (c + i < vocab) __stcs(out + i, v[i]);
+  }
+}
+
 template <int kMode>
 __device__ __forceinline__ void epilogue_tile(const LmParams& P, uint32_t acc_addr, int m0, int n0,
                                               int vt, int q, int lane) {
@@ -202,10 +222,12 @@ __device__ __forceinline__ void epilogue_tile(const LmParams& P, uint32_t acc_ad
       if (pos < P.token_stride) t = P.tokens[static_cast<long>(seq) * P.token_stride + pos];
     }
     float o = -INFINITY, sum = 0.f, xt = 0.f;
+    const bool vec = (P.vocab % 4) == 0;
 #pragma unroll 1
     for (int c0 = 0; c0 < kBN; c0 += 32) {
       float v[32];
       tmem_ld32(lane_addr + c0, v);
+      if (P.logits && r < P.rows) store_logits32(P.logits + (P.row_offset + r) * P.vocab, n0 + c0, P.vocab, vec, v);
       float cm = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -230,25 +252,12 @@ __device__ __forceinline__ void epilogue_tile(const LmParams& P, uint32_t acc_ad
       if (t >= n0 && t < n0 + kBN) P.gathered[P.row_offset + r] = xt;
     }
   } else {
-    // 16-byte stores when the row's 32 columns are 16-byte aligned and inside
-    // the vocabulary (every full tile of a vocabulary that is a multiple of 4)
     const bool vec = (P.vocab % 4) == 0;
 #pragma unroll 1
     for (int c0 = 0; c0 < kBN; c0 += 32) {
       float v[32];
       tmem_ld32(lane_addr + c0, v);
-      if (r < P.rows) {
-        float* out = P.logits + static_cast<long>(r) * P.vocab + n0 + c0;
-        if (vec && n0 + c0 + 32 <= P.vocab) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(out + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (n0 + c0 + i < P.vocab) out[i] = v[i];
-        }
-      }
+      if (r < P.rows) store_logits32(P.logits + static_cast<long>(r) * P.vocab, n0 + c0, P.vocab, vec, v);
     }
   }
 }

@@ -438,6 +438,31 @@ constexpr int kMaxGamma = 255;
 // through L2 (ld.global.cg), never from a possibly stale L1 line.
 template <bool kCg>
 __device__ __forceinline__ double row_lse2(const RowPartial* parts, int S, int& valid) {
+  if (S <= 8) {
+    // every partial's 16-byte record loaded at once (one memory round trip);
+    // then the same two passes, in the same order, as the general loop
+    float o[8];
+    double s[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      if (r < S) {
+        const uint4 v = kCg ? __ldcg(reinterpret_cast<const uint4*>(parts) + r)
+                            : *(reinterpret_cast<const uint4*>(parts) + r);
+        s[r] = __hiloint2double(static_cast<int>(v.y), static_cast<int>(v.x));
+        o[r] = __uint_as_float(v.z);
+      }
+    }
+    float O = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (r < S) O = fmaxf(O, o[r]);
+    double sum = 0.0;
+#pragma unroll
+    for (int r = 0; r < 8; ++r)
+      if (r < S) sum += (o[r] == -INFINITY) ? s[r] * 0.0 : s[r] * exp2(static_cast<double>(o[r]) - O);
+    valid = (O != -INFINITY) && isfinite(sum) && sum > 0.0;
+    return static_cast<double>(O) + log2(sum);
+  }
   float O = -INFINITY;
   for (int r = 0; r < S; ++r) O = fmaxf(O, kCg ? __ldcg(&parts[r].o) : parts[r].o);
   double sum = 0.0;

@@ -73,6 +73,8 @@ SIGNATURES = {
     "specverify_lmhead_profile_end": (_i, [_vp, ctypes.POINTER(_f), ctypes.POINTER(_f),
                                            ctypes.POINTER(_i)]),
     "specverify_lmhead_destroy": (None, [_vp]),
+    "specverify_lmhead_set_keep_logits": (_i, [_vp, _i]),
+    "specverify_lmhead_get_keep_logits": (_i, [_vp, ctypes.POINTER(_i)]),
     "specverify_status_string": (ctypes.c_char_p, [_i]),
     "specverify_last_error": (ctypes.c_char_p, []),
 }
@@ -311,6 +313,18 @@ def specverify_lmhead_profile_end(h) -> dict:
     _check(_lib.specverify_lmhead_profile_end(h, ctypes.byref(a), ctypes.byref(c),
                                               ctypes.byref(n)), "specverify_lmhead_profile_end")
     return {"stats_ms": a.value, "rest_ms": c.value, "runs": n.value}
+
+
+def specverify_lmhead_set_keep_logits(h, keep: bool) -> int:
+    return _check(_lib.specverify_lmhead_set_keep_logits(h, 1 if keep else 0),
+                  "specverify_lmhead_set_keep_logits")
+
+
+def specverify_lmhead_get_keep_logits(h) -> bool:
+    k = ctypes.c_int()
+    _check(_lib.specverify_lmhead_get_keep_logits(h, ctypes.byref(k)),
+           "specverify_lmhead_get_keep_logits")
+    return bool(k.value)
 
 
 def specverify_lmhead_destroy(h) -> None:
@@ -629,6 +643,15 @@ class LmHeadVerify:
         if getattr(self, "handle", None):
             specverify_lmhead_destroy(self.handle)
             self.handle = None
+
+    @property
+    def keep_logits(self) -> bool:
+        """Whether the statistics GEMMs keep every row's logits for the draw."""
+        return specverify_lmhead_get_keep_logits(self.handle)
+
+    @keep_logits.setter
+    def keep_logits(self, keep: bool):
+        specverify_lmhead_set_keep_logits(self.handle, keep)
 
     def __del__(self):
         try:

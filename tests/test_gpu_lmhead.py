@@ -39,12 +39,16 @@ def _f(a, dtype=np.float32):
     return torch.from_numpy(np.ascontiguousarray(a, dtype)).cuda()
 
 
-def run_fused(w, lm=None):
+def run_fused(w, lm=None, keep=None):
+    """One fused step; ``keep``: kept logits (True), recomputed drawn rows
+    (False), or the handle's default (None)."""
     from speculative_decoding_verification_90_b200.specverify import LmHeadVerify
     own = lm is None
     if own:
         lm = LmHeadVerify(w.batch, w.gamma, w.vocab, w.hidden)
     try:
+        if keep is not None:
+            lm.keep_logits = keep
         B, G = w.batch, w.gamma
         ht, wt = _bf(w.target_hidden), _bf(w.target_weight)
         hd = _bf(w.draft_hidden)
@@ -79,9 +83,9 @@ def oracle_fused(w, logits=None):
                          float(np.float32(w.temperature)), threads=os.cpu_count() or 1)
 
 
-def _parity(w, name):
+def _parity(w, name, keep=None):
     import parity
-    g = run_fused(w)
+    g = run_fused(w, keep=keep)
     logits = oracle_logits(w)
     o = oracle_fused(w, logits)
     old = parity.MARGIN
@@ -137,17 +141,38 @@ def test_gemm_against_float64_logits(rows, hidden, vocab):
     (3, 0, 2000, 128, True),      # bonus draw only
     (6, 9, 1000, 64, True),       # the smallest hidden size
 ])
-def test_fused_parity(B, G, V, D, shared):
+@pytest.mark.parametrize("keep", [True, False])
+def test_fused_parity(B, G, V, D, shared, keep):
     w = workloads.lmhead(seed=B + G + V, batch=B, gamma=G, vocab=V, hidden=D, shared_weight=shared)
-    g, o, s = _parity(w, f"fused B={B} G={G} V={V} D={D} shared={shared}")
+    g, o, s = _parity(w, f"fused B={B} G={G} V={V} D={D} shared={shared} keep={keep}", keep)
     assert g["status"] == 0
 
 
-def test_fused_parity_full_size():
-    """64 sequences, gamma 8, V = 128256, hidden 4096 (the benchmark case)."""
+@pytest.mark.parametrize("keep", [True, False])
+def test_fused_parity_full_size(keep):
+    """64 sequences, gamma 8, V = 128256, hidden 4096 (the benchmark case),
+    in both forms: the logits kept by the statistics GEMMs, and the drawn
+    rows recomputed by a second GEMM."""
     w = workloads.lmhead()
-    g, o, s = _parity(w, "fused full size")
+    g, o, s = _parity(w, f"fused full size keep={keep}", keep)
     assert g["status"] == 0
+
+
+def test_kept_and_recomputed_logits_agree_exactly():
+    """Both forms take the drawn rows' logits from the same tensor-core
+    arithmetic (per element the same products in the same order), so their
+    outputs and readbacks are identical; the default is the kept form."""
+    from speculative_decoding_verification_90_b200.specverify import LmHeadVerify
+    w = workloads.lmhead(seed=11, batch=12, gamma=5, vocab=20000, hidden=512)
+    with LmHeadVerify(w.batch, w.gamma, w.vocab, w.hidden) as lm:
+        assert lm.keep_logits
+        a = run_fused(w, lm, keep=True)
+        b = run_fused(w, lm, keep=False)
+        assert not lm.keep_logits
+        c = run_fused(w, lm, keep=True)
+    for k in ("out_tokens", "out_num_accepted", "resid_mass", "target_lse", "q_tok"):
+        np.testing.assert_array_equal(a[k], b[k])
+        np.testing.assert_array_equal(a[k], c[k])
 
 
 def test_fused_token_range_and_repeat():
