@@ -968,33 +968,44 @@ __device__ __forceinline__ float key16_value(unsigned k) {
 }
 
 struct XState {
-  bool off = false;  // an entry above the window, NaN or +inf: the general path takes the row
-  float tail = 0.f;  // kTail: sum 2^(x c - o) below the window
+  unsigned kmax2 = 0u;            // per 16-bit half: the largest key seen
+  unsigned kmin2 = 0xffffffffu;   // per 16-bit half: the smallest key seen
+  float2 tail = make_float2(0.f, 0.f);  // kTail: sum 2^(x c - o) below the window (per half)
 };
 
 // One 32-bit word of two bf16 entries, branch-free: both keys in one register
 // (each half h -> h ^ 0x8000 for a positive value, ~h for a negative one);
-// a key in the window [klo, klo + span] adds 1 to its count (a predicated
-// shared atomic at index key - klo); one unsigned compare flags a key above
-// the window, +inf or NaN of either sign; the mass below the window is an ex2
-// of -inf where it does not apply.
+// a key in the window [klo, klo + span] adds 1 to its count (a shared
+// reduction at index key - klo, predicated in the instruction itself); the
+// largest and smallest keys of both halves are kept with packed 16-bit
+// max / min, which after the scan flag a key above the window, +inf or NaN
+// of either sign; the mass below the window is an ex2 of -inf where it does
+// not apply.  hb: the shared-memory address of the count of key 0.
 template <bool kTail>
-__device__ __forceinline__ void x_word(unsigned w, unsigned klo, unsigned span, unsigned top,
-                                       unsigned* hist, float c_hi, float c_lo, float o,
-                                       XState& st) {
+__device__ __forceinline__ void x_word(unsigned w, unsigned klo, unsigned span, unsigned hb,
+                                       float c_hi, float c_lo, float o, XState& st) {
   const unsigned neg = (w >> 15) & 0x00010001u;              // sign of each half
   const unsigned k2 = w ^ (0x80008000u | (neg * 0x7fffu));   // both keys
+  asm("max.u16x2 %0, %0, %1;" : "+r"(st.kmax2) : "r"(k2));
+  asm("min.u16x2 %0, %0, %1;" : "+r"(st.kmin2) : "r"(k2));
+  unsigned idx[2];
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     const unsigned k = half ? (k2 >> 16) : (k2 & 0xffffu);
-    const unsigned i = k - klo;
-    const bool in = i <= span;
-    if (in) atomicAdd(hist + i, 1u);
-    st.off |= (k - kKeyNegInf) > top;  // top = window top - key(-inf)
-    if constexpr (kTail) {
-      const float x = __uint_as_float(half ? (w & 0xffff0000u) : (w << 16));
-      st.tail += ex2(in ? -INFINITY : specverify::arg2(x, c_hi, c_lo, o));
-    }
+    idx[half] = k - klo;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.le.u32 p, %0, %1;\n\t@p red.shared.add.u32 [%2], 1;\n\t}"
+        ::"r"(idx[half]), "r"(span), "r"(hb + 4u * k));
+  }
+  if constexpr (kTail) {
+    // both halves' exponents with the packed fp32x2 instructions (x c - o
+    // as two FMAs each, as everywhere); ex2 of -inf for entries in the window
+    const float2 x = make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    const float2 y = __ffma2_rn(x, make_float2(c_lo, c_lo),
+                                __ffma2_rn(x, make_float2(c_hi, c_hi), make_float2(-o, -o)));
+    const float2 e = make_float2(ex2(idx[0] <= span ? -INFINITY : y.x),
+                                 ex2(idx[1] <= span ? -INFINITY : y.y));
+    st.tail = __fadd2_rn(st.tail, e);
   }
 }
 
@@ -1034,12 +1045,13 @@ __device__ bool exact_select(const SampParams& P, long r, long nT, const __nv_bf
   // the window: keys klo .. khi (never the key of -inf); count index = key - klo
   const int klo = max(khi - kXBins + 1, static_cast<int>(kKeyNegInf) + 1);
   const unsigned span = static_cast<unsigned>(khi - klo);
-  const unsigned top = static_cast<unsigned>(khi) - kKeyNegInf;
+  // the count of key k lives at hist[k - klo] (only keys in the window are counted)
+  const unsigned hb = static_cast<unsigned>(__cvta_generic_to_shared(hist)) - 4u * static_cast<unsigned>(klo);
   const float o = key16_value(ks) * c_hi;  // weights of the entries below the window
 
   XState st;
   {
-    constexpr int kU = 4;
+    constexpr int kU = 8;  // 16-byte loads in flight per thread
     const long stride = static_cast<long>(kSelThreads) * kU;
     for (long g0 = tid; g0 < groups; g0 += stride) {
       uint4 v[kU];
@@ -1052,17 +1064,23 @@ __device__ bool exact_select(const SampParams& P, long r, long nT, const __nv_bf
       for (int u = 0; u < kU; ++u) {
         const long g = g0 + static_cast<long>(u) * kSelThreads;
         if (g >= groups) break;
-        x_word<kTail>(v[u].x, static_cast<unsigned>(klo), span, top, hist, c_hi, c_lo, o, st);
-        x_word<kTail>(v[u].y, static_cast<unsigned>(klo), span, top, hist, c_hi, c_lo, o, st);
-        x_word<kTail>(v[u].z, static_cast<unsigned>(klo), span, top, hist, c_hi, c_lo, o, st);
-        x_word<kTail>(v[u].w, static_cast<unsigned>(klo), span, top, hist, c_hi, c_lo, o, st);
+        x_word<kTail>(v[u].x, static_cast<unsigned>(klo), span, hb, c_hi, c_lo, o, st);
+        x_word<kTail>(v[u].y, static_cast<unsigned>(klo), span, hb, c_hi, c_lo, o, st);
+        x_word<kTail>(v[u].z, static_cast<unsigned>(klo), span, hb, c_hi, c_lo, o, st);
+        x_word<kTail>(v[u].w, static_cast<unsigned>(klo), span, hb, c_hi, c_lo, o, st);
       }
     }
   }
   // rows with an entry above the window, NaN or +inf go to the general path
-  // (which also reports the invalid ones)
-  if (__syncthreads_or(st.off)) return false;
-  const double tail_o = kTail ? block_sum<kSelThreads>(static_cast<double>(st.tail), smd) : 0.0;
+  // (which also reports the invalid ones); a key below that of -inf is a
+  // negative NaN
+  const unsigned kmx = max(st.kmax2 & 0xffffu, st.kmax2 >> 16);
+  const unsigned kmn = min(st.kmin2 & 0xffffu, st.kmin2 >> 16);
+  const bool off = kmx > static_cast<unsigned>(khi) || kmn < kKeyNegInf;
+  if (__syncthreads_or(off)) return false;
+  const double tail_o =
+      kTail ? block_sum<kSelThreads>(static_cast<double>(st.tail.x) + static_cast<double>(st.tail.y), smd)
+            : 0.0;
   // the window in descending order: rank q = khi - key, count hist[span - q]
   // (ranks past span lie below the window: no count); the row maximum is the
   // first rank with a count (none: every entry is below the window or -inf,
