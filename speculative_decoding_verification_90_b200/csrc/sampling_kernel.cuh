@@ -1695,16 +1695,75 @@ __global__ void __launch_bounds__(kDrawThreads) draw_kernel(const SampParams P) 
     return s;
   };
 
+  // 16-byte aligned rows with one chunk of kDrawChunk elements per thread
+  // and tile: the chunks are read as kQ 16-byte loads per row, four tiles'
+  // loads in flight together (the same elements, sums and order as
+  // chunk_sum)
+  constexpr int kVec = specverify::Elem<T>::kVec;
+  constexpr int kQ = kDrawChunk / kVec;  // 16-byte loads per row and chunk
+  constexpr int kTB = 4;                 // tiles whose loads are in flight together
+  const bool vec = L == kDrawChunk && (static_cast<long>(V) * sizeof(T)) % 16 == 0 &&
+                   reinterpret_cast<uintptr_t>(rowT) % 16 == 0 &&
+                   (G == 0 || reinterpret_cast<uintptr_t>(rowD) % 16 == 0);
+  auto load_chunk = [&](int tile, int md, uint4 (&vt)[kQ], uint4 (&vd)[kQ]) {
+    const long i0 = static_cast<long>(tile) * E + static_cast<long>(threadIdx.x) * L;
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) {
+      const long i = i0 + q * kVec;
+      if (i < V) {  // V is a multiple of kVec here: the group is whole
+        vt[q] = __ldg(reinterpret_cast<const uint4*>(rowT + i));
+        if (md == kModeResidual) vd[q] = __ldg(reinterpret_cast<const uint4*>(rowD + i));
+      }
+    }
+  };
+  auto chunk_sum_vec = [&](int tile, int md, const uint4 (&vt)[kQ], const uint4 (&vd)[kQ],
+                           int* last) -> float {
+    const long i0 = static_cast<long>(tile) * E + static_cast<long>(threadIdx.x) * L;
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < kQ; ++q) {
+      if (i0 + q * kVec >= V) break;
+      float xt[kVec], xd[kVec];
+      specverify::Elem<T>::unpack(vt[q], xt);
+      if (md == kModeResidual) specverify::Elem<T>::unpack(vd[q], xd);
+#pragma unroll
+      for (int e = 0; e < kVec; ++e) {
+        const float rv = resid_elem(xt[e], md == kModeResidual ? xd[e] : 0.f, md, d, c_hi, c_lo,
+                                    lt_hi, lt_lo, k_hi, k_lo);
+        s += rv;
+        if (rv > 0.f) *last = static_cast<int>(i0 + q * kVec + e);
+      }
+    }
+    return s;
+  };
+
   // pass 1: the mass of every tile (warp partials, no barrier in the loop)
   double Z = 0.0;
   int last_pos = -1;
   for (int attempt = 0; attempt < 2; ++attempt) {
     int lp = -1;
-    for (int t = 0; t < ntiles; ++t) {
-      float s = chunk_sum(t, mode, &lp);
+    if (vec) {
+      for (int t0 = 0; t0 < ntiles; t0 += kTB) {
+        uint4 vt[kTB][kQ], vd[kTB][kQ];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) s_part[t][warp] = s;
+        for (int j = 0; j < kTB; ++j)
+          if (t0 + j < ntiles) load_chunk(t0 + j, mode, vt[j], vd[j]);
+#pragma unroll
+        for (int j = 0; j < kTB; ++j) {
+          if (t0 + j >= ntiles) break;
+          float s = chunk_sum_vec(t0 + j, mode, vt[j], vd[j], &lp);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          if (lane == 0) s_part[t0 + j][warp] = s;
+        }
+      }
+    } else {
+      for (int t = 0; t < ntiles; ++t) {
+        float s = chunk_sum(t, mode, &lp);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) s_part[t][warp] = s;
+      }
     }
     __syncthreads();
     double zt = 0.0;
