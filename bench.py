@@ -81,6 +81,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-shared-rows", action="store_true",
                     help="skip the timing of the shared-row entry point (multibranch)")
+    ap.add_argument("--fused", action="store_true",
+                    help="time the headline step in the single-launch form (specverify_set_fused)")
+    ap.add_argument("--no-single-launch", action="store_true",
+                    help="skip the extra timing of the single-launch form on the bench batch")
     ap.add_argument("--no-sampling", action="store_true",
                     help="skip the timing of the sampling variants")
     ap.add_argument("--sampling", default=None,
@@ -371,6 +375,8 @@ def run_ours(args):
     out_n = torch.empty((B,), dtype=torch.int32, device=dev)
 
     sv = SpecVerify(B, G, V, wl.dtype, local)
+    if args.fused:
+        sv.set_fused(True)
     if args.slices or args.threads or args.draw_slices:
         c0, t0 = sv.launch()
         sv.set_launch(args.slices or c0, args.threads or t0, args.draw_slices)
@@ -467,6 +473,11 @@ def run_ours(args):
     if extras and not args.no_sampling:
         sampling = time_sampling(args, wl, sv, sets, n_sets, out_t, out_n, dev, world, local)
 
+    # the same batch in the single-launch form (one persistent kernel)
+    single = None
+    if extras and not args.fused and not args.no_single_launch:
+        single = time_single_launch(args, sv, step, dev, world, local)
+
     # the same batch through the shared-row entry point: each distinct row once
     shared = None
     if extras and wl.mapped and not args.no_shared_rows:
@@ -506,7 +517,8 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic, "peak_source": peak_src,
                          "algorithmic_bytes_per_launch": step_bytes,
-                         "kernel": "stats_kernel (streams every logit once)"},
+                         "kernel": ("fused_kernel (the whole step in one launch)" if args.fused
+                                    else "stats_kernel (streams every logit once)")},
             "kernels_us_per_step": {"stats": 1e3 * kern["stats_ms"],
                                     "decide_and_draw": 1e3 * kern["draw_ms"],
                                     "runs": kern["runs"],
@@ -537,6 +549,14 @@ def run_ours(args):
                        "decide_and_draw_us": v["decide_and_draw_us"],
                        "status_after": v["status"]}
                 for name, v in sampling.items()}
+        if single is not None:
+            line["single_launch"] = {
+                "entry": "specverify_run with specverify_set_fused(h, 1, 0, 0, -1)",
+                "value": positions * args.steps / (single["ms_max"] / 1e3), "unit": UNIT,
+                "ms_per_step": single["ms_max"] / args.steps,
+                "kernel_us": 1e3 * single["stats_ms"], "kernels_per_step": single["kernels"],
+                "step_hbm_gbs": step_bytes / (single["ms_max"] / 1e3 / args.steps) / 1e9,
+                "status_after": single["status"]}
         if shared is not None:
             sh_bytes = shared["bytes"]
             sh_ach = sh_bytes / (shared["stats_ms"] / 1e3) / 1e9
@@ -784,6 +804,25 @@ def others_summary(res, peak):
     return out
 
 
+def time_single_launch(args, sv, step, dev, world, local):
+    """Time the bench's steps with the handle in the single-launch form, then
+    restore the three-kernel form."""
+    import torch
+    sv.set_fused(True)
+    try:
+        for i in range(max(3, args.warmup)):
+            step(i)
+        torch.cuda.synchronize()
+        ms, kern = timed_then_profiled(step, args.steps, sv.profile_begin, sv.profile_end, world,
+                                       local)
+        st, _ = sv.status()
+        kernels = sv.kernels_per_run()
+    finally:
+        sv.set_fused(False)
+    return {"ms_max": svdist.max_over_ranks(ms, device=dev), "stats_ms": kern["stats_ms"],
+            "status": st, "kernels": kernels}
+
+
 def time_shared_rows(args, wl, sv, put, out_t, out_n, dev, world, local):
     """Time specverify_run_mapped on the workload's distinct rows and row maps."""
     import torch
@@ -893,12 +932,14 @@ def time_lmhead(args, dev, world, local):
                                    world, local)
     ms_max = svdist.max_over_ranks(ms, device=dev)
     st, _ = lm.status()
+    keep = lm.keep_logits
     lm.close()
     rows = B * (2 * G + 1)
     return {"workload": w.name, "steps": steps, "ms_max": ms_max, "stats_ms": kern["stats_ms"],
-            "rest_ms": kern["rest_ms"], "positions": B * G * world,
+            "rest_ms": kern["rest_ms"], "positions": B * G * world, "keep_logits": keep,
             "stats_flops": 2.0 * rows * w.vocab * w.hidden,
-            "draw_flops": 2.0 * 2 * B * w.vocab * w.hidden,
+            # the drawn rows' logits come from the kept logits, or from a second GEMM
+            "draw_flops": 0.0 if keep else 2.0 * 2 * B * w.vocab * w.hidden,
             "weight_bytes": w.vocab * w.hidden * 2 * (1 if w.draft_weight is w.target_weight else 2),
             "status": st}
 
@@ -917,7 +958,11 @@ def lmhead_summary(g):
                      "algorithmic_flops_per_step": g["stats_flops"]},
         "step_tflops": step_tf,
         "stats_gemm_us": 1e3 * g["stats_ms"], "rest_us": 1e3 * g["rest_ms"],
-        "logits_written_per_step": "only the 2 drawn rows per sequence (fp32)",
+        "logits_kept": g.get("keep_logits"),
+        "logits_written_per_step": ("every row's fp32 logits (kept by the statistics GEMMs; "
+                                    "the draw reads its 2 rows per sequence there)"
+                                    if g.get("keep_logits") else
+                                    "only the 2 drawn rows per sequence (fp32, a second GEMM)"),
         "status_after": g["status"],
     }
 

@@ -5,7 +5,7 @@
 // is one ordered list of tasks that the warps take from a global counter:
 //
 //   statistics unit  one warp streams a contiguous run of 16-byte groups of
-//                    one logit row (sixteen 128-bit loads in flight per lane)
+//                    one logit row (eight 128-bit loads in flight per lane)
 //                    and writes its (offset, sum) partial;
 //   draw chunk       one warp computes the residual (or target) masses of a
 //                    run of tiles of the rows a sequence draws from.
