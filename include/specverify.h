@@ -82,7 +82,10 @@ typedef enum {
   SV_ERR_ROW_INDEX = 19,   /* device: a row map entry was outside the rows given */
   SV_ERR_PARENT = 20,      /* device (fold gate): a parent entry out of range, a self link or a cycle */
   SV_ERR_TEMPERATURE = 21, /* device (sampling variants): a temperature < 0, NaN or infinite */
-  SV_ERR_PIPELINE = 22     /* device: a bounded wait gave up (LM-head pipeline, single-launch step) */
+  SV_ERR_PIPELINE = 22,    /* device: a bounded wait gave up (LM-head pipeline, single-launch step) */
+  SV_ERR_BOUNDS = 23       /* device, debug builds only (libspecverify_debug.so, compiled with
+                              -DSV_DEBUG_BOUNDS=1): an index the kernels derived fell outside its
+                              buffer; the access was skipped */
 } sv_status;
 
 /*

@@ -694,6 +694,7 @@ sv_status specverify_get_status(specverify_t h, void* stream, uint32_t* bits) {
     if (e != cudaSuccess) return cuda_fail(e);
     return SV_ERR_PIPELINE;
   }
+  if (v & specverify::kStatBounds) return SV_ERR_BOUNDS;
   if (v & specverify::kStatRowIndex) return SV_ERR_ROW_INDEX;
   if (v & specsamp::kStatTemperature) return SV_ERR_TEMPERATURE;
   if (v & specverify::kStatTokenRange) return SV_ERR_TOKEN_RANGE;
@@ -859,6 +860,7 @@ const char* specverify_status_string(sv_status s) {
     case SV_ERR_ROW_INDEX: return "row map entry outside the logit rows given";
     case SV_ERR_PARENT: return "parent index out of range, self link or cycle";
     case SV_ERR_TEMPERATURE: return "temperature negative, NaN or infinite";
+    case SV_ERR_BOUNDS: return "device: a bounds check of a debug build failed";
     case SV_ERR_PIPELINE: return "a bounded device wait gave up (tensor-core pipeline or single-launch step)";
   }
   return "unknown status";

@@ -58,14 +58,36 @@ constexpr int kMaxSlices = 64;
 enum : int { kFlagReject = 0, kFlagAccept = 1, kFlagTokenRange = 2, kFlagNonFinite = 3 };
 // status word bits
 // (16 is the sampling variants' temperature bit; 32: a bounded wait of the
-// single-launch step gave up)
+// single-launch step gave up; 64: a bounds check of a debug build failed)
 enum : unsigned {
   kStatTokenRange = 1u,
   kStatNonFinite = 2u,
   kStatZeroMass = 4u,
   kStatRowIndex = 8u,
-  kStatWait = 32u
+  kStatWait = 32u,
+  kStatBounds = 64u
 };
+
+// Debug builds (compiled with -DSV_DEBUG_BOUNDS=1) check the indices that
+// the kernels derive from launch geometry and from decisions before they
+// touch the workspace or the outputs: a failed check sets kStatBounds in the
+// status word and the access is skipped (nothing traps).  In normal builds
+// every check is the constant true.
+#ifndef SV_DEBUG_BOUNDS
+#define SV_DEBUG_BOUNDS 0
+#endif
+__device__ __forceinline__ bool bounds_ok(long i, long n, unsigned* status) {
+#if SV_DEBUG_BOUNDS
+  if (i >= 0 && i < n) return true;
+  atomicOr(status, kStatBounds);
+  return false;
+#else
+  (void)i;
+  (void)n;
+  (void)status;
+  return true;
+#endif
+}
 // what the draw kernel draws from
 enum : int { kDrawResidual = 0, kDrawTarget = 1, kDrawNone = 2 };
 
@@ -621,6 +643,7 @@ __global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Param
   const long r = unit / S;
   const int slice = static_cast<int>(unit - r * S);
   const long nT = P.target_rows;
+  if (!bounds_ok(r, nT + P.draft_rows, P.status)) return;  // (block-uniform)
   const T* row = (r < nT) ? static_cast<const T*>(P.target) + r * V
                           : static_cast<const T*>(P.draft) + (r - nT) * V;
   const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
@@ -1128,13 +1151,13 @@ __device__ __noinline__ void locate(const Params* Pp, int b, int n, int mode, co
   }
   if (!one_round) find_in_table(table, ntiles, u * Z, found, tl);
   int token = -1;
-  if (found >= 0) {
+  if (found >= 0 && bounds_ok(found, ntiles, P.status)) {
     token = (mode == kDrawResidual)
                 ? scan_tile<T, kAligned, kDrawResidual>(rowT, rowD, k, found, ngroups, V, tl)
                 : scan_tile<T, kAligned, kDrawTarget>(rowT, rowD, k, found, ngroups, V, tl);
   }
   if (lane == 0) {
-    P.out_tokens[static_cast<long>(b) * (G + 1) + n] = token;
+    if (bounds_ok(n, G + 1, P.status)) P.out_tokens[static_cast<long>(b) * (G + 1) + n] = token;
     P.resid_mass[b] = Z;
     if (extra_bits) atomicOr(P.status, extra_bits);
     P.draw_ticket[b] = 0u;  // ready for the next launch
@@ -1160,7 +1183,12 @@ __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(co
     const long row0 = static_cast<long>(b) * ntiles;
     const long end = (hi < row0 + ntiles) ? hi : row0 + ntiles;
     const SeqDecision d = P.decision[b];
-    if (d.mode != kDrawNone) {
+    // (a debug build skips a sequence whose rows drawn from lie outside the
+    // logit buffers, in every warp alike, so its ticket stays untouched)
+    const bool rows_ok = d.mode == kDrawNone ||
+                         (bounds_ok(d.trow, P.target_rows, P.status) &&
+                          (d.mode != kDrawResidual || bounds_ok(d.drow, P.draft_rows, P.status)));
+    if (d.mode != kDrawNone && rows_ok) {
       const T* rowT = static_cast<const T*>(P.target) + d.trow * V;
       const T* rowD = (d.mode == kDrawResidual) ? static_cast<const T*>(P.draft) + d.drow * V
                                                 : nullptr;

@@ -6,7 +6,10 @@ takes torch tensors (device memory and streams come from PyTorch).
 
 Importing this module loads the library and fails loudly if it has not been
 built (``python -m speculative_decoding_verification_90_b200.build``).  There
-is no CPU fallback.
+is no CPU fallback.  With SPECVERIFY_DEBUG_BOUNDS=1 in the environment it
+loads ``libspecverify_debug.so`` instead: the same library compiled with
+device bounds checks that report SV_ERR_BOUNDS instead of touching memory
+outside a buffer.
 """
 from __future__ import annotations
 
@@ -16,7 +19,8 @@ import os
 import numpy as np
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libspecverify.so")
+DEBUG_BOUNDS = os.environ.get("SPECVERIFY_DEBUG_BOUNDS", "0") == "1"
+LIB_PATH = os.path.join(_PKG, "libspecverify_debug.so" if DEBUG_BOUNDS else "libspecverify.so")
 
 SV_DTYPE_F32 = 0
 SV_DTYPE_BF16 = 1
@@ -33,6 +37,7 @@ SV_ERR_ROW_INDEX = 19
 SV_ERR_PARENT = 20
 SV_ERR_TEMPERATURE = 21
 SV_ERR_PIPELINE = 22
+SV_ERR_BOUNDS = 23
 
 # every function declared in include/*.h, with its ctypes signature
 _vp, _i, _f, _u32p = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.POINTER(ctypes.c_uint32)
