@@ -43,7 +43,11 @@ constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK * 2;   // 16 KB
 constexpr int kBBytes = kBN * kBK * 2;   // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kSmemBytes = kStages * kStageBytes + 1024;  // + room to align to 1024
+// the epilogue warps' staging buffers for the logits they store: 32 rows x
+// kStageLd floats each (rows 16-byte aligned, conflict-free quarter warps)
+constexpr int kStageLd = 36;
+constexpr int kEpiStageBytes = 32 * kStageLd * 4;
+constexpr int kSmemBytes = kStages * kStageBytes + 4 * kEpiStageBytes + 1024;  // + room to align to 1024
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s per wait
 
 enum : int { kModeStats = 0, kModeLogits = 1 };
@@ -191,28 +195,47 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
 // the epilogue of one tile (one warp: its 32 TMEM lanes = rows q*32 .. q*32+31)
 // ---------------------------------------------------------------------------
 
-// columns c .. c+31 of one fp32 logit row: 16-byte stores when they are
-// 16-byte aligned and inside the vocabulary (every full tile of a vocabulary
-// that is a multiple of 4), else one store per column inside it.  Streaming
-// stores (evict-first in L2): the logits are read back at most once, later,
-// and must not push the operand tiles that concurrent CTAs share out of L2.
-__device__ __forceinline__ void store_logits32(float* row, int c, int vocab, bool vec,
-                                               const float (&v)[32]) {
-  float* out = row + c;
-  if (vec && c + 32 <= vocab) {
+// The 32 x 32 chunk of fp32 logits of rows r0 .. r0+31 (lane l holds row
+// r0 + l's values v[0..31]) and columns c .. c+31, stored to base[row *
+// vocab + column] for the rows below nrows and the columns inside the
+// vocabulary.  The chunk goes through the warp's staging buffer so that each
+// store instruction writes whole 128-byte row segments (8 lanes per row, 4
+// rows per instruction) instead of 16 bytes of 32 different rows.  16-byte
+// stores when the vocabulary is a multiple of 4 (16-byte aligned rows), else
+// one per column.  Streaming stores (evict-first in L2): the logits are read
+// back at most once, later, and must not push the operand tiles that
+// concurrent CTAs share out of L2.
+__device__ __forceinline__ void store_chunk_staged(float* base, long r0, int nrows, int c,
+                                                   int vocab, bool vec, const float (&v)[32],
+                                                   float* stage) {
+  const int lane = threadIdx.x & 31;
+  float4* mine = reinterpret_cast<float4*>(stage + lane * kStageLd);
 #pragma unroll
-    for (int i = 0; i < 32; i += 4)
-      __stcs(reinterpret_cast<float4*>(out + i), make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]));
-  } else {
+  for (int k = 0; k < 8; ++k) mine[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+  __syncwarp();
+  const int sub = lane >> 3, col = c + 4 * (lane & 7);
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (c + i < vocab) __stcs(out + i, v[i]);
+  for (int i = 0; i < 8; ++i) {
+    const int rr = 4 * i + sub;
+    const float4 x = *reinterpret_cast<const float4*>(stage + rr * kStageLd + 4 * (lane & 7));
+    if (rr < nrows) {
+      float* out = base + (r0 + rr) * vocab + col;
+      if (vec && col + 4 <= vocab) {
+        __stcs(reinterpret_cast<float4*>(out), x);
+      } else {
+        if (col < vocab) __stcs(out, x.x);
+        if (col + 1 < vocab) __stcs(out + 1, x.y);
+        if (col + 2 < vocab) __stcs(out + 2, x.z);
+        if (col + 3 < vocab) __stcs(out + 3, x.w);
+      }
+    }
   }
+  __syncwarp();  // the buffer is rewritten by the next chunk
 }
 
 template <int kMode>
 __device__ __forceinline__ void epilogue_tile(const LmParams& P, uint32_t acc_addr, int m0, int n0,
-                                              int vt, int q, int lane) {
+                                              int vt, int q, int lane, float* stage) {
   const int r = m0 + q * 32 + lane;
   const uint32_t lane_addr = acc_addr + (static_cast<uint32_t>(q * 32) << 16);
   if constexpr (kMode == kModeStats) {
@@ -227,7 +250,9 @@ __device__ __forceinline__ void epilogue_tile(const LmParams& P, uint32_t acc_ad
     for (int c0 = 0; c0 < kBN; c0 += 32) {
       float v[32];
       tmem_ld32(lane_addr + c0, v);
-      if (P.logits && r < P.rows) store_logits32(P.logits + (P.row_offset + r) * P.vocab, n0 + c0, P.vocab, vec, v);
+      if (P.logits)
+        store_chunk_staged(P.logits + P.row_offset * P.vocab, m0 + q * 32, P.rows - (m0 + q * 32),
+                           n0 + c0, P.vocab, vec, v, stage);
       float cm = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -257,7 +282,8 @@ __device__ __forceinline__ void epilogue_tile(const LmParams& P, uint32_t acc_ad
     for (int c0 = 0; c0 < kBN; c0 += 32) {
       float v[32];
       tmem_ld32(lane_addr + c0, v);
-      if (r < P.rows) store_logits32(P.logits + static_cast<long>(r) * P.vocab, n0 + c0, P.vocab, vec, v);
+      store_chunk_staged(P.logits, m0 + q * 32, P.rows - (m0 + q * 32), n0 + c0, P.vocab, vec, v,
+                         stage);
     }
   }
 }
@@ -385,6 +411,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     __syncwarp();
   } else {
     const int q = warp % 4;  // TMEM lane quarter of this warp
+    float* stage = reinterpret_cast<float*>(smem + kStages * kStageBytes + (warp - 2) * kEpiStageBytes);
     long i = 0;
     for (long t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
       const int acc = static_cast<int>(i & 1);
@@ -405,7 +432,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
         P.logits = P0.logits2;
       }
       epilogue_tile<kMode>(P, tmem + static_cast<uint32_t>(acc * kBN),
-                           (second ? rt - tiles1 : rt) * kBM, vt * kBN, vt, q, lane);
+                           (second ? rt - tiles1 : rt) * kBM, vt * kBN, vt, q, lane, stage);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[acc]);
