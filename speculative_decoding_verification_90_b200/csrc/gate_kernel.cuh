@@ -304,14 +304,23 @@ __global__ void __launch_bounds__(kSlotThreads) scan_kernel(const GateParams P) 
   // (the flag array is 256-byte aligned and padded to a multiple of 4)
   const long chunk = ((P.rows + kSlotThreads - 1) / kSlotThreads + 3) & ~3L;
   const long lo = min(P.rows, chunk * threadIdx.x), hi = min(P.rows, lo + chunk);
+  // kW words (4 flags each) loaded together, so a thread's chunk costs one
+  // memory round trip per 4 kW rows in each of the two passes
+  constexpr int kW = 8;
+  const unsigned* fw = reinterpret_cast<const unsigned*>(P.flag);
   int v = 0;
-  for (long i = lo; i < hi; i += 4) {
-    const unsigned w = __ldcg(reinterpret_cast<const unsigned*>(P.flag + i));
-    // bytes past `hi` (the next chunk's rows, or padding past the last row)
-    // are masked off
-    const long left = hi - i;
-    const unsigned keep = left >= 4 ? 0xffffffffu : ((1u << (8 * left)) - 1u);
-    v += __popc(w & keep & 0x01010101u);
+  for (long i0 = lo; i0 < hi; i0 += 4 * kW) {
+    unsigned w[kW];
+#pragma unroll
+    for (int k = 0; k < kW; ++k) w[k] = (i0 + 4 * k < hi) ? __ldcg(fw + (i0 + 4 * k) / 4) : 0u;
+#pragma unroll
+    for (int k = 0; k < kW; ++k) {
+      // bytes past `hi` (the next chunk's rows, or padding past the last
+      // row) are masked off
+      const long left = hi - (i0 + 4 * k);
+      const unsigned keep = left >= 4 ? 0xffffffffu : (left > 0 ? ((1u << (8 * left)) - 1u) : 0u);
+      v += __popc(w[k] & keep & 0x01010101u);
+    }
   }
   int x = v;
 #pragma unroll
@@ -332,8 +341,18 @@ __global__ void __launch_bounds__(kSlotThreads) scan_kernel(const GateParams P) 
   }
   __syncthreads();
   int slot = (warp > 0 ? s_warp[warp - 1] : 0) + x - v;
-  for (long i = lo; i < hi; ++i)
-    if (__ldcg(P.flag + i) != 0) P.rank[i] = slot++;
+  for (long i0 = lo; i0 < hi; i0 += 4 * kW) {
+    unsigned w[kW];
+#pragma unroll
+    for (int k = 0; k < kW; ++k) w[k] = (i0 + 4 * k < hi) ? __ldcg(fw + (i0 + 4 * k) / 4) : 0u;
+#pragma unroll
+    for (int k = 0; k < kW; ++k)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const long i = i0 + 4 * k + q;
+        if (i < hi && ((w[k] >> (8 * q)) & 0xffu) != 0u) P.rank[i] = slot++;
+      }
+  }
   if (threadIdx.x == kSlotThreads - 1) *P.n_packed = s_warp[kWarp - 1];
 }
 
