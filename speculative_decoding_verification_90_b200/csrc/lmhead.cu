@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(256) combine_rows_kernel(const RowPartial* in,
                                                            long rows, RowPartial* out) {
   const int lane = threadIdx.x & 31;
   const long r = static_cast<long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  cudaGridDependencySynchronize();  // the GEMM's partials (programmatic dependent launch)
   if (r >= rows) return;
   const RowPartial* p = in + r * ntiles;
   float O = -INFINITY;
@@ -166,10 +167,22 @@ __global__ void __launch_bounds__(256) combine_rows_kernel(const RowPartial* in,
   if (lane == 0) out[r] = RowPartial{S, O, 0};
 }
 
-template <typename K>
-cudaError_t launch_plain(K kernel, unsigned grid, unsigned block, cudaStream_t s, const Params& p) {
-  kernel<<<grid, block, 0, s>>>(p);
-  return cudaGetLastError();
+// a launch that may start before its predecessor on the stream has finished
+// (programmatic dependent launch); the kernel waits in a grid-dependency
+// barrier before it reads the predecessor's results
+template <typename K, typename... A>
+cudaError_t launch_pdl(K kernel, unsigned grid, unsigned block, cudaStream_t s, A... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 // the kept-logits buffer is allocated by default up to this size
@@ -461,15 +474,13 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   p.gathered_target = h->gathered;
   p.gathered_draft = h->gathered + nT;
   p.draw_compact = keep ? 0 : 1;
-  if (e == cudaSuccess) {
-    combine_rows_kernel<<<static_cast<unsigned>((nT + nD + 7) / 8), 256, 0, s>>>(
-        h->partial, h->ntiles, nT + nD, h->combined);
-    e = cudaGetLastError();
-  }
+  if (e == cudaSuccess)
+    e = launch_pdl(combine_rows_kernel, static_cast<unsigned>((nT + nD + 7) / 8), 256u, s,
+                   static_cast<const RowPartial*>(h->partial), h->ntiles, nT + nD, h->combined);
   const int per = specverify::kDecideThreads / specverify::kWarp;
   if (e == cudaSuccess)
-    e = launch_plain(specverify::decide_kernel<float>, static_cast<unsigned>((B + per - 1) / per),
-                     specverify::kDecideThreads, s, p);
+    e = launch_pdl(specverify::decide_kernel<float>, static_cast<unsigned>((B + per - 1) / per),
+                   static_cast<unsigned>(specverify::kDecideThreads), s, p);
 
   // 3. without kept logits: the two rows each sequence draws from, and their logits
   if (e == cudaSuccess && !keep) {
@@ -505,8 +516,8 @@ sv_status specverify_lmhead_run(specverify_lmhead_t h, const void* target_hidden
   // 4. the draw on fp32 rows
   const bool aligned = (static_cast<size_t>(V) * 4) % 16 == 0;
   if (e == cudaSuccess)
-    e = aligned ? specverify::launch_draw<float, true>(p, static_cast<unsigned>(h->draw_slices), s, false)
-                : specverify::launch_draw<float, false>(p, static_cast<unsigned>(h->draw_slices), s, false);
+    e = aligned ? specverify::launch_draw<float, true>(p, static_cast<unsigned>(h->draw_slices), s, true)
+                : specverify::launch_draw<float, false>(p, static_cast<unsigned>(h->draw_slices), s, true);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
   if (e != cudaSuccess) return cuda_fail(e);
   return SV_OK;
