@@ -34,6 +34,10 @@ struct specverify_ctx {
   int max_slices = 1;  // the partial-statistics workspace holds this many per position
   int draw_slices = 64; // at most this many draw blocks per sequence
   int num_sms = 148;
+  // tapered statistics grid (0: every row in `slices` slices): all but the
+  // last taper_tail rows of a run in taper_slices long slices
+  long taper_tail = 0;
+  int taper_slices = 0;
   void* ws = nullptr;  // one device allocation for the whole workspace
   RowPartial* partial = nullptr;
   RowStat* tstat = nullptr;
@@ -89,11 +93,20 @@ long num_groups(const specverify_ctx* h) {
   return (static_cast<long>(h->vocab) + ve - 1) / ve;
 }
 
+// Tapered grid: rows in long slices first, then about one wave of short
+// blocks (kTaperShort slices per row) at the end of the grid.
+constexpr int kTaperLong = 2;
+constexpr int kTaperShort = 8;
+constexpr double kTaperWaves = 1.0;
+
 // Default launch shape of the statistics kernel: 128 threads per block,
 // every logit row split over `slices` blocks (at most 8) so that the grid
 // holds about four waves of blocks where the batch allows (the last, partial
 // wave then costs little; more, smaller blocks only add per-block overhead),
-// with at least one 16-byte group per thread.
+// with at least one 16-byte group per thread.  Batches of several waves of
+// rows of 64 KB or more take the tapered grid instead: long blocks (less
+// start-up per byte) with the short ones dispatched last, so that the SMs
+// run out of work together.
 void default_shape(specverify_ctx* h) {
   const int threads = 128;
   const long rows = static_cast<long>(h->batch) * (2L * h->gamma + 1);
@@ -109,6 +122,16 @@ void default_shape(specverify_ctx* h) {
   }
   h->slices = best;
   h->threads = threads;
+  h->taper_tail = 0;
+  h->taper_slices = 0;
+  const int shortS = cap < kTaperShort ? cap : kTaperShort;
+  const long tail = static_cast<long>(kTaperWaves * static_cast<double>(slots) / shortS + 0.999);
+  if (shortS > kTaperLong && ngroups >= 4096 && rows >= 2 * tail &&
+      (rows - tail) * kTaperLong + tail * shortS >= 2 * slots) {
+    h->slices = shortS;
+    h->taper_slices = kTaperLong;
+    h->taper_tail = tail;
+  }
 }
 
 // Draw blocks per sequence, at most: the draw kernel's grid is also capped at
@@ -141,10 +164,12 @@ cudaError_t launch_pdl(K kernel, unsigned blocks, unsigned threads, cudaStream_t
   return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
+// The statistics kernel is a programmatic dependent of whatever precedes it
+// on the stream: its blocks may become resident during the predecessor's
+// tail and wait for it to complete before their first load.
 template <typename T, int NT, bool A>
 cudaError_t launch_stats_nt(const Params& p, long blocks, cudaStream_t s) {
-  specverify::stats_kernel<T, NT, A><<<static_cast<unsigned>(blocks), NT, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(specverify::stats_kernel<T, NT, A>, static_cast<unsigned>(blocks), NT, s, p);
 }
 
 // One step: statistics, decide, draw.  events[0..2] (may be null): before
@@ -153,7 +178,7 @@ template <typename T, bool A>
 cudaError_t launch_step(const Params& p, int NT, unsigned draw_blocks, cudaStream_t s,
                         cudaEvent_t* ev) {
   const long rows = p.target_rows + p.draft_rows;
-  const long blocks = rows * p.slices;
+  const long blocks = p.taper_rows * p.taper_slices + (rows - p.taper_rows) * p.slices;
   cudaError_t e = cudaSuccess;
   if (ev) e = cudaEventRecord(ev[0], s);
   if (e != cudaSuccess) return e;
@@ -230,6 +255,7 @@ template <typename T>
 cudaError_t launch_fused(const specverify_ctx* h, Params p, cudaStream_t s, cudaEvent_t* ev) {
   const specverify::FusedShape fs = fused_shape_of(h);
   p.slices = fs.units_per_row;  // the partial table holds max_slices >= this per row
+  p.taper_rows = 0;
   specverify::FusedParams f;
   f.task_next = h->fctl;
   f.exit_count = h->fctl + 1;
@@ -331,6 +357,12 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
   const long ngroups = num_groups(h);
   p.slices = h->slices;
   p.groups_per_slice = static_cast<int>((ngroups + h->slices - 1) / h->slices);
+  const long rows = target_rows + draft_rows;
+  p.taper_rows = (h->taper_slices > 0 && rows > h->taper_tail) ? rows - h->taper_tail : 0;
+  p.taper_slices = h->taper_slices;
+  p.taper_groups = h->taper_slices > 0
+                       ? static_cast<int>((ngroups + h->taper_slices - 1) / h->taper_slices)
+                       : 0;
   p.draw_tiles = draw_tiles(h);
   const unsigned nd = draw_blocks(h);
   p.c_hi = c_hi;
@@ -742,6 +774,8 @@ sv_status specverify_set_launch(specverify_t h, int slices, int threads, int dra
   if (draw_slices > 64) return SV_ERR_INVALID_ARG;
   h->slices = slices;
   h->threads = threads;
+  h->taper_tail = 0;  // an explicit shape cuts every row alike
+  h->taper_slices = 0;
   h->draw_slices = (draw_slices >= 1) ? draw_slices : draw_shape(h);
   return SV_OK;
 }

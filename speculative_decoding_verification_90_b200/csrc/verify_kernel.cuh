@@ -156,6 +156,15 @@ struct Params {
   const float* gathered_target;
   const float* gathered_draft;
   int draw_compact;
+  // tapered slicing of the statistics grid: the first taper_rows rows are
+  // cut into taper_slices slices of taper_groups groups each, the remaining
+  // rows into `slices` slices of groups_per_slice groups, so that the blocks
+  // dispatched last are short and the grid's last wave ends together.  The
+  // partial table keeps `slices` entries per row; a tapered row fills its
+  // entries past taper_slices with empty partials.  taper_rows 0: every row
+  // alike.
+  long taper_rows;
+  int taper_slices, taper_groups;
 };
 
 // ---------------------------------------------------------------------------
@@ -636,23 +645,45 @@ constexpr int min_blocks() {
 template <typename T, int NT, bool kAligned>
 __global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Params P) {
   constexpr int kVec = Elem<T>::kVec;
+  // the logits may be the previous kernel's output (programmatic launch):
+  // the block may be resident before it completes, and waits for it here
+  cudaGridDependencySynchronize();
   const int V = P.vocab, S = P.slices;
   // one unit = one block = one slice of one row; the target tensor's rows
   // come first, then the draft tensor's, so the grid walks memory in order
+  // (the tapered rows first, in long slices)
   const long unit = blockIdx.x;
-  const long r = unit / S;
-  const int slice = static_cast<int>(unit - r * S);
+  const long uA = P.taper_rows * P.taper_slices;
+  long r, slice, gps, Sr;
+  if (unit < uA) {
+    r = unit / P.taper_slices;
+    slice = unit - r * P.taper_slices;
+    gps = P.taper_groups;
+    Sr = P.taper_slices;
+  } else {
+    const long u2 = unit - uA;
+    const long q = u2 / S;
+    r = P.taper_rows + q;
+    slice = u2 - q * S;
+    gps = P.groups_per_slice;
+    Sr = S;
+  }
   const long nT = P.target_rows;
   if (!bounds_ok(r, nT + P.draft_rows, P.status)) return;  // (block-uniform)
   const T* row = (r < nT) ? static_cast<const T*>(P.target) + r * V
                           : static_cast<const T*>(P.draft) + (r - nT) * V;
   const long ngroups = (static_cast<long>(V) + kVec - 1) / kVec;
-  long glo = static_cast<long>(slice) * P.groups_per_slice;
-  long ghi = glo + P.groups_per_slice;
+  long glo = slice * gps;
+  long ghi = glo + gps;
   if (glo > ngroups) glo = ngroups;
   if (ghi > ngroups) ghi = ngroups;
   const RowPartial part = slice_stats<T, NT, kAligned, 8>(row, glo, ghi, V, P.c_hi, P.c_lo);
-  if (threadIdx.x == 0) P.partial[unit] = part;
+  if (threadIdx.x == 0) {
+    P.partial[r * S + slice] = part;
+    // a tapered row's table entries past its slices: empty partials
+    if (slice == 0)
+      for (long j = Sr; j < S; ++j) P.partial[r * S + j] = RowPartial{0.0, -INFINITY, 0};
+  }
   cudaTriggerProgrammaticLaunchCompletion();
 }
 
