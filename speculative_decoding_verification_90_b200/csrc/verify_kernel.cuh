@@ -506,19 +506,62 @@ __device__ __forceinline__ double row_lse2(const RowPartial* parts, int S, int& 
   return static_cast<double>(O) + log2(sum);  // log2 sum_i 2^(x_i c)
 }
 
+// What lane j of a deciding warp reads from the caller's buffers for position
+// j of sequence b (j <= gamma): its rows, the drafted token, its uniform and
+// the two logits at the token.  None of it comes from this library's kernels,
+// so a programmatic dependent may load it before its grid-dependency wait.
+struct LaneInputs {
+  long tr, dr;  // rows of the logit buffers that hold the position
+  int t;        // drafted token
+  float u, xt, xd;
+  bool tok_bad, map_bad;
+};
+
+template <typename T>
+__device__ __forceinline__ LaneInputs lane_inputs(const Params& P, int b, int j) {
+  const int G = P.gamma, V = P.vocab;
+  LaneInputs in{0, 0, 0, 0.f, 0.f, 0.f, false, false};
+  if (j > G) return in;
+  const long position = static_cast<long>(b) * (G + 1) + j;
+  const long pj = static_cast<long>(b) * G + j;
+  const bool has_draft = j < G;
+  in.tr = P.target_map ? static_cast<long>(P.target_map[position]) : position;
+  in.dr = has_draft ? (P.draft_map ? static_cast<long>(P.draft_map[pj]) : pj) : 0;
+  in.map_bad = in.tr < 0 || in.tr >= P.target_rows ||
+               (has_draft && (in.dr < 0 || in.dr >= P.draft_rows));
+  if (has_draft) {
+    in.t = P.tokens[pj];
+    in.u = P.u_accept[pj];
+    in.tok_bad = (in.t < 0 || in.t >= V);
+    if (!in.tok_bad && !in.map_bad) {
+      in.xt = P.gathered_target ? P.gathered_target[in.tr]
+                                : Elem<T>::load1(static_cast<const T*>(P.target) + in.tr * V, in.t);
+      in.xd = P.gathered_draft ? P.gathered_draft[in.dr]
+                               : Elem<T>::load1(static_cast<const T*>(P.draft) + in.dr * V, in.t);
+    }
+  }
+  return in;
+}
+
 // The decision of sequence b by the calling warp (all 32 lanes): lane j
 // combines the partials of position j's rows, forms q(t), p(t) and the ratio
 // in fp64 and tests u < ratio (step 2); a warp ballot finds the first
-// rejection n (step 3).  Writes the accepted prefix, the padding, the count,
-// the per-position readback records and what the draw kernel draws from.
+// rejection n (step 3).  Returns what the draw draws from (in every lane).
+// write: also writes the accepted prefix, the padding, the count, the
+// per-position readback records, the status bits and the decision record
+// (exactly one warp per sequence writes; others only use the result).
 // kCg: the partials come from other warps of the same launch (see row_lse2).
 // staged (unmapped rows only): the sequence's partials were copied to shared
 // memory, its gamma+1 target rows then its gamma draft rows, S per row.
+// pre (may be null): this lane's lane_inputs for positions 0 .. 31, loaded
+// earlier.
 template <typename T, bool kCg = false>
-__device__ __forceinline__ void decide_sequence(const Params& P, int b,
-                                                const RowPartial* staged = nullptr) {
+__device__ __forceinline__ SeqDecision decide_sequence(const Params& P, int b,
+                                                       const RowPartial* staged = nullptr,
+                                                       bool write = true,
+                                                       const LaneInputs* pre = nullptr) {
   const int lane = threadIdx.x & (kWarp - 1);
-  const int G = P.gamma, V = P.vocab, S = P.slices;
+  const int G = P.gamma, S = P.slices;
   const double c = P.c;
   int n = G;          // first rejection, gamma if none
   unsigned bits = 0;  // data errors of the sequence
@@ -534,24 +577,13 @@ __device__ __forceinline__ void decide_sequence(const Params& P, int b,
       const long position = static_cast<long>(b) * (G + 1) + j;
       const long pj = static_cast<long>(b) * G + j;
       const bool has_draft = j < G;
-      // rows of the logit buffers that hold this position
-      tr = P.target_map ? static_cast<long>(P.target_map[position]) : position;
-      dr = has_draft ? (P.draft_map ? static_cast<long>(P.draft_map[pj]) : pj) : 0;
-      map_bad = tr < 0 || tr >= P.target_rows || (has_draft && (dr < 0 || dr >= P.draft_rows));
       // the acceptance test's inputs first: their loads overlap the combine
-      int t = 0;
-      float u = 0.f, xt = 0.f, xd = 0.f;
-      if (has_draft) {
-        t = P.tokens[pj];
-        u = P.u_accept[pj];
-        tok_bad = (t < 0 || t >= V);
-        if (!tok_bad && !map_bad) {
-          xt = P.gathered_target ? P.gathered_target[tr]
-                                 : Elem<T>::load1(static_cast<const T*>(P.target) + tr * V, t);
-          xd = P.gathered_draft ? P.gathered_draft[dr]
-                                : Elem<T>::load1(static_cast<const T*>(P.draft) + dr * V, t);
-        }
-      }
+      const LaneInputs in = (pre && base == 0) ? *pre : lane_inputs<T>(P, b, j);
+      tr = in.tr;
+      dr = in.dr;
+      map_bad = in.map_bad;
+      tok_bad = in.tok_bad;
+      const float u = in.u, xt = in.xt, xd = in.xd;
       int validT = 0, validD = 1;
       if (!map_bad) {
         if (staged) {
@@ -562,8 +594,10 @@ __device__ __forceinline__ void decide_sequence(const Params& P, int b,
           if (has_draft) lD = row_lse2<kCg>(P.partial + (P.target_rows + dr) * S, S, validD);
         }
       }
-      P.tstat[position] = RowStat{lT, validT, 0};
-      if (has_draft) P.dstat[pj] = RowStat{lD, validD, 0};
+      if (write) {
+        P.tstat[position] = RowStat{lT, validT, 0};
+        if (has_draft) P.dstat[pj] = RowStat{lD, validD, 0};
+      }
       row_bad = !map_bad && (!validT || !validD);
       if (has_draft) {
         PosInfo info{0.0, 0.0, 0.0, kFlagReject, 0};
@@ -581,7 +615,7 @@ __device__ __forceinline__ void decide_sequence(const Params& P, int b,
           else info.ratio = exp2(lq - lp);
           info.flag = (static_cast<double>(u) < info.ratio) ? kFlagAccept : kFlagReject;
         }
-        P.pos[pj] = info;
+        if (write) P.pos[pj] = info;
         flag = info.flag;
       }
     }
@@ -606,12 +640,22 @@ __device__ __forceinline__ void decide_sequence(const Params& P, int b,
     }
   }
   const long bo = static_cast<long>(b) * (G + 1);
+  SeqDecision d{0.0, 0.0, 0, 0, 0, kDrawNone, bits, 0.f, 0.f, 0.f, 1.f};
+  if (!bits) {
+    d = SeqDecision{lT_n, lD_n, P.draw_compact ? b : tr_n, P.draw_compact ? b : dr_n, n,
+                    (n < G) ? kDrawResidual : kDrawTarget, 0u, 0.f, 0.f, 0.f, 1.f};
+    float lt_lo;
+    split2(lT_n, d.lt_hi, lt_lo);
+    split2(lT_n - lD_n, d.k_hi, d.k_lo);
+    d.fT = static_cast<float>(exp2(-static_cast<double>(lt_lo)));
+  }
+  if (!write) return d;
   if (bits) {
     for (int q = lane; q <= G; q += kWarp) P.out_tokens[bo + q] = -1;
     if (lane == 0) {
       P.out_num_accepted[b] = 0;
       P.resid_mass[b] = NAN;
-      P.decision[b] = SeqDecision{0.0, 0.0, 0, 0, 0, kDrawNone, bits, 0.f, 0.f, 0.f, 1.f};
+      P.decision[b] = d;
       atomicOr(P.status, bits);
     }
   } else {
@@ -622,15 +666,10 @@ __device__ __forceinline__ void decide_sequence(const Params& P, int b,
     }
     if (lane == 0) {
       P.out_num_accepted[b] = n;
-      SeqDecision d{lT_n, lD_n, P.draw_compact ? b : tr_n, P.draw_compact ? b : dr_n, n,
-                    (n < G) ? kDrawResidual : kDrawTarget, 0u, 0.f, 0.f, 0.f, 1.f};
-      float lt_lo;
-      split2(lT_n, d.lt_hi, lt_lo);
-      split2(lT_n - lD_n, d.k_hi, d.k_lo);
-      d.fT = static_cast<float>(exp2(-static_cast<double>(lt_lo)));
       P.decision[b] = d;
     }
   }
+  return d;
 }
 
 // ---------------------------------------------------------------------------
@@ -648,6 +687,10 @@ __global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Param
   // the logits may be the previous kernel's output (programmatic launch):
   // the block may be resident before it completes, and waits for it here
   cudaGridDependencySynchronize();
+  // From here every input of the caller is complete, so the next kernel may
+  // be scheduled: it reads the caller's inputs at once, and this grid's
+  // results only after its own grid-dependency wait.
+  cudaTriggerProgrammaticLaunchCompletion();
   const int V = P.vocab, S = P.slices;
   // one unit = one block = one slice of one row; the target tensor's rows
   // come first, then the draft tensor's, so the grid walks memory in order
@@ -684,20 +727,28 @@ __global__ void __launch_bounds__(NT, min_blocks<NT>()) stats_kernel(const Param
     if (slice == 0)
       for (long j = Sr; j < S; ++j) P.partial[r * S + j] = RowPartial{0.0, -INFINITY, 0};
   }
-  cudaTriggerProgrammaticLaunchCompletion();
 }
 
 // ---------------------------------------------------------------------------
 // kernel 2: decide (one warp per sequence)
 // ---------------------------------------------------------------------------
 
+// The caller's inputs to a decision (tokens, uniforms, row maps, the logits
+// at the tokens) are loaded before the grid-dependency wait: the statistics
+// kernel lets this one be scheduled only once they are complete.  Logits
+// gathered by an earlier kernel of this library are read after the wait.
+// The draw kernel reads nothing before its own wait, so it may be scheduled
+// at once.
 template <typename T>
 __global__ void __launch_bounds__(kDecideThreads) decide_kernel(const Params P) {
+  const int b = blockIdx.x * (kDecideThreads / kWarp) + (threadIdx.x >> 5);
+  const bool early = b < P.batch && !P.gathered_target && !P.gathered_draft;
+  LaneInputs pre{0, 0, 0, 0.f, 0.f, 0.f, false, false};
+  if (early) pre = lane_inputs<T>(P, b, threadIdx.x & (kWarp - 1));
+  cudaTriggerProgrammaticLaunchCompletion();
   // the statistics of the previous kernel must be complete and visible
   cudaGridDependencySynchronize();
-  const int b = blockIdx.x * (kDecideThreads / kWarp) + (threadIdx.x >> 5);
-  if (b < P.batch) decide_sequence<T>(P, b);  // warp-uniform
-  cudaTriggerProgrammaticLaunchCompletion();
+  if (b < P.batch) decide_sequence<T>(P, b, nullptr, true, early ? &pre : nullptr);  // warp-uniform
 }
 
 // ---------------------------------------------------------------------------
@@ -1195,7 +1246,22 @@ __device__ __noinline__ void locate(const Params* Pp, int b, int n, int mode, co
   }
 }
 
-template <typename T, bool kAligned>
+// The decision of sequence b inside the draw kernel, as a call of its own so
+// that none of its registers is live across the draw's tile loop.
+template <typename T>
+__device__ __noinline__ void decide_in_draw(const Params* Pp, int b, bool write,
+                                            const LaneInputs* pre, SeqDecision* out) {
+  *out = decide_sequence<T>(*Pp, b, nullptr, write, pre);
+}
+
+// kInline: the kernel follows the statistics kernel directly and every warp
+// takes the decision of each sequence its run touches itself (the same
+// arithmetic in every warp, so all agree); the warp whose run holds the
+// sequence's first tile writes the decision's outputs.  The caller's inputs
+// to the first decision are loaded before the grid-dependency wait.  Chosen
+// for grids of less than one wave with no more sequences than warps (a run
+// then touches at most two sequences).
+template <typename T, bool kAligned, bool kInline = false>
 __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(const __grid_constant__ Params P) {
   constexpr int kVec = Elem<T>::kVec;
   extern __shared__ uint4 draw_smem[];
@@ -1208,12 +1274,21 @@ __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(co
   const long W = static_cast<long>(gridDim.x) * kDrawWarps;
   const long w = static_cast<long>(blockIdx.x) * kDrawWarps + (threadIdx.x >> 5);
   const long lo = total * w / W, hi = total * (w + 1) / W;
-  cudaGridDependencySynchronize();  // the decisions of the previous kernel
+  const int b_pre = (lo < hi) ? static_cast<int>(lo / ntiles) : -1;
+  LaneInputs pre{0, 0, 0, 0.f, 0.f, 0.f, false, false};
+  if constexpr (kInline) {
+    if (b_pre >= 0) pre = lane_inputs<T>(P, b_pre, lane);
+  }
+  cudaGridDependencySynchronize();  // the statistics (or decisions) of the previous kernel
   for (long t = lo; t < hi;) {
     const int b = static_cast<int>(t / ntiles);
     const long row0 = static_cast<long>(b) * ntiles;
     const long end = (hi < row0 + ntiles) ? hi : row0 + ntiles;
-    const SeqDecision d = P.decision[b];
+    SeqDecision d;
+    if constexpr (kInline)
+      decide_in_draw<T>(&P, b, t == row0, b == b_pre ? &pre : nullptr, &d);
+    else
+      d = P.decision[b];
     // (a debug build skips a sequence whose rows drawn from lie outside the
     // logit buffers, in every warp alike, so its ticket stays untouched)
     const bool rows_ok = d.mode == kDrawNone ||
@@ -1258,16 +1333,26 @@ __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(co
   }
 }
 
+// Whether the draw kernel takes the decisions itself (kInline): a draw grid of
+// less than one resident wave (a small, launch-bound batch: one launch and
+// one grid-dependency wait fewer), with no more sequences than warps.  On
+// batches that fill the wave every warp's serial decision costs more than the
+// separate decide kernel saves.
+inline bool draw_decides(long batch, unsigned grid, int num_sms) {
+  return static_cast<long>(grid) < static_cast<long>(num_sms) * kDrawBlocksPerSM &&
+         batch <= static_cast<long>(grid) * kDrawWarps;
+}
+
 // Host: launch the draw kernel (its ring needs more than the default 48 KB of
 // dynamic shared memory per block), optionally as a programmatic dependent
 // launch of the previous kernel on the stream.
-template <typename T, bool kAligned>
+template <typename T, bool kAligned, bool kInline = false>
 inline cudaError_t launch_draw(const Params& p, unsigned grid, cudaStream_t s, bool pdl) {
   const size_t smem = kAligned ? kDrawSmem : 0;
   cudaError_t e = cudaSuccess;
   if (kAligned)
-    e = cudaFuncSetAttribute(draw_kernel<T, kAligned>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
+    e = cudaFuncSetAttribute(draw_kernel<T, kAligned, kInline>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
@@ -1279,7 +1364,7 @@ inline cudaError_t launch_draw(const Params& p, unsigned grid, cudaStream_t s, b
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, draw_kernel<T, kAligned>, p);
+  return cudaLaunchKernelEx(&cfg, draw_kernel<T, kAligned, kInline>, p);
 }
 
 }  // namespace specverify
