@@ -36,7 +36,10 @@
  * device workspace (per-branch validated parents, per-row flags, provenance
  * and packed slots, a status word).  Errors: argument
  * errors return before anything is enqueued; a bad parent array never traps:
- * it sets status bit 1, read (and cleared) by specfold_gate_get_status.
+ * it sets status bit 1, read (and cleared) by specfold_gate_get_status.  On
+ * 16-byte aligned rows of at most 50 KB the difference test streams row pairs
+ * into shared memory by bulk copies; its waits are bounded (2 s), and a wait
+ * that gives up (it never should) sets status bit 2 instead of hanging.
  */
 #ifndef SPECFOLD_GATE_H
 #define SPECFOLD_GATE_H
@@ -81,9 +84,10 @@ sv_status specfold_gate_run(specfold_gate_t h, const void *hidden, const int32_t
                             int32_t *packed_rows, int32_t *n_packed, void *packed_hidden,
                             void *stream);
 
-/* Wait for `stream`, read and clear the status word: SV_ERR_PARENT if some
- * parent entry was invalid since the last call, else SV_OK.  `*bits` (may be
- * NULL) receives the raw bits (1: invalid parent). */
+/* Wait for `stream`, read and clear the status word: SV_ERR_PIPELINE if a
+ * bounded wait of the difference test gave up since the last call, else
+ * SV_ERR_PARENT if some parent entry was invalid, else SV_OK.  `*bits` (may
+ * be NULL) receives the raw bits (1: invalid parent, 2: a wait gave up). */
 sv_status specfold_gate_get_status(specfold_gate_t h, void *stream, uint32_t *bits);
 
 /* Record CUDA events around each of the next `max_runs` runs' kernels

@@ -13,7 +13,9 @@
 //                each warp streams its rows' H[c, j] and H[parent, j] with
 //                128-bit loads, eight in flight per lane, sums squares with
 //                packed fp32 pairs per lane and in fp64 across the warp, and
-//                decides recompute = !(d <= tau);
+//                decides recompute = !(d <= tau); on 16-byte aligned rows
+//                of at most 50 KB the bulk-copy form rows_bulk_kernel does
+//                the same test from shared memory (one block per SM);
 //   scan_kernel  one block: the packed slot of every recomputed row (an
 //                exclusive prefix sum of the flags) and their count;
 //   pack_kernel  one warp per row: writes the packed row index, follows the
@@ -43,6 +45,9 @@ struct GateParams {
   int branches, positions, dim;
   long rows;
   int blocks;               // rows_kernel grid (persistent warps)
+  int bulk_stages;          // > 0: rows_bulk_kernel with this many ring stages
+  int bulk_consumers;       // its consumer warps that take rows (bulk_stages is a multiple)
+  int bulk_parts;           // stage loads per row pair: 1, or 2 (halves of the rows)
   int pack_blocks;          // pack_kernel grid (8 rows per block)
   // outputs (rel_diff, provenance, source, packed_hidden may be null)
   float* rel_diff;
@@ -286,6 +291,248 @@ __global__ void __launch_bounds__(kThreads, kRowsBlocksPerSM) rows_kernel(const 
     }
   }
 
+}
+
+// ---------------------------------------------------------------------------
+// kernel 2, bulk-copy form (16-byte aligned rows of at most kBulkMaxRowBytes)
+// ---------------------------------------------------------------------------
+//
+// One persistent block per SM takes rows blockIdx.x + k G (G blocks), as the
+// register form's warps do, so every block moves through the tensor with the
+// others and a parent row is still in L2 when its children read it.  C warps
+// of the block take the block's rows k = c, c + C, ... (warp c) that have a
+// parent; each warp streams its rows through a private ring of R stages of
+// shared memory, every stage one (child row, parent row) pair brought in by
+// two 1-D bulk copies (the copy engine generates the addresses: one
+// instruction per row) whose completion the stage's mbarrier counts in bytes.
+// A warp reduces the pair of its oldest stage and refills that stage with
+// its load R ahead.  The reduction of a pair is one dependent chain per lane,
+// so the most warps with one stage each do best; where whole row pairs would
+// leave fewer than 12 stages, a stage holds half of each row (the two halves
+// of a row go through the same warp, one after the other).  With hidden size
+// 4096, bf16: 12 warps of one 16 KB stage, 96 KB of child rows per SM in
+// flight or being reduced, where the register form keeps about 64 KB of
+// child rows in flight at its full occupancy.  A stage only ever holds its own
+// warp's rows, in order, so no wait can run a phase ahead of its barrier (a
+// parity wait could not tell two phases apart) and no stage needs a release
+// barrier.  The parents of a warp's rows are looked up 32 at a time, one
+// lane per row, with the next 32 in flight.  Each lane adds the groups lane,
+// lane + 32, ... of both rows in the register form's order (a half row holds
+// a multiple of 32 groups), so the sums are the same bits.  Every wait is bounded (2 s of the global timer): a wait
+// that runs out sets kStatWait, and the warp waits (bounded) for the copies
+// it issued before it leaves.
+
+constexpr int kBulkWarps = 24;  // warps launched; P.bulk_consumers of them take rows
+constexpr int kBulkThreads = kBulkWarps * kWarp;
+constexpr int kBulkMaxStages = 24;
+constexpr int kBulkRingBytes = 200 * 1024;                  // dynamic shared memory, at most
+constexpr long kBulkMaxRowBytes = kBulkRingBytes / 4;       // at least 2 whole-row stages
+constexpr unsigned long long kBulkWaitNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ unsigned smem_u32(const void* p) {
+  return static_cast<unsigned>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, unsigned count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint64_t* bar, unsigned bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, unsigned parity) {
+  unsigned ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// wait for the phase of `parity` to complete; false after 2 s
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, unsigned parity) {
+  if (mbar_test(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (!mbar_test(bar, parity))
+    if (global_ns() - t0 > kBulkWaitNs) return false;
+  return true;
+}
+// bytes from global to this block's shared memory (both 16-byte aligned,
+// bytes a multiple of 16), counted on `bar`; no multicast
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, unsigned bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+enum : unsigned { kStatWait = 2u };
+
+template <typename T>
+__global__ void __launch_bounds__(kBulkThreads, 1) rows_bulk_kernel(const GateParams P) {
+  extern __shared__ __align__(128) unsigned char ring[];  // C rings of R (child row, parent row) stages
+  __shared__ uint64_t full[kBulkMaxStages];
+  __shared__ int item_row[kBulkMaxStages], item_par[kBulkMaxStages], item_part[kBulkMaxStages];
+  const int warp = threadIdx.x / kWarp, lane = threadIdx.x & (kWarp - 1);
+  const int C = P.bulk_consumers;      // warps that take rows, 1 .. kBulkWarps
+  const int R = P.bulk_stages / C;     // stages per warp (bulk_stages is a multiple of C)
+  const int parts = P.bulk_parts;      // 1 or 2 stage loads per row pair
+  const long G = gridDim.x;
+  const unsigned rb = static_cast<unsigned>(P.dim * sizeof(T));  // a multiple of 16
+  const unsigned pb = rb / parts;      // bytes of one row per stage: a multiple of 512 when parts = 2
+  const T* base = static_cast<const T*>(P.hidden);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C * R; ++s) mbar_init(&full[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncthreads();
+  cudaGridDependencySynchronize();  // validated parents
+
+  // the block's rows are blockIdx.x + k G, k = 0 .. nk - 1 (rows < 2^31)
+  const int nk = static_cast<int>((P.rows - blockIdx.x + G - 1) / G);
+  auto row_of = [&](int k) -> int { return static_cast<int>(blockIdx.x + static_cast<long>(k) * G); };
+  // rows without a parent are decided without reading anything, lane by lane
+  // across all warps of the block
+  for (int k = warp + kBulkWarps * lane; k < nk; k += kBulkWarps * kWarp) {
+    const int row = row_of(k);
+    if (P.eff_parent[row / P.positions] < 0) finish_row(P, row, -1, 0, 0.0, 0.0);
+  }
+  const int c = warp;
+  if (c >= C) return;
+
+  // warp c's rows: m-th = k = c + m C, m = 0 .. mc - 1; lane l looks up the
+  // parent of m = m0 + l, the next 32 lookups in flight
+  const int mc = (nk > c) ? (nk - c + C - 1) / C : 0;
+  auto lookup = [&](int m) -> int {
+    return (m < mc) ? P.eff_parent[row_of(c + m * C) / P.positions] : -1;
+  };
+  int m0 = 0;
+  int par_cur = lookup(lane);
+  int par_next = lookup(kWarp + lane);
+  unsigned todo = __ballot_sync(0xffffffffu, par_cur >= 0);
+  // the next row of the warp that has a parent (warp-uniform); false at the end
+  auto next_item = [&](int& row, int& par) -> bool {
+    while (todo == 0u) {
+      if (m0 + kWarp >= mc) return false;
+      m0 += kWarp;
+      par_cur = par_next;
+      par_next = lookup(m0 + kWarp + lane);
+      todo = __ballot_sync(0xffffffffu, par_cur >= 0);
+    }
+    const int bit = __ffs(todo) - 1;
+    todo &= todo - 1u;
+    par = __shfl_sync(0xffffffffu, par_cur, bit);
+    row = row_of(c + (m0 + bit) * C);
+    return true;
+  };
+  uint64_t* bar = full + c * R;
+  unsigned char* mine = ring + static_cast<size_t>(c) * R * 2 * pb;
+  // the stage loads of a warp: part h = 0 .. parts - 1 of each of its rows
+  // with a parent, in order (warp-uniform); false at the end
+  int cur_row = 0, cur_par = 0, cur_part = parts;
+  auto next_load = [&](int& row, int& par, int& part) -> bool {
+    if (cur_part == parts) {
+      if (!next_item(cur_row, cur_par)) return false;
+      cur_part = 0;
+    }
+    row = cur_row;
+    par = cur_par;
+    part = cur_part++;
+    return true;
+  };
+  // the copies of part h of (row, par) into stage s of this warp's ring (lane 0)
+  auto issue = [&](int s, int row, int par, int part) {
+    if (lane == 0) {
+      item_row[c * R + s] = row;
+      item_par[c * R + s] = par;
+      item_part[c * R + s] = part;
+      const int j = row % P.positions;
+      unsigned char* dst = mine + static_cast<size_t>(s) * 2 * pb;
+      const char* child = reinterpret_cast<const char*>(base + static_cast<long>(row) * P.dim);
+      const char* parent =
+          reinterpret_cast<const char*>(base + (static_cast<long>(par) * P.positions + j) * P.dim);
+      // the warp's generic reads of this stage (synchronised by the caller)
+      // come before the copy engine's writes
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_tx(&bar[s], 2 * pb);
+      bulk_load(dst, child + static_cast<size_t>(part) * pb, pb, &bar[s]);
+      bulk_load(dst + pb, parent + static_cast<size_t>(part) * pb, pb, &bar[s]);
+    }
+  };
+
+  int issued = 0;
+  bool more = true;
+  while (issued < R) {
+    int row, par, part;
+    if (!(more = next_load(row, par, part))) break;
+    issue(issued, row, par, part);
+    ++issued;
+  }
+  // a part holds groups/parts groups, a multiple of 32 when parts = 2, so
+  // each lane meets its groups lane, lane + 32, ... of the row in order
+  const int pgroups = static_cast<int>(pb / 16);
+  int t = 0, s = 0;
+  unsigned ph = 0;
+  bool ok = true;
+  float2 d = make_float2(0.f, 0.f), n = make_float2(0.f, 0.f);
+  for (; t < issued; ++t) {
+    if (!mbar_wait(&bar[s], ph)) {
+      ok = false;
+      break;
+    }
+    __syncwarp();
+    const int row = item_row[c * R + s];
+    const int par = item_par[c * R + s];
+    const int part = item_part[c * R + s];
+    const uint4* hc = reinterpret_cast<const uint4*>(mine + static_cast<size_t>(s) * 2 * pb);
+    const uint4* hp = hc + pgroups;
+#pragma unroll 4
+    for (int g = lane; g < pgroups; g += kWarp) HElem<T>::accumulate2(hc[g], hp[g], d, n);
+    __syncwarp();  // every lane's reads of the stage are done
+    if (more) {
+      int r2, p2, h2;
+      if ((more = next_load(r2, p2, h2))) {
+        issue(s, r2, p2, h2);
+        ++issued;
+      }
+    }
+    if (part == parts - 1) {
+      double num = static_cast<double>(d.x) + static_cast<double>(d.y);
+      double den = static_cast<double>(n.x) + static_cast<double>(n.y);
+#pragma unroll
+      for (int o = kWarp / 2; o > 0; o >>= 1) {
+        num += __shfl_xor_sync(0xffffffffu, num, o);
+        den += __shfl_xor_sync(0xffffffffu, den, o);
+      }
+      if (lane == 0) finish_row(P, row, par, row % P.positions, num, den);
+      d = make_float2(0.f, 0.f);
+      n = make_float2(0.f, 0.f);
+    }
+    if (++s == R) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+  if (!ok) {
+    if (lane == 0) {
+      atomicOr(P.status, kStatWait);
+      // the copies still in flight must land before the warp leaves
+      for (int u = t; u < issued; ++u)
+        if (!mbar_wait(&bar[u % R], static_cast<unsigned>((u / R) & 1))) break;
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------

@@ -25,6 +25,10 @@ struct specfold_gate_ctx {
   int branches = 0, positions = 0, dim = 0;
   long rows = 0;
   int blocks = 0;       // difference kernel (persistent)
+  int bulk_stages = 0;  // bulk-copy difference kernel: ring stages (0: register form only)
+  int bulk_consumers = 0;  // its consumer warps (bulk_stages is a multiple)
+  int bulk_parts = 1;      // stage loads per row pair (2: half rows)
+  int bulk_blocks = 0;  // its grid: one block per SM
   int pack_blocks = 0;  // packing kernel
   sv_dtype dtype = SV_DTYPE_F32;
   void* ws = nullptr;
@@ -61,15 +65,22 @@ cudaError_t launch_pdl(K kernel, unsigned grid, unsigned block, size_t smem, cud
 }
 
 template <typename T, bool A>
-cudaError_t launch_pass(const GateParams& p, cudaStream_t s, cudaEvent_t* ev) {
+cudaError_t launch_pass(const GateParams& p, int bulk_blocks, cudaStream_t s, cudaEvent_t* ev) {
   const size_t smem = 2 * sizeof(int32_t) * static_cast<size_t>(p.branches);
   cudaError_t e = cudaSuccess;
   specfold::tree_kernel<<<1, specfold::kTreeThreads, smem, s>>>(p);
   e = cudaGetLastError();
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[0], s);
-  if (e == cudaSuccess)
-    e = launch_pdl(specfold::rows_kernel<T, A>, static_cast<unsigned>(p.blocks),
-                   specfold::kThreads, 0, s, p);
+  if (e == cudaSuccess) {
+    if (A && p.bulk_stages > 0)
+      e = launch_pdl(specfold::rows_bulk_kernel<T>, static_cast<unsigned>(bulk_blocks),
+                     specfold::kBulkThreads,
+                     static_cast<size_t>(p.bulk_stages) * 2 * sizeof(T) * p.dim / p.bulk_parts, s,
+                     p);
+    else
+      e = launch_pdl(specfold::rows_kernel<T, A>, static_cast<unsigned>(p.blocks),
+                     specfold::kThreads, 0, s, p);
+  }
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
   if (e == cudaSuccess)
     e = launch_pdl(specfold::scan_kernel, 1u, specfold::kSlotThreads, 0, s, p);
@@ -136,6 +147,43 @@ sv_status specfold_gate_create(specfold_gate_t* out, int branches, int positions
     }
     const long want = static_cast<long>(sms) * (occ > 0 ? occ : 1);
     h->blocks = static_cast<int>(want < rows ? want : rows);
+    // rows of 16-byte multiples up to a quarter of the ring take the
+    // bulk-copy form on aligned inputs: one block per SM, as many stages of
+    // (child, parent) row pairs as the ring holds (at most kBulkMaxStages).
+    // Each warp that takes rows owns S / C stages.  A warp's reduction of a
+    // row pair is one long dependent chain per lane, so the most warps with
+    // one stage each beat fewer warps with deeper rings (measured on the
+    // 4096-wide bf16 rows: 12 warps x 1 stage 49.9 us, 8 x 1 53.5 us,
+    // 6 x 2 65.0 us, 4 x 3 74.1 us, 3 x 4 94.4 us; 24 warps of half rows
+    // 50.7 us).  Where the ring holds fewer than 12 whole row pairs and a row
+    // has a multiple of 64 groups, a stage holds half of each row instead
+    // (twice the warps).
+    const long rb = static_cast<long>(dim) * static_cast<long>(gate_elem_size(dtype));
+    if (rb % 16 == 0 && rb <= specfold::kBulkMaxRowBytes) {
+      int parts = 1;
+      long smax = specfold::kBulkRingBytes / (2 * rb);  // >= 2
+      if (smax < specfold::kBulkMaxStages / 2 && (rb / 16) % 64 == 0) {
+        parts = 2;
+        smax = specfold::kBulkRingBytes / rb;
+      }
+      if (smax > specfold::kBulkMaxStages) smax = specfold::kBulkMaxStages;
+      long cons = smax;
+      if (cons > specfold::kBulkWarps) cons = specfold::kBulkWarps;
+      h->bulk_parts = parts;
+      h->bulk_stages = static_cast<int>(cons * (smax / cons));
+      h->bulk_consumers = static_cast<int>(cons);
+      h->bulk_blocks = static_cast<int>(sms < rows ? sms : rows);
+      // the attribute is per function, shared by all handles: the ring's maximum
+      const void* kb = (dtype == SV_DTYPE_BF16)
+                           ? reinterpret_cast<const void*>(specfold::rows_bulk_kernel<__nv_bfloat16>)
+                           : reinterpret_cast<const void*>(specfold::rows_bulk_kernel<float>);
+      e = cudaFuncSetAttribute(kb, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               specfold::kBulkRingBytes);
+      if (e != cudaSuccess) {
+        delete h;
+        return cuda_fail(e);
+      }
+    }
   }
 
   size_t off = 0;
@@ -200,6 +248,9 @@ sv_status specfold_gate_run(specfold_gate_t h, const void* hidden, const int32_t
   p.dim = h->dim;
   p.rows = h->rows;
   p.blocks = h->blocks;
+  p.bulk_stages = h->bulk_stages;
+  p.bulk_consumers = h->bulk_consumers;
+  p.bulk_parts = h->bulk_parts;
   p.pack_blocks = h->pack_blocks;
   p.rel_diff = rel_diff;
   p.provenance = provenance;
@@ -220,9 +271,11 @@ sv_status specfold_gate_run(specfold_gate_t h, const void* hidden, const int32_t
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (h->dtype == SV_DTYPE_BF16)
-    e = aligned ? launch_pass<__nv_bfloat16, true>(p, s, ev) : launch_pass<__nv_bfloat16, false>(p, s, ev);
+    e = aligned ? launch_pass<__nv_bfloat16, true>(p, h->bulk_blocks, s, ev)
+                : launch_pass<__nv_bfloat16, false>(p, h->bulk_blocks, s, ev);
   else
-    e = aligned ? launch_pass<float, true>(p, s, ev) : launch_pass<float, false>(p, s, ev);
+    e = aligned ? launch_pass<float, true>(p, h->bulk_blocks, s, ev)
+                : launch_pass<float, false>(p, h->bulk_blocks, s, ev);
   if (e != cudaSuccess) return cuda_fail(e);
   return SV_OK;
 }
@@ -238,6 +291,7 @@ sv_status specfold_gate_get_status(specfold_gate_t h, void* stream, uint32_t* bi
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(e);
   if (bits) *bits = v;
+  if (v & specfold::kStatWait) return SV_ERR_PIPELINE;
   return (v & specfold::kStatParent) ? SV_ERR_PARENT : SV_OK;
 }
 

@@ -110,6 +110,11 @@ def test_gate_full_size():
     (2, 3, 3, 100, "bf16", 0.05),     # 200-byte rows: scalar loads
     (40, 8, 32, 256, "bf16", 0.05),   # 10240 rows: 1280 blocks, several scan chunks
     (1, 1, 1, 8, "f32", 0.05),        # one row, no parent
+    (5, 8, 32, 4096, "f32", 0.05),    # 16 KB rows: half-row stages of the bulk-copy ring
+    (2, 4, 3, 3000, "bf16", 0.05),    # 6000-byte rows: 17 whole-row stages, one warp each
+    (2, 4, 3, 12800, "f32", 0.05),    # 51200-byte rows: the largest the ring takes (4 half-row stages)
+    (2, 4, 3, 12804, "f32", 0.05),    # 51216-byte rows: register form
+    (1, 3, 2, 2048, "bf16", 0.05),    # 6 rows: fewer rows than SMs, two blocks with nothing to read
 ])
 def test_gate_shapes(seqs, branches, positions, dim, dtype, tau):
     w = workloads.gate_tree(seed=seqs + dim, sequences=seqs, branches=branches,
