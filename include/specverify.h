@@ -254,10 +254,9 @@ sv_status specverify_get_launch(specverify_t h, int *slices, int *threads, int *
 
 /*
  * Number of kernels one run of the handle enqueues (`mapped` nonzero: a run
- * of specverify_run_mapped): statistics, decide and draw (3); statistics and
- * a draw that takes the decisions itself (2) when the draw grid is less than
- * one wave of the device (small batches); one for an aligned unmapped run in
- * the single-launch form (specverify_set_fused); none for an empty batch.
+ * of specverify_run_mapped): statistics, decide and draw (3); one for an
+ * aligned unmapped run in the single-launch form (specverify_set_fused); none
+ * for an empty batch.
  */
 sv_status specverify_kernels_per_run(specverify_t h, int mapped, int *kernels);
 

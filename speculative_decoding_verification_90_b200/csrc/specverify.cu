@@ -172,12 +172,10 @@ cudaError_t launch_stats_nt(const Params& p, long blocks, cudaStream_t s) {
   return launch_pdl(specverify::stats_kernel<T, NT, A>, static_cast<unsigned>(blocks), NT, s, p);
 }
 
-// One step: statistics, decide, draw; statistics then a draw that decides
-// (two launches) when the draw grid is less than one wave (see
-// draw_decides).  events[0..2] (may be null): before stats, after stats,
-// after draw.
+// One step: statistics, decide, draw.  events[0..2] (may be null): before
+// stats, after stats, after draw.
 template <typename T, bool A>
-cudaError_t launch_step(const Params& p, int NT, unsigned draw_blocks, int num_sms, cudaStream_t s,
+cudaError_t launch_step(const Params& p, int NT, unsigned draw_blocks, cudaStream_t s,
                         cudaEvent_t* ev) {
   const long rows = p.target_rows + p.draft_rows;
   const long blocks = p.taper_rows * p.taper_slices + (rows - p.taper_rows) * p.slices;
@@ -192,24 +190,20 @@ cudaError_t launch_step(const Params& p, int NT, unsigned draw_blocks, int num_s
   }
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[1], s);
   if (e != cudaSuccess) return e;
-  if (specverify::draw_decides(p.batch, draw_blocks, num_sms)) {
-    e = specverify::launch_draw<T, A, true>(p, draw_blocks, s, true);
-  } else {
-    const int per = specverify::kDecideThreads / specverify::kWarp;
-    e = launch_pdl(specverify::decide_kernel<T>, static_cast<unsigned>((p.batch + per - 1) / per),
-                   specverify::kDecideThreads, s, p);
-    if (e != cudaSuccess) return e;
-    e = specverify::launch_draw<T, A>(p, draw_blocks, s, true);
-  }
+  const int per = specverify::kDecideThreads / specverify::kWarp;
+  e = launch_pdl(specverify::decide_kernel<T>, static_cast<unsigned>((p.batch + per - 1) / per),
+                 specverify::kDecideThreads, s, p);
+  if (e != cudaSuccess) return e;
+  e = specverify::launch_draw<T, A>(p, draw_blocks, s, true);
   if (e == cudaSuccess && ev) e = cudaEventRecord(ev[2], s);
   return e;
 }
 
 template <typename T>
-cudaError_t launch_dtype(const Params& p, int NT, unsigned draw_blocks, int num_sms, bool aligned,
+cudaError_t launch_dtype(const Params& p, int NT, unsigned draw_blocks, bool aligned,
                          cudaStream_t s, cudaEvent_t* ev) {
-  return aligned ? launch_step<T, true>(p, NT, draw_blocks, num_sms, s, ev)
-                 : launch_step<T, false>(p, NT, draw_blocks, num_sms, s, ev);
+  return aligned ? launch_step<T, true>(p, NT, draw_blocks, s, ev)
+                 : launch_step<T, false>(p, NT, draw_blocks, s, ev);
 }
 
 bool aligned_to(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -388,8 +382,8 @@ sv_status enqueue(specverify_t h, const void* target, const void* draft, const i
     return SV_OK;
   }
   cudaError_t e = (h->dtype == SV_DTYPE_BF16)
-                      ? launch_dtype<__nv_bfloat16>(p, h->threads, nd, h->num_sms, aligned, stream, ev)
-                      : launch_dtype<float>(p, h->threads, nd, h->num_sms, aligned, stream, ev);
+                      ? launch_dtype<__nv_bfloat16>(p, h->threads, nd, aligned, stream, ev)
+                      : launch_dtype<float>(p, h->threads, nd, aligned, stream, ev);
   if (e != cudaSuccess) return cuda_fail(e);
   return SV_OK;
 }
@@ -796,13 +790,12 @@ sv_status specverify_get_launch(specverify_t h, int* slices, int* threads, int* 
 
 sv_status specverify_kernels_per_run(specverify_t h, int mapped, int* kernels) {
   if (!h || !kernels) return SV_ERR_INVALID_ARG;
-  // statistics, decide, draw (statistics and a deciding draw when the draw
-  // grid is less than one wave); one launch for an
-  // unmapped run in fused mode (the count for 16-byte aligned logits with
-  // vocab * sizeof(dtype) a multiple of 16)
+  // statistics, decide, draw; one launch for an unmapped run in fused mode
+  // (the count for 16-byte aligned logits with vocab * sizeof(dtype) a
+  // multiple of 16)
   if (h->batch == 0) *kernels = 0;
   else if (!mapped && use_fused(h, nullptr)) *kernels = 1;
-  else *kernels = specverify::draw_decides(h->batch, draw_blocks(h), h->num_sms) ? 2 : 3;
+  else *kernels = 3;
   return SV_OK;
 }
 

@@ -1246,22 +1246,7 @@ __device__ __noinline__ void locate(const Params* Pp, int b, int n, int mode, co
   }
 }
 
-// The decision of sequence b inside the draw kernel, as a call of its own so
-// that none of its registers is live across the draw's tile loop.
-template <typename T>
-__device__ __noinline__ void decide_in_draw(const Params* Pp, int b, bool write,
-                                            const LaneInputs* pre, SeqDecision* out) {
-  *out = decide_sequence<T>(*Pp, b, nullptr, write, pre);
-}
-
-// kInline: the kernel follows the statistics kernel directly and every warp
-// takes the decision of each sequence its run touches itself (the same
-// arithmetic in every warp, so all agree); the warp whose run holds the
-// sequence's first tile writes the decision's outputs.  The caller's inputs
-// to the first decision are loaded before the grid-dependency wait.  Chosen
-// for grids of less than one wave with no more sequences than warps (a run
-// then touches at most two sequences).
-template <typename T, bool kAligned, bool kInline = false>
+template <typename T, bool kAligned>
 __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(const __grid_constant__ Params P) {
   constexpr int kVec = Elem<T>::kVec;
   extern __shared__ uint4 draw_smem[];
@@ -1274,21 +1259,12 @@ __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(co
   const long W = static_cast<long>(gridDim.x) * kDrawWarps;
   const long w = static_cast<long>(blockIdx.x) * kDrawWarps + (threadIdx.x >> 5);
   const long lo = total * w / W, hi = total * (w + 1) / W;
-  const int b_pre = (lo < hi) ? static_cast<int>(lo / ntiles) : -1;
-  LaneInputs pre{0, 0, 0, 0.f, 0.f, 0.f, false, false};
-  if constexpr (kInline) {
-    if (b_pre >= 0) pre = lane_inputs<T>(P, b_pre, lane);
-  }
-  cudaGridDependencySynchronize();  // the statistics (or decisions) of the previous kernel
+  cudaGridDependencySynchronize();  // the decisions of the previous kernel
   for (long t = lo; t < hi;) {
     const int b = static_cast<int>(t / ntiles);
     const long row0 = static_cast<long>(b) * ntiles;
     const long end = (hi < row0 + ntiles) ? hi : row0 + ntiles;
-    SeqDecision d;
-    if constexpr (kInline)
-      decide_in_draw<T>(&P, b, t == row0, b == b_pre ? &pre : nullptr, &d);
-    else
-      d = P.decision[b];
+    const SeqDecision d = P.decision[b];
     // (a debug build skips a sequence whose rows drawn from lie outside the
     // logit buffers, in every warp alike, so its ticket stays untouched)
     const bool rows_ok = d.mode == kDrawNone ||
@@ -1333,25 +1309,15 @@ __global__ void __launch_bounds__(kDrawThreads, kDrawBlocksPerSM) draw_kernel(co
   }
 }
 
-// Whether the draw kernel takes the decisions itself (kInline): a draw grid of
-// less than one resident wave (a small, launch-bound batch: one launch and
-// one grid-dependency wait fewer), with no more sequences than warps.  On
-// batches that fill the wave every warp's serial decision costs more than the
-// separate decide kernel saves.
-inline bool draw_decides(long batch, unsigned grid, int num_sms) {
-  return static_cast<long>(grid) < static_cast<long>(num_sms) * kDrawBlocksPerSM &&
-         batch <= static_cast<long>(grid) * kDrawWarps;
-}
-
 // Host: launch the draw kernel (its ring needs more than the default 48 KB of
 // dynamic shared memory per block), optionally as a programmatic dependent
 // launch of the previous kernel on the stream.
-template <typename T, bool kAligned, bool kInline = false>
+template <typename T, bool kAligned>
 inline cudaError_t launch_draw(const Params& p, unsigned grid, cudaStream_t s, bool pdl) {
   const size_t smem = kAligned ? kDrawSmem : 0;
   cudaError_t e = cudaSuccess;
   if (kAligned)
-    e = cudaFuncSetAttribute(draw_kernel<T, kAligned, kInline>,
+    e = cudaFuncSetAttribute(draw_kernel<T, kAligned>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
@@ -1364,7 +1330,7 @@ inline cudaError_t launch_draw(const Params& p, unsigned grid, cudaStream_t s, b
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, draw_kernel<T, kAligned, kInline>, p);
+  return cudaLaunchKernelEx(&cfg, draw_kernel<T, kAligned>, p);
 }
 
 }  // namespace specverify

@@ -40,17 +40,16 @@ def _check(wl, fused=True):
 
 
 def test_single_launch_counts_one_kernel():
-    """Launch counts: one in fused mode; otherwise statistics and a draw that
-    decides (two) while the draw grid is less than one wave, statistics,
-    decide and draw (three) from one wave on."""
+    """Launch counts: one in fused mode; otherwise statistics, decide and draw
+    (three) at every batch size."""
     from speculative_decoding_verification_90_b200.specverify import SpecVerify
     with SpecVerify(4, 3, 4096, "bf16") as sv:
-        assert sv.kernels_per_run() == 2 and sv.fused()[0] == 0  # off by default
+        assert sv.kernels_per_run() == 3 and sv.fused()[0] == 0  # off by default
         sv.set_fused(True)
         assert sv.kernels_per_run() == 1 and sv.fused()[0] == 1
-        assert sv.kernels_per_run(mapped=True) == 2  # the mapped form keeps the kernels
+        assert sv.kernels_per_run(mapped=True) == 3  # the mapped form keeps the kernels
         sv.set_fused(False)
-        assert sv.kernels_per_run() == 2
+        assert sv.kernels_per_run() == 3
     for B, G, V, dt in ((60000, 1, 4096, "f32"), (64, 8, 128256, "bf16")):
         with SpecVerify(B, G, V, dt) as sv:
             assert sv.kernels_per_run() == 3 and sv.kernels_per_run(mapped=True) == 3
