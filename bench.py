@@ -995,10 +995,22 @@ def time_gate(args, dev, world, local):
     ms, kern = timed_then_profiled(lambda i: step(), steps, gate.profile_begin, gate.profile_end,
                                    world, local)
     ms_max = svdist.max_over_ranks(ms, device=dev)
+    k = int(n.item())
+    # diagnostic: the same passes without the packed batch (the packing kernel
+    # then writes no rows), so the difference kernel does not run while the
+    # previous pass's 105 MB of packed rows are written back from L2
+    def step_unpacked():
+        gate.run(H, par, w.tau, packed, n, rel_diff=rel, provenance=prov, source=src)
+
+    for _ in range(3):
+        step_unpacked()
+    torch.cuda.synchronize()
+    _, kern_u = timed_then_profiled(lambda i: step_unpacked(), steps, gate.profile_begin,
+                                    gate.profile_end, world, local)
     st, _ = gate.status()
     gate.close()
-    k = int(n.item())
     return {"workload": w.name, "steps": steps, "ms_max": ms_max, "rows_ms": kern["rows_ms"],
+            "rows_ms_unpacked": kern_u["rows_ms"],
             "pack_ms": kern["pack_ms"], "rows": rows, "packed": k,
             "read_bytes": w.rows_read() * w.dim * w.elem_size,
             "packed_bytes": k * w.dim * w.elem_size, "hidden_bytes": w.hidden.nbytes,
@@ -1018,6 +1030,12 @@ def gate_summary(g, peak):
         "difference_kernel": {"us": 1e3 * g["rows_ms"], "algorithmic_bytes": g["read_bytes"],
                               "achieved_gbs": rows_gbs, "peak_gbs": peak,
                               "frac": rows_gbs / peak},
+        # the same kernel in passes that write no packed rows (a diagnostic:
+        # the figure above includes the write-back of the previous pass's
+        # packed batch from L2)
+        "difference_kernel_without_packed_rows": {
+            "us": 1e3 * g["rows_ms_unpacked"],
+            "frac": g["read_bytes"] / (g["rows_ms_unpacked"] / 1e3) / 1e9 / peak},
         "pack_kernel": {"us": 1e3 * g["pack_ms"], "algorithmic_bytes": g["packed_bytes"],
                         "achieved_gbs": pack_gbs},
         "l2": "inputs larger than L2 (%.0f MB of hidden states per pass)" % (g["hidden_bytes"] / 1e6),

@@ -297,10 +297,10 @@ __global__ void __launch_bounds__(kThreads, kRowsBlocksPerSM) rows_kernel(const 
 // kernel 2, bulk-copy form (16-byte aligned rows of at most kBulkMaxRowBytes)
 // ---------------------------------------------------------------------------
 //
-// One persistent block per SM takes rows blockIdx.x + k G (G blocks), as the
-// register form's warps do, so every block moves through the tensor with the
-// others and a parent row is still in L2 when its children read it.  C warps
-// of the block take the block's rows k = c, c + C, ... (warp c) that have a
+// One persistent block per SM (C warps) takes rows blockIdx.x + k G (G
+// blocks), as the register form's warps do, so every block moves through the
+// tensor with the others and a parent row is still in L2 when its children
+// read it.  The warps take the block's rows k = c, c + C, ... (warp c) that have a
 // parent; each warp streams its rows through a private ring of R stages of
 // shared memory, every stage one (child row, parent row) pair brought in by
 // two 1-D bulk copies (the copy engine generates the addresses: one
@@ -322,7 +322,7 @@ __global__ void __launch_bounds__(kThreads, kRowsBlocksPerSM) rows_kernel(const 
 // that runs out sets kStatWait, and the warp waits (bounded) for the copies
 // it issued before it leaves.
 
-constexpr int kBulkWarps = 24;  // warps launched; P.bulk_consumers of them take rows
+constexpr int kBulkWarps = 24;  // warps per block at most; the launch has P.bulk_consumers
 constexpr int kBulkThreads = kBulkWarps * kWarp;
 constexpr int kBulkMaxStages = 24;
 constexpr int kBulkRingBytes = 200 * 1024;                  // dynamic shared memory, at most
@@ -405,7 +405,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) rows_bulk_kernel(const GatePa
   auto row_of = [&](int k) -> int { return static_cast<int>(blockIdx.x + static_cast<long>(k) * G); };
   // rows without a parent are decided without reading anything, lane by lane
   // across all warps of the block
-  for (int k = warp + kBulkWarps * lane; k < nk; k += kBulkWarps * kWarp) {
+  const int nwarps = static_cast<int>(blockDim.x) / kWarp;
+  for (int k = warp + nwarps * lane; k < nk; k += nwarps * kWarp) {
     const int row = row_of(k);
     if (P.eff_parent[row / P.positions] < 0) finish_row(P, row, -1, 0, 0.0, 0.0);
   }
@@ -488,7 +489,8 @@ __global__ void __launch_bounds__(kBulkThreads, 1) rows_bulk_kernel(const GatePa
   bool ok = true;
   float2 d = make_float2(0.f, 0.f), n = make_float2(0.f, 0.f);
   for (; t < issued; ++t) {
-    if (!mbar_wait(&bar[s], ph)) {
+    // every lane waits; the warp leaves together if any lane's wait gave up
+    if (!__all_sync(0xffffffffu, mbar_wait(&bar[s], ph))) {
       ok = false;
       break;
     }

@@ -74,7 +74,7 @@ cudaError_t launch_pass(const GateParams& p, int bulk_blocks, cudaStream_t s, cu
   if (e == cudaSuccess) {
     if (A && p.bulk_stages > 0)
       e = launch_pdl(specfold::rows_bulk_kernel<T>, static_cast<unsigned>(bulk_blocks),
-                     specfold::kBulkThreads,
+                     static_cast<unsigned>(p.bulk_consumers * specfold::kWarp),
                      static_cast<size_t>(p.bulk_stages) * 2 * sizeof(T) * p.dim / p.bulk_parts, s,
                      p);
     else
